@@ -1,0 +1,258 @@
+"""Cube-routed block-sparse attention for B200 (sm_100a): thin Python binding of libsa.
+
+Every step of the path runs in the CUDA kernels of ``libsa.so``; this module only
+marshals arguments (device pointers, sizes, the current CUDA stream) and allocates
+outputs and workspaces with torch.  There is no CPU fallback: importing works without
+a GPU, but every compute call needs the built library and a CUDA device.
+
+Entry points mirror the C ABI in ``include/sa.h``:
+
+* :func:`plan`      router -> ``kv_index [B,H,T,cap]``, ``kv_count [B,H,T]``
+* :func:`forward`   fine stage -> ``out [B,H,Npad,D]`` bf16, ``lse [B,H,Npad]`` fp32
+* :func:`backward`  -> ``dq, dk, dv`` fp32
+* :func:`tile` / :func:`untile`  latent order <-> cube-major padded order
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsa.so")
+
+SA_OK = 0
+STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_ALIGNMENT",
+                4: "SA_ERR_CAPACITY", 5: "SA_ERR_WORKSPACE", 6: "SA_ERR_LAUNCH", 7: "SA_ERR_DEVICE_TIMEOUT",
+                8: "SA_ERR_DEVICE_INDEX"}
+OP_PLAN, OP_FORWARD, OP_BACKWARD = 0, 1, 2
+BF16, FP8_E4M3 = 0, 1
+DEBUG_SKIP_LOADS = 1
+
+# every symbol include/sa.h declares
+EXPORTS = ("sa_padded_tokens", "sa_num_cubes", "sa_topk_from_fraction", "sa_workspace_size", "sa_tile",
+           "sa_untile", "sa_plan", "sa_forward", "sa_backward", "sa_get_device_status", "sa_status_string",
+           "sa_last_launch_count")
+
+
+class SAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("D", ctypes.c_int),
+                ("lat_t", ctypes.c_int), ("lat_h", ctypes.c_int), ("lat_w", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("top_p", ctypes.c_float), ("kv_capacity", ctypes.c_int),
+                ("qk_dtype", ctypes.c_int), ("softmax_scale", ctypes.c_float),
+                ("timeout_ms", ctypes.c_uint), ("debug_flags", ctypes.c_uint)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libsa.so and declare its signatures.  Raises when the library is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libsa.so not built at {path}; run `python -m block_sparse_attention_cubes_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(Params)
+    vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    sig = {
+        "sa_padded_tokens": (i32, [P]),
+        "sa_num_cubes": (i32, [P]),
+        "sa_topk_from_fraction": (i32, [ctypes.c_double, i32]),
+        "sa_workspace_size": (sz, [P, i32]),
+        "sa_tile": (i32, [vp, vp, P, i32, vp]),
+        "sa_untile": (i32, [vp, vp, P, i32, vp]),
+        "sa_plan": (i32, [vp, vp, vp, vp, P, vp, vp, vp, sz, vp]),
+        "sa_forward": (i32, [vp, vp, vp, vp, vp, vp, vp, P, vp, vp, vp, sz, vp]),
+        "sa_backward": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, P, vp, vp, vp, vp, sz, vp]),
+        "sa_get_device_status": (i32, [vp, vp]),
+        "sa_status_string": (ctypes.c_char_p, [i32]),
+        "sa_last_launch_count": (i32, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype, f.argtypes = res, args
+    _lib = lib
+    return lib
+
+
+def make_params(B: int, H: int, D: int, lat, top_k: int, top_p: float, kv_capacity: int | None = None,
+                qk_dtype: int = BF16, softmax_scale: float = 0.0, timeout_ms: int = 0, debug_flags: int = 0) -> Params:
+    lt, lh, lw = lat
+    T = math.ceil(lt / 4) * math.ceil(lh / 4) * math.ceil(lw / 4)
+    cap = T if kv_capacity is None else kv_capacity
+    return Params(B, H, D, lt, lh, lw, top_k, top_p, cap, qk_dtype, softmax_scale, timeout_ms, debug_flags)
+
+
+def geometry(p: Params):
+    """(Npad, T) for the parameters."""
+    lib = load_library()
+    return lib.sa_padded_tokens(ctypes.byref(p)), lib.sa_num_cubes(ctypes.byref(p))
+
+
+def workspace_size(p: Params, op: int) -> int:
+    return int(load_library().sa_workspace_size(ctypes.byref(p), op))
+
+
+def last_launch_count() -> int:
+    return int(load_library().sa_last_launch_count())
+
+
+def _torch():
+    import torch
+    if not torch.cuda.is_available():
+        raise RuntimeError("libsa needs a CUDA device; there is no CPU path")
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != SA_OK:
+        raise SAError(status, what)
+
+
+def _contig(t, name, dtype=None, device=None):
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    return t
+
+
+def new_workspace(p: Params, op: int, device=None):
+    torch = _torch()
+    return torch.empty(max(workspace_size(p, op), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def device_status(ws, stream=None) -> int:
+    """Synchronise the stream and return the status recorded in the workspace (0 = SA_OK)."""
+    return int(load_library().sa_get_device_status(_ptr(ws), _stream(stream)))
+
+
+def tile(x, p: Params, out=None, stream=None):
+    """Latent ``[B,H,L,D]`` -> cube-major ``[B,H,Npad,D]`` (same dtype, padding zero)."""
+    torch = _torch()
+    _contig(x, "x")
+    npad, _ = geometry(p)
+    if out is None:
+        out = torch.empty((p.B, p.H, npad, x.shape[-1]), dtype=x.dtype, device=x.device)
+    q = Params.from_buffer_copy(p)
+    q.D = x.shape[-1]
+    _check(load_library().sa_tile(_ptr(x), _ptr(out), ctypes.byref(q), x.element_size(), _stream(stream)), "sa_tile")
+    return out
+
+
+def untile(y, p: Params, out=None, stream=None):
+    torch = _torch()
+    _contig(y, "y")
+    L = p.lat_t * p.lat_h * p.lat_w
+    if out is None:
+        out = torch.empty((p.B, p.H, L, y.shape[-1]), dtype=y.dtype, device=y.device)
+    q = Params.from_buffer_copy(p)
+    q.D = y.shape[-1]
+    _check(load_library().sa_untile(_ptr(y), _ptr(out), ctypes.byref(q), y.element_size(), _stream(stream)),
+           "sa_untile")
+    return out
+
+
+def plan(q, k, p: Params, q_scale=None, k_scale=None, kv_index=None, kv_count=None, ws=None, stream=None):
+    """Router: returns (kv_index [B,H,T,cap] int32, kv_count [B,H,T] int32)."""
+    torch = _torch()
+    _contig(q, "q")
+    _contig(k, "k")
+    _, T = geometry(p)
+    dev = q.device
+    if kv_index is None:
+        kv_index = torch.empty((p.B, p.H, T, p.kv_capacity), dtype=torch.int32, device=dev)
+    if kv_count is None:
+        kv_count = torch.empty((p.B, p.H, T), dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = new_workspace(p, OP_PLAN, dev)
+    st = load_library().sa_plan(_ptr(q), _ptr(k), _ptr(q_scale), _ptr(k_scale), ctypes.byref(p), _ptr(kv_index),
+                                _ptr(kv_count), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "sa_plan")
+    return kv_index, kv_count
+
+
+def forward(q, k, v, kv_index, kv_count, p: Params, q_scale=None, k_scale=None, out=None, lse=None, ws=None,
+            stream=None):
+    """Fine stage forward: returns (out [B,H,Npad,D] bf16, lse [B,H,Npad] fp32)."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (kv_index, "kv_index"), (kv_count, "kv_count")):
+        _contig(t, n)
+    npad, _ = geometry(p)
+    dev = q.device
+    if out is None:
+        out = torch.empty((p.B, p.H, npad, p.D), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((p.B, p.H, npad), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = new_workspace(p, OP_FORWARD, dev)
+    st = load_library().sa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(q_scale), _ptr(k_scale), _ptr(kv_index),
+                                   _ptr(kv_count), ctypes.byref(p), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                   _stream(stream))
+    _check(st, "sa_forward")
+    return out, lse
+
+
+def backward(q, k, v, out, lse, dout, kv_index, kv_count, p: Params, dq=None, dk=None, dv=None, ws=None,
+             stream=None):
+    """Fine stage backward: returns (dq, dk, dv), each [B,H,Npad,D] fp32."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (lse, "lse"), (dout, "dout"),
+                 (kv_index, "kv_index"), (kv_count, "kv_count")):
+        _contig(t, n)
+    dev = q.device
+    shape = tuple(q.shape)
+    dq = torch.empty(shape, dtype=torch.float32, device=dev) if dq is None else dq
+    dk = torch.empty(shape, dtype=torch.float32, device=dev) if dk is None else dk
+    dv = torch.empty(shape, dtype=torch.float32, device=dev) if dv is None else dv
+    if ws is None:
+        ws = new_workspace(p, OP_BACKWARD, dev)
+    st = load_library().sa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(kv_index),
+                                    _ptr(kv_count), ctypes.byref(p), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                                    ws.numel(), _stream(stream))
+    _check(st, "sa_backward")
+    return dq, dk, dv
+
+
+@dataclass
+class Attention:
+    """Router + fine stage with buffers kept between calls (one layer's worth)."""
+    params: Params
+
+    def __post_init__(self):
+        self._ws = {}
+
+    def _w(self, op, dev):
+        if op not in self._ws:
+            self._ws[op] = new_workspace(self.params, op, dev)
+        return self._ws[op]
+
+    def plan(self, q, k, q_scale=None, k_scale=None):
+        return plan(q, k, self.params, q_scale, k_scale, ws=self._w(OP_PLAN, q.device))
+
+    def forward(self, q, k, v, kv_index, kv_count, q_scale=None, k_scale=None):
+        return forward(q, k, v, kv_index, kv_count, self.params, q_scale, k_scale, ws=self._w(OP_FORWARD, q.device))
+
+    def backward(self, q, k, v, out, lse, dout, kv_index, kv_count):
+        return backward(q, k, v, out, lse, dout, kv_index, kv_count, self.params, ws=self._w(OP_BACKWARD, q.device))

@@ -1,0 +1,317 @@
+// C ABI of libsa: argument validation, workspace carving, TMA descriptors and launches.
+// Every check here runs on the host before anything is launched.
+#include <cmath>
+#include <cstring>
+
+#include "../../include/sa.h"
+#include "attn_common.cuh"
+#include "kernels.h"
+
+namespace {
+
+using sa::Geom;
+
+thread_local int g_last_launches = 0;
+
+constexpr size_t kHeader = 256;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool make_geom(const sa_params* p, Geom* g) {
+  if (!p || p->lat_t < 1 || p->lat_h < 1 || p->lat_w < 1) return false;
+  g->lat_t = p->lat_t;
+  g->lat_h = p->lat_h;
+  g->lat_w = p->lat_w;
+  g->Nt = (p->lat_t + 3) / 4;
+  g->Nh = (p->lat_h + 3) / 4;
+  g->Nw = (p->lat_w + 3) / 4;
+  const long long T = static_cast<long long>(g->Nt) * g->Nh * g->Nw;
+  if (T > (1 << 20)) return false;
+  g->T = static_cast<int>(T);
+  g->Npad = g->T * 64;
+  return true;
+}
+
+// Shape checks common to all ops.
+sa_status check_params(const sa_params* p, Geom* g) {
+  if (!p) return SA_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || !make_geom(p, g)) return SA_ERR_INVALID_ARG;
+  if (p->D != 64 && p->D != 128) return SA_ERR_UNSUPPORTED;
+  if (g->T > 8192) return SA_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(p->B) * p->H;
+  if (BH * g->Npad >= (1LL << 31) - 64) return SA_ERR_UNSUPPORTED;
+  if (p->top_k < 0 || !std::isfinite(p->top_p)) return SA_ERR_INVALID_ARG;
+  if (p->kv_capacity < 1 || p->kv_capacity > g->T) return SA_ERR_INVALID_ARG;
+  if (BH * g->T * static_cast<long long>(p->kv_capacity) >= (1LL << 31)) return SA_ERR_UNSUPPORTED;
+  if (p->qk_dtype != SA_BF16 && p->qk_dtype != SA_FP8_E4M3) return SA_ERR_INVALID_ARG;
+  if (!std::isfinite(p->softmax_scale) || p->softmax_scale < 0.0f) return SA_ERR_INVALID_ARG;
+  return SA_OK;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
+
+double softmax_scale(const sa_params* p) {
+  return p->softmax_scale > 0.0f ? static_cast<double>(p->softmax_scale) : 1.0 / std::sqrt(static_cast<double>(p->D));
+}
+
+struct WsLayout {
+  size_t qbar = 0, kbar = 0, scores = 0;                   // plan
+  size_t delta = 0, qcnt = 0, qoff = 0, qidx = 0;          // backward
+  size_t total = 0;
+};
+
+WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
+  WsLayout w;
+  const size_t BH = static_cast<size_t>(p->B) * p->H;
+  size_t off = kHeader;
+  if (op == SA_OP_PLAN) {
+    w.qbar = off;
+    off = align256(off + BH * g.T * p->D * sizeof(double));
+    w.kbar = off;
+    off = align256(off + BH * g.T * p->D * sizeof(double));
+    w.scores = off;
+    off = align256(off + BH * g.T * static_cast<size_t>(g.T) * sizeof(double));
+  } else if (op == SA_OP_BACKWARD) {
+    w.delta = off;
+    off = align256(off + BH * g.Npad * sizeof(float));
+    w.qcnt = off;
+    off = align256(off + BH * g.T * sizeof(int32_t));
+    w.qoff = off;
+    off = align256(off + BH * (g.T + 1) * sizeof(int32_t));
+    w.qidx = off;
+    off = align256(off + BH * g.T * static_cast<size_t>(p->kv_capacity) * sizeof(int32_t));
+  }
+  w.total = off;
+  return w;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D map over [rows][D] elements with 64-row boxes of 128 bytes, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int D, int esize) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const CUtensorMapDataType dt = esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * esize};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 64};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+sa_status reset_status(void* ws, cudaStream_t s) {
+  return cudaMemsetAsync(ws, 0, kHeader, s) == cudaSuccess ? SA_OK : SA_ERR_LAUNCH;
+}
+
+sa::AttnArgs base_args(const sa_params* p, const Geom& g, void* ws) {
+  sa::AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.g = g;
+  a.BH = p->B * p->H;
+  a.D = p->D;
+  a.cap = p->kv_capacity;
+  a.rows_total = a.BH * g.Npad;
+  const double sc = softmax_scale(p);
+  a.scale = static_cast<float>(sc);
+  a.scale_log2 = static_cast<float>(sc * 1.4426950408889634);
+  const unsigned ms = p->timeout_ms ? p->timeout_ms : 2000u;
+  a.timeout_ns = static_cast<unsigned long long>(ms) * 1000000ull;
+  a.debug = p->debug_flags;
+  a.st = static_cast<sa::DevStatus*>(ws);
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sa_padded_tokens(const sa_params* p) {
+  Geom g;
+  return make_geom(p, &g) ? g.Npad : 0;
+}
+
+int sa_num_cubes(const sa_params* p) {
+  Geom g;
+  return make_geom(p, &g) ? g.T : 0;
+}
+
+int sa_topk_from_fraction(double frac, int T) {
+  if (!(frac >= 0.0) || T < 0) return 0;
+  return static_cast<int>(std::ceil(frac * T - 1e-12));
+}
+
+size_t sa_workspace_size(const sa_params* p, int op) {
+  Geom g;
+  if (check_params(p, &g) != SA_OK || op < 0 || op > 2) return 0;
+  return ws_layout(p, g, op).total;
+}
+
+static sa_status tile_common(const void* src, void* dst, const sa_params* p, int elem_bytes, sa_stream_t stream,
+                             bool to_tiled) {
+  Geom g;
+  g_last_launches = 0;
+  if (!p || !src || !dst || p->B < 1 || p->H < 1 || !make_geom(p, &g)) return SA_ERR_INVALID_ARG;
+  if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4) return SA_ERR_INVALID_ARG;
+  if (p->D < 1) return SA_ERR_INVALID_ARG;
+  const int row_bytes = p->D * elem_bytes;
+  if (row_bytes % 16 != 0) return SA_ERR_UNSUPPORTED;
+  if (!aligned16(src) || !aligned16(dst)) return SA_ERR_ALIGNMENT;
+  if (sa::launch_tile(src, dst, g, p->B * p->H, row_bytes, to_tiled, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return SA_ERR_LAUNCH;
+  g_last_launches = 1;
+  return SA_OK;
+}
+
+sa_status sa_tile(const void* x_latent, void* x_tiled, const sa_params* p, int elem_bytes, sa_stream_t stream) {
+  return tile_common(x_latent, x_tiled, p, elem_bytes, stream, true);
+}
+
+sa_status sa_untile(const void* x_tiled, void* x_latent, const sa_params* p, int elem_bytes, sa_stream_t stream) {
+  return tile_common(x_tiled, x_latent, p, elem_bytes, stream, false);
+}
+
+sa_status sa_plan(const void* q, const void* k, const float* q_scale, const float* k_scale, const sa_params* p,
+                  int32_t* kv_index, int32_t* kv_count, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  Geom g;
+  g_last_launches = 0;
+  sa_status s = check_params(p, &g);
+  if (s != SA_OK) return s;
+  if (!q || !k || !kv_index || !kv_count) return SA_ERR_INVALID_ARG;
+  const bool fp8 = p->qk_dtype == SA_FP8_E4M3;
+  if (fp8 && (!q_scale || !k_scale)) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned4(kv_index) || !aligned4(kv_count)) return SA_ERR_ALIGNMENT;
+  if (fp8 && (!aligned4(q_scale) || !aligned4(k_scale))) return SA_ERR_ALIGNMENT;
+  const WsLayout w = ws_layout(p, g, SA_OP_PLAN);
+  if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SA_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  int launches = 0;
+  if (sa::launch_plan(q, k, q_scale, k_scale, g, p->B * p->H, p->D, fp8, softmax_scale(p), p->top_k, p->top_p,
+                      p->kv_capacity, kv_index, kv_count, reinterpret_cast<double*>(wb + w.qbar),
+                      reinterpret_cast<double*>(wb + w.kbar), reinterpret_cast<double*>(wb + w.scores),
+                      static_cast<sa::DevStatus*>(ws), st, &launches) != cudaSuccess)
+    return SA_ERR_LAUNCH;
+  g_last_launches = launches;
+  return SA_OK;
+}
+
+sa_status sa_forward(const void* q, const void* k, const void* v, const float* q_scale, const float* k_scale,
+                     const int32_t* kv_index, const int32_t* kv_count, const sa_params* p, void* out, float* lse,
+                     void* ws, size_t ws_bytes, sa_stream_t stream) {
+  Geom g;
+  g_last_launches = 0;
+  sa_status s = check_params(p, &g);
+  if (s != SA_OK) return s;
+  if (!q || !k || !v || !kv_index || !kv_count || !out || !lse) return SA_ERR_INVALID_ARG;
+  if (p->qk_dtype == SA_FP8_E4M3) return SA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(lse) || !aligned4(kv_index) ||
+      !aligned4(kv_count))
+    return SA_ERR_ALIGNMENT;
+  const WsLayout w = ws_layout(p, g, SA_OP_FORWARD);
+  if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SA_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  sa::AttnArgs a = base_args(p, g, ws);
+  a.kv_index = kv_index;
+  a.kv_count = kv_count;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, a.rows_total, p->D, 2) || !make_map(&tk, k, a.rows_total, p->D, 2) ||
+      !make_map(&tv, v, a.rows_total, p->D, 2))
+    return SA_ERR_LAUNCH;
+  if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
+  if (sa::launch_forward(tq, tk, tv, a, st) != cudaSuccess) return SA_ERR_LAUNCH;
+  g_last_launches = 1;
+  return SA_OK;
+}
+
+sa_status sa_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                      const void* dout, const int32_t* kv_index, const int32_t* kv_count, const sa_params* p,
+                      float* dq, float* dk, float* dv, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  Geom g;
+  g_last_launches = 0;
+  sa_status s = check_params(p, &g);
+  if (s != SA_OK) return s;
+  if (!q || !k || !v || !out || !lse || !dout || !kv_index || !kv_count || !dq || !dk || !dv)
+    return SA_ERR_INVALID_ARG;
+  if (p->qk_dtype != SA_BF16) return SA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned4(lse) || !aligned4(kv_index) || !aligned4(kv_count))
+    return SA_ERR_ALIGNMENT;
+  const WsLayout w = ws_layout(p, g, SA_OP_BACKWARD);
+  if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SA_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  sa::AttnArgs a = base_args(p, g, ws);
+  a.kv_index = kv_index;
+  a.kv_count = kv_count;
+  a.lse = const_cast<float*>(lse);
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map(&tq, q, a.rows_total, p->D, 2) || !make_map(&tk, k, a.rows_total, p->D, 2) ||
+      !make_map(&tv, v, a.rows_total, p->D, 2) || !make_map(&tdo, dout, a.rows_total, p->D, 2))
+    return SA_ERR_LAUNCH;
+  if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  int launches = 0;
+  if (sa::launch_backward(tq, tk, tv, tdo, out, dout, a, reinterpret_cast<int32_t*>(wb + w.qcnt),
+                          reinterpret_cast<int32_t*>(wb + w.qoff), reinterpret_cast<int32_t*>(wb + w.qidx),
+                          reinterpret_cast<float*>(wb + w.delta), st, &launches) != cudaSuccess)
+    return SA_ERR_LAUNCH;
+  g_last_launches = launches;
+  return SA_OK;
+}
+
+sa_status sa_get_device_status(const void* ws, sa_stream_t stream) {
+  if (!ws) return SA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SA_ERR_LAUNCH;
+  sa::DevStatus h;
+  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return SA_ERR_LAUNCH;
+  if (h.error & sa::DEVERR_TIMEOUT) return SA_ERR_DEVICE_TIMEOUT;
+  if (h.error & sa::DEVERR_INDEX) return SA_ERR_DEVICE_INDEX;
+  if (h.error & sa::DEVERR_CAPACITY) return SA_ERR_CAPACITY;
+  return SA_OK;
+}
+
+const char* sa_status_string(sa_status s) {
+  switch (s) {
+    case SA_OK: return "ok";
+    case SA_ERR_INVALID_ARG: return "invalid argument";
+    case SA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case SA_ERR_CAPACITY: return "a row selected more blocks than kv_capacity";
+    case SA_ERR_WORKSPACE: return "workspace missing or too small";
+    case SA_ERR_LAUNCH: return "CUDA launch or driver call failed";
+    case SA_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel timed out";
+    case SA_ERR_DEVICE_INDEX: return "kv_index entry or kv_count out of range";
+  }
+  return "unknown status";
+}
+
+int sa_last_launch_count(void) { return g_last_launches; }
+
+}  // extern "C"

@@ -1,0 +1,141 @@
+// Pieces shared by the fine-stage kernels (forward, dQ, dK/dV).
+#pragma once
+#include <cuda_bf16.h>
+
+#include "geometry.cuh"
+#include "ptx.cuh"
+
+namespace sa {
+
+struct AttnArgs {
+  const int32_t* kv_index;  // [BH, T, cap]
+  const int32_t* kv_count;  // [BH, T]
+  const float* q_scale;     // [BH, T] (fp8 only)
+  const float* k_scale;
+  __nv_bfloat16* out;       // forward output [BH, Npad, D]
+  float* lse;               // [BH, Npad]
+  const float* delta;       // backward: rowsum(dO * O) [BH, Npad]
+  const int32_t* q_off;     // backward: transposed lists, CSR offsets [BH, T+1]
+  const int32_t* q_idx;     // backward: transposed lists, entries
+  float* dq;
+  float* dk;
+  float* dv;
+  DevStatus* st;
+  Geom g;
+  int BH, D, cap;
+  int rows_total;           // BH * Npad, the first out-of-range row for zero-filled loads
+  float scale;              // softmax scale
+  float scale_log2;         // softmax scale * log2(e)
+  unsigned long long timeout_ns;
+  unsigned int debug;
+};
+
+// Block id t of query block i's list, or -1 when t is past the count or the entry is
+// out of range (the latter is recorded as an index error).
+__device__ __forceinline__ int list_entry(const AttnArgs& a, int bh, int i, int n, int t, bool report) {
+  if (t >= n) return -1;
+  const int j = __ldg(a.kv_index + (static_cast<size_t>(bh) * a.g.T + i) * a.cap + t);
+  if (j < 0 || j >= a.g.T) {
+    if (report) flag_error(a.st, DEVERR_INDEX, 0);
+    return -1;
+  }
+  return j;
+}
+
+__device__ __forceinline__ int list_count(const AttnArgs& a, int bh, int i, bool report) {
+  int n = __ldg(a.kv_count + static_cast<size_t>(bh) * a.g.T + i);
+  if (n < 0 || n > a.cap) {
+    if (report) flag_error(a.st, DEVERR_INDEX, 0);
+    n = n < 0 ? 0 : a.cap;
+  }
+  return n;
+}
+
+struct OpMax {
+  __device__ __forceinline__ float operator()(float a, float b) const { return fmaxf(a, b); }
+};
+struct OpSum {
+  __device__ __forceinline__ float operator()(float a, float b) const { return a + b; }
+};
+
+// Reduce 64 per-thread column values over the 32 lanes of a warp by recursive halving:
+// at the end lane l holds columns c0, c0+1 with c0 = 32*b4 + 16*b3 + 8*b2 + 4*b1 + 2*b0
+// (b = bits of l) in v[0], v[1].  62 shuffles instead of 64 x 5.
+template <class Op>
+__device__ __forceinline__ int warp_colreduce64(float (&v)[64], int lane, Op op) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const bool hi = lane & 16;
+    const float send = hi ? v[i] : v[i + 32];
+    const float keep = hi ? v[i + 32] : v[i];
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const bool hi = lane & 8;
+    const float send = hi ? v[i] : v[i + 16];
+    const float keep = hi ? v[i + 16] : v[i];
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool hi = lane & 4;
+    const float send = hi ? v[i] : v[i + 8];
+    const float keep = hi ? v[i + 8] : v[i];
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool hi = lane & 2;
+    const float send = hi ? v[i] : v[i + 4];
+    const float keep = hi ? v[i + 4] : v[i];
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool hi = lane & 1;
+    const float send = hi ? v[i] : v[i + 2];
+    const float keep = hi ? v[i + 2] : v[i];
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 1));
+  }
+  return 32 * ((lane >> 4) & 1) + 16 * ((lane >> 3) & 1) + 8 * ((lane >> 2) & 1) + 4 * ((lane >> 1) & 1) +
+         2 * (lane & 1);
+}
+
+// Store one 64-element bf16 row (128 bytes) of a 128-byte-swizzled tile.
+__device__ __forceinline__ void store_row_bf16_sw128(uint32_t tile_base, uint32_t row, const float (&v)[64]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t a = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
+    const uint32_t b = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+    const uint32_t cc = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+    const uint32_t d = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+    st_shared_v4(tile_base + sw128_offset(row, c), a, b, cc, d);
+  }
+}
+
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r0[32], r1[32];
+  tmem_ld32(taddr, r0);
+  tmem_ld32(taddr + 32, r1);
+  tmem_ld_wait();
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    v[c] = __uint_as_float(r0[c]);
+    v[c + 32] = __uint_as_float(r1[c]);
+  }
+}
+
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const float (&v)[64]) {
+  uint32_t r0[32], r1[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    r0[c] = __float_as_uint(v[c]);
+    r1[c] = __float_as_uint(v[c + 32]);
+  }
+  tmem_st32(taddr, r0);
+  tmem_st32(taddr + 32, r1);
+  tmem_st_wait();
+}
+
+}  // namespace sa

@@ -1,0 +1,30 @@
+// Launch functions of the library's kernels (host side, internal).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "geometry.cuh"
+
+namespace sa {
+
+struct DevStatus;
+struct AttnArgs;
+
+cudaError_t launch_tile(const void* src, void* dst, const Geom& g, int BH, int row_bytes, bool to_tiled,
+                        cudaStream_t stream);
+
+cudaError_t launch_plan(const void* q, const void* k, const float* q_scale, const float* k_scale, const Geom& g,
+                        int BH, int D, bool fp8, double scale, int top_k, float top_p, int cap, int32_t* kv_index,
+                        int32_t* kv_count, double* qbar, double* kbar, double* S, DevStatus* st,
+                        cudaStream_t stream, int* launches);
+
+cudaError_t launch_forward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
+                           cudaStream_t stream);
+
+cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const void* out, const void* dout, AttnArgs a, int32_t* qcnt,
+                            int32_t* qoff, int32_t* qidx, float* delta, cudaStream_t stream, int* launches);
+
+}  // namespace sa

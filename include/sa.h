@@ -1,0 +1,153 @@
+/*
+ * sa.h - C ABI of the cube-routed block-sparse attention library (libsa.so, sm_100a).
+ *
+ * The method: a coarse router mean-pools Q and K over 4x4x4 cubes of 64 tokens, scores
+ * every (query cube, key cube) pair, applies a row softmax and keeps the union of the
+ * Top-k and Top-p key cubes of each query cube (SpargeAttention2 page, "Block-Pooled
+ * Attention for Efficient Mask Construction" and "The Hybrid Top-k+Top-p Masking Rule",
+ * equation 9).  A fine stage then runs softmax attention over only the selected 64x64
+ * tiles, forward and backward (SpargeAttention2 page, "Kernel Implementation of the
+ * Hybrid-Masked Block-Sparse Attention"; VSA page, "The Fine Stage").
+ *
+ * Conventions shared by every entry point
+ *  - All tensor arguments are DEVICE pointers owned by the caller.  The library never
+ *    allocates or frees device memory and never synchronises, except where stated.
+ *  - Token tensors are contiguous [B, H, Npad, D] in cube-major padded order (see
+ *    sa_tile), Npad = 64 * N_t * N_h * N_w with N_x = ceil(lat_x / 4).  Row pitch is
+ *    D elements; base pointers must be 16-byte aligned.
+ *  - T = N_t * N_h * N_w is the number of cubes (query blocks = key blocks).
+ *  - Every launch is asynchronous on `stream` (a cudaStream_t; NULL = legacy stream).
+ *  - Host-side argument errors are returned synchronously before anything is
+ *    launched.  Problems found on the device (a bounded wait that timed out, an index
+ *    list entry out of range, too many selected blocks for kv_capacity) are recorded in
+ *    the status block at the start of the workspace and read with
+ *    sa_get_device_status.  Every entry point that takes a workspace clears that block
+ *    first, so the status reports the most recent call on that workspace.
+ */
+#ifndef SA_H_
+#define SA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SA_API __attribute__((visibility("default")))
+#else
+#define SA_API
+#endif
+
+typedef struct CUstream_st* sa_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,    /* null pointer, bad shape, k < 0, p not finite, ... */
+  SA_ERR_UNSUPPORTED = 2,    /* a valid request outside what is built (e.g. D not in {64,128}) */
+  SA_ERR_ALIGNMENT = 3,      /* a pointer not aligned to 16 bytes */
+  SA_ERR_CAPACITY = 4,       /* device: a row selected more than kv_capacity blocks */
+  SA_ERR_WORKSPACE = 5,      /* ws == NULL or ws_bytes < sa_workspace_size(...) */
+  SA_ERR_LAUNCH = 6,         /* a CUDA launch or driver call failed */
+  SA_ERR_DEVICE_TIMEOUT = 7, /* device: a bounded wait inside a kernel gave up */
+  SA_ERR_DEVICE_INDEX = 8    /* device: a kv_index entry outside [0,T) or a count outside [0,cap] */
+} sa_status;
+
+typedef enum { SA_BF16 = 0, SA_FP8_E4M3 = 1 } sa_qk_dtype;
+
+typedef enum { SA_OP_PLAN = 0, SA_OP_FORWARD = 1, SA_OP_BACKWARD = 2 } sa_op;
+
+typedef struct {
+  int B, H, D;                /* batch, heads, head dim (D in {64, 128}) */
+  int lat_t, lat_h, lat_w;    /* valid latent grid, e.g. 21, 45, 80 */
+  int top_k;                  /* Top-k block count, >= 0 (clamped to T); see sa_topk_from_fraction */
+  float top_p;                /* Top-p mass fraction; >= 1 keeps every block, <= 0 adds none */
+  int kv_capacity;            /* row stride of kv_index; 1 <= kv_capacity <= T */
+  int qk_dtype;               /* sa_qk_dtype; SA_FP8_E4M3 needs q_scale / k_scale */
+  float softmax_scale;        /* 0 -> 1/sqrt(D) */
+  unsigned int timeout_ms;    /* bound of every in-kernel wait; 0 -> 2000 ms */
+  unsigned int debug_flags;   /* 0 in normal use; SA_DEBUG_* below */
+} sa_params;
+
+/* Test hook: the forward kernel's producer issues no loads, so its consumers' bounded
+ * waits run out and the call reports SA_ERR_DEVICE_TIMEOUT without faulting. */
+#define SA_DEBUG_SKIP_LOADS 1u
+
+/* Padded token count Npad and cube count T implied by the latent grid (0 on bad input). */
+SA_API int sa_padded_tokens(const sa_params* p);
+SA_API int sa_num_cubes(const sa_params* p);
+
+/* ceil(frac * T): SpargeAttention2's k% rule ("Definition of the two component
+ * selectors": the largest ceil(k% x T_n) entries). */
+SA_API int sa_topk_from_fraction(double frac, int T);
+
+/* Bytes of device workspace `op` (sa_op) needs for these parameters; 0 on bad input.
+ * Plan: status block + pooled Q and K (fp64) + block scores (fp64, B*H*T*T).
+ * Forward: status block.  Backward: status block + Delta (fp32, B*H*Npad) + the
+ * transposed index lists (int32, B*H*(2T+1) + B*H*T*kv_capacity). */
+SA_API size_t sa_workspace_size(const sa_params* p, int op);
+
+/* Layout helper (VSA page, "Cube Partitioning and Token Re-Indexing"; VSA2 page,
+ * section 2.2 "Permutation" and "Kernel Implementation" for padding).
+ * x_latent: [B, H, lat_t*lat_h*lat_w, D] row-major (t, h, w) token order.
+ * x_tiled:  [B, H, Npad, D] cube-major; token (t,h,w) goes to slot
+ *   ((t/4)*N_h*N_w + (h/4)*N_w + w/4)*64 + (t%4)*16 + (h%4)*4 + (w%4); padding slots are 0.
+ * elem_bytes is 1, 2 or 4.  sa_untile is the inverse (padding dropped). */
+SA_API sa_status sa_tile(const void* x_latent, void* x_tiled, const sa_params* p, int elem_bytes, sa_stream_t stream);
+SA_API sa_status sa_untile(const void* x_tiled, void* x_latent, const sa_params* p, int elem_bytes, sa_stream_t stream);
+
+/* Router (SpargeAttention2 page, "Block-Pooled Attention", steps 2-4, and equation 9;
+ * VSA page, "Kernel Implementation": contiguous arrays of block indices).
+ * q, k: [B,H,Npad,D] bf16, or e4m3 bytes when qk_dtype == SA_FP8_E4M3, in which case
+ *   q_scale, k_scale are [B,H,T] fp32 (value = code * scale of its cube); else NULL.
+ * Pooling averages the valid tokens of each cube; scores are Qbar Kbar^T * scale; the
+ * row softmax, Top-k (top_k largest) and Top-p (shortest prefix of the descending order
+ * whose mass reaches top_p of the row) are taken in that order, ties broken by the
+ * smaller block id, and at least one block is kept.
+ * Outputs: kv_count [B,H,T] int32 = number of kept blocks (clipped to kv_capacity, with
+ * SA_ERR_CAPACITY recorded when clipping happened); kv_index [B,H,T,kv_capacity] int32
+ * holds the kept block ids in ascending order in its first kv_count entries (the rest
+ * are left untouched).  Deterministic. */
+SA_API sa_status sa_plan(const void* q, const void* k, const float* q_scale, const float* k_scale, const sa_params* p,
+                  int32_t* kv_index, int32_t* kv_count, void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* Fine stage forward (SpargeAttention2 page, "Kernel Implementation", online softmax;
+ * VSA2 page 2.1, O = softmax(QK^T/sqrt(D) + M) V with M = 0 on selected 64x64 tiles,
+ * -inf elsewhere and on padding keys).
+ * q, k: as for sa_plan; v: [B,H,Npad,D] bf16; kv_index/kv_count: as written by sa_plan
+ *   (entries must lie in [0,T), counts in [0,kv_capacity]; violations are recorded as
+ *   SA_ERR_DEVICE_INDEX and the offending entries skipped).
+ * out: [B,H,Npad,D] bf16; lse: [B,H,Npad] fp32, natural log of each row's softmax
+ * normaliser of the scaled scores.  Padding query rows get out = 0, lse = 0; a row with
+ * count 0 gets out = 0, lse = -inf.  Deterministic. */
+SA_API sa_status sa_forward(const void* q, const void* k, const void* v, const float* q_scale, const float* k_scale,
+                     const int32_t* kv_index, const int32_t* kv_count, const sa_params* p, void* out, float* lse,
+                     void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* Fine stage backward with the block mask held constant (VSA2 page 2.1: the router's
+ * output carries no gradient).  Inputs as for sa_forward plus out and lse from it and
+ * dout [B,H,Npad,D] bf16.  Outputs dq, dk, dv: [B,H,Npad,D] fp32:
+ *   P = exp(scale*QK^T - lse), dV = P^T dO, dP = dO V^T, Delta = rowsum(dO * O),
+ *   dS = P * (dP - Delta), dQ = scale * dS K, dK = scale * dS^T Q.
+ * Padding rows of every output are 0; dout of padding rows is ignored.
+ * bf16 only (qk_dtype must be SA_BF16).  Deterministic. */
+SA_API sa_status sa_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                      const void* dout, const int32_t* kv_index, const int32_t* kv_count, const sa_params* p,
+                      float* dq, float* dk, float* dv, void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* Synchronises `stream`, then maps the workspace's device status block to a status:
+ * SA_OK, SA_ERR_DEVICE_TIMEOUT, SA_ERR_DEVICE_INDEX or SA_ERR_CAPACITY (first that
+ * applies, in that order of precedence: timeout, index, capacity). */
+SA_API sa_status sa_get_device_status(const void* ws, sa_stream_t stream);
+
+SA_API const char* sa_status_string(sa_status s);
+
+/* Number of kernels the most recent call of each entry point launched on this host
+ * thread (for launch accounting in benchmarks). */
+SA_API int sa_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SA_H_ */

@@ -1,0 +1,88 @@
+"""The C ABI library loads and exports every symbol include/sa.h declares; host-side
+validation answers without touching a GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_cubes_b200 as sa
+from block_sparse_attention_cubes_b200 import build as sa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sa_build.build()
+    return sa.load_library()
+
+
+def test_header_declares_exactly_the_exports(lib):
+    hdr = open(os.path.join(ROOT, "include", "sa.h")).read()
+    declared = set(re.findall(r"SA_API\s+[\w\s\*]+?\b(sa_\w+)\s*\(", hdr))
+    assert declared == set(sa.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_exported_dynamic_symbols(lib):
+    out = os.popen(f"nm -D --defined-only {sa.LIB_PATH}").read()
+    for name in sa.EXPORTS:
+        assert re.search(rf"\bT {name}\b", out), name
+
+
+def test_geometry_and_workspace(lib):
+    p = sa.make_params(1, 40, 128, (21, 45, 80), 44, 0.9)
+    assert sa.geometry(p) == (92160, 1440)
+    assert lib.sa_topk_from_fraction(0.03, 1440) == 44
+    assert lib.sa_topk_from_fraction(0.03, 1562) == 47
+    T, BH = 1440, 40
+    plan_ws = sa.workspace_size(p, sa.OP_PLAN)
+    assert plan_ws >= 256 + 2 * BH * T * 128 * 8 + BH * T * T * 8
+    assert sa.workspace_size(p, sa.OP_FORWARD) == 256
+    assert sa.workspace_size(p, sa.OP_BACKWARD) >= BH * 92160 * 4 + BH * T * T * 4
+
+
+def test_host_validation_without_gpu(lib):
+    p = sa.make_params(1, 2, 96, (8, 8, 8), 4, 0.5)          # D = 96 is not built
+    assert sa.workspace_size(p, 0) == 0
+    bad = ctypes.c_void_p(16)
+    st = lib.sa_plan(bad, bad, None, None, ctypes.byref(p), bad, bad, bad, 1 << 20, None)
+    assert st == 2  # SA_ERR_UNSUPPORTED, returned before any launch
+    p = sa.make_params(1, 2, 64, (8, 8, 8), -1, 0.5)
+    assert lib.sa_plan(bad, bad, None, None, ctypes.byref(p), bad, bad, bad, 1 << 20, None) == 1
+    p = sa.make_params(1, 2, 64, (8, 8, 8), 4, float("nan"))
+    assert lib.sa_plan(bad, bad, None, None, ctypes.byref(p), bad, bad, bad, 1 << 20, None) == 1
+    p = sa.make_params(1, 2, 64, (8, 8, 8), 4, 0.5, kv_capacity=9)   # T = 8
+    assert lib.sa_plan(bad, bad, None, None, ctypes.byref(p), bad, bad, bad, 1 << 20, None) == 1
+    p = sa.make_params(1, 2, 64, (8, 8, 8), 4, 0.5)
+    assert lib.sa_plan(None, bad, None, None, ctypes.byref(p), bad, bad, bad, 1 << 20, None) == 1
+    odd = ctypes.c_void_p(24)                                    # 8 bytes off a 16-byte boundary
+    assert lib.sa_plan(odd, bad, None, None, ctypes.byref(p), bad, bad, bad, 1 << 20, None) == 3
+    assert lib.sa_plan(bad, bad, None, None, ctypes.byref(p), bad, bad, bad, 16, None) == 5
+    fp8 = sa.make_params(1, 2, 128, (8, 8, 8), 4, 0.5, qk_dtype=sa.FP8_E4M3)
+    assert lib.sa_plan(bad, bad, None, None, ctypes.byref(fp8), bad, bad, bad, 1 << 30, None) == 1
+    assert lib.sa_status_string(7) == b"a bounded wait inside a kernel timed out"
+    assert lib.sa_last_launch_count() == 0
+
+
+def test_product_path_has_no_cpu_fallback():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    p = sa.make_params(1, 1, 64, (4, 4, 4), 1, 0.5)
+    with pytest.raises(RuntimeError):
+        sa.plan(torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16), torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16), p)
+
+
+def test_package_does_not_import_oracle():
+    import ast
+    pkg = os.path.join(ROOT, "block_sparse_attention_cubes_b200")
+    for fn in os.listdir(pkg):
+        if fn.endswith(".py"):
+            tree = ast.parse(open(os.path.join(pkg, fn)).read())
+            for node in ast.walk(tree):
+                if isinstance(node, (ast.Import, ast.ImportFrom)):
+                    names = [a.name for a in node.names] if isinstance(node, ast.Import) else [node.module or ""]
+                    assert not any(n.split(".")[0] == "oracle" for n in names), fn

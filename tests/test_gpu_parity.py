@@ -1,0 +1,162 @@
+"""CUDA path vs the fp64 oracle on the same seeded inputs, through the C ABI.
+
+Index lists must match bit for bit except tie rows (counted); outputs and gradients
+must be within max-abs 2e-2 and mean-abs 2e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_cubes_b200 as sa
+import oracle as O
+import synth
+from parity import (assert_close, classify_router_rows, gpu_inputs, gpu_lists, lists_to_device, oracle_head)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _need_gpu(cuda_ok):
+    from block_sparse_attention_cubes_b200 import build
+    build.build()
+    yield
+
+
+def _check_layout(cfg, x, tiled):
+    lay = O.cube_layout(cfg.lat)
+    for n, t in tiled.items():
+        ref = O.tile(x[n][0].float().numpy(), lay)
+        assert np.array_equal(t[0].float().cpu().numpy(), ref), n
+        back = sa.untile(t, sa.make_params(cfg.B, t.shape[1], cfg.D, cfg.lat, 1, 0.5))
+        assert torch.equal(back.cpu(), x[n]), n
+
+
+def _router_case(cfg, heads=None, allow_tie_frac=1e-3):
+    x, p, t = gpu_inputs(cfg, names=("q", "k"), heads=heads)
+    idx, cnt = sa.plan(t["q"], t["k"], p)
+    torch.cuda.synchronize()
+    lay = O.cube_layout(cfg.lat)
+    tot_mis, tot_ties, rows = 0, 0, 0
+    for hh in range(p.H):
+        tr = O.route_head(oracle_head(x, "q", 0, hh, lay), oracle_head(x, "k", 0, hh, lay), lay.valid,
+                          cfg.top_k, cfg.top_p)
+        mis, ties, bad = classify_router_rows(tr, gpu_lists(idx, cnt, 0, hh), cfg.top_p)
+        assert mis == 0, f"head {hh}: {mis} mismatching rows, e.g. {bad[:5]}"
+        tot_ties += ties
+        rows += lay.n_cubes
+    assert tot_ties <= max(2, allow_tie_frac * rows)
+    return x, p, t, idx, cnt
+
+
+def test_tile_matches_oracle_layout():
+    cfg = synth.small_config("pad", 1, 2, 64, (5, 6, 7), 2, 0.5)
+    x, p, t = gpu_inputs(cfg, names=("q", "v"))
+    _check_layout(cfg, x, t)
+
+
+@pytest.mark.parametrize("name", ["tiny"])
+def test_router_tiny(name):
+    _router_case(synth.get_config(name))
+
+
+@pytest.mark.parametrize("lat,k,pp", [((4, 4, 4), 1, 0.9), ((5, 8, 12), 3, 0.9), ((8, 8, 8), 0, 0.0),
+                                      ((8, 12, 16), 2, 0.5), ((9, 9, 9), 50, 0.3), ((8, 8, 8), 4, 1.0)])
+def test_router_small_edge(lat, k, pp):
+    _router_case(synth.small_config("e", 1, 2, 128, lat, k, pp))
+
+
+def _fwd_case(cfg, lists_src="oracle", heads=None, q_blocks=None):
+    x, p, t = gpu_inputs(cfg, heads=heads)
+    lay = O.cube_layout(cfg.lat)
+    H = p.H
+    trs = {}
+    for hh in range(H):
+        trs[(0, hh)] = O.route_head(oracle_head(x, "q", 0, hh, lay), oracle_head(x, "k", 0, hh, lay), lay.valid,
+                                    cfg.top_k, cfg.top_p).lists
+    idx, cnt = lists_to_device(trs, 1, H, lay.n_cubes, p.kv_capacity)
+    out, lse = sa.forward(t["q"], t["k"], t["v"], idx, cnt, p)
+    torch.cuda.synchronize()
+    for hh in range(H):
+        q, k, v = (oracle_head(x, n, 0, hh, lay) for n in ("q", "k", "v"))
+        o_ref, lse_ref = O.attention_forward_head(q, k, v, trs[(0, hh)], lay.valid, q_blocks=q_blocks)
+        rows = lay.valid.copy()
+        if q_blocks is not None:
+            m = np.zeros_like(rows)
+            for i in q_blocks:
+                m[i * 64:(i + 1) * 64] = True
+            rows &= m
+        got = out[0, hh].float().cpu().numpy()
+        assert_close(f"out h{hh}", got[rows], o_ref[rows])
+        assert np.all(got[~lay.valid] == 0)
+        gl = lse[0, hh].cpu().numpy()
+        assert np.max(np.abs(gl[rows] - lse_ref[rows])) < 1e-3
+        assert np.all(gl[~lay.valid] == 0)
+    return x, p, t, idx, cnt, out, lse, trs
+
+
+def test_forward_tiny():
+    _fwd_case(synth.get_config("tiny"))
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("lat,k,pp", [((4, 4, 4), 1, 0.9), ((5, 8, 12), 3, 0.9), ((8, 12, 16), 2, 0.5),
+                                      ((9, 9, 9), 50, 0.3), ((8, 8, 8), 8, 1.0)])
+def test_forward_small(D, lat, k, pp):
+    _fwd_case(synth.small_config("f", 1, 2, D, lat, k, pp))
+
+
+def _bwd_case(cfg):
+    x, p, t, idx, cnt, out, lse, trs = _fwd_case(cfg)
+    dq, dk, dv = sa.backward(t["q"], t["k"], t["v"], out, lse, t["do"], idx, cnt, p)
+    torch.cuda.synchronize()
+    lay = O.cube_layout(cfg.lat)
+    for hh in range(p.H):
+        q, k, v, do = (oracle_head(x, n, 0, hh, lay) for n in ("q", "k", "v", "do"))
+        g = O.attention_backward_head(q, k, v, do, trs[(0, hh)], lay.valid)
+        for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), g):
+            a = got[0, hh].cpu().numpy()
+            assert_close(f"{name} h{hh}", a, ref)
+            assert np.all(a[~lay.valid] == 0)
+
+
+def test_backward_tiny():
+    _bwd_case(synth.get_config("tiny"))
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("lat,k,pp", [((4, 4, 4), 1, 0.9), ((5, 8, 12), 3, 0.9), ((8, 12, 16), 2, 0.5),
+                                      ((9, 9, 9), 50, 0.3)])
+def test_backward_small(D, lat, k, pp):
+    _bwd_case(synth.small_config("b", 1, 2, D, lat, k, pp))
+
+
+def test_end_to_end_with_gpu_lists():
+    cfg = synth.small_config("e2e", 1, 4, 128, (8, 16, 20), 4, 0.9)
+    x, p, t, idx, cnt = _router_case(cfg)
+    out, lse = sa.forward(t["q"], t["k"], t["v"], idx, cnt, p)
+    dq, dk, dv = sa.backward(t["q"], t["k"], t["v"], out, lse, t["do"], idx, cnt, p)
+    torch.cuda.synchronize()
+    lay = O.cube_layout(cfg.lat)
+    for hh in range(p.H):
+        lists = gpu_lists(idx, cnt, 0, hh)
+        q, k, v, do = (oracle_head(x, n, 0, hh, lay) for n in ("q", "k", "v", "do"))
+        o_ref, _ = O.attention_forward_head(q, k, v, lists, lay.valid)
+        assert_close("out", out[0, hh].float().cpu().numpy(), o_ref)
+        g = O.attention_backward_head(q, k, v, do, lists, lay.valid)
+        for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), g):
+            assert_close(name, got[0, hh].cpu().numpy(), ref)
+
+
+def test_deterministic_repeat():
+    cfg = synth.small_config("det", 1, 2, 128, (8, 12, 16), 3, 0.9)
+    x, p, t = gpu_inputs(cfg)
+    r1 = sa.plan(t["q"], t["k"], p)
+    r2 = sa.plan(t["q"], t["k"], p)
+    assert torch.equal(r1[1], r2[1]) and torch.equal(r1[0], r2[0])
+    o1 = sa.forward(t["q"], t["k"], t["v"], *r1, p)
+    o2 = sa.forward(t["q"], t["k"], t["v"], *r1, p)
+    assert torch.equal(o1[0], o2[0]) and torch.equal(o1[1], o2[1])
+    g1 = sa.backward(t["q"], t["k"], t["v"], *o1, t["do"], *r1, p)
+    g2 = sa.backward(t["q"], t["k"], t["v"], *o1, t["do"], *r1, p)
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
