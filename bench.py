@@ -1,0 +1,396 @@
+"""Benchmark: one step = router + fine-stage forward + backward (sa_plan, sa_forward,
+sa_backward) at the Wan2.1-14B-720p attention shape, 95% block sparsity.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 720p]
+
+Prints ONE JSON line on rank 0.  ``value`` is effective TFLOP/s over the whole step
+(all ranks' work / max-over-ranks device time), counting only the selected 64x64 tiles:
+forward 4*D*64*64 and backward 10*D*64*64 FLOPs per selected tile (VSA page, FLOP
+accounting: 4 * D * S * H * d * 3.5, i.e. forward 1 + backward 2.5).  Each rank runs an
+independent problem of the same shape (weak scaling, no collective on the data path).
+Inputs are larger than L2 and L2 is also flushed between steps (256 MiB write).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn fwd+bwd ms & effective TFLOPS at Wan-720p shape, 95% sparsity"
+UNIT = "TFLOP/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def tile_flops(D: int, ntiles: int):
+    fwd = 4.0 * D * 64 * 64 * ntiles
+    return fwd, 2.5 * fwd
+
+
+# ---------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out" if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else "",
+                                 f".clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={CLOCK_QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        power = [num(r[3]) for r in rows if num(r[3]) is not None]
+        under_load = [s for s, pw in zip(sm, power) if pw is not None and pw > 300] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(under_load) if under_load else None,
+                "sm_max_mhz": max(num(r[2]) or 0 for r in rows), "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------------- ours
+def run_ours(args, rank, world, dist):
+    import torch
+
+    import block_sparse_attention_cubes_b200 as sa
+    import synth
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = synth.get_config(args.config)
+    t_gen = time.time()
+    host = synth.make_inputs(cfg, seed=rank)
+    t_gen = time.time() - t_gen
+    p = sa.make_params(cfg.B, cfg.H, cfg.D, cfg.lat, cfg.top_k, cfg.top_p)
+    npad, T = sa.geometry(p)
+    x = {n: sa.tile(host[n].to(dev), p) for n in ("q", "k", "v", "do")}
+    A = sa.Attention(p)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    launches = {"n": 0}
+
+    def step(rec=None):
+        if rec is not None:
+            rec[0].record()
+        idx, cnt = A.plan(x["q"], x["k"])
+        launches["n"] += sa.last_launch_count()
+        if rec is not None:
+            rec[1].record()
+        out, lse, out32 = A.forward(x["q"], x["k"], x["v"], idx, cnt)
+        launches["n"] += sa.last_launch_count()
+        if rec is not None:
+            rec[2].record()
+        g = A.backward(x["q"], x["k"], x["v"], out, lse, x["do"], idx, cnt, out_f32=out32)
+        launches["n"] += sa.last_launch_count()
+        if rec is not None:
+            rec[3].record()
+        return idx, cnt, out, lse, g
+
+    for _ in range(args.warmup):
+        idx, cnt, *_ = step()
+    torch.cuda.synchronize()
+    for op in (sa.OP_PLAN, sa.OP_FORWARD, sa.OP_BACKWARD):
+        st = sa.device_status(A._ws[op])
+        if st != 0:
+            raise RuntimeError(f"device status {sa.STATUS_NAMES.get(st, st)} after warm-up")
+    ntiles = int(cnt.sum().item())
+    density = ntiles / (cfg.B * cfg.H * T * T)
+    fwd_fl, bwd_fl = tile_flops(cfg.D, ntiles)
+
+    recs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    launches["n"] = 0
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for s in range(args.steps):
+            flush.fill_(s & 0xff)     # evict L2 between steps (not timed)
+            step(recs[s])
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    plan_ms = [r[0].elapsed_time(r[1]) for r in recs]
+    fwd_ms = [r[1].elapsed_time(r[2]) for r in recs]
+    bwd_ms = [r[2].elapsed_time(r[3]) for r in recs]
+    step_ms = [a + b + c for a, b, c in zip(plan_ms, fwd_ms, bwd_ms)]
+    total_ms = sum(step_ms)
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    step_flops = (fwd_fl + bwd_fl) * world
+    value = step_flops / (ms_per_step * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    fwd_avg = statistics.mean(fwd_ms)
+    bwd_avg = statistics.mean(bwd_ms)
+    plan_avg = statistics.mean(plan_ms)
+    # dominant kernel: the forward kernel is the only launch of sa_forward; it is timed
+    # on the launching (current) stream inside the timed region
+    fwd_tf = fwd_fl / (fwd_avg * 1e-3) / 1e12
+    peak_tf = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
+    roofline = {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": round(fwd_tf, 2),
+                "peak": peak_tf, "unit": "TFLOP/s", "frac": round(fwd_tf / peak_tf, 4),
+                "traffic": traffic_for("attn_fwd_kernel", ntiles),
+                "peak_source": f"{peak_src} bf16 dense, sustained",
+                "algorithmic_flops_per_launch": fwd_fl}
+    router_bytes = 2 * cfg.B * cfg.H * npad * cfg.D * 2 + 4 * (ntiles + cfg.B * cfg.H * T)
+    router_gbs = router_bytes / (plan_avg * 1e-3) / 1e9
+
+    result = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"Wan2.1-14B-720p-shaped attention ({args.config}): B=1, H=40, D=128, latent 21x45x80 "
+                               f"-> 24x48x80 cube grid, T=1440 cubes of 64, Npad=92160; top_k={cfg.top_k}, top_p={cfg.top_p}; "
+                               "step = sa_plan + sa_forward + sa_backward",
+                   "B": cfg.B, "H": cfg.H, "D": cfg.D, "lat": list(cfg.lat), "T": T, "top_k": cfg.top_k,
+                   "top_p": cfg.top_p, "density": round(density, 5), "selected_tiles": ntiles,
+                   "l2": "inputs larger than L2; 256 MiB flush between steps",
+                   "per_rank": "independent problem per rank (seed = rank)"},
+        "breakdown_ms": {"plan": round(plan_avg, 4), "forward": round(fwd_avg, 4), "backward": round(bwd_avg, 4),
+                         "fwd_plus_bwd": round(fwd_avg + bwd_avg, 4)},
+        "fwd_bwd_tflops": round((fwd_fl + bwd_fl) / ((fwd_avg + bwd_avg) * 1e-3) / 1e12, 3),
+        "router": {"achieved_gbs": round(router_gbs, 1), "peak_gbs": peaks.get("hbm_gbs"),
+                   "frac": round(router_gbs / peaks.get("hbm_gbs"), 4), "algorithmic_bytes": router_bytes},
+        "roofline": roofline,
+        "gpu_launches": launches["n"],
+        "clocks": clocks.summary(),
+        "gen_s": round(t_gen, 1),
+    }
+    if args.e2e_steps > 0:
+        result["e2e"] = run_e2e(args, sa, A, p, host, dev, fwd_fl + bwd_fl, world, dist)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(cfg, host, seconds=args.cpu_seconds)
+    return result
+
+
+def traffic_for(kernel: str, ntiles: int):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f).get(kernel)
+    if not d or d.get("source_sha") != source_sha():
+        return None
+    # scale by selected tiles when the capture ran a smaller case
+    per_tile = d["dram_bytes"] / d["tiles"]
+    return int(per_tile * ntiles)
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_attention_cubes_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def run_e2e(args, sa, A, p, host, dev, flops, world, dist):
+    """Same step through the public API with host buffers: pinned latent-order inputs are
+    copied in, tiled, routed, run forward and backward, and out/dq/dk/dv are untiled and
+    copied back, all inside the timed region."""
+    import torch
+    pinned = {n: host[n].pin_memory() for n in ("q", "k", "v", "do")}
+    L = p.lat_t * p.lat_h * p.lat_w
+    outs = {"out": torch.empty((p.B, p.H, L, p.D), dtype=torch.bfloat16).pin_memory()}
+    for n in ("dq", "dk", "dv"):
+        outs[n] = torch.empty((p.B, p.H, L, p.D), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+
+    def e2e_step():
+        d = {n: t.to(dev, non_blocking=True) for n, t in pinned.items()}
+        x = {n: sa.tile(d[n], p) for n in d}
+        idx, cnt = A.plan(x["q"], x["k"])
+        out, lse, out32 = A.forward(x["q"], x["k"], x["v"], idx, cnt)
+        dq, dk, dv = A.backward(x["q"], x["k"], x["v"], out, lse, x["do"], idx, cnt, out_f32=out32)
+        for n, t in (("out", out), ("dq", dq), ("dk", dk), ("dv", dv)):
+            outs[n].copy_(sa.untile(t, p), non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.e2e_steps
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(flops * world / (ms * 1e-3) / 1e12, 3), "unit": UNIT, "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+# ---------------------------------------------------------------------------------- oracle
+def oracle_sample(cfg, host, head: int, frac: float, seed: int = 0):
+    """Run the fp64 oracle on one head: the full router, then forward and backward for a
+    fixed sample of query blocks.  Returns (seconds, effective FLOPs of the sampled tiles)."""
+    import numpy as np
+
+    import oracle as O
+    lay = O.cube_layout(cfg.lat)
+    t = {n: O.tile(host[n][0, head].double().numpy(), lay) for n in ("q", "k", "v", "do")}
+    T = lay.n_cubes
+    rng = np.random.default_rng(seed)
+    sample = np.sort(rng.choice(T, size=max(1, int(round(frac * T))), replace=False))
+    t0 = time.perf_counter()
+    tr = O.route_head(t["q"], t["k"], lay.valid, cfg.top_k, cfg.top_p)
+    O.attention_forward_head(t["q"], t["k"], t["v"], tr.lists, lay.valid, q_blocks=sample)
+    O.attention_backward_head(t["q"], t["k"], t["v"], t["do"], tr.lists, lay.valid, q_blocks=sample,
+                              kv_blocks=range(T), visit=sample)
+    secs = time.perf_counter() - t0
+    ntiles = sum(len(tr.lists[i]) for i in sample)
+    f, b = tile_flops(cfg.D, ntiles)
+    return secs, f + b, len(sample)
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, host, seconds: float = 15.0):
+    # calibrate the sample size on a small piece, then run ~`seconds` of oracle work
+    s0, _, n0 = oracle_sample(cfg, host, head=0, frac=0.02)
+    frac = min(1.0, max(0.02, 0.02 * seconds / max(s0, 1e-3)))
+    secs, flops, n = oracle_sample(cfg, host, head=0, frac=frac, seed=1)
+    return {"value": round(flops / secs / 1e12, 6), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"head 0 of {cfg.name}: full fp64 router + forward and backward of {n} of "
+                      f"{(cfg.lat[0]+3)//4*((cfg.lat[1]+3)//4)*((cfg.lat[2]+3)//4)} query cubes ({secs:.1f} s)"}
+
+
+def run_reference(args, rank, world):
+    import synth
+    cfg = synth.get_config(args.config)
+    host = synth.make_inputs(cfg, seed=0, heads=[0])
+    # sample size: the whole run (warm-up + timed) should take about two minutes
+    s0, _, _ = oracle_sample(cfg, host, head=0, frac=0.02)
+    per_step = 120.0 / max(1, args.steps + args.warmup)
+    frac = min(1.0, max(0.005, 0.02 * per_step / max(s0, 1e-3)))
+    for w in range(args.warmup):
+        oracle_sample(cfg, host, 0, frac, seed=100 + w)
+    tot_s, tot_f, n = 0.0, 0.0, 0
+    for s in range(args.steps):
+        secs, fl, n = oracle_sample(cfg, host, 0, frac, seed=s)
+        tot_s += secs
+        tot_f += fl
+    value = tot_f / tot_s / 1e12
+    cores = cpu_cores()
+    sample = f"per step: head 0 of {cfg.name}, full fp64 router + forward and backward of {n} query cubes"
+    return {"metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"Wan2.1-14B-720p-shaped attention ({args.config}), fp64 CPU oracle sample",
+                       "sample": sample},
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="720p")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    try:
+        res = run_ours(args, rank, world, dist)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

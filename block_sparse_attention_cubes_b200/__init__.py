@@ -71,8 +71,8 @@ def load_library(path: str = LIB_PATH):
         "sa_tile": (i32, [vp, vp, P, i32, vp]),
         "sa_untile": (i32, [vp, vp, P, i32, vp]),
         "sa_plan": (i32, [vp, vp, vp, vp, P, vp, vp, vp, sz, vp]),
-        "sa_forward": (i32, [vp, vp, vp, vp, vp, vp, vp, P, vp, vp, vp, sz, vp]),
-        "sa_backward": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, P, vp, vp, vp, vp, sz, vp]),
+        "sa_forward": (i32, [vp, vp, vp, vp, vp, vp, vp, P, vp, vp, vp, vp, sz, vp]),
+        "sa_backward": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, P, vp, vp, vp, vp, sz, vp]),
         "sa_get_device_status": (i32, [vp, vp]),
         "sa_status_string": (ctypes.c_char_p, [i32]),
         "sa_last_launch_count": (i32, []),
@@ -138,6 +138,19 @@ def _contig(t, name, dtype=None, device=None):
     return t
 
 
+def _shape(t, shape, name):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _token_tensor(t, p: Params, name, elem_bytes):
+    npad, _ = geometry(p)
+    _contig(t, name)
+    _shape(t, (p.B, p.H, npad, p.D), name)
+    if t.element_size() != elem_bytes:
+        raise TypeError(f"{name} must have {elem_bytes}-byte elements")
+
+
 def new_workspace(p: Params, op: int, device=None):
     torch = _torch()
     return torch.empty(max(workspace_size(p, op), 256), dtype=torch.uint8, device=device or "cuda")
@@ -177,8 +190,9 @@ def untile(y, p: Params, out=None, stream=None):
 def plan(q, k, p: Params, q_scale=None, k_scale=None, kv_index=None, kv_count=None, ws=None, stream=None):
     """Router: returns (kv_index [B,H,T,cap] int32, kv_count [B,H,T] int32)."""
     torch = _torch()
-    _contig(q, "q")
-    _contig(k, "k")
+    eb = 1 if p.qk_dtype == FP8_E4M3 else 2
+    _token_tensor(q, p, "q", eb)
+    _token_tensor(k, p, "k", eb)
     _, T = geometry(p)
     dev = q.device
     if kv_index is None:
@@ -194,33 +208,51 @@ def plan(q, k, p: Params, q_scale=None, k_scale=None, kv_index=None, kv_count=No
 
 
 def forward(q, k, v, kv_index, kv_count, p: Params, q_scale=None, k_scale=None, out=None, lse=None, ws=None,
-            stream=None):
-    """Fine stage forward: returns (out [B,H,Npad,D] bf16, lse [B,H,Npad] fp32)."""
+            stream=None, with_f32: bool = False, out_f32=None):
+    """Fine stage forward: returns (out [B,H,Npad,D] bf16, lse [B,H,Npad] fp32), plus the
+    fp32 copy of out as a third element when ``with_f32`` is set (for an exact backward)."""
     torch = _torch()
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (kv_index, "kv_index"), (kv_count, "kv_count")):
-        _contig(t, n)
-    npad, _ = geometry(p)
+    npad, T = geometry(p)
+    eb = 1 if p.qk_dtype == FP8_E4M3 else 2
+    _token_tensor(q, p, "q", eb)
+    _token_tensor(k, p, "k", eb)
+    _token_tensor(v, p, "v", 2)
+    _contig(kv_index, "kv_index", torch.int32)
+    _contig(kv_count, "kv_count", torch.int32)
+    _shape(kv_index, (p.B, p.H, T, p.kv_capacity), "kv_index")
+    _shape(kv_count, (p.B, p.H, T), "kv_count")
     dev = q.device
     if out is None:
         out = torch.empty((p.B, p.H, npad, p.D), dtype=torch.bfloat16, device=dev)
     if lse is None:
         lse = torch.empty((p.B, p.H, npad), dtype=torch.float32, device=dev)
+    if with_f32 and out_f32 is None:
+        out_f32 = torch.empty((p.B, p.H, npad, p.D), dtype=torch.float32, device=dev)
     if ws is None:
         ws = new_workspace(p, OP_FORWARD, dev)
     st = load_library().sa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(q_scale), _ptr(k_scale), _ptr(kv_index),
-                                   _ptr(kv_count), ctypes.byref(p), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
-                                   _stream(stream))
+                                   _ptr(kv_count), ctypes.byref(p), _ptr(out), _ptr(lse), _ptr(out_f32), _ptr(ws),
+                                   ws.numel(), _stream(stream))
     _check(st, "sa_forward")
-    return out, lse
+    return (out, lse, out_f32) if with_f32 else (out, lse)
 
 
 def backward(q, k, v, out, lse, dout, kv_index, kv_count, p: Params, dq=None, dk=None, dv=None, ws=None,
-             stream=None):
-    """Fine stage backward: returns (dq, dk, dv), each [B,H,Npad,D] fp32."""
+             stream=None, out_f32=None):
+    """Fine stage backward: returns (dq, dk, dv), each [B,H,Npad,D] fp32.  Pass the
+    forward's ``out_f32`` to take Delta = rowsum(dO * O) from the unrounded output."""
     torch = _torch()
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (lse, "lse"), (dout, "dout"),
-                 (kv_index, "kv_index"), (kv_count, "kv_count")):
-        _contig(t, n)
+    npad, T = geometry(p)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _token_tensor(t, p, n, 2)
+    if out_f32 is not None:
+        _token_tensor(out_f32, p, "out_f32", 4)
+    _contig(lse, "lse", torch.float32)
+    _shape(lse, (p.B, p.H, npad), "lse")
+    _contig(kv_index, "kv_index", torch.int32)
+    _contig(kv_count, "kv_count", torch.int32)
+    _shape(kv_index, (p.B, p.H, T, p.kv_capacity), "kv_index")
+    _shape(kv_count, (p.B, p.H, T), "kv_count")
     dev = q.device
     shape = tuple(q.shape)
     dq = torch.empty(shape, dtype=torch.float32, device=dev) if dq is None else dq
@@ -228,7 +260,8 @@ def backward(q, k, v, out, lse, dout, kv_index, kv_count, p: Params, dq=None, dk
     dv = torch.empty(shape, dtype=torch.float32, device=dev) if dv is None else dv
     if ws is None:
         ws = new_workspace(p, OP_BACKWARD, dev)
-    st = load_library().sa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(kv_index),
+    st = load_library().sa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(out_f32), _ptr(lse), _ptr(dout),
+                                    _ptr(kv_index),
                                     _ptr(kv_count), ctypes.byref(p), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
                                     ws.numel(), _stream(stream))
     _check(st, "sa_backward")
@@ -251,8 +284,12 @@ class Attention:
     def plan(self, q, k, q_scale=None, k_scale=None):
         return plan(q, k, self.params, q_scale, k_scale, ws=self._w(OP_PLAN, q.device))
 
-    def forward(self, q, k, v, kv_index, kv_count, q_scale=None, k_scale=None):
-        return forward(q, k, v, kv_index, kv_count, self.params, q_scale, k_scale, ws=self._w(OP_FORWARD, q.device))
+    def forward(self, q, k, v, kv_index, kv_count, q_scale=None, k_scale=None, with_f32=True):
+        """Returns (out, lse, out_f32) (out_f32 is None when ``with_f32`` is False)."""
+        r = forward(q, k, v, kv_index, kv_count, self.params, q_scale, k_scale, ws=self._w(OP_FORWARD, q.device),
+                    with_f32=with_f32)
+        return r if with_f32 else (r[0], r[1], None)
 
-    def backward(self, q, k, v, out, lse, dout, kv_index, kv_count):
-        return backward(q, k, v, out, lse, dout, kv_index, kv_count, self.params, ws=self._w(OP_BACKWARD, q.device))
+    def backward(self, q, k, v, out, lse, dout, kv_index, kv_count, out_f32=None):
+        return backward(q, k, v, out, lse, dout, kv_index, kv_count, self.params, ws=self._w(OP_BACKWARD, q.device),
+                        out_f32=out_f32)

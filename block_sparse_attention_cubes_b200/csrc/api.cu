@@ -218,7 +218,7 @@ sa_status sa_plan(const void* q, const void* k, const float* q_scale, const floa
 
 sa_status sa_forward(const void* q, const void* k, const void* v, const float* q_scale, const float* k_scale,
                      const int32_t* kv_index, const int32_t* kv_count, const sa_params* p, void* out, float* lse,
-                     void* ws, size_t ws_bytes, sa_stream_t stream) {
+                     float* out_f32, void* ws, size_t ws_bytes, sa_stream_t stream) {
   Geom g;
   g_last_launches = 0;
   sa_status s = check_params(p, &g);
@@ -226,7 +226,7 @@ sa_status sa_forward(const void* q, const void* k, const void* v, const float* q
   if (!q || !k || !v || !kv_index || !kv_count || !out || !lse) return SA_ERR_INVALID_ARG;
   if (p->qk_dtype == SA_FP8_E4M3) return SA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(lse) || !aligned4(kv_index) ||
-      !aligned4(kv_count))
+      !aligned4(kv_count) || (out_f32 && !aligned16(out_f32)))
     return SA_ERR_ALIGNMENT;
   const WsLayout w = ws_layout(p, g, SA_OP_FORWARD);
   if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
@@ -236,6 +236,7 @@ sa_status sa_forward(const void* q, const void* k, const void* v, const float* q
   a.kv_index = kv_index;
   a.kv_count = kv_count;
   a.out = static_cast<__nv_bfloat16*>(out);
+  a.out_f32 = out_f32;
   a.lse = lse;
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, a.rows_total, p->D, 2) || !make_map(&tk, k, a.rows_total, p->D, 2) ||
@@ -247,8 +248,8 @@ sa_status sa_forward(const void* q, const void* k, const void* v, const float* q
   return SA_OK;
 }
 
-sa_status sa_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
-                      const void* dout, const int32_t* kv_index, const int32_t* kv_count, const sa_params* p,
+sa_status sa_backward(const void* q, const void* k, const void* v, const void* out, const float* out_f32,
+                      const float* lse, const void* dout, const int32_t* kv_index, const int32_t* kv_count, const sa_params* p,
                       float* dq, float* dk, float* dv, void* ws, size_t ws_bytes, sa_stream_t stream) {
   Geom g;
   g_last_launches = 0;
@@ -258,7 +259,8 @@ sa_status sa_backward(const void* q, const void* k, const void* v, const void* o
     return SA_ERR_INVALID_ARG;
   if (p->qk_dtype != SA_BF16) return SA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
-      !aligned16(dk) || !aligned16(dv) || !aligned4(lse) || !aligned4(kv_index) || !aligned4(kv_count))
+      !aligned16(dk) || !aligned16(dv) || !aligned4(lse) || !aligned4(kv_index) || !aligned4(kv_count) ||
+      (out_f32 && !aligned16(out_f32)))
     return SA_ERR_ALIGNMENT;
   const WsLayout w = ws_layout(p, g, SA_OP_BACKWARD);
   if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
@@ -278,7 +280,7 @@ sa_status sa_backward(const void* q, const void* k, const void* v, const void* o
   if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
   uint8_t* wb = static_cast<uint8_t*>(ws);
   int launches = 0;
-  if (sa::launch_backward(tq, tk, tv, tdo, out, dout, a, reinterpret_cast<int32_t*>(wb + w.qcnt),
+  if (sa::launch_backward(tq, tk, tv, tdo, out, out_f32, dout, a, reinterpret_cast<int32_t*>(wb + w.qcnt),
                           reinterpret_cast<int32_t*>(wb + w.qoff), reinterpret_cast<int32_t*>(wb + w.qidx),
                           reinterpret_cast<float*>(wb + w.delta), st, &launches) != cudaSuccess)
     return SA_ERR_LAUNCH;

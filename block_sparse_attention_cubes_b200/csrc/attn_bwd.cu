@@ -25,7 +25,9 @@
 namespace sa {
 
 // ------------------------------------------------------------------------ Delta
+// O is read from its fp32 copy when there is one, else from the bf16 output.
 __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ o,
+                                                    const float* __restrict__ o32,
                                                     const __nv_bfloat16* __restrict__ dout,
                                                     float* __restrict__ delta, Geom g, int BH, int D) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -34,16 +36,22 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restr
   const int p = static_cast<int>(row % g.Npad);
   float acc = 0.0f;
   if (token_valid(g, p >> 6, p & 63)) {
-    const uint2* a = reinterpret_cast<const uint2*>(o + row * D);
     const uint2* b = reinterpret_cast<const uint2*>(dout + row * D);
     for (int c = lane; c < D / 4; c += 32) {
-      const uint2 x = a[c], y = b[c];
-      const uint32_t xs[2] = {x.x, x.y}, ys[2] = {y.x, y.y};
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        acc += __uint_as_float(xs[u] << 16) * __uint_as_float(ys[u] << 16);
-        acc += __uint_as_float(xs[u] & 0xffff0000u) * __uint_as_float(ys[u] & 0xffff0000u);
+      const uint2 y = b[c];
+      float ov[4];
+      if (o32) {
+        const float4 x = reinterpret_cast<const float4*>(o32 + row * D)[c];
+        ov[0] = x.x; ov[1] = x.y; ov[2] = x.z; ov[3] = x.w;
+      } else {
+        const uint2 x = reinterpret_cast<const uint2*>(o + row * D)[c];
+        ov[0] = __uint_as_float(x.x << 16); ov[1] = __uint_as_float(x.x & 0xffff0000u);
+        ov[2] = __uint_as_float(x.y << 16); ov[3] = __uint_as_float(x.y & 0xffff0000u);
       }
+      acc += ov[0] * __uint_as_float(y.x << 16);
+      acc += ov[1] * __uint_as_float(y.x & 0xffff0000u);
+      acc += ov[2] * __uint_as_float(y.y << 16);
+      acc += ov[3] * __uint_as_float(y.y & 0xffff0000u);
     }
   }
 #pragma unroll
@@ -542,7 +550,8 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
 
 // ------------------------------------------------------------------------ launch
 cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const void* out, const void* dout, AttnArgs a, int32_t* qcnt,
+                            const CUtensorMap& tdo, const void* out, const float* out_f32, const void* dout,
+                            AttnArgs a, int32_t* qcnt,
                             int32_t* qoff, int32_t* qidx, float* delta, cudaStream_t stream, int* launches) {
   static bool attr_set = false;
   if (!attr_set) {
@@ -555,7 +564,8 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   const Geom& g = a.g;
   const long long rows = static_cast<long long>(a.BH) * g.Npad;
   delta_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), delta, g, a.BH, a.D);
+      static_cast<const __nv_bfloat16*>(out), out_f32, static_cast<const __nv_bfloat16*>(dout), delta, g, a.BH,
+      a.D);
   cudaError_t e = cudaMemsetAsync(qcnt, 0, sizeof(int32_t) * static_cast<size_t>(a.BH) * g.T, stream);
   if (e != cudaSuccess) return e;
   const long long qrows = static_cast<long long>(a.BH) * g.T;

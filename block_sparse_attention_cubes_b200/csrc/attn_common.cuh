@@ -13,6 +13,7 @@ struct AttnArgs {
   const float* q_scale;     // [BH, T] (fp8 only)
   const float* k_scale;
   __nv_bfloat16* out;       // forward output [BH, Npad, D]
+  float* out_f32;           // optional fp32 copy of the forward output
   float* lse;               // [BH, Npad]
   const float* delta;       // backward: rowsum(dO * O) [BH, Npad]
   const int32_t* q_off;     // backward: transposed lists, CSR offsets [BH, T+1]

@@ -258,12 +258,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     }
     if (r < a.D) {
       __nv_bfloat16* outp = a.out + static_cast<size_t>(row0) * a.D + r;
+      float* outf = a.out_f32 ? a.out_f32 + static_cast<size_t>(row0) * a.D + r : nullptr;
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         const float l = l_sh[c];
         const bool qv = token_valid(g, i, c);
         const float val = (qv && ok && nsteps > 0 && l > 0.0f) ? o[c] / l : 0.0f;
         outp[static_cast<size_t>(c) * a.D] = __float2bfloat16_rn(val);
+        if (outf) outf[static_cast<size_t>(c) * a.D] = val;
       }
     }
     if (r < 64) {

@@ -24,7 +24,8 @@ cudaError_t launch_forward(const CUtensorMap& tq, const CUtensorMap& tk, const C
                            cudaStream_t stream);
 
 cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const void* out, const void* dout, AttnArgs a, int32_t* qcnt,
+                            const CUtensorMap& tdo, const void* out, const float* out_f32, const void* dout,
+                            AttnArgs a, int32_t* qcnt,
                             int32_t* qoff, int32_t* qidx, float* delta, cudaStream_t stream, int* launches);
 
 }  // namespace sa

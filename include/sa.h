@@ -120,20 +120,26 @@ SA_API sa_status sa_plan(const void* q, const void* k, const float* q_scale, con
  *   SA_ERR_DEVICE_INDEX and the offending entries skipped).
  * out: [B,H,Npad,D] bf16; lse: [B,H,Npad] fp32, natural log of each row's softmax
  * normaliser of the scaled scores.  Padding query rows get out = 0, lse = 0; a row with
- * count 0 gets out = 0, lse = -inf.  Deterministic. */
+ * count 0 gets out = 0, lse = -inf.  out_f32 (may be NULL): [B,H,Npad,D] fp32, the same
+ * output before rounding to bf16; pass it on to sa_backward for an exact Delta.
+ * Deterministic. */
 SA_API sa_status sa_forward(const void* q, const void* k, const void* v, const float* q_scale, const float* k_scale,
                      const int32_t* kv_index, const int32_t* kv_count, const sa_params* p, void* out, float* lse,
-                     void* ws, size_t ws_bytes, sa_stream_t stream);
+                     float* out_f32, void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /* Fine stage backward with the block mask held constant (VSA2 page 2.1: the router's
- * output carries no gradient).  Inputs as for sa_forward plus out and lse from it and
- * dout [B,H,Npad,D] bf16.  Outputs dq, dk, dv: [B,H,Npad,D] fp32:
+ * output carries no gradient).  Inputs as for sa_forward plus out, out_f32 and lse from
+ * it and dout [B,H,Npad,D] bf16.  Delta = rowsum(dO * O) is taken from out_f32 when it is
+ * not NULL, else from the bf16 out; bf16 rounding of O enters dS = P * (dP - Delta) as an
+ * absolute error on every selected key and is multiplied by |k| in dQ, which matters for
+ * sink keys of large norm, so pass out_f32 when training.
+ * Outputs dq, dk, dv: [B,H,Npad,D] fp32:
  *   P = exp(scale*QK^T - lse), dV = P^T dO, dP = dO V^T, Delta = rowsum(dO * O),
  *   dS = P * (dP - Delta), dQ = scale * dS K, dK = scale * dS^T Q.
  * Padding rows of every output are 0; dout of padding rows is ignored.
  * bf16 only (qk_dtype must be SA_BF16).  Deterministic. */
-SA_API sa_status sa_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
-                      const void* dout, const int32_t* kv_index, const int32_t* kv_count, const sa_params* p,
+SA_API sa_status sa_backward(const void* q, const void* k, const void* v, const void* out, const float* out_f32,
+                      const float* lse, const void* dout, const int32_t* kv_index, const int32_t* kv_count, const sa_params* p,
                       float* dq, float* dk, float* dv, void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /* Synchronises `stream`, then maps the workspace's device status block to a status:

@@ -231,13 +231,15 @@ def attention_forward_head(q, k, v, lists, valid, scale=None, block=64, q_blocks
 
 
 def attention_backward_head(q, k, v, do, lists, valid, scale=None, block=64,
-                            q_blocks=None, kv_blocks=None):
+                            q_blocks=None, kv_blocks=None, visit=None):
     """dQ, dK, dV of O = softmax(scale*QK^T + M) V with M fixed, for one head.
 
     dV_c = sum_r P_rc dO_r ; dP_rc = dO_r . v_c ; Delta_r = sum_c P_rc dP_rc ;
     dS = P * (dP - Delta) ; dQ_r = scale sum_c dS_rc k_c ; dK_c = scale sum_r dS_rc q_r.
     ``q_blocks`` limits which dQ rows are produced; ``kv_blocks`` limits which dK/dV
     rows are produced (all query blocks that attend them are still visited).
+    ``visit`` limits the query blocks whose contributions are computed at all (a sample
+    of the work, used for timing); by default every query block is visited.
     """
     n_pad, D = q.shape
     scale = 1.0 / math.sqrt(D) if scale is None else scale
@@ -247,7 +249,7 @@ def attention_backward_head(q, k, v, do, lists, valid, scale=None, block=64,
     dv = np.zeros_like(v, dtype=np.float64)
     want_kv = None if kv_blocks is None else set(int(j) for j in kv_blocks)
     want_q = None if q_blocks is None else set(int(i) for i in q_blocks)
-    for i in range(T):
+    for i in (range(T) if visit is None else visit):
         sel = lists[i]
         need_q = want_q is None or i in want_q
         need_kv = want_kv is None or any(int(j) in want_kv for j in sel)

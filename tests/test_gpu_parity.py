@@ -74,8 +74,9 @@ def _fwd_case(cfg, lists_src="oracle", heads=None, q_blocks=None):
         trs[(0, hh)] = O.route_head(oracle_head(x, "q", 0, hh, lay), oracle_head(x, "k", 0, hh, lay), lay.valid,
                                     cfg.top_k, cfg.top_p).lists
     idx, cnt = lists_to_device(trs, 1, H, lay.n_cubes, p.kv_capacity)
-    out, lse = sa.forward(t["q"], t["k"], t["v"], idx, cnt, p)
+    out, lse, out32 = sa.forward(t["q"], t["k"], t["v"], idx, cnt, p, with_f32=True)
     torch.cuda.synchronize()
+    assert torch.equal(out32.to(torch.bfloat16), out)
     for hh in range(H):
         q, k, v = (oracle_head(x, n, 0, hh, lay) for n in ("q", "k", "v"))
         o_ref, lse_ref = O.attention_forward_head(q, k, v, trs[(0, hh)], lay.valid, q_blocks=q_blocks)
@@ -91,7 +92,7 @@ def _fwd_case(cfg, lists_src="oracle", heads=None, q_blocks=None):
         gl = lse[0, hh].cpu().numpy()
         assert np.max(np.abs(gl[rows] - lse_ref[rows])) < 1e-3
         assert np.all(gl[~lay.valid] == 0)
-    return x, p, t, idx, cnt, out, lse, trs
+    return x, p, t, idx, cnt, out, lse, out32, trs
 
 
 def test_forward_tiny():
@@ -106,8 +107,8 @@ def test_forward_small(D, lat, k, pp):
 
 
 def _bwd_case(cfg):
-    x, p, t, idx, cnt, out, lse, trs = _fwd_case(cfg)
-    dq, dk, dv = sa.backward(t["q"], t["k"], t["v"], out, lse, t["do"], idx, cnt, p)
+    x, p, t, idx, cnt, out, lse, out32, trs = _fwd_case(cfg)
+    dq, dk, dv = sa.backward(t["q"], t["k"], t["v"], out, lse, t["do"], idx, cnt, p, out_f32=out32)
     torch.cuda.synchronize()
     lay = O.cube_layout(cfg.lat)
     for hh in range(p.H):
@@ -133,8 +134,8 @@ def test_backward_small(D, lat, k, pp):
 def test_end_to_end_with_gpu_lists():
     cfg = synth.small_config("e2e", 1, 4, 128, (8, 16, 20), 4, 0.9)
     x, p, t, idx, cnt = _router_case(cfg)
-    out, lse = sa.forward(t["q"], t["k"], t["v"], idx, cnt, p)
-    dq, dk, dv = sa.backward(t["q"], t["k"], t["v"], out, lse, t["do"], idx, cnt, p)
+    out, lse, out32 = sa.forward(t["q"], t["k"], t["v"], idx, cnt, p, with_f32=True)
+    dq, dk, dv = sa.backward(t["q"], t["k"], t["v"], out, lse, t["do"], idx, cnt, p, out_f32=out32)
     torch.cuda.synchronize()
     lay = O.cube_layout(cfg.lat)
     for hh in range(p.H):
@@ -153,10 +154,15 @@ def test_deterministic_repeat():
     r1 = sa.plan(t["q"], t["k"], p)
     r2 = sa.plan(t["q"], t["k"], p)
     assert torch.equal(r1[1], r2[1]) and torch.equal(r1[0], r2[0])
-    o1 = sa.forward(t["q"], t["k"], t["v"], *r1, p)
-    o2 = sa.forward(t["q"], t["k"], t["v"], *r1, p)
-    assert torch.equal(o1[0], o2[0]) and torch.equal(o1[1], o2[1])
-    g1 = sa.backward(t["q"], t["k"], t["v"], *o1, t["do"], *r1, p)
-    g2 = sa.backward(t["q"], t["k"], t["v"], *o1, t["do"], *r1, p)
+    o1 = sa.forward(t["q"], t["k"], t["v"], *r1, p, with_f32=True)
+    o2 = sa.forward(t["q"], t["k"], t["v"], *r1, p, with_f32=True)
+    assert all(torch.equal(a, b) for a, b in zip(o1, o2))
+    g1 = sa.backward(t["q"], t["k"], t["v"], o1[0], o1[1], t["do"], *r1, p, out_f32=o1[2])
+    g2 = sa.backward(t["q"], t["k"], t["v"], o1[0], o1[1], t["do"], *r1, p, out_f32=o1[2])
     for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
+    # without the fp32 copy Delta comes from the bf16 output: same as passing it upcast
+    g3 = sa.backward(t["q"], t["k"], t["v"], o1[0], o1[1], t["do"], *r1, p)
+    g4 = sa.backward(t["q"], t["k"], t["v"], o1[0], o1[1], t["do"], *r1, p, out_f32=o1[0].float())
+    for a, b in zip(g3, g4):
         assert torch.equal(a, b)
