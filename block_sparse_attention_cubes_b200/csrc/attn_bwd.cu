@@ -138,8 +138,8 @@ constexpr uint32_t OFF_Q = 0;          // [2 halves][64][128 B]
 constexpr uint32_t OFF_DO = 16384;     // same
 constexpr uint32_t OFF_K = 32768;      // 2 stages x [2 halves][128][128 B]
 constexpr uint32_t OFF_V = 98304;      // same
-constexpr uint32_t OFF_DS = 163840;    // 2 buffers x [128 keys][64 q] bf16
-constexpr uint32_t OFF_BAR = 196608;
+constexpr uint32_t OFF_DS = 163840;    // 2 buffers x {hi, lo} x [128 keys][64 q] bf16
+constexpr uint32_t OFF_BAR = 229376;
 constexpr uint32_t OFF_SLOT = OFF_BAR + 192;
 constexpr uint32_t OFF_FLAG = OFF_BAR + 200;
 constexpr uint32_t OFF_LSE = OFF_BAR + 256;    // [64] lse * log2(e)
@@ -258,11 +258,12 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         if (!mbar_wait(&bars[B_DSF + st], (s >> 1) & 1, a.st, a.timeout_ns, 54)) break;
         tc_fence_after();
         const uint32_t kst = sbase + OFF_K + st * 32768;
-        const uint32_t dsb = sbase + OFF_DS + st * 16384;
+        const uint32_t dsb = sbase + OFF_DS + st * 32768;
 #pragma unroll 1
-        for (int ks = 0; ks < 8; ++ks) {
-          umma_f16_ss(tmem + 256, sw128_desc(kst + ks * 2048, 16384, 1024), sw128_desc(dsb + ks * 2048, 8192, 1024),
-                      idesc_mn, (s > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < 16; ++ks) {  // 8 k-steps over dS_hi, then 8 over dS_lo
+          const uint32_t kk = ks & 7, part = ks >> 3;
+          umma_f16_ss(tmem + 256, sw128_desc(kst + kk * 2048, 16384, 1024),
+                      sw128_desc(dsb + part * 16384 + kk * 2048, 8192, 1024), idesc_mn, (s > 0 || ks > 0) ? 1u : 0u);
         }
         umma_commit(&bars[B_EMPTY + st]);
         umma_commit(&bars[B_DSFREE + st]);
@@ -307,7 +308,7 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         sv[c] = p * (dp[c] - delta_sh[c]);
       }
       if (s >= 2 && !mbar_wait(&bars[B_DSFREE + b], ((s >> 1) + 1) & 1, a.st, a.timeout_ns, 62)) *grp_abort = 1;
-      store_row_bf16_sw128(sbase + OFF_DS + b * 16384, r, sv);
+      store_row_bf16x2_sw128(sbase + OFF_DS + b * 32768, sbase + OFF_DS + b * 32768 + 16384, r, sv);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[B_DSF + b]);
@@ -347,9 +348,9 @@ constexpr uint32_t OFF_K = 0;          // [2 halves][64][128 B]
 constexpr uint32_t OFF_V = 16384;      // same
 constexpr uint32_t OFF_Q = 32768;      // 2 stages x [2 halves][128][128 B]
 constexpr uint32_t OFF_DO = 98304;     // same
-constexpr uint32_t OFF_P = 163840;     // [128 q][64 keys] bf16
-constexpr uint32_t OFF_DS = 180224;    // same
-constexpr uint32_t OFF_BAR = 196608;
+constexpr uint32_t OFF_P = 163840;     // {hi, lo} x [128 q][64 keys] bf16
+constexpr uint32_t OFF_DS = 196608;    // same
+constexpr uint32_t OFF_BAR = 229376;
 constexpr uint32_t OFF_SLOT = OFF_BAR + 192;
 constexpr uint32_t OFF_FLAG = OFF_BAR + 200;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
@@ -462,14 +463,18 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
         tc_fence_after();
         const uint32_t qst = sbase + OFF_Q + st * 32768, dst = sbase + OFF_DO + st * 32768;
 #pragma unroll 1
-        for (int ks = 0; ks < 8; ++ks) {
-          umma_f16_ss(tmem + 256, sw128_desc(dst + ks * 2048, 16384, 1024),
-                      sw128_desc(sbase + OFF_P + ks * 2048, 8192, 1024), idesc_mn, (s > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < 16; ++ks) {  // P_hi then P_lo
+          const uint32_t kk = ks & 7, part = ks >> 3;
+          umma_f16_ss(tmem + 256, sw128_desc(dst + kk * 2048, 16384, 1024),
+                      sw128_desc(sbase + OFF_P + part * 16384 + kk * 2048, 8192, 1024), idesc_mn,
+                      (s > 0 || ks > 0) ? 1u : 0u);
         }
 #pragma unroll 1
-        for (int ks = 0; ks < 8; ++ks) {
-          umma_f16_ss(tmem + 320, sw128_desc(qst + ks * 2048, 16384, 1024),
-                      sw128_desc(sbase + OFF_DS + ks * 2048, 8192, 1024), idesc_mn, (s > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < 16; ++ks) {  // dS_hi then dS_lo
+          const uint32_t kk = ks & 7, part = ks >> 3;
+          umma_f16_ss(tmem + 320, sw128_desc(qst + kk * 2048, 16384, 1024),
+                      sw128_desc(sbase + OFF_DS + part * 16384 + kk * 2048, 8192, 1024), idesc_mn,
+                      (s > 0 || ks > 0) ? 1u : 0u);
         }
         umma_commit(&bars[B_EMPTY + st]);
         umma_commit(&bars[B_PDSFREE]);
@@ -511,8 +516,8 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
         dp[c] = p * (dp[c] - dlt);
       }
       if (s >= 1 && !mbar_wait(&bars[B_PDSFREE], (s - 1) & 1, a.st, a.timeout_ns, 92)) *grp_abort = 1;
-      store_row_bf16_sw128(sbase + OFF_P, r, sv);
-      store_row_bf16_sw128(sbase + OFF_DS, r, dp);
+      store_row_bf16x2_sw128(sbase + OFF_P, sbase + OFF_P + 16384, r, sv);
+      store_row_bf16x2_sw128(sbase + OFF_DS, sbase + OFF_DS + 16384, r, dp);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[B_PDS]);

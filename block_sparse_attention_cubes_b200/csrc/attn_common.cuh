@@ -115,6 +115,27 @@ __device__ __forceinline__ void store_row_bf16_sw128(uint32_t tile_base, uint32_
   }
 }
 
+// Store a 64-element row as two bf16 rows hi + lo with hi = bf16(v) and lo = bf16(v - hi),
+// so that hi + lo carries v to about 2^-16 relative.  Products that are summed over many
+// query rows (dV of a popular key, dK and dQ next to a large sink key) use both halves.
+__device__ __forceinline__ void store_row_bf16x2_sw128(uint32_t base_hi, uint32_t base_lo, uint32_t row,
+                                                       const float (&v)[64]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float a = v[8 * c + 2 * u], b = v[8 * c + 2 * u + 1];
+      h[u] = pack_bf16x2(a, b);
+      const float ha = __uint_as_float(h[u] << 16), hb = __uint_as_float(h[u] & 0xffff0000u);
+      l[u] = pack_bf16x2(a - ha, b - hb);
+    }
+    const uint32_t off = sw128_offset(row, c);
+    st_shared_v4(base_hi + off, h[0], h[1], h[2], h[3]);
+    st_shared_v4(base_lo + off, l[0], l[1], l[2], l[3]);
+  }
+}
+
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
   uint32_t r0[32], r1[32];
   tmem_ld32(taddr, r0);
