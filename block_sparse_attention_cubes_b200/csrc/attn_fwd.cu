@@ -30,8 +30,8 @@ constexpr int kThreads = 192;
 constexpr uint32_t OFF_Q = 0;            // 2 halves x [64 rows][128 B]
 constexpr uint32_t OFF_K = 16384;        // 2 stages x 2 halves x [128 rows][128 B]
 constexpr uint32_t OFF_V = 81920;        // same
-constexpr uint32_t OFF_P = 147456;       // 2 buffers x [128 keys][64 queries] bf16
-constexpr uint32_t OFF_BAR = 180224;
+constexpr uint32_t OFF_P = 147456;       // 2 buffers x {hi, lo} x [128 keys][64 queries] bf16
+constexpr uint32_t OFF_BAR = 212992;
 constexpr uint32_t OFF_SLOT = OFF_BAR + 128;
 constexpr uint32_t OFF_FLAG = OFF_BAR + 136;
 constexpr uint32_t OFF_RED = OFF_BAR + 256;  // [4][64] float
@@ -85,6 +85,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   const int n = list_count(a, bh, i, threadIdx.x == 0);
   const int nsteps = skip_all ? 0 : (n + 1) >> 1;
   const int row0 = bh * g.Npad + i * 64;
+  // When the caller keeps the fp32 output (for the backward's Delta), P enters the PV
+  // product as bf16 hi + lo so that O is exact to ~2^-16 instead of bf16's 2^-9.
+  const bool split_pv = a.out_f32 != nullptr;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
@@ -127,6 +130,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       const uint32_t idesc_s = make_idesc(128, 64, FMT_BF16, false, false);
       const uint32_t idesc_o = make_idesc(128, 64, FMT_BF16, true, true);
       const int ksteps = a.D / 16;
+      const int nk_pv = split_pv ? 16 : 8;
       auto issue_s = [&](int s) {
         const uint32_t kst = sbase + OFF_K + (s & 1) * 32768;
         const uint32_t d_tmem = tmem + (s & 1) * 64;
@@ -153,11 +157,12 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t vst = sbase + OFF_V + st * 32768;
-        const uint32_t pb = sbase + OFF_P + st * 16384;
+        const uint32_t pb = sbase + OFF_P + st * 32768;
 #pragma unroll 1
-        for (int ks = 0; ks < 8; ++ks) {
-          umma_f16_ss(tmem + 128, sw128_desc(vst + ks * 2048, 16384, 1024), sw128_desc(pb + ks * 2048, 8192, 1024),
-                      idesc_o, (s > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < nk_pv; ++ks) {  // 8 k-steps over P (or P_hi), then 8 over P_lo
+          const uint32_t kk = ks & 7, part = ks >> 3;
+          umma_f16_ss(tmem + 128, sw128_desc(vst + kk * 2048, 16384, 1024),
+                      sw128_desc(pb + part * 16384 + kk * 2048, 8192, 1024), idesc_o, (s > 0 || ks > 0) ? 1u : 0u);
         }
         umma_commit(&bars[B_EMPTY + st]);
         umma_commit(&bars[B_OD]);
@@ -226,7 +231,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         rescale |= (al != 1.0f);
       }
       if (s >= 1 && !mbar_wait(&bars[B_OD], (s - 1) & 1, a.st, a.timeout_ns, 32)) *grp_abort = 1;
-      store_row_bf16_sw128(sbase + OFF_P + b * 16384, r, v);
+      if (split_pv)
+        store_row_bf16x2_sw128(sbase + OFF_P + b * 32768, sbase + OFF_P + b * 32768 + 16384, r, v);
+      else
+        store_row_bf16_sw128(sbase + OFF_P + b * 32768, r, v);
       if (rescale && s >= 1) {
         tc_fence_after();
         float o[64];

@@ -75,8 +75,10 @@ def _fwd_case(cfg, lists_src="oracle", heads=None, q_blocks=None):
                                     cfg.top_k, cfg.top_p).lists
     idx, cnt = lists_to_device(trs, 1, H, lay.n_cubes, p.kv_capacity)
     out, lse, out32 = sa.forward(t["q"], t["k"], t["v"], idx, cnt, p, with_f32=True)
+    out_inf, lse_inf = sa.forward(t["q"], t["k"], t["v"], idx, cnt, p)      # inference path: single bf16 P
     torch.cuda.synchronize()
     assert torch.equal(out32.to(torch.bfloat16), out)
+    assert torch.equal(lse_inf, lse)
     for hh in range(H):
         q, k, v = (oracle_head(x, n, 0, hh, lay) for n in ("q", "k", "v"))
         o_ref, lse_ref = O.attention_forward_head(q, k, v, trs[(0, hh)], lay.valid, q_blocks=q_blocks)
@@ -88,6 +90,7 @@ def _fwd_case(cfg, lists_src="oracle", heads=None, q_blocks=None):
             rows &= m
         got = out[0, hh].float().cpu().numpy()
         assert_close(f"out h{hh}", got[rows], o_ref[rows])
+        assert_close(f"out (bf16 P) h{hh}", out_inf[0, hh].float().cpu().numpy()[rows], o_ref[rows])
         assert np.all(got[~lay.valid] == 0)
         gl = lse[0, hh].cpu().numpy()
         assert np.max(np.abs(gl[rows] - lse_ref[rows])) < 1e-3
