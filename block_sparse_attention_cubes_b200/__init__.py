@@ -33,7 +33,7 @@ DEBUG_SKIP_LOADS = 1
 # every symbol include/sa.h declares
 EXPORTS = ("sa_padded_tokens", "sa_num_cubes", "sa_topk_from_fraction", "sa_workspace_size", "sa_tile",
            "sa_untile", "sa_plan", "sa_forward", "sa_backward", "sa_get_device_status", "sa_status_string",
-           "sa_last_launch_count")
+           "sa_last_launch_count", "sa_plan_static")
 
 
 class SAError(RuntimeError):
@@ -76,6 +76,7 @@ def load_library(path: str = LIB_PATH):
         "sa_get_device_status": (i32, [vp, vp]),
         "sa_status_string": (ctypes.c_char_p, [i32]),
         "sa_last_launch_count": (i32, []),
+        "sa_plan_static": (i32, [vp, vp, vp, vp, P, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -204,6 +205,18 @@ def plan(q, k, p: Params, q_scale=None, k_scale=None, kv_index=None, kv_count=No
     st = load_library().sa_plan(_ptr(q), _ptr(k), _ptr(q_scale), _ptr(k_scale), ctypes.byref(p), _ptr(kv_index),
                                 _ptr(kv_count), _ptr(ws), ws.numel(), _stream(stream))
     _check(st, "sa_plan")
+    return kv_index, kv_count
+
+
+def plan_static(q, k, p: Params, kv_index, kv_count, q_scale=None, k_scale=None, stream=None):
+    """Router with the library's fixed 64 MiB scratch instead of a workspace (see
+    ``sa_plan_static`` in include/sa.h).  Outputs are caller-provided; nothing is allocated."""
+    eb = 1 if p.qk_dtype == FP8_E4M3 else 2
+    _token_tensor(q, p, "q", eb)
+    _token_tensor(k, p, "k", eb)
+    st = load_library().sa_plan_static(_ptr(q), _ptr(k), _ptr(q_scale), _ptr(k_scale), ctypes.byref(p),
+                                       _ptr(kv_index), _ptr(kv_count), _stream(stream))
+    _check(st, "sa_plan_static")
     return kv_index, kv_count
 
 

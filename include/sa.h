@@ -142,6 +142,20 @@ SA_API sa_status sa_backward(const void* q, const void* k, const void* v, const 
                       const float* lse, const void* dout, const int32_t* kv_index, const int32_t* kv_count, const sa_params* p,
                       float* dq, float* dk, float* dv, void* ws, size_t ws_bytes, sa_stream_t stream);
 
+/* sa_plan without a workspace: the same router and the same results, for callers that
+ * cannot allocate device memory (code running under a CUDA stream capture, serving
+ * processes confined to a pre-reserved memory arena, C callers with no device
+ * allocator).  The pages have no counterpart to it; it is a deployment convenience.
+ * Scratch lives in one fixed device array of 64 MiB that every GPU loading the library
+ * holds until exit; problems needing more (sa_workspace_size(p, SA_OP_PLAN) > 64 MiB,
+ * e.g. 12 heads at the 480p shape fit, 40 heads at 720p do not) return SA_ERR_WORKSPACE.
+ * kv_capacity must equal T, so no row can be clipped and there is no device status to
+ * read.  The first call on a device looks up the array's device address (make it before
+ * any stream capture).  All calls share the array: calls that overlap on the GPU race and
+ * must be serialised by the caller.  Allocates nothing (no cudaMalloc/cudaFree). */
+SA_API sa_status sa_plan_static(const void* q, const void* k, const float* q_scale, const float* k_scale,
+                                const sa_params* p, int32_t* kv_index, int32_t* kv_count, sa_stream_t stream);
+
 /* Synchronises `stream`, then maps the workspace's device status block to a status:
  * SA_OK, SA_ERR_DEVICE_TIMEOUT, SA_ERR_DEVICE_INDEX or SA_ERR_CAPACITY (first that
  * applies, in that order of precedence: timeout, index, capacity). */
