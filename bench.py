@@ -114,7 +114,7 @@ def run_ours(args, rank, world, dist):
     dev = torch.device("cuda", local)
     cfg = synth.get_config(args.config)
     t_gen = time.time()
-    host = synth.make_inputs(cfg, seed=rank)
+    host = synth.make_inputs(cfg, seed=rank_seed(rank))
     t_gen = time.time() - t_gen
     p = sa.make_params(cfg.B, cfg.H, cfg.D, cfg.lat, cfg.top_k, cfg.top_p)
     npad, T = sa.geometry(p)
@@ -168,11 +168,7 @@ def run_ours(args, rank, world, dist):
     fwd_ms = [r[1].elapsed_time(r[2]) for r in recs]
     bwd_ms = [r[2].elapsed_time(r[3]) for r in recs]
     step_ms = [a + b + c for a, b, c in zip(plan_ms, fwd_ms, bwd_ms)]
-    total_ms = sum(step_ms)
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, dev)
     ms_per_step = total_ms / args.steps
     step_flops = (fwd_fl + bwd_fl) * world
     value = step_flops / (ms_per_step * 1e-3) / 1e12
@@ -219,6 +215,21 @@ def run_ours(args, rank, world, dist):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(cfg, host, seconds=args.cpu_seconds)
     return result
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws an independent problem of the same shape."""
+    return rank
 
 
 def traffic_for(kernel: str, ntiles: int):
@@ -276,11 +287,7 @@ def run_e2e(args, sa, A, p, host, dev, flops, world, dist):
         e2e_step()
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.e2e_steps
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dist, dev)
     return {"value": round(flops * world / (ms * 1e-3) / 1e12, 3), "unit": UNIT, "ms_per_step": round(ms, 3),
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 

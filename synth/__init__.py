@@ -147,18 +147,28 @@ def _to_bf16(x: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16)
 
 
-def _one_head(cfg: Config, seed: int, name: str, b: int, h: int) -> torch.Tensor:
-    ht = cfg.head_types[h]
+def components(cfg: Config, seed: int, name: str, b: int, h: int):
+    """The two draws behind one head of one tensor: (noise, phi), both fp64 [L, D]
+    (phi is None for do)."""
     rng = np.random.Generator(np.random.Philox(np.random.SeedSequence([seed, TENSOR_IDS[name], b, h])))
-    x = rng.standard_normal((cfg.L, cfg.D))
+    noise = rng.standard_normal((cfg.L, cfg.D))
+    return noise, (None if name == "do" else _phi(cfg, seed, b, h))
+
+
+def combine(name: str, noise: np.ndarray, phi, ht: HeadType) -> torch.Tensor:
+    """Assemble one head from its draws with the head type's amplitude, scale and sink."""
+    x = noise.copy()
     if name != "do":
-        phi = _phi(cfg, seed, b, h)
-        amp = ht.alpha * (0.5 if name == "v" else 1.0)
-        x += amp * phi
+        x += ht.alpha * (0.5 if name == "v" else 1.0) * phi
         if name == "k":
             x *= ht.kscale
             x[0] *= ht.sink
     return _to_bf16(x)
+
+
+def _one_head(cfg: Config, seed: int, name: str, b: int, h: int) -> torch.Tensor:
+    noise, phi = components(cfg, seed, name, b, h)
+    return combine(name, noise, phi, cfg.head_types[h])
 
 
 def make_inputs(cfg: Config, seed: int = 0, names=("q", "k", "v", "do"), heads=None,
