@@ -56,6 +56,7 @@ double softmax_scale(const sa_params* p) {
 }
 
 struct WsLayout {
+  size_t cmask = 0;                                        // forward, backward: [T] cube masks
   size_t qbar = 0, kbar = 0, scores = 0;                   // plan
   size_t delta = 0, qcnt = 0, qoff = 0, qidx = 0;          // backward
   size_t total = 0;
@@ -72,7 +73,12 @@ WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
     off = align256(off + BH * g.T * p->D * sizeof(double));
     w.scores = off;
     off = align256(off + BH * g.T * static_cast<size_t>(g.T) * sizeof(double));
+  } else if (op == SA_OP_FORWARD) {
+    w.cmask = off;
+    off = align256(off + static_cast<size_t>(g.T) * sizeof(unsigned long long));
   } else if (op == SA_OP_BACKWARD) {
+    w.cmask = off;
+    off = align256(off + static_cast<size_t>(g.T) * sizeof(unsigned long long));
     w.delta = off;
     off = align256(off + BH * g.Npad * sizeof(float));
     w.qcnt = off;
@@ -243,8 +249,12 @@ sa_status sa_forward(const void* q, const void* k, const void* v, const float* q
       !make_map(&tv, v, a.rows_total, p->D, 2))
     return SA_ERR_LAUNCH;
   if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
+  a.cube_mask = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(ws) + w.cmask);
+  if (sa::launch_cube_mask(g, reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(ws) + w.cmask), st) !=
+      cudaSuccess)
+    return SA_ERR_LAUNCH;
   if (sa::launch_forward(tq, tk, tv, a, st) != cudaSuccess) return SA_ERR_LAUNCH;
-  g_last_launches = 1;
+  g_last_launches = 2;
   return SA_OK;
 }
 
@@ -279,12 +289,15 @@ sa_status sa_backward(const void* q, const void* k, const void* v, const void* o
     return SA_ERR_LAUNCH;
   if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
   uint8_t* wb = static_cast<uint8_t*>(ws);
+  a.cube_mask = reinterpret_cast<unsigned long long*>(wb + w.cmask);
+  if (sa::launch_cube_mask(g, reinterpret_cast<unsigned long long*>(wb + w.cmask), st) != cudaSuccess)
+    return SA_ERR_LAUNCH;
   int launches = 0;
   if (sa::launch_backward(tq, tk, tv, tdo, out, out_f32, dout, a, reinterpret_cast<int32_t*>(wb + w.qcnt),
                           reinterpret_cast<int32_t*>(wb + w.qoff), reinterpret_cast<int32_t*>(wb + w.qidx),
                           reinterpret_cast<float*>(wb + w.delta), st, &launches) != cudaSuccess)
     return SA_ERR_LAUNCH;
-  g_last_launches = launches;
+  g_last_launches = launches + 1;
   return SA_OK;
 }
 

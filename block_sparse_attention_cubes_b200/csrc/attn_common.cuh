@@ -14,6 +14,7 @@ struct AttnArgs {
   const float* k_scale;
   __nv_bfloat16* out;       // forward output [BH, Npad, D]
   float* out_f32;           // optional fp32 copy of the forward output
+  const unsigned long long* cube_mask;  // [T] valid-slot mask of every cube
   float* lse;               // [BH, Npad]
   const float* delta;       // backward: rowsum(dO * O) [BH, Npad]
   const int32_t* q_off;     // backward: transposed lists, CSR offsets [BH, T+1]
@@ -101,6 +102,78 @@ __device__ __forceinline__ int warp_colreduce64(float (&v)[64], int lane, Op op)
   }
   return 32 * ((lane >> 4) & 1) + 16 * ((lane >> 3) & 1) + 8 * ((lane >> 2) & 1) + 4 * ((lane >> 1) & 1) +
          2 * (lane & 1);
+}
+
+// Same reduction for 32 column values: lane l ends with column l in v[0] (31 shuffles).
+template <class Op>
+__device__ __forceinline__ int warp_colreduce32(float (&v)[32], int lane, Op op) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const bool hi = lane & 16;
+    const float send = hi ? v[i] : v[i + 16];
+    const float keep = hi ? v[i + 16] : v[i];
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool hi = lane & 8;
+    const float send = hi ? v[i] : v[i + 8];
+    const float keep = hi ? v[i + 8] : v[i];
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool hi = lane & 4;
+    const float send = hi ? v[i] : v[i + 4];
+    const float keep = hi ? v[i + 4] : v[i];
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool hi = lane & 2;
+    const float send = hi ? v[i] : v[i + 2];
+    const float keep = hi ? v[i + 2] : v[i];
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+  }
+  {
+    const bool hi = lane & 1;
+    const float send = hi ? v[0] : v[1];
+    const float keep = hi ? v[1] : v[0];
+    v[0] = op(keep, __shfl_xor_sync(0xffffffffu, send, 1));
+  }
+  return lane;
+}
+
+// Store 32 bf16 values as columns 32*half .. 32*half+31 (64 bytes, chunks 4*half..4*half+3)
+// of row `row` of a 128-byte-swizzled tile.
+__device__ __forceinline__ void store_half_row_bf16_sw128(uint32_t tile_base, uint32_t row, int half,
+                                                          const float (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint32_t a = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
+    const uint32_t b = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+    const uint32_t cc = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+    const uint32_t d = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+    st_shared_v4(tile_base + sw128_offset(row, 4 * half + c), a, b, cc, d);
+  }
+}
+
+// hi + lo version of the above (hi = bf16(v), lo = bf16(v - hi))
+__device__ __forceinline__ void store_half_row_bf16x2_sw128(uint32_t base_hi, uint32_t base_lo, uint32_t row,
+                                                            int half, const float (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float x0 = v[8 * c + 2 * u], x1 = v[8 * c + 2 * u + 1];
+      h[u] = pack_bf16x2(x0, x1);
+      l[u] = pack_bf16x2(x0 - __uint_as_float(h[u] << 16), x1 - __uint_as_float(h[u] & 0xffff0000u));
+    }
+    const uint32_t off = sw128_offset(row, 4 * half + c);
+    st_shared_v4(base_hi + off, h[0], h[1], h[2], h[3]);
+    st_shared_v4(base_lo + off, l[0], l[1], l[2], l[3]);
+  }
 }
 
 // Store one 64-element bf16 row (128 bytes) of a 128-byte-swizzled tile.

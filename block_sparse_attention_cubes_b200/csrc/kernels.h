@@ -20,6 +20,9 @@ cudaError_t launch_plan(const void* q, const void* k, const float* q_scale, cons
                         int32_t* kv_count, double* qbar, double* kbar, double* S, DevStatus* st,
                         cudaStream_t stream, int* launches);
 
+cudaError_t launch_cube_mask(const Geom& g, unsigned long long* mask, cudaStream_t stream);
+int num_sms();
+
 cudaError_t launch_forward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
                            cudaStream_t stream);
 
