@@ -10,10 +10,12 @@
 //     S^T[128 keys x 64 queries]  = [K_j0; K_j1] . Q_i^T         (M=128, N=64, K=D)
 //     O^T[D x 64 queries]        += [V_j0; V_j1]^T . P^T          (M=D,   N=64, K=128)
 // with both accumulators in TMEM.  Persistent CTAs (one per SM) walk the query cubes
-// round-robin; the K/V ring, the S^T buffers and the step counters run on across cubes,
-// and Q and O^T are double-buffered so that one cube's epilogue overlaps the next cube's
-// first products.  Warp roles (320 threads):
-//   warp 0      TMA producer: Q of each cube, K/V tile pairs into a 2-stage ring
+// round-robin; the K and V rings, the S^T buffers and the step counters run on across
+// cubes, and O^T is double-buffered so that one cube's epilogue overlaps the next cube's
+// products.  K tiles live in a 3-stage ring released as soon as their S^T product is
+// done, V tiles in a 2-stage ring released after PV, so K loads run well ahead of the MMA.
+// Warp roles (320 threads):
+//   warp 0      TMA producers: lane 0 loads Q and K tile pairs, lane 1 loads V tile pairs
 //   warp 1      TMEM owner and the single MMA-issuing thread
 //   warps 2-9   two groups of four warps; group g owns query columns 32g..32g+31 and
 //               thread r of a group owns key r of the pair (TMEM lane r).
@@ -31,11 +33,13 @@ namespace fwd {
 constexpr int kThreads = 320;
 constexpr float kTau = 8.0f;       // log2 headroom before a running maximum is raised
 constexpr float kNegBig = -1e30f;  // finite "minus infinity" for running maxima
-constexpr uint32_t OFF_Q = 0;          // 2 buffers x [2 halves][64 rows][128 B]
-constexpr uint32_t OFF_K = 32768;      // 2 stages x [2 halves][128 rows][128 B]
-constexpr uint32_t OFF_V = 98304;      // same
-constexpr uint32_t OFF_P = 163840;     // {hi, lo} x [128 keys][64 queries] bf16
-constexpr uint32_t OFF_BAR = 196608;
+constexpr int KST = 3;                 // K ring stages
+constexpr int VST = 2;                 // V ring stages
+constexpr uint32_t OFF_Q = 0;          // [2 halves][64 rows][128 B]
+constexpr uint32_t OFF_K = 16384;      // KST stages x [2 halves][128 rows][128 B]
+constexpr uint32_t OFF_V = OFF_K + KST * 32768;  // VST stages, same shape
+constexpr uint32_t OFF_P = OFF_V + VST * 32768;  // {hi, lo} x [128 keys][64 queries] bf16
+constexpr uint32_t OFF_BAR = OFF_P + 32768;
 constexpr uint32_t OFF_SLOT = OFF_BAR + 256;
 constexpr uint32_t OFF_FLAG = OFF_BAR + 264;  // [2] per-group abort flags
 constexpr uint32_t OFF_VOTE = OFF_BAR + 272;  // [2 step parities][2 groups][4 warps] "new maximum" votes
@@ -46,8 +50,8 @@ constexpr uint32_t OFF_L = OFF_ALPHA + 256;   // [2][32] 1/l for the epilogue
 constexpr uint32_t SMEM_BYTES = OFF_L + 256 + 1024;
 constexpr uint32_t TMEM_COLS = 256;  // S^T[b] at 64b (b = 0,1), O^T[ob] at 128 + 64ob
 enum {
-  B_QF = 0, B_QE = 2, B_KF = 4, B_VF = 6, B_KVE = 8, B_SF = 10, B_PF = 12, B_PFREE = 13, B_OR = 14, B_OFREE = 16,
-  B_FIN = 18, NBAR = 19
+  B_QF = 0, B_QE = 1, B_KF = 2, B_KE = 5, B_VF = 8, B_VE = 10, B_SF = 12, B_PF = 14, B_PFREE = 15, B_OR = 16,
+  B_OFREE = 18, B_FIN = 20, NBAR = 21
 };
 }  // namespace fwd
 
@@ -100,54 +104,60 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   const bool split_pv = a.out_f32 != nullptr;
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ producer
-    if (lane == 0 && !skip_all && !(a.debug & 1u)) {
-      uint32_t gs = 0;  // global step counter (K/V ring)
+    // ------------------------------------------------------------------ producers
+    if (lane < 2 && !skip_all && !(a.debug & 1u)) {
+      const bool kq = lane == 0;  // lane 0: Q and K tiles; lane 1: V tiles
+      const CUtensorMap* tmap = kq ? &tm_k : &tm_v;
+      uint32_t gs = 0;            // global step counter
       int issued_q = 0;
       bool ok = true;
       for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
         const int bh = it / g.T, i = it % g.T;
-        const int cnt = list_count(a, bh, i, true);
-        const int qb = n & 1;
-        if (n >= 2 && !mbar_wait(&bars[B_QE + qb], ((n >> 1) + 1) & 1, a.st, a.timeout_ns, 11)) break;
-        const int row0 = bh * g.Npad + i * 64;
-        mbar_arrive_expect_tx(&bars[B_QF + qb], 16384);
-        tma_load_2d(smem + OFF_Q + qb * 16384, &tm_q, &bars[B_QF + qb], 0, row0);
-        tma_load_2d(smem + OFF_Q + qb * 16384 + 8192, &tm_q, &bars[B_QF + qb], 64, row0);
-        ++issued_q;
+        const int cnt = list_count(a, bh, i, kq);
+        if (kq) {
+          if (n >= 1 && !mbar_wait(&bars[B_QE], (n - 1) & 1, a.st, a.timeout_ns, 11)) break;
+          const int row0 = bh * g.Npad + i * 64;
+          mbar_arrive_expect_tx(&bars[B_QF], 16384);
+          tma_load_2d(smem + OFF_Q, &tm_q, &bars[B_QF], 0, row0);
+          tma_load_2d(smem + OFF_Q + 8192, &tm_q, &bars[B_QF], 64, row0);
+          ++issued_q;
+        }
         const int nsteps = (cnt + 1) >> 1;
         for (int s = 0; s < nsteps; ++s) {
-          const uint32_t st = gs & 1;
-          if (gs >= 2 && !mbar_wait(&bars[B_KVE + st], ((gs >> 1) + 1) & 1, a.st, a.timeout_ns, 12)) {
-            ok = false;
-            break;
+          uint32_t st, full;
+          if (kq) {
+            st = gs % KST;
+            if (gs >= KST && !mbar_wait(&bars[B_KE + st], ((gs / KST) + 1) & 1, a.st, a.timeout_ns, 12)) {
+              ok = false;
+              break;
+            }
+            full = B_KF + st;
+          } else {
+            st = gs % VST;
+            if (gs >= VST && !mbar_wait(&bars[B_VE + st], ((gs / VST) + 1) & 1, a.st, a.timeout_ns, 12)) {
+              ok = false;
+              break;
+            }
+            full = B_VF + st;
           }
-          const int j0 = list_entry(a, bh, i, cnt, 2 * s, true);
-          const int j1 = list_entry(a, bh, i, cnt, 2 * s + 1, true);
+          const int j0 = list_entry(a, bh, i, cnt, 2 * s, kq);
+          const int j1 = list_entry(a, bh, i, cnt, 2 * s + 1, kq);
           const int y0 = j0 >= 0 ? bh * g.Npad + j0 * 64 : a.rows_total;
           const int y1 = j1 >= 0 ? bh * g.Npad + j1 * 64 : a.rows_total;
-          uint8_t* kst = smem + OFF_K + st * 32768;
-          uint8_t* vst = smem + OFF_V + st * 32768;
-          mbar_arrive_expect_tx(&bars[B_KF + st], 32768);
-          tma_load_2d(kst, &tm_k, &bars[B_KF + st], 0, y0);
-          tma_load_2d(kst + 8192, &tm_k, &bars[B_KF + st], 0, y1);
-          tma_load_2d(kst + 16384, &tm_k, &bars[B_KF + st], 64, y0);
-          tma_load_2d(kst + 24576, &tm_k, &bars[B_KF + st], 64, y1);
-          mbar_arrive_expect_tx(&bars[B_VF + st], 32768);
-          tma_load_2d(vst, &tm_v, &bars[B_VF + st], 0, y0);
-          tma_load_2d(vst + 8192, &tm_v, &bars[B_VF + st], 0, y1);
-          tma_load_2d(vst + 16384, &tm_v, &bars[B_VF + st], 64, y0);
-          tma_load_2d(vst + 24576, &tm_v, &bars[B_VF + st], 64, y1);
+          uint8_t* dst = smem + (kq ? OFF_K : OFF_V) + st * 32768;
+          mbar_arrive_expect_tx(&bars[full], 32768);
+          tma_load_2d(dst, tmap, &bars[full], 0, y0);
+          tma_load_2d(dst + 8192, tmap, &bars[full], 0, y1);
+          tma_load_2d(dst + 16384, tmap, &bars[full], 64, y0);
+          tma_load_2d(dst + 24576, tmap, &bars[full], 64, y1);
           ++gs;
         }
       }
       // drain: never leave the CTA with copies in flight
-      for (int n = (issued_q > 2 ? issued_q - 2 : 0); n < issued_q; ++n)
-        mbar_wait(&bars[B_QF + (n & 1)], (n >> 1) & 1, a.st, a.timeout_ns, 13);
-      for (uint32_t s = (gs > 2 ? gs - 2 : 0); s < gs; ++s) {
-        mbar_wait(&bars[B_KF + (s & 1)], (s >> 1) & 1, a.st, a.timeout_ns, 14);
-        mbar_wait(&bars[B_VF + (s & 1)], (s >> 1) & 1, a.st, a.timeout_ns, 15);
-      }
+      if (kq && issued_q > 0) mbar_wait(&bars[B_QF], (issued_q - 1) & 1, a.st, a.timeout_ns, 13);
+      const uint32_t nst = kq ? KST : VST;
+      for (uint32_t s = (gs > nst ? gs - nst : 0); s < gs; ++s)
+        mbar_wait(&bars[(kq ? B_KF : B_VF) + s % nst], (s / nst) & 1, a.st, a.timeout_ns, 14);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -158,37 +168,37 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       const int nk_pv = split_pv ? 16 : 8;
       uint32_t gs_s = 0, gs_o = 0;  // global steps whose S (resp. PV) product was issued
       bool ok = true;
-      // S^T for the next global step, from the Q buffer qb.  Its S buffer (gs_s & 1) was
+      // S^T for the next global step.  Its S buffer (gs_s & 1) was
       // last read by the softmax of step gs_s - 2, whose P_FULL arrival this thread has
       // already waited for before issuing PV(gs_s - 2).
-      auto issue_s = [&](int qb) -> bool {
-        const uint32_t st = gs_s & 1;
-        if (!mbar_wait(&bars[B_KF + st], (gs_s >> 1) & 1, a.st, a.timeout_ns, 21)) return false;
+      auto issue_s = [&]() -> bool {
+        const uint32_t kst_i = gs_s % KST, sb = gs_s & 1;
+        if (!mbar_wait(&bars[B_KF + kst_i], (gs_s / KST) & 1, a.st, a.timeout_ns, 21)) return false;
         tc_fence_after();
-        const uint32_t kst = sbase + OFF_K + st * 32768;
-        const uint32_t qs = sbase + OFF_Q + qb * 16384;
+        const uint32_t kst = sbase + OFF_K + kst_i * 32768;
         for (int ks = 0; ks < ksteps; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
           const uint32_t qoff = (ks >> 2) * 8192 + (ks & 3) * 32;
-          umma_f16_ss(tmem + st * 64, sw128_desc(kst + off, 16, 1024), sw128_desc(qs + qoff, 16, 1024), idesc_s,
-                      ks > 0 ? 1u : 0u);
+          umma_f16_ss(tmem + sb * 64, sw128_desc(kst + off, 16, 1024), sw128_desc(sbase + OFF_Q + qoff, 16, 1024),
+                      idesc_s, ks > 0 ? 1u : 0u);
         }
-        umma_commit(&bars[B_SF + st]);
+        umma_commit(&bars[B_SF + sb]);
+        umma_commit(&bars[B_KE + kst_i]);  // the K stage is free once this product completes
         ++gs_s;
         return true;
       };
       for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
         const int bh = it / g.T, i = it % g.T;
         const int nsteps = (list_count(a, bh, i, false) + 1) >> 1;
-        const int qb = n & 1, ob = n & 1;
-        if (!mbar_wait(&bars[B_QF + qb], (n >> 1) & 1, a.st, a.timeout_ns, 22)) break;
-        for (int s = 0; ok && s < nsteps && s < 2; ++s) ok = issue_s(qb);
+        const int ob = n & 1;
+        if (!mbar_wait(&bars[B_QF], n & 1, a.st, a.timeout_ns, 22)) break;
+        for (int s = 0; ok && s < nsteps && s < 2; ++s) ok = issue_s();
         if (ok && n >= 2 && nsteps > 0)
           ok = mbar_wait(&bars[B_OFREE + ob], ((n >> 1) + 1) & 1, a.st, a.timeout_ns, 23);
         for (int s = 0; ok && s < nsteps; ++s) {
-          const uint32_t st = gs_o & 1;
+          const uint32_t st = gs_o % VST;
           ok = mbar_wait(&bars[B_PF], gs_o & 1, a.st, a.timeout_ns, 24) &&
-               mbar_wait(&bars[B_VF + st], (gs_o >> 1) & 1, a.st, a.timeout_ns, 25);
+               mbar_wait(&bars[B_VF + st], (gs_o / VST) & 1, a.st, a.timeout_ns, 25);
           if (!ok) break;
           tc_fence_after();
           const uint32_t vst = sbase + OFF_V + st * 32768;
@@ -199,13 +209,13 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
                         sw128_desc(sbase + OFF_P + part * 16384 + kk * 2048, 8192, 1024), idesc_o,
                         (s > 0 || ks > 0) ? 1u : 0u);
           }
-          umma_commit(&bars[B_KVE + st]);
+          umma_commit(&bars[B_VE + st]);
           umma_commit(&bars[B_PFREE]);
           ++gs_o;
-          if (s + 2 < nsteps) ok = issue_s(qb);
+          if (s + 2 < nsteps) ok = issue_s();
         }
         if (!ok) break;
-        umma_commit(&bars[B_QE + qb]);  // every product reading this Q buffer has been issued
+        umma_commit(&bars[B_QE]);       // every product reading Q has been issued
         umma_commit(&bars[B_OR + ob]);  // O^T of this cube is final once these complete
       }
       // every issued product must complete before TMEM is freed
