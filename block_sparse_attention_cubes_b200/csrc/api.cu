@@ -57,6 +57,7 @@ double softmax_scale(const sa_params* p) {
 
 struct WsLayout {
   size_t cmask = 0;                                        // forward, backward: [T] cube masks
+  size_t ulist = 0, ucnt = 0;                              // forward: query-pair union lists
   size_t qbar = 0, kbar = 0, scores = 0;                   // plan
   size_t delta = 0, qcnt = 0, qoff = 0, qidx = 0;          // backward
   size_t total = 0;
@@ -76,6 +77,11 @@ WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
   } else if (op == SA_OP_FORWARD) {
     w.cmask = off;
     off = align256(off + static_cast<size_t>(g.T) * sizeof(unsigned long long));
+    const size_t P = static_cast<size_t>((g.T + 1) / 2);
+    w.ucnt = off;
+    off = align256(off + BH * P * sizeof(int32_t));
+    w.ulist = off;
+    off = align256(off + BH * P * 2 * static_cast<size_t>(p->kv_capacity) * sizeof(int32_t));
   } else if (op == SA_OP_BACKWARD) {
     w.cmask = off;
     off = align256(off + static_cast<size_t>(g.T) * sizeof(unsigned long long));
@@ -249,12 +255,17 @@ sa_status sa_forward(const void* q, const void* k, const void* v, const float* q
       !make_map(&tv, v, a.rows_total, p->D, 2))
     return SA_ERR_LAUNCH;
   if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
-  a.cube_mask = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(ws) + w.cmask);
-  if (sa::launch_cube_mask(g, reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(ws) + w.cmask), st) !=
-      cudaSuccess)
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  a.cube_mask = reinterpret_cast<unsigned long long*>(wb + w.cmask);
+  a.u_list = reinterpret_cast<int32_t*>(wb + w.ulist);
+  a.u_cnt = reinterpret_cast<int32_t*>(wb + w.ucnt);
+  if (sa::launch_cube_mask(g, reinterpret_cast<unsigned long long*>(wb + w.cmask), st) != cudaSuccess ||
+      sa::launch_query_pair_union(kv_index, kv_count, reinterpret_cast<int32_t*>(wb + w.ulist),
+                                  reinterpret_cast<int32_t*>(wb + w.ucnt), a.BH, g.T, p->kv_capacity, a.st,
+                                  st) != cudaSuccess)
     return SA_ERR_LAUNCH;
   if (sa::launch_forward(tq, tk, tv, a, st) != cudaSuccess) return SA_ERR_LAUNCH;
-  g_last_launches = 2;
+  g_last_launches = 3;
   return SA_OK;
 }
 

@@ -6,6 +6,7 @@
 #include <cstdint>
 
 #include "geometry.cuh"
+#include "ptx.cuh"
 
 namespace sa {
 
@@ -19,6 +20,11 @@ cudaError_t launch_plan(const void* q, const void* k, const float* q_scale, cons
                         int BH, int D, bool fp8, double scale, int top_k, float top_p, int cap, int32_t* kv_index,
                         int32_t* kv_count, double* qbar, double* kbar, double* S, DevStatus* st,
                         cudaStream_t stream, int* launches);
+
+cudaError_t launch_query_pair_union(const int32_t* kv_index, const int32_t* kv_count, int32_t* u_list,
+                                    int32_t* u_cnt, int BH, int T, int cap, DevStatus* st, cudaStream_t stream);
+cudaError_t launch_key_pair_union(const int32_t* q_off, const int32_t* q_idx, int32_t* u_list, int32_t* u_cnt,
+                                  int BH, int T, int cap, cudaStream_t stream);
 
 cudaError_t launch_cube_mask(const Geom& g, unsigned long long* mask, cudaStream_t stream);
 int num_sms();

@@ -84,7 +84,8 @@ SA_API int sa_topk_from_fraction(double frac, int T);
 
 /* Bytes of device workspace `op` (sa_op) needs for these parameters; 0 on bad input.
  * Plan: status block + pooled Q and K (fp64) + block scores (fp64, B*H*T*T).
- * Forward: status block + one 64-bit valid-slot mask per cube (T).  Backward: status block
+ * Forward: status block + one 64-bit valid-slot mask per cube (T) + the union lists of
+ * adjacent query-cube pairs (int32, B*H*ceil(T/2)*(1 + 2*kv_capacity)).  Backward: status block
  * + cube masks + Delta (fp32, B*H*Npad) + the transposed index lists (int32,
  * B*H*(2T+1) + B*H*T*kv_capacity). */
 SA_API size_t sa_workspace_size(const sa_params* p, int op);
