@@ -55,11 +55,14 @@ double softmax_scale(const sa_params* p) {
   return p->softmax_scale > 0.0f ? static_cast<double>(p->softmax_scale) : 1.0 / std::sqrt(static_cast<double>(p->D));
 }
 
+int union_cap(const sa_params* p, const Geom& g) { return 2 * p->kv_capacity < g.T ? 2 * p->kv_capacity : g.T; }
+
 struct WsLayout {
   size_t cmask = 0;                                        // forward, backward: [T] cube masks
   size_t ulist = 0, ucnt = 0;                              // forward: query-pair union lists
   size_t qbar = 0, kbar = 0, scores = 0;                   // plan
   size_t delta = 0, qcnt = 0, qoff = 0, qidx = 0;          // backward
+  size_t ukcnt = 0, uklist = 0;                            // backward: key-pair unions
   size_t total = 0;
 };
 
@@ -81,7 +84,7 @@ WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
     w.ucnt = off;
     off = align256(off + BH * P * sizeof(int32_t));
     w.ulist = off;
-    off = align256(off + BH * P * 2 * static_cast<size_t>(p->kv_capacity) * sizeof(int32_t));
+    off = align256(off + BH * P * static_cast<size_t>(union_cap(p, g)) * sizeof(int32_t));
   } else if (op == SA_OP_BACKWARD) {
     w.cmask = off;
     off = align256(off + static_cast<size_t>(g.T) * sizeof(unsigned long long));
@@ -93,6 +96,15 @@ WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
     off = align256(off + BH * (g.T + 1) * sizeof(int32_t));
     w.qidx = off;
     off = align256(off + BH * g.T * static_cast<size_t>(p->kv_capacity) * sizeof(int32_t));
+    const size_t P = static_cast<size_t>((g.T + 1) / 2);
+    w.ucnt = off;
+    off = align256(off + BH * P * sizeof(int32_t));
+    w.ulist = off;
+    off = align256(off + BH * P * static_cast<size_t>(union_cap(p, g)) * sizeof(int32_t));
+    w.ukcnt = off;
+    off = align256(off + BH * P * sizeof(int32_t));
+    w.uklist = off;
+    off = align256(off + BH * P * static_cast<size_t>(g.T) * sizeof(int32_t));
   }
   w.total = off;
   return w;
@@ -259,6 +271,7 @@ sa_status sa_forward(const void* q, const void* k, const void* v, const float* q
   a.cube_mask = reinterpret_cast<unsigned long long*>(wb + w.cmask);
   a.u_list = reinterpret_cast<int32_t*>(wb + w.ulist);
   a.u_cnt = reinterpret_cast<int32_t*>(wb + w.ucnt);
+  a.ucap = union_cap(p, g);
   if (sa::launch_cube_mask(g, reinterpret_cast<unsigned long long*>(wb + w.cmask), st) != cudaSuccess ||
       sa::launch_query_pair_union(kv_index, kv_count, reinterpret_cast<int32_t*>(wb + w.ulist),
                                   reinterpret_cast<int32_t*>(wb + w.ucnt), a.BH, g.T, p->kv_capacity, a.st,
@@ -304,9 +317,12 @@ sa_status sa_backward(const void* q, const void* k, const void* v, const void* o
   if (sa::launch_cube_mask(g, reinterpret_cast<unsigned long long*>(wb + w.cmask), st) != cudaSuccess)
     return SA_ERR_LAUNCH;
   int launches = 0;
+  a.ucap = union_cap(p, g);
   if (sa::launch_backward(tq, tk, tv, tdo, out, out_f32, dout, a, reinterpret_cast<int32_t*>(wb + w.qcnt),
                           reinterpret_cast<int32_t*>(wb + w.qoff), reinterpret_cast<int32_t*>(wb + w.qidx),
-                          reinterpret_cast<float*>(wb + w.delta), st, &launches) != cudaSuccess)
+                          reinterpret_cast<float*>(wb + w.delta), reinterpret_cast<int32_t*>(wb + w.ulist),
+                          reinterpret_cast<int32_t*>(wb + w.ucnt), reinterpret_cast<int32_t*>(wb + w.uklist),
+                          reinterpret_cast<int32_t*>(wb + w.ukcnt), st, &launches) != cudaSuccess)
     return SA_ERR_LAUNCH;
   g_last_launches = launches + 1;
   return SA_OK;

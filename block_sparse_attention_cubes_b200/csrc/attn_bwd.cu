@@ -9,14 +9,12 @@
 //   delta_kernel      Delta per query row (one warp per row).
 //   count/scan/fill   the transposed lists: for each key cube j the ascending query cubes
 //                     whose list holds j (CSR, deterministic).
-//   attn_dq_kernel    per query cube, transposed like the forward: over pairs of its key
-//                     tiles, S^T = K2 Q^T and dP^T = V2 dO^T (M=128), dS^T in shared memory,
-//                     dQ^T += K2^T dS^T (M=D).
-//   attn_dkdv_kernel  per key cube, over pairs of the query cubes that selected it:
-//                     S = Q2 K^T and dP = dO2 V^T (M=128 query rows), P and dS in shared
-//                     memory, dV^T += dO2^T P and dK^T += Q2^T dS (M=D).
-// Both main kernels keep every accumulator in TMEM and use the same warp roles as the
-// forward (TMA producer, MMA issuer, 128-thread elementwise group).
+//   pair unions       (pairs.cu) query-cube pairs over their KV lists, key-cube pairs over
+//                     their transposed lists.
+//   attn_dq_kernel    row form over query-cube pairs (M = 128 rows, N = 128 keys).
+//   attn_dkdv_kernel  transposed form over key-cube pairs (M = 128 keys, N = 128 queries).
+// All products are full-rate 128 x 128 tcgen05 MMAs with accumulators in TMEM; P and dS
+// enter the dV, dK and dQ products as bf16 hi + lo pairs read from TMEM.
 #include <cmath>
 
 #include "attn_common.cuh"
@@ -132,21 +130,28 @@ __global__ void __launch_bounds__(256) fill_kernel(const int32_t* __restrict__ k
 }
 
 // ------------------------------------------------------------------------ dQ
+// One item = two adjacent query cubes (128 rows) over the union of their KV lists, two key
+// tiles per step:  S = Q2 K2^T,  dP = dO2 V2^T  (SS, N=128),  P = exp(S*scale - lse),
+// dS = P (dP - Delta) written as bf16 hi + lo into this step's S columns of TMEM, and
+// dQ += dS K2 as a TS product (N = D).  Thread r of group g owns row r and the 64 keys of
+// tile t_g, and writes its dS over its own S columns, so the groups never wait on each
+// other.  S is double-buffered; dQ(s) overlaps the elementwise work of step s + 1.
 namespace dqk {
-constexpr int kThreads = 192;
-constexpr uint32_t OFF_Q = 0;          // [2 halves][64][128 B]
-constexpr uint32_t OFF_DO = 16384;     // same
-constexpr uint32_t OFF_K = 32768;      // 2 stages x [2 halves][128][128 B]
-constexpr uint32_t OFF_V = 98304;      // same
-constexpr uint32_t OFF_DS = 163840;    // 2 buffers x {hi, lo} x [128 keys][64 q] bf16
-constexpr uint32_t OFF_BAR = 229376;
-constexpr uint32_t OFF_SLOT = OFF_BAR + 192;
-constexpr uint32_t OFF_FLAG = OFF_BAR + 200;
-constexpr uint32_t OFF_LSE = OFF_BAR + 256;    // [64] lse * log2(e)
-constexpr uint32_t OFF_DELTA = OFF_LSE + 256;  // [64]
-constexpr uint32_t SMEM_BYTES = OFF_DELTA + 256 + 1024;
-constexpr uint32_t TMEM_COLS = 512;  // S^T[b] at 128b, dP^T[b] at 128b+64, dQ^T at 256
-enum { B_QD = 0, B_KF = 1, B_VF = 3, B_EMPTY = 5, B_SDP = 7, B_DSF = 9, B_DSFREE = 11, B_FIN = 13, NBAR = 14 };
+constexpr int kThreads = 320;
+constexpr int KST = 3, VST = 2;
+constexpr uint32_t OFF_Q = 0;       // Q2  [2 halves][128 rows][128 B]
+constexpr uint32_t OFF_DO = 32768;  // dO2 same
+constexpr uint32_t OFF_K = 65536;   // KST x [2 halves][128 keys][128 B]
+constexpr uint32_t OFF_V = OFF_K + KST * 32768;
+constexpr uint32_t OFF_BAR = OFF_V + VST * 32768;
+constexpr uint32_t OFF_SLOT = OFF_BAR + 256;
+constexpr uint32_t OFF_ABORT = OFF_BAR + 264;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;
+constexpr uint32_t TMEM_COLS = 512;  // S/dS[b] at 128b, dP at 256, dQ at 384
+enum {
+  B_QF = 0, B_QE = 1, B_KF = 2, B_KE = 5, B_VF = 8, B_VE = 10, B_SF = 12, B_DPF = 14, B_PF = 15, B_DQR = 16,
+  B_DQFREE = 17, B_FIN = 18, NBAR = 19
+};
 }  // namespace dqk
 
 __global__ void __launch_bounds__(dqk::kThreads, 1)
@@ -159,18 +164,16 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_SLOT);
-  volatile int* grp_abort = reinterpret_cast<volatile int*>(smem + OFF_FLAG);
-  float* lse2_sh = reinterpret_cast<float*>(smem + OFF_LSE);
-  float* delta_sh = reinterpret_cast<float*>(smem + OFF_DELTA);
+  volatile int* sm_abort = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.x % a.g.T;
-  const int bh = blockIdx.x / a.g.T;
   const Geom& g = a.g;
+  const int npairs = (g.T + 1) >> 1;
+  const int n_items = a.BH * npairs;
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < NBAR; ++b) mbar_init(&bars[b], (b == B_DSF || b == B_DSF + 1) ? 128u : 1u);
-    *grp_abort = aborted(a.st) ? 1 : 0;
+    for (int b = 0; b < NBAR; ++b) mbar_init(&bars[b], b == B_PF ? 256u : (b == B_DQFREE ? 8u : 1u));
+    *sm_abort = aborted(a.st) ? 1 : 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -181,159 +184,225 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const bool skip_all = *grp_abort != 0;
-  const int n = list_count(a, bh, i, threadIdx.x == 0);
-  const int nsteps = skip_all ? 0 : (n + 1) >> 1;
-  const int row0 = bh * g.Npad + i * 64;
+  const bool skip_all = *sm_abort != 0;
 
   if (warp == 0) {
-    if (lane == 0 && nsteps > 0) {
-      mbar_arrive_expect_tx(&bars[B_QD], 32768);
-      tma_load_2d(smem + OFF_Q, &tm_q, &bars[B_QD], 0, row0);
-      tma_load_2d(smem + OFF_Q + 8192, &tm_q, &bars[B_QD], 64, row0);
-      tma_load_2d(smem + OFF_DO, &tm_do, &bars[B_QD], 0, row0);
-      tma_load_2d(smem + OFF_DO + 8192, &tm_do, &bars[B_QD], 64, row0);
-      int issued = 0;
-      for (int s = 0; s < nsteps; ++s) {
-        const int st = s & 1;
-        if (s >= 2 && !mbar_wait(&bars[B_EMPTY + st], ((s >> 1) + 1) & 1, a.st, a.timeout_ns, 41)) break;
-        const int j0 = list_entry(a, bh, i, n, 2 * s, true);
-        const int j1 = list_entry(a, bh, i, n, 2 * s + 1, true);
-        const int y0 = j0 >= 0 ? bh * g.Npad + j0 * 64 : a.rows_total;
-        const int y1 = j1 >= 0 ? bh * g.Npad + j1 * 64 : a.rows_total;
-        uint8_t* kst = smem + OFF_K + st * 32768;
-        uint8_t* vst = smem + OFF_V + st * 32768;
-        mbar_arrive_expect_tx(&bars[B_KF + st], 32768);
-        tma_load_2d(kst, &tm_k, &bars[B_KF + st], 0, y0);
-        tma_load_2d(kst + 8192, &tm_k, &bars[B_KF + st], 0, y1);
-        tma_load_2d(kst + 16384, &tm_k, &bars[B_KF + st], 64, y0);
-        tma_load_2d(kst + 24576, &tm_k, &bars[B_KF + st], 64, y1);
-        mbar_arrive_expect_tx(&bars[B_VF + st], 32768);
-        tma_load_2d(vst, &tm_v, &bars[B_VF + st], 0, y0);
-        tma_load_2d(vst + 8192, &tm_v, &bars[B_VF + st], 0, y1);
-        tma_load_2d(vst + 16384, &tm_v, &bars[B_VF + st], 64, y0);
-        tma_load_2d(vst + 24576, &tm_v, &bars[B_VF + st], 64, y1);
-        ++issued;
+    if (lane < 2 && !skip_all) {
+      const bool kq = lane == 0;  // lane 0: Q2, dO2 and K tiles; lane 1: V tiles
+      const CUtensorMap* tmap = kq ? &tm_k : &tm_v;
+      uint32_t gs = 0;
+      int issued_q = 0;
+      bool ok = true;
+      for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+        const int bh = it / npairs, pr = it % npairs;
+        const int nu = a.u_cnt[it];
+        const int32_t* ul = a.u_list + static_cast<size_t>(it) * a.ucap;
+        if (kq) {
+          if (n >= 1 && !mbar_wait(&bars[B_QE], (n - 1) & 1, a.st, a.timeout_ns, 41)) break;
+          const int r0 = bh * g.Npad + (2 * pr) * 64;
+          const int r1 = (2 * pr + 1 < g.T) ? r0 + 64 : a.rows_total;
+          mbar_arrive_expect_tx(&bars[B_QF], 65536);
+          tma_load_2d(smem + OFF_Q, &tm_q, &bars[B_QF], 0, r0);
+          tma_load_2d(smem + OFF_Q + 8192, &tm_q, &bars[B_QF], 0, r1);
+          tma_load_2d(smem + OFF_Q + 16384, &tm_q, &bars[B_QF], 64, r0);
+          tma_load_2d(smem + OFF_Q + 24576, &tm_q, &bars[B_QF], 64, r1);
+          tma_load_2d(smem + OFF_DO, &tm_do, &bars[B_QF], 0, r0);
+          tma_load_2d(smem + OFF_DO + 8192, &tm_do, &bars[B_QF], 0, r1);
+          tma_load_2d(smem + OFF_DO + 16384, &tm_do, &bars[B_QF], 64, r0);
+          tma_load_2d(smem + OFF_DO + 24576, &tm_do, &bars[B_QF], 64, r1);
+          ++issued_q;
+        }
+        const int nsteps = (nu + 1) >> 1;
+        for (int s = 0; s < nsteps; ++s) {
+          const uint32_t nst = kq ? KST : VST;
+          const uint32_t st = gs % nst;
+          if (gs >= nst &&
+              !mbar_wait(&bars[(kq ? B_KE : B_VE) + st], ((gs / nst) + 1) & 1, a.st, a.timeout_ns, 42)) {
+            ok = false;
+            break;
+          }
+          const int t0 = ul[2 * s] >> 2;
+          const int t1 = (2 * s + 1 < nu) ? (ul[2 * s + 1] >> 2) : -1;
+          const int y0 = bh * g.Npad + t0 * 64;
+          const int y1 = t1 >= 0 ? bh * g.Npad + t1 * 64 : a.rows_total;
+          const uint32_t full = (kq ? B_KF : B_VF) + st;
+          uint8_t* dst = smem + (kq ? OFF_K : OFF_V) + st * 32768;
+          mbar_arrive_expect_tx(&bars[full], 32768);
+          tma_load_2d(dst, tmap, &bars[full], 0, y0);
+          tma_load_2d(dst + 8192, tmap, &bars[full], 0, y1);
+          tma_load_2d(dst + 16384, tmap, &bars[full], 64, y0);
+          tma_load_2d(dst + 24576, tmap, &bars[full], 64, y1);
+          ++gs;
+        }
       }
-      mbar_wait(&bars[B_QD], 0, a.st, a.timeout_ns, 42);
-      for (int s = (issued > 2 ? issued - 2 : 0); s < issued; ++s) {
-        mbar_wait(&bars[B_KF + (s & 1)], (s >> 1) & 1, a.st, a.timeout_ns, 43);
-        mbar_wait(&bars[B_VF + (s & 1)], (s >> 1) & 1, a.st, a.timeout_ns, 44);
-      }
+      if (kq && issued_q > 0) mbar_wait(&bars[B_QF], (issued_q - 1) & 1, a.st, a.timeout_ns, 43);
+      const uint32_t nst = kq ? KST : VST;
+      for (uint32_t s = (gs > nst ? gs - nst : 0); s < gs; ++s)
+        mbar_wait(&bars[(kq ? B_KF : B_VF) + s % nst], (s / nst) & 1, a.st, a.timeout_ns, 44);
     }
   } else if (warp == 1) {
-    if (lane == 0 && nsteps > 0) {
-      const uint32_t idesc_kk = make_idesc(128, 64, FMT_BF16, false, false);
-      const uint32_t idesc_mn = make_idesc(128, 64, FMT_BF16, true, true);
+    if (lane == 0 && !skip_all) {
+      const uint32_t idesc_kk = make_idesc(128, 128, FMT_BF16, false, false);
+      const uint32_t idesc_q = make_idesc(128, 128, FMT_BF16, false, true);
       const int ksteps = a.D / 16;
-      auto issue_sdp = [&](int s) {
-        const int st = s & 1;
-        const uint32_t kst = sbase + OFF_K + st * 32768, vst = sbase + OFF_V + st * 32768;
-        const uint32_t d_s = tmem + st * 128, d_dp = tmem + st * 128 + 64;
+      uint32_t gs_s = 0, gs_p = 0, gs_q = 0;  // global steps whose S, dP, dQ products were issued
+      bool ok = true;
+      auto issue_s = [&]() -> bool {
+        const uint32_t ks_i = gs_s % KST, sb = gs_s & 1;
+        if (!mbar_wait(&bars[B_KF + ks_i], (gs_s / KST) & 1, a.st, a.timeout_ns, 51)) return false;
+        tc_fence_after();
+        const uint32_t kst = sbase + OFF_K + ks_i * 32768;
         for (int ks = 0; ks < ksteps; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          const uint32_t qoff = (ks >> 2) * 8192 + (ks & 3) * 32;
-          umma_f16_ss(d_s, sw128_desc(kst + off, 16, 1024), sw128_desc(sbase + OFF_Q + qoff, 16, 1024), idesc_kk,
-                      ks > 0 ? 1u : 0u);
-        }
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          const uint32_t qoff = (ks >> 2) * 8192 + (ks & 3) * 32;
-          umma_f16_ss(d_dp, sw128_desc(vst + off, 16, 1024), sw128_desc(sbase + OFF_DO + qoff, 16, 1024),
+          umma_f16_ss(tmem + sb * 128, sw128_desc(sbase + OFF_Q + off, 16, 1024), sw128_desc(kst + off, 16, 1024),
                       idesc_kk, ks > 0 ? 1u : 0u);
         }
-        umma_commit(&bars[B_SDP + st]);
+        umma_commit(&bars[B_SF + sb]);
+        ++gs_s;
+        return true;
       };
-      bool ok = mbar_wait(&bars[B_QD], 0, a.st, a.timeout_ns, 51);
-      for (int s = 0; ok && s < 2 && s < nsteps; ++s) {
-        ok = mbar_wait(&bars[B_KF + s], 0, a.st, a.timeout_ns, 52) &&
-             mbar_wait(&bars[B_VF + s], 0, a.st, a.timeout_ns, 53);
-        if (ok) {
-          tc_fence_after();
-          issue_sdp(s);
-        }
-      }
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int st = s & 1;
-        if (!mbar_wait(&bars[B_DSF + st], (s >> 1) & 1, a.st, a.timeout_ns, 54)) break;
+      auto issue_dp = [&]() -> bool {
+        const uint32_t vs = gs_p % VST;
+        if (!mbar_wait(&bars[B_VF + vs], (gs_p / VST) & 1, a.st, a.timeout_ns, 52)) return false;
         tc_fence_after();
-        const uint32_t kst = sbase + OFF_K + st * 32768;
-        const uint32_t dsb = sbase + OFF_DS + st * 32768;
-#pragma unroll 1
-        for (int ks = 0; ks < 16; ++ks) {  // 8 k-steps over dS_hi, then 8 over dS_lo
-          const uint32_t kk = ks & 7, part = ks >> 3;
-          umma_f16_ss(tmem + 256, sw128_desc(kst + kk * 2048, 16384, 1024),
-                      sw128_desc(dsb + part * 16384 + kk * 2048, 8192, 1024), idesc_mn, (s > 0 || ks > 0) ? 1u : 0u);
+        const uint32_t vst = sbase + OFF_V + vs * 32768;
+        for (int ks = 0; ks < ksteps; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          umma_f16_ss(tmem + 256, sw128_desc(sbase + OFF_DO + off, 16, 1024), sw128_desc(vst + off, 16, 1024),
+                      idesc_kk, ks > 0 ? 1u : 0u);
         }
-        umma_commit(&bars[B_EMPTY + st]);
-        umma_commit(&bars[B_DSFREE + st]);
-        if (s + 2 < nsteps) {
-          ok = mbar_wait(&bars[B_KF + st], ((s + 2) >> 1) & 1, a.st, a.timeout_ns, 55) &&
-               mbar_wait(&bars[B_VF + st], ((s + 2) >> 1) & 1, a.st, a.timeout_ns, 56);
-          if (!ok) break;
+        umma_commit(&bars[B_DPF]);
+        umma_commit(&bars[B_VE + vs]);
+        ++gs_p;
+        return true;
+      };
+      for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+        const int nsteps = (a.u_cnt[it] + 1) >> 1;
+        if (!mbar_wait(&bars[B_QF], n & 1, a.st, a.timeout_ns, 53)) break;
+        if (nsteps > 0) ok = issue_s() && issue_dp();
+        if (ok && n >= 1 && nsteps > 0) ok = mbar_wait(&bars[B_DQFREE], (n - 1) & 1, a.st, a.timeout_ns, 54);
+        for (int s = 0; ok && s < nsteps; ++s) {
+          // S(s+1) goes to the other S buffer, whose dS(s-1) was read by the earlier dQ(s-1)
+          if (s + 1 < nsteps) ok = issue_s();
+          if (!ok || !mbar_wait(&bars[B_PF], gs_q & 1, a.st, a.timeout_ns, 55)) {
+            ok = false;
+            break;
+          }
+          // dP(s) has been read: its buffer takes dP(s+1), issued ahead of dQ(s)
+          if (s + 1 < nsteps && !issue_dp()) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          issue_sdp(s + 2);
+          const uint32_t ks_i = gs_q % KST, sb = gs_q & 1;
+          const uint32_t kst = sbase + OFF_K + ks_i * 32768;
+#pragma unroll 1
+          for (int ks = 0; ks < 16; ++ks) {  // 8 k-steps over dS_hi, then 8 over dS_lo
+            const uint32_t kk = ks & 7, part = ks >> 3;
+            const uint32_t acol = sb * 128 + (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
+            umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(kst + kk * 2048, 16384, 1024), idesc_q,
+                        (s > 0 || ks > 0) ? 1u : 0u);
+          }
+          umma_commit(&bars[B_KE + ks_i]);  // K(s) was read by S(s) and dQ(s)
+          ++gs_q;
         }
+        if (!ok) break;
+        umma_commit(&bars[B_QE]);
+        umma_commit(&bars[B_DQR]);
       }
       umma_commit(&bars[B_FIN]);
-      mbar_wait(&bars[B_FIN], 0, a.st, a.timeout_ns, 57);
+      mbar_wait(&bars[B_FIN], 0, a.st, a.timeout_ns, 56);
     }
   } else {
+    const int grp = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
+    const int half = r >> 6;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    if (r < 64) {
-      const bool qv = token_valid(g, i, r);
-      lse2_sh[r] = qv ? a.lse[row0 + r] * 1.4426950408889634f : 0.0f;
-      delta_sh[r] = qv ? a.delta[row0 + r] : 0.0f;
-    }
-    named_bar_sync(1, 128);
-    uint64_t qmask = 0;  // valid query columns of this cube
-    for (int c = 0; c < 64; ++c)
-      if (token_valid(g, i, c)) qmask |= 1ull << c;
-    bool ok = true;
-    for (int s = 0; s < nsteps; ++s) {
-      const int b = s & 1;
-      if (!mbar_wait(&bars[B_SDP + b], (s >> 1) & 1, a.st, a.timeout_ns, 61)) *grp_abort = 1;
-      tc_fence_after();
-      float sv[64], dp[64];
-      tmem_ld64(t_lane + b * 128, sv);
-      tmem_ld64(t_lane + b * 128 + 64, dp);
-      const int tile = list_entry(a, bh, i, n, 2 * s + (r >> 6), false);
-      const bool kvalid = tile >= 0 && token_valid(g, tile, r & 63);
+    uint32_t gs = 0;
+    bool ok = !skip_all;
+    for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+      const int bh = it / npairs, pr = it % npairs;
+      const int icube = 2 * pr + half;
+      const bool row_exists = icube < g.T;
+      const bool row_valid = row_exists && ((a.cube_mask[icube] >> (r & 63)) & 1ull);
+      const size_t qrow = static_cast<size_t>(bh) * g.Npad + static_cast<size_t>(icube) * 64 + (r & 63);
+      const float lse2 = row_valid ? a.lse[qrow] * 1.4426950408889634f : 0.0f;
+      const float dlt = row_valid ? a.delta[qrow] : 0.0f;
+      const int nu = a.u_cnt[it];
+      const int32_t* ul = a.u_list + static_cast<size_t>(it) * a.ucap;
+      const int nsteps = (nu + 1) >> 1;
+      for (int s = 0; s < nsteps; ++s, ++gs) {
+        const uint32_t b = gs & 1;
+        const int e = (2 * s + grp < nu) ? ul[2 * s + grp] : 0;
+        const int tile = e >> 2;
+        const bool active = ((e >> half) & 1) && row_valid;
+        const bool w_active = __any_sync(0xffffffffu, active);
+        const bool ok1 = mbar_wait(&bars[B_SF + b], (gs >> 1) & 1, a.st, a.timeout_ns, 61);
+        const bool ok2 = mbar_wait(&bars[B_DPF], gs & 1, a.st, a.timeout_ns, 62);
+        if (!(ok1 && ok2)) *sm_abort = 1;
+        tc_fence_after();
+        uint32_t hi[32], lo[32];
+        if (w_active) {
+          uint32_t s0[32], s1[32], p0[32], p1[32];
+          tmem_ld32(t_lane + b * 128 + grp * 64, s0);
+          tmem_ld32(t_lane + b * 128 + grp * 64 + 32, s1);
+          tmem_ld32(t_lane + 256 + grp * 64, p0);
+          tmem_ld32(t_lane + 256 + grp * 64 + 32, p1);
+          tmem_ld_wait();
+          const unsigned long long km = active ? a.cube_mask[tile] : 0ull;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const bool on = kvalid && ((qmask >> c) & 1ull);
-        const float p = on ? exp2f(sv[c] * a.scale_log2 - lse2_sh[c]) : 0.0f;
-        sv[c] = p * (dp[c] - delta_sh[c]);
+          for (int c = 0; c < 32; ++c) {
+            const int c0 = 2 * c, c1 = 2 * c + 1;
+            const uint32_t sa0 = c0 < 32 ? s0[c0] : s1[c0 - 32], sa1 = c1 < 32 ? s0[c1] : s1[c1 - 32];
+            const uint32_t pa0 = c0 < 32 ? p0[c0] : p1[c0 - 32], pa1 = c1 < 32 ? p0[c1] : p1[c1 - 32];
+            const float e0 = ((km >> c0) & 1ull) ? ex2_approx(fmaf(__uint_as_float(sa0), a.scale_log2, -lse2)) : 0.0f;
+            const float e1 = ((km >> c1) & 1ull) ? ex2_approx(fmaf(__uint_as_float(sa1), a.scale_log2, -lse2)) : 0.0f;
+            const float d0 = e0 * (__uint_as_float(pa0) - dlt), d1 = e1 * (__uint_as_float(pa1) - dlt);
+            hi[c] = pack_bf16x2(d0, d1);
+            lo[c] = pack_bf16x2(d0 - __uint_as_float(hi[c] << 16), d1 - __uint_as_float(hi[c] & 0xffff0000u));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) hi[c] = lo[c] = 0u;
+        }
+        // dS over this group's own S columns: hi at +0, lo at +32
+        tmem_st32(t_lane + b * 128 + grp * 64, hi);
+        tmem_st32(t_lane + b * 128 + grp * 64 + 32, lo);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars[B_PF]);
       }
-      if (s >= 2 && !mbar_wait(&bars[B_DSFREE + b], ((s >> 1) + 1) & 1, a.st, a.timeout_ns, 62)) *grp_abort = 1;
-      store_row_bf16x2_sw128(sbase + OFF_DS + b * 32768, sbase + OFF_DS + b * 32768 + 16384, r, sv);
-      fence_proxy_async_smem();
+      // epilogue: dQ row r, columns 64grp..64grp+63, times the softmax scale
+      float o[64];
+      if (nsteps > 0) {
+        if (!mbar_wait(&bars[B_DQR], n & 1, a.st, a.timeout_ns, 63)) *sm_abort = 1;
+        tc_fence_after();
+        uint32_t o0[32], o1[32];
+        tmem_ld32(t_lane + 384 + grp * 64, o0);
+        tmem_ld32(t_lane + 384 + grp * 64 + 32, o1);
+        tmem_ld_wait();
+        const float sc = row_valid ? a.scale : 0.0f;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          o[c] = __uint_as_float(o0[c]) * sc;
+          o[c + 32] = __uint_as_float(o1[c]) * sc;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) o[c] = 0.0f;
+      }
       tc_fence_before();
-      mbar_arrive(&bars[B_DSF + b]);
-      named_bar_sync(1, 128);
-      if (*grp_abort) {
-        ok = false;
-        break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_DQFREE]);
+      if (row_exists && grp * 64 < a.D) {
+        float4* dst = reinterpret_cast<float4*>(a.dq + qrow * a.D + grp * 64);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
       }
-    }
-    if (ok && nsteps > 0) {
-      if (!mbar_wait(&bars[B_DSFREE + ((nsteps - 1) & 1)], ((nsteps - 1) >> 1) & 1, a.st, a.timeout_ns, 63))
-        ok = false;
-    }
-    tc_fence_after();
-    float o[64];
-    if (nsteps > 0 && ok) {
-      tmem_ld64(t_lane + 256, o);
-    } else {
-#pragma unroll
-      for (int c = 0; c < 64; ++c) o[c] = 0.0f;
-    }
-    if (r < a.D) {
-      float* dst = a.dq + static_cast<size_t>(row0) * a.D + r;
-#pragma unroll
-      for (int c = 0; c < 64; ++c) dst[static_cast<size_t>(c) * a.D] = ((qmask >> c) & 1ull) ? o[c] * a.scale : 0.0f;
+      // an abort seen by any thread reaches every thread at the item boundary
+      named_bar_sync(1, 256);
+      if (*sm_abort) break;
     }
   }
   tc_fence_before();
@@ -342,20 +411,30 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
 }
 
 // ------------------------------------------------------------------------ dK, dV
+// One item = two adjacent key cubes (128 keys) over the union of their transposed lists,
+// two query cubes per step:  S^T = K2 Q2^T,  dP^T = V2 dO2^T  (SS, M = 128 keys, N = 128
+// queries), P^T = exp(S^T*scale - lse_q), dS^T = P^T (dP^T - Delta_q), both written as bf16
+// hi + lo over their own TMEM columns, then  dV += P^T dO2  and  dK += dS^T Q2  (TS, N = D).
+// Thread r of group g owns key row r and the 64 queries of query cube g of the step; the
+// step's lse and Delta arrive with the Q and dO tiles (1-D bulk copies).
 namespace dkv {
-constexpr int kThreads = 192;
-constexpr uint32_t OFF_K = 0;          // [2 halves][64][128 B]
-constexpr uint32_t OFF_V = 16384;      // same
-constexpr uint32_t OFF_Q = 32768;      // 2 stages x [2 halves][128][128 B]
-constexpr uint32_t OFF_DO = 98304;     // same
-constexpr uint32_t OFF_P = 163840;     // {hi, lo} x [128 q][64 keys] bf16
-constexpr uint32_t OFF_DS = 196608;    // same
-constexpr uint32_t OFF_BAR = 229376;
-constexpr uint32_t OFF_SLOT = OFF_BAR + 192;
-constexpr uint32_t OFF_FLAG = OFF_BAR + 200;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
-constexpr uint32_t TMEM_COLS = 512;  // S[b] at 128b, dP[b] at 128b+64, dV^T at 256, dK^T at 320
-enum { B_KV = 0, B_QF = 1, B_EMPTY = 3, B_SDP = 5, B_PDS = 7, B_PDSFREE = 8, B_FIN = 9, NBAR = 10 };
+constexpr int kThreads = 320;
+constexpr int QST = 2;              // Q/dO ring depth
+constexpr uint32_t OFF_K = 0;       // K2 [2 halves][128 keys][128 B]
+constexpr uint32_t OFF_V = 32768;   // V2 same
+constexpr uint32_t OFF_Q = 65536;   // QST x Q2  [2 halves][128 q][128 B]
+constexpr uint32_t OFF_DO = OFF_Q + QST * 32768;
+constexpr uint32_t OFF_LSE = OFF_DO + QST * 32768;  // QST x [128] float
+constexpr uint32_t OFF_DLT = OFF_LSE + QST * 512;   // QST x [128] float
+constexpr uint32_t OFF_BAR = OFF_DLT + QST * 512;
+constexpr uint32_t OFF_SLOT = OFF_BAR + 256;
+constexpr uint32_t OFF_ABORT = OFF_BAR + 264;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;
+constexpr uint32_t TMEM_COLS = 512;  // S^T/P^T at 0, dP^T/dS^T at 128, dV at 256, dK at 384
+enum {
+  B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DF = 6, B_DE = 8, B_SF = 10, B_PF = 11, B_DVR = 12, B_DVFREE = 13,
+  B_FIN = 14, NBAR = 15
+};
 }  // namespace dkv
 
 __global__ void __launch_bounds__(dkv::kThreads, 1)
@@ -368,18 +447,18 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_SLOT);
-  volatile int* grp_abort = reinterpret_cast<volatile int*>(smem + OFF_FLAG);
+  volatile int* sm_abort = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
+  const float* lse_sh = reinterpret_cast<const float*>(smem + OFF_LSE);
+  const float* dlt_sh = reinterpret_cast<const float*>(smem + OFF_DLT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x % a.g.T;
-  const int bh = blockIdx.x / a.g.T;
   const Geom& g = a.g;
-  const int qbeg = a.q_off[static_cast<size_t>(bh) * (g.T + 1) + j];
-  const int nq = a.q_off[static_cast<size_t>(bh) * (g.T + 1) + j + 1] - qbeg;
+  const int npairs = (g.T + 1) >> 1;
+  const int n_items = a.BH * npairs;
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < NBAR; ++b) mbar_init(&bars[b], b == B_PDS ? 128u : 1u);
-    *grp_abort = aborted(a.st) ? 1 : 0;
+    for (int b = 0; b < NBAR; ++b) mbar_init(&bars[b], b == B_PF ? 256u : (b == B_DVFREE ? 8u : 1u));
+    *sm_abort = aborted(a.st) ? 1 : 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -390,162 +469,227 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const bool skip_all = *grp_abort != 0;
-  const int nsteps = skip_all ? 0 : (nq + 1) >> 1;
-  const int krow0 = bh * g.Npad + j * 64;
-  auto qcube = [&](int t) -> int { return t < nq ? a.q_idx[qbeg + t] : -1; };
+  const bool skip_all = *sm_abort != 0;
 
   if (warp == 0) {
-    if (lane == 0 && nsteps > 0) {
-      mbar_arrive_expect_tx(&bars[B_KV], 32768);
-      tma_load_2d(smem + OFF_K, &tm_k, &bars[B_KV], 0, krow0);
-      tma_load_2d(smem + OFF_K + 8192, &tm_k, &bars[B_KV], 64, krow0);
-      tma_load_2d(smem + OFF_V, &tm_v, &bars[B_KV], 0, krow0);
-      tma_load_2d(smem + OFF_V + 8192, &tm_v, &bars[B_KV], 64, krow0);
-      int issued = 0;
-      for (int s = 0; s < nsteps; ++s) {
-        const int st = s & 1;
-        if (s >= 2 && !mbar_wait(&bars[B_EMPTY + st], ((s >> 1) + 1) & 1, a.st, a.timeout_ns, 71)) break;
-        const int i0 = qcube(2 * s), i1 = qcube(2 * s + 1);
-        const int y0 = i0 >= 0 ? bh * g.Npad + i0 * 64 : a.rows_total;
-        const int y1 = i1 >= 0 ? bh * g.Npad + i1 * 64 : a.rows_total;
-        uint8_t* qst = smem + OFF_Q + st * 32768;
-        uint8_t* dst = smem + OFF_DO + st * 32768;
-        mbar_arrive_expect_tx(&bars[B_QF + st], 65536);
-        tma_load_2d(qst, &tm_q, &bars[B_QF + st], 0, y0);
-        tma_load_2d(qst + 8192, &tm_q, &bars[B_QF + st], 0, y1);
-        tma_load_2d(qst + 16384, &tm_q, &bars[B_QF + st], 64, y0);
-        tma_load_2d(qst + 24576, &tm_q, &bars[B_QF + st], 64, y1);
-        tma_load_2d(dst, &tm_do, &bars[B_QF + st], 0, y0);
-        tma_load_2d(dst + 8192, &tm_do, &bars[B_QF + st], 0, y1);
-        tma_load_2d(dst + 16384, &tm_do, &bars[B_QF + st], 64, y0);
-        tma_load_2d(dst + 24576, &tm_do, &bars[B_QF + st], 64, y1);
-        ++issued;
+    if (lane < 2 && !skip_all) {
+      const bool qside = lane == 0;  // lane 0: K2, V2, Q2 + lse; lane 1: dO2 + Delta
+      const CUtensorMap* tmap = qside ? &tm_q : &tm_do;
+      const float* vec = qside ? a.lse : a.delta;
+      uint32_t gs = 0;
+      int issued_kv = 0;
+      bool ok = true;
+      for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+        const int bh = it / npairs, pr = it % npairs;
+        const int nu = a.uk_cnt[it];
+        const int32_t* ul = a.uk_list + static_cast<size_t>(it) * g.T;
+        if (qside) {
+          if (n >= 1 && !mbar_wait(&bars[B_KVE], (n - 1) & 1, a.st, a.timeout_ns, 71)) break;
+          const int r0 = bh * g.Npad + (2 * pr) * 64;
+          const int r1 = (2 * pr + 1 < g.T) ? r0 + 64 : a.rows_total;
+          mbar_arrive_expect_tx(&bars[B_KVF], 65536);
+          tma_load_2d(smem + OFF_K, &tm_k, &bars[B_KVF], 0, r0);
+          tma_load_2d(smem + OFF_K + 8192, &tm_k, &bars[B_KVF], 0, r1);
+          tma_load_2d(smem + OFF_K + 16384, &tm_k, &bars[B_KVF], 64, r0);
+          tma_load_2d(smem + OFF_K + 24576, &tm_k, &bars[B_KVF], 64, r1);
+          tma_load_2d(smem + OFF_V, &tm_v, &bars[B_KVF], 0, r0);
+          tma_load_2d(smem + OFF_V + 8192, &tm_v, &bars[B_KVF], 0, r1);
+          tma_load_2d(smem + OFF_V + 16384, &tm_v, &bars[B_KVF], 64, r0);
+          tma_load_2d(smem + OFF_V + 24576, &tm_v, &bars[B_KVF], 64, r1);
+          ++issued_kv;
+        }
+        const int nsteps = (nu + 1) >> 1;
+        for (int s = 0; s < nsteps; ++s) {
+          const uint32_t st = gs % QST;
+          const uint32_t empty = (qside ? B_QE : B_DE) + st, full = (qside ? B_QF : B_DF) + st;
+          if (gs >= QST && !mbar_wait(&bars[empty], ((gs / QST) + 1) & 1, a.st, a.timeout_ns, 72)) {
+            ok = false;
+            break;
+          }
+          const int u0 = ul[2 * s] >> 2;
+          const int u1 = (2 * s + 1 < nu) ? (ul[2 * s + 1] >> 2) : -1;
+          const int y0 = bh * g.Npad + u0 * 64;
+          const int y1 = u1 >= 0 ? bh * g.Npad + u1 * 64 : a.rows_total;
+          uint8_t* dst = smem + (qside ? OFF_Q : OFF_DO) + st * 32768;
+          uint8_t* vdst = smem + (qside ? OFF_LSE : OFF_DLT) + st * 512;
+          mbar_arrive_expect_tx(&bars[full], 32768 + (u1 >= 0 ? 512 : 256));
+          tma_load_2d(dst, tmap, &bars[full], 0, y0);
+          tma_load_2d(dst + 8192, tmap, &bars[full], 0, y1);
+          tma_load_2d(dst + 16384, tmap, &bars[full], 64, y0);
+          tma_load_2d(dst + 24576, tmap, &bars[full], 64, y1);
+          bulk_load(vdst, vec + y0, 256, &bars[full]);
+          if (u1 >= 0) bulk_load(vdst + 256, vec + y1, 256, &bars[full]);
+          ++gs;
+        }
       }
-      mbar_wait(&bars[B_KV], 0, a.st, a.timeout_ns, 72);
-      for (int s = (issued > 2 ? issued - 2 : 0); s < issued; ++s)
-        mbar_wait(&bars[B_QF + (s & 1)], (s >> 1) & 1, a.st, a.timeout_ns, 73);
+      if (qside && issued_kv > 0) mbar_wait(&bars[B_KVF], (issued_kv - 1) & 1, a.st, a.timeout_ns, 73);
+      for (uint32_t s = (gs > QST ? gs - QST : 0); s < gs; ++s)
+        mbar_wait(&bars[(qside ? B_QF : B_DF) + s % QST], (s / QST) & 1, a.st, a.timeout_ns, 74);
     }
   } else if (warp == 1) {
-    if (lane == 0 && nsteps > 0) {
-      const uint32_t idesc_kk = make_idesc(128, 64, FMT_BF16, false, false);
-      const uint32_t idesc_mn = make_idesc(128, 64, FMT_BF16, true, true);
+    if (lane == 0 && !skip_all) {
+      const uint32_t idesc_kk = make_idesc(128, 128, FMT_BF16, false, false);
+      const uint32_t idesc_mn = make_idesc(128, 128, FMT_BF16, false, true);
       const int ksteps = a.D / 16;
-      auto issue_sdp = [&](int s) {
-        const int st = s & 1;
-        const uint32_t qst = sbase + OFF_Q + st * 32768, dst = sbase + OFF_DO + st * 32768;
-        const uint32_t d_s = tmem + st * 128, d_dp = tmem + st * 128 + 64;
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          const uint32_t koff = (ks >> 2) * 8192 + (ks & 3) * 32;
-          umma_f16_ss(d_s, sw128_desc(qst + off, 16, 1024), sw128_desc(sbase + OFF_K + koff, 16, 1024), idesc_kk,
-                      ks > 0 ? 1u : 0u);
-        }
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          const uint32_t koff = (ks >> 2) * 8192 + (ks & 3) * 32;
-          umma_f16_ss(d_dp, sw128_desc(dst + off, 16, 1024), sw128_desc(sbase + OFF_V + koff, 16, 1024), idesc_kk,
-                      ks > 0 ? 1u : 0u);
-        }
-        umma_commit(&bars[B_SDP + st]);
-      };
-      bool ok = mbar_wait(&bars[B_KV], 0, a.st, a.timeout_ns, 81);
-      for (int s = 0; ok && s < 2 && s < nsteps; ++s) {
-        ok = mbar_wait(&bars[B_QF + s], 0, a.st, a.timeout_ns, 82);
-        if (ok) {
-          tc_fence_after();
-          issue_sdp(s);
-        }
-      }
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int st = s & 1;
-        if (!mbar_wait(&bars[B_PDS], s & 1, a.st, a.timeout_ns, 83)) break;
-        tc_fence_after();
-        const uint32_t qst = sbase + OFF_Q + st * 32768, dst = sbase + OFF_DO + st * 32768;
-#pragma unroll 1
-        for (int ks = 0; ks < 16; ++ks) {  // P_hi then P_lo
-          const uint32_t kk = ks & 7, part = ks >> 3;
-          umma_f16_ss(tmem + 256, sw128_desc(dst + kk * 2048, 16384, 1024),
-                      sw128_desc(sbase + OFF_P + part * 16384 + kk * 2048, 8192, 1024), idesc_mn,
-                      (s > 0 || ks > 0) ? 1u : 0u);
-        }
-#pragma unroll 1
-        for (int ks = 0; ks < 16; ++ks) {  // dS_hi then dS_lo
-          const uint32_t kk = ks & 7, part = ks >> 3;
-          umma_f16_ss(tmem + 320, sw128_desc(qst + kk * 2048, 16384, 1024),
-                      sw128_desc(sbase + OFF_DS + part * 16384 + kk * 2048, 8192, 1024), idesc_mn,
-                      (s > 0 || ks > 0) ? 1u : 0u);
-        }
-        umma_commit(&bars[B_EMPTY + st]);
-        umma_commit(&bars[B_PDSFREE]);
-        if (s + 2 < nsteps) {
-          ok = mbar_wait(&bars[B_QF + st], ((s + 2) >> 1) & 1, a.st, a.timeout_ns, 84);
+      uint32_t gs = 0;
+      bool ok = true;
+      for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+        const int nsteps = (a.uk_cnt[it] + 1) >> 1;
+        if (!mbar_wait(&bars[B_KVF], n & 1, a.st, a.timeout_ns, 81)) break;
+        if (n >= 1 && nsteps > 0 && !mbar_wait(&bars[B_DVFREE], (n - 1) & 1, a.st, a.timeout_ns, 82)) break;
+        for (int s = 0; ok && s < nsteps; ++s, ++gs) {
+          const uint32_t st = gs % QST;
+          ok = mbar_wait(&bars[B_QF + st], (gs / QST) & 1, a.st, a.timeout_ns, 83) &&
+               mbar_wait(&bars[B_DF + st], (gs / QST) & 1, a.st, a.timeout_ns, 84);
           if (!ok) break;
           tc_fence_after();
-          issue_sdp(s + 2);
+          const uint32_t qst = sbase + OFF_Q + st * 32768, dst = sbase + OFF_DO + st * 32768;
+          // S^T and dP^T overwrite the previous step's P^T / dS^T, read by dV / dK issued
+          // earlier by this thread (in-order execution)
+          for (int ks = 0; ks < ksteps; ++ks) {
+            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+            umma_f16_ss(tmem + 0, sw128_desc(sbase + OFF_K + off, 16, 1024), sw128_desc(qst + off, 16, 1024),
+                        idesc_kk, ks > 0 ? 1u : 0u);
+          }
+          for (int ks = 0; ks < ksteps; ++ks) {
+            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+            umma_f16_ss(tmem + 128, sw128_desc(sbase + OFF_V + off, 16, 1024), sw128_desc(dst + off, 16, 1024),
+                        idesc_kk, ks > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars[B_SF]);
+          if (!mbar_wait(&bars[B_PF], gs & 1, a.st, a.timeout_ns, 85)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int ks = 0; ks < 16; ++ks) {  // dV += P^T dO2 (hi then lo)
+            const uint32_t kk = ks & 7, part = ks >> 3;
+            const uint32_t acol = (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
+            umma_f16_ts(tmem + 256, tmem + acol, sw128_desc(dst + kk * 2048, 16384, 1024), idesc_mn,
+                        (s > 0 || ks > 0) ? 1u : 0u);
+          }
+#pragma unroll 1
+          for (int ks = 0; ks < 16; ++ks) {  // dK += dS^T Q2 (hi then lo)
+            const uint32_t kk = ks & 7, part = ks >> 3;
+            const uint32_t acol = 128 + (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
+            umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(qst + kk * 2048, 16384, 1024), idesc_mn,
+                        (s > 0 || ks > 0) ? 1u : 0u);
+          }
+          umma_commit(&bars[B_QE + st]);
+          umma_commit(&bars[B_DE + st]);
         }
+        if (!ok) break;
+        umma_commit(&bars[B_KVE]);
+        umma_commit(&bars[B_DVR]);
       }
       umma_commit(&bars[B_FIN]);
-      mbar_wait(&bars[B_FIN], 0, a.st, a.timeout_ns, 85);
+      mbar_wait(&bars[B_FIN], 0, a.st, a.timeout_ns, 86);
     }
   } else {
+    const int grp = (warp - 2) >> 2;      // query cube grp of each step
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // query row of the pair == TMEM lane
+    const int r = quarter * 32 + lane;    // key row of the pair == TMEM lane
+    const int khalf = r >> 6;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    uint64_t kmask = 0;  // valid key columns of cube j
-    for (int c = 0; c < 64; ++c)
-      if (token_valid(g, j, c)) kmask |= 1ull << c;
-    bool ok = true;
-    for (int s = 0; s < nsteps; ++s) {
-      const int b = s & 1;
-      const int icube = qcube(2 * s + (r >> 6));
-      const bool qv = icube >= 0 && token_valid(g, icube, r & 63);
-      const size_t qrow = static_cast<size_t>(bh) * g.Npad + static_cast<size_t>(icube < 0 ? 0 : icube) * 64 + (r & 63);
-      const float lse2 = qv ? a.lse[qrow] * 1.4426950408889634f : 0.0f;
-      const float dlt = qv ? a.delta[qrow] : 0.0f;
-      if (!mbar_wait(&bars[B_SDP + b], (s >> 1) & 1, a.st, a.timeout_ns, 91)) *grp_abort = 1;
-      tc_fence_after();
-      float sv[64], dp[64];
-      tmem_ld64(t_lane + b * 128, sv);
-      tmem_ld64(t_lane + b * 128 + 64, dp);
+    uint32_t gs = 0;
+    bool ok = !skip_all;
+    for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+      const int bh = it / npairs, pr = it % npairs;
+      const int kcube = 2 * pr + khalf;
+      const bool key_exists = kcube < g.T;
+      const bool key_valid = key_exists && ((a.cube_mask[kcube] >> (r & 63)) & 1ull);
+      const int nu = a.uk_cnt[it];
+      const int32_t* ul = a.uk_list + static_cast<size_t>(it) * g.T;
+      const int nsteps = (nu + 1) >> 1;
+      for (int s = 0; s < nsteps; ++s, ++gs) {
+        const uint32_t st = gs % QST;
+        const int e = (2 * s + grp < nu) ? ul[2 * s + grp] : 0;
+        const int qcube = e >> 2;
+        const bool active = ((e >> khalf) & 1) && key_valid;
+        const bool w_active = __any_sync(0xffffffffu, active);
+        if (!mbar_wait(&bars[B_SF], gs & 1, a.st, a.timeout_ns, 91)) *sm_abort = 1;
+        tc_fence_after();
+        uint32_t ph[32], pl[32], dh[32], dl[32];
+        if (w_active) {
+          uint32_t s0[32], s1[32], p0[32], p1[32];
+          tmem_ld32(t_lane + grp * 64, s0);
+          tmem_ld32(t_lane + grp * 64 + 32, s1);
+          tmem_ld32(t_lane + 128 + grp * 64, p0);
+          tmem_ld32(t_lane + 128 + grp * 64 + 32, p1);
+          tmem_ld_wait();
+          const unsigned long long qm = active ? a.cube_mask[qcube] : 0ull;
+          const float* lq = lse_sh + st * 128 + grp * 64;
+          const float* dq_ = dlt_sh + st * 128 + grp * 64;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const bool on = qv && ((kmask >> c) & 1ull);
-        const float p = on ? exp2f(sv[c] * a.scale_log2 - lse2) : 0.0f;
-        sv[c] = p;
-        dp[c] = p * (dp[c] - dlt);
+          for (int c = 0; c < 32; ++c) {
+            const int c0 = 2 * c, c1 = 2 * c + 1;
+            const uint32_t sa0 = c0 < 32 ? s0[c0] : s1[c0 - 32], sa1 = c1 < 32 ? s0[c1] : s1[c1 - 32];
+            const uint32_t pa0 = c0 < 32 ? p0[c0] : p1[c0 - 32], pa1 = c1 < 32 ? p0[c1] : p1[c1 - 32];
+            const float2 l2 = *reinterpret_cast<const float2*>(lq + c0);
+            const float2 d2 = *reinterpret_cast<const float2*>(dq_ + c0);
+            const float e0 =
+                ((qm >> c0) & 1ull) ? ex2_approx(fmaf(__uint_as_float(sa0), a.scale_log2, -l2.x * 1.4426950408889634f))
+                                    : 0.0f;
+            const float e1 =
+                ((qm >> c1) & 1ull) ? ex2_approx(fmaf(__uint_as_float(sa1), a.scale_log2, -l2.y * 1.4426950408889634f))
+                                    : 0.0f;
+            const float g0 = e0 * (__uint_as_float(pa0) - d2.x), g1 = e1 * (__uint_as_float(pa1) - d2.y);
+            ph[c] = pack_bf16x2(e0, e1);
+            pl[c] = pack_bf16x2(e0 - __uint_as_float(ph[c] << 16), e1 - __uint_as_float(ph[c] & 0xffff0000u));
+            dh[c] = pack_bf16x2(g0, g1);
+            dl[c] = pack_bf16x2(g0 - __uint_as_float(dh[c] << 16), g1 - __uint_as_float(dh[c] & 0xffff0000u));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ph[c] = pl[c] = dh[c] = dl[c] = 0u;
+        }
+        tmem_st32(t_lane + grp * 64, ph);
+        tmem_st32(t_lane + grp * 64 + 32, pl);
+        tmem_st32(t_lane + 128 + grp * 64, dh);
+        tmem_st32(t_lane + 128 + grp * 64 + 32, dl);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars[B_PF]);
       }
-      if (s >= 1 && !mbar_wait(&bars[B_PDSFREE], (s - 1) & 1, a.st, a.timeout_ns, 92)) *grp_abort = 1;
-      store_row_bf16x2_sw128(sbase + OFF_P, sbase + OFF_P + 16384, r, sv);
-      store_row_bf16x2_sw128(sbase + OFF_DS, sbase + OFF_DS + 16384, r, dp);
-      fence_proxy_async_smem();
+      // epilogue: key row r, columns 64grp..64grp+63 of dV and dK (dK times the scale)
+      float gv[64], gk[64];
+      if (nsteps > 0) {
+        if (!mbar_wait(&bars[B_DVR], n & 1, a.st, a.timeout_ns, 92)) *sm_abort = 1;
+        tc_fence_after();
+        uint32_t v0[32], v1[32], k0[32], k1[32];
+        tmem_ld32(t_lane + 256 + grp * 64, v0);
+        tmem_ld32(t_lane + 256 + grp * 64 + 32, v1);
+        tmem_ld32(t_lane + 384 + grp * 64, k0);
+        tmem_ld32(t_lane + 384 + grp * 64 + 32, k1);
+        tmem_ld_wait();
+        const float vs = key_valid ? 1.0f : 0.0f, ks = key_valid ? a.scale : 0.0f;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          gv[c] = __uint_as_float(v0[c]) * vs;
+          gv[c + 32] = __uint_as_float(v1[c]) * vs;
+          gk[c] = __uint_as_float(k0[c]) * ks;
+          gk[c + 32] = __uint_as_float(k1[c]) * ks;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) gv[c] = gk[c] = 0.0f;
+      }
       tc_fence_before();
-      mbar_arrive(&bars[B_PDS]);
-      named_bar_sync(1, 128);
-      if (*grp_abort) {
-        ok = false;
-        break;
-      }
-    }
-    if (ok && nsteps > 0 && !mbar_wait(&bars[B_PDSFREE], (nsteps - 1) & 1, a.st, a.timeout_ns, 93)) ok = false;
-    tc_fence_after();
-    float gv[64], gk[64];
-    if (nsteps > 0 && ok) {
-      tmem_ld64(t_lane + 256, gv);
-      tmem_ld64(t_lane + 320, gk);
-    } else {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_DVFREE]);
+      if (key_exists && grp * 64 < a.D) {
+        const size_t krow = static_cast<size_t>(bh) * g.Npad + static_cast<size_t>(kcube) * 64 + (r & 63);
+        float4* pv = reinterpret_cast<float4*>(a.dv + krow * a.D + grp * 64);
+        float4* pk = reinterpret_cast<float4*>(a.dk + krow * a.D + grp * 64);
 #pragma unroll
-      for (int c = 0; c < 64; ++c) gv[c] = gk[c] = 0.0f;
-    }
-    if (r < a.D) {
-      float* pv = a.dv + static_cast<size_t>(krow0) * a.D + r;
-      float* pk = a.dk + static_cast<size_t>(krow0) * a.D + r;
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const bool kv = (kmask >> c) & 1ull;
-        pv[static_cast<size_t>(c) * a.D] = kv ? gv[c] : 0.0f;
-        pk[static_cast<size_t>(c) * a.D] = kv ? gk[c] * a.scale : 0.0f;
+        for (int c = 0; c < 16; ++c) {
+          pv[c] = make_float4(gv[4 * c], gv[4 * c + 1], gv[4 * c + 2], gv[4 * c + 3]);
+          pk[c] = make_float4(gk[4 * c], gk[4 * c + 1], gk[4 * c + 2], gk[4 * c + 3]);
+        }
       }
+      named_bar_sync(1, 256);
+      if (*sm_abort) break;
     }
   }
   tc_fence_before();
@@ -556,8 +700,8 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
 // ------------------------------------------------------------------------ launch
 cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const void* out, const float* out_f32, const void* dout,
-                            AttnArgs a, int32_t* qcnt,
-                            int32_t* qoff, int32_t* qidx, float* delta, cudaStream_t stream, int* launches) {
+                            AttnArgs a, int32_t* qcnt, int32_t* qoff, int32_t* qidx, float* delta, int32_t* uq_list,
+                            int32_t* uq_cnt, int32_t* uk_list, int32_t* uk_cnt, cudaStream_t stream, int* launches) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(attn_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::SMEM_BYTES);
@@ -579,13 +723,23 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   scan_kernel<<<a.BH, 1024, 0, stream>>>(qcnt, qoff, g.T, a.cap);
   fill_kernel<<<static_cast<unsigned>((qrows + 7) / 8), 256, 0, stream>>>(a.kv_index, a.kv_count, qoff, qidx, a.BH,
                                                                           g.T, a.cap);
+  e = launch_query_pair_union(a.kv_index, a.kv_count, uq_list, uq_cnt, a.BH, g.T, a.cap, a.st, stream);
+  if (e != cudaSuccess) return e;
+  e = launch_key_pair_union(qoff, qidx, uk_list, uk_cnt, a.BH, g.T, a.cap, stream);
+  if (e != cudaSuccess) return e;
   a.delta = delta;
   a.q_off = qoff;
   a.q_idx = qidx;
-  const unsigned grid = static_cast<unsigned>(a.BH) * g.T;
+  a.u_list = uq_list;
+  a.u_cnt = uq_cnt;
+  a.uk_list = uk_list;
+  a.uk_cnt = uk_cnt;
+  const int sms = num_sms();
+  const int items = a.BH * ((g.T + 1) >> 1);
+  const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
   attn_dq_kernel<<<grid, dqk::kThreads, dqk::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
   attn_dkdv_kernel<<<grid, dkv::kThreads, dkv::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
-  *launches = 6;
+  *launches = 8;
   return cudaGetLastError();
 }
 

@@ -15,8 +15,11 @@ struct AttnArgs {
   __nv_bfloat16* out;       // forward output [BH, Npad, D]
   float* out_f32;           // optional fp32 copy of the forward output
   const unsigned long long* cube_mask;  // [T] valid-slot mask of every cube
-  const int32_t* u_list;    // pair unions: [BH, ceil(T/2), 2*cap] (block << 2 | membership bits)
+  const int32_t* u_list;    // query-pair unions: [BH, ceil(T/2), ucap] (block << 2 | membership bits)
   const int32_t* u_cnt;     // [BH, ceil(T/2)]
+  const int32_t* uk_list;   // key-pair unions of the transposed lists: [BH, ceil(T/2), T]
+  const int32_t* uk_cnt;
+  int ucap;                 // row stride of u_list: min(2 * cap, T)
   float* lse;               // [BH, Npad]
   const float* delta;       // backward: rowsum(dO * O) [BH, Npad]
   const int32_t* q_off;     // backward: transposed lists, CSR offsets [BH, T+1]

@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   const Geom& g = a.g;
   const int npairs = (g.T + 1) >> 1;
   const int n_items = a.BH * npairs;
-  const int ucap = 2 * a.cap;
+  const int ucap = a.ucap;
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < NBAR; ++b) {

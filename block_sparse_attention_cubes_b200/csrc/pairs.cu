@@ -35,11 +35,11 @@ __device__ __forceinline__ int merge_two(const int32_t* a, int n0, const int32_t
 }
 
 // Query-cube pairs: union of kv_index rows 2p and 2p+1 of each (b, h).
-// u_list: [BH, P, 2*cap], u_cnt: [BH, P] with P = ceil(T/2).  Entries outside [0, T) or
+// u_list: [BH, P, ucap] with ucap = min(2*cap, T), u_cnt: [BH, P], P = ceil(T/2).  Entries outside [0, T) or
 // counts outside [0, cap] are dropped (and reported as index errors).
 __global__ void query_pair_union_kernel(const int32_t* __restrict__ kv_index, const int32_t* __restrict__ kv_count,
                                         int32_t* __restrict__ u_list, int32_t* __restrict__ u_cnt, int BH, int T,
-                                        int cap, DevStatus* st) {
+                                        int cap, int ucap, DevStatus* st) {
   const int P = (T + 1) >> 1;
   const long long id = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (id >= static_cast<long long>(BH) * P) return;
@@ -59,7 +59,7 @@ __global__ void query_pair_union_kernel(const int32_t* __restrict__ kv_index, co
     n[u] = c;
     src[u] = kv_index + r * cap;
   }
-  int32_t* out = u_list + id * (2LL * cap);
+  int32_t* out = u_list + id * static_cast<long long>(ucap);
   // drop out-of-range entries while merging: copy valid prefixes through local filtering
   int x = 0, y = 0, k = 0;
   while (x < n[0] || y < n[1]) {
@@ -95,7 +95,8 @@ __global__ void query_pair_union_kernel(const int32_t* __restrict__ kv_index, co
   u_cnt[id] = k;
 }
 
-// Key-cube pairs: union of the transposed lists (CSR q_off/q_idx) of cubes 2p and 2p+1.
+// Key-cube pairs: union of the transposed lists (CSR q_off/q_idx) of cubes 2p and 2p+1
+// (row stride T: a union of query cubes has at most T entries).
 __global__ void key_pair_union_kernel(const int32_t* __restrict__ q_off, const int32_t* __restrict__ q_idx,
                                       int32_t* __restrict__ u_list, int32_t* __restrict__ u_cnt, int BH, int T,
                                       int cap) {
@@ -111,14 +112,15 @@ __global__ void key_pair_union_kernel(const int32_t* __restrict__ q_off, const i
     b1 = off[j1];
     n1 = off[j1 + 1] - b1;
   }
-  u_cnt[id] = merge_two(q_idx + b0, n0, q_idx + b1, n1, u_list + id * (2LL * cap));
+  u_cnt[id] = merge_two(q_idx + b0, n0, q_idx + b1, n1, u_list + id * static_cast<long long>(T));
 }
 
 cudaError_t launch_query_pair_union(const int32_t* kv_index, const int32_t* kv_count, int32_t* u_list,
                                     int32_t* u_cnt, int BH, int T, int cap, DevStatus* st, cudaStream_t stream) {
   const long long n = static_cast<long long>(BH) * ((T + 1) >> 1);
+  const int ucap = 2 * cap < T ? 2 * cap : T;
   query_pair_union_kernel<<<static_cast<unsigned>((n + 127) / 128), 128, 0, stream>>>(kv_index, kv_count, u_list,
-                                                                                       u_cnt, BH, T, cap, st);
+                                                                                       u_cnt, BH, T, cap, ucap, st);
   return cudaGetLastError();
 }
 
