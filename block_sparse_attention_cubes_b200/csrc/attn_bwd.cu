@@ -332,10 +332,11 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       const int nu = a.u_cnt[it];
       const int32_t* ul = a.u_list + static_cast<size_t>(it) * a.ucap;
       const int nsteps = (nu + 1) >> 1;
+      int e = (grp < nu) ? ul[grp] : 0;
+      unsigned long long km_cur = a.cube_mask[e >> 2];
       for (int s = 0; s < nsteps; ++s, ++gs) {
         const uint32_t b = gs & 1;
-        const int e = (2 * s + grp < nu) ? ul[2 * s + grp] : 0;
-        const int tile = e >> 2;
+        const int e_next = (2 * s + 2 + grp < nu) ? ul[2 * s + 2 + grp] : 0;
         const bool active = ((e >> half) & 1) && row_valid;
         const bool w_active = __any_sync(0xffffffffu, active);
         const bool ok1 = mbar_wait(&bars[B_SF + b], (gs >> 1) & 1, a.st, a.timeout_ns, 61);
@@ -350,7 +351,7 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
           tmem_ld32(t_lane + 256 + grp * 64, p0);
           tmem_ld32(t_lane + 256 + grp * 64 + 32, p1);
           tmem_ld_wait();
-          const unsigned long long km = active ? a.cube_mask[tile] : 0ull;
+          const unsigned long long km = active ? km_cur : 0ull;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const int c0 = 2 * c, c1 = 2 * c + 1;
@@ -369,6 +370,8 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         // dS over this group's own S columns: hi at +0, lo at +32
         tmem_st32(t_lane + b * 128 + grp * 64, hi);
         tmem_st32(t_lane + b * 128 + grp * 64 + 32, lo);
+        e = e_next;
+        km_cur = a.cube_mask[e >> 2];
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars[B_PF]);
@@ -432,8 +435,8 @@ constexpr uint32_t OFF_ABORT = OFF_BAR + 264;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;
 constexpr uint32_t TMEM_COLS = 512;  // S^T/P^T at 0, dP^T/dS^T at 128, dV at 256, dK at 384
 enum {
-  B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DF = 6, B_DE = 8, B_SF = 10, B_PF = 11, B_DVR = 12, B_DVFREE = 13,
-  B_FIN = 14, NBAR = 15
+  B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DF = 6, B_DE = 8, B_SF = 10, B_DPF = 11, B_PF = 12, B_DSF = 13,
+  B_DVR = 14, B_DVFREE = 15, B_FIN = 16, NBAR = 17
 };
 }  // namespace dkv
 
@@ -457,7 +460,8 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
   const int n_items = a.BH * npairs;
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < NBAR; ++b) mbar_init(&bars[b], b == B_PF ? 256u : (b == B_DVFREE ? 8u : 1u));
+    for (int b = 0; b < NBAR; ++b)
+      mbar_init(&bars[b], (b == B_PF || b == B_DSF) ? 256u : (b == B_DVFREE ? 8u : 1u));
     *sm_abort = aborted(a.st) ? 1 : 0;
     fence_barrier_init();
   }
@@ -551,24 +555,30 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
             umma_f16_ss(tmem + 0, sw128_desc(sbase + OFF_K + off, 16, 1024), sw128_desc(qst + off, 16, 1024),
                         idesc_kk, ks > 0 ? 1u : 0u);
           }
+          umma_commit(&bars[B_SF]);  // the exponentials can start while dP^T is computed
           for (int ks = 0; ks < ksteps; ++ks) {
             const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
             umma_f16_ss(tmem + 128, sw128_desc(sbase + OFF_V + off, 16, 1024), sw128_desc(dst + off, 16, 1024),
                         idesc_kk, ks > 0 ? 1u : 0u);
           }
-          umma_commit(&bars[B_SF]);
+          umma_commit(&bars[B_DPF]);
           if (!mbar_wait(&bars[B_PF], gs & 1, a.st, a.timeout_ns, 85)) {
             ok = false;
             break;
           }
           tc_fence_after();
 #pragma unroll 1
-          for (int ks = 0; ks < 16; ++ks) {  // dV += P^T dO2 (hi then lo)
+          for (int ks = 0; ks < 16; ++ks) {  // dV += P^T dO2 (hi then lo), overlapping dS^T
             const uint32_t kk = ks & 7, part = ks >> 3;
             const uint32_t acol = (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
             umma_f16_ts(tmem + 256, tmem + acol, sw128_desc(dst + kk * 2048, 16384, 1024), idesc_mn,
                         (s > 0 || ks > 0) ? 1u : 0u);
           }
+          if (!mbar_wait(&bars[B_DSF], gs & 1, a.st, a.timeout_ns, 87)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll 1
           for (int ks = 0; ks < 16; ++ks) {  // dK += dS^T Q2 (hi then lo)
             const uint32_t kk = ks & 7, part = ks >> 3;
@@ -602,55 +612,99 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
       const int nu = a.uk_cnt[it];
       const int32_t* ul = a.uk_list + static_cast<size_t>(it) * g.T;
       const int nsteps = (nu + 1) >> 1;
+      int e = (grp < nu) ? ul[grp] : 0;
+      unsigned long long qm_cur = a.cube_mask[e >> 2];
       for (int s = 0; s < nsteps; ++s, ++gs) {
         const uint32_t st = gs % QST;
-        const int e = (2 * s + grp < nu) ? ul[2 * s + grp] : 0;
-        const int qcube = e >> 2;
+        const int e_next = (2 * s + 2 + grp < nu) ? ul[2 * s + 2 + grp] : 0;
         const bool active = ((e >> khalf) & 1) && key_valid;
         const bool w_active = __any_sync(0xffffffffu, active);
+        const unsigned long long qm = active ? qm_cur : 0ull;
         if (!mbar_wait(&bars[B_SF], gs & 1, a.st, a.timeout_ns, 91)) *sm_abort = 1;
         tc_fence_after();
-        uint32_t ph[32], pl[32], dh[32], dl[32];
-        if (w_active) {
-          uint32_t s0[32], s1[32], p0[32], p1[32];
-          tmem_ld32(t_lane + grp * 64, s0);
-          tmem_ld32(t_lane + grp * 64 + 32, s1);
-          tmem_ld32(t_lane + 128 + grp * 64, p0);
-          tmem_ld32(t_lane + 128 + grp * 64 + 32, p1);
-          tmem_ld_wait();
-          const unsigned long long qm = active ? a.cube_mask[qcube] : 0ull;
-          const float* lq = lse_sh + st * 128 + grp * 64;
-          const float* dq_ = dlt_sh + st * 128 + grp * 64;
+        // P^T = exp(S^T * scale - lse_q): written as soon as it is known so that dV can start
+        float pe[64];
+        {
+          uint32_t ph[32], pl[32];
+          if (w_active) {
+            uint32_t s0[32], s1[32];
+            tmem_ld32(t_lane + grp * 64, s0);
+            tmem_ld32(t_lane + grp * 64 + 32, s1);
+            tmem_ld_wait();
+            const float* lq = lse_sh + st * 128 + grp * 64;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int c0 = 2 * c, c1 = 2 * c + 1;
-            const uint32_t sa0 = c0 < 32 ? s0[c0] : s1[c0 - 32], sa1 = c1 < 32 ? s0[c1] : s1[c1 - 32];
-            const uint32_t pa0 = c0 < 32 ? p0[c0] : p1[c0 - 32], pa1 = c1 < 32 ? p0[c1] : p1[c1 - 32];
-            const float2 l2 = *reinterpret_cast<const float2*>(lq + c0);
-            const float2 d2 = *reinterpret_cast<const float2*>(dq_ + c0);
-            const float e0 =
-                ((qm >> c0) & 1ull) ? ex2_approx(fmaf(__uint_as_float(sa0), a.scale_log2, -l2.x * 1.4426950408889634f))
-                                    : 0.0f;
-            const float e1 =
-                ((qm >> c1) & 1ull) ? ex2_approx(fmaf(__uint_as_float(sa1), a.scale_log2, -l2.y * 1.4426950408889634f))
-                                    : 0.0f;
-            const float g0 = e0 * (__uint_as_float(pa0) - d2.x), g1 = e1 * (__uint_as_float(pa1) - d2.y);
-            ph[c] = pack_bf16x2(e0, e1);
-            pl[c] = pack_bf16x2(e0 - __uint_as_float(ph[c] << 16), e1 - __uint_as_float(ph[c] & 0xffff0000u));
-            dh[c] = pack_bf16x2(g0, g1);
-            dl[c] = pack_bf16x2(g0 - __uint_as_float(dh[c] << 16), g1 - __uint_as_float(dh[c] & 0xffff0000u));
+            for (int c4 = 0; c4 < 16; ++c4) {
+              const float4 l4 = *reinterpret_cast<const float4*>(lq + 4 * c4);
+              const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int c = 4 * c4 + u;
+                const uint32_t sv = c < 32 ? s0[c] : s1[c - 32];
+                pe[c] = ((qm >> c) & 1ull)
+                            ? ex2_approx(fmaf(__uint_as_float(sv), a.scale_log2, -lv[u] * 1.4426950408889634f))
+                            : 0.0f;
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              ph[c] = pack_bf16x2(pe[2 * c], pe[2 * c + 1]);
+              pl[c] = pack_bf16x2(pe[2 * c] - __uint_as_float(ph[c] << 16),
+                                  pe[2 * c + 1] - __uint_as_float(ph[c] & 0xffff0000u));
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) pe[c] = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ph[c] = pl[c] = 0u;
           }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) ph[c] = pl[c] = dh[c] = dl[c] = 0u;
+          // P^T over S^T: every S^T read of this thread's own columns is done
+          tmem_st32(t_lane + grp * 64, ph);
+          tmem_st32(t_lane + grp * 64 + 32, pl);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&bars[B_PF]);
         }
-        tmem_st32(t_lane + grp * 64, ph);
-        tmem_st32(t_lane + grp * 64 + 32, pl);
-        tmem_st32(t_lane + 128 + grp * 64, dh);
-        tmem_st32(t_lane + 128 + grp * 64 + 32, dl);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bars[B_PF]);
+        // dS^T = P^T (dP^T - Delta_q)
+        if (!mbar_wait(&bars[B_DPF], gs & 1, a.st, a.timeout_ns, 93)) *sm_abort = 1;
+        tc_fence_after();
+        {
+          uint32_t dh[32], dl[32];
+          if (w_active) {
+            uint32_t p0[32], p1[32];
+            tmem_ld32(t_lane + 128 + grp * 64, p0);
+            tmem_ld32(t_lane + 128 + grp * 64 + 32, p1);
+            tmem_ld_wait();
+            const float* dq_ = dlt_sh + st * 128 + grp * 64;
+            float dsv[64];
+#pragma unroll
+            for (int c4 = 0; c4 < 16; ++c4) {
+              const float4 d4 = *reinterpret_cast<const float4*>(dq_ + 4 * c4);
+              const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int c = 4 * c4 + u;
+                const uint32_t pv = c < 32 ? p0[c] : p1[c - 32];
+                dsv[c] = pe[c] * (__uint_as_float(pv) - dv4[u]);
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              dh[c] = pack_bf16x2(dsv[2 * c], dsv[2 * c + 1]);
+              dl[c] = pack_bf16x2(dsv[2 * c] - __uint_as_float(dh[c] << 16),
+                                  dsv[2 * c + 1] - __uint_as_float(dh[c] & 0xffff0000u));
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) dh[c] = dl[c] = 0u;
+          }
+          tmem_st32(t_lane + 128 + grp * 64, dh);
+          tmem_st32(t_lane + 128 + grp * 64 + 32, dl);
+          e = e_next;
+          qm_cur = a.cube_mask[e >> 2];
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&bars[B_DSF]);
+        }
       }
       // epilogue: key row r, columns 64grp..64grp+63 of dV and dK (dK times the scale)
       float gv[64], gk[64];

@@ -228,9 +228,12 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       float qs = 1.0f;
       if (a.q_scale && row_exists) qs = a.q_scale[static_cast<size_t>(bh) * g.T + icube];
       float m_run = kNegBig, l_part = 0.0f;
+      // this step's and the next step's list entries and key masks are loaded one step ahead
+      int e = (grp < nu) ? ul[grp] : 0;
+      unsigned long long km = a.cube_mask[e >> 2];
       for (int s = 0; s < nsteps; ++s, ++gs) {
         const uint32_t b = gs & 1;
-        const int e = (2 * s + grp < nu) ? ul[2 * s + grp] : 0;
+        const int e_next = (2 * s + 2 + grp < nu) ? ul[2 * s + 2 + grp] : 0;
         const int tile = e >> 2;
         const bool active = ((e >> half) & 1) && row_exists;  // uniform over each warp
         float sc = a.scale_log2 * qs;
@@ -244,7 +247,6 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           tmem_ld32(t_lane + b * 128 + grp * 64, r0);
           tmem_ld32(t_lane + b * 128 + grp * 64 + 32, r1);
           tmem_ld_wait();
-          const unsigned long long km = a.cube_mask[tile];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             x[c] = __uint_as_float(r0[c]);
@@ -315,6 +317,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         }
         tmem_st32(t_lane + b * 128 + grp * 32, ph);
         if (split_pv) tmem_st32(t_lane + b * 128 + 64 + grp * 32, pl);
+        e = e_next;
+        km = a.cube_mask[e >> 2];
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars[B_PF]);
