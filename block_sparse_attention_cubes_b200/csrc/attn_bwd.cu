@@ -154,6 +154,7 @@ enum {
 };
 }  // namespace dqk
 
+template <int KS>  // D / 16; MMA loops unrolled (a counted loop costs more than the MMA)
 __global__ void __launch_bounds__(dqk::kThreads, 1)
     attn_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -235,56 +236,66 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
           ++gs;
         }
       }
-      if (kq && issued_q > 0) mbar_wait(&bars[B_QF], (issued_q - 1) & 1, a.st, a.timeout_ns, 43);
+      if (kq && issued_q > 0) mbar_wait_drain(&bars[B_QF], (issued_q - 1) & 1, a.st, a.timeout_ns, 43);
       const uint32_t nst = kq ? KST : VST;
       for (uint32_t s = (gs > nst ? gs - nst : 0); s < gs; ++s)
-        mbar_wait(&bars[(kq ? B_KF : B_VF) + s % nst], (s / nst) & 1, a.st, a.timeout_ns, 44);
+        mbar_wait_drain(&bars[(kq ? B_KF : B_VF) + s % nst], (s / nst) & 1, a.st, a.timeout_ns, 44);
     }
   } else if (warp == 1) {
-    if (lane == 0 && !skip_all) {
+    // the whole warp runs the loop; one elected lane issues (see elect_one)
+    if (!skip_all) {
       const uint32_t idesc_kk = make_idesc(128, 128, FMT_BF16, false, false);
       const uint32_t idesc_q = make_idesc(128, 128, FMT_BF16, false, true);
-      const int ksteps = a.D / 16;
       uint32_t gs_s = 0, gs_p = 0, gs_q = 0;  // global steps whose S, dP, dQ products were issued
       bool ok = true;
       auto issue_s = [&]() -> bool {
         const uint32_t ks_i = gs_s % KST, sb = gs_s & 1;
-        if (!mbar_wait(&bars[B_KF + ks_i], (gs_s / KST) & 1, a.st, a.timeout_ns, 51)) return false;
+        if (!mbar_wait_warp(&bars[B_KF + ks_i], (gs_s / KST) & 1, a.st, a.timeout_ns, 51)) return false;
         tc_fence_after();
         const uint32_t kst = sbase + OFF_K + ks_i * 32768;
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          umma_f16_ss(tmem + sb * 128, sw128_desc(sbase + OFF_Q + off, 16, 1024), sw128_desc(kst + off, 16, 1024),
-                      idesc_kk, ks > 0 ? 1u : 0u);
+        if (elect_one()) {
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+            umma_f16_ss(tmem + sb * 128, sw128_desc(sbase + OFF_Q + off, 16, 1024), sw128_desc(kst + off, 16, 1024),
+                        idesc_kk, ks > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars[B_SF + sb]);
         }
-        umma_commit(&bars[B_SF + sb]);
+        __syncwarp();
         ++gs_s;
         return true;
       };
       auto issue_dp = [&]() -> bool {
         const uint32_t vs = gs_p % VST;
-        if (!mbar_wait(&bars[B_VF + vs], (gs_p / VST) & 1, a.st, a.timeout_ns, 52)) return false;
+        if (!mbar_wait_warp(&bars[B_VF + vs], (gs_p / VST) & 1, a.st, a.timeout_ns, 52)) return false;
         tc_fence_after();
         const uint32_t vst = sbase + OFF_V + vs * 32768;
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          umma_f16_ss(tmem + 256, sw128_desc(sbase + OFF_DO + off, 16, 1024), sw128_desc(vst + off, 16, 1024),
-                      idesc_kk, ks > 0 ? 1u : 0u);
+        if (elect_one()) {
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+            umma_f16_ss(tmem + 256, sw128_desc(sbase + OFF_DO + off, 16, 1024), sw128_desc(vst + off, 16, 1024),
+                        idesc_kk, ks > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars[B_DPF]);
+          umma_commit(&bars[B_VE + vs]);
         }
-        umma_commit(&bars[B_DPF]);
-        umma_commit(&bars[B_VE + vs]);
+        __syncwarp();
         ++gs_p;
         return true;
       };
       for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
         const int nsteps = (a.u_cnt[it] + 1) >> 1;
-        if (!mbar_wait(&bars[B_QF], n & 1, a.st, a.timeout_ns, 53)) break;
+        if (!mbar_wait_warp(&bars[B_QF], n & 1, a.st, a.timeout_ns, 53)) break;
         if (nsteps > 0) ok = issue_s() && issue_dp();
-        if (ok && n >= 1 && nsteps > 0) ok = mbar_wait(&bars[B_DQFREE], (n - 1) & 1, a.st, a.timeout_ns, 54);
+        // dQ of the previous item must have been read out before this item's dQ (or, for an
+        // empty item, its ready signal): one phase of DQR / DQFREE per item, never two unobserved
+        if (ok && n >= 1) ok = mbar_wait_warp(&bars[B_DQFREE], (n - 1) & 1, a.st, a.timeout_ns, 54);
         for (int s = 0; ok && s < nsteps; ++s) {
           // S(s+1) goes to the other S buffer, whose dS(s-1) was read by the earlier dQ(s-1)
           if (s + 1 < nsteps) ok = issue_s();
-          if (!ok || !mbar_wait(&bars[B_PF], gs_q & 1, a.st, a.timeout_ns, 55)) {
+          if (!ok || !mbar_wait_warp(&bars[B_PF], gs_q & 1, a.st, a.timeout_ns, 55)) {
             ok = false;
             break;
           }
@@ -296,22 +307,29 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
           tc_fence_after();
           const uint32_t ks_i = gs_q % KST, sb = gs_q & 1;
           const uint32_t kst = sbase + OFF_K + ks_i * 32768;
-#pragma unroll 1
-          for (int ks = 0; ks < 16; ++ks) {  // 8 k-steps over dS_hi, then 8 over dS_lo
-            const uint32_t kk = ks & 7, part = ks >> 3;
-            const uint32_t acol = sb * 128 + (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
-            umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(kst + kk * 2048, 16384, 1024), idesc_q,
-                        (s > 0 || ks > 0) ? 1u : 0u);
+          if (elect_one()) {
+#pragma unroll
+            for (int ks = 0; ks < 16; ++ks) {  // 8 k-steps over dS_hi, then 8 over dS_lo
+              const uint32_t kk = ks & 7, part = ks >> 3;
+              const uint32_t acol = sb * 128 + (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
+              umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(kst + kk * 2048, 16384, 1024), idesc_q,
+                          (s > 0 || ks > 0) ? 1u : 0u);
+            }
+            umma_commit(&bars[B_KE + ks_i]);  // K(s) was read by S(s) and dQ(s)
           }
-          umma_commit(&bars[B_KE + ks_i]);  // K(s) was read by S(s) and dQ(s)
+          __syncwarp();
           ++gs_q;
         }
         if (!ok) break;
-        umma_commit(&bars[B_QE]);
-        umma_commit(&bars[B_DQR]);
+        if (elect_one()) {
+          umma_commit(&bars[B_QE]);
+          umma_commit(&bars[B_DQR]);
+        }
+        __syncwarp();
       }
-      umma_commit(&bars[B_FIN]);
-      mbar_wait(&bars[B_FIN], 0, a.st, a.timeout_ns, 56);
+      if (elect_one()) umma_commit(&bars[B_FIN]);
+      __syncwarp();
+      mbar_wait_drain(&bars[B_FIN], 0, a.st, a.timeout_ns, 56);
     }
   } else {
     const int grp = (warp - 2) >> 2;
@@ -378,8 +396,8 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       }
       // epilogue: dQ row r, columns 64grp..64grp+63, times the softmax scale
       float o[64];
+      if (!mbar_wait(&bars[B_DQR], n & 1, a.st, a.timeout_ns, 63)) *sm_abort = 1;  // every item
       if (nsteps > 0) {
-        if (!mbar_wait(&bars[B_DQR], n & 1, a.st, a.timeout_ns, 63)) *sm_abort = 1;
         tc_fence_after();
         uint32_t o0[32], o1[32];
         tmem_ld32(t_lane + 384 + grp * 64, o0);
@@ -440,6 +458,7 @@ enum {
 };
 }  // namespace dkv
 
+template <int KS>  // D / 16; MMA loops unrolled (a counted loop costs more than the MMA)
 __global__ void __launch_bounds__(dkv::kThreads, 1)
     attn_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -526,75 +545,91 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
           ++gs;
         }
       }
-      if (qside && issued_kv > 0) mbar_wait(&bars[B_KVF], (issued_kv - 1) & 1, a.st, a.timeout_ns, 73);
+      if (qside && issued_kv > 0) mbar_wait_drain(&bars[B_KVF], (issued_kv - 1) & 1, a.st, a.timeout_ns, 73);
       for (uint32_t s = (gs > QST ? gs - QST : 0); s < gs; ++s)
-        mbar_wait(&bars[(qside ? B_QF : B_DF) + s % QST], (s / QST) & 1, a.st, a.timeout_ns, 74);
+        mbar_wait_drain(&bars[(qside ? B_QF : B_DF) + s % QST], (s / QST) & 1, a.st, a.timeout_ns, 74);
     }
   } else if (warp == 1) {
-    if (lane == 0 && !skip_all) {
+    // the whole warp runs the loop; one elected lane issues (see elect_one)
+    if (!skip_all) {
       const uint32_t idesc_kk = make_idesc(128, 128, FMT_BF16, false, false);
       const uint32_t idesc_mn = make_idesc(128, 128, FMT_BF16, false, true);
-      const int ksteps = a.D / 16;
       uint32_t gs = 0;
       bool ok = true;
       for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
         const int nsteps = (a.uk_cnt[it] + 1) >> 1;
-        if (!mbar_wait(&bars[B_KVF], n & 1, a.st, a.timeout_ns, 81)) break;
-        if (n >= 1 && nsteps > 0 && !mbar_wait(&bars[B_DVFREE], (n - 1) & 1, a.st, a.timeout_ns, 82)) break;
+        if (!mbar_wait_warp(&bars[B_KVF], n & 1, a.st, a.timeout_ns, 81)) break;
+        // one phase of DVR / DVFREE per item, empty items included (see the dQ kernel)
+        if (n >= 1 && !mbar_wait_warp(&bars[B_DVFREE], (n - 1) & 1, a.st, a.timeout_ns, 82)) break;
         for (int s = 0; ok && s < nsteps; ++s, ++gs) {
           const uint32_t st = gs % QST;
-          ok = mbar_wait(&bars[B_QF + st], (gs / QST) & 1, a.st, a.timeout_ns, 83) &&
-               mbar_wait(&bars[B_DF + st], (gs / QST) & 1, a.st, a.timeout_ns, 84);
+          ok = mbar_wait_warp(&bars[B_QF + st], (gs / QST) & 1, a.st, a.timeout_ns, 83) &&
+               mbar_wait_warp(&bars[B_DF + st], (gs / QST) & 1, a.st, a.timeout_ns, 84);
           if (!ok) break;
           tc_fence_after();
           const uint32_t qst = sbase + OFF_Q + st * 32768, dst = sbase + OFF_DO + st * 32768;
           // S^T and dP^T overwrite the previous step's P^T / dS^T, read by dV / dK issued
-          // earlier by this thread (in-order execution)
-          for (int ks = 0; ks < ksteps; ++ks) {
-            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-            umma_f16_ss(tmem + 0, sw128_desc(sbase + OFF_K + off, 16, 1024), sw128_desc(qst + off, 16, 1024),
-                        idesc_kk, ks > 0 ? 1u : 0u);
+          // earlier by the same lane (in-order execution)
+          if (elect_one()) {
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+              const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+              umma_f16_ss(tmem + 0, sw128_desc(sbase + OFF_K + off, 16, 1024), sw128_desc(qst + off, 16, 1024),
+                          idesc_kk, ks > 0 ? 1u : 0u);
+            }
+            umma_commit(&bars[B_SF]);  // the exponentials can start while dP^T is computed
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+              const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+              umma_f16_ss(tmem + 128, sw128_desc(sbase + OFF_V + off, 16, 1024), sw128_desc(dst + off, 16, 1024),
+                          idesc_kk, ks > 0 ? 1u : 0u);
+            }
+            umma_commit(&bars[B_DPF]);
           }
-          umma_commit(&bars[B_SF]);  // the exponentials can start while dP^T is computed
-          for (int ks = 0; ks < ksteps; ++ks) {
-            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-            umma_f16_ss(tmem + 128, sw128_desc(sbase + OFF_V + off, 16, 1024), sw128_desc(dst + off, 16, 1024),
-                        idesc_kk, ks > 0 ? 1u : 0u);
-          }
-          umma_commit(&bars[B_DPF]);
-          if (!mbar_wait(&bars[B_PF], gs & 1, a.st, a.timeout_ns, 85)) {
+          __syncwarp();
+          if (!mbar_wait_warp(&bars[B_PF], gs & 1, a.st, a.timeout_ns, 85)) {
             ok = false;
             break;
           }
           tc_fence_after();
-#pragma unroll 1
-          for (int ks = 0; ks < 16; ++ks) {  // dV += P^T dO2 (hi then lo), overlapping dS^T
-            const uint32_t kk = ks & 7, part = ks >> 3;
-            const uint32_t acol = (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
-            umma_f16_ts(tmem + 256, tmem + acol, sw128_desc(dst + kk * 2048, 16384, 1024), idesc_mn,
-                        (s > 0 || ks > 0) ? 1u : 0u);
+          if (elect_one()) {
+#pragma unroll
+            for (int ks = 0; ks < 16; ++ks) {  // dV += P^T dO2 (hi then lo), overlapping dS^T
+              const uint32_t kk = ks & 7, part = ks >> 3;
+              const uint32_t acol = (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
+              umma_f16_ts(tmem + 256, tmem + acol, sw128_desc(dst + kk * 2048, 16384, 1024), idesc_mn,
+                          (s > 0 || ks > 0) ? 1u : 0u);
+            }
           }
-          if (!mbar_wait(&bars[B_DSF], gs & 1, a.st, a.timeout_ns, 87)) {
+          __syncwarp();
+          if (!mbar_wait_warp(&bars[B_DSF], gs & 1, a.st, a.timeout_ns, 87)) {
             ok = false;
             break;
           }
           tc_fence_after();
-#pragma unroll 1
-          for (int ks = 0; ks < 16; ++ks) {  // dK += dS^T Q2 (hi then lo)
-            const uint32_t kk = ks & 7, part = ks >> 3;
-            const uint32_t acol = 128 + (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
-            umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(qst + kk * 2048, 16384, 1024), idesc_mn,
-                        (s > 0 || ks > 0) ? 1u : 0u);
+          if (elect_one()) {
+#pragma unroll
+            for (int ks = 0; ks < 16; ++ks) {  // dK += dS^T Q2 (hi then lo)
+              const uint32_t kk = ks & 7, part = ks >> 3;
+              const uint32_t acol = 128 + (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
+              umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(qst + kk * 2048, 16384, 1024), idesc_mn,
+                          (s > 0 || ks > 0) ? 1u : 0u);
+            }
+            umma_commit(&bars[B_QE + st]);
+            umma_commit(&bars[B_DE + st]);
           }
-          umma_commit(&bars[B_QE + st]);
-          umma_commit(&bars[B_DE + st]);
+          __syncwarp();
         }
         if (!ok) break;
-        umma_commit(&bars[B_KVE]);
-        umma_commit(&bars[B_DVR]);
+        if (elect_one()) {
+          umma_commit(&bars[B_KVE]);
+          umma_commit(&bars[B_DVR]);
+        }
+        __syncwarp();
       }
-      umma_commit(&bars[B_FIN]);
-      mbar_wait(&bars[B_FIN], 0, a.st, a.timeout_ns, 86);
+      if (elect_one()) umma_commit(&bars[B_FIN]);
+      __syncwarp();
+      mbar_wait_drain(&bars[B_FIN], 0, a.st, a.timeout_ns, 86);
     }
   } else {
     const int grp = (warp - 2) >> 2;      // query cube grp of each step
@@ -708,8 +743,8 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
       }
       // epilogue: key row r, columns 64grp..64grp+63 of dV and dK (dK times the scale)
       float gv[64], gk[64];
+      if (!mbar_wait(&bars[B_DVR], n & 1, a.st, a.timeout_ns, 92)) *sm_abort = 1;  // every item
       if (nsteps > 0) {
-        if (!mbar_wait(&bars[B_DVR], n & 1, a.st, a.timeout_ns, 92)) *sm_abort = 1;
         tc_fence_after();
         uint32_t v0[32], v1[32], k0[32], k1[32];
         tmem_ld32(t_lane + 256 + grp * 64, v0);
@@ -758,9 +793,11 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             int32_t* uq_cnt, int32_t* uk_list, int32_t* uk_cnt, cudaStream_t stream, int* launches) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM_BYTES);
+    cudaError_t e = cudaSuccess;
+    for (auto fn : {attn_dq_kernel<4>, attn_dq_kernel<8>})
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::SMEM_BYTES);
+    for (auto fn : {attn_dkdv_kernel<4>, attn_dkdv_kernel<8>})
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -791,8 +828,13 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   const int sms = num_sms();
   const int items = a.BH * ((g.T + 1) >> 1);
   const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
-  attn_dq_kernel<<<grid, dqk::kThreads, dqk::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
-  attn_dkdv_kernel<<<grid, dkv::kThreads, dkv::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+  if (a.D == 64) {
+    attn_dq_kernel<4><<<grid, dqk::kThreads, dqk::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+    attn_dkdv_kernel<4><<<grid, dkv::kThreads, dkv::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+  } else {
+    attn_dq_kernel<8><<<grid, dqk::kThreads, dqk::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+    attn_dkdv_kernel<8><<<grid, dkv::kThreads, dkv::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+  }
   *launches = 8;
   return cudaGetLastError();
 }

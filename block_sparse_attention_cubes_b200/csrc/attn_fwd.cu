@@ -16,11 +16,12 @@
 // Warp roles (320 threads):
 //   warp 0      TMA producers: lane 0 loads Q2 and K tile pairs (3-stage ring, released when
 //               S is done), lane 1 loads V tile pairs (2-stage ring, released after PV)
-//   warp 1      TMEM owner and the single MMA-issuing thread
+//   warp 1      TMEM owner and MMA warp: the whole warp runs the issue loop and one elected
+//               lane issues every tcgen05.mma / commit
 //   warps 2-9   two groups of 128 threads; thread r of group g owns query row r and the 64
 //               key columns of tile t_g.  The two halves' row maxima are exchanged once per
 //               step through shared memory; the running maximum is raised (and that row of O
-//               rescaled in TMEM) only when a score exceeds it by more than 2^8.
+//               rescaled in TMEM) only when a score exceeds it by more than 2^16.
 #include <cmath>
 
 #include "attn_common.cuh"
@@ -30,7 +31,7 @@ namespace sa {
 
 namespace fwd {
 constexpr int kThreads = 320;
-constexpr float kTau = 8.0f;       // log2 headroom before a running maximum is raised
+constexpr float kTau = 16.0f;      // log2 headroom before a running maximum is raised
 constexpr float kNegBig = -1e30f;  // finite "minus infinity" for running maxima
 constexpr int KST = 3, VST = 2;    // K and V ring depths
 constexpr uint32_t OFF_Q = 0;                    // Q2: [2 halves][128 rows][128 B]
@@ -43,12 +44,19 @@ constexpr uint32_t OFF_XMAX = OFF_BAR + 512;     // [2 step parities][2 groups][
 constexpr uint32_t OFF_XL = OFF_XMAX + 2048;     // [2 groups][128 rows] float
 constexpr uint32_t SMEM_BYTES = OFF_XL + 1024 + 1024;
 constexpr uint32_t TMEM_COLS = 512;  // S/P[b] at 128b (b = 0,1), O[ob] at 256 + 128ob
+// P-full is one barrier per S buffer: the softmax of step s+1 can start before the MMA thread
+// has observed P(s) (S(s+1) is issued ahead of PV(s)), so a single barrier could complete two
+// phases unobserved.  The softmax of step s+2 needs S(s+2), issued only after PV(s).
 enum {
-  B_QF = 0, B_QE = 1, B_KF = 2, B_KE = 5, B_VF = 8, B_VE = 10, B_SF = 12, B_PF = 14, B_PFREE = 15, B_OR = 16,
-  B_OFREE = 18, B_FIN = 20, NBAR = 21
+  B_QF = 0, B_QE = 1, B_KF = 2, B_KE = 5, B_VF = 8, B_VE = 10, B_SF = 12, B_PF = 14, B_PFREE = 16, B_OR = 17,
+  B_OFREE = 19, B_FIN = 21, NBAR = 22
 };
 }  // namespace fwd
 
+// KS = D / 16 k-steps per S product.  Every MMA loop below has a compile-time trip count and
+// is unrolled: a single issuing thread running a counted loop spends far more than the
+// tensor core's 64 cycles per 128x128x16 product on the loop itself.
+template <int KS>
 __global__ void __launch_bounds__(fwd::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
@@ -71,7 +79,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int b = 0; b < NBAR; ++b) {
       uint32_t cnt = 1;
-      if (b == B_PF) cnt = 256;
+      if (b == B_PF || b == B_PF + 1) cnt = 256;
       if (b == B_OFREE || b == B_OFREE + 1) cnt = 8;
       mbar_init(&bars[b], cnt);
     }
@@ -143,18 +151,16 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         }
       }
       // drain: never leave the CTA with copies in flight
-      if (kq && issued_q > 0) mbar_wait(&bars[B_QF], (issued_q - 1) & 1, a.st, a.timeout_ns, 13);
+      if (kq && issued_q > 0) mbar_wait_drain(&bars[B_QF], (issued_q - 1) & 1, a.st, a.timeout_ns, 13);
       const uint32_t nst = kq ? KST : VST;
       for (uint32_t s = (gs > nst ? gs - nst : 0); s < gs; ++s)
-        mbar_wait(&bars[(kq ? B_KF : B_VF) + s % nst], (s / nst) & 1, a.st, a.timeout_ns, 14);
+        mbar_wait_drain(&bars[(kq ? B_KF : B_VF) + s % nst], (s / nst) & 1, a.st, a.timeout_ns, 14);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && !skip_all) {
+    if (!skip_all) {
       const uint32_t idesc_s = make_idesc(128, 128, FMT_BF16, false, false);
       const uint32_t idesc_o = make_idesc(128, 128, FMT_BF16, false, true);
-      const int ksteps = a.D / 16;
-      const int nk_pv = split_pv ? 16 : 8;
       uint32_t gs_s = 0, gs_o = 0;
       bool ok = true;
       // S for the next global step into S buffer gs_s & 1.  That buffer last held P of step
@@ -162,50 +168,64 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       // operations of one thread execute in issue order.
       auto issue_s = [&]() -> bool {
         const uint32_t kst_i = gs_s % KST, sb = gs_s & 1;
-        if (!mbar_wait(&bars[B_KF + kst_i], (gs_s / KST) & 1, a.st, a.timeout_ns, 21)) return false;
+        if (!mbar_wait_warp(&bars[B_KF + kst_i], (gs_s / KST) & 1, a.st, a.timeout_ns, 21)) return false;
         tc_fence_after();
         const uint32_t kst = sbase + OFF_K + kst_i * 32768;
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          umma_f16_ss(tmem + sb * 128, sw128_desc(sbase + OFF_Q + off, 16, 1024), sw128_desc(kst + off, 16, 1024),
-                      idesc_s, ks > 0 ? 1u : 0u);
+        if (elect_one()) {
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+            umma_f16_ss(tmem + sb * 128, sw128_desc(sbase + OFF_Q + off, 16, 1024), sw128_desc(kst + off, 16, 1024),
+                        idesc_s, ks > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars[B_SF + sb]);
+          umma_commit(&bars[B_KE + kst_i]);
         }
-        umma_commit(&bars[B_SF + sb]);
-        umma_commit(&bars[B_KE + kst_i]);
+        __syncwarp();
         ++gs_s;
         return true;
       };
       for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
         const int nsteps = (a.u_cnt[it] + 1) >> 1;
         const int ob = n & 1;
-        if (!mbar_wait(&bars[B_QF], n & 1, a.st, a.timeout_ns, 22)) break;
+        if (!mbar_wait_warp(&bars[B_QF], n & 1, a.st, a.timeout_ns, 22)) break;
         for (int s = 0; ok && s < nsteps && s < 2; ++s) ok = issue_s();
-        if (ok && n >= 2 && nsteps > 0)
-          ok = mbar_wait(&bars[B_OFREE + ob], ((n >> 1) + 1) & 1, a.st, a.timeout_ns, 23);
+        if (ok && n >= 2) ok = mbar_wait_warp(&bars[B_OFREE + ob], ((n >> 1) + 1) & 1, a.st, a.timeout_ns, 23);
         for (int s = 0; ok && s < nsteps; ++s) {
           const uint32_t vs = gs_o % VST, pb = gs_o & 1;
-          ok = mbar_wait(&bars[B_PF], gs_o & 1, a.st, a.timeout_ns, 24) &&
-               mbar_wait(&bars[B_VF + vs], (gs_o / VST) & 1, a.st, a.timeout_ns, 25);
+          ok = mbar_wait_warp(&bars[B_PF + pb], (gs_o >> 1) & 1, a.st, a.timeout_ns, 24) &&
+               mbar_wait_warp(&bars[B_VF + vs], (gs_o / VST) & 1, a.st, a.timeout_ns, 25);
           if (!ok) break;
           tc_fence_after();
           const uint32_t vst = sbase + OFF_V + vs * 32768;
-#pragma unroll 1
-          for (int ks = 0; ks < nk_pv; ++ks) {  // 8 k-steps over P (or P_hi), then 8 over P_lo
-            const uint32_t kk = ks & 7, part = ks >> 3;
-            umma_f16_ts(tmem + 256 + ob * 128, tmem + pb * 128 + part * 64 + kk * 8,
-                        sw128_desc(vst + kk * 2048, 16384, 1024), idesc_o, (s > 0 || ks > 0) ? 1u : 0u);
+          const uint32_t o_acc = tmem + 256 + ob * 128, p_col = tmem + pb * 128;
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // 8 k-steps over P (or P_hi) ...
+              umma_f16_ts(o_acc, p_col + kk * 8, sw128_desc(vst + kk * 2048, 16384, 1024), idesc_o,
+                          (s > 0 || kk > 0) ? 1u : 0u);
+            if (split_pv) {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)  // ... then 8 over P_lo
+                umma_f16_ts(o_acc, p_col + 64 + kk * 8, sw128_desc(vst + kk * 2048, 16384, 1024), idesc_o, 1u);
+            }
+            umma_commit(&bars[B_VE + vs]);
+            umma_commit(&bars[B_PFREE]);
           }
-          umma_commit(&bars[B_VE + vs]);
-          umma_commit(&bars[B_PFREE]);
+          __syncwarp();
           ++gs_o;
           if (s + 2 < nsteps) ok = issue_s();
         }
         if (!ok) break;
-        umma_commit(&bars[B_QE]);       // every product reading Q2 has been issued
-        umma_commit(&bars[B_OR + ob]);  // O of this pair is final once these complete
+        if (elect_one()) {
+          umma_commit(&bars[B_QE]);       // every product reading Q2 has been issued
+          umma_commit(&bars[B_OR + ob]);  // O of this pair is final once these complete
+        }
+        __syncwarp();
       }
-      umma_commit(&bars[B_FIN]);
-      mbar_wait(&bars[B_FIN], 0, a.st, a.timeout_ns, 26);
+      if (elect_one()) umma_commit(&bars[B_FIN]);
+      __syncwarp();
+      mbar_wait_drain(&bars[B_FIN], 0, a.st, a.timeout_ns, 26);
     }
   } else {
     // ------------------------------------------------------------------ softmax groups
@@ -300,17 +320,23 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         }
         uint32_t ph[32], pl[32];
         if (active) {
-          const float nm = -m_run;
-          float lsum = 0.0f;
+          const uint64_t sc2 = pk2(sc, sc), nm2 = pk2(-m_run, -m_run);
+          uint64_t l2 = pk2(0.0f, 0.0f);
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2_approx(fmaf(x[2 * c], sc, nm));
-            const float p1 = ex2_approx(fmaf(x[2 * c + 1], sc, nm));
-            lsum += p0 + p1;
+            float d0, d1;
+            upk2(fma2(pk2(x[2 * c], x[2 * c + 1]), sc2, nm2), d0, d1);
+            const float p0 = ex2_approx(d0), p1 = ex2_approx(d1);
+            const uint64_t pp = pk2(p0, p1);
+            l2 = add2(l2, pp);
             ph[c] = pack_bf16x2(p0, p1);
-            pl[c] = pack_bf16x2(p0 - __uint_as_float(ph[c] << 16), p1 - __uint_as_float(ph[c] & 0xffff0000u));
+            float r0, r1;
+            upk2(sub2(pp, pk2(__uint_as_float(ph[c] << 16), __uint_as_float(ph[c] & 0xffff0000u))), r0, r1);
+            pl[c] = pack_bf16x2(r0, r1);
           }
-          l_part += lsum;
+          float la, lb;
+          upk2(l2, la, lb);
+          l_part += la + lb;
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) ph[c] = pl[c] = 0u;
@@ -321,7 +347,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         km = a.cube_mask[e >> 2];
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bars[B_PF]);
+        mbar_arrive(&bars[B_PF + b]);
       }
       if (!ok) break;
       // -------------------------------------------------------------- epilogue
@@ -335,8 +361,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       if (grp == 0 && row_exists)
         a.lse[qrow] = row_valid ? (has ? (m_run + log2f(l)) * 0.69314718055994531f : -INFINITY) : 0.0f;
       float o[64];
+      if (!mbar_wait(&bars[B_OR + ob], (n >> 1) & 1, a.st, a.timeout_ns, 33)) *sm_abort = 1;  // every item
       if (nsteps > 0) {
-        if (!mbar_wait(&bars[B_OR + ob], (n >> 1) & 1, a.st, a.timeout_ns, 33)) *sm_abort = 1;
         tc_fence_after();
         uint32_t o0[32], o1[32];
         tmem_ld32(t_lane + 256 + ob * 128 + grp * 64, o0);
@@ -405,15 +431,20 @@ cudaError_t launch_forward(const CUtensorMap& tq, const CUtensorMap& tk, const C
                            cudaStream_t stream) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          fwd::SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_fwd_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int items = a.BH * ((a.g.T + 1) >> 1);
   const int sms = num_sms();
   const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
-  attn_fwd_kernel<<<grid, fwd::kThreads, fwd::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  if (a.D == 64)
+    attn_fwd_kernel<4><<<grid, fwd::kThreads, fwd::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  else
+    attn_fwd_kernel<8><<<grid, fwd::kThreads, fwd::SMEM_BYTES, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 

@@ -171,3 +171,54 @@ def test_deterministic_repeat():
     g4 = sa.backward(t["q"], t["k"], t["v"], o1[0], o1[1], t["do"], *r1, p, out_f32=o1[0].float())
     for a, b in zip(g3, g4):
         assert torch.equal(a, b)
+
+
+def test_empty_lists_and_unselected_key_cubes():
+    """Caller-supplied lists with runs of empty query-cube pairs and of key-cube pairs that
+    no query selects: with 8 heads x 128 pairs every CTA walks several items per stream,
+    empty ones among them.  Empty rows give out = 0, lse = -inf, dQ = 0 (the header's
+    contract for a count of 0); all other rows match the oracle restricted to them."""
+    cfg = synth.small_config("holes", 1, 8, 128, (16, 32, 32), 6, 0.9)
+    x, p, t = gpu_inputs(cfg)
+    lay = O.cube_layout(cfg.lat)
+    T = lay.n_cubes
+    drop_q = {i for i in range(T) if (i // 2) % 3 != 0}
+    drop_k = {j for j in range(T) if (j // 2) % 3 == 1}
+    trs = {}
+    for hh in range(p.H):
+        lists = O.route_head(oracle_head(x, "q", 0, hh, lay), oracle_head(x, "k", 0, hh, lay), lay.valid,
+                             cfg.top_k, cfg.top_p).lists
+        trs[(0, hh)] = [np.array([], np.int64) if i in drop_q else np.array([j for j in l if j not in drop_k],
+                                                                            np.int64) for i, l in enumerate(lists)]
+    idx, cnt = lists_to_device(trs, 1, p.H, T, p.kv_capacity)
+    out, lse, out32 = sa.forward(t["q"], t["k"], t["v"], idx, cnt, p, with_f32=True)
+    dq, dk, dv = sa.backward(t["q"], t["k"], t["v"], out, lse, t["do"], idx, cnt, p, out_f32=out32)
+    torch.cuda.synchronize()
+    for hh in range(p.H):
+        lists = trs[(0, hh)]
+        live = [i for i in range(T) if len(lists[i]) > 0]
+        assert 0 < len(live) < T
+        empty_rows = np.zeros(lay.valid.shape, bool)
+        for i in range(T):
+            if len(lists[i]) == 0:
+                empty_rows[i * 64:(i + 1) * 64] = True
+        empty_rows &= lay.valid
+        q, k, v, do = (oracle_head(x, n, 0, hh, lay) for n in ("q", "k", "v", "do"))
+        o_ref, lse_ref = O.attention_forward_head(q, k, v, lists, lay.valid, q_blocks=live)
+        rows = lay.valid & ~empty_rows
+        got = out[0, hh].float().cpu().numpy()
+        assert_close(f"out h{hh}", got[rows], o_ref[rows])
+        assert np.all(got[empty_rows] == 0)
+        gl = lse[0, hh].cpu().numpy()
+        assert np.max(np.abs(gl[rows] - lse_ref[rows])) < 1e-3
+        assert np.all(np.isneginf(gl[empty_rows]))
+        g = O.attention_backward_head(q, k, v, do, lists, lay.valid, visit=live)
+        for name, got_g, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), g):
+            a = got_g[0, hh].cpu().numpy()
+            assert_close(f"{name} h{hh}", a, ref)
+        assert np.all(dq[0, hh].cpu().numpy()[empty_rows] == 0)
+        unselected = sorted(set(range(T)) - {int(j) for l in lists for j in l})
+        assert len(unselected) >= 4
+        for j in unselected:
+            assert np.all(dk[0, hh, j * 64:(j + 1) * 64].cpu().numpy() == 0)
+            assert np.all(dv[0, hh, j * 64:(j + 1) * 64].cpu().numpy() == 0)
