@@ -193,9 +193,9 @@ def run_ours(args, rank, world, dist):
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"Wan2.1-14B-720p-shaped attention ({args.config}): B=1, H=40, D=128, latent 21x45x80 "
-                               f"-> 24x48x80 cube grid, T=1440 cubes of 64, Npad=92160; top_k={cfg.top_k}, top_p={cfg.top_p}; "
-                               "step = sa_plan + sa_forward + sa_backward",
+        "config": {"workload": f"Wan2.1-shaped attention ({args.config}): B={cfg.B}, H={cfg.H}, D={cfg.D}, latent "
+                               f"{'x'.join(map(str, cfg.lat))} -> T={T} cubes of 64, Npad={npad}; top_k={cfg.top_k}, "
+                               f"top_p={cfg.top_p}; step = sa_plan + sa_forward + sa_backward",
                    "B": cfg.B, "H": cfg.H, "D": cfg.D, "lat": list(cfg.lat), "T": T, "top_k": cfg.top_k,
                    "top_p": cfg.top_p, "density": round(density, 5), "selected_tiles": ntiles,
                    "l2": "inputs larger than L2; 256 MiB flush between steps",
@@ -212,9 +212,71 @@ def run_ours(args, rank, world, dist):
     }
     if args.e2e_steps > 0:
         result["e2e"] = run_e2e(args, sa, A, p, host, dev, fwd_fl + bwd_fl, world, dist)
+    if args.config == "720p" and not args.no_fp8:
+        del x, A
+        result["fp8_forward"] = run_fp8_forward(args, sa, synth, rank, dev, flush, peak_tf, peaks.get("hbm_gbs"), dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(cfg, host, seconds=args.cpu_seconds)
     return result
+
+
+def run_fp8_forward(args, sa, synth, rank, dev, flush, bf16_peak, hbm_peak, dist):
+    """The e4m3 Q/K configuration (config "720p_fp8": k = 22, p = 0.9, ~97% sparsity):
+    sa_plan + sa_forward with Q, K quantised per cube from the bf16 draws, V bf16.  The
+    forward's S product runs at the fp8 rate and PV at the bf16 rate, so its tensor peak
+    is 4/3 of the bf16 peak (half the FLOPs at twice the rate)."""
+    import torch
+    cfg = synth.get_config("720p_fp8")
+    host = synth.make_inputs(cfg, seed=rank_seed(rank), names=("q", "k", "v"))
+    pb = sa.make_params(cfg.B, cfg.H, cfg.D, cfg.lat, cfg.top_k, cfg.top_p)
+    p = sa.make_params(cfg.B, cfg.H, cfg.D, cfg.lat, cfg.top_k, cfg.top_p, qk_dtype=sa.FP8_E4M3)
+    npad, T = sa.geometry(p)
+    t = {n: sa.tile(host[n].to(dev), pb) for n in host}
+    q8, qs = synth.quantize_e4m3_rows(t["q"])
+    k8, ks = synth.quantize_e4m3_rows(t["k"])
+    del t["q"], t["k"]
+    A = sa.Attention(p)
+
+    def step(rec=None):
+        if rec is not None:
+            rec[0].record()
+        idx, cnt = A.plan(q8, k8, qs, ks)
+        if rec is not None:
+            rec[1].record()
+        A.forward(q8, k8, t["v"], idx, cnt, qs, ks, with_f32=False)
+        if rec is not None:
+            rec[2].record()
+        return cnt
+
+    for _ in range(max(3, args.warmup)):
+        cnt = step()
+    torch.cuda.synchronize()
+    for op in (sa.OP_PLAN, sa.OP_FORWARD):
+        st = sa.device_status(A._ws[op])
+        if st != 0:
+            raise RuntimeError(f"fp8: device status {sa.STATUS_NAMES.get(st, st)}")
+    ntiles = int(cnt.sum().item())
+    steps = max(3, min(args.steps, 10))
+    recs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for s in range(steps):
+        flush.fill_(s & 0xff)
+        step(recs[s])
+    torch.cuda.synchronize()
+    plan_ms = statistics.mean(r[0].elapsed_time(r[1]) for r in recs)
+    fwd_ms = statistics.mean(r[1].elapsed_time(r[2]) for r in recs)
+    fwd_fl, _ = tile_flops(cfg.D, ntiles)
+    tf = fwd_fl / (fwd_ms * 1e-3) / 1e12
+    peak = bf16_peak * 4.0 / 3.0
+    router_bytes = 2 * cfg.B * cfg.H * npad * cfg.D + 2 * 4 * cfg.B * cfg.H * T + 4 * (ntiles + cfg.B * cfg.H * T)
+    return {"config": f"{cfg.name}: e4m3 Q/K with per-cube scales, V bf16, top_k={cfg.top_k}, top_p={cfg.top_p}",
+            "density": round(ntiles / (cfg.B * cfg.H * T * T), 5), "selected_tiles": ntiles, "steps": steps,
+            "plan_ms": round(plan_ms, 4), "forward_ms": round(fwd_ms, 4), "forward_tflops": round(tf, 2),
+            "forward_peak_tflops": round(peak, 1), "forward_frac": round(tf / peak, 4),
+            "router_gbs": round(router_bytes / (plan_ms * 1e-3) / 1e9, 1),
+            "router_frac": round(router_bytes / (plan_ms * 1e-3) / 1e9 / hbm_peak, 4)}
 
 
 def max_over_ranks(x: float, dist, device) -> float:
@@ -372,6 +434,7 @@ def main():
     ap.add_argument("--config", default="720p")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the e4m3 Q/K forward section")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

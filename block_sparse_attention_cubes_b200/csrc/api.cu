@@ -248,9 +248,11 @@ sa_status sa_forward(const void* q, const void* k, const void* v, const float* q
   sa_status s = check_params(p, &g);
   if (s != SA_OK) return s;
   if (!q || !k || !v || !kv_index || !kv_count || !out || !lse) return SA_ERR_INVALID_ARG;
-  if (p->qk_dtype == SA_FP8_E4M3) return SA_ERR_UNSUPPORTED;
+  const bool fp8 = p->qk_dtype == SA_FP8_E4M3;
+  if (fp8 && p->D != 128) return SA_ERR_UNSUPPORTED;  // one 128-byte e4m3 row per token
+  if (fp8 && (!q_scale || !k_scale)) return SA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(lse) || !aligned4(kv_index) ||
-      !aligned4(kv_count) || (out_f32 && !aligned16(out_f32)))
+      !aligned4(kv_count) || (out_f32 && !aligned16(out_f32)) || (fp8 && (!aligned4(q_scale) || !aligned4(k_scale))))
     return SA_ERR_ALIGNMENT;
   const WsLayout w = ws_layout(p, g, SA_OP_FORWARD);
   if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
@@ -262,8 +264,14 @@ sa_status sa_forward(const void* q, const void* k, const void* v, const float* q
   a.out = static_cast<__nv_bfloat16*>(out);
   a.out_f32 = out_f32;
   a.lse = lse;
+  a.qk_fp8 = fp8 ? 1 : 0;
+  if (fp8) {
+    a.q_scale = q_scale;
+    a.k_scale = k_scale;
+  }
+  const int qk_esize = fp8 ? 1 : 2;
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, a.rows_total, p->D, 2) || !make_map(&tk, k, a.rows_total, p->D, 2) ||
+  if (!make_map(&tq, q, a.rows_total, p->D, qk_esize) || !make_map(&tk, k, a.rows_total, p->D, qk_esize) ||
       !make_map(&tv, v, a.rows_total, p->D, 2))
     return SA_ERR_LAUNCH;
   if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;

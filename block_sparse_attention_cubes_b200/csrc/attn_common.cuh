@@ -30,6 +30,7 @@ struct AttnArgs {
   DevStatus* st;
   Geom g;
   int BH, D, cap;
+  int qk_fp8;               // Q and K are e4m3 bytes with per-cube scales q_scale / k_scale
   int rows_total;           // BH * Npad, the first out-of-range row for zero-filled loads
   float scale;              // softmax scale
   float scale_log2;         // softmax scale * log2(e)

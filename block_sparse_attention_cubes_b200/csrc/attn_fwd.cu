@@ -56,7 +56,10 @@ enum {
 // KS = D / 16 k-steps per S product.  Every MMA loop below has a compile-time trip count and
 // is unrolled: a single issuing thread running a counted loop spends far more than the
 // tensor core's 64 cycles per 128x128x16 product on the loop itself.
-template <int KS>
+// FP8: Q and K are e4m3 bytes (one 128-byte row per token at D = 128) and S comes from a
+// kind::f8f6f4 product (K = 32 per instruction, 4 k-steps); the per-cube scales enter in
+// the softmax.  V and the PV product stay bf16.
+template <int KS, bool FP8>
 __global__ void __launch_bounds__(fwd::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
@@ -120,11 +123,13 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           if (n >= 1 && !mbar_wait(&bars[B_QE], (n - 1) & 1, a.st, a.timeout_ns, 11)) break;
           const int r0 = bh * g.Npad + (2 * pr) * 64;
           const int r1 = (2 * pr + 1 < g.T) ? r0 + 64 : a.rows_total;
-          mbar_arrive_expect_tx(&bars[B_QF], 32768);
+          mbar_arrive_expect_tx(&bars[B_QF], FP8 ? 16384 : 32768);
           tma_load_2d(smem + OFF_Q, &tm_q, &bars[B_QF], 0, r0);
           tma_load_2d(smem + OFF_Q + 8192, &tm_q, &bars[B_QF], 0, r1);
-          tma_load_2d(smem + OFF_Q + 16384, &tm_q, &bars[B_QF], 64, r0);
-          tma_load_2d(smem + OFF_Q + 24576, &tm_q, &bars[B_QF], 64, r1);
+          if (!FP8) {
+            tma_load_2d(smem + OFF_Q + 16384, &tm_q, &bars[B_QF], 64, r0);
+            tma_load_2d(smem + OFF_Q + 24576, &tm_q, &bars[B_QF], 64, r1);
+          }
           ++issued_q;
         }
         const int nsteps = (nu + 1) >> 1;
@@ -142,11 +147,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           const int y1 = t1 >= 0 ? bh * g.Npad + t1 * 64 : a.rows_total;
           const uint32_t full = (kq ? B_KF : B_VF) + st;
           uint8_t* dst = smem + (kq ? OFF_K : OFF_V) + st * 32768;
-          mbar_arrive_expect_tx(&bars[full], 32768);
+          const bool one_box = FP8 && kq;  // an e4m3 K row is a single 128-byte box
+          mbar_arrive_expect_tx(&bars[full], one_box ? 16384 : 32768);
           tma_load_2d(dst, tmap, &bars[full], 0, y0);
           tma_load_2d(dst + 8192, tmap, &bars[full], 0, y1);
-          tma_load_2d(dst + 16384, tmap, &bars[full], 64, y0);
-          tma_load_2d(dst + 24576, tmap, &bars[full], 64, y1);
+          if (!one_box) {
+            tma_load_2d(dst + 16384, tmap, &bars[full], 64, y0);
+            tma_load_2d(dst + 24576, tmap, &bars[full], 64, y1);
+          }
           ++gs;
         }
       }
@@ -160,6 +168,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (!skip_all) {
       const uint32_t idesc_s = make_idesc(128, 128, FMT_BF16, false, false);
+      const uint32_t idesc_s8 = make_idesc(128, 128, FMT_E4M3, false, false);
       const uint32_t idesc_o = make_idesc(128, 128, FMT_BF16, false, true);
       uint32_t gs_s = 0, gs_o = 0;
       bool ok = true;
@@ -172,11 +181,18 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         tc_fence_after();
         const uint32_t kst = sbase + OFF_K + kst_i * 32768;
         if (elect_one()) {
+          if (FP8) {
 #pragma unroll
-          for (int ks = 0; ks < KS; ++ks) {
-            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-            umma_f16_ss(tmem + sb * 128, sw128_desc(sbase + OFF_Q + off, 16, 1024), sw128_desc(kst + off, 16, 1024),
-                        idesc_s, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < 4; ++ks)  // 32 e4m3 elements = 32 bytes per k-step
+              umma_f8_ss(tmem + sb * 128, sw128_desc(sbase + OFF_Q + ks * 32, 16, 1024),
+                         sw128_desc(kst + ks * 32, 16, 1024), idesc_s8, ks > 0 ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+              const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+              umma_f16_ss(tmem + sb * 128, sw128_desc(sbase + OFF_Q + off, 16, 1024),
+                          sw128_desc(kst + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+            }
           }
           umma_commit(&bars[B_SF + sb]);
           umma_commit(&bars[B_KE + kst_i]);
@@ -431,20 +447,18 @@ cudaError_t launch_forward(const CUtensorMap& tq, const CUtensorMap& tk, const C
                            cudaStream_t stream) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         fwd::SMEM_BYTES);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn_fwd_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::SMEM_BYTES);
+    cudaError_t e = cudaSuccess;
+    for (auto fn : {attn_fwd_kernel<4, false>, attn_fwd_kernel<8, false>, attn_fwd_kernel<8, true>})
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int items = a.BH * ((a.g.T + 1) >> 1);
   const int sms = num_sms();
   const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
-  if (a.D == 64)
-    attn_fwd_kernel<4><<<grid, fwd::kThreads, fwd::SMEM_BYTES, stream>>>(tq, tk, tv, a);
-  else
-    attn_fwd_kernel<8><<<grid, fwd::kThreads, fwd::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  // e4m3 Q/K is built for D = 128 only (the host rejects other head sizes)
+  auto fn = a.qk_fp8 ? attn_fwd_kernel<8, true> : (a.D == 64 ? attn_fwd_kernel<4, false> : attn_fwd_kernel<8, false>);
+  fn<<<grid, fwd::kThreads, fwd::SMEM_BYTES, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 

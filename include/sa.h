@@ -121,6 +121,10 @@ SA_API sa_status sa_plan(const void* q, const void* k, const float* q_scale, con
  * q, k: as for sa_plan; v: [B,H,Npad,D] bf16; kv_index/kv_count: as written by sa_plan
  *   (entries must lie in [0,T), counts in [0,kv_capacity]; violations are recorded as
  *   SA_ERR_DEVICE_INDEX and the offending entries skipped).
+ * With qk_dtype == SA_FP8_E4M3 (D = 128 only, else SA_ERR_UNSUPPORTED; q_scale and k_scale
+ * required, else SA_ERR_INVALID_ARG): S = (Q8 K8^T) * q_scale[i] * k_scale[j] * scale from an
+ * e4m3 tensor-core product with fp32 accumulation (SparkDiffusion page, section 4.3, E4M3);
+ * P and V stay bf16.
  * out: [B,H,Npad,D] bf16; lse: [B,H,Npad] fp32, natural log of each row's softmax
  * normaliser of the scaled scores.  Padding query rows get out = 0, lse = 0; a row with
  * count 0 gets out = 0, lse = -inf.  out_f32 (may be NULL): [B,H,Npad,D] fp32, the same

@@ -78,3 +78,46 @@ def test_480p_full_router_sampled_attention():
 
 def test_720p_full_router_sampled_attention():
     _full("720p", sample_heads=(0, 20), nq=8, nkv=4)
+
+
+def test_720p_fp8_full_router_sampled_forward():
+    """The e4m3 Q/K configuration: Q and K quantised per cube from the same bf16 draws;
+    router and forward against the oracle on the dequantised values (V stays bf16)."""
+    cfg = synth.get_config("720p_fp8")
+    x = synth.make_inputs(cfg, 0, names=("q", "k", "v"))
+    p = sa.make_params(cfg.B, cfg.H, cfg.D, cfg.lat, cfg.top_k, cfg.top_p, qk_dtype=sa.FP8_E4M3)
+    pb = sa.make_params(cfg.B, cfg.H, cfg.D, cfg.lat, cfg.top_k, cfg.top_p)
+    dev = torch.device("cuda")
+    t = {n: sa.tile(x[n].to(dev), pb) for n in x}
+    q8, qs = synth.quantize_e4m3_rows(t["q"])
+    k8, ks = synth.quantize_e4m3_rows(t["k"])
+    A = sa.Attention(p)
+    idx, cnt = A.plan(q8, k8, qs, ks)
+    out, lse, _ = A.forward(q8, k8, t["v"], idx, cnt, qs, ks, with_f32=False)
+    torch.cuda.synchronize()
+    for op in (sa.OP_PLAN, sa.OP_FORWARD):
+        assert sa.device_status(A._ws[op]) == 0
+    lay = O.cube_layout(cfg.lat)
+    T = lay.n_cubes
+    q8n, k8n, qsn, ksn = (a.cpu().numpy() for a in (q8, k8, qs, ks))
+    ties = 0
+    for h in range(cfg.H):
+        q = O.dequantize_rows(q8n[0, h], qsn[0, h])
+        k = O.dequantize_rows(k8n[0, h], ksn[0, h])
+        tr = O.route_head(q, k, lay.valid, cfg.top_k, cfg.top_p)
+        lists = gpu_lists(idx, cnt, 0, h)
+        mis, tie, bad = classify_router_rows(tr, lists, cfg.top_p)
+        assert mis == 0, f"head {h}: rows {bad[:5]}"
+        ties += tie
+        if h not in (0, 20):
+            continue
+        rng = np.random.default_rng(h)
+        qb = np.sort(rng.choice(T, 8, replace=False))
+        qb[0] = T - 1
+        v = O.tile(x["v"][0, h].double().numpy(), lay)
+        o_ref, lse_ref = O.attention_forward_head(q, k, v, lists, lay.valid, q_blocks=qb)
+        rows = np.concatenate([np.arange(i * 64, (i + 1) * 64) for i in qb])
+        rows = rows[lay.valid[rows]]
+        assert_close(f"out h{h}", out[0, h].float().cpu().numpy()[rows], o_ref[rows])
+        assert np.max(np.abs(lse[0, h].cpu().numpy()[rows] - lse_ref[rows])) < 1e-3
+    assert ties <= max(2, 1e-3 * cfg.H * T)

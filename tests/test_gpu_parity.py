@@ -222,3 +222,47 @@ def test_empty_lists_and_unselected_key_cubes():
         for j in unselected:
             assert np.all(dk[0, hh, j * 64:(j + 1) * 64].cpu().numpy() == 0)
             assert np.all(dv[0, hh, j * 64:(j + 1) * 64].cpu().numpy() == 0)
+
+
+@pytest.mark.parametrize("lat,k,pp", [((4, 4, 4), 1, 0.9), ((5, 8, 12), 3, 0.9), ((9, 9, 9), 50, 0.3)])
+def test_fp8_router_and_forward_small(lat, k, pp):
+    """e4m3 Q/K with one scale per cube (quantised from the bf16 draws): router lists and
+    forward against the oracle run on the dequantised Q and K."""
+    cfg = synth.small_config("f8", 1, 2, 128, lat, k, pp)
+    x, pb, t = gpu_inputs(cfg, names=("q", "k", "v"))
+    p = sa.make_params(cfg.B, cfg.H, cfg.D, cfg.lat, cfg.top_k, cfg.top_p, qk_dtype=sa.FP8_E4M3)
+    q8, qs = synth.quantize_e4m3_rows(t["q"])
+    k8, ks = synth.quantize_e4m3_rows(t["k"])
+    idx, cnt = sa.plan(q8, k8, p, qs, ks)
+    out, lse = sa.forward(q8, k8, t["v"], idx, cnt, p, qs, ks)
+    out_f, lse_f, out32 = sa.forward(q8, k8, t["v"], idx, cnt, p, qs, ks, with_f32=True)
+    torch.cuda.synchronize()
+    assert torch.equal(out32.to(torch.bfloat16), out_f)
+    lay = O.cube_layout(cfg.lat)
+    q8n, k8n, qsn, ksn = (a.cpu().numpy() for a in (q8, k8, qs, ks))
+    for hh in range(p.H):
+        q = O.dequantize_rows(q8n[0, hh], qsn[0, hh])
+        kk = O.dequantize_rows(k8n[0, hh], ksn[0, hh])
+        tr = O.route_head(q, kk, lay.valid, cfg.top_k, cfg.top_p)
+        lists = gpu_lists(idx, cnt, 0, hh)
+        mis, ties, bad = classify_router_rows(tr, lists, cfg.top_p)
+        assert mis == 0, f"head {hh}: rows {bad[:5]}"
+        v = oracle_head(x, "v", 0, hh, lay)
+        o_ref, lse_ref = O.attention_forward_head(q, kk, v, lists, lay.valid)
+        rows = lay.valid
+        for name, o in (("out", out), ("out (split P)", out_f)):
+            got = o[0, hh].float().cpu().numpy()
+            assert_close(f"{name} h{hh}", got[rows], o_ref[rows])
+            assert np.all(got[~rows] == 0)
+        assert np.max(np.abs(lse[0, hh].cpu().numpy()[rows] - lse_ref[rows])) < 1e-3
+
+
+def test_fp8_host_checks(cuda_ok):
+    p = sa.make_params(1, 1, 64, (4, 4, 4), 1, 0.5, qk_dtype=sa.FP8_E4M3)   # e4m3 needs D = 128
+    z8 = torch.zeros(1, 1, 64, 64, dtype=torch.uint8, device="cuda")
+    zb = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16, device="cuda")
+    sc = torch.ones(1, 1, 1, device="cuda")
+    idx = torch.zeros(1, 1, 1, 1, dtype=torch.int32, device="cuda")
+    cnt = torch.ones(1, 1, 1, dtype=torch.int32, device="cuda")
+    with pytest.raises(RuntimeError, match="UNSUPPORTED"):
+        sa.forward(z8, z8, zb, idx, cnt, p, sc, sc)
