@@ -279,6 +279,119 @@ def run_fp8_forward(args, sa, synth, rank, dev, flush, bf16_peak, hbm_peak, dist
             "router_frac": round(router_bytes / (plan_ms * 1e-3) / 1e9 / hbm_peak, 4)}
 
 
+def cta_balance(masks, sms: int):
+    """Per-CTA work of the persistent attention kernels, from the selection alone.
+
+    ``masks``: one boolean [T, T] matrix per (b, h), M[i, j] = query cube i selected key
+    cube j.  The forward and dQ kernels take query-cube pairs (rows 2p, 2p+1), the dK/dV
+    kernel key-cube pairs (columns 2p, 2p+1); item it = bh * ceil(T/2) + pair goes to CTA
+    it mod G with G = min(items, sms); one step covers two union entries (128 keys).
+    Returns max/mean of per-CTA steps and tiles for both kernels, and the union
+    inflation (union entries walked per selected tile)."""
+    import numpy as np
+
+    def pair_items(M):
+        T = M.shape[0]
+        if T % 2:
+            M = np.concatenate([M, np.zeros((1, M.shape[1]), bool)])
+        a, b = M[0::2], M[1::2]
+        return (((a | b).sum(1) + 1) // 2), a.sum(1) + b.sum(1), (a | b).sum(1)
+
+    def stats(item_steps, item_tiles):
+        n = len(item_steps)
+        G = min(n, sms)
+        st = np.bincount(np.arange(n) % G, weights=item_steps, minlength=G)
+        tl = np.bincount(np.arange(n) % G, weights=item_tiles, minlength=G)
+        return {"ctas": G, "steps_max_over_mean": round(float(st.max() / st.mean()), 4),
+                "tiles_max_over_mean": round(float(tl.max() / tl.mean()), 4),
+                "steps_per_cta_mean": round(float(st.mean()), 1), "steps_per_cta_max": int(st.max())}
+
+    q = [pair_items(M) for M in masks]
+    k = [pair_items(M.T) for M in masks]
+    qs, qt, qu = (np.concatenate([x[c] for x in q]) for c in range(3))
+    ks, kt, _ = (np.concatenate([x[c] for x in k]) for c in range(3))
+    return {"forward_dq": stats(qs, qt), "dkdv": stats(ks, kt),
+            "union_entries_per_tile": round(float(qu.sum() / max(1, qt.sum())), 4)}
+
+
+def selection_masks(idx, cnt):
+    """[B,H,T,cap] index lists + counts -> one boolean [T, T] selection matrix per (b, h)."""
+    import numpy as np
+    ic, cc = idx.cpu().numpy(), cnt.cpu().numpy()
+    B, H, T, cap = ic.shape
+    masks = []
+    for b in range(B):
+        for h in range(H):
+            M = np.zeros((T, T), bool)
+            used = np.arange(cap)[None, :] < cc[b, h][:, None]
+            rows = np.broadcast_to(np.arange(T)[:, None], (T, cap))
+            M[rows[used], ic[b, h][used]] = True
+            masks.append(M)
+    return masks
+
+
+def run_sweep(args):
+    """Config-4 sweep at the 720p shape: k = 4, p in {0.8, 0.9, 0.95}, locality amplitude calibrated
+    (at p = 0.9) for 80..98% sparsity.  One JSON line per point: step timings and the per-CTA
+    load balance of the persistent attention kernels."""
+    import torch
+
+    import block_sparse_attention_cubes_b200 as sa
+    import synth
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    for sp in (80, 85, 90, 95, 98):
+        for pp in (0.8, 0.9, 0.95):
+            cfg = synth.get_config(f"sweep_{pp}_{sp}")
+            host = synth.make_inputs(cfg, seed=0)
+            p = sa.make_params(cfg.B, cfg.H, cfg.D, cfg.lat, cfg.top_k, cfg.top_p)
+            npad, T = sa.geometry(p)
+            x = {n: sa.tile(host[n].to(dev), p) for n in ("q", "k", "v", "do")}
+            A = sa.Attention(p)
+
+            def step(rec=None):
+                if rec is not None:
+                    rec[0].record()
+                idx, cnt = A.plan(x["q"], x["k"])
+                if rec is not None:
+                    rec[1].record()
+                out, lse, out32 = A.forward(x["q"], x["k"], x["v"], idx, cnt)
+                if rec is not None:
+                    rec[2].record()
+                A.backward(x["q"], x["k"], x["v"], out, lse, x["do"], idx, cnt, out_f32=out32)
+                if rec is not None:
+                    rec[3].record()
+                return idx, cnt
+
+            for _ in range(3):
+                idx, cnt = step()
+            torch.cuda.synchronize()
+            for op in (sa.OP_PLAN, sa.OP_FORWARD, sa.OP_BACKWARD):
+                if sa.device_status(A._ws[op]) != 0:
+                    raise RuntimeError(f"sweep {cfg.name}: device status {sa.device_status(A._ws[op])}")
+            recs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+            for s in range(args.steps):
+                flush.fill_(s & 0xff)
+                step(recs[s])
+            torch.cuda.synchronize()
+            ms = [statistics.mean(r[k].elapsed_time(r[k + 1]) for r in recs) for k in range(3)]
+            ntiles = int(cnt.sum().item())
+            fwd_fl, bwd_fl = tile_flops(cfg.D, ntiles)
+            masks = selection_masks(idx, cnt)
+            row_n = cnt[0].cpu().numpy().astype(float)
+            line = {"config": cfg.name, "top_k": cfg.top_k, "top_p": cfg.top_p,
+                    "sparsity": round(1 - ntiles / (cfg.H * T * T), 4), "selected_tiles": ntiles,
+                    "blocks_per_row": {"mean": round(float(row_n.mean()), 1), "min": int(row_n.min()),
+                                       "max": int(row_n.max())},
+                    "plan_ms": round(ms[0], 3), "forward_ms": round(ms[1], 3), "backward_ms": round(ms[2], 3),
+                    "forward_tflops": round(fwd_fl / (ms[1] * 1e-3) / 1e12, 1),
+                    "backward_tflops": round(bwd_fl / (ms[2] * 1e-3) / 1e12, 1),
+                    "balance": cta_balance(masks, sms)}
+            print(json.dumps(line), flush=True)
+            del x, A
+
+
 def max_over_ranks(x: float, dist, device) -> float:
     """Max of a per-rank scalar over all ranks (identity without a process group)."""
     if dist is None:
@@ -435,12 +548,18 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the e4m3 Q/K forward section")
+    ap.add_argument("--sweep", action="store_true",
+                    help="config-4 sweep (k=4, p x sparsity grid): one JSON line per point with load balance")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.sweep:
+        if rank == 0:
+            run_sweep(args)
+        return
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args, rank, world)), flush=True)

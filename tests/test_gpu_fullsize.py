@@ -121,3 +121,9 @@ def test_720p_fp8_full_router_sampled_forward():
         assert_close(f"out h{h}", out[0, h].float().cpu().numpy()[rows], o_ref[rows])
         assert np.max(np.abs(lse[0, h].cpu().numpy()[rows] - lse_ref[rows])) < 1e-3
     assert ties <= max(2, 1e-3 * cfg.H * T)
+
+
+def test_sweep_densest_full_router_sampled_attention():
+    """Config-4 sweep point with the longest lists (k = 4, p = 0.8 at the amplitude
+    calibrated for 80% sparsity): ragged unions of up to min(2 cap, T) entries."""
+    _full("sweep_0.8_80", sample_heads=(0, 20), nq=6, nkv=3)
