@@ -561,32 +561,34 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
         if (!mbar_wait_warp(&bars[B_KVF], n & 1, a.st, a.timeout_ns, 81)) break;
         // one phase of DVR / DVFREE per item, empty items included (see the dQ kernel)
         if (n >= 1 && !mbar_wait_warp(&bars[B_DVFREE], (n - 1) & 1, a.st, a.timeout_ns, 82)) break;
-        for (int s = 0; ok && s < nsteps; ++s, ++gs) {
-          const uint32_t st = gs % QST;
-          ok = mbar_wait_warp(&bars[B_QF + st], (gs / QST) & 1, a.st, a.timeout_ns, 83) &&
-               mbar_wait_warp(&bars[B_DF + st], (gs / QST) & 1, a.st, a.timeout_ns, 84);
-          if (!ok) break;
+        // Issue order per step s:  dV(s), S^T(s+1), dK(s), dP^T(s+1).  S^T(s+1) overwrites P^T(s),
+        // already read by dV(s); dP^T(s+1) overwrites dS^T(s), already read by dK(s) (one lane
+        // issues everything, so the products execute in this order).  The exponentials of step
+        // s+1 then overlap dK(s), and dS^T(s+1) overlaps dV(s+1).
+        auto issue_sdp = [&](uint32_t g, bool want_s) -> bool {
+          const uint32_t st = g % QST;
+          if (!mbar_wait_warp(want_s ? &bars[B_QF + st] : &bars[B_DF + st], (g / QST) & 1, a.st, a.timeout_ns,
+                              want_s ? 83 : 84))
+            return false;
           tc_fence_after();
-          const uint32_t qst = sbase + OFF_Q + st * 32768, dst = sbase + OFF_DO + st * 32768;
-          // S^T and dP^T overwrite the previous step's P^T / dS^T, read by dV / dK issued
-          // earlier by the same lane (in-order execution)
+          const uint32_t opnd = sbase + (want_s ? OFF_Q : OFF_DO) + st * 32768;
+          const uint32_t kv = sbase + (want_s ? OFF_K : OFF_V);
           if (elect_one()) {
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
               const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-              umma_f16_ss(tmem + 0, sw128_desc(sbase + OFF_K + off, 16, 1024), sw128_desc(qst + off, 16, 1024),
+              umma_f16_ss(tmem + (want_s ? 0 : 128), sw128_desc(kv + off, 16, 1024), sw128_desc(opnd + off, 16, 1024),
                           idesc_kk, ks > 0 ? 1u : 0u);
             }
-            umma_commit(&bars[B_SF]);  // the exponentials can start while dP^T is computed
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-              const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-              umma_f16_ss(tmem + 128, sw128_desc(sbase + OFF_V + off, 16, 1024), sw128_desc(dst + off, 16, 1024),
-                          idesc_kk, ks > 0 ? 1u : 0u);
-            }
-            umma_commit(&bars[B_DPF]);
+            umma_commit(&bars[want_s ? B_SF : B_DPF]);
           }
           __syncwarp();
+          return true;
+        };
+        if (nsteps > 0) ok = issue_sdp(gs, true) && issue_sdp(gs, false);
+        for (int s = 0; ok && s < nsteps; ++s, ++gs) {
+          const uint32_t st = gs % QST;
+          const uint32_t qst = sbase + OFF_Q + st * 32768, dst = sbase + OFF_DO + st * 32768;
           if (!mbar_wait_warp(&bars[B_PF], gs & 1, a.st, a.timeout_ns, 85)) {
             ok = false;
             break;
@@ -602,6 +604,10 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
             }
           }
           __syncwarp();
+          if (s + 1 < nsteps && !issue_sdp(gs + 1, true)) {
+            ok = false;
+            break;
+          }
           if (!mbar_wait_warp(&bars[B_DSF], gs & 1, a.st, a.timeout_ns, 87)) {
             ok = false;
             break;
@@ -615,10 +621,15 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
               umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(qst + kk * 2048, 16384, 1024), idesc_mn,
                           (s > 0 || ks > 0) ? 1u : 0u);
             }
+            // the Q and dO stages (with their lse and Delta, read by the softmax before DSF) are free
             umma_commit(&bars[B_QE + st]);
             umma_commit(&bars[B_DE + st]);
           }
           __syncwarp();
+          if (s + 1 < nsteps && !issue_sdp(gs + 1, false)) {
+            ok = false;
+            break;
+          }
         }
         if (!ok) break;
         if (elect_one()) {
