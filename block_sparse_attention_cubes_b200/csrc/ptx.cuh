@@ -81,7 +81,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, DevSta
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 0u) {
+    if ((it & 255u) == 0u) {
       if (aborted(st)) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
         flag_error(st, DEVERR_TIMEOUT, where);

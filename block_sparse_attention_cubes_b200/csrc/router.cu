@@ -96,51 +96,57 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint8_t* __restrict__ q
 }
 
 // ------------------------------------------------------------------------ block scores
-// S[bh][i][j] = scale * sum_d Qbar[bh][i][d] * Kbar[bh][j][d], fp64, 64x64 tile per CTA.
+// S[bh][i][j] = scale * sum_d Qbar[bh][i][d] * Kbar[bh][j][d], fp64.  One 128x128 tile per
+// CTA, 16-deep slices of Qbar and Kbar staged in shared memory; each of the 256 threads
+// accumulates an 8x8 block of rows ty + 16u and columns tx + 16v (u, v < 8), so a warp's
+// Qbar reads are two broadcast addresses and its Kbar reads 16 consecutive doubles.
+constexpr int SC_TILE = 128, SC_K = 16, SC_PAD = SC_TILE + 2;
 __global__ void __launch_bounds__(256) score_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
                                                     double* __restrict__ S, int T, int D, double scale) {
-  __shared__ double As[16][65];
-  __shared__ double Bs[16][65];
+  __shared__ double As[SC_K][SC_PAD];
+  __shared__ double Bs[SC_K][SC_PAD];
   const int bh = blockIdx.z;
-  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
+  const int i0 = blockIdx.y * SC_TILE, j0 = blockIdx.x * SC_TILE;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const double* Q = qbar + static_cast<size_t>(bh) * T * D;
   const double* K = kbar + static_cast<size_t>(bh) * T * D;
-  double acc[4][4];
+  double acc[8][8];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int u = 0; u < 8; ++u)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
-  for (int d0 = 0; d0 < D; d0 += 16) {
-    for (int e = threadIdx.x; e < 1024; e += 256) {
-      const int r = e >> 4, dd = e & 15;
+    for (int v = 0; v < 8; ++v) acc[u][v] = 0.0;
+  for (int d0 = 0; d0 < D; d0 += SC_K) {
+    // 128 rows x 16 doubles of each operand: thread e takes row e / 16 + 16 w, column e % 16
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const int r = (threadIdx.x >> 4) + 16 * w, dd = threadIdx.x & 15;
       As[dd][r] = (i0 + r < T) ? Q[static_cast<size_t>(i0 + r) * D + d0 + dd] : 0.0;
       Bs[dd][r] = (j0 + r < T) ? K[static_cast<size_t>(j0 + r) * D + d0 + dd] : 0.0;
     }
     __syncthreads();
 #pragma unroll
-    for (int dd = 0; dd < 16; ++dd) {
-      double a[4], b[4];
+    for (int dd = 0; dd < SC_K; ++dd) {
+      double a[8], b[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        a[u] = As[dd][ty * 4 + u];
-        b[u] = Bs[dd][tx * 4 + u];
+      for (int u = 0; u < 8; ++u) {
+        a[u] = As[dd][ty + 16 * u];
+        b[u] = Bs[dd][tx + 16 * u];
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < 8; ++u)
 #pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] = fma(a[u], b[v], acc[u][v]);
+        for (int v = 0; v < 8; ++v) acc[u][v] = fma(a[u], b[v], acc[u][v]);
     }
     __syncthreads();
   }
   double* out = S + static_cast<size_t>(bh) * T * T;
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int i = i0 + ty * 4 + u;
+  for (int u = 0; u < 8; ++u) {
+    const int i = i0 + ty + 16 * u;
     if (i >= T) continue;
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int j = j0 + tx * 4 + v;
+    for (int v = 0; v < 8; ++v) {
+      const int j = j0 + tx + 16 * v;
       if (j < T) out[static_cast<size_t>(i) * T + j] = acc[u][v] * scale;
     }
   }
@@ -195,13 +201,37 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
         mass[d] = 0ull;
       }
       __syncwarp();
-      for (int j = lane; j < T; j += 32) {
-        const double x = s[j];
-        const uint64_t kj = desc_key(x);
-        if (shift == 56 || (kj >> (shift + 8)) == (prefix >> (shift + 8))) {
-          const int d = static_cast<int>((kj >> shift) & 255u);
+      // Keys of one binade share their top bytes, so in the first passes most lanes of a warp
+      // fall in the same bucket: then the warp adds its count and (exact, fixed-point) mass
+      // once instead of 32 colliding shared-memory atomics.
+      for (int j0 = 0; j0 < T; j0 += 32) {
+        const int j = j0 + lane;
+        bool part = false;
+        int d = 0;
+        unsigned long long mj = 0ull;
+        if (j < T) {
+          const double x = s[j];
+          const uint64_t kj = desc_key(x);
+          if (shift == 56 || (kj >> (shift + 8)) == (prefix >> (shift + 8))) {
+            part = true;
+            d = static_cast<int>((kj >> shift) & 255u);
+            mj = static_cast<unsigned long long>(mass_fx(x, m));
+          }
+        }
+        const uint32_t act = __ballot_sync(0xffffffffu, part);
+        if (act == 0u) continue;
+        const int dl = __shfl_sync(0xffffffffu, d, __ffs(act) - 1);
+        if (__all_sync(0xffffffffu, !part || d == dl)) {
+          unsigned long long ms = mj;
+#pragma unroll
+          for (int o = 16; o; o >>= 1) ms += __shfl_xor_sync(0xffffffffu, ms, o);
+          if (lane == 0) {
+            atomicAdd(&cnt[dl], static_cast<uint32_t>(__popc(act)));
+            atomicAdd(&mass[dl], ms);
+          }
+        } else if (part) {
           atomicAdd(&cnt[d], 1u);
-          atomicAdd(&mass[d], static_cast<unsigned long long>(mass_fx(x, m)));
+          atomicAdd(&mass[d], mj);
         }
       }
       __syncwarp();
@@ -330,7 +360,7 @@ cudaError_t launch_plan(const void* q, const void* k, const float* q_scale, cons
   else
     pool_kernel<2><<<pg, 256, 0, stream>>>(static_cast<const uint8_t*>(q), static_cast<const uint8_t*>(k), q_scale,
                                            k_scale, qbar, kbar, g, D);
-  dim3 sg((g.T + 63) / 64, (g.T + 63) / 64, BH);
+  dim3 sg((g.T + SC_TILE - 1) / SC_TILE, (g.T + SC_TILE - 1) / SC_TILE, BH);
   score_kernel<<<sg, 256, 0, stream>>>(qbar, kbar, S, g.T, D, scale);
   const int rows = BH * g.T;
   select_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(S, kv_index, kv_count, rows, g.T, top_k, top_p, cap, st);
