@@ -369,17 +369,25 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
           tmem_ld32(t_lane + 256 + grp * 64, p0);
           tmem_ld32(t_lane + 256 + grp * 64 + 32, p1);
           tmem_ld_wait();
+          // the key mask is first used here, so its load (issued a step earlier) hides behind the waits
           const unsigned long long km = active ? km_cur : 0ull;
+          const uint64_t sc2 = pk2(a.scale_log2, a.scale_log2), nl2 = pk2(-lse2, -lse2), dl2 = pk2(dlt, dlt);
+          const bool full = km == ~0ull;  // uniform over the warp
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const int c0 = 2 * c, c1 = 2 * c + 1;
             const uint32_t sa0 = c0 < 32 ? s0[c0] : s1[c0 - 32], sa1 = c1 < 32 ? s0[c1] : s1[c1 - 32];
             const uint32_t pa0 = c0 < 32 ? p0[c0] : p1[c0 - 32], pa1 = c1 < 32 ? p0[c1] : p1[c1 - 32];
-            const float e0 = ((km >> c0) & 1ull) ? ex2_approx(fmaf(__uint_as_float(sa0), a.scale_log2, -lse2)) : 0.0f;
-            const float e1 = ((km >> c1) & 1ull) ? ex2_approx(fmaf(__uint_as_float(sa1), a.scale_log2, -lse2)) : 0.0f;
-            const float d0 = e0 * (__uint_as_float(pa0) - dlt), d1 = e1 * (__uint_as_float(pa1) - dlt);
-            hi[c] = pack_bf16x2(d0, d1);
-            lo[c] = pack_bf16x2(d0 - __uint_as_float(hi[c] << 16), d1 - __uint_as_float(hi[c] & 0xffff0000u));
+            float x0, x1;
+            upk2(fma2(pk2(__uint_as_float(sa0), __uint_as_float(sa1)), sc2, nl2), x0, x1);
+            float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+            if (!full) {
+              if (!((km >> c0) & 1ull)) e0 = 0.0f;
+              if (!((km >> c1) & 1ull)) e1 = 0.0f;
+            }
+            float d0, d1;
+            upk2(mul2(pk2(e0, e1), sub2(pk2(__uint_as_float(pa0), __uint_as_float(pa1)), dl2)), d0, d1);
+            split_bf16x2(d0, d1, hi[c], lo[c]);
           }
         } else {
 #pragma unroll
@@ -665,7 +673,6 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
         const int e_next = (2 * s + 2 + grp < nu) ? ul[2 * s + 2 + grp] : 0;
         const bool active = ((e >> khalf) & 1) && key_valid;
         const bool w_active = __any_sync(0xffffffffu, active);
-        const unsigned long long qm = active ? qm_cur : 0ull;
         if (!mbar_wait(&bars[B_SF], gs & 1, a.st, a.timeout_ns, 91)) *sm_abort = 1;
         tc_fence_after();
         // P^T = exp(S^T * scale - lse_q): written as soon as it is known so that dV can start
@@ -677,6 +684,9 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
             tmem_ld32(t_lane + grp * 64, s0);
             tmem_ld32(t_lane + grp * 64 + 32, s1);
             tmem_ld_wait();
+            // the query mask is first used here, so its load hides behind the waits
+            const unsigned long long qm = active ? qm_cur : 0ull;
+            const bool full = qm == ~0ull;  // uniform over the warp
             const float* lq = lse_sh + st * 128 + grp * 64;
 #pragma unroll
             for (int c4 = 0; c4 < 16; ++c4) {
@@ -686,9 +696,8 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
               for (int u = 0; u < 4; ++u) {
                 const int c = 4 * c4 + u;
                 const uint32_t sv = c < 32 ? s0[c] : s1[c - 32];
-                pe[c] = ((qm >> c) & 1ull)
-                            ? ex2_approx(fmaf(__uint_as_float(sv), a.scale_log2, -lv[u] * 1.4426950408889634f))
-                            : 0.0f;
+                pe[c] = ex2_approx(fmaf(__uint_as_float(sv), a.scale_log2, -lv[u] * 1.4426950408889634f));
+                if (!full && !((qm >> c) & 1ull)) pe[c] = 0.0f;
               }
             }
 #pragma unroll

@@ -38,6 +38,15 @@ struct AttnArgs {
   unsigned int debug;
 };
 
+// bf16 pair of (v0, v1) into hi, and with the remainders (v - bf16(v)) as a second bf16 pair
+// into lo: hi + lo carries v to about 16 bits.
+__device__ __forceinline__ void split_bf16x2(float v0, float v1, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(v0, v1);
+  float r0, r1;
+  upk2(sub2(pk2(v0, v1), pk2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u))), r0, r1);
+  lo = pack_bf16x2(r0, r1);
+}
+
 // Block id t of query block i's list, or -1 when t is past the count or the entry is
 // out of range (the latter is recorded as an index error).
 __device__ __forceinline__ int list_entry(const AttnArgs& a, int bh, int i, int n, int t, bool report) {

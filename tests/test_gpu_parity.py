@@ -266,3 +266,35 @@ def test_fp8_host_checks(cuda_ok):
     cnt = torch.ones(1, 1, 1, dtype=torch.int32, device="cuda")
     with pytest.raises(RuntimeError, match="UNSUPPORTED"):
         sa.forward(z8, z8, zb, idx, cnt, p, sc, sc)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_batch2_odd_heads_router_forward_backward(D):
+    """B = 2 with an odd head count: router lists, forward and backward of every (b, h)
+    against the oracle (the kernels index rows by b * H + h)."""
+    cfg = synth.small_config("b2", 2, 3, D, (6, 9, 10), 3, 0.9)
+    x, p, t = gpu_inputs(cfg)
+    lay = O.cube_layout(cfg.lat)
+    T = lay.n_cubes
+    idx, cnt = sa.plan(t["q"], t["k"], p)
+    trs = {}
+    for b in range(cfg.B):
+        for hh in range(cfg.H):
+            tr = O.route_head(oracle_head(x, "q", b, hh, lay), oracle_head(x, "k", b, hh, lay), lay.valid,
+                              cfg.top_k, cfg.top_p)
+            mis, ties, bad = classify_router_rows(tr, gpu_lists(idx, cnt, b, hh), cfg.top_p)
+            assert mis == 0, f"b{b} h{hh}: rows {bad[:5]}"
+            trs[(b, hh)] = tr.lists
+    idx_o, cnt_o = lists_to_device(trs, cfg.B, cfg.H, T, p.kv_capacity)
+    out, lse, out32 = sa.forward(t["q"], t["k"], t["v"], idx_o, cnt_o, p, with_f32=True)
+    dq, dk, dv = sa.backward(t["q"], t["k"], t["v"], out, lse, t["do"], idx_o, cnt_o, p, out_f32=out32)
+    torch.cuda.synchronize()
+    for b in range(cfg.B):
+        for hh in range(cfg.H):
+            q, k, v, do = (oracle_head(x, n, b, hh, lay) for n in ("q", "k", "v", "do"))
+            o_ref, lse_ref = O.attention_forward_head(q, k, v, trs[(b, hh)], lay.valid)
+            assert_close(f"out b{b}h{hh}", out[b, hh].float().cpu().numpy()[lay.valid], o_ref[lay.valid])
+            assert np.max(np.abs(lse[b, hh].cpu().numpy()[lay.valid] - lse_ref[lay.valid])) < 1e-3
+            g = O.attention_backward_head(q, k, v, do, trs[(b, hh)], lay.valid)
+            for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), g):
+                assert_close(f"{name} b{b}h{hh}", got[b, hh].cpu().numpy(), ref)
