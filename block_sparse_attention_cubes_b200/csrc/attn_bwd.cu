@@ -23,11 +23,13 @@
 namespace sa {
 
 // ------------------------------------------------------------------------ Delta
-// O is read from its fp32 copy when there is one, else from the bf16 output.
+// O is read from its fp32 copy when there is one, else from the bf16 output.  The same pass
+// writes -lse * log2(e) per row, the form in which the dK/dV kernel's exponentials use it.
 __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ o,
                                                     const float* __restrict__ o32,
                                                     const __nv_bfloat16* __restrict__ dout,
-                                                    float* __restrict__ delta, Geom g, int BH, int D) {
+                                                    const float* __restrict__ lse, float* __restrict__ delta,
+                                                    float* __restrict__ nlse2, Geom g, int BH, int D) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = blockIdx.x * 8LL + warp;
   if (row >= static_cast<long long>(BH) * g.Npad) return;
@@ -54,7 +56,10 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restr
   }
 #pragma unroll
   for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) delta[row] = acc;
+  if (lane == 0) {
+    delta[row] = acc;
+    nlse2[row] = -lse[row] * 1.4426950408889634f;
+  }
 }
 
 // ------------------------------------------------------------------------ transposed lists
@@ -506,7 +511,7 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
     if (lane < 2 && !skip_all) {
       const bool qside = lane == 0;  // lane 0: K2, V2, Q2 + lse; lane 1: dO2 + Delta
       const CUtensorMap* tmap = qside ? &tm_q : &tm_do;
-      const float* vec = qside ? a.lse : a.delta;
+      const float* vec = qside ? a.nlse2 : a.delta;
       uint32_t gs = 0;
       int issued_kv = 0;
       bool ok = true;
@@ -696,7 +701,7 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
               for (int u = 0; u < 4; ++u) {
                 const int c = 4 * c4 + u;
                 const uint32_t sv = c < 32 ? s0[c] : s1[c - 32];
-                pe[c] = ex2_approx(fmaf(__uint_as_float(sv), a.scale_log2, -lv[u] * 1.4426950408889634f));
+                pe[c] = ex2_approx(fmaf(__uint_as_float(sv), a.scale_log2, lv[u]));  // lv = -lse log2(e)
                 if (!full && !((qm >> c) & 1ull)) pe[c] = 0.0f;
               }
             }
@@ -809,7 +814,8 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
 // ------------------------------------------------------------------------ launch
 cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const void* out, const float* out_f32, const void* dout,
-                            AttnArgs a, int32_t* qcnt, int32_t* qoff, int32_t* qidx, float* delta, int32_t* uq_list,
+                            AttnArgs a, int32_t* qcnt, int32_t* qoff, int32_t* qidx, float* delta, float* nlse2,
+                            int32_t* uq_list,
                             int32_t* uq_cnt, int32_t* uk_list, int32_t* uk_cnt, cudaStream_t stream, int* launches) {
   static bool attr_set = false;
   if (!attr_set) {
@@ -824,8 +830,8 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   const Geom& g = a.g;
   const long long rows = static_cast<long long>(a.BH) * g.Npad;
   delta_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(out), out_f32, static_cast<const __nv_bfloat16*>(dout), delta, g, a.BH,
-      a.D);
+      static_cast<const __nv_bfloat16*>(out), out_f32, static_cast<const __nv_bfloat16*>(dout), a.lse, delta, nlse2,
+      g, a.BH, a.D);
   cudaError_t e = cudaMemsetAsync(qcnt, 0, sizeof(int32_t) * static_cast<size_t>(a.BH) * g.T, stream);
   if (e != cudaSuccess) return e;
   const long long qrows = static_cast<long long>(a.BH) * g.T;
@@ -839,6 +845,7 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   e = launch_key_pair_union(qoff, qidx, uk_list, uk_cnt, a.BH, g.T, a.cap, stream);
   if (e != cudaSuccess) return e;
   a.delta = delta;
+  a.nlse2 = nlse2;
   a.q_off = qoff;
   a.q_idx = qidx;
   a.u_list = uq_list;

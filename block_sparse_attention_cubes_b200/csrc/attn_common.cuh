@@ -22,6 +22,7 @@ struct AttnArgs {
   int ucap;                 // row stride of u_list: min(2 * cap, T)
   float* lse;               // [BH, Npad]
   const float* delta;       // backward: rowsum(dO * O) [BH, Npad]
+  const float* nlse2;       // backward: -lse * log2(e) [BH, Npad]
   const int32_t* q_off;     // backward: transposed lists, CSR offsets [BH, T+1]
   const int32_t* q_idx;     // backward: transposed lists, entries
   float* dq;

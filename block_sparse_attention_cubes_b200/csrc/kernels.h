@@ -34,7 +34,8 @@ cudaError_t launch_forward(const CUtensorMap& tq, const CUtensorMap& tk, const C
 
 cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const void* out, const float* out_f32, const void* dout,
-                            AttnArgs a, int32_t* qcnt, int32_t* qoff, int32_t* qidx, float* delta, int32_t* uq_list,
+                            AttnArgs a, int32_t* qcnt, int32_t* qoff, int32_t* qidx, float* delta, float* nlse2,
+                            int32_t* uq_list,
                             int32_t* uq_cnt, int32_t* uk_list, int32_t* uk_cnt, cudaStream_t stream, int* launches);
 
 }  // namespace sa
