@@ -61,7 +61,7 @@ struct WsLayout {
   size_t cmask = 0;                                        // forward, backward: [T] cube masks
   size_t ulist = 0, ucnt = 0;                              // forward: query-pair union lists
   size_t qbar = 0, kbar = 0, scores = 0;                   // plan
-  size_t delta = 0, nlse2 = 0, qcnt = 0, qoff = 0, qidx = 0;  // backward
+  size_t delta = 0, nlse2 = 0, bits = 0;                  // backward
   size_t ukcnt = 0, uklist = 0;                            // backward: key-pair unions
   size_t total = 0;
 };
@@ -92,12 +92,8 @@ WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
     off = align256(off + BH * g.Npad * sizeof(float));
     w.nlse2 = off;
     off = align256(off + BH * g.Npad * sizeof(float));
-    w.qcnt = off;
-    off = align256(off + BH * g.T * sizeof(int32_t));
-    w.qoff = off;
-    off = align256(off + BH * (g.T + 1) * sizeof(int32_t));
-    w.qidx = off;
-    off = align256(off + BH * g.T * static_cast<size_t>(p->kv_capacity) * sizeof(int32_t));
+    w.bits = off;  // selection bit matrix [BH, T, ceil(T/32)]
+    off = align256(off + BH * g.T * static_cast<size_t>((g.T + 31) / 32) * sizeof(uint32_t));
     const size_t P = static_cast<size_t>((g.T + 1) / 2);
     w.ucnt = off;
     off = align256(off + BH * P * sizeof(int32_t));
@@ -328,8 +324,7 @@ sa_status sa_backward(const void* q, const void* k, const void* v, const void* o
     return SA_ERR_LAUNCH;
   int launches = 0;
   a.ucap = union_cap(p, g);
-  if (sa::launch_backward(tq, tk, tv, tdo, out, out_f32, dout, a, reinterpret_cast<int32_t*>(wb + w.qcnt),
-                          reinterpret_cast<int32_t*>(wb + w.qoff), reinterpret_cast<int32_t*>(wb + w.qidx),
+  if (sa::launch_backward(tq, tk, tv, tdo, out, out_f32, dout, a, reinterpret_cast<uint32_t*>(wb + w.bits),
                           reinterpret_cast<float*>(wb + w.delta), reinterpret_cast<float*>(wb + w.nlse2),
                           reinterpret_cast<int32_t*>(wb + w.ulist),
                           reinterpret_cast<int32_t*>(wb + w.ucnt), reinterpret_cast<int32_t*>(wb + w.uklist),

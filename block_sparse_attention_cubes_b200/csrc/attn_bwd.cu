@@ -6,11 +6,10 @@
 //     dQ = scale * dS K,  dK = scale * dS^T Q.
 //
 // Kernels:
-//   delta_kernel      Delta per query row (one warp per row).
-//   count/scan/fill   the transposed lists: for each key cube j the ascending query cubes
-//                     whose list holds j (CSR, deterministic).
-//   pair unions       (pairs.cu) query-cube pairs over their KV lists, key-cube pairs over
-//                     their transposed lists.
+//   delta_kernel      Delta and -lse * log2(e) per query row (one warp per row).
+//   pair unions       (pairs.cu) query-cube pairs over their KV lists; key-cube pairs over
+//                     the transposed selection, read from a bit matrix that the lists are
+//                     scattered into with atomicOr (deterministic, ascending query cubes).
 //   attn_dq_kernel    row form over query-cube pairs (M = 128 rows, N = 128 keys).
 //   attn_dkdv_kernel  transposed form over key-cube pairs (M = 128 keys, N = 128 queries).
 // All products are full-rate 128 x 128 tcgen05 MMAs with accumulators in TMEM; P and dS
@@ -59,78 +58,6 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restr
   if (lane == 0) {
     delta[row] = acc;
     nlse2[row] = -lse[row] * 1.4426950408889634f;
-  }
-}
-
-// ------------------------------------------------------------------------ transposed lists
-__global__ void count_kernel(const int32_t* __restrict__ kv_index, const int32_t* __restrict__ kv_count,
-                             int32_t* __restrict__ qcnt, int BH, int T, int cap) {
-  const long long row = blockIdx.x * (long long)blockDim.y + threadIdx.y;  // (bh, i)
-  if (row >= static_cast<long long>(BH) * T) return;
-  const int bh = static_cast<int>(row / T);
-  int n = kv_count[row];
-  n = n < 0 ? 0 : (n > cap ? cap : n);
-  for (int t = threadIdx.x; t < n; t += blockDim.x) {
-    const int j = kv_index[row * cap + t];
-    if (j >= 0 && j < T) atomicAdd(&qcnt[static_cast<size_t>(bh) * T + j], 1);
-  }
-}
-
-// exclusive scan of qcnt[bh][0..T) into qoff[bh][0..T], one CTA per bh
-__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ qcnt, int32_t* __restrict__ qoff,
-                                                    int T, int cap) {
-  __shared__ int32_t part[1024];
-  const int bh = blockIdx.x;
-  const int per = (T + 1023) / 1024;
-  const int beg = threadIdx.x * per;
-  int s = 0;
-  for (int j = beg; j < beg + per && j < T; ++j) s += qcnt[static_cast<size_t>(bh) * T + j];
-  part[threadIdx.x] = s;
-  __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {
-    const int v = threadIdx.x >= off ? part[threadIdx.x - off] : 0;
-    __syncthreads();
-    part[threadIdx.x] += v;
-    __syncthreads();
-  }
-  // entries of head bh start at bh * T * cap (an upper bound of its total)
-  int run = static_cast<int>(static_cast<size_t>(bh) * T * cap) + (threadIdx.x ? part[threadIdx.x - 1] : 0);
-  for (int j = beg; j < beg + per && j < T; ++j) {
-    qoff[static_cast<size_t>(bh) * (T + 1) + j] = run;
-    run += qcnt[static_cast<size_t>(bh) * T + j];
-  }
-  if (threadIdx.x == 1023) qoff[static_cast<size_t>(bh) * (T + 1) + T] = run;
-}
-
-// One warp per (bh, key cube j): visit query cubes in ascending order and binary-search j in
-// each ascending list; append hits in order.
-__global__ void __launch_bounds__(256) fill_kernel(const int32_t* __restrict__ kv_index,
-                                                   const int32_t* __restrict__ kv_count,
-                                                   const int32_t* __restrict__ qoff, int32_t* __restrict__ qidx,
-                                                   int BH, int T, int cap) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long col = blockIdx.x * 8LL + warp;
-  if (col >= static_cast<long long>(BH) * T) return;
-  const int bh = static_cast<int>(col / T), j = static_cast<int>(col % T);
-  int pos = qoff[static_cast<size_t>(bh) * (T + 1) + j];
-  for (int i0 = 0; i0 < T; i0 += 32) {
-    const int i = i0 + lane;
-    bool hit = false;
-    if (i < T) {
-      const size_t r = static_cast<size_t>(bh) * T + i;
-      int n = kv_count[r];
-      n = n < 0 ? 0 : (n > cap ? cap : n);
-      const int32_t* lst = kv_index + r * cap;
-      int lo = 0, hi = n;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (lst[mid] < j) lo = mid + 1; else hi = mid;
-      }
-      hit = lo < n && lst[lo] == j;
-    }
-    const uint32_t bal = __ballot_sync(0xffffffffu, hit);
-    if (hit) qidx[pos + __popc(bal & ((1u << lane) - 1u))] = i;
-    pos += __popc(bal);
   }
 }
 
@@ -814,7 +741,7 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
 // ------------------------------------------------------------------------ launch
 cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const void* out, const float* out_f32, const void* dout,
-                            AttnArgs a, int32_t* qcnt, int32_t* qoff, int32_t* qidx, float* delta, float* nlse2,
+                            AttnArgs a, uint32_t* bits, float* delta, float* nlse2,
                             int32_t* uq_list,
                             int32_t* uq_cnt, int32_t* uk_list, int32_t* uk_cnt, cudaStream_t stream, int* launches) {
   static bool attr_set = false;
@@ -832,22 +759,12 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   delta_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(out), out_f32, static_cast<const __nv_bfloat16*>(dout), a.lse, delta, nlse2,
       g, a.BH, a.D);
-  cudaError_t e = cudaMemsetAsync(qcnt, 0, sizeof(int32_t) * static_cast<size_t>(a.BH) * g.T, stream);
+  cudaError_t e = launch_query_pair_union(a.kv_index, a.kv_count, uq_list, uq_cnt, a.BH, g.T, a.cap, a.st, stream);
   if (e != cudaSuccess) return e;
-  const long long qrows = static_cast<long long>(a.BH) * g.T;
-  count_kernel<<<static_cast<unsigned>((qrows + 7) / 8), dim3(32, 8), 0, stream>>>(a.kv_index, a.kv_count, qcnt,
-                                                                                    a.BH, g.T, a.cap);
-  scan_kernel<<<a.BH, 1024, 0, stream>>>(qcnt, qoff, g.T, a.cap);
-  fill_kernel<<<static_cast<unsigned>((qrows + 7) / 8), 256, 0, stream>>>(a.kv_index, a.kv_count, qoff, qidx, a.BH,
-                                                                          g.T, a.cap);
-  e = launch_query_pair_union(a.kv_index, a.kv_count, uq_list, uq_cnt, a.BH, g.T, a.cap, a.st, stream);
-  if (e != cudaSuccess) return e;
-  e = launch_key_pair_union(qoff, qidx, uk_list, uk_cnt, a.BH, g.T, a.cap, stream);
+  e = launch_key_pair_union(a.kv_index, a.kv_count, bits, uk_list, uk_cnt, a.BH, g.T, a.cap, a.st, stream);
   if (e != cudaSuccess) return e;
   a.delta = delta;
   a.nlse2 = nlse2;
-  a.q_off = qoff;
-  a.q_idx = qidx;
   a.u_list = uq_list;
   a.u_cnt = uq_cnt;
   a.uk_list = uk_list;
@@ -862,7 +779,7 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
     attn_dq_kernel<8><<<grid, dqk::kThreads, dqk::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
     attn_dkdv_kernel<8><<<grid, dkv::kThreads, dkv::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
   }
-  *launches = 8;
+  *launches = 6;
   return cudaGetLastError();
 }
 

@@ -23,8 +23,6 @@ struct AttnArgs {
   float* lse;               // [BH, Npad]
   const float* delta;       // backward: rowsum(dO * O) [BH, Npad]
   const float* nlse2;       // backward: -lse * log2(e) [BH, Npad]
-  const int32_t* q_off;     // backward: transposed lists, CSR offsets [BH, T+1]
-  const int32_t* q_idx;     // backward: transposed lists, entries
   float* dq;
   float* dk;
   float* dv;

@@ -23,8 +23,9 @@ cudaError_t launch_plan(const void* q, const void* k, const float* q_scale, cons
 
 cudaError_t launch_query_pair_union(const int32_t* kv_index, const int32_t* kv_count, int32_t* u_list,
                                     int32_t* u_cnt, int BH, int T, int cap, DevStatus* st, cudaStream_t stream);
-cudaError_t launch_key_pair_union(const int32_t* q_off, const int32_t* q_idx, int32_t* u_list, int32_t* u_cnt,
-                                  int BH, int T, int cap, cudaStream_t stream);
+// Key-cube pair unions of the transposed selection, through a [BH, T, ceil(T/32)] bit matrix.
+cudaError_t launch_key_pair_union(const int32_t* kv_index, const int32_t* kv_count, uint32_t* bits, int32_t* u_list,
+                                  int32_t* u_cnt, int BH, int T, int cap, DevStatus* st, cudaStream_t stream);
 
 cudaError_t launch_cube_mask(const Geom& g, unsigned long long* mask, cudaStream_t stream);
 int num_sms();
@@ -34,7 +35,7 @@ cudaError_t launch_forward(const CUtensorMap& tq, const CUtensorMap& tk, const C
 
 cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const void* out, const float* out_f32, const void* dout,
-                            AttnArgs a, int32_t* qcnt, int32_t* qoff, int32_t* qidx, float* delta, float* nlse2,
+                            AttnArgs a, uint32_t* bits, float* delta, float* nlse2,
                             int32_t* uq_list,
                             int32_t* uq_cnt, int32_t* uk_list, int32_t* uk_cnt, cudaStream_t stream, int* launches);
 

@@ -13,27 +13,6 @@
 
 namespace sa {
 
-// One thread per pair: merge two ascending lists of length n0, n1 (second may be absent).
-__device__ __forceinline__ int merge_two(const int32_t* a, int n0, const int32_t* b, int n1, int32_t* out) {
-  int x = 0, y = 0, k = 0;
-  while (x < n0 || y < n1) {
-    const int va = x < n0 ? a[x] : 0x7fffffff;
-    const int vb = y < n1 ? b[y] : 0x7fffffff;
-    if (va == vb) {
-      out[k++] = (va << 2) | 3;
-      ++x;
-      ++y;
-    } else if (va < vb) {
-      out[k++] = (va << 2) | 1;
-      ++x;
-    } else {
-      out[k++] = (vb << 2) | 2;
-      ++y;
-    }
-  }
-  return k;
-}
-
 // Query-cube pairs: union of kv_index rows 2p and 2p+1 of each (b, h).
 // u_list: [BH, P, ucap] with ucap = min(2*cap, T), u_cnt: [BH, P], P = ceil(T/2).  Entries outside [0, T) or
 // counts outside [0, cap] are dropped (and reported as index errors).
@@ -95,24 +74,69 @@ __global__ void query_pair_union_kernel(const int32_t* __restrict__ kv_index, co
   u_cnt[id] = k;
 }
 
-// Key-cube pairs: union of the transposed lists (CSR q_off/q_idx) of cubes 2p and 2p+1
-// (row stride T: a union of query cubes has at most T entries).
-__global__ void key_pair_union_kernel(const int32_t* __restrict__ q_off, const int32_t* __restrict__ q_idx,
-                                      int32_t* __restrict__ u_list, int32_t* __restrict__ u_cnt, int BH, int T,
-                                      int cap) {
+// ---------------------------------------------------------------- key-cube pairs
+// The selection as a bit matrix: bit i of bits[bh][j] (words of 32 query cubes) is set when
+// query cube i selected key cube j.  atomicOr makes the result independent of the order of
+// the writes.  One warp per query row (bh, i).
+__global__ void selection_bits_kernel(const int32_t* __restrict__ kv_index, const int32_t* __restrict__ kv_count,
+                                      uint32_t* __restrict__ bits, int BH, int T, int cap, int W, DevStatus* st) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = blockIdx.x * 8LL + warp;
+  if (row >= static_cast<long long>(BH) * T) return;
+  const int bh = static_cast<int>(row / T), i = static_cast<int>(row % T);
+  int n = kv_count[row];
+  if (n < 0 || n > cap) {
+    if (lane == 0) flag_error(st, DEVERR_INDEX, 0);
+    n = n < 0 ? 0 : cap;
+  }
+  const int32_t* lst = kv_index + row * cap;
+  uint32_t* col0 = bits + static_cast<size_t>(bh) * T * W;
+  for (int t = lane; t < n; t += 32) {
+    const int j = lst[t];
+    if (j < 0 || j >= T) {
+      flag_error(st, DEVERR_INDEX, 0);
+      continue;
+    }
+    atomicOr(col0 + static_cast<size_t>(j) * W + (i >> 5), 1u << (i & 31));
+  }
+}
+
+// Key-cube pairs: union of the query cubes that selected key cube 2p or 2p+1, ascending, as
+// entries (query cube << 2) | (1 if it selected 2p) | (2 if it selected 2p+1); row stride T.
+// One warp per pair: lane w takes words w, w+32, ...; a warp prefix sum places each word's
+// entries.
+__global__ void key_pair_union_kernel(const uint32_t* __restrict__ bits, int32_t* __restrict__ u_list,
+                                      int32_t* __restrict__ u_cnt, int BH, int T, int W) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int P = (T + 1) >> 1;
-  const long long id = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const long long id = blockIdx.x * 8LL + warp;
   if (id >= static_cast<long long>(BH) * P) return;
   const int bh = static_cast<int>(id / P), p = static_cast<int>(id % P);
-  const int j0 = 2 * p, j1 = 2 * p + 1;
-  const int32_t* off = q_off + static_cast<size_t>(bh) * (T + 1);
-  const int b0 = off[j0], n0 = off[j0 + 1] - b0;
-  int b1 = 0, n1 = 0;
-  if (j1 < T) {
-    b1 = off[j1];
-    n1 = off[j1 + 1] - b1;
+  const uint32_t* c0 = bits + (static_cast<size_t>(bh) * T + 2 * p) * W;
+  const uint32_t* c1 = (2 * p + 1 < T) ? c0 + W : nullptr;
+  int32_t* out = u_list + id * static_cast<long long>(T);
+  int base = 0;
+  for (int w0 = 0; w0 < W; w0 += 32) {
+    const int w = w0 + lane;
+    const uint32_t a = w < W ? c0[w] : 0u;
+    const uint32_t b = (w < W && c1) ? c1[w] : 0u;
+    uint32_t u = a | b;
+    const int cnt = __popc(u);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int k = base + incl - cnt;
+    while (u) {
+      const int bit = __ffs(u) - 1;
+      u &= u - 1u;
+      out[k++] = ((w * 32 + bit) << 2) | static_cast<int>((a >> bit) & 1u) | (static_cast<int>((b >> bit) & 1u) << 1);
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
   }
-  u_cnt[id] = merge_two(q_idx + b0, n0, q_idx + b1, n1, u_list + id * static_cast<long long>(T));
+  if (lane == 0) u_cnt[id] = base;
 }
 
 cudaError_t launch_query_pair_union(const int32_t* kv_index, const int32_t* kv_count, int32_t* u_list,
@@ -124,11 +148,16 @@ cudaError_t launch_query_pair_union(const int32_t* kv_index, const int32_t* kv_c
   return cudaGetLastError();
 }
 
-cudaError_t launch_key_pair_union(const int32_t* q_off, const int32_t* q_idx, int32_t* u_list, int32_t* u_cnt,
-                                  int BH, int T, int cap, cudaStream_t stream) {
-  const long long n = static_cast<long long>(BH) * ((T + 1) >> 1);
-  key_pair_union_kernel<<<static_cast<unsigned>((n + 127) / 128), 128, 0, stream>>>(q_off, q_idx, u_list, u_cnt, BH,
-                                                                                     T, cap);
+cudaError_t launch_key_pair_union(const int32_t* kv_index, const int32_t* kv_count, uint32_t* bits, int32_t* u_list,
+                                  int32_t* u_cnt, int BH, int T, int cap, DevStatus* st, cudaStream_t stream) {
+  const int W = (T + 31) / 32;
+  cudaError_t e = cudaMemsetAsync(bits, 0, sizeof(uint32_t) * static_cast<size_t>(BH) * T * W, stream);
+  if (e != cudaSuccess) return e;
+  const long long rows = static_cast<long long>(BH) * T;
+  selection_bits_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(kv_index, kv_count, bits, BH, T,
+                                                                                   cap, W, st);
+  const long long pairs = static_cast<long long>(BH) * ((T + 1) >> 1);
+  key_pair_union_kernel<<<static_cast<unsigned>((pairs + 7) / 8), 256, 0, stream>>>(bits, u_list, u_cnt, BH, T, W);
   return cudaGetLastError();
 }
 

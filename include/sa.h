@@ -86,8 +86,8 @@ SA_API int sa_topk_from_fraction(double frac, int T);
  * Plan: status block + pooled Q and K (fp64) + block scores (fp64, B*H*T*T).
  * Forward: status block + one 64-bit valid-slot mask per cube (T) + the union lists of
  * adjacent query-cube pairs (int32, B*H*ceil(T/2)*(1 + 2*kv_capacity)).  Backward: status block
- * + cube masks + Delta (fp32, B*H*Npad) + the transposed index lists (int32,
- * B*H*(2T+1) + B*H*T*kv_capacity) + the query-pair and key-pair union lists (int32,
+ * + cube masks + Delta and -lse*log2(e) (fp32, 2*B*H*Npad) + the selection as a bit matrix
+ * (B*H*T*ceil(T/32) words) + the query-pair and key-pair union lists (int32,
  * B*H*ceil(T/2)*(2 + min(2*kv_capacity, T) + T)). */
 SA_API size_t sa_workspace_size(const sa_params* p, int op);
 
