@@ -15,63 +15,69 @@ namespace sa {
 
 // Query-cube pairs: union of kv_index rows 2p and 2p+1 of each (b, h).
 // u_list: [BH, P, ucap] with ucap = min(2*cap, T), u_cnt: [BH, P], P = ceil(T/2).  Entries outside [0, T) or
-// counts outside [0, cap] are dropped (and reported as index errors).
-__global__ void query_pair_union_kernel(const int32_t* __restrict__ kv_index, const int32_t* __restrict__ kv_count,
-                                        int32_t* __restrict__ u_list, int32_t* __restrict__ u_cnt, int BH, int T,
-                                        int cap, int ucap, DevStatus* st) {
-  const int P = (T + 1) >> 1;
-  const long long id = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+// counts outside [0, cap] are dropped (and reported as index errors).  One warp per pair: both
+// lists are scattered into two bit rows in shared memory (order-independent), then read out in
+// ascending block order with a warp prefix sum placing each word's entries.
+constexpr int QPU_WARPS = 8;
+__global__ void __launch_bounds__(QPU_WARPS * 32)
+    query_pair_union_kernel(const int32_t* __restrict__ kv_index, const int32_t* __restrict__ kv_count,
+                            int32_t* __restrict__ u_list, int32_t* __restrict__ u_cnt, int BH, int T, int cap,
+                            int ucap, DevStatus* st) {
+  extern __shared__ uint32_t qpu_bits[];  // [QPU_WARPS][2][W]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int P = (T + 1) >> 1, W = (T + 31) >> 5;
+  const long long id = blockIdx.x * static_cast<long long>(QPU_WARPS) + warp;
   if (id >= static_cast<long long>(BH) * P) return;
   const int bh = static_cast<int>(id / P), p = static_cast<int>(id % P);
-  const int i0 = 2 * p, i1 = 2 * p + 1;
-  int n[2] = {0, 0};
-  const int32_t* src[2] = {nullptr, nullptr};
+  uint32_t* ba = qpu_bits + static_cast<size_t>(warp) * 2 * W;
+  uint32_t* bb = ba + W;
+  for (int w = lane; w < 2 * W; w += 32) ba[w] = 0u;
+  __syncwarp();
   for (int u = 0; u < 2; ++u) {
-    const int i = u ? i1 : i0;
+    const int i = 2 * p + u;
     if (i >= T) continue;
     const size_t r = static_cast<size_t>(bh) * T + i;
     int c = kv_count[r];
     if (c < 0 || c > cap) {
-      flag_error(st, DEVERR_INDEX, 0);
+      if (lane == 0) flag_error(st, DEVERR_INDEX, 0);
       c = c < 0 ? 0 : cap;
     }
-    n[u] = c;
-    src[u] = kv_index + r * cap;
+    const int32_t* src = kv_index + r * cap;
+    uint32_t* dst = u ? bb : ba;
+    for (int t = lane; t < c; t += 32) {
+      const int j = src[t];
+      if (j < 0 || j >= T) {
+        flag_error(st, DEVERR_INDEX, 0);
+        continue;
+      }
+      atomicOr(dst + (j >> 5), 1u << (j & 31));
+    }
   }
+  __syncwarp();
   int32_t* out = u_list + id * static_cast<long long>(ucap);
-  // drop out-of-range entries while merging: copy valid prefixes through local filtering
-  int x = 0, y = 0, k = 0;
-  while (x < n[0] || y < n[1]) {
-    int va = 0x7fffffff, vb = 0x7fffffff;
-    if (x < n[0]) {
-      va = src[0][x];
-      if (va < 0 || va >= T) {
-        flag_error(st, DEVERR_INDEX, 0);
-        ++x;
-        continue;
-      }
+  int base = 0;
+  for (int w0 = 0; w0 < W; w0 += 32) {
+    const int w = w0 + lane;
+    const uint32_t a = w < W ? ba[w] : 0u, b = w < W ? bb[w] : 0u;
+    uint32_t u = a | b;
+    const int cnt = __popc(u);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
     }
-    if (y < n[1]) {
-      vb = src[1][y];
-      if (vb < 0 || vb >= T) {
-        flag_error(st, DEVERR_INDEX, 0);
-        ++y;
-        continue;
-      }
+    int k = base + incl - cnt;
+    while (u) {
+      const int bit = __ffs(u) - 1;
+      u &= u - 1u;
+      if (k < ucap)
+        out[k] = ((w * 32 + bit) << 2) | static_cast<int>((a >> bit) & 1u) | (static_cast<int>((b >> bit) & 1u) << 1);
+      ++k;
     }
-    if (va == vb) {
-      out[k++] = (va << 2) | 3;
-      ++x;
-      ++y;
-    } else if (va < vb) {
-      out[k++] = (va << 2) | 1;
-      ++x;
-    } else {
-      out[k++] = (vb << 2) | 2;
-      ++y;
-    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
   }
-  u_cnt[id] = k;
+  if (lane == 0) u_cnt[id] = base < ucap ? base : ucap;
 }
 
 // ---------------------------------------------------------------- key-cube pairs
@@ -143,8 +149,9 @@ cudaError_t launch_query_pair_union(const int32_t* kv_index, const int32_t* kv_c
                                     int32_t* u_cnt, int BH, int T, int cap, DevStatus* st, cudaStream_t stream) {
   const long long n = static_cast<long long>(BH) * ((T + 1) >> 1);
   const int ucap = 2 * cap < T ? 2 * cap : T;
-  query_pair_union_kernel<<<static_cast<unsigned>((n + 127) / 128), 128, 0, stream>>>(kv_index, kv_count, u_list,
-                                                                                       u_cnt, BH, T, cap, ucap, st);
+  const size_t smem = sizeof(uint32_t) * QPU_WARPS * 2 * ((T + 31) / 32);  // 16 KB at T = 8192
+  query_pair_union_kernel<<<static_cast<unsigned>((n + QPU_WARPS - 1) / QPU_WARPS), QPU_WARPS * 32, smem, stream>>>(
+      kv_index, kv_count, u_list, u_cnt, BH, T, cap, ucap, st);
   return cudaGetLastError();
 }
 

@@ -59,19 +59,30 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint8_t* __restrict__ q
     cube_extent(g, c, vt, vh, vw);
     const size_t row_bytes = static_cast<size_t>(D) * ESZ;
     const uint8_t* base = src + (static_cast<size_t>(bh) * g.Npad + static_cast<size_t>(c) * 64) * row_bytes;
-    for (int r = roff; r < 64; r += rows_per_iter) {
-      if (!slot_valid(vt, vh, vw, r)) continue;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + r * row_bytes) + chunk);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    // four rows' loads in flight per thread before any of them is accumulated
+    for (int r0 = roff; r0 < 64; r0 += 4 * rows_per_iter) {
+      uint4 v[4];
+      bool ok[4];
 #pragma unroll
-      for (int e = 0; e < EPT; ++e) {
-        float f;
-        if constexpr (ESZ == 2) {
-          f = __uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
-        } else {
-          f = e4m3_value((w[e >> 2] >> (8 * (e & 3))) & 0xffu);
+      for (int u = 0; u < 4; ++u) {
+        const int r = r0 + u * rows_per_iter;
+        ok[u] = r < 64 && slot_valid(vt, vh, vw, r);
+        v[u] = ok[u] ? __ldg(reinterpret_cast<const uint4*>(base + r * row_bytes) + chunk) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (!ok[u]) continue;
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+          float f;
+          if constexpr (ESZ == 2) {
+            f = __uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
+          } else {
+            f = e4m3_value((w[e >> 2] >> (8 * (e & 3))) & 0xffu);
+          }
+          acc[e] += static_cast<double>(f);
         }
-        acc[e] += static_cast<double>(f);
       }
     }
   }
