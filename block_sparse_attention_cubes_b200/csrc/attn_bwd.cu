@@ -24,40 +24,63 @@ namespace sa {
 // ------------------------------------------------------------------------ Delta
 // O is read from its fp32 copy when there is one, else from the bf16 output.  The same pass
 // writes -lse * log2(e) per row, the form in which the dK/dV kernel's exponentials use it.
+// One warp per 4 consecutive rows, all loads issued before any arithmetic (padding rows are
+// read too and zeroed afterwards), so each warp keeps 4 rows of O and dO in flight.
+constexpr int DELTA_ROWS = 4;
 __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ o,
                                                     const float* __restrict__ o32,
                                                     const __nv_bfloat16* __restrict__ dout,
                                                     const float* __restrict__ lse, float* __restrict__ delta,
                                                     float* __restrict__ nlse2, Geom g, int BH, int D) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row = blockIdx.x * 8LL + warp;
-  if (row >= static_cast<long long>(BH) * g.Npad) return;
-  const int p = static_cast<int>(row % g.Npad);
-  float acc = 0.0f;
-  if (token_valid(g, p >> 6, p & 63)) {
-    const uint2* b = reinterpret_cast<const uint2*>(dout + row * D);
-    for (int c = lane; c < D / 4; c += 32) {
-      const uint2 y = b[c];
-      float ov[4];
+  const long long rows = static_cast<long long>(BH) * g.Npad;
+  const long long row0 = (blockIdx.x * 8LL + warp) * DELTA_ROWS;
+  if (row0 >= rows) return;
+  // D is 64 or 128: lane c holds elements 4c..4c+3 of a row (lanes >= D/4 idle)
+  const int c = lane;
+  const bool on = c < D / 4;
+  uint2 y[DELTA_ROWS];
+  float4 x[DELTA_ROWS];
+#pragma unroll
+  for (int u = 0; u < DELTA_ROWS; ++u) {
+    const long long row = row0 + u;
+    y[u] = make_uint2(0u, 0u);
+    x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (on && row < rows) {
+      y[u] = reinterpret_cast<const uint2*>(dout + row * D)[c];
       if (o32) {
-        const float4 x = reinterpret_cast<const float4*>(o32 + row * D)[c];
-        ov[0] = x.x; ov[1] = x.y; ov[2] = x.z; ov[3] = x.w;
+        x[u] = reinterpret_cast<const float4*>(o32 + row * D)[c];
       } else {
-        const uint2 x = reinterpret_cast<const uint2*>(o + row * D)[c];
-        ov[0] = __uint_as_float(x.x << 16); ov[1] = __uint_as_float(x.x & 0xffff0000u);
-        ov[2] = __uint_as_float(x.y << 16); ov[3] = __uint_as_float(x.y & 0xffff0000u);
+        const uint2 b = reinterpret_cast<const uint2*>(o + row * D)[c];
+        x[u] = make_float4(__uint_as_float(b.x << 16), __uint_as_float(b.x & 0xffff0000u),
+                           __uint_as_float(b.y << 16), __uint_as_float(b.y & 0xffff0000u));
       }
-      acc += ov[0] * __uint_as_float(y.x << 16);
-      acc += ov[1] * __uint_as_float(y.x & 0xffff0000u);
-      acc += ov[2] * __uint_as_float(y.y << 16);
-      acc += ov[3] * __uint_as_float(y.y & 0xffff0000u);
     }
   }
+  float acc[DELTA_ROWS];
 #pragma unroll
-  for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) {
-    delta[row] = acc;
-    nlse2[row] = -lse[row] * 1.4426950408889634f;
+  for (int u = 0; u < DELTA_ROWS; ++u) {
+    acc[u] = x[u].x * __uint_as_float(y[u].x << 16);
+    acc[u] += x[u].y * __uint_as_float(y[u].x & 0xffff0000u);
+    acc[u] += x[u].z * __uint_as_float(y[u].y << 16);
+    acc[u] += x[u].w * __uint_as_float(y[u].y & 0xffff0000u);
+  }
+#pragma unroll
+  for (int u = 0; u < DELTA_ROWS; ++u) {
+#pragma unroll
+    for (int off = 16; off; off >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], off);
+  }
+  if (lane < DELTA_ROWS) {
+    float a = acc[0];
+#pragma unroll
+    for (int u = 1; u < DELTA_ROWS; ++u)
+      if (lane == u) a = acc[u];
+    const long long row = row0 + lane;
+    if (row < rows) {
+      const int p = static_cast<int>(row % g.Npad);
+      delta[row] = token_valid(g, p >> 6, p & 63) ? a : 0.0f;
+      nlse2[row] = -lse[row] * 1.4426950408889634f;
+    }
   }
 }
 
@@ -756,7 +779,7 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   }
   const Geom& g = a.g;
   const long long rows = static_cast<long long>(a.BH) * g.Npad;
-  delta_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+  delta_kernel<<<static_cast<unsigned>((rows + 8 * DELTA_ROWS - 1) / (8 * DELTA_ROWS)), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(out), out_f32, static_cast<const __nv_bfloat16*>(dout), a.lse, delta, nlse2,
       g, a.BH, a.D);
   cudaError_t e = launch_query_pair_union(a.kv_index, a.kv_count, uq_list, uq_cnt, a.BH, g.T, a.cap, a.st, stream);
