@@ -215,34 +215,46 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
       // Keys of one binade share their top bytes, so in the first passes most lanes of a warp
       // fall in the same bucket: then the warp adds its count and (exact, fixed-point) mass
       // once instead of 32 colliding shared-memory atomics.
-      for (int j0 = 0; j0 < T; j0 += 32) {
-        const int j = j0 + lane;
-        bool part = false;
-        int d = 0;
-        unsigned long long mj = 0ull;
-        if (j < T) {
-          const double x = s[j];
-          const uint64_t kj = desc_key(x);
-          if (shift == 56 || (kj >> (shift + 8)) == (prefix >> (shift + 8))) {
-            part = true;
-            d = static_cast<int>((kj >> shift) & 255u);
-            mj = static_cast<unsigned long long>(mass_fx(x, m));
-          }
-        }
-        const uint32_t act = __ballot_sync(0xffffffffu, part);
-        if (act == 0u) continue;
-        const int dl = __shfl_sync(0xffffffffu, d, __ffs(act) - 1);
-        if (__all_sync(0xffffffffu, !part || d == dl)) {
-          unsigned long long ms = mj;
+      // The chunks of 32 scores carry warp collectives, so the loads of four chunks are issued
+      // before any of them is processed (otherwise every chunk waits out a full L2 round trip).
+      for (int j0 = 0; j0 < T; j0 += 128) {
+        double xs[4];
 #pragma unroll
-          for (int o = 16; o; o >>= 1) ms += __shfl_xor_sync(0xffffffffu, ms, o);
-          if (lane == 0) {
-            atomicAdd(&cnt[dl], static_cast<uint32_t>(__popc(act)));
-            atomicAdd(&mass[dl], ms);
+        for (int u = 0; u < 4; ++u) {
+          const int j = j0 + 32 * u + lane;
+          xs[u] = j < T ? s[j] : 0.0;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (j0 + 32 * u >= T) break;
+          const int j = j0 + 32 * u + lane;
+          bool part = false;
+          int d = 0;
+          unsigned long long mj = 0ull;
+          if (j < T) {
+            const double x = xs[u];
+            const uint64_t kj = desc_key(x);
+            if (shift == 56 || (kj >> (shift + 8)) == (prefix >> (shift + 8))) {
+              part = true;
+              d = static_cast<int>((kj >> shift) & 255u);
+              mj = static_cast<unsigned long long>(mass_fx(x, m));
+            }
           }
-        } else if (part) {
-          atomicAdd(&cnt[d], 1u);
-          atomicAdd(&mass[d], mj);
+          const uint32_t act = __ballot_sync(0xffffffffu, part);
+          if (act == 0u) continue;
+          const int dl = __shfl_sync(0xffffffffu, d, __ffs(act) - 1);
+          if (__all_sync(0xffffffffu, !part || d == dl)) {
+            unsigned long long ms = mj;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) ms += __shfl_xor_sync(0xffffffffu, ms, o);
+            if (lane == 0) {
+              atomicAdd(&cnt[dl], static_cast<uint32_t>(__popc(act)));
+              atomicAdd(&mass[dl], ms);
+            }
+          } else if (part) {
+            atomicAdd(&cnt[d], 1u);
+            atomicAdd(&mass[d], mj);
+          }
         }
       }
       __syncwarp();
@@ -341,17 +353,26 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   // emit the kept ids in ascending order
   int n = 0;
   int32_t* out = kv_index + static_cast<size_t>(row) * cap;
-  for (int j0 = 0; j0 < T; j0 += 32) {
-    const int j = j0 + lane;
-    bool sel = false;
-    if (j < T) {
-      const uint64_t kj = desc_key(s[j]);
-      sel = kj < kb || (kj == kb && j <= jb);
+  for (int j0 = 0; j0 < T; j0 += 128) {
+    double xs[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + 32 * u + lane;
+      xs[u] = j < T ? s[j] : 0.0;
     }
-    const uint32_t bal = __ballot_sync(0xffffffffu, sel);
-    const int pos = n + __popc(bal & ((1u << lane) - 1u));
-    if (sel && pos < cap) out[pos] = j;
-    n += __popc(bal);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + 32 * u + lane;
+      bool sel = false;
+      if (j < T) {
+        const uint64_t kj = desc_key(xs[u]);
+        sel = kj < kb || (kj == kb && j <= jb);
+      }
+      const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+      const int pos = n + __popc(bal & ((1u << lane) - 1u));
+      if (sel && pos < cap) out[pos] = j;
+      n += __popc(bal);
+    }
   }
   if (lane == 0) {
     if (n > cap) flag_error(st, DEVERR_CAPACITY, 0);
