@@ -195,6 +195,7 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   unsigned long long* mass = mass_s[warp];
 
   double m = -DBL_MAX;
+#pragma unroll 4
   for (int j = lane; j < T; j += 32) m = fmax(m, s[j]);
 #pragma unroll
   for (int o = 16; o; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -310,40 +311,51 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
         uint64_t c_acc = cnt_above, m_acc = mass_above;
         const uint64_t mask = (shift == 0) ? ~0ull : ~((1ull << shift) - 1ull);
         bool done = false;
-        for (int j0 = 0; j0 < T && !done; j0 += 32) {
-          const int j = j0 + lane;
-          uint64_t kj = 0, mj = 0;
-          bool cand = false;
-          if (j < T) {
-            const double x = s[j];
-            kj = desc_key(x);
-            cand = (kj & mask) == prefix;
-            if (cand) mj = mass_fx(x, m);
-          }
-          // candidates share one key when shift == 0; a single candidate otherwise
-          const uint32_t cb = __ballot_sync(0xffffffffu, cand);
-          unsigned long long pm = cand ? mj : 0ull;
-          uint32_t pc = cand ? 1u : 0u;
+        for (int j1 = 0; j1 < T && !done; j1 += 128) {
+          double xs[4];
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const unsigned long long t1 = __shfl_up_sync(0xffffffffu, pm, o);
-            const uint32_t t2 = __shfl_up_sync(0xffffffffu, pc, o);
-            if (lane >= o) {
-              pm += t1;
-              pc += t2;
-            }
+          for (int u = 0; u < 4; ++u) {
+            const int j = j1 + 32 * u + lane;
+            xs[u] = j < T ? s[j] : 0.0;
           }
-          const bool ok = cand && (c_acc + pc >= static_cast<uint64_t>(nk)) &&
-                          (static_cast<double>(m_acc + pm) >= target);
-          const uint32_t okb = __ballot_sync(0xffffffffu, ok);
-          if (okb) {
-            const int L = __ffs(okb) - 1;
-            jb = j0 + L;
-            kb = __shfl_sync(0xffffffffu, kj, L);
-            done = true;
-          } else if (cb) {
-            c_acc += __shfl_sync(0xffffffffu, pc, 31);
-            m_acc += __shfl_sync(0xffffffffu, pm, 31);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j0 = j1 + 32 * u;
+            if (done || j0 >= T) break;
+            const int j = j0 + lane;
+            uint64_t kj = 0, mj = 0;
+            bool cand = false;
+            if (j < T) {
+              const double x = xs[u];
+              kj = desc_key(x);
+              cand = (kj & mask) == prefix;
+              if (cand) mj = mass_fx(x, m);
+            }
+            // candidates share one key when shift == 0; a single candidate otherwise
+            const uint32_t cb = __ballot_sync(0xffffffffu, cand);
+            unsigned long long pm = cand ? mj : 0ull;
+            uint32_t pc = cand ? 1u : 0u;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const unsigned long long t1 = __shfl_up_sync(0xffffffffu, pm, o);
+              const uint32_t t2 = __shfl_up_sync(0xffffffffu, pc, o);
+              if (lane >= o) {
+                pm += t1;
+                pc += t2;
+              }
+            }
+            const bool ok = cand && (c_acc + pc >= static_cast<uint64_t>(nk)) &&
+                            (static_cast<double>(m_acc + pm) >= target);
+            const uint32_t okb = __ballot_sync(0xffffffffu, ok);
+            if (okb) {
+              const int L = __ffs(okb) - 1;
+              jb = j0 + L;
+              kb = __shfl_sync(0xffffffffu, kj, L);
+              done = true;
+            } else if (cb) {
+              c_acc += __shfl_sync(0xffffffffu, pc, 31);
+              m_acc += __shfl_sync(0xffffffffu, pm, 31);
+            }
           }
         }
         break;
