@@ -127,3 +127,46 @@ def test_sweep_densest_full_router_sampled_attention():
     """Config-4 sweep point with the longest lists (k = 4, p = 0.8 at the amplitude
     calibrated for 80% sparsity): ragged unions of up to min(2 cap, T) entries."""
     _full("sweep_0.8_80", sample_heads=(0, 20), nq=6, nkv=3)
+
+
+def test_t4096_ragged_router_and_sampled_attention():
+    """T = 4096 cubes (latent 63 x 62 x 61: every axis ragged), D = 64, one head: every router
+    row against the oracle, and forward / backward of sampled cubes (among them the last,
+    partial cube) with the GPU's lists."""
+    cfg = synth.small_config("t4096", 1, 1, 64, (63, 62, 61), 8, 0.5)
+    x = synth.make_inputs(cfg, 0)
+    p = sa.make_params(cfg.B, cfg.H, cfg.D, cfg.lat, cfg.top_k, cfg.top_p)
+    npad, T = sa.geometry(p)
+    assert T == 4096
+    dev = torch.device("cuda")
+    t = {n: sa.tile(x[n].to(dev), p) for n in x}
+    A = sa.Attention(p)
+    idx, cnt = A.plan(t["q"], t["k"])
+    out, lse, out32 = A.forward(t["q"], t["k"], t["v"], idx, cnt)
+    dq, dk, dv = A.backward(t["q"], t["k"], t["v"], out, lse, t["do"], idx, cnt, out_f32=out32)
+    torch.cuda.synchronize()
+    for op in (sa.OP_PLAN, sa.OP_FORWARD, sa.OP_BACKWARD):
+        assert sa.device_status(A._ws[op]) == 0
+    lay = O.cube_layout(cfg.lat)
+    q, k, v, do = (O.tile(x[n][0, 0].double().numpy(), lay) for n in ("q", "k", "v", "do"))
+    tr = O.route_head(q, k, lay.valid, cfg.top_k, cfg.top_p)
+    lists = gpu_lists(idx, cnt, 0, 0)
+    mis, ties, bad = classify_router_rows(tr, lists, cfg.top_p)
+    assert mis == 0, f"rows {bad[:5]}"
+    assert ties <= max(2, 1e-3 * T)
+    rng = np.random.default_rng(7)
+    qb = np.sort(rng.choice(T, 6, replace=False))
+    qb[-1] = T - 1
+    kb = np.sort(rng.choice(T, 4, replace=False))
+    kb[-1] = T - 1
+    o_ref, lse_ref = O.attention_forward_head(q, k, v, lists, lay.valid, q_blocks=qb)
+    g = O.attention_backward_head(q, k, v, do, lists, lay.valid, q_blocks=qb, kv_blocks=kb)
+    rows = np.concatenate([np.arange(i * 64, (i + 1) * 64) for i in qb])
+    rows = rows[lay.valid[rows]]
+    cols = np.concatenate([np.arange(j * 64, (j + 1) * 64) for j in kb])
+    cols = cols[lay.valid[cols]]
+    assert_close("out", out[0, 0].float().cpu().numpy()[rows], o_ref[rows])
+    assert np.max(np.abs(lse[0, 0].cpu().numpy()[rows] - lse_ref[rows])) < 1e-3
+    assert_close("dq", dq[0, 0].cpu().numpy()[rows], g[0][rows])
+    assert_close("dk", dk[0, 0].cpu().numpy()[cols], g[1][cols])
+    assert_close("dv", dv[0, 0].cpu().numpy()[cols], g[2][cols])
