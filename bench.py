@@ -177,8 +177,9 @@ def run_ours(args, rank, world, dist):
     fwd_avg = statistics.mean(fwd_ms)
     bwd_avg = statistics.mean(bwd_ms)
     plan_avg = statistics.mean(plan_ms)
-    # dominant kernel: the forward kernel is the only launch of sa_forward; it is timed
-    # on the launching (current) stream inside the timed region
+    # dominant kernel: the forward kernel, timed with events around sa_forward on the launching
+    # (current) stream inside the timed region; the call's two other launches (cube mask, query
+    # pair union) are about 0.3% of its time, so this slightly understates the kernel's own rate
     fwd_tf = fwd_fl / (fwd_avg * 1e-3) / 1e12
     peak_tf = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
     roofline = {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": round(fwd_tf, 2),
