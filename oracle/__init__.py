@@ -23,6 +23,9 @@ float64, with numpy matmuls and sorts as the only library steps:
                          constant (VSA2 page section 2.1: the router output M carries
                          no gradient)
 * error decomposition .. SpargeAttention2 page, equation 8
+* coarse branch, gate .. VSA page, "Big-Picture Architecture" and "Gated Combination";
+                         VSA2 page section 2.2, "Coarse Branch" and the gate equation
+                         (module ``coarse``)
 
 Parity pinning: every function here is pinned by the ``-m "not gpu"`` tests in
 ``tests/test_oracle_*.py`` against worked numbers printed on the pages, closed
@@ -34,4 +37,7 @@ from .attention import (  # noqa: F401
     attention_forward_head, attention_backward_head, dense_attention_head,
     e4m3_decode, dequantize_rows, eq8_error_terms, block_grid_shape, vsa_sparsity,
     topk_from_fraction,
+)
+from .coarse import (  # noqa: F401
+    coarse_forward_head, repeat_cubes, gated_forward_head, gated_backward_head,
 )
