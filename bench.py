@@ -422,12 +422,24 @@ def traffic_for(kernel: str, ntiles: int):
     return int(per_tile * ntiles)
 
 
+# What decides the forward kernel's DRAM traffic: its own source and device headers, and in
+# the C ABI the tensor-map encoding, the argument setup and the forward entry point.
+FWD_SOURCES = ("attn_fwd.cu", "attn_common.cuh", "geometry.cuh", "ptx.cuh")
+FWD_ABI_FUNCTIONS = ("bool make_map(", "sa::AttnArgs base_args(", "sa_status sa_forward(")
+
+
 def source_sha() -> str:
+    """Hash of the forward kernel's sources (see FWD_SOURCES, FWD_ABI_FUNCTIONS)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_attention_cubes_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in FWD_SOURCES:
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
+    with open(os.path.join(csrc, "api.cu")) as f:
+        api = f.read()
+    for sig in FWD_ABI_FUNCTIONS:
+        i = api.index(sig)
+        h.update(api[i:api.index("\n}\n", i) + 3].encode())
     return h.hexdigest()[:16]
 
 
