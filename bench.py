@@ -213,9 +213,12 @@ def run_ours(args, rank, world, dist):
     }
     if args.e2e_steps > 0:
         result["e2e"] = run_e2e(args, sa, A, p, host, dev, fwd_fl + bwd_fl, world, dist)
-    if args.config == "720p" and not args.no_fp8:
+    if args.config == "720p" and not (args.no_fp8 and args.no_gated):
         del x, A
+    if args.config == "720p" and not args.no_fp8:
         result["fp8_forward"] = run_fp8_forward(args, sa, synth, rank, dev, flush, peak_tf, peaks.get("hbm_gbs"), dist)
+    if args.config == "720p" and not args.no_gated:
+        result["gated"] = run_gated(args, sa, synth, cfg, host, rank, dev, flush, result["breakdown_ms"], dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(cfg, host, seconds=args.cpu_seconds)
     return result
@@ -278,6 +281,82 @@ def run_fp8_forward(args, sa, synth, rank, dev, flush, bf16_peak, hbm_peak, dist
             "forward_peak_tflops": round(peak, 1), "forward_frac": round(tf / peak, 4),
             "router_gbs": round(router_bytes / (plan_ms * 1e-3) / 1e9, 1),
             "router_frac": round(router_bytes / (plan_ms * 1e-3) / 1e9 / hbm_peak, 4)}
+
+
+def run_gated(args, sa, synth, cfg, host, rank, dev, flush, plain_ms, dist):
+    """The full gated layer at the same shape: sa_plan_coarse (router + coarse branch),
+    sa_forward_gated (fine stage + O = G * Repeat(Oc) + O_f) and sa_backward_gated (fine +
+    coarse gradients, dG), timed like the main step.  Reports each phase and what the coarse
+    branch adds to the plain step.  Its cube-level products (T x T x D per head: one in the
+    forward, five in the backward) run on the fp32 FMA pipe."""
+    import torch
+    p = sa.make_params(cfg.B, cfg.H, cfg.D, cfg.lat, cfg.top_k, cfg.top_p)
+    npad, T = sa.geometry(p)
+    t = {n: sa.tile(host[n].to(dev), p) for n in ("q", "k", "v", "do")}
+    gate = synth.make_gate(cfg, seed=rank_seed(rank)).to(dev)
+    ws = {op: sa.new_workspace(p, op, dev) for op in (sa.OP_PLAN_COARSE, sa.OP_FORWARD, sa.OP_BACKWARD_GATED)}
+    co = sa.Coarse.empty(p, dev)
+    shape = tuple(t["q"].shape)
+    out = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    out32 = torch.empty(shape, dtype=torch.float32, device=dev)
+    lse = torch.empty((cfg.B, cfg.H, npad), dtype=torch.float32, device=dev)
+    grads = [torch.empty(shape, dtype=torch.float32, device=dev) for _ in range(3)]
+    dgate = torch.empty((cfg.B, cfg.H, npad), dtype=torch.float32, device=dev)
+    idx = torch.empty((cfg.B, cfg.H, T, p.kv_capacity), dtype=torch.int32, device=dev)
+    cnt = torch.empty((cfg.B, cfg.H, T), dtype=torch.int32, device=dev)
+    launches = {"n": 0}
+
+    def step(rec=None):
+        n = 0
+        if rec is not None:
+            rec[0].record()
+        sa.plan_coarse(t["q"], t["k"], t["v"], p, kv_index=idx, kv_count=cnt, coarse=co, ws=ws[sa.OP_PLAN_COARSE])
+        n += sa.last_launch_count()
+        if rec is not None:
+            rec[1].record()
+        sa.forward_gated(t["q"], t["k"], t["v"], idx, cnt, p, co, gate, out=out, lse=lse, ws=ws[sa.OP_FORWARD],
+                         with_f32=True, out_f32=out32)
+        n += sa.last_launch_count()
+        if rec is not None:
+            rec[2].record()
+        sa.backward_gated(t["q"], t["k"], t["v"], out, lse, t["do"], gate, idx, cnt, p, co, dq=grads[0], dk=grads[1],
+                          dv=grads[2], dgate=dgate, ws=ws[sa.OP_BACKWARD_GATED], out_f32=out32)
+        n += sa.last_launch_count()
+        if rec is not None:
+            rec[3].record()
+        launches["n"] += n
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    for op, w in ws.items():
+        st = sa.device_status(w)
+        if st != 0:
+            raise RuntimeError(f"gated: device status {sa.STATUS_NAMES.get(st, st)} (op {op})")
+    ntiles = int(cnt.sum().item())
+    steps = max(3, min(args.steps, 10))
+    recs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches["n"] = 0
+    for s in range(steps):
+        flush.fill_(s & 0xff)
+        step(recs[s])
+    torch.cuda.synchronize()
+    ms = [statistics.mean(r[i].elapsed_time(r[i + 1]) for r in recs) for i in range(3)]
+    fwd_fl, bwd_fl = tile_flops(cfg.D, ntiles)
+    cube_fl = 2.0 * cfg.B * cfg.H * T * T * cfg.D      # one cube-level product
+    total_ms = sum(ms)
+    return {"config": f"{cfg.name}: O = G * Repeat(Oc) + O_f, gates tanh(N(0,1)), fp32 out kept",
+            "steps": steps, "selected_tiles": ntiles,
+            "plan_coarse_ms": round(ms[0], 4), "forward_gated_ms": round(ms[1], 4),
+            "backward_gated_ms": round(ms[2], 4), "ms_per_step": round(total_ms, 4),
+            "added_ms": {"plan": round(ms[0] - plain_ms["plan"], 4), "forward": round(ms[1] - plain_ms["forward"], 4),
+                         "backward": round(ms[2] - plain_ms["backward"], 4)},
+            "cube_level_gflop": round(6 * cube_fl / 1e9, 2),
+            "effective_tflops": round((fwd_fl + bwd_fl + 6 * cube_fl) / (total_ms * 1e-3) / 1e12, 3),
+            "gpu_launches_per_step": launches["n"] // steps}
 
 
 def cta_balance(masks, sms: int):
@@ -561,6 +640,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the e4m3 Q/K forward section")
+    ap.add_argument("--no-gated", action="store_true", help="skip the gated (coarse + fine) layer section")
     ap.add_argument("--sweep", action="store_true",
                     help="config-4 sweep (k=4, p x sparsity grid): one JSON line per point with load balance")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

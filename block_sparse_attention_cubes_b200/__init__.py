@@ -11,6 +11,9 @@ Entry points mirror the C ABI in ``include/sa.h``:
 * :func:`forward`   fine stage -> ``out [B,H,Npad,D]`` bf16, ``lse [B,H,Npad]`` fp32
 * :func:`backward`  -> ``dq, dk, dv`` fp32
 * :func:`tile` / :func:`untile`  latent order <-> cube-major padded order
+* :func:`plan_coarse`     router + coarse branch -> lists and a :class:`Coarse`
+* :func:`forward_gated`   fine stage, then ``O = G * Repeat(Oc) + O_f``
+* :func:`backward_gated`  -> ``dq, dk, dv`` (fine + coarse) and ``dgate``
 """
 from __future__ import annotations
 
@@ -26,14 +29,14 @@ SA_OK = 0
 STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_ALIGNMENT",
                 4: "SA_ERR_CAPACITY", 5: "SA_ERR_WORKSPACE", 6: "SA_ERR_LAUNCH", 7: "SA_ERR_DEVICE_TIMEOUT",
                 8: "SA_ERR_DEVICE_INDEX"}
-OP_PLAN, OP_FORWARD, OP_BACKWARD = 0, 1, 2
+OP_PLAN, OP_FORWARD, OP_BACKWARD, OP_PLAN_COARSE, OP_BACKWARD_GATED = 0, 1, 2, 3, 4
 BF16, FP8_E4M3 = 0, 1
 DEBUG_SKIP_LOADS = 1
 
 # every symbol include/sa.h declares
 EXPORTS = ("sa_padded_tokens", "sa_num_cubes", "sa_topk_from_fraction", "sa_workspace_size", "sa_tile",
            "sa_untile", "sa_plan", "sa_forward", "sa_backward", "sa_get_device_status", "sa_status_string",
-           "sa_last_launch_count", "sa_plan_static")
+           "sa_last_launch_count", "sa_plan_static", "sa_plan_coarse", "sa_forward_gated", "sa_backward_gated")
 
 
 class SAError(RuntimeError):
@@ -48,6 +51,11 @@ class Params(ctypes.Structure):
                 ("top_k", ctypes.c_int), ("top_p", ctypes.c_float), ("kv_capacity", ctypes.c_int),
                 ("qk_dtype", ctypes.c_int), ("softmax_scale", ctypes.c_float),
                 ("timeout_ms", ctypes.c_uint), ("debug_flags", ctypes.c_uint)]
+
+
+class CoarseC(ctypes.Structure):
+    _fields_ = [("qbar", ctypes.c_void_p), ("kbar", ctypes.c_void_p), ("vbar", ctypes.c_void_p),
+                ("oc", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
 
 
 _lib = None
@@ -77,6 +85,10 @@ def load_library(path: str = LIB_PATH):
         "sa_status_string": (ctypes.c_char_p, [i32]),
         "sa_last_launch_count": (i32, []),
         "sa_plan_static": (i32, [vp, vp, vp, vp, P, vp, vp, vp]),
+        "sa_plan_coarse": (i32, [vp, vp, vp, P, vp, vp, ctypes.POINTER(CoarseC), vp, sz, vp]),
+        "sa_forward_gated": (i32, [vp, vp, vp, vp, vp, P, ctypes.POINTER(CoarseC), vp, vp, vp, vp, vp, sz, vp]),
+        "sa_backward_gated": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, P, ctypes.POINTER(CoarseC), vp, vp, vp,
+                                    vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -279,6 +291,127 @@ def backward(q, k, v, out, lse, dout, kv_index, kv_count, p: Params, dq=None, dk
                                     ws.numel(), _stream(stream))
     _check(st, "sa_backward")
     return dq, dk, dv
+
+
+@dataclass
+class Coarse:
+    """Cube-level tensors of the coarse branch, fp32: qbar, kbar, vbar, oc ``[B,H,T,D]`` and
+    lse ``[B,H,T]`` (written by :func:`plan_coarse`, read by the gated backward)."""
+    qbar: object
+    kbar: object
+    vbar: object
+    oc: object
+    lse: object
+
+    @classmethod
+    def empty(cls, p: Params, device=None):
+        torch = _torch()
+        _, T = geometry(p)
+        f = lambda *shape: torch.empty(shape, dtype=torch.float32, device=device or "cuda")
+        return cls(f(p.B, p.H, T, p.D), f(p.B, p.H, T, p.D), f(p.B, p.H, T, p.D), f(p.B, p.H, T, p.D),
+                   f(p.B, p.H, T))
+
+    def c_struct(self, p: Params) -> CoarseC:
+        torch = _torch()
+        _, T = geometry(p)
+        for n in ("qbar", "kbar", "vbar", "oc"):
+            t = getattr(self, n)
+            _contig(t, n, torch.float32)
+            _shape(t, (p.B, p.H, T, p.D), n)
+        _contig(self.lse, "lse", torch.float32)
+        _shape(self.lse, (p.B, p.H, T), "lse")
+        return CoarseC(*(t.data_ptr() for t in (self.qbar, self.kbar, self.vbar, self.oc, self.lse)))
+
+
+def _gate_tensor(gate, p: Params, name="gate"):
+    torch = _torch()
+    npad, _ = geometry(p)
+    _contig(gate, name, torch.float32)
+    _shape(gate, (p.B, p.H, npad), name)
+
+
+def plan_coarse(q, k, v, p: Params, kv_index=None, kv_count=None, coarse=None, ws=None, stream=None):
+    """Router and coarse branch in one call: returns (kv_index, kv_count, :class:`Coarse`)."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _token_tensor(t, p, n, 2)
+    _, T = geometry(p)
+    dev = q.device
+    if kv_index is None:
+        kv_index = torch.empty((p.B, p.H, T, p.kv_capacity), dtype=torch.int32, device=dev)
+    if kv_count is None:
+        kv_count = torch.empty((p.B, p.H, T), dtype=torch.int32, device=dev)
+    if coarse is None:
+        coarse = Coarse.empty(p, dev)
+    if ws is None:
+        ws = new_workspace(p, OP_PLAN_COARSE, dev)
+    cs = coarse.c_struct(p)
+    st = load_library().sa_plan_coarse(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(p), _ptr(kv_index), _ptr(kv_count),
+                                       ctypes.byref(cs), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "sa_plan_coarse")
+    return kv_index, kv_count, coarse
+
+
+def forward_gated(q, k, v, kv_index, kv_count, p: Params, coarse: Coarse, gate, out=None, lse=None, ws=None,
+                  stream=None, with_f32: bool = False, out_f32=None):
+    """Fine stage then ``O = G * Repeat(Oc) + O_f``; returns (out, lse[, out_f32]) like :func:`forward`."""
+    torch = _torch()
+    npad, T = geometry(p)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _token_tensor(t, p, n, 2)
+    _gate_tensor(gate, p)
+    _contig(kv_index, "kv_index", torch.int32)
+    _contig(kv_count, "kv_count", torch.int32)
+    _shape(kv_index, (p.B, p.H, T, p.kv_capacity), "kv_index")
+    _shape(kv_count, (p.B, p.H, T), "kv_count")
+    dev = q.device
+    if out is None:
+        out = torch.empty((p.B, p.H, npad, p.D), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((p.B, p.H, npad), dtype=torch.float32, device=dev)
+    if with_f32 and out_f32 is None:
+        out_f32 = torch.empty((p.B, p.H, npad, p.D), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = new_workspace(p, OP_FORWARD, dev)
+    cs = coarse.c_struct(p)
+    st = load_library().sa_forward_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_index), _ptr(kv_count), ctypes.byref(p),
+                                         ctypes.byref(cs), _ptr(gate), _ptr(out), _ptr(lse), _ptr(out_f32), _ptr(ws),
+                                         ws.numel(), _stream(stream))
+    _check(st, "sa_forward_gated")
+    return (out, lse, out_f32) if with_f32 else (out, lse)
+
+
+def backward_gated(q, k, v, out, lse, dout, gate, kv_index, kv_count, p: Params, coarse: Coarse, dq=None, dk=None,
+                   dv=None, dgate=None, ws=None, stream=None, out_f32=None):
+    """Gradients of the gated output: returns (dq, dk, dv, dgate), fp32."""
+    torch = _torch()
+    npad, T = geometry(p)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _token_tensor(t, p, n, 2)
+    if out_f32 is not None:
+        _token_tensor(out_f32, p, "out_f32", 4)
+    _gate_tensor(gate, p)
+    _contig(lse, "lse", torch.float32)
+    _shape(lse, (p.B, p.H, npad), "lse")
+    _contig(kv_index, "kv_index", torch.int32)
+    _contig(kv_count, "kv_count", torch.int32)
+    _shape(kv_index, (p.B, p.H, T, p.kv_capacity), "kv_index")
+    _shape(kv_count, (p.B, p.H, T), "kv_count")
+    dev = q.device
+    shape = tuple(q.shape)
+    dq = torch.empty(shape, dtype=torch.float32, device=dev) if dq is None else dq
+    dk = torch.empty(shape, dtype=torch.float32, device=dev) if dk is None else dk
+    dv = torch.empty(shape, dtype=torch.float32, device=dev) if dv is None else dv
+    dgate = torch.empty((p.B, p.H, npad), dtype=torch.float32, device=dev) if dgate is None else dgate
+    if ws is None:
+        ws = new_workspace(p, OP_BACKWARD_GATED, dev)
+    cs = coarse.c_struct(p)
+    st = load_library().sa_backward_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(out_f32), _ptr(lse), _ptr(dout),
+                                          _ptr(gate), _ptr(kv_index), _ptr(kv_count), ctypes.byref(p),
+                                          ctypes.byref(cs), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgate), _ptr(ws),
+                                          ws.numel(), _stream(stream))
+    _check(st, "sa_backward_gated")
+    return dq, dk, dv, dgate
 
 
 @dataclass

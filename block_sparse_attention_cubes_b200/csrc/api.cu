@@ -63,12 +63,43 @@ struct WsLayout {
   size_t qbar = 0, kbar = 0, scores = 0;                   // plan
   size_t delta = 0, nlse2 = 0, bits = 0;                  // backward
   size_t ukcnt = 0, uklist = 0;                            // backward: key-pair unions
+  size_t p32 = 0;                                          // plan + coarse: Pc [BH, T, T] fp32
+  size_t doc = 0, dltc = 0, s32 = 0, ds32 = 0;             // gated backward: coarse scratch
+  size_t cq = 0, ck = 0, cv = 0;
   size_t total = 0;
 };
 
 WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
   WsLayout w;
   const size_t BH = static_cast<size_t>(p->B) * p->H;
+  if (op == SA_OP_PLAN_COARSE || op == SA_OP_BACKWARD_GATED) {
+    // the plain layout, then the coarse branch's buffers
+    w = ws_layout(p, g, op == SA_OP_PLAN_COARSE ? SA_OP_PLAN : SA_OP_BACKWARD);
+    const size_t TT = BH * g.T * static_cast<size_t>(g.T) * sizeof(float);
+    const size_t TD = BH * g.T * static_cast<size_t>(p->D) * sizeof(float);
+    size_t off = w.total;
+    if (op == SA_OP_PLAN_COARSE) {
+      w.p32 = off;
+      off = align256(off + TT);
+    } else {
+      w.doc = off;
+      off = align256(off + TD);
+      w.dltc = off;
+      off = align256(off + BH * g.T * sizeof(float));
+      w.s32 = off;
+      off = align256(off + TT);
+      w.ds32 = off;
+      off = align256(off + TT);
+      w.cq = off;
+      off = align256(off + TD);
+      w.ck = off;
+      off = align256(off + TD);
+      w.cv = off;
+      off = align256(off + TD);
+    }
+    w.total = off;
+    return w;
+  }
   size_t off = kHeader;
   if (op == SA_OP_PLAN) {
     w.qbar = off;
@@ -182,7 +213,7 @@ int sa_topk_from_fraction(double frac, int T) {
 
 size_t sa_workspace_size(const sa_params* p, int op) {
   Geom g;
-  if (check_params(p, &g) != SA_OK || op < 0 || op > 2) return 0;
+  if (check_params(p, &g) != SA_OK || op < SA_OP_PLAN || op > SA_OP_BACKWARD_GATED) return 0;
   return ws_layout(p, g, op).total;
 }
 
@@ -288,9 +319,26 @@ sa_status sa_forward(const void* q, const void* k, const void* v, const float* q
   return SA_OK;
 }
 
-sa_status sa_backward(const void* q, const void* k, const void* v, const void* out, const float* out_f32,
-                      const float* lse, const void* dout, const int32_t* kv_index, const int32_t* kv_count, const sa_params* p,
-                      float* dq, float* dk, float* dv, void* ws, size_t ws_bytes, sa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+sa_status check_coarse(const sa_coarse* c) {
+  if (!c || !c->qbar || !c->kbar || !c->vbar || !c->oc || !c->lse) return SA_ERR_INVALID_ARG;
+  if (!aligned16(c->qbar) || !aligned16(c->kbar) || !aligned16(c->vbar) || !aligned16(c->oc) || !aligned4(c->lse))
+    return SA_ERR_ALIGNMENT;
+  return SA_OK;
+}
+
+sa::CoarseTensors coarse_tensors(const sa_coarse* c) {
+  return sa::CoarseTensors{c->qbar, c->kbar, c->vbar, c->oc, c->lse};
+}
+
+// sa_backward, and with `coarse` set sa_backward_gated (gate, dgate and the coarse tensors).
+sa_status backward_impl(const void* q, const void* k, const void* v, const void* out, const float* out_f32,
+                        const float* lse, const void* dout, const float* gate, const int32_t* kv_index,
+                        const int32_t* kv_count, const sa_params* p, const sa_coarse* coarse, float* dq, float* dk,
+                        float* dv, float* dgate, void* ws, size_t ws_bytes, sa_stream_t stream) {
   Geom g;
   g_last_launches = 0;
   sa_status s = check_params(p, &g);
@@ -302,7 +350,14 @@ sa_status sa_backward(const void* q, const void* k, const void* v, const void* o
       !aligned16(dk) || !aligned16(dv) || !aligned4(lse) || !aligned4(kv_index) || !aligned4(kv_count) ||
       (out_f32 && !aligned16(out_f32)))
     return SA_ERR_ALIGNMENT;
-  const WsLayout w = ws_layout(p, g, SA_OP_BACKWARD);
+  const bool gated = coarse != nullptr;
+  if (gated) {
+    if (!gate || !dgate) return SA_ERR_INVALID_ARG;
+    if ((s = check_coarse(coarse)) != SA_OK) return s;
+    if (!aligned4(gate) || !aligned4(dgate)) return SA_ERR_ALIGNMENT;
+    if (p->B * p->H > 65535) return SA_ERR_UNSUPPORTED;  // one grid layer per head
+  }
+  const WsLayout w = ws_layout(p, g, gated ? SA_OP_BACKWARD_GATED : SA_OP_BACKWARD);
   if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
   if (!aligned16(ws)) return SA_ERR_ALIGNMENT;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -322,16 +377,103 @@ sa_status sa_backward(const void* q, const void* k, const void* v, const void* o
   a.cube_mask = reinterpret_cast<unsigned long long*>(wb + w.cmask);
   if (sa::launch_cube_mask(g, reinterpret_cast<unsigned long long*>(wb + w.cmask), st) != cudaSuccess)
     return SA_ERR_LAUNCH;
+  float* delta = reinterpret_cast<float*>(wb + w.delta);
+  float* nlse2 = reinterpret_cast<float*>(wb + w.nlse2);
+  int coarse_launches = 0;
+  sa::CoarseAdd add{};
+  if (gated) {
+    const sa::CoarseGradWs cw{reinterpret_cast<float*>(wb + w.doc), reinterpret_cast<float*>(wb + w.dltc),
+                              reinterpret_cast<float*>(wb + w.s32),  reinterpret_cast<float*>(wb + w.ds32),
+                              reinterpret_cast<float*>(wb + w.cq),   reinterpret_cast<float*>(wb + w.ck),
+                              reinterpret_cast<float*>(wb + w.cv)};
+    if (sa::launch_coarse_backward(out, out_f32, dout, lse, gate, coarse_tensors(coarse), dgate, delta, nlse2, cw,
+                                   a.scale, g, a.BH, p->D, st, &coarse_launches) != cudaSuccess)
+      return SA_ERR_LAUNCH;
+    add = sa::CoarseAdd{cw.cq, cw.ck, cw.cv};
+  }
   int launches = 0;
   a.ucap = union_cap(p, g);
-  if (sa::launch_backward(tq, tk, tv, tdo, out, out_f32, dout, a, reinterpret_cast<uint32_t*>(wb + w.bits),
-                          reinterpret_cast<float*>(wb + w.delta), reinterpret_cast<float*>(wb + w.nlse2),
-                          reinterpret_cast<int32_t*>(wb + w.ulist),
-                          reinterpret_cast<int32_t*>(wb + w.ucnt), reinterpret_cast<int32_t*>(wb + w.uklist),
-                          reinterpret_cast<int32_t*>(wb + w.ukcnt), st, &launches) != cudaSuccess)
+  if (sa::launch_backward(tq, tk, tv, tdo, out, out_f32, dout, a, reinterpret_cast<uint32_t*>(wb + w.bits), delta,
+                          nlse2, reinterpret_cast<int32_t*>(wb + w.ulist), reinterpret_cast<int32_t*>(wb + w.ucnt),
+                          reinterpret_cast<int32_t*>(wb + w.uklist), reinterpret_cast<int32_t*>(wb + w.ukcnt), add,
+                          gated, st, &launches) != cudaSuccess)
     return SA_ERR_LAUNCH;
-  g_last_launches = launches + 1;
+  g_last_launches = 1 + coarse_launches + launches;
   return SA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sa_status sa_backward(const void* q, const void* k, const void* v, const void* out, const float* out_f32,
+                      const float* lse, const void* dout, const int32_t* kv_index, const int32_t* kv_count, const sa_params* p,
+                      float* dq, float* dk, float* dv, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  return backward_impl(q, k, v, out, out_f32, lse, dout, nullptr, kv_index, kv_count, p, nullptr, dq, dk, dv, nullptr,
+                       ws, ws_bytes, stream);
+}
+
+sa_status sa_plan_coarse(const void* q, const void* k, const void* v, const sa_params* p, int32_t* kv_index,
+                         int32_t* kv_count, const sa_coarse* coarse, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  Geom g;
+  g_last_launches = 0;
+  sa_status s = check_params(p, &g);
+  if (s != SA_OK) return s;
+  if (!q || !k || !v || !kv_index || !kv_count) return SA_ERR_INVALID_ARG;
+  if (p->qk_dtype != SA_BF16) return SA_ERR_UNSUPPORTED;
+  if ((s = check_coarse(coarse)) != SA_OK) return s;
+  if (p->B * p->H > 65535) return SA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(kv_index) || !aligned4(kv_count))
+    return SA_ERR_ALIGNMENT;
+  const WsLayout w = ws_layout(p, g, SA_OP_PLAN_COARSE);
+  if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SA_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  const int BH = p->B * p->H;
+  double* qbar = reinterpret_cast<double*>(wb + w.qbar);
+  double* kbar = reinterpret_cast<double*>(wb + w.kbar);
+  double* S = reinterpret_cast<double*>(wb + w.scores);
+  int plan_launches = 0, coarse_launches = 0;
+  if (sa::launch_plan(q, k, nullptr, nullptr, g, BH, p->D, false, softmax_scale(p), p->top_k, p->top_p,
+                      p->kv_capacity, kv_index, kv_count, qbar, kbar, S, static_cast<sa::DevStatus*>(ws), st,
+                      &plan_launches) != cudaSuccess ||
+      sa::launch_coarse_forward(v, qbar, kbar, S, reinterpret_cast<float*>(wb + w.p32), coarse_tensors(coarse), g, BH,
+                                p->D, st, &coarse_launches) != cudaSuccess)
+    return SA_ERR_LAUNCH;
+  g_last_launches = plan_launches + coarse_launches;
+  return SA_OK;
+}
+
+sa_status sa_forward_gated(const void* q, const void* k, const void* v, const int32_t* kv_index,
+                           const int32_t* kv_count, const sa_params* p, const sa_coarse* coarse, const float* gate,
+                           void* out, float* lse, float* out_f32, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  Geom g;
+  g_last_launches = 0;
+  sa_status s = check_params(p, &g);
+  if (s != SA_OK) return s;
+  if (p->qk_dtype != SA_BF16) return SA_ERR_UNSUPPORTED;
+  if (!gate) return SA_ERR_INVALID_ARG;
+  if ((s = check_coarse(coarse)) != SA_OK) return s;
+  if (!aligned4(gate)) return SA_ERR_ALIGNMENT;
+  s = sa_forward(q, k, v, nullptr, nullptr, kv_index, kv_count, p, out, lse, out_f32, ws, ws_bytes, stream);
+  if (s != SA_OK) return s;
+  const int fine_launches = g_last_launches;
+  if (sa::launch_coarse_combine(out, out_f32, gate, coarse->oc, g, p->B * p->H, p->D,
+                                reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SA_ERR_LAUNCH;
+  g_last_launches = fine_launches + 1;
+  return SA_OK;
+}
+
+sa_status sa_backward_gated(const void* q, const void* k, const void* v, const void* out, const float* out_f32,
+                            const float* lse, const void* dout, const float* gate, const int32_t* kv_index,
+                            const int32_t* kv_count, const sa_params* p, const sa_coarse* coarse, float* dq, float* dk,
+                            float* dv, float* dgate, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  if (!coarse) return SA_ERR_INVALID_ARG;
+  return backward_impl(q, k, v, out, out_f32, lse, dout, gate, kv_index, kv_count, p, coarse, dq, dk, dv, dgate, ws,
+                       ws_bytes, stream);
 }
 
 sa_status sa_get_device_status(const void* ws, sa_stream_t stream) {

@@ -113,7 +113,7 @@ template <int KS>  // D / 16; MMA loops unrolled (a counted loop costs more than
 __global__ void __launch_bounds__(dqk::kThreads, 1)
     attn_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                   const AttnArgs a) {
+                   const AttnArgs a, const CoarseAdd add) {
   using namespace dqk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -381,8 +381,19 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       if (lane == 0) mbar_arrive(&bars[B_DQFREE]);
       if (row_exists && grp * 64 < a.D) {
         float4* dst = reinterpret_cast<float4*>(a.dq + qrow * a.D + grp * 64);
+        // the coarse branch's term of this cube (valid rows only), when there is one
+        const float4* cq = (add.q && row_valid) ? reinterpret_cast<const float4*>(
+                                                      add.q + (static_cast<size_t>(bh) * g.T + icube) * a.D + grp * 64)
+                                                : nullptr;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        for (int c = 0; c < 16; ++c) {
+          float4 w = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          if (cq) {
+            const float4 t = __ldg(cq + c);
+            w.x += t.x, w.y += t.y, w.z += t.z, w.w += t.w;
+          }
+          dst[c] = w;
+        }
       }
       // an abort seen by any thread reaches every thread at the item boundary
       named_bar_sync(1, 256);
@@ -425,7 +436,7 @@ template <int KS>  // D / 16; MMA loops unrolled (a counted loop costs more than
 __global__ void __launch_bounds__(dkv::kThreads, 1)
     attn_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                     const AttnArgs a) {
+                     const AttnArgs a, const CoarseAdd add) {
   using namespace dkv;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -746,10 +757,21 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
         const size_t krow = static_cast<size_t>(bh) * g.Npad + static_cast<size_t>(kcube) * 64 + (r & 63);
         float4* pv = reinterpret_cast<float4*>(a.dv + krow * a.D + grp * 64);
         float4* pk = reinterpret_cast<float4*>(a.dk + krow * a.D + grp * 64);
+        // the coarse branch's terms of this cube (valid keys only), when there are some
+        const size_t co = (static_cast<size_t>(bh) * g.T + kcube) * a.D + grp * 64;
+        const bool has_add = add.k && key_valid;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          pv[c] = make_float4(gv[4 * c], gv[4 * c + 1], gv[4 * c + 2], gv[4 * c + 3]);
-          pk[c] = make_float4(gk[4 * c], gk[4 * c + 1], gk[4 * c + 2], gk[4 * c + 3]);
+          float4 wv = make_float4(gv[4 * c], gv[4 * c + 1], gv[4 * c + 2], gv[4 * c + 3]);
+          float4 wk = make_float4(gk[4 * c], gk[4 * c + 1], gk[4 * c + 2], gk[4 * c + 3]);
+          if (has_add) {
+            const float4 tv = __ldg(reinterpret_cast<const float4*>(add.v + co) + c);
+            const float4 tk = __ldg(reinterpret_cast<const float4*>(add.k + co) + c);
+            wv.x += tv.x, wv.y += tv.y, wv.z += tv.z, wv.w += tv.w;
+            wk.x += tk.x, wk.y += tk.y, wk.z += tk.z, wk.w += tk.w;
+          }
+          pv[c] = wv;
+          pk[c] = wk;
         }
       }
       named_bar_sync(1, 256);
@@ -766,7 +788,8 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const CUtensorMap& tdo, const void* out, const float* out_f32, const void* dout,
                             AttnArgs a, uint32_t* bits, float* delta, float* nlse2,
                             int32_t* uq_list,
-                            int32_t* uq_cnt, int32_t* uk_list, int32_t* uk_cnt, cudaStream_t stream, int* launches) {
+                            int32_t* uq_cnt, int32_t* uk_list, int32_t* uk_cnt, const CoarseAdd& add,
+                            bool delta_ready, cudaStream_t stream, int* launches) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaSuccess;
@@ -779,9 +802,10 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   }
   const Geom& g = a.g;
   const long long rows = static_cast<long long>(a.BH) * g.Npad;
-  delta_kernel<<<static_cast<unsigned>((rows + 8 * DELTA_ROWS - 1) / (8 * DELTA_ROWS)), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(out), out_f32, static_cast<const __nv_bfloat16*>(dout), a.lse, delta, nlse2,
-      g, a.BH, a.D);
+  if (!delta_ready)
+    delta_kernel<<<static_cast<unsigned>((rows + 8 * DELTA_ROWS - 1) / (8 * DELTA_ROWS)), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(out), out_f32, static_cast<const __nv_bfloat16*>(dout), a.lse, delta,
+        nlse2, g, a.BH, a.D);
   cudaError_t e = launch_query_pair_union(a.kv_index, a.kv_count, uq_list, uq_cnt, a.BH, g.T, a.cap, a.st, stream);
   if (e != cudaSuccess) return e;
   e = launch_key_pair_union(a.kv_index, a.kv_count, bits, uk_list, uk_cnt, a.BH, g.T, a.cap, a.st, stream);
@@ -796,13 +820,13 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   const int items = a.BH * ((g.T + 1) >> 1);
   const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
   if (a.D == 64) {
-    attn_dq_kernel<4><<<grid, dqk::kThreads, dqk::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
-    attn_dkdv_kernel<4><<<grid, dkv::kThreads, dkv::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+    attn_dq_kernel<4><<<grid, dqk::kThreads, dqk::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a, add);
+    attn_dkdv_kernel<4><<<grid, dkv::kThreads, dkv::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a, add);
   } else {
-    attn_dq_kernel<8><<<grid, dqk::kThreads, dqk::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
-    attn_dkdv_kernel<8><<<grid, dkv::kThreads, dkv::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+    attn_dq_kernel<8><<<grid, dqk::kThreads, dqk::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a, add);
+    attn_dkdv_kernel<8><<<grid, dkv::kThreads, dkv::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a, add);
   }
-  *launches = 6;
+  *launches = delta_ready ? 5 : 6;
   return cudaGetLastError();
 }
 

@@ -33,10 +33,56 @@ int num_sms();
 cudaError_t launch_forward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
                            cudaStream_t stream);
 
+// Per-cube terms the backward kernels add to every valid row of a cube (the coarse branch's
+// gradients through the mean pool), [BH, T, D] fp32 each; all NULL for the fine stage alone.
+struct CoarseAdd {
+  const float* q;
+  const float* k;
+  const float* v;
+};
+
+// With delta_ready, Delta and -lse*log2(e) are already in `delta` / `nlse2` and the Delta
+// pass is not launched.
 cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const void* out, const float* out_f32, const void* dout,
                             AttnArgs a, uint32_t* bits, float* delta, float* nlse2,
                             int32_t* uq_list,
-                            int32_t* uq_cnt, int32_t* uk_list, int32_t* uk_cnt, cudaStream_t stream, int* launches);
+                            int32_t* uq_cnt, int32_t* uk_list, int32_t* uk_cnt, const CoarseAdd& add,
+                            bool delta_ready, cudaStream_t stream, int* launches);
+
+// Coarse branch (cube-level tensors, fp32, [BH, T, D] and lse [BH, T]).
+struct CoarseTensors {
+  float* qbar;
+  float* kbar;
+  float* vbar;
+  float* oc;
+  float* lse;
+};
+
+// Backward scratch of the coarse branch.
+struct CoarseGradWs {
+  float* doc;   // [BH, T, D]  dOc^
+  float* dltc;  // [BH, T]     <dOc^, Oc^>
+  float* s;     // [BH, T, T]  scaled scores, then P
+  float* ds;    // [BH, T, T]  dS
+  float* cq;    // [BH, T, D]  dQc / n, dKc / n, dVc / n
+  float* ck;
+  float* cv;
+};
+
+// Vc pooled from v, fp32 copies of the router's fp64 Qc and Kc, Pc from the router's fp64
+// scores and Oc^ = Pc Vc (3 launches).
+cudaError_t launch_coarse_forward(const void* v, const double* qbar64, const double* kbar64, const double* S64,
+                                  float* P32, const CoarseTensors& c, const Geom& g, int BH, int D,
+                                  cudaStream_t stream, int* launches);
+// O = G * Oc^[cube] + O in place on the valid rows of out (bf16) and out_f32 (if not NULL).
+cudaError_t launch_coarse_combine(void* out, float* out_f32, const float* gate, const float* oc, const Geom& g,
+                                  int BH, int D, cudaStream_t stream);
+// dG, the fine branch's Delta and -lse*log2(e), and the coarse branch's per-cube gradient
+// terms w.cq, w.ck, w.cv (6 launches).
+cudaError_t launch_coarse_backward(const void* out, const float* out_f32, const void* dout, const float* lse,
+                                   const float* gate, const CoarseTensors& c, float* dgate, float* delta,
+                                   float* nlse2, const CoarseGradWs& w, float scale, const Geom& g, int BH, int D,
+                                   cudaStream_t stream, int* launches);
 
 }  // namespace sa

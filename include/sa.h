@@ -56,7 +56,13 @@ typedef enum {
 
 typedef enum { SA_BF16 = 0, SA_FP8_E4M3 = 1 } sa_qk_dtype;
 
-typedef enum { SA_OP_PLAN = 0, SA_OP_FORWARD = 1, SA_OP_BACKWARD = 2 } sa_op;
+typedef enum {
+  SA_OP_PLAN = 0,
+  SA_OP_FORWARD = 1,          /* also sa_forward_gated */
+  SA_OP_BACKWARD = 2,
+  SA_OP_PLAN_COARSE = 3,      /* sa_plan_coarse */
+  SA_OP_BACKWARD_GATED = 4    /* sa_backward_gated */
+} sa_op;
 
 typedef struct {
   int B, H, D;                /* batch, heads, head dim (D in {64, 128}) */
@@ -88,7 +94,10 @@ SA_API int sa_topk_from_fraction(double frac, int T);
  * adjacent query-cube pairs (int32, B*H*ceil(T/2)*(1 + 2*kv_capacity)).  Backward: status block
  * + cube masks + Delta and -lse*log2(e) (fp32, 2*B*H*Npad) + the selection as a bit matrix
  * (B*H*T*ceil(T/32) words) + the query-pair and key-pair union lists (int32,
- * B*H*ceil(T/2)*(2 + min(2*kv_capacity, T) + T)). */
+ * B*H*ceil(T/2)*(2 + min(2*kv_capacity, T) + T)).  Plan + coarse: the plan's, then the
+ * cube-level softmax Pc (fp32, B*H*T*T).  Gated backward: the backward's, then dOc^ and
+ * the three per-cube gradient terms (fp32, 4*B*H*T*D), <dOc^, Oc^> (B*H*T) and the
+ * cube-level scores and dS (fp32, 2*B*H*T*T). */
 SA_API size_t sa_workspace_size(const sa_params* p, int op);
 
 /* Layout helper (VSA page, "Cube Partitioning and Token Re-Indexing"; VSA2 page,
@@ -148,6 +157,60 @@ SA_API sa_status sa_forward(const void* q, const void* k, const void* v, const f
 SA_API sa_status sa_backward(const void* q, const void* k, const void* v, const void* out, const float* out_f32,
                       const float* lse, const void* dout, const int32_t* kv_index, const int32_t* kv_count, const sa_params* p,
                       float* dq, float* dk, float* dv, void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* ---- Coarse branch and gated combination ----
+ * VSA page, "Big-Picture Architecture" item 2, "What the coarse attention output O_c
+ * provides" and "Gated Combination"; VSA2 page, section 2.2 "Coarse Branch" and the gate
+ * equation.  Per head, with Qc, Kc, Vc the means of the valid tokens of each cube:
+ *   Pc = softmax(Qc Kc^T * scale)  (dense, T x T),   Oc^ = Pc Vc,
+ *   O  = G (.) Repeat_64(Oc^) + O_f,   O_f the fine stage's output (sa_forward).
+ * G is one scalar per token and head, the gate VALUE (VSA2's tanh(X W_g); the projection
+ * and its tanh belong to the caller's linear layers, and the backward returns dL/dG).
+ * VSA's fine gate is taken as 1 (its sparse adaptation removes it).  Padding slots get
+ * O = 0 whatever G holds there, and dG = 0.  bf16 only (qk_dtype SA_BF16, else
+ * SA_ERR_UNSUPPORTED); B*H <= 65535.  The cube-level tensors are caller-owned fp32 device
+ * arrays: qbar, kbar, vbar, oc [B,H,T,D] (16-byte aligned), lse [B,H,T] (natural log of
+ * each row's normaliser of the scaled cube scores). */
+typedef struct {
+  float* qbar;
+  float* kbar;
+  float* vbar;
+  float* oc;
+  float* lse;
+} sa_coarse;
+
+/* Router and coarse branch in one call: the same kv_index / kv_count as sa_plan (same
+ * kernels, bit-identical), and the cube-level tensors of `coarse` (written).  Q and K are
+ * pooled once for both (the coarse branch reads the router's fp64 means and scores).
+ * v: [B,H,Npad,D] bf16.  Workspace: sa_workspace_size(p, SA_OP_PLAN_COARSE).
+ * Deterministic. */
+SA_API sa_status sa_plan_coarse(const void* q, const void* k, const void* v, const sa_params* p, int32_t* kv_index,
+                                int32_t* kv_count, const sa_coarse* coarse, void* ws, size_t ws_bytes,
+                                sa_stream_t stream);
+
+/* sa_forward (arguments, errors and outputs as there, bf16 only), then
+ * O = G (.) Repeat_64(coarse->oc) + O_f written in place over out (and over out_f32 when
+ * given: then out is the bf16 rounding of the fp32 sum).  gate: [B,H,Npad] fp32.  lse is
+ * the fine stage's.  Workspace: sa_workspace_size(p, SA_OP_FORWARD).  Deterministic. */
+SA_API sa_status sa_forward_gated(const void* q, const void* k, const void* v, const int32_t* kv_index,
+                                  const int32_t* kv_count, const sa_params* p, const sa_coarse* coarse,
+                                  const float* gate, void* out, float* lse, float* out_f32, void* ws, size_t ws_bytes,
+                                  sa_stream_t stream);
+
+/* Gradients of the gated output, mask held constant: dq, dk, dv [B,H,Npad,D] fp32 are the
+ * fine stage's (as sa_backward, with dO_f = dO) plus the coarse branch's,
+ *   dG_t = <dO_t, Oc^[i]>,  dOc^[i] = sum_t G_t dO_t  (t over the valid tokens of cube i),
+ *   dVc = Pc^T dOc^,  dPc = dOc^ Vc^T,  dSc = Pc (.) (dPc - rowsum(Pc (.) dPc)),
+ *   dQc = scale dSc Kc,  dKc = scale dSc^T Qc,
+ * each cube-level gradient handed to the n_i valid tokens of its cube as dXc[i] / n_i.
+ * out / out_f32: the combined output from sa_forward_gated (the fine stage's Delta is taken
+ * as <dO, O> - G dG).  coarse: as written by sa_plan_coarse (read only).  gate: [B,H,Npad]
+ * fp32; dgate: [B,H,Npad] fp32 (0 on padding slots).  Workspace:
+ * sa_workspace_size(p, SA_OP_BACKWARD_GATED).  Deterministic. */
+SA_API sa_status sa_backward_gated(const void* q, const void* k, const void* v, const void* out, const float* out_f32,
+                                   const float* lse, const void* dout, const float* gate, const int32_t* kv_index,
+                                   const int32_t* kv_count, const sa_params* p, const sa_coarse* coarse, float* dq,
+                                   float* dk, float* dv, float* dgate, void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /* sa_plan without a workspace: the same router and the same results, for callers that
  * cannot allocate device memory (code running under a CUDA stream capture, serving

@@ -19,6 +19,8 @@ Recipe (per batch b, head h, tensor X in {q, k, v, do}):
   ``v = noise + 0.5 * alpha * phi``, ``do = noise``.
 * Sink heads multiply the key of latent token 0 by ``sink`` (8 by default).
 * Values are rounded fp64 -> fp32 -> bf16, each step round-to-nearest-even.
+* Gates of the gated combination (``make_gate``): ``tanh(N(0, 1))`` per cube-major token
+  slot, fp32, keyed by ``SeedSequence([seed, 4, b, h])``.
 
 ``alpha`` is set per head type ("uniform" or "sink"); for the configurations
 with a sparsity target it was calibrated once against the fp64 oracle router
@@ -184,6 +186,25 @@ def make_inputs(cfg: Config, seed: int = 0, names=("q", "k", "v", "do"), heads=N
         t = torch.stack(parts).reshape(cfg.B, len(heads), cfg.L, cfg.D)
         out[name] = t
     return out
+
+
+GATE_ID = 4
+
+
+def make_gate(cfg: Config, seed: int = 0, heads=None) -> torch.Tensor:
+    """Gate values of the gated combination, fp32 ``[B, len(heads), Npad]`` in cube-major slot
+    order (one per token slot; the slot order does not matter to an i.i.d. draw):
+    ``tanh(N(0, 1))`` from a Philox generator keyed by ``SeedSequence([seed, 4, b, h])``,
+    i.e. values spread over the open range of a tanh gate.  Padding slots get values too;
+    both sides must ignore them."""
+    heads = list(range(cfg.H)) if heads is None else list(heads)
+    npad = 64 * math.prod(-(-n // 4) for n in cfg.lat)
+    parts = []
+    for b in range(cfg.B):
+        for h in heads:
+            rng = np.random.Generator(np.random.Philox(np.random.SeedSequence([seed, GATE_ID, b, h])))
+            parts.append(np.tanh(rng.standard_normal(npad)).astype(np.float32))
+    return torch.from_numpy(np.stack(parts).reshape(cfg.B, len(heads), npad))
 
 
 def quantize_e4m3_rows(x: torch.Tensor, rows: int = 64):

@@ -86,3 +86,40 @@ def test_package_does_not_import_oracle():
                 if isinstance(node, (ast.Import, ast.ImportFrom)):
                     names = [a.name for a in node.names] if isinstance(node, ast.Import) else [node.module or ""]
                     assert not any(n.split(".")[0] == "oracle" for n in names), fn
+
+
+def test_coarse_entry_points_validate_on_the_host(lib):
+    p = sa.make_params(2, 3, 64, (8, 8, 8), 4, 0.5)          # T = 8, B*H = 6
+    T, BH, D, npad = 8, 6, 64, 512
+    plan, bwd = sa.workspace_size(p, sa.OP_PLAN), sa.workspace_size(p, sa.OP_BACKWARD)
+    # plan + Pc; backward + dOc^, three per-cube terms, delta_c, scores and dS (each 256-byte aligned)
+    assert sa.workspace_size(p, sa.OP_PLAN_COARSE) >= plan + BH * T * T * 4
+    assert sa.workspace_size(p, sa.OP_BACKWARD_GATED) >= bwd + 4 * BH * T * D * 4 + BH * T * 4 + 2 * BH * T * T * 4
+    assert sa.workspace_size(p, 5) == 0
+    bad = ctypes.c_void_p(16)
+    c = sa.CoarseC(16, 16, 16, 16, 16)
+    cref = ctypes.byref(c)
+    # every error below is returned before anything touches the device
+    assert lib.sa_plan_coarse(bad, bad, bad, ctypes.byref(p), bad, bad, None, bad, 1 << 30, None) == 1
+    assert lib.sa_plan_coarse(bad, bad, None, ctypes.byref(p), bad, bad, cref, bad, 1 << 30, None) == 1
+    assert lib.sa_plan_coarse(bad, bad, bad, ctypes.byref(p), bad, bad, cref, bad, 16, None) == 5
+    odd = sa.CoarseC(16, 16, 24, 16, 16)
+    assert lib.sa_plan_coarse(bad, bad, bad, ctypes.byref(p), bad, bad, ctypes.byref(odd), bad, 1 << 30, None) == 3
+    nul = sa.CoarseC(16, 16, 16, None, 16)
+    assert lib.sa_plan_coarse(bad, bad, bad, ctypes.byref(p), bad, bad, ctypes.byref(nul), bad, 1 << 30, None) == 1
+    fp8 = sa.make_params(2, 3, 128, (8, 8, 8), 4, 0.5, qk_dtype=sa.FP8_E4M3)
+    assert lib.sa_plan_coarse(bad, bad, bad, ctypes.byref(fp8), bad, bad, cref, bad, 1 << 30, None) == 2
+    # gated forward: gate required; the fine stage's checks follow
+    assert lib.sa_forward_gated(bad, bad, bad, bad, bad, ctypes.byref(p), cref, None, bad, bad, None, bad, 1 << 30,
+                                None) == 1
+    assert lib.sa_forward_gated(bad, bad, bad, bad, bad, ctypes.byref(p), cref, bad, bad, bad, None, bad, 16,
+                                None) == 5
+    # gated backward: coarse, gate and dgate required, the gated workspace size enforced
+    args = [bad] * 10
+    assert lib.sa_backward_gated(*args, ctypes.byref(p), None, bad, bad, bad, bad, bad, 1 << 30, None) == 1
+    args_nogate = [bad] * 7 + [None] + [bad] * 2
+    assert lib.sa_backward_gated(*args_nogate, ctypes.byref(p), cref, bad, bad, bad, bad, bad, 1 << 30, None) == 1
+    assert lib.sa_backward_gated(*args, ctypes.byref(p), cref, bad, bad, bad, bad, bad, bwd, None) == 5
+    many = sa.make_params(1, 70000, 64, (4, 4, 4), 1, 0.5)      # B*H above one grid layer per head
+    assert lib.sa_plan_coarse(bad, bad, bad, ctypes.byref(many), bad, bad, cref, bad, 1 << 40, None) == 2
+    assert lib.sa_last_launch_count() == 0
