@@ -62,6 +62,14 @@ class ClockSampler:
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+        # wait for the first sample, so nvidia-smi's start-up (NVML initialisation) is over
+        # before the timed region begins
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < 5.0:
+            self.f.flush()
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.05)
         time.sleep(0.3)
         return self
 
@@ -203,6 +211,8 @@ def run_ours(args, rank, world, dist):
                    "per_rank": "independent problem per rank (seed = rank)"},
         "breakdown_ms": {"plan": round(plan_avg, 4), "forward": round(fwd_avg, 4), "backward": round(bwd_avg, 4),
                          "fwd_plus_bwd": round(fwd_avg + bwd_avg, 4)},
+        "per_step_ms": {"plan": [round(v, 3) for v in plan_ms], "forward": [round(v, 3) for v in fwd_ms],
+                        "backward": [round(v, 3) for v in bwd_ms]},
         "fwd_bwd_tflops": round((fwd_fl + bwd_fl) / ((fwd_avg + bwd_avg) * 1e-3) / 1e12, 3),
         "router": {"achieved_gbs": round(router_gbs, 1), "peak_gbs": peaks.get("hbm_gbs"),
                    "frac": round(router_gbs / peaks.get("hbm_gbs"), 4), "algorithmic_bytes": router_bytes},
@@ -315,7 +325,7 @@ def run_gated(args, sa, synth, cfg, host, rank, dev, flush, plain_ms, dist):
         if rec is not None:
             rec[1].record()
         sa.forward_gated(t["q"], t["k"], t["v"], idx, cnt, p, co, gate, out=out, lse=lse, ws=ws[sa.OP_FORWARD],
-                         with_f32=True, out_f32=out32)
+                         out_f32=out32)
         n += sa.last_launch_count()
         if rec is not None:
             rec[2].record()
@@ -344,7 +354,8 @@ def run_gated(args, sa, synth, cfg, host, rank, dev, flush, plain_ms, dist):
         flush.fill_(s & 0xff)
         step(recs[s])
     torch.cuda.synchronize()
-    ms = [statistics.mean(r[i].elapsed_time(r[i + 1]) for r in recs) for i in range(3)]
+    per_step = [[r[i].elapsed_time(r[i + 1]) for r in recs] for i in range(3)]
+    ms = [statistics.mean(v) for v in per_step]
     fwd_fl, bwd_fl = tile_flops(cfg.D, ntiles)
     cube_fl = 2.0 * cfg.B * cfg.H * T * T * cfg.D      # one cube-level product
     total_ms = sum(ms)
@@ -356,7 +367,9 @@ def run_gated(args, sa, synth, cfg, host, rank, dev, flush, plain_ms, dist):
                          "backward": round(ms[2] - plain_ms["backward"], 4)},
             "cube_level_gflop": round(6 * cube_fl / 1e9, 2),
             "effective_tflops": round((fwd_fl + bwd_fl + 6 * cube_fl) / (total_ms * 1e-3) / 1e12, 3),
-            "gpu_launches_per_step": launches["n"] // steps}
+            "gpu_launches_per_step": launches["n"] // steps,
+            "per_step_ms": {n: [round(v, 3) for v in vals]
+                            for n, vals in zip(("plan_coarse", "forward_gated", "backward_gated"), per_step)}}
 
 
 def cta_balance(masks, sms: int):

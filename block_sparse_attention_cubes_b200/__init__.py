@@ -353,8 +353,9 @@ def plan_coarse(q, k, v, p: Params, kv_index=None, kv_count=None, coarse=None, w
 
 
 def forward_gated(q, k, v, kv_index, kv_count, p: Params, coarse: Coarse, gate, out=None, lse=None, ws=None,
-                  stream=None, with_f32: bool = False, out_f32=None):
-    """Fine stage then ``O = G * Repeat(Oc) + O_f``; returns (out, lse[, out_f32]) like :func:`forward`."""
+                  stream=None, out_f32=None):
+    """Fine stage then ``O = G * Repeat(Oc) + O_f``; returns (out, lse, out_f32).  The fp32
+    copy is always produced (the library forms the sum in fp32)."""
     torch = _torch()
     npad, T = geometry(p)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -369,7 +370,7 @@ def forward_gated(q, k, v, kv_index, kv_count, p: Params, coarse: Coarse, gate, 
         out = torch.empty((p.B, p.H, npad, p.D), dtype=torch.bfloat16, device=dev)
     if lse is None:
         lse = torch.empty((p.B, p.H, npad), dtype=torch.float32, device=dev)
-    if with_f32 and out_f32 is None:
+    if out_f32 is None:
         out_f32 = torch.empty((p.B, p.H, npad, p.D), dtype=torch.float32, device=dev)
     if ws is None:
         ws = new_workspace(p, OP_FORWARD, dev)
@@ -378,12 +379,13 @@ def forward_gated(q, k, v, kv_index, kv_count, p: Params, coarse: Coarse, gate, 
                                          ctypes.byref(cs), _ptr(gate), _ptr(out), _ptr(lse), _ptr(out_f32), _ptr(ws),
                                          ws.numel(), _stream(stream))
     _check(st, "sa_forward_gated")
-    return (out, lse, out_f32) if with_f32 else (out, lse)
+    return out, lse, out_f32
 
 
 def backward_gated(q, k, v, out, lse, dout, gate, kv_index, kv_count, p: Params, coarse: Coarse, dq=None, dk=None,
                    dv=None, dgate=None, ws=None, stream=None, out_f32=None):
-    """Gradients of the gated output: returns (dq, dk, dv, dgate), fp32."""
+    """Gradients of the gated output: returns (dq, dk, dv, dgate), fp32.  ``out_f32`` (the fp32
+    copy from :func:`forward_gated` with ``with_f32=True``) is required by the library."""
     torch = _torch()
     npad, T = geometry(p)
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):

@@ -352,7 +352,9 @@ sa_status backward_impl(const void* q, const void* k, const void* v, const void*
     return SA_ERR_ALIGNMENT;
   const bool gated = coarse != nullptr;
   if (gated) {
-    if (!gate || !dgate) return SA_ERR_INVALID_ARG;
+    // Delta of the fine branch is recovered from the combined output; from its bf16 rounding
+    // (2^-9 of |G Oc^ + O_f|) it misses the gradient bounds, so the fp32 copy is required
+    if (!gate || !dgate || !out_f32) return SA_ERR_INVALID_ARG;
     if ((s = check_coarse(coarse)) != SA_OK) return s;
     if (!aligned4(gate) || !aligned4(dgate)) return SA_ERR_ALIGNMENT;
     if (p->B * p->H > 65535) return SA_ERR_UNSUPPORTED;  // one grid layer per head
@@ -454,7 +456,9 @@ sa_status sa_forward_gated(const void* q, const void* k, const void* v, const in
   sa_status s = check_params(p, &g);
   if (s != SA_OK) return s;
   if (p->qk_dtype != SA_BF16) return SA_ERR_UNSUPPORTED;
-  if (!gate) return SA_ERR_INVALID_ARG;
+  // the sum is formed from the fine stage's fp32 output: a bf16 O_f rounded again after
+  // the sum misses the output error bounds
+  if (!gate || !out_f32) return SA_ERR_INVALID_ARG;
   if ((s = check_coarse(coarse)) != SA_OK) return s;
   if (!aligned4(gate)) return SA_ERR_ALIGNMENT;
   s = sa_forward(q, k, v, nullptr, nullptr, kv_index, kv_count, p, out, lse, out_f32, ws, ws_bytes, stream);

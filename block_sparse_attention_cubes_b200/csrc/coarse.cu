@@ -266,7 +266,8 @@ cudaError_t gemm(const GemmArgs& a, int batch, cudaStream_t stream) {
 
 // ------------------------------------------------------------------------ combine
 // O = G * Oc^[cube] + O_f on valid rows, in place on the bf16 output and, when present, its
-// fp32 copy (then the bf16 value is the rounded fp32 sum).  One thread per 4 columns of a row.
+// fp32 copy (then the bf16 value is the rounded fp32 sum; the C ABI always passes the copy).
+// One thread per 4 columns of a row.
 __global__ void __launch_bounds__(256) coarse_combine_kernel(__nv_bfloat16* __restrict__ out,
                                                              float* __restrict__ o32, const float* __restrict__ gate,
                                                              const float* __restrict__ oc, Geom g, int BH, int D) {

@@ -189,9 +189,11 @@ SA_API sa_status sa_plan_coarse(const void* q, const void* k, const void* v, con
                                 sa_stream_t stream);
 
 /* sa_forward (arguments, errors and outputs as there, bf16 only), then
- * O = G (.) Repeat_64(coarse->oc) + O_f written in place over out (and over out_f32 when
- * given: then out is the bf16 rounding of the fp32 sum).  gate: [B,H,Npad] fp32.  lse is
- * the fine stage's.  Workspace: sa_workspace_size(p, SA_OP_FORWARD).  Deterministic. */
+ * O = G (.) Repeat_64(coarse->oc) + O_f written in place over out_f32 and out (out is the
+ * bf16 rounding of the fp32 sum).  out_f32 is REQUIRED (SA_ERR_INVALID_ARG when NULL):
+ * summing into an already rounded bf16 O_f rounds twice, past the output error bounds.
+ * gate: [B,H,Npad] fp32.  lse is the fine stage's.  Workspace:
+ * sa_workspace_size(p, SA_OP_FORWARD).  Deterministic. */
 SA_API sa_status sa_forward_gated(const void* q, const void* k, const void* v, const int32_t* kv_index,
                                   const int32_t* kv_count, const sa_params* p, const sa_coarse* coarse,
                                   const float* gate, void* out, float* lse, float* out_f32, void* ws, size_t ws_bytes,
@@ -203,8 +205,9 @@ SA_API sa_status sa_forward_gated(const void* q, const void* k, const void* v, c
  *   dVc = Pc^T dOc^,  dPc = dOc^ Vc^T,  dSc = Pc (.) (dPc - rowsum(Pc (.) dPc)),
  *   dQc = scale dSc Kc,  dKc = scale dSc^T Qc,
  * each cube-level gradient handed to the n_i valid tokens of its cube as dXc[i] / n_i.
- * out / out_f32: the combined output from sa_forward_gated (the fine stage's Delta is taken
- * as <dO, O> - G dG).  coarse: as written by sa_plan_coarse (read only).  gate: [B,H,Npad]
+ * out / out_f32: the combined output from sa_forward_gated; out_f32 is REQUIRED here
+ * (SA_ERR_INVALID_ARG when NULL): the fine stage's Delta is taken as <dO, O> - G dG, and
+ * from the bf16 rounding of the combined O it exceeds the gradient error bounds.  coarse: as written by sa_plan_coarse (read only).  gate: [B,H,Npad]
  * fp32; dgate: [B,H,Npad] fp32 (0 on padding slots).  Workspace:
  * sa_workspace_size(p, SA_OP_BACKWARD_GATED).  Deterministic. */
 SA_API sa_status sa_backward_gated(const void* q, const void* k, const void* v, const void* out, const float* out_f32,

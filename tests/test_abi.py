@@ -112,7 +112,9 @@ def test_coarse_entry_points_validate_on_the_host(lib):
     # gated forward: gate required; the fine stage's checks follow
     assert lib.sa_forward_gated(bad, bad, bad, bad, bad, ctypes.byref(p), cref, None, bad, bad, None, bad, 1 << 30,
                                 None) == 1
-    assert lib.sa_forward_gated(bad, bad, bad, bad, bad, ctypes.byref(p), cref, bad, bad, bad, None, bad, 16,
+    assert lib.sa_forward_gated(bad, bad, bad, bad, bad, ctypes.byref(p), cref, bad, bad, bad, None, bad, 1 << 30,
+                                None) == 1                      # out_f32 is required
+    assert lib.sa_forward_gated(bad, bad, bad, bad, bad, ctypes.byref(p), cref, bad, bad, bad, bad, bad, 16,
                                 None) == 5
     # gated backward: coarse, gate and dgate required, the gated workspace size enforced
     args = [bad] * 10
@@ -120,6 +122,8 @@ def test_coarse_entry_points_validate_on_the_host(lib):
     args_nogate = [bad] * 7 + [None] + [bad] * 2
     assert lib.sa_backward_gated(*args_nogate, ctypes.byref(p), cref, bad, bad, bad, bad, bad, 1 << 30, None) == 1
     assert lib.sa_backward_gated(*args, ctypes.byref(p), cref, bad, bad, bad, bad, bad, bwd, None) == 5
+    args_no32 = [bad] * 4 + [None] + [bad] * 5                  # out_f32 is required
+    assert lib.sa_backward_gated(*args_no32, ctypes.byref(p), cref, bad, bad, bad, bad, bad, 1 << 30, None) == 1
     many = sa.make_params(1, 70000, 64, (4, 4, 4), 1, 0.5)      # B*H above one grid layer per head
     assert lib.sa_plan_coarse(bad, bad, bad, ctypes.byref(many), bad, bad, cref, bad, 1 << 40, None) == 2
     assert lib.sa_last_launch_count() == 0

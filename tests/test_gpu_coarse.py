@@ -68,9 +68,8 @@ def test_plan_coarse_lists_and_cube_tensors(case):
             _check_coarse(co, x, lay, b, h, f"b{b}h{h}")
 
 
-@pytest.mark.parametrize("with_f32", [True, False])
 @pytest.mark.parametrize("case", sorted(SMALL))
-def test_gated_forward_backward(case, with_f32):
+def test_gated_forward_backward(case):
     cfg = synth.small_config(*SMALL[case])
     x, p, t = gpu_inputs(cfg)
     gate = synth.make_gate(cfg).cuda()
@@ -84,9 +83,7 @@ def test_gated_forward_backward(case, with_f32):
             lists[(b, h)] = O.route_head(oracle_head(x, "q", b, h, lay), oracle_head(x, "k", b, h, lay), lay.valid,
                                          cfg.top_k, cfg.top_p).lists
     idx, cnt = lists_to_device(lists, cfg.B, cfg.H, T, p.kv_capacity)
-    r = sa.forward_gated(t["q"], t["k"], t["v"], idx, cnt, p, co, gate, with_f32=with_f32)
-    out, lse = r[0], r[1]
-    out32 = r[2] if with_f32 else None
+    out, lse, out32 = sa.forward_gated(t["q"], t["k"], t["v"], idx, cnt, p, co, gate)
     dq, dk, dv, dg = sa.backward_gated(t["q"], t["k"], t["v"], out, lse, t["do"], gate, idx, cnt, p, co,
                                        out_f32=out32)
     torch.cuda.synchronize()
@@ -100,10 +97,9 @@ def test_gated_forward_backward(case, with_f32):
             o = out[b, h].float().cpu().numpy()
             assert_close(f"out {tag}", o[lay.valid], o_ref[lay.valid])
             assert np.all(o[pad] == 0), tag
-            if with_f32:
-                assert_close(f"out_f32 {tag}", out32[b, h].cpu().numpy()[lay.valid], o_ref[lay.valid])
-                # the bf16 output is the rounding of the fp32 one
-                assert torch.equal(out[b, h], out32[b, h].to(torch.bfloat16))
+            assert_close(f"out_f32 {tag}", out32[b, h].cpu().numpy()[lay.valid], o_ref[lay.valid])
+            # the bf16 output is the rounding of the fp32 one
+            assert torch.equal(out[b, h], out32[b, h].to(torch.bfloat16))
             assert np.max(np.abs(lse[b, h].cpu().numpy()[lay.valid] - lse_ref[lay.valid])) < 1e-3
             grads = O.gated_backward_head(q, k, v, do, g, lists[(b, h)], lay.valid)
             for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), grads[:3]):
@@ -122,7 +118,7 @@ def test_zero_gate_reproduces_the_fine_stage():
     x, p, t = gpu_inputs(cfg)
     idx, cnt, co = sa.plan_coarse(t["q"], t["k"], t["v"], p)
     zero = torch.zeros((cfg.B, cfg.H, t["q"].shape[2]), dtype=torch.float32, device="cuda")
-    out_g, lse_g, o32_g = sa.forward_gated(t["q"], t["k"], t["v"], idx, cnt, p, co, zero, with_f32=True)
+    out_g, lse_g, o32_g = sa.forward_gated(t["q"], t["k"], t["v"], idx, cnt, p, co, zero)
     out_f, lse_f, o32_f = sa.forward(t["q"], t["k"], t["v"], idx, cnt, p, with_f32=True)
     torch.cuda.synchronize()
     assert torch.equal(out_g, out_f) and torch.equal(o32_g, o32_f) and torch.equal(lse_g, lse_f)
@@ -150,8 +146,7 @@ def test_720p_gated_sampled():
     t = {n: sa.tile(x[n].cuda(), p) for n in x}
     ws = {op: sa.new_workspace(p, op) for op in (sa.OP_PLAN_COARSE, sa.OP_FORWARD, sa.OP_BACKWARD_GATED)}
     idx, cnt, co = sa.plan_coarse(t["q"], t["k"], t["v"], p, ws=ws[sa.OP_PLAN_COARSE])
-    out, lse, out32 = sa.forward_gated(t["q"], t["k"], t["v"], idx, cnt, p, co, gate, ws=ws[sa.OP_FORWARD],
-                                       with_f32=True)
+    out, lse, out32 = sa.forward_gated(t["q"], t["k"], t["v"], idx, cnt, p, co, gate, ws=ws[sa.OP_FORWARD])
     dq, dk, dv, dg = sa.backward_gated(t["q"], t["k"], t["v"], out, lse, t["do"], gate, idx, cnt, p, co,
                                        ws=ws[sa.OP_BACKWARD_GATED], out_f32=out32)
     torch.cuda.synchronize()
