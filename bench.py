@@ -223,11 +223,12 @@ def run_ours(args, rank, world, dist):
     }
     if args.e2e_steps > 0:
         result["e2e"] = run_e2e(args, sa, A, p, host, dev, fwd_fl + bwd_fl, world, dist)
-    if args.config == "720p" and not (args.no_fp8 and args.no_gated):
+    run_fp8 = args.config == "720p" and not args.no_fp8
+    if run_fp8 or not args.no_gated:
         del x, A
-    if args.config == "720p" and not args.no_fp8:
+    if run_fp8:
         result["fp8_forward"] = run_fp8_forward(args, sa, synth, rank, dev, flush, peak_tf, peaks.get("hbm_gbs"), dist)
-    if args.config == "720p" and not args.no_gated:
+    if not args.no_gated:
         result["gated"] = run_gated(args, sa, synth, cfg, host, rank, dev, flush, result["breakdown_ms"], dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(cfg, host, seconds=args.cpu_seconds)
