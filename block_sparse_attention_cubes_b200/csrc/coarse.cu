@@ -16,9 +16,9 @@
 //   coarse_gate_bwd_kernel  one pass over dO: dG, the fine branch's Delta and -lse*log2(e),
 //                           dOc^ = sum_t G_t dO_t and delta_c = <dOc^, Oc^> per cube
 //
-// The cube-level matrices are T x T per head (T = 1440 at the 720p shape), so the products
-// here are about 1/2000 of the fine stage's work at 95% sparsity; they run on the fp32 FMA
-// pipe, which keeps the branch within fp32 rounding of the fp64 definition.
+// The cube-level matrices are T x T per head (T = 1440 at the 720p shape), so the six products
+// of a forward and backward are about 1/250 of the fine stage's FLOPs at 95% sparsity; they run
+// on the fp32 FMA pipe, which keeps the branch within fp32 rounding of the fp64 definition.
 #include <cuda_bf16.h>
 
 #include <cmath>
