@@ -14,6 +14,7 @@ Entry points mirror the C ABI in ``include/sa.h``:
 * :func:`plan_coarse`     router + coarse branch -> lists and a :class:`Coarse`
 * :func:`forward_gated`   fine stage, then ``O = G * Repeat(Oc) + O_f``
 * :func:`backward_gated`  -> ``dq, dk, dv`` (fine + coarse) and ``dgate``
+* :func:`recall`          router recall diagnostic from two forward lse's
 """
 from __future__ import annotations
 
@@ -36,7 +37,7 @@ DEBUG_SKIP_LOADS = 1
 # every symbol include/sa.h declares
 EXPORTS = ("sa_padded_tokens", "sa_num_cubes", "sa_topk_from_fraction", "sa_workspace_size", "sa_tile",
            "sa_untile", "sa_plan", "sa_forward", "sa_backward", "sa_get_device_status", "sa_status_string",
-           "sa_last_launch_count", "sa_plan_static", "sa_plan_coarse", "sa_forward_gated", "sa_backward_gated")
+           "sa_last_launch_count", "sa_plan_static", "sa_plan_coarse", "sa_forward_gated", "sa_backward_gated", "sa_recall")
 
 
 class SAError(RuntimeError):
@@ -89,6 +90,7 @@ def load_library(path: str = LIB_PATH):
         "sa_forward_gated": (i32, [vp, vp, vp, vp, vp, P, ctypes.POINTER(CoarseC), vp, vp, vp, vp, vp, sz, vp]),
         "sa_backward_gated": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, P, ctypes.POINTER(CoarseC), vp, vp, vp,
                                     vp, vp, sz, vp]),
+        "sa_recall": (i32, [vp, vp, P, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -414,6 +416,23 @@ def backward_gated(q, k, v, out, lse, dout, gate, kv_index, kv_count, p: Params,
                                           ws.numel(), _stream(stream))
     _check(st, "sa_backward_gated")
     return dq, dk, dv, dgate
+
+
+def recall(lse_kept, lse_all, p: Params, stream=None):
+    """Router recall: (tau per token [B,H,Npad], its mean per query cube [B,H,T]), fp32, with
+    tau = exp(lse_kept - lse_all) (lse of :func:`forward` on the router's lists and on lists
+    holding every block)."""
+    torch = _torch()
+    npad, T = geometry(p)
+    for t, n in ((lse_kept, "lse_kept"), (lse_all, "lse_all")):
+        _contig(t, n, torch.float32)
+        _shape(t, (p.B, p.H, npad), n)
+    tau = torch.empty((p.B, p.H, npad), dtype=torch.float32, device=lse_kept.device)
+    cube = torch.empty((p.B, p.H, T), dtype=torch.float32, device=lse_kept.device)
+    st = load_library().sa_recall(_ptr(lse_kept), _ptr(lse_all), ctypes.byref(p), _ptr(tau), _ptr(cube),
+                                  _stream(stream))
+    _check(st, "sa_recall")
+    return tau, cube
 
 
 @dataclass

@@ -480,6 +480,23 @@ sa_status sa_backward_gated(const void* q, const void* k, const void* v, const v
                        ws_bytes, stream);
 }
 
+sa_status sa_recall(const float* lse_kept, const float* lse_all, const sa_params* p, float* recall,
+                    float* cube_recall, sa_stream_t stream) {
+  Geom g;
+  g_last_launches = 0;
+  sa_status s = check_params(p, &g);
+  if (s != SA_OK) return s;
+  if (!lse_kept || !lse_all || (!recall && !cube_recall)) return SA_ERR_INVALID_ARG;
+  if (!aligned4(lse_kept) || !aligned4(lse_all) || (recall && !aligned4(recall)) ||
+      (cube_recall && !aligned4(cube_recall)))
+    return SA_ERR_ALIGNMENT;
+  if (sa::launch_recall(lse_kept, lse_all, recall, cube_recall, g, p->B * p->H,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SA_ERR_LAUNCH;
+  g_last_launches = 1;
+  return SA_OK;
+}
+
 sa_status sa_get_device_status(const void* ws, sa_stream_t stream) {
   if (!ws) return SA_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SA_ERR_LAUNCH;

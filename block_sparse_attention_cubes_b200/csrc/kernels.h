@@ -85,4 +85,9 @@ cudaError_t launch_coarse_backward(const void* out, const float* out_f32, const 
                                    float* nlse2, const CoarseGradWs& w, float scale, const Geom& g, int BH, int D,
                                    cudaStream_t stream, int* launches);
 
+// tau = exp(lse_kept - lse_all) per valid row (0 on padding) into recall, and its mean over each
+// cube's valid rows into cube_recall; either output may be NULL.
+cudaError_t launch_recall(const float* lse_kept, const float* lse_all, float* recall, float* cube_recall,
+                          const Geom& g, int BH, cudaStream_t stream);
+
 }  // namespace sa

@@ -215,6 +215,17 @@ SA_API sa_status sa_backward_gated(const void* q, const void* k, const void* v, 
                                    const int32_t* kv_count, const sa_params* p, const sa_coarse* coarse, float* dq,
                                    float* dk, float* dv, float* dgate, void* ws, size_t ws_bytes, sa_stream_t stream);
 
+/* Router recall diagnostic (SpargeAttention2 page, equation 8: tau = sum_j p_j m_j, the share of a
+ * query's true softmax mass inside its kept blocks; VSA page, "Kernel Implementation": Top-32
+ * keeps 50-90%).  Since lse is the log of a row's softmax normaliser, tau = exp(lse_kept -
+ * lse_all), with lse_kept from sa_forward on the router's lists and lse_all from sa_forward on
+ * lists holding every block (kv_capacity = T).  lse_kept, lse_all: [B,H,Npad] fp32.
+ * recall: [B,H,Npad] fp32, tau per valid row, 0 on padding rows (may be NULL).
+ * cube_recall: [B,H,T] fp32, the mean of tau over each cube's valid rows (may be NULL; not both).
+ * Asynchronous, one launch, no workspace.  Deterministic. */
+SA_API sa_status sa_recall(const float* lse_kept, const float* lse_all, const sa_params* p, float* recall,
+                           float* cube_recall, sa_stream_t stream);
+
 /* sa_plan without a workspace: the same router and the same results, for callers that
  * cannot allocate device memory (code running under a CUDA stream capture, serving
  * processes confined to a pre-reserved memory arena, C callers with no device

@@ -127,3 +127,12 @@ def test_coarse_entry_points_validate_on_the_host(lib):
     many = sa.make_params(1, 70000, 64, (4, 4, 4), 1, 0.5)      # B*H above one grid layer per head
     assert lib.sa_plan_coarse(bad, bad, bad, ctypes.byref(many), bad, bad, cref, bad, 1 << 40, None) == 2
     assert lib.sa_last_launch_count() == 0
+
+
+def test_recall_validates_on_the_host(lib):
+    p = sa.make_params(1, 2, 64, (8, 8, 8), 4, 0.5)
+    bad = ctypes.c_void_p(16)
+    assert lib.sa_recall(bad, bad, ctypes.byref(p), None, None, None) == 1      # no output
+    assert lib.sa_recall(None, bad, ctypes.byref(p), bad, bad, None) == 1
+    assert lib.sa_recall(bad, ctypes.c_void_p(18), ctypes.byref(p), bad, None, None) == 3
+    assert lib.sa_last_launch_count() == 0
