@@ -15,6 +15,7 @@ Entry points mirror the C ABI in ``include/sa.h``:
 * :func:`forward_gated`   fine stage, then ``O = G * Repeat(Oc) + O_f``
 * :func:`backward_gated`  -> ``dq, dk, dv`` (fine + coarse) and ``dgate``
 * :func:`recall`          router recall diagnostic from two forward lse's
+* :func:`plan_bq128`      router with 128-token query blocks (cube pairs)
 """
 from __future__ import annotations
 
@@ -30,14 +31,14 @@ SA_OK = 0
 STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_ALIGNMENT",
                 4: "SA_ERR_CAPACITY", 5: "SA_ERR_WORKSPACE", 6: "SA_ERR_LAUNCH", 7: "SA_ERR_DEVICE_TIMEOUT",
                 8: "SA_ERR_DEVICE_INDEX"}
-OP_PLAN, OP_FORWARD, OP_BACKWARD, OP_PLAN_COARSE, OP_BACKWARD_GATED = 0, 1, 2, 3, 4
+OP_PLAN, OP_FORWARD, OP_BACKWARD, OP_PLAN_COARSE, OP_BACKWARD_GATED, OP_PLAN_BQ128 = 0, 1, 2, 3, 4, 5
 BF16, FP8_E4M3 = 0, 1
 DEBUG_SKIP_LOADS = 1
 
 # every symbol include/sa.h declares
 EXPORTS = ("sa_padded_tokens", "sa_num_cubes", "sa_topk_from_fraction", "sa_workspace_size", "sa_tile",
            "sa_untile", "sa_plan", "sa_forward", "sa_backward", "sa_get_device_status", "sa_status_string",
-           "sa_last_launch_count", "sa_plan_static", "sa_plan_coarse", "sa_forward_gated", "sa_backward_gated", "sa_recall")
+           "sa_last_launch_count", "sa_plan_static", "sa_plan_coarse", "sa_forward_gated", "sa_backward_gated", "sa_recall", "sa_plan_bq128")
 
 
 class SAError(RuntimeError):
@@ -91,6 +92,7 @@ def load_library(path: str = LIB_PATH):
         "sa_backward_gated": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, P, ctypes.POINTER(CoarseC), vp, vp, vp,
                                     vp, vp, sz, vp]),
         "sa_recall": (i32, [vp, vp, P, vp, vp, vp]),
+        "sa_plan_bq128": (i32, [vp, vp, P, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -416,6 +418,26 @@ def backward_gated(q, k, v, out, lse, dout, gate, kv_index, kv_count, p: Params,
                                           ws.numel(), _stream(stream))
     _check(st, "sa_backward_gated")
     return dq, dk, dv, dgate
+
+
+def plan_bq128(q, k, p: Params, kv_index=None, kv_count=None, ws=None, stream=None):
+    """Router with 128-token query blocks (cube pairs): per-cube lists like :func:`plan`, both
+    cubes of a block holding the block's list."""
+    torch = _torch()
+    _token_tensor(q, p, "q", 2)
+    _token_tensor(k, p, "k", 2)
+    _, T = geometry(p)
+    dev = q.device
+    if kv_index is None:
+        kv_index = torch.empty((p.B, p.H, T, p.kv_capacity), dtype=torch.int32, device=dev)
+    if kv_count is None:
+        kv_count = torch.empty((p.B, p.H, T), dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = new_workspace(p, OP_PLAN_BQ128, dev)
+    st = load_library().sa_plan_bq128(_ptr(q), _ptr(k), ctypes.byref(p), _ptr(kv_index), _ptr(kv_count), _ptr(ws),
+                                      ws.numel(), _stream(stream))
+    _check(st, "sa_plan_bq128")
+    return kv_index, kv_count
 
 
 def recall(lse_kept, lse_all, p: Params, stream=None):

@@ -66,12 +66,27 @@ struct WsLayout {
   size_t p32 = 0;                                          // plan + coarse: Pc [BH, T, T] fp32
   size_t doc = 0, dltc = 0, s32 = 0, ds32 = 0;             // gated backward: coarse scratch
   size_t cq = 0, ck = 0, cv = 0;
+  size_t qpair = 0, blk_index = 0, blk_count = 0;          // plan with 128-token query blocks
   size_t total = 0;
 };
 
 WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
   WsLayout w;
   const size_t BH = static_cast<size_t>(p->B) * p->H;
+  if (op == SA_OP_PLAN_BQ128) {
+    // the plan's (the score rows of the first ceil(T/2) blocks are used), then the block means and lists
+    w = ws_layout(p, g, SA_OP_PLAN);
+    const size_t M = static_cast<size_t>((g.T + 1) / 2);
+    size_t off = w.total;
+    w.qpair = off;
+    off = align256(off + BH * M * p->D * sizeof(double));
+    w.blk_count = off;
+    off = align256(off + BH * M * sizeof(int32_t));
+    w.blk_index = off;
+    off = align256(off + BH * M * static_cast<size_t>(p->kv_capacity) * sizeof(int32_t));
+    w.total = off;
+    return w;
+  }
   if (op == SA_OP_PLAN_COARSE || op == SA_OP_BACKWARD_GATED) {
     // the plain layout, then the coarse branch's buffers
     w = ws_layout(p, g, op == SA_OP_PLAN_COARSE ? SA_OP_PLAN : SA_OP_BACKWARD);
@@ -213,7 +228,7 @@ int sa_topk_from_fraction(double frac, int T) {
 
 size_t sa_workspace_size(const sa_params* p, int op) {
   Geom g;
-  if (check_params(p, &g) != SA_OK || op < SA_OP_PLAN || op > SA_OP_BACKWARD_GATED) return 0;
+  if (check_params(p, &g) != SA_OK || op < SA_OP_PLAN || op > SA_OP_PLAN_BQ128) return 0;
   return ws_layout(p, g, op).total;
 }
 
@@ -478,6 +493,34 @@ sa_status sa_backward_gated(const void* q, const void* k, const void* v, const v
   if (!coarse) return SA_ERR_INVALID_ARG;
   return backward_impl(q, k, v, out, out_f32, lse, dout, gate, kv_index, kv_count, p, coarse, dq, dk, dv, dgate, ws,
                        ws_bytes, stream);
+}
+
+sa_status sa_plan_bq128(const void* q, const void* k, const sa_params* p, int32_t* kv_index, int32_t* kv_count,
+                        void* ws, size_t ws_bytes, sa_stream_t stream) {
+  Geom g;
+  g_last_launches = 0;
+  sa_status s = check_params(p, &g);
+  if (s != SA_OK) return s;
+  if (!q || !k || !kv_index || !kv_count) return SA_ERR_INVALID_ARG;
+  if (p->qk_dtype != SA_BF16) return SA_ERR_UNSUPPORTED;
+  if (p->B * p->H > 65535) return SA_ERR_UNSUPPORTED;  // one grid layer per head
+  if (!aligned16(q) || !aligned16(k) || !aligned4(kv_index) || !aligned4(kv_count)) return SA_ERR_ALIGNMENT;
+  const WsLayout w = ws_layout(p, g, SA_OP_PLAN_BQ128);
+  if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SA_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  int launches = 0;
+  if (sa::launch_plan_bq128(q, k, g, p->B * p->H, p->D, softmax_scale(p), p->top_k, p->top_p, p->kv_capacity,
+                            kv_index, kv_count, reinterpret_cast<double*>(wb + w.qbar),
+                            reinterpret_cast<double*>(wb + w.kbar), reinterpret_cast<double*>(wb + w.qpair),
+                            reinterpret_cast<double*>(wb + w.scores), reinterpret_cast<int32_t*>(wb + w.blk_index),
+                            reinterpret_cast<int32_t*>(wb + w.blk_count), static_cast<sa::DevStatus*>(ws), st,
+                            &launches) != cudaSuccess)
+    return SA_ERR_LAUNCH;
+  g_last_launches = launches;
+  return SA_OK;
 }
 
 sa_status sa_recall(const float* lse_kept, const float* lse_all, const sa_params* p, float* recall,

@@ -85,6 +85,18 @@ cudaError_t launch_coarse_backward(const void* out, const float* out_f32, const 
                                    float* nlse2, const CoarseGradWs& w, float scale, const Geom& g, int BH, int D,
                                    cudaStream_t stream, int* launches);
 
+// The cube router's pooling (bf16) and selection passes on their own.
+cudaError_t launch_pool(const void* q, const void* k, const Geom& g, int BH, int D, double* qbar, double* kbar,
+                        cudaStream_t stream);
+cudaError_t launch_select(const double* S, int32_t* kv_index, int32_t* kv_count, int rows, int T, int top_k,
+                          float top_p, int cap, DevStatus* st, cudaStream_t stream);
+// Router with 128-token query blocks (cube pairs); writes each block's list for both its cubes
+// (5 launches).  qpair [BH, ceil(T/2), D] fp64, S [BH, ceil(T/2), T] fp64, blk_* the block lists.
+cudaError_t launch_plan_bq128(const void* q, const void* k, const Geom& g, int BH, int D, double scale, int top_k,
+                              float top_p, int cap, int32_t* kv_index, int32_t* kv_count, double* qbar, double* kbar,
+                              double* qpair, double* S, int32_t* blk_index, int32_t* blk_count, DevStatus* st,
+                              cudaStream_t stream, int* launches);
+
 // tau = exp(lse_kept - lse_all) per valid row (0 on padding) into recall, and its mean over each
 // cube's valid rows into cube_recall; either output may be NULL.
 cudaError_t launch_recall(const float* lse_kept, const float* lse_all, float* recall, float* cube_recall,

@@ -412,4 +412,20 @@ cudaError_t launch_plan(const void* q, const void* k, const float* q_scale, cons
   return cudaGetLastError();
 }
 
+// The pooling and selection passes on their own, for routers that score a different matrix
+// (bf16 Q and K; the same kernels and launch shapes as launch_plan).
+cudaError_t launch_pool(const void* q, const void* k, const Geom& g, int BH, int D, double* qbar, double* kbar,
+                        cudaStream_t stream) {
+  dim3 pg((g.T + 3) / 4, BH, 2);
+  pool_kernel<2><<<pg, 256, 0, stream>>>(static_cast<const uint8_t*>(q), static_cast<const uint8_t*>(k), nullptr,
+                                         nullptr, qbar, kbar, g, D);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const double* S, int32_t* kv_index, int32_t* kv_count, int rows, int T, int top_k,
+                          float top_p, int cap, DevStatus* st, cudaStream_t stream) {
+  select_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(S, kv_index, kv_count, rows, T, top_k, top_p, cap, st);
+  return cudaGetLastError();
+}
+
 }  // namespace sa

@@ -61,7 +61,8 @@ typedef enum {
   SA_OP_FORWARD = 1,          /* also sa_forward_gated */
   SA_OP_BACKWARD = 2,
   SA_OP_PLAN_COARSE = 3,      /* sa_plan_coarse */
-  SA_OP_BACKWARD_GATED = 4    /* sa_backward_gated */
+  SA_OP_BACKWARD_GATED = 4,   /* sa_backward_gated */
+  SA_OP_PLAN_BQ128 = 5        /* sa_plan_bq128 */
 } sa_op;
 
 typedef struct {
@@ -214,6 +215,18 @@ SA_API sa_status sa_backward_gated(const void* q, const void* k, const void* v, 
                                    const float* lse, const void* dout, const float* gate, const int32_t* kv_index,
                                    const int32_t* kv_count, const sa_params* p, const sa_coarse* coarse, float* dq,
                                    float* dk, float* dv, float* dgate, void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* Router with 128-token query blocks and 64-token key blocks (SpargeAttention2 page,
+ * "Block-Pooled Attention for Efficient Mask Construction" step 1: b_q = 128, b_kv = 64 in all
+ * its experiments).  On the cube layout query block i is cubes 2i and 2i+1 (the last block is
+ * one cube when T is odd), pooled over the valid tokens of both; keys stay per cube.  Scores,
+ * row softmax, Top-k / Top-p and ties as sa_plan, over the ceil(T/2) x T block matrix (top_k
+ * counts key cubes).  Output in sa_plan's per-cube layout, kv_index [B,H,T,kv_capacity] and
+ * kv_count [B,H,T], with both cubes of a block holding the block's list, so sa_forward and
+ * sa_backward take it as is.  bf16 only.  B*H <= 65535.  Workspace:
+ * sa_workspace_size(p, SA_OP_PLAN_BQ128).  Deterministic. */
+SA_API sa_status sa_plan_bq128(const void* q, const void* k, const sa_params* p, int32_t* kv_index, int32_t* kv_count,
+                               void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /* Router recall diagnostic (SpargeAttention2 page, equation 8: tau = sum_j p_j m_j, the share of a
  * query's true softmax mass inside its kept blocks; VSA page, "Kernel Implementation": Top-32

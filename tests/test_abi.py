@@ -95,7 +95,7 @@ def test_coarse_entry_points_validate_on_the_host(lib):
     # plan + Pc; backward + dOc^, three per-cube terms, delta_c, scores and dS (each 256-byte aligned)
     assert sa.workspace_size(p, sa.OP_PLAN_COARSE) >= plan + BH * T * T * 4
     assert sa.workspace_size(p, sa.OP_BACKWARD_GATED) >= bwd + 4 * BH * T * D * 4 + BH * T * 4 + 2 * BH * T * T * 4
-    assert sa.workspace_size(p, 5) == 0
+    assert sa.workspace_size(p, 6) == 0
     bad = ctypes.c_void_p(16)
     c = sa.CoarseC(16, 16, 16, 16, 16)
     cref = ctypes.byref(c)
@@ -135,4 +135,20 @@ def test_recall_validates_on_the_host(lib):
     assert lib.sa_recall(bad, bad, ctypes.byref(p), None, None, None) == 1      # no output
     assert lib.sa_recall(None, bad, ctypes.byref(p), bad, bad, None) == 1
     assert lib.sa_recall(bad, ctypes.c_void_p(18), ctypes.byref(p), bad, None, None) == 3
+    assert lib.sa_last_launch_count() == 0
+
+
+def test_plan_bq128_validates_on_the_host(lib):
+    p = sa.make_params(1, 2, 64, (8, 8, 12), 4, 0.5)          # T = 12: 6 query blocks
+    T, BH, M, D = 12, 2, 6, 64
+    plan = sa.workspace_size(p, sa.OP_PLAN)
+    # the plan's, then the block means (fp64) and the block lists and counts
+    assert sa.workspace_size(p, sa.OP_PLAN_BQ128) >= plan + BH * M * D * 8 + BH * M * (T + 1) * 4
+    bad = ctypes.c_void_p(16)
+    assert lib.sa_plan_bq128(None, bad, ctypes.byref(p), bad, bad, bad, 1 << 30, None) == 1
+    assert lib.sa_plan_bq128(bad, bad, ctypes.byref(p), bad, bad, bad, plan, None) == 5
+    fp8 = sa.make_params(1, 2, 128, (8, 8, 12), 4, 0.5, qk_dtype=sa.FP8_E4M3)
+    assert lib.sa_plan_bq128(bad, bad, ctypes.byref(fp8), bad, bad, bad, 1 << 30, None) == 2
+    many = sa.make_params(1, 70000, 64, (4, 4, 4), 1, 0.5)
+    assert lib.sa_plan_bq128(bad, bad, ctypes.byref(many), bad, bad, bad, 1 << 40, None) == 2
     assert lib.sa_last_launch_count() == 0
