@@ -9,6 +9,9 @@ forward 4*D*64*64 and backward 10*D*64*64 FLOPs per selected tile (VSA page, FLO
 accounting: 4 * D * S * H * d * 3.5, i.e. forward 1 + backward 2.5).  Each rank runs an
 independent problem of the same shape (weak scaling, no collective on the data path).
 Inputs are larger than L2 and L2 is also flushed between steps (256 MiB write).
+Extra sections on the same line: ``fp8_forward`` (e4m3 Q/K configuration, 720p only) and
+``gated`` (the coarse branch + gate layer: sa_plan_coarse, sa_forward_gated,
+sa_backward_gated), skipped with ``--no-fp8`` / ``--no-gated``.
 """
 from __future__ import annotations
 
