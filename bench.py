@@ -233,6 +233,8 @@ def run_ours(args, rank, world, dist):
         result["fp8_forward"] = run_fp8_forward(args, sa, synth, rank, dev, flush, peak_tf, peaks.get("hbm_gbs"), dist)
     if not args.no_gated:
         result["gated"] = run_gated(args, sa, synth, cfg, host, rank, dev, flush, result["breakdown_ms"], dist)
+    if args.extras:
+        result["extras"] = run_extras(args, sa, cfg, host, dev, flush, dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(cfg, host, seconds=args.cpu_seconds)
     return result
@@ -374,6 +376,73 @@ def run_gated(args, sa, synth, cfg, host, rank, dev, flush, plain_ms, dist):
             "gpu_launches_per_step": launches["n"] // steps,
             "per_step_ms": {n: [round(v, 3) for v in vals]
                             for n, vals in zip(("plan_coarse", "forward_gated", "backward_gated"), per_step)}}
+
+
+def run_extras(args, sa, cfg, host, dev, flush, dist):
+    """The other routers at the same shape (off by default, ``--extras``): sa_plan_bq128
+    (128-token query blocks) timed with the fine forward and backward on its lists, like the
+    main step; and the recall diagnostic, sa_recall on the lse of the forward with the cube
+    router's lists and with every block (the dense forward is not timed), with its result."""
+    import torch
+    p = sa.make_params(cfg.B, cfg.H, cfg.D, cfg.lat, cfg.top_k, cfg.top_p)
+    npad, T = sa.geometry(p)
+    t = {n: sa.tile(host[n].to(dev), p) for n in ("q", "k", "v", "do")}
+    ws = {op: sa.new_workspace(p, op, dev) for op in (sa.OP_PLAN_BQ128, sa.OP_FORWARD, sa.OP_BACKWARD)}
+
+    def step(rec=None):
+        if rec is not None:
+            rec[0].record()
+        idx, cnt = sa.plan_bq128(t["q"], t["k"], p, ws=ws[sa.OP_PLAN_BQ128])
+        if rec is not None:
+            rec[1].record()
+        out, lse, o32 = sa.forward(t["q"], t["k"], t["v"], idx, cnt, p, ws=ws[sa.OP_FORWARD], with_f32=True)
+        if rec is not None:
+            rec[2].record()
+        sa.backward(t["q"], t["k"], t["v"], out, lse, t["do"], idx, cnt, p, ws=ws[sa.OP_BACKWARD], out_f32=o32)
+        if rec is not None:
+            rec[3].record()
+        return cnt
+
+    for _ in range(max(3, args.warmup)):
+        cnt = step()
+    torch.cuda.synchronize()
+    for op, w in ws.items():
+        st = sa.device_status(w)
+        if st != 0:
+            raise RuntimeError(f"extras: device status {sa.STATUS_NAMES.get(st, st)} (op {op})")
+    ntiles = int(cnt.sum().item())
+    steps = max(3, min(args.steps, 5))
+    recs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for s in range(steps):
+        flush.fill_(s & 0xff)
+        step(recs[s])
+    torch.cuda.synchronize()
+    ms = [statistics.mean(r[i].elapsed_time(r[i + 1]) for r in recs) for i in range(3)]
+    fwd_fl, bwd_fl = tile_flops(cfg.D, ntiles)
+    bq = {"plan_ms": round(ms[0], 4), "forward_ms": round(ms[1], 4), "backward_ms": round(ms[2], 4),
+          "selected_tiles": ntiles, "density": round(ntiles / (cfg.B * cfg.H * T * T), 5),
+          "effective_tflops": round((fwd_fl + bwd_fl) / (sum(ms) * 1e-3) / 1e12, 3)}
+    # recall of the cube router's selection
+    idx, cnt = sa.plan(t["q"], t["k"], p)
+    _, lse_kept = sa.forward(t["q"], t["k"], t["v"], idx, cnt, p)
+    every = torch.arange(T, dtype=torch.int32, device=dev).expand(cfg.B, cfg.H, T, T).contiguous()
+    full = torch.full((cfg.B, cfg.H, T), T, dtype=torch.int32, device=dev)
+    _, lse_all = sa.forward(t["q"], t["k"], t["v"], every, full, p)
+    del every
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    sa.recall(lse_kept, lse_all, p)
+    ev[0].record()
+    tau, cube = sa.recall(lse_kept, lse_all, p)
+    ev[1].record()
+    torch.cuda.synchronize()
+    cube_cpu = cube.float().cpu()
+    rec = {"recall_ms": round(ev[0].elapsed_time(ev[1]), 4), "mean_cube_recall": round(float(cube_cpu.mean()), 4),
+           "min_cube_recall": round(float(cube_cpu.min()), 4),
+           "cubes_below_half": round(float((cube_cpu < 0.5).float().mean()), 4),
+           "mean_blocks_per_row": round(float(cnt.float().mean()), 2)}
+    return {"config": f"{cfg.name}: sa_plan_bq128 + fine stage on its lists; recall of sa_plan's lists",
+            "steps": steps, "bq128": bq, "recall": rec}
 
 
 def cta_balance(masks, sms: int):
@@ -658,6 +727,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the e4m3 Q/K forward section")
     ap.add_argument("--no-gated", action="store_true", help="skip the gated (coarse + fine) layer section")
+    ap.add_argument("--extras", action="store_true",
+                    help="also time the 128-token query-block router and the recall diagnostic")
     ap.add_argument("--sweep", action="store_true",
                     help="config-4 sweep (k=4, p x sparsity grid): one JSON line per point with load balance")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
