@@ -365,7 +365,10 @@ def run_gated(args, sa, synth, cfg, host, rank, dev, flush, plain_ms, dist):
     fwd_fl, bwd_fl = tile_flops(cfg.D, ntiles)
     cube_fl = 2.0 * cfg.B * cfg.H * T * T * cfg.D      # one cube-level product
     total_ms = sum(ms)
-    return {"config": f"{cfg.name}: O = G * Repeat(Oc) + O_f, gates tanh(N(0,1)), fp32 out kept",
+    extra = {}
+    if dist is None and not args.no_cpu_baseline:
+        extra["cpu_baseline"] = cpu_baseline_gated(cfg, host, gate.cpu(), seconds=args.cpu_seconds)
+    return {**extra, "config": f"{cfg.name}: O = G * Repeat(Oc) + O_f, gates tanh(N(0,1)), fp32 out kept",
             "steps": steps, "selected_tiles": ntiles,
             "plan_coarse_ms": round(ms[0], 4), "forward_gated_ms": round(ms[1], 4),
             "backward_gated_ms": round(ms[2], 4), "ms_per_step": round(total_ms, 4),
@@ -666,6 +669,40 @@ def oracle_sample(cfg, host, head: int, frac: float, seed: int = 0):
     ntiles = sum(len(tr.lists[i]) for i in sample)
     f, b = tile_flops(cfg.D, ntiles)
     return secs, f + b, len(sample)
+
+
+def oracle_gated_sample(cfg, host, gate, head: int, frac: float, seed: int = 0):
+    """The fp64 oracle's gated layer on one head: the full router and cube-level branch,
+    the fine forward and backward on a fixed sample of query blocks (as ``oracle_sample``).
+    Returns (seconds, effective FLOPs: the sampled tiles plus the six cube-level products)."""
+    import numpy as np
+
+    import oracle as O
+    lay = O.cube_layout(cfg.lat)
+    t = {n: O.tile(host[n][0, head].double().numpy(), lay) for n in ("q", "k", "v", "do")}
+    g = gate[0, head].double().numpy()
+    T = lay.n_cubes
+    rng = np.random.default_rng(seed)
+    sample = np.sort(rng.choice(T, size=max(1, int(round(frac * T))), replace=False))
+    t0 = time.perf_counter()
+    tr = O.route_head(t["q"], t["k"], lay.valid, cfg.top_k, cfg.top_p)
+    O.gated_forward_head(t["q"], t["k"], t["v"], g, tr.lists, lay.valid, q_blocks=sample)
+    O.gated_backward_head(t["q"], t["k"], t["v"], t["do"], g, tr.lists, lay.valid, q_blocks=sample,
+                          kv_blocks=range(T), visit=sample)
+    secs = time.perf_counter() - t0
+    ntiles = sum(len(tr.lists[i]) for i in sample)
+    f, b = tile_flops(cfg.D, ntiles)
+    return secs, f + b + 6 * 2.0 * T * T * cfg.D, len(sample)
+
+
+def cpu_baseline_gated(cfg, host, gate, seconds: float = 15.0):
+    s0, _, _ = oracle_gated_sample(cfg, host, gate, head=0, frac=0.02)
+    frac = min(1.0, max(0.02, 0.02 * seconds / max(s0, 1e-3)))
+    secs, flops, n = oracle_gated_sample(cfg, host, gate, head=0, frac=frac, seed=1)
+    T = (cfg.lat[0] + 3) // 4 * ((cfg.lat[1] + 3) // 4) * ((cfg.lat[2] + 3) // 4)
+    return {"value": round(flops / secs / 1e12, 6), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"head 0 of {cfg.name}: full fp64 router and coarse branch, gated forward and backward of "
+                      f"{n} of {T} query cubes ({secs:.1f} s)"}
 
 
 def cpu_cores():

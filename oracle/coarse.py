@@ -80,7 +80,8 @@ def gated_forward_head(q, k, v, gate, lists, valid, scale=None, block=64, q_bloc
     return o, o_f, lse, coarse
 
 
-def gated_backward_head(q, k, v, do, gate, lists, valid, scale=None, block=64, q_blocks=None, kv_blocks=None):
+def gated_backward_head(q, k, v, do, gate, lists, valid, scale=None, block=64, q_blocks=None, kv_blocks=None,
+                        visit=None):
     """dQ, dK, dV (fine plus coarse) and dG of L = <dO, O>, O as in :func:`gated_forward_head`.
 
     Fine branch: its output enters O with weight 1, so it takes dO as is.
@@ -89,14 +90,14 @@ def gated_backward_head(q, k, v, do, gate, lists, valid, scale=None, block=64, q
         dV_c = P_c^T dO^_c;          dP_c = dO^_c V_c^T
         dS_c = P_c (.) (dP_c - rowsum(P_c (.) dP_c))
         dQ_c = scale dS_c K_c;       dK_c = scale dS_c^T Q_c
-    and each valid token of cube i receives dX_c[i] / n_i.  ``q_blocks`` / ``kv_blocks``
-    restrict the fine branch's dQ rows / dK, dV rows as in :func:`attention_backward_head`
-    (the cube-level part is always complete).
+    and each valid token of cube i receives dX_c[i] / n_i.  ``q_blocks`` / ``kv_blocks`` /
+    ``visit`` restrict the fine branch's dQ rows / dK, dV rows / visited query blocks as in
+    :func:`attention_backward_head` (the cube-level part is always complete).
     """
     n_pad, D = q.shape
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     T = n_pad // block
-    dq, dk, dv = attention_backward_head(q, k, v, do, lists, valid, scale, block, q_blocks, kv_blocks)
+    dq, dk, dv = attention_backward_head(q, k, v, do, lists, valid, scale, block, q_blocks, kv_blocks, visit)
     qbar, kbar, vbar, oc_hat, _, P = coarse_forward_head(q, k, v, valid, scale, block)
     g = np.asarray(gate, np.float64) * valid
     dgate = (do * repeat_cubes(oc_hat, valid, block)).sum(axis=1)
