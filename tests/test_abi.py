@@ -152,3 +152,41 @@ def test_plan_bq128_validates_on_the_host(lib):
     many = sa.make_params(1, 70000, 64, (4, 4, 4), 1, 0.5)
     assert lib.sa_plan_bq128(bad, bad, ctypes.byref(many), bad, bad, bad, 1 << 40, None) == 2
     assert lib.sa_last_launch_count() == 0
+
+
+def test_fine_stage_layout_and_static_plan_validate_on_the_host(lib):
+    """Error paths of sa_forward, sa_backward, sa_tile / sa_untile, sa_plan_static and
+    sa_get_device_status that return before anything touches the device."""
+    p = sa.make_params(1, 2, 64, (8, 8, 8), 4, 0.5)            # T = 8
+    P = ctypes.byref(p)
+    bad, odd = ctypes.c_void_p(16), ctypes.c_void_p(24)
+    big = 1 << 30
+    # sa_forward(q, k, v, q_scale, k_scale, kv_index, kv_count, p, out, lse, out_f32, ws, ws_bytes, stream)
+    assert lib.sa_forward(bad, bad, None, None, None, bad, bad, P, bad, bad, None, bad, big, None) == 1
+    assert lib.sa_forward(bad, bad, odd, None, None, bad, bad, P, bad, bad, None, bad, big, None) == 3
+    assert lib.sa_forward(bad, bad, bad, None, None, bad, bad, P, bad, bad, odd, bad, big, None) == 3
+    assert lib.sa_forward(bad, bad, bad, None, None, bad, bad, P, bad, bad, None, bad, 16, None) == 5
+    f8 = sa.make_params(1, 2, 64, (8, 8, 8), 4, 0.5, qk_dtype=sa.FP8_E4M3)
+    assert lib.sa_forward(bad, bad, bad, bad, bad, bad, bad, ctypes.byref(f8), bad, bad, None, bad, big, None) == 2
+    f8d = sa.make_params(1, 2, 128, (8, 8, 8), 4, 0.5, qk_dtype=sa.FP8_E4M3)
+    assert lib.sa_forward(bad, bad, bad, None, bad, bad, bad, ctypes.byref(f8d), bad, bad, None, bad, big, None) == 1
+    # sa_backward(q, k, v, out, out_f32, lse, dout, kv_index, kv_count, p, dq, dk, dv, ws, ws_bytes, stream)
+    assert lib.sa_backward(bad, bad, bad, bad, None, bad, bad, bad, bad, P, None, bad, bad, bad, big, None) == 1
+    assert lib.sa_backward(bad, bad, bad, bad, None, bad, odd, bad, bad, P, bad, bad, bad, bad, big, None) == 3
+    assert lib.sa_backward(bad, bad, bad, bad, None, bad, bad, bad, bad, P, bad, bad, bad, bad, 16, None) == 5
+    assert lib.sa_backward(bad, bad, bad, bad, None, bad, bad, bad, bad, ctypes.byref(f8d), bad, bad, bad, bad,
+                           big, None) == 2
+    # sa_tile / sa_untile(src, dst, p, elem_bytes, stream)
+    assert lib.sa_tile(bad, bad, P, 3, None) == 1                # element size not 1, 2 or 4
+    assert lib.sa_tile(None, bad, P, 2, None) == 1
+    p4 = sa.make_params(1, 2, 4, (8, 8, 8), 4, 0.5)             # 8-byte rows: not a multiple of 16
+    assert lib.sa_untile(bad, bad, ctypes.byref(p4), 2, None) == 2
+    assert lib.sa_untile(bad, odd, P, 2, None) == 3
+    # sa_plan_static(q, k, q_scale, k_scale, p, kv_index, kv_count, stream)
+    pc = sa.make_params(1, 2, 64, (8, 8, 8), 4, 0.5, kv_capacity=4)
+    assert lib.sa_plan_static(bad, bad, None, None, ctypes.byref(pc), bad, bad, None) == 1   # capacity != T
+    assert lib.sa_plan_static(odd, bad, None, None, P, bad, bad, None) == 3
+    huge = sa.make_params(1, 40, 128, (21, 45, 80), 44, 0.9)   # needs far more than the 64 MiB array
+    assert lib.sa_plan_static(bad, bad, None, None, ctypes.byref(huge), bad, bad, None) == 5
+    assert lib.sa_get_device_status(None, None) == 1
+    assert lib.sa_last_launch_count() == 0
