@@ -204,14 +204,40 @@ def untile(y, p: Params, out=None, stream=None):
     return out
 
 
-def plan(q, k, p: Params, q_scale=None, k_scale=None, kv_index=None, kv_count=None, ws=None, stream=None):
-    """Router: returns (kv_index [B,H,T,cap] int32, kv_count [B,H,T] int32)."""
+def _router_args(q, k, p: Params, q_scale, k_scale, kv_index, kv_count):
+    """Checks shared by the routers before anything reaches the library: token tensors,
+    caller-given output buffers (int32, contiguous, [B,H,T,cap] / [B,H,T], on q's device)
+    and, for e4m3 Q/K, the per-cube fp32 scales [B,H,T] on q's device."""
     torch = _torch()
     eb = 1 if p.qk_dtype == FP8_E4M3 else 2
     _token_tensor(q, p, "q", eb)
     _token_tensor(k, p, "k", eb)
     _, T = geometry(p)
     dev = q.device
+    if k.device != dev:
+        raise ValueError("q and k must be on the same device")
+    for t, name, shape in ((kv_index, "kv_index", (p.B, p.H, T, p.kv_capacity)), (kv_count, "kv_count", (p.B, p.H, T))):
+        if t is None:
+            continue
+        _contig(t, name, torch.int32)
+        _shape(t, shape, name)
+        if t.device != dev:
+            raise ValueError(f"{name} must be on {dev}")
+    if p.qk_dtype == FP8_E4M3:
+        for t, name in ((q_scale, "q_scale"), (k_scale, "k_scale")):
+            if t is None:
+                raise ValueError(f"{name} is required for e4m3 Q/K")
+            _contig(t, name, torch.float32)
+            _shape(t, (p.B, p.H, T), name)
+            if t.device != dev:
+                raise ValueError(f"{name} must be on {dev}")
+    return T, dev
+
+
+def plan(q, k, p: Params, q_scale=None, k_scale=None, kv_index=None, kv_count=None, ws=None, stream=None):
+    """Router: returns (kv_index [B,H,T,cap] int32, kv_count [B,H,T] int32)."""
+    torch = _torch()
+    T, dev = _router_args(q, k, p, q_scale, k_scale, kv_index, kv_count)
     if kv_index is None:
         kv_index = torch.empty((p.B, p.H, T, p.kv_capacity), dtype=torch.int32, device=dev)
     if kv_count is None:
@@ -227,9 +253,9 @@ def plan(q, k, p: Params, q_scale=None, k_scale=None, kv_index=None, kv_count=No
 def plan_static(q, k, p: Params, kv_index, kv_count, q_scale=None, k_scale=None, stream=None):
     """Router with the library's fixed 64 MiB scratch instead of a workspace (see
     ``sa_plan_static`` in include/sa.h).  Outputs are caller-provided; nothing is allocated."""
-    eb = 1 if p.qk_dtype == FP8_E4M3 else 2
-    _token_tensor(q, p, "q", eb)
-    _token_tensor(k, p, "k", eb)
+    if kv_index is None or kv_count is None:
+        raise ValueError("plan_static writes into caller-given kv_index and kv_count")
+    _router_args(q, k, p, q_scale, k_scale, kv_index, kv_count)
     st = load_library().sa_plan_static(_ptr(q), _ptr(k), _ptr(q_scale), _ptr(k_scale), ctypes.byref(p),
                                        _ptr(kv_index), _ptr(kv_count), _stream(stream))
     _check(st, "sa_plan_static")

@@ -209,6 +209,53 @@ sa::AttnArgs base_args(const sa_params* p, const Geom& g, void* ws) {
 
 }  // namespace
 
+namespace sa {
+
+// sa_plan's host-side argument checks (nothing touches the device); *ws_needed receives the
+// workspace size the router needs.
+sa_status plan_check(const void* q, const void* k, const float* q_scale, const float* k_scale, const sa_params* p,
+                     const int32_t* kv_index, const int32_t* kv_count, size_t* ws_needed) {
+  Geom g;
+  sa_status s = check_params(p, &g);
+  if (s != SA_OK) return s;
+  if (!q || !k || !kv_index || !kv_count) return SA_ERR_INVALID_ARG;
+  const bool fp8 = p->qk_dtype == SA_FP8_E4M3;
+  if (fp8 && (!q_scale || !k_scale)) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned4(kv_index) || !aligned4(kv_count)) return SA_ERR_ALIGNMENT;
+  if (fp8 && (!aligned4(q_scale) || !aligned4(k_scale))) return SA_ERR_ALIGNMENT;
+  *ws_needed = ws_layout(p, g, SA_OP_PLAN).total;
+  return SA_OK;
+}
+
+// The same checks, then the workspace carving and launches of sa_plan on the scratch `ws`
+// (a caller's workspace, or the fixed array of sa_plan_static); records the launch count.
+sa_status plan_on_scratch(const void* q, const void* k, const float* q_scale, const float* k_scale,
+                          const sa_params* p, int32_t* kv_index, int32_t* kv_count, void* ws, size_t ws_bytes,
+                          cudaStream_t st) {
+  g_last_launches = 0;
+  size_t need = 0;
+  sa_status s = plan_check(q, k, q_scale, k_scale, p, kv_index, kv_count, &need);
+  if (s != SA_OK) return s;
+  Geom g;
+  make_geom(p, &g);
+  const bool fp8 = p->qk_dtype == SA_FP8_E4M3;
+  const WsLayout w = ws_layout(p, g, SA_OP_PLAN);
+  if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SA_ERR_ALIGNMENT;
+  if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  int launches = 0;
+  if (launch_plan(q, k, q_scale, k_scale, g, p->B * p->H, p->D, fp8, softmax_scale(p), p->top_k, p->top_p,
+                  p->kv_capacity, kv_index, kv_count, reinterpret_cast<double*>(wb + w.qbar),
+                  reinterpret_cast<double*>(wb + w.kbar), reinterpret_cast<double*>(wb + w.scores),
+                  static_cast<DevStatus*>(ws), st, &launches) != cudaSuccess)
+    return SA_ERR_LAUNCH;
+  g_last_launches = launches;
+  return SA_OK;
+}
+
+}  // namespace sa
+
 extern "C" {
 
 int sa_padded_tokens(const sa_params* p) {
@@ -259,29 +306,8 @@ sa_status sa_untile(const void* x_tiled, void* x_latent, const sa_params* p, int
 
 sa_status sa_plan(const void* q, const void* k, const float* q_scale, const float* k_scale, const sa_params* p,
                   int32_t* kv_index, int32_t* kv_count, void* ws, size_t ws_bytes, sa_stream_t stream) {
-  Geom g;
-  g_last_launches = 0;
-  sa_status s = check_params(p, &g);
-  if (s != SA_OK) return s;
-  if (!q || !k || !kv_index || !kv_count) return SA_ERR_INVALID_ARG;
-  const bool fp8 = p->qk_dtype == SA_FP8_E4M3;
-  if (fp8 && (!q_scale || !k_scale)) return SA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned4(kv_index) || !aligned4(kv_count)) return SA_ERR_ALIGNMENT;
-  if (fp8 && (!aligned4(q_scale) || !aligned4(k_scale))) return SA_ERR_ALIGNMENT;
-  const WsLayout w = ws_layout(p, g, SA_OP_PLAN);
-  if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
-  if (!aligned16(ws)) return SA_ERR_ALIGNMENT;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
-  uint8_t* wb = static_cast<uint8_t*>(ws);
-  int launches = 0;
-  if (sa::launch_plan(q, k, q_scale, k_scale, g, p->B * p->H, p->D, fp8, softmax_scale(p), p->top_k, p->top_p,
-                      p->kv_capacity, kv_index, kv_count, reinterpret_cast<double*>(wb + w.qbar),
-                      reinterpret_cast<double*>(wb + w.kbar), reinterpret_cast<double*>(wb + w.scores),
-                      static_cast<sa::DevStatus*>(ws), st, &launches) != cudaSuccess)
-    return SA_ERR_LAUNCH;
-  g_last_launches = launches;
-  return SA_OK;
+  return sa::plan_on_scratch(q, k, q_scale, k_scale, p, kv_index, kv_count, ws, ws_bytes,
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 sa_status sa_forward(const void* q, const void* k, const void* v, const float* q_scale, const float* k_scale,

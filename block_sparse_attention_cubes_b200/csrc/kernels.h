@@ -5,10 +5,21 @@
 
 #include <cstdint>
 
+#include "../../include/sa.h"
 #include "geometry.cuh"
 #include "ptx.cuh"
 
 namespace sa {
+
+// sa_plan's host-side argument checks; *ws_needed receives the router's workspace size (api.cu).
+sa_status plan_check(const void* q, const void* k, const float* q_scale, const float* k_scale, const sa_params* p,
+                     const int32_t* kv_index, const int32_t* kv_count, size_t* ws_needed);
+// sa_plan on the scratch `ws` of `ws_bytes` (a caller's workspace or the library's fixed
+// array): the host checks, the workspace carving and the launches of sa_plan, and the launch
+// count that sa_last_launch_count reports (api.cu).
+sa_status plan_on_scratch(const void* q, const void* k, const float* q_scale, const float* k_scale,
+                          const sa_params* p, int32_t* kv_index, int32_t* kv_count, void* ws, size_t ws_bytes,
+                          cudaStream_t stream);
 
 struct DevStatus;
 struct AttnArgs;

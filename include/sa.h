@@ -247,8 +247,9 @@ SA_API sa_status sa_recall(const float* lse_kept, const float* lse_all, const sa
  * holds until exit; problems needing more (sa_workspace_size(p, SA_OP_PLAN) > 64 MiB,
  * e.g. 12 heads at the 480p shape fit, 40 heads at 720p do not) return SA_ERR_WORKSPACE.
  * kv_capacity must equal T, so no row can be clipped and there is no device status to
- * read.  The first call on a device looks up the array's device address (make it before
- * any stream capture).  All calls share the array: calls that overlap on the GPU race and
+ * read.  Outside a stream capture every call looks up the array's device address on the
+ * current device; inside a capture the address cached by an earlier call is used, so the first
+ * call on a device must come before any stream capture.  All calls share the array: calls that overlap on the GPU race and
  * must be serialised by the caller.  Allocates nothing (no cudaMalloc/cudaFree). */
 SA_API sa_status sa_plan_static(const void* q, const void* k, const float* q_scale, const float* k_scale,
                                 const sa_params* p, int32_t* kv_index, int32_t* kv_count, sa_stream_t stream);

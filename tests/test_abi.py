@@ -186,6 +186,10 @@ def test_fine_stage_layout_and_static_plan_validate_on_the_host(lib):
     pc = sa.make_params(1, 2, 64, (8, 8, 8), 4, 0.5, kv_capacity=4)
     assert lib.sa_plan_static(bad, bad, None, None, ctypes.byref(pc), bad, bad, None) == 1   # capacity != T
     assert lib.sa_plan_static(odd, bad, None, None, P, bad, bad, None) == 3
+    f8s = sa.make_params(1, 2, 128, (8, 8, 8), 4, 0.5, qk_dtype=sa.FP8_E4M3)
+    odd4 = ctypes.c_void_p(18)                                   # fp32 scales must be 4-byte aligned
+    assert lib.sa_plan_static(bad, bad, odd4, bad, ctypes.byref(f8s), bad, bad, None) == 3
+    assert lib.sa_plan_static(bad, bad, None, bad, ctypes.byref(f8s), bad, bad, None) == 1   # scale missing
     huge = sa.make_params(1, 40, 128, (21, 45, 80), 44, 0.9)   # needs far more than the 64 MiB array
     assert lib.sa_plan_static(bad, bad, None, None, ctypes.byref(huge), bad, bad, None) == 5
     assert lib.sa_get_device_status(None, None) == 1
