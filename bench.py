@@ -8,7 +8,8 @@ Prints ONE JSON line on rank 0.  ``value`` is effective TFLOP/s over the whole s
 forward 4*D*64*64 and backward 10*D*64*64 FLOPs per selected tile (VSA page, FLOP
 accounting: 4 * D * S * H * d * 3.5, i.e. forward 1 + backward 2.5).  Each rank runs an
 independent problem of the same shape (weak scaling, no collective on the data path).
-Inputs are larger than L2 and L2 is also flushed between steps (256 MiB write).
+Inputs are larger than L2 and L2 is also flushed between steps (256 MiB write); every
+time reported is the median over the timed steps (per-step values are on the line too).
 Extra sections on the same line: ``fp8_forward`` (e4m3 Q/K configuration, 720p only) and
 ``gated`` (the coarse branch + gate layer: sa_plan_coarse, sa_forward_gated,
 sa_backward_gated), skipped with ``--no-fp8`` / ``--no-gated``.
@@ -22,6 +23,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -51,11 +53,15 @@ def tile_flops(D: int, ntiles: int):
 
 # ---------------------------------------------------------------------------------- clocks
 class ClockSampler:
+    """nvidia-smi clock/power/throttle samples every 200 ms in a temporary file.  Started
+    before the warm-up (so its start-up is over long before the timed region) and
+    summarised over the lines written between two ``mark()`` calls."""
+
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out" if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else "",
-                                 f".clocks_{os.getpid()}.csv")
+        fd, self.path = tempfile.mkstemp(prefix="sa_clocks_", suffix=".csv")
+        os.close(fd)
 
     def __enter__(self):
         try:
@@ -65,16 +71,20 @@ class ClockSampler:
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
-        # wait for the first sample, so nvidia-smi's start-up (NVML initialisation) is over
-        # before the timed region begins
         t0 = time.time()
         while self.proc is not None and time.time() - t0 < 5.0:
             self.f.flush()
             if os.path.getsize(self.path) > 0:
                 break
             time.sleep(0.05)
-        time.sleep(0.3)
         return self
+
+    def mark(self) -> int:
+        """Number of complete sample lines written so far."""
+        if self.proc is None:
+            return 0
+        with open(self.path) as f:
+            return sum(1 for line in f if line.endswith("\n"))
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -85,20 +95,22 @@ class ClockSampler:
                 self.proc.kill()
             self.f.close()
 
-    def summary(self):
+    def summary(self, first: int = 0, last: int | None = None):
+        """Median SM clock under load and throttle reasons over sample lines [first, last]
+        (one line past ``last`` is included: the sample that closes the interval)."""
         if self.proc is None or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
+        lines = open(self.path).read().splitlines()
         try:
             os.remove(self.path)
         except OSError:
             pass
+        window = lines[first:(None if last is None else last + 1)]
+        rows = [[x.strip() for x in line.split(",")] for line in window]
+        rows = [r for r in rows if len(r) >= 9]
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
         def num(x):
             try:
                 return float(x)
@@ -111,6 +123,11 @@ class ClockSampler:
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
         return {"sm_mhz": statistics.median(under_load) if under_load else None,
                 "sm_max_mhz": max(num(r[2]) or 0 for r in rows), "reasons": reasons, "samples": len(rows)}
+
+
+def stats_ms(v):
+    return {"median": round(statistics.median(v), 4), "mean": round(statistics.mean(v), 4),
+            "min": round(min(v), 4), "max": round(max(v), 4)}
 
 
 # ---------------------------------------------------------------------------------- ours
@@ -152,54 +169,75 @@ def run_ours(args, rank, world, dist):
             rec[3].record()
         return idx, cnt, out, lse, g
 
-    for _ in range(args.warmup):
-        idx, cnt, *_ = step()
-    torch.cuda.synchronize()
-    for op in (sa.OP_PLAN, sa.OP_FORWARD, sa.OP_BACKWARD):
-        st = sa.device_status(A._ws[op])
-        if st != 0:
-            raise RuntimeError(f"device status {sa.STATUS_NAMES.get(st, st)} after warm-up")
-    ntiles = int(cnt.sum().item())
-    density = ntiles / (cfg.B * cfg.H * T * T)
-    fwd_fl, bwd_fl = tile_flops(cfg.D, ntiles)
+    def phases(recs):
+        return [[r[i].elapsed_time(r[i + 1]) for r in recs] for i in range(3)]
 
-    recs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    launches["n"] = 0
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
+    # the clock sampler runs from before the warm-up to after the timed steps; its samples
+    # are summarised over the timed region only
     with ClockSampler(local) as clocks:
+        wrecs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.warmup)]
+        for w in range(args.warmup):
+            flush.fill_(w & 0xff)
+            last = step(wrecs[w])
+        torch.cuda.synchronize()
+        warm_phases = phases(wrecs)
+        for op in (sa.OP_PLAN, sa.OP_FORWARD, sa.OP_BACKWARD):
+            st = sa.device_status(A._ws[op])
+            if st != 0:
+                raise RuntimeError(f"device status {sa.STATUS_NAMES.get(st, st)} after warm-up")
+        cnt = last[1]
+        ntiles = int(cnt.sum().item())
+        valid_fl = valid_only_flops(sa, p, cfg, last[0], cnt, dev)
+        del last
+
+        recs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        launches["n"] = 0
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        line0 = clocks.mark()
         for s in range(args.steps):
             flush.fill_(s & 0xff)     # evict L2 between steps (not timed)
-            step(recs[s])
+            res = step(recs[s])
         torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    plan_ms = [r[0].elapsed_time(r[1]) for r in recs]
-    fwd_ms = [r[1].elapsed_time(r[2]) for r in recs]
-    bwd_ms = [r[2].elapsed_time(r[3]) for r in recs]
+        line1 = clocks.mark()
+        gpu_launches = launches["n"]
+        if dist is not None:
+            dist.barrier()
+        # warm L2: the same step without the flush in between (context, not the headline)
+        wl = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(5)]
+        for s in range(5):
+            step(wl[s])
+        torch.cuda.synchronize()
+    clock_summary = clocks.summary(line0, line1)
+    plan_ms, fwd_ms, bwd_ms = phases(recs)
     step_ms = [a + b + c for a, b, c in zip(plan_ms, fwd_ms, bwd_ms)]
-    total_ms = max_over_ranks(sum(step_ms), dist, dev)
-    ms_per_step = total_ms / args.steps
+    ms_per_step = max_over_ranks(statistics.median(step_ms), dist, dev)
+    fwd_fl, bwd_fl = tile_flops(cfg.D, ntiles)
     step_flops = (fwd_fl + bwd_fl) * world
     value = step_flops / (ms_per_step * 1e-3) / 1e12
 
     peaks, peak_src = load_peaks()
-    fwd_avg = statistics.mean(fwd_ms)
-    bwd_avg = statistics.mean(bwd_ms)
-    plan_avg = statistics.mean(plan_ms)
+    fwd_med, bwd_med, plan_med = (statistics.median(v) for v in (fwd_ms, bwd_ms, plan_ms))
     # dominant kernel: the forward kernel, timed with events around sa_forward on the launching
     # (current) stream inside the timed region; the call's two other launches (cube mask, query
-    # pair union) are about 0.3% of its time, so this slightly understates the kernel's own rate
-    fwd_tf = fwd_fl / (fwd_avg * 1e-3) / 1e12
-    peak_tf = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
+    # pair union) are about 0.3% of its time, so this slightly understates the kernel's own rate.
+    # A kernel timed on its own (tens of ms) takes the burst peak, measured with the same clocks free.
+    fwd_tf = fwd_fl / (fwd_med * 1e-3) / 1e12
+    fb_tf = (fwd_fl + bwd_fl) / ((fwd_med + bwd_med) * 1e-3) / 1e12
+    peak_tf = peaks.get("bf16_tflops")
     roofline = {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": round(fwd_tf, 2),
                 "peak": peak_tf, "unit": "TFLOP/s", "frac": round(fwd_tf / peak_tf, 4),
                 "traffic": traffic_for("attn_fwd_kernel", ntiles),
-                "peak_source": f"{peak_src} bf16 dense, sustained",
-                "algorithmic_flops_per_launch": fwd_fl}
+                "peak_source": f"{peak_src} bf16 dense, burst (cuBLAS, best of 10)",
+                "algorithmic_flops_per_launch": fwd_fl,
+                "fwd_bwd": {"achieved": round(fb_tf, 2), "frac": round(fb_tf / peak_tf, 4),
+                            "frac_of_sustained": round(fb_tf / peaks.get("bf16_tflops_sustained", peak_tf), 4)},
+                "run_sm_mhz": clock_summary.get("sm_mhz"),
+                "peak_sustained_sm_mhz": (peaks.get("clocks_under_load") or {}).get("sm_mhz_median")}
     router_bytes = 2 * cfg.B * cfg.H * npad * cfg.D * 2 + 4 * (ntiles + cfg.B * cfg.H * T)
-    router_gbs = router_bytes / (plan_avg * 1e-3) / 1e9
+    router_gbs = router_bytes / (plan_med * 1e-3) / 1e9
+    warm = phases(wl)
 
     result = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -209,23 +247,33 @@ def run_ours(args, rank, world, dist):
                                f"{'x'.join(map(str, cfg.lat))} -> T={T} cubes of 64, Npad={npad}; top_k={cfg.top_k}, "
                                f"top_p={cfg.top_p}; step = sa_plan + sa_forward + sa_backward",
                    "B": cfg.B, "H": cfg.H, "D": cfg.D, "lat": list(cfg.lat), "T": T, "top_k": cfg.top_k,
-                   "top_p": cfg.top_p, "density": round(density, 5), "selected_tiles": ntiles,
+                   "top_p": cfg.top_p, "density": round(ntiles / (cfg.B * cfg.H * T * T), 5), "selected_tiles": ntiles,
                    "l2": "inputs larger than L2; 256 MiB flush between steps",
-                   "per_rank": "independent problem per rank (seed = rank)"},
-        "breakdown_ms": {"plan": round(plan_avg, 4), "forward": round(fwd_avg, 4), "backward": round(bwd_avg, 4),
-                         "fwd_plus_bwd": round(fwd_avg + bwd_avg, 4)},
+                   "per_rank": "independent problem per rank (seed = rank)",
+                   "timing": "median of the timed steps (CUDA events on the launching stream)"},
+        "breakdown_ms": {"plan": round(plan_med, 4), "forward": round(fwd_med, 4), "backward": round(bwd_med, 4),
+                         "fwd_plus_bwd": round(fwd_med + bwd_med, 4)},
+        "step_ms": stats_ms(step_ms),
         "per_step_ms": {"plan": [round(v, 3) for v in plan_ms], "forward": [round(v, 3) for v in fwd_ms],
                         "backward": [round(v, 3) for v in bwd_ms]},
-        "fwd_bwd_tflops": round((fwd_fl + bwd_fl) / ((fwd_avg + bwd_avg) * 1e-3) / 1e12, 3),
+        "warmup_ms": {n: [round(v, 3) for v in vals] for n, vals in zip(("plan", "forward", "backward"), warm_phases)},
+        "warm_l2_ms": {n: round(statistics.median(vals), 4) for n, vals in zip(("plan", "forward", "backward"), warm)},
+        "fwd_bwd_tflops": round(fb_tf, 3),
+        "valid_only": {"flops_fwd_bwd": valid_fl, "tflops": round(valid_fl / ((fwd_med + bwd_med) * 1e-3) / 1e12, 3),
+                       "note": "4*D and 10*D FLOPs per valid (query row, key) pair of the selected tiles"},
         "router": {"achieved_gbs": round(router_gbs, 1), "peak_gbs": peaks.get("hbm_gbs"),
                    "frac": round(router_gbs / peaks.get("hbm_gbs"), 4), "algorithmic_bytes": router_bytes},
         "roofline": roofline,
-        "gpu_launches": launches["n"],
-        "clocks": clocks.summary(),
+        "gpu_launches": gpu_launches,
+        "clocks": clock_summary,
         "gen_s": round(t_gen, 1),
     }
     if args.e2e_steps > 0:
         result["e2e"] = run_e2e(args, sa, A, p, host, dev, fwd_fl + bwd_fl, world, dist)
+    gpu_sample = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gpu_sample = gpu_outputs_for_heads(res, cfg, oracle_heads(cfg.H))
+    del res
     run_fp8 = args.config == "720p" and not args.no_fp8
     if run_fp8 or not args.no_gated:
         del x, A
@@ -235,9 +283,51 @@ def run_ours(args, rank, world, dist):
         result["gated"] = run_gated(args, sa, synth, cfg, host, rank, dev, flush, result["breakdown_ms"], dist)
     if args.extras:
         result["extras"] = run_extras(args, sa, cfg, host, dev, flush, dist)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(cfg, host, seconds=args.cpu_seconds)
+    if gpu_sample is not None:
+        result["cpu_baseline"], result["parity_sample"] = cpu_baseline(cfg, host, gpu_sample, ntiles,
+                                                                       seconds=args.cpu_seconds)
     return result
+
+
+def valid_only_flops(sa, p, cfg, idx, cnt, dev):
+    """Forward + backward FLOPs counting only valid (query row, key) pairs of the selected
+    tiles: sum over selected (i, j) of 14 * D * n_i * n_j, n = valid tokens of a cube."""
+    import torch
+    T = idx.shape[2]
+    nv = torch.tensor(cube_valid_counts(cfg.lat), dtype=torch.float64, device=dev)
+    total = 0.0
+    for b in range(idx.shape[0]):
+        for h in range(idx.shape[1]):
+            used = torch.arange(idx.shape[3], device=dev)[None, :] < cnt[b, h][:, None]
+            nk = torch.where(used, nv[idx[b, h].clamp(0, T - 1).long()], torch.zeros((), dtype=torch.float64,
+                                                                                   device=dev)).sum(1)
+            total += float((nk * nv).sum().item())
+    return 14.0 * cfg.D * total
+
+
+def cube_valid_counts(lat):
+    """Valid tokens of every 4x4x4 cube of a latent grid, in cube order."""
+    lt, lh, lw = lat
+    out = []
+    for ct in range((lt + 3) // 4):
+        for ch in range((lh + 3) // 4):
+            for cw in range((lw + 3) // 4):
+                out.append(min(4, lt - 4 * ct) * min(4, lh - 4 * ch) * min(4, lw - 4 * cw))
+    return out
+
+
+def oracle_heads(H: int):
+    """The heads the oracle leg runs on: the first two of each head type (uniform first half,
+    sink second half)."""
+    return sorted({0, min(1, H - 1), H // 2, min(H // 2 + 1, H - 1)})
+
+
+def gpu_outputs_for_heads(res, cfg, heads):
+    """Host copies of the last timed step's lists and outputs on the oracle leg's heads."""
+    idx, cnt, out, lse, (dq, dk, dv) = res
+    pick = lambda t: t[0, heads].cpu()
+    return {"heads": heads, "idx": pick(idx), "cnt": pick(cnt), "out": pick(out).float(), "dq": pick(dq),
+            "dk": pick(dk), "dv": pick(dv)}
 
 
 def run_fp8_forward(args, sa, synth, rank, dev, flush, bf16_peak, hbm_peak, dist):
@@ -285,8 +375,8 @@ def run_fp8_forward(args, sa, synth, rank, dev, flush, bf16_peak, hbm_peak, dist
         flush.fill_(s & 0xff)
         step(recs[s])
     torch.cuda.synchronize()
-    plan_ms = statistics.mean(r[0].elapsed_time(r[1]) for r in recs)
-    fwd_ms = statistics.mean(r[1].elapsed_time(r[2]) for r in recs)
+    plan_ms = statistics.median(r[0].elapsed_time(r[1]) for r in recs)
+    fwd_ms = statistics.median(r[1].elapsed_time(r[2]) for r in recs)
     fwd_fl, _ = tile_flops(cfg.D, ntiles)
     tf = fwd_fl / (fwd_ms * 1e-3) / 1e12
     peak = bf16_peak * 4.0 / 3.0
@@ -361,7 +451,7 @@ def run_gated(args, sa, synth, cfg, host, rank, dev, flush, plain_ms, dist):
         step(recs[s])
     torch.cuda.synchronize()
     per_step = [[r[i].elapsed_time(r[i + 1]) for r in recs] for i in range(3)]
-    ms = [statistics.mean(v) for v in per_step]
+    ms = [statistics.median(v) for v in per_step]
     fwd_fl, bwd_fl = tile_flops(cfg.D, ntiles)
     cube_fl = 2.0 * cfg.B * cfg.H * T * T * cfg.D      # one cube-level product
     total_ms = sum(ms)
@@ -421,7 +511,7 @@ def run_extras(args, sa, cfg, host, dev, flush, dist):
         flush.fill_(s & 0xff)
         step(recs[s])
     torch.cuda.synchronize()
-    ms = [statistics.mean(r[i].elapsed_time(r[i + 1]) for r in recs) for i in range(3)]
+    ms = [statistics.median(r[i].elapsed_time(r[i + 1]) for r in recs) for i in range(3)]
     fwd_fl, bwd_fl = tile_flops(cfg.D, ntiles)
     bq = {"plan_ms": round(ms[0], 4), "forward_ms": round(ms[1], 4), "backward_ms": round(ms[2], 4),
           "selected_tiles": ntiles, "density": round(ntiles / (cfg.B * cfg.H * T * T), 5),
@@ -544,7 +634,7 @@ def run_sweep(args):
                 flush.fill_(s & 0xff)
                 step(recs[s])
             torch.cuda.synchronize()
-            ms = [statistics.mean(r[k].elapsed_time(r[k + 1]) for r in recs) for k in range(3)]
+            ms = [statistics.median(r[k].elapsed_time(r[k + 1]) for r in recs) for k in range(3)]
             ntiles = int(cnt.sum().item())
             fwd_fl, bwd_fl = tile_flops(cfg.D, ntiles)
             masks = selection_masks(idx, cnt)
@@ -700,56 +790,159 @@ def cpu_baseline_gated(cfg, host, gate, seconds: float = 15.0):
     frac = min(1.0, max(0.02, 0.02 * seconds / max(s0, 1e-3)))
     secs, flops, n = oracle_gated_sample(cfg, host, gate, head=0, frac=frac, seed=1)
     T = (cfg.lat[0] + 3) // 4 * ((cfg.lat[1] + 3) // 4) * ((cfg.lat[2] + 3) // 4)
-    return {"value": round(flops / secs / 1e12, 6), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+    cores = cpu_cores()
+    return {"value": round(flops / secs / 1e12, 6), "unit": UNIT, "cores": cores["used"], "host_cpus": cores["host"],
+            "kind": "oracle",
             "sample": f"head 0 of {cfg.name}: full fp64 router and coarse branch, gated forward and backward of "
                       f"{n} of {T} query cubes ({secs:.1f} s)"}
 
 
 def cpu_cores():
+    """Threads the oracle's BLAS uses, and the host's logical CPUs (nproc)."""
+    used = None
     try:
         from threadpoolctl import threadpool_info
-        info = threadpool_info()
-        n = max((i.get("num_threads", 1) for i in info), default=1)
-        return int(n)
+        used = max((i.get("num_threads", 1) for i in threadpool_info()), default=None)
     except Exception:
-        return os.cpu_count() or 1
+        pass
+    host = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    return {"used": int(used or host), "host": int(host)}
 
 
-def cpu_baseline(cfg, host, seconds: float = 15.0):
-    # calibrate the sample size on a small piece, then run ~`seconds` of oracle work
-    s0, _, n0 = oracle_sample(cfg, host, head=0, frac=0.02)
-    frac = min(1.0, max(0.02, 0.02 * seconds / max(s0, 1e-3)))
-    secs, flops, n = oracle_sample(cfg, host, head=0, frac=frac, seed=1)
-    return {"value": round(flops / secs / 1e12, 6), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"head 0 of {cfg.name}: full fp64 router + forward and backward of {n} of "
-                      f"{(cfg.lat[0]+3)//4*((cfg.lat[1]+3)//4)*((cfg.lat[2]+3)//4)} query cubes ({secs:.1f} s)"}
+def cpu_baseline(cfg, host, gpu, ntiles_total: int, seconds: float = 15.0):
+    """The fp64 oracle on the host cores, on a bounded sample of the timed workload: the full
+    router of the heads ``gpu["heads"]`` (two near-uniform, two sink heads) and the forward and
+    backward of one fixed sample of query cubes on each.  Returns (baseline, parity):
+
+    * baseline: the measured seconds, and the whole step (all heads, every selected tile)
+      extrapolated linearly (router time per head x heads, attention time per tile x tiles);
+      ``value`` is the step's FLOPs over that extrapolated time.
+    * parity: the last timed step's lists, outputs and gradients on the same heads against the
+      oracle: tie rows (the tie band of ``oracle.parity``), mismatching rows, and max/mean abs
+      errors of out and dQ on the sampled query cubes and of dK, dV on a few key cubes (over
+      every query cube that selects them).  Cubes touched by a row whose lists differ are left
+      out of the error figures."""
+    import numpy as np
+
+    import oracle as O
+    heads = gpu["heads"]
+    lay = O.cube_layout(cfg.lat)
+    T = lay.n_cubes
+    per_head = {h: {n: O.tile(host[n][0, h].double().numpy(), lay) for n in ("q", "k", "v", "do")} for h in heads}
+    # size the query-cube sample from a 1% calibration run on the first head (not counted)
+    t = per_head[heads[0]]
+    tr0 = O.route_head(t["q"], t["k"], lay.valid, cfg.top_k, cfg.top_p)
+    cal = np.arange(0, T, 100)
+    c0 = time.perf_counter()
+    O.attention_forward_head(t["q"], t["k"], t["v"], tr0.lists, lay.valid, q_blocks=cal)
+    O.attention_backward_head(t["q"], t["k"], t["v"], t["do"], tr0.lists, lay.valid, q_blocks=cal,
+                              kv_blocks=range(T), visit=cal)
+    per_cube = (time.perf_counter() - c0) / len(cal)
+    n_sample = int(min(T, max(4, seconds / len(heads) / max(per_cube, 1e-4))))
+    rng = np.random.default_rng(1)
+    sample = np.sort(rng.choice(T, size=n_sample, replace=False))
+    router_s, attn_s, tiles = 0.0, 0.0, 0
+    rows = eq = ties = mism = 0
+    err = {n: [0.0, 0.0, 0] for n in ("out", "dq", "dk", "dv")}    # max, sum, count
+    for hi, h in enumerate(heads):
+        t = per_head[h]
+        c0 = time.perf_counter()
+        tr = O.route_head(t["q"], t["k"], lay.valid, cfg.top_k, cfg.top_p)
+        c1 = time.perf_counter()
+        o_ref, _ = O.attention_forward_head(t["q"], t["k"], t["v"], tr.lists, lay.valid, q_blocks=sample)
+        dq_ref, _, _ = O.attention_backward_head(t["q"], t["k"], t["v"], t["do"], tr.lists, lay.valid,
+                                                 q_blocks=sample, kv_blocks=range(T), visit=sample)
+        c2 = time.perf_counter()
+        router_s += c1 - c0
+        attn_s += c2 - c1
+        tiles += sum(len(tr.lists[i]) for i in sample)
+        # ---- parity of the GPU's last timed step on this head
+        ci, cc = gpu["idx"][hi].numpy(), gpu["cnt"][hi].numpy()
+        got = [ci[i, :cc[i]].astype(np.int64) for i in range(T)]
+        m, tie, _ = O.parity.classify_router_rows(tr, got, cfg.top_p)
+        same = np.array([len(a) == len(b) and np.array_equal(a, b) for a, b in zip(tr.lists, got)])
+        rows += T
+        eq += int(same.sum())
+        ties += tie
+        mism += m
+
+        def acc(name, got_rows, ref_rows):
+            if got_rows.size == 0:
+                return
+            e = np.abs(got_rows.astype(np.float64) - ref_rows)
+            err[name][0] = max(err[name][0], float(e.max()))
+            err[name][1] += float(e.sum())
+            err[name][2] += e.size
+        qc = [i for i in sample if same[i]]
+        rws = np.concatenate([np.arange(i * 64, i * 64 + 64) for i in qc]) if qc else np.zeros(0, np.int64)
+        acc("out", gpu["out"][hi].numpy()[rws], o_ref[rws])
+        acc("dq", gpu["dq"][hi].numpy()[rws], dq_ref[rws])
+        # dK, dV of a few key cubes whose selecting query cubes all have equal lists
+        sel_by = [[] for _ in range(T)]
+        for i, l in enumerate(tr.lists):
+            for j in l:
+                sel_by[int(j)].append(i)
+        kc = [j for j in rng.choice(T, size=min(T, 16), replace=False) if all(same[i] for i in sel_by[j])][:4]
+        if kc:
+            _, dk_ref, dv_ref = O.attention_backward_head(t["q"], t["k"], t["v"], t["do"], tr.lists, lay.valid,
+                                                          q_blocks=[], kv_blocks=kc)
+            kr = np.concatenate([np.arange(j * 64, j * 64 + 64) for j in kc])
+            acc("dk", gpu["dk"][hi].numpy()[kr], dk_ref[kr])
+            acc("dv", gpu["dv"][hi].numpy()[kr], dv_ref[kr])
+    H = cfg.B * cfg.H
+    est_s = router_s / len(heads) * H + attn_s / max(tiles, 1) * ntiles_total
+    fwd, bwd = tile_flops(cfg.D, ntiles_total)
+    cores = cpu_cores()
+    sample_txt = (f"heads {heads} of {cfg.name}: full fp64 router of each, forward and backward of the same "
+                  f"{n_sample} of {T} query cubes on each ({tiles} tiles); measured {router_s:.1f} s router + "
+                  f"{attn_s:.1f} s attention; the whole step ({H} heads, {ntiles_total} tiles) extrapolated "
+                  f"linearly to {est_s:.0f} s")
+    baseline = {"value": round((fwd + bwd) / est_s / 1e12, 6), "unit": UNIT, "cores": cores["used"],
+                "host_cpus": cores["host"], "kind": "oracle", "sample": sample_txt,
+                "measured_s": {"router": round(router_s, 2), "attention": round(attn_s, 2)},
+                "sampled_tflops": round(tile_flops(cfg.D, tiles)[0] * 3.5 / attn_s / 1e12, 6),
+                "extrapolated_step_s": round(est_s, 1), "extrapolated": True}
+    parity = {"heads": heads, "rows": rows, "equal_rows": eq, "tie_rows": ties, "mismatch_rows": mism,
+              "tie_band": O.parity.TIE_REL,
+              "max_abs": {n: round(v[0], 6) for n, v in err.items() if v[2]},
+              "mean_abs": {n: round(v[1] / v[2], 7) for n, v in err.items() if v[2]},
+              "bounds": {"max_abs": 2e-2, "mean_abs": 2e-3},
+              "sample": f"last timed step; out and dq on {n_sample} query cubes per head, dk and dv on up to 4 "
+                        f"key cubes per head (over every query cube selecting them)"}
+    return baseline, parity
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle as it stands, on the host cores.  Step s runs the
+    full router of one head (cycling over the two near-uniform and two sink heads the oracle
+    leg uses) and the forward and backward of a fixed-size sample of its query cubes."""
     import synth
     cfg = synth.get_config(args.config)
-    host = synth.make_inputs(cfg, seed=0, heads=[0])
+    heads = oracle_heads(cfg.H)
+    host = synth.make_inputs(cfg, seed=0, heads=heads)
+    # make_inputs(heads=...) returns only those heads, in that order
     # sample size: the whole run (warm-up + timed) should take about two minutes
     s0, _, _ = oracle_sample(cfg, host, head=0, frac=0.02)
     per_step = 120.0 / max(1, args.steps + args.warmup)
     frac = min(1.0, max(0.005, 0.02 * per_step / max(s0, 1e-3)))
     for w in range(args.warmup):
-        oracle_sample(cfg, host, 0, frac, seed=100 + w)
+        oracle_sample(cfg, host, w % len(heads), frac, seed=100 + w)
     tot_s, tot_f, n = 0.0, 0.0, 0
     for s in range(args.steps):
-        secs, fl, n = oracle_sample(cfg, host, 0, frac, seed=s)
+        secs, fl, n = oracle_sample(cfg, host, s % len(heads), frac, seed=s)
         tot_s += secs
         tot_f += fl
     value = tot_f / tot_s / 1e12
     cores = cpu_cores()
-    sample = f"per step: head 0 of {cfg.name}, full fp64 router + forward and backward of {n} query cubes"
+    sample = (f"per step: one of heads {heads} of {cfg.name} in turn, full fp64 router + forward and backward "
+              f"of {n} query cubes")
     return {"metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": f"Wan2.1-14B-720p-shaped attention ({args.config}), fp64 CPU oracle sample",
                        "sample": sample},
-            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores["used"],
+                             "host_cpus": cores["host"], "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 

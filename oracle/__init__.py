@@ -23,6 +23,7 @@ float64, with numpy matmuls and sorts as the only library steps:
                          constant (VSA2 page section 2.1: the router output M carries
                          no gradient)
 * error decomposition .. SpargeAttention2 page, equation 8
+* parity rule ......... tie rows at the k / p boundary (module ``parity``)
 * coarse branch, gate .. VSA page, "Big-Picture Architecture" and "Gated Combination";
                          VSA2 page section 2.2, "Coarse Branch" and the gate equation
                          (module ``coarse``)
@@ -38,7 +39,7 @@ from .attention import (  # noqa: F401
     e4m3_decode, dequantize_rows, eq8_error_terms, block_grid_shape, vsa_sparsity,
     topk_from_fraction,
 )
-from . import blocks128, vsa2_router  # noqa: F401
+from . import blocks128, parity, vsa2_router  # noqa: F401
 from .coarse import (  # noqa: F401
     coarse_forward_head, repeat_cubes, gated_forward_head, gated_backward_head,
 )

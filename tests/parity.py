@@ -11,7 +11,8 @@ import synth
 
 ATOL_MAX = 2e-2    # max-abs error bound for bf16 inputs with fp32 accumulation
 ATOL_MEAN = 2e-3   # mean-abs error bound
-TIE_REL = 1e-6     # block-score tie band at the k / p boundary
+TIE_REL = O.parity.TIE_REL   # block-score tie band at the k / p boundary
+classify_router_rows = O.parity.classify_router_rows
 
 
 def gpu_inputs(cfg, seed=0, names=("q", "k", "v", "do"), heads=None):
@@ -31,35 +32,6 @@ def gpu_lists(idx, cnt, b, h):
     idx = idx[b, h].cpu().numpy()
     cnt = cnt[b, h].cpu().numpy()
     return [idx[i, :cnt[i]].astype(np.int64) for i in range(len(cnt))]
-
-
-def classify_router_rows(tr: O.RouterTrace, got_lists, top_p: float):
-    """Count (mismatch, tie) rows.  A differing row is a tie row when every block of the
-    symmetric difference has an oracle probability within TIE_REL of the oracle's boundary
-    value, or the oracle's cumulative mass at the Top-p crossing is within TIE_REL of p."""
-    mismatch, ties, bad_rows = 0, 0, []
-    for i, (ref, got) in enumerate(zip(tr.lists, got_lists)):
-        if len(ref) == len(got) and np.array_equal(ref, got):
-            continue
-        row = tr.pbar[i]
-        order = O.descending_order(row)
-        n = len(ref)
-        bval = row[order[n - 1]]
-        sym = np.setxor1d(ref, got)
-        tie_a = len(sym) > 0 and bool(np.all(np.abs(row[sym] - bval) <= TIE_REL * bval))
-        tie_b = False
-        if 0 < top_p < 1:
-            csum = np.cumsum(row[order])
-            target = top_p * row.sum()
-            for m in (tr.n_p[i] - 1, tr.n_p[i]):
-                if 1 <= m <= len(row) and abs(csum[m - 1] - target) <= TIE_REL * target:
-                    tie_b = True
-        if tie_a or tie_b:
-            ties += 1
-        else:
-            mismatch += 1
-            bad_rows.append(i)
-    return mismatch, ties, bad_rows
 
 
 def errs(got: np.ndarray, ref: np.ndarray):
