@@ -39,7 +39,7 @@ from .attention import (  # noqa: F401
     e4m3_decode, dequantize_rows, eq8_error_terms, block_grid_shape, vsa_sparsity,
     topk_from_fraction,
 )
-from . import blocks128, parity, vsa2_router  # noqa: F401
+from . import blocks128, parity, rope, vsa2_router  # noqa: F401
 from .coarse import (  # noqa: F401
     coarse_forward_head, repeat_cubes, gated_forward_head, gated_backward_head,
 )
