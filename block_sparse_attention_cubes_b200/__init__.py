@@ -34,11 +34,13 @@ STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3:
 OP_PLAN, OP_FORWARD, OP_BACKWARD, OP_PLAN_COARSE, OP_BACKWARD_GATED, OP_PLAN_BQ128 = 0, 1, 2, 3, 4, 5
 BF16, FP8_E4M3 = 0, 1
 DEBUG_SKIP_LOADS = 1
+DEBUG_ROUTER_FALLBACK = 2
 
 # every symbol include/sa.h declares
 EXPORTS = ("sa_padded_tokens", "sa_num_cubes", "sa_topk_from_fraction", "sa_workspace_size", "sa_tile",
            "sa_untile", "sa_plan", "sa_forward", "sa_backward", "sa_get_device_status", "sa_status_string",
-           "sa_last_launch_count", "sa_plan_static", "sa_plan_coarse", "sa_forward_gated", "sa_backward_gated", "sa_recall", "sa_plan_bq128")
+           "sa_last_launch_count", "sa_plan_static", "sa_plan_coarse", "sa_forward_gated", "sa_backward_gated", "sa_recall", "sa_plan_bq128",
+           "sa_plan_fallback_rows", "sa_tile_rope", "sa_untile_rope")
 
 
 class SAError(RuntimeError):
@@ -93,6 +95,9 @@ def load_library(path: str = LIB_PATH):
                                     vp, vp, sz, vp]),
         "sa_recall": (i32, [vp, vp, P, vp, vp, vp]),
         "sa_plan_bq128": (i32, [vp, vp, P, vp, vp, vp, sz, vp]),
+        "sa_plan_fallback_rows": (i32, [vp, vp]),
+        "sa_tile_rope": (i32, [vp, vp, P, i32, i32, i32, i32, vp, vp, vp]),
+        "sa_untile_rope": (i32, [vp, vp, P, i32, i32, i32, i32, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -178,6 +183,16 @@ def device_status(ws, stream=None) -> int:
     return int(load_library().sa_get_device_status(_ptr(ws), _stream(stream)))
 
 
+def plan_fallback_rows(ws, stream=None) -> int:
+    """Synchronise the stream and return how many rows the last :func:`plan` on workspace
+    ``ws`` decided on its fp64 path (rows whose tensor-core decision was within the error
+    bounds of changing)."""
+    n = int(load_library().sa_plan_fallback_rows(_ptr(ws), _stream(stream)))
+    if n < 0:
+        raise SAError(6, "sa_plan_fallback_rows")
+    return n
+
+
 def tile(x, p: Params, out=None, stream=None):
     """Latent ``[B,H,L,D]`` -> cube-major ``[B,H,Npad,D]`` (same dtype, padding zero)."""
     torch = _torch()
@@ -188,6 +203,47 @@ def tile(x, p: Params, out=None, stream=None):
     q = Params.from_buffer_copy(p)
     q.D = x.shape[-1]
     _check(load_library().sa_tile(_ptr(x), _ptr(out), ctypes.byref(q), x.element_size(), _stream(stream)), "sa_tile")
+    return out
+
+
+def _rope_tables(p: Params, sections, rope_cos, rope_sin, device):
+    torch = _torch()
+    dt, dh, dw = sections
+    n = p.lat_t * (dt // 2) + p.lat_h * (dh // 2) + p.lat_w * (dw // 2)
+    for t, name in ((rope_cos, "rope_cos"), (rope_sin, "rope_sin")):
+        _contig(t, name, torch.float32)
+        if t.numel() != n or t.device != device:
+            raise ValueError(f"{name} must hold {n} fp32 values on {device}")
+
+
+def tile_rope(x, p: Params, sections, rope_cos, rope_sin, out=None, stream=None):
+    """Latent ``[B,H,L,D]`` -> cube-major ``[B,H,Npad,D]`` with each token rotated by its 3-D
+    RoPE angles (``sections`` = (d_t, d_h, d_w); tables as in ``sa_tile_rope``)."""
+    torch = _torch()
+    _contig(x, "x")
+    npad, _ = geometry(p)
+    _rope_tables(p, sections, rope_cos, rope_sin, x.device)
+    if out is None:
+        out = torch.empty((p.B, p.H, npad, x.shape[-1]), dtype=x.dtype, device=x.device)
+    q = Params.from_buffer_copy(p)
+    q.D = x.shape[-1]
+    _check(load_library().sa_tile_rope(_ptr(x), _ptr(out), ctypes.byref(q), x.element_size(), *sections,
+                                       _ptr(rope_cos), _ptr(rope_sin), _stream(stream)), "sa_tile_rope")
+    return out
+
+
+def untile_rope(y, p: Params, sections, rope_cos, rope_sin, out=None, stream=None):
+    """Inverse of :func:`tile_rope`: cube-major -> latent order with the inverse rotation."""
+    torch = _torch()
+    _contig(y, "y")
+    L = p.lat_t * p.lat_h * p.lat_w
+    _rope_tables(p, sections, rope_cos, rope_sin, y.device)
+    if out is None:
+        out = torch.empty((p.B, p.H, L, y.shape[-1]), dtype=y.dtype, device=y.device)
+    q = Params.from_buffer_copy(p)
+    q.D = y.shape[-1]
+    _check(load_library().sa_untile_rope(_ptr(y), _ptr(out), ctypes.byref(q), y.element_size(), *sections,
+                                         _ptr(rope_cos), _ptr(rope_sin), _stream(stream)), "sa_untile_rope")
     return out
 
 

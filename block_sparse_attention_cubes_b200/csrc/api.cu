@@ -67,15 +67,22 @@ struct WsLayout {
   size_t doc = 0, dltc = 0, s32 = 0, ds32 = 0;             // gated backward: coarse scratch
   size_t cq = 0, ck = 0, cv = 0;
   size_t qpair = 0, blk_index = 0, blk_count = 0;          // plan with 128-token query blocks
+  size_t qlimb = 0, klimb = 0, qexp = 0, kexp = 0, ql1 = 0;  // plan on the tensor cores
+  size_t kexpmax = 0, meta = 0, keys = 0, flist = 0, fbs = 0;
+  int Tk = 0;
   size_t total = 0;
 };
+
+// The routers that keep every fp64 score (the coarse branch reads them; the 128-token block
+// router scores blocks of two cubes): status, Qbar, Kbar, S [BH, T, T] fp64.
+constexpr int kOpPlanFp64 = 100;
 
 WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
   WsLayout w;
   const size_t BH = static_cast<size_t>(p->B) * p->H;
   if (op == SA_OP_PLAN_BQ128) {
-    // the plan's (the score rows of the first ceil(T/2) blocks are used), then the block means and lists
-    w = ws_layout(p, g, SA_OP_PLAN);
+    // the fp64 plan's (the score rows of the first ceil(T/2) blocks are used), then the block means and lists
+    w = ws_layout(p, g, kOpPlanFp64);
     const size_t M = static_cast<size_t>((g.T + 1) / 2);
     size_t off = w.total;
     w.qpair = off;
@@ -89,7 +96,7 @@ WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
   }
   if (op == SA_OP_PLAN_COARSE || op == SA_OP_BACKWARD_GATED) {
     // the plain layout, then the coarse branch's buffers
-    w = ws_layout(p, g, op == SA_OP_PLAN_COARSE ? SA_OP_PLAN : SA_OP_BACKWARD);
+    w = ws_layout(p, g, op == SA_OP_PLAN_COARSE ? kOpPlanFp64 : SA_OP_BACKWARD);
     const size_t TT = BH * g.T * static_cast<size_t>(g.T) * sizeof(float);
     const size_t TD = BH * g.T * static_cast<size_t>(p->D) * sizeof(float);
     size_t off = w.total;
@@ -117,6 +124,33 @@ WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
   }
   size_t off = kHeader;
   if (op == SA_OP_PLAN) {
+    const size_t rows = BH * g.T;
+    w.qbar = off;
+    off = align256(off + rows * p->D * sizeof(double));
+    w.kbar = off;
+    off = align256(off + rows * p->D * sizeof(double));
+    w.qlimb = off;
+    off = align256(off + BH * 4 * g.T * 128);
+    w.klimb = off;
+    off = align256(off + BH * 4 * g.T * 128);
+    w.qexp = off;
+    off = align256(off + rows * sizeof(int));
+    w.kexp = off;
+    off = align256(off + rows * sizeof(int));
+    w.ql1 = off;
+    off = align256(off + rows * sizeof(double));
+    w.kexpmax = off;
+    off = align256(off + BH * sizeof(unsigned));
+    w.meta = off;
+    off = align256(off + rows * 32);
+    w.Tk = (g.T + 3) & ~3;
+    w.keys = off;
+    off = align256(off + rows * static_cast<size_t>(w.Tk) * sizeof(int));
+    w.flist = off;
+    off = align256(off + rows * sizeof(int));
+    w.fbs = off;
+    off = align256(off + static_cast<size_t>(sa::plan_fallback_ctas()) * 4 * g.T * sizeof(double));
+  } else if (op == kOpPlanFp64) {
     w.qbar = off;
     off = align256(off + BH * g.T * p->D * sizeof(double));
     w.kbar = off;
@@ -185,6 +219,20 @@ bool make_map(CUtensorMap* m, const void* base, long long rows, int D, int esize
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over limb rows {128 bytes, T rows, BH*4 slabs}: 128 x 128 boxes, 128-byte swizzle;
+// rows past T read as zeros.
+bool make_limb_map(CUtensorMap* m, const void* base, int T, long long slabs) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(slabs)};
+  cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(T) * 128};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 sa_status reset_status(void* ws, cudaStream_t s) {
   return cudaMemsetAsync(ws, 0, kHeader, s) == cudaSuccess ? SA_OK : SA_ERR_LAUNCH;
 }
@@ -242,13 +290,31 @@ sa_status plan_on_scratch(const void* q, const void* k, const float* q_scale, co
   const WsLayout w = ws_layout(p, g, SA_OP_PLAN);
   if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
   if (!aligned16(ws)) return SA_ERR_ALIGNMENT;
-  if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
   uint8_t* wb = static_cast<uint8_t*>(ws);
+  const int BH = p->B * p->H;
+  PlanFastWs f;
+  f.qbar = reinterpret_cast<double*>(wb + w.qbar);
+  f.kbar = reinterpret_cast<double*>(wb + w.kbar);
+  f.qlimb = reinterpret_cast<int8_t*>(wb + w.qlimb);
+  f.klimb = reinterpret_cast<int8_t*>(wb + w.klimb);
+  f.qexp = reinterpret_cast<int*>(wb + w.qexp);
+  f.kexp = reinterpret_cast<int*>(wb + w.kexp);
+  f.ql1 = reinterpret_cast<double*>(wb + w.ql1);
+  f.kexp_max = reinterpret_cast<unsigned*>(wb + w.kexpmax);
+  f.meta = wb + w.meta;
+  f.keys = reinterpret_cast<int*>(wb + w.keys);
+  f.Tk = w.Tk;
+  f.flist = reinterpret_cast<int*>(wb + w.flist);
+  f.fb_scratch = reinterpret_cast<double*>(wb + w.fbs);
+  CUtensorMap tq, tk;
+  if (!make_limb_map(&tq, f.qlimb, g.T, 4LL * BH) || !make_limb_map(&tk, f.klimb, g.T, 4LL * BH))
+    return SA_ERR_LAUNCH;
+  if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
+  const unsigned ms = p->timeout_ms ? p->timeout_ms : 2000u;
   int launches = 0;
-  if (launch_plan(q, k, q_scale, k_scale, g, p->B * p->H, p->D, fp8, softmax_scale(p), p->top_k, p->top_p,
-                  p->kv_capacity, kv_index, kv_count, reinterpret_cast<double*>(wb + w.qbar),
-                  reinterpret_cast<double*>(wb + w.kbar), reinterpret_cast<double*>(wb + w.scores),
-                  static_cast<DevStatus*>(ws), st, &launches) != cudaSuccess)
+  if (launch_plan_fast(q, k, q_scale, k_scale, tq, tk, g, BH, p->D, fp8, softmax_scale(p), p->top_k, p->top_p,
+                       p->kv_capacity, p->debug_flags, static_cast<unsigned long long>(ms) * 1000000ull, f, kv_index,
+                       kv_count, static_cast<DevStatus*>(ws), st, &launches) != cudaSuccess)
     return SA_ERR_LAUNCH;
   g_last_launches = launches;
   return SA_OK;
@@ -294,6 +360,35 @@ static sa_status tile_common(const void* src, void* dst, const sa_params* p, int
     return SA_ERR_LAUNCH;
   g_last_launches = 1;
   return SA_OK;
+}
+
+static sa_status tile_rope_common(const void* src, void* dst, const sa_params* p, int elem_bytes, int dt, int dh,
+                                  int dw, const float* cs, const float* sn, sa_stream_t stream, bool to_tiled) {
+  Geom g;
+  g_last_launches = 0;
+  if (!p || !src || !dst || !cs || !sn || p->B < 1 || p->H < 1 || !make_geom(p, &g)) return SA_ERR_INVALID_ARG;
+  if (elem_bytes != 2 && elem_bytes != 4) return SA_ERR_INVALID_ARG;
+  if (dt < 0 || dh < 0 || dw < 0 || (dt | dh | dw) & 1 || p->D < 2 || dt + dh + dw != p->D) return SA_ERR_INVALID_ARG;
+  if ((p->D * elem_bytes) % 16 != 0) return SA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(p->B) * p->H * g.Npad * p->D >= (1LL << 40)) return SA_ERR_UNSUPPORTED;
+  if (!aligned16(src) || !aligned16(dst) || !aligned4(cs) || !aligned4(sn)) return SA_ERR_ALIGNMENT;
+  if (sa::launch_tile_rope(src, dst, g, p->B * p->H, p->D, elem_bytes, to_tiled, dt, dh, dw, cs, sn,
+                           reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SA_ERR_LAUNCH;
+  g_last_launches = 1;
+  return SA_OK;
+}
+
+sa_status sa_tile_rope(const void* x_latent, void* x_tiled, const sa_params* p, int elem_bytes, int rope_dt,
+                       int rope_dh, int rope_dw, const float* rope_cos, const float* rope_sin, sa_stream_t stream) {
+  return tile_rope_common(x_latent, x_tiled, p, elem_bytes, rope_dt, rope_dh, rope_dw, rope_cos, rope_sin, stream,
+                          true);
+}
+
+sa_status sa_untile_rope(const void* x_tiled, void* x_latent, const sa_params* p, int elem_bytes, int rope_dt,
+                         int rope_dh, int rope_dw, const float* rope_cos, const float* rope_sin, sa_stream_t stream) {
+  return tile_rope_common(x_tiled, x_latent, p, elem_bytes, rope_dt, rope_dh, rope_dw, rope_cos, rope_sin, stream,
+                          false);
 }
 
 sa_status sa_tile(const void* x_latent, void* x_tiled, const sa_params* p, int elem_bytes, sa_stream_t stream) {
@@ -575,6 +670,14 @@ sa_status sa_get_device_status(const void* ws, sa_stream_t stream) {
   if (h.error & sa::DEVERR_INDEX) return SA_ERR_DEVICE_INDEX;
   if (h.error & sa::DEVERR_CAPACITY) return SA_ERR_CAPACITY;
   return SA_OK;
+}
+
+int sa_plan_fallback_rows(const void* ws, sa_stream_t stream) {
+  if (!ws) return -1;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return -1;
+  sa::DevStatus h;
+  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return -1;
+  return static_cast<int>(h.router_fallback);
 }
 
 const char* sa_status_string(sa_status s) {

@@ -27,10 +27,40 @@ struct AttnArgs;
 cudaError_t launch_tile(const void* src, void* dst, const Geom& g, int BH, int row_bytes, bool to_tiled,
                         cudaStream_t stream);
 
+// Tile (to_tiled) or untile with the 3-D RoPE rotation of each token (inverse when untiling).
+cudaError_t launch_tile_rope(const void* src, void* dst, const Geom& g, int BH, int D, int elem_bytes, bool to_tiled,
+                             int dt, int dh, int dw, const float* cs, const float* sn, cudaStream_t stream);
+
 cudaError_t launch_plan(const void* q, const void* k, const float* q_scale, const float* k_scale, const Geom& g,
                         int BH, int D, bool fp8, double scale, int top_k, float top_p, int cap, int32_t* kv_index,
                         int32_t* kv_count, double* qbar, double* kbar, double* S, DevStatus* st,
                         cudaStream_t stream, int* launches);
+
+// Scratch of the tensor-core router (carved from the plan workspace by api.cu).
+struct PlanFastWs {
+  double* qbar;        // [BH*T, D] fp64 pooled means (also read by the fp64 fallback rows)
+  double* kbar;
+  int8_t* qlimb;       // [BH, 4, T, 128] int8 limbs of the pooled rows
+  int8_t* klimb;
+  int* qexp;           // [BH*T] binary exponent of each pooled row
+  int* kexp;
+  double* ql1;         // [BH*T] 1-norm of each pooled query row
+  unsigned* kexp_max;  // [BH] largest key exponent per head (biased)
+  void* meta;          // [BH*T] per-row key scaling and error bounds (32 bytes each)
+  int* keys;           // [BH*T, Tk] fixed-point score keys
+  int Tk;              // row stride of keys (T rounded up to 4)
+  int* flist;          // [BH*T] rows left to the fp64 path
+  double* fb_scratch;  // [plan_fallback_ctas() * 4, T] one fp64 score row per fallback warp
+};
+int plan_fallback_ctas();
+// Router on the tensor cores (pool + limbs, exact limb products -> keys, key selection, fp64
+// rows): 5 launches and one memset.  tm_qlimb / tm_klimb: 3-D maps {128 B, T, BH*4} over the
+// limb buffers with 128 x 128 boxes and the 128-byte swizzle.
+cudaError_t launch_plan_fast(const void* q, const void* k, const float* q_scale, const float* k_scale,
+                             const CUtensorMap& tm_qlimb, const CUtensorMap& tm_klimb, const Geom& g, int BH, int D,
+                             bool fp8, double scale, int top_k, float top_p, int cap, unsigned debug,
+                             unsigned long long timeout_ns, const PlanFastWs& w, int32_t* kv_index, int32_t* kv_count,
+                             DevStatus* st, cudaStream_t stream, int* launches);
 
 cudaError_t launch_query_pair_union(const int32_t* kv_index, const int32_t* kv_count, int32_t* u_list,
                                     int32_t* u_cnt, int BH, int T, int cap, DevStatus* st, cudaStream_t stream);

@@ -14,7 +14,8 @@ struct DevStatus {
   unsigned int error;      // OR of SA_DEVERR_* bits
   unsigned int abort;      // set once any CTA gave up; later CTAs return at once
   unsigned int where;      // code of the first wait that timed out
-  unsigned int pad[61];
+  unsigned int router_fallback;  // rows the router decided again in fp64 (and the length of its row list)
+  unsigned int pad[60];
 };
 enum : unsigned int {
   DEVERR_TIMEOUT = 1u,
@@ -143,6 +144,15 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
+// 3-D tiled load (x innermost), this CTA only
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int32_t x,
+                                            int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
 // 1-D bulk copy global -> shared (both 16-byte aligned, size a multiple of 16), this CTA only
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -205,6 +215,17 @@ __device__ __forceinline__ void umma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uin
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::i8 (signed 8-bit inputs, exact s32 accumulate)
+__device__ __forceinline__ void umma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // arrive on `bar` once every previously issued tcgen05.mma of this thread has completed
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -260,6 +281,10 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t M, uint32_t N, uint32
 }
 constexpr uint32_t FMT_BF16 = 1u;
 constexpr uint32_t FMT_E4M3 = 0u;
+// kind::i8 with signed 8-bit A and B (format 1) and a signed 32-bit accumulator (D format 2)
+__host__ __device__ constexpr uint32_t make_idesc_s8(uint32_t M, uint32_t N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
 
 // byte offset of element (row, 16-byte chunk) inside a 128-byte-swizzled tile whose rows are 128 bytes
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk16) {

@@ -182,17 +182,12 @@ __device__ __forceinline__ uint64_t mass_fx(double x, double m) {
 // the first position n-1 such that n >= max(k, 1) and the first n masses reach p * Z,
 // by an 8-bit radix descent over the 64-bit order keys in which every bucket carries
 // its count and its exact fixed-point mass.  Then writes the kept ids in ascending order.
-__global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ S, int32_t* __restrict__ kv_index,
-                                                     int32_t* __restrict__ kv_count, int rows, int T, int top_k,
-                                                     float top_p, int cap, DevStatus* st) {
-  __shared__ uint32_t cnt_s[8][256];
-  __shared__ unsigned long long mass_s[8][256];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + warp;
-  if (row >= rows) return;
-  const double* s = S + static_cast<size_t>(row) * T;
-  uint32_t* cnt = cnt_s[warp];
-  unsigned long long* mass = mass_s[warp];
+// `s` is the row's T scores, `cnt` / `mass` a 256-entry scratch histogram of this warp; the
+// kept ids go to `out` (at most cap) and their number to *count.  Called by a whole warp.
+__device__ void select_row_fp64(const double* __restrict__ s, int T, int top_k, float top_p, int cap,
+                                int32_t* __restrict__ out, int32_t* __restrict__ count, DevStatus* st,
+                                uint32_t* cnt, unsigned long long* mass) {
+  const int lane = threadIdx.x & 31;
 
   double m = -DBL_MAX;
 #pragma unroll 4
@@ -364,7 +359,6 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   }
   // emit the kept ids in ascending order
   int n = 0;
-  int32_t* out = kv_index + static_cast<size_t>(row) * cap;
   for (int j0 = 0; j0 < T; j0 += 128) {
     double xs[4];
 #pragma unroll
@@ -388,7 +382,725 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   }
   if (lane == 0) {
     if (n > cap) flag_error(st, DEVERR_CAPACITY, 0);
-    kv_count[row] = min(n, cap);
+    *count = min(n, cap);
+  }
+}
+
+__global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ S, int32_t* __restrict__ kv_index,
+                                                     int32_t* __restrict__ kv_count, int rows, int T, int top_k,
+                                                     float top_p, int cap, DevStatus* st) {
+  __shared__ uint32_t cnt_s[8][256];
+  __shared__ unsigned long long mass_s[8][256];
+  const int warp = threadIdx.x >> 5;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= rows) return;
+  select_row_fp64(S + static_cast<size_t>(row) * T, T, top_k, top_p, cap, kv_index + static_cast<size_t>(row) * cap,
+                  kv_count + row, st, cnt_s[warp], mass_s[warp]);
+}
+
+// ======================================================================== fast router
+// The same decisions as the fp64 path above, at tensor-core speed.
+//
+//  * pooling .... as above, and each pooled row x (D values, fp64) is also written as an
+//                 exact fixed-point integer X = rint(x * 2^(30-E)) (E: the row's binary
+//                 exponent, |x_d| < 2^E) split into four signed 8-bit limbs,
+//                 X = d0 256^3 + d1 256^2 + d2 256 + d3 (d0 in [-64, 64], others [-128, 127]).
+//  * scores ..... Qbar Kbar^T from limb products on the tensor cores (tcgen05 kind::i8,
+//                 exact s32 accumulation): the products of limb pairs (a, b) with a + b = w
+//                 accumulate into level w (w = 0..3, ten products), and
+//                 v = L0 2^24 + L1 2^16 + L2 2^8 + L3 is the dot product in units of
+//                 2^(Eq + Ek - 36).  Dropping the levels w >= 4 and rounding the rows to 30
+//                 bits bound the error of a raw score by 4.03 * 2^-23 * 2^(Eq + Ek).
+//                 Each score is written as a 32-bit fixed-point key, key = rint(raw / 2^f_i),
+//                 with f_i chosen from a bound on the row (|raw| <= |Qbar_i|_1 2^Ekmax) so that
+//                 |key| <= 2^30.
+//  * selection .. one warp per row: radix descent on u = max_key - key (ascending u is
+//                 descending score), every bucket carrying its count and its fixed-point mass
+//                 exp(s - max) * 2^50 (exponential from ex2.approx on the fractional part,
+//                 relative error below 2^-21); the last bucket's few candidates are sorted
+//                 exactly (u, then id).  A row is accepted only if its decision cannot change
+//                 within the error bounds: the boundary key is more than twice the score bound
+//                 from the next key, and the Top-p crossing is farther from p * Z than the
+//                 masses' relative error.  Other rows (exact ties among them) are queued and
+//                 decided again by the fp64 path, so every row ends with the fp64 decision.
+
+struct RowMeta {
+  double cunit;    // log2 units of exp(s - max) per key unit: 2^f * scale * log2(e)
+  double eps_key;  // bound on a key's error, in key units
+  double eps_s;    // bound on a score's error, natural units (scaled)
+  double pad;
+};
+
+constexpr int kLimbRow = 128;  // bytes per limb row: K = 128 int8 (D = 64 rows are zero-padded)
+constexpr int kExpZero = -1100;  // exponent recorded for an all-zero row
+constexpr int kExpBias = 2048;   // exponents are kept as E + 2048 > 0 for the per-head atomicMax
+
+// grid (ceil(T/4), BH, 2); as pool_kernel, plus the limbs, exponents and (Q) 1-norms.
+template <int ESZ>
+__global__ void __launch_bounds__(256) pool_limbs_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ k,
+                                                         const float* __restrict__ q_scale,
+                                                         const float* __restrict__ k_scale, double* __restrict__ qbar,
+                                                         double* __restrict__ kbar, int8_t* __restrict__ qlimb,
+                                                         int8_t* __restrict__ klimb, int* __restrict__ qexp,
+                                                         int* __restrict__ kexp, double* __restrict__ ql1,
+                                                         unsigned* __restrict__ kexp_max, Geom g, int D) {
+  constexpr int EPT = 16 / ESZ;  // elements per 16-byte vector
+  __shared__ double red[4][64][EPT];
+  const int grp = threadIdx.x >> 6, t64 = threadIdx.x & 63;
+  const int c = blockIdx.x * 4 + grp;
+  const int bh = blockIdx.y;
+  const bool is_k = blockIdx.z == 1;
+  const uint8_t* src = is_k ? k : q;
+  const int tpr = D * ESZ / 16;  // threads per token row (4, 8 or 16: lanes 0..tpr-1 of the group's first warp)
+  const int rows_per_iter = 64 / tpr;
+  const int chunk = t64 % tpr, roff = t64 / tpr;
+  double acc[EPT];
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) acc[e] = 0.0;
+  int vt = 0, vh = 0, vw = 0;
+  if (c < g.T) {
+    cube_extent(g, c, vt, vh, vw);
+    const size_t row_bytes = static_cast<size_t>(D) * ESZ;
+    const uint8_t* base = src + (static_cast<size_t>(bh) * g.Npad + static_cast<size_t>(c) * 64) * row_bytes;
+    // eight rows' loads in flight per thread before any of them is accumulated
+    for (int r0 = roff; r0 < 64; r0 += 8 * rows_per_iter) {
+      uint4 v[8];
+      bool ok[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int r = r0 + u * rows_per_iter;
+        ok[u] = r < 64 && slot_valid(vt, vh, vw, r);
+        v[u] = ok[u] ? __ldg(reinterpret_cast<const uint4*>(base + r * row_bytes) + chunk) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (!ok[u]) continue;
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+          float f;
+          if constexpr (ESZ == 2) {
+            f = __uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
+          } else {
+            f = e4m3_value((w[e >> 2] >> (8 * (e & 3))) & 0xffu);
+          }
+          acc[e] += static_cast<double>(f);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) red[grp][t64][e] = acc[e];
+  __syncthreads();
+  if (c >= g.T || t64 >= tpr) return;
+  const int n = vt * vh * vw;
+  double scale = 1.0;
+  if constexpr (ESZ == 1) {
+    const float* sc = is_k ? k_scale : q_scale;
+    scale = static_cast<double>(sc[static_cast<size_t>(bh) * g.T + c]);
+  }
+  const size_t rowid = static_cast<size_t>(bh) * g.T + c;
+  double* dst = (is_k ? kbar : qbar) + rowid * D + chunk * EPT;
+  double x[EPT];
+  double amax = 0.0, l1 = 0.0;
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) {
+    double s = 0.0;
+    for (int r = 0; r < rows_per_iter; ++r) s += red[grp][t64 + r * tpr][e];
+    x[e] = s * scale / static_cast<double>(n);
+    dst[e] = x[e];
+    amax = fmax(amax, fabs(x[e]));
+    l1 += fabs(x[e]);
+  }
+  // row maximum and 1-norm over the tpr lanes holding the row
+  const unsigned mask = (tpr >= 32) ? 0xffffffffu : ((1u << tpr) - 1u);
+  for (int o = 1; o < tpr; o <<= 1) {
+    amax = fmax(amax, __shfl_xor_sync(mask, amax, o));
+    l1 += __shfl_xor_sync(mask, l1, o);
+  }
+  int E = kExpZero;
+  if (amax > 0.0) frexp(amax, &E);  // amax = m 2^E, m in [0.5, 1): every |x_d| < 2^E
+  const double up = amax > 0.0 ? ldexp(1.0, 30 - E) : 0.0;
+  uint32_t limb[4][EPT / 4];
+#pragma unroll
+  for (int w = 0; w < EPT / 4; ++w) limb[0][w] = limb[1][w] = limb[2][w] = limb[3][w] = 0u;
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) {
+    int X = static_cast<int>(rint(x[e] * up));  // |X| <= 2^30
+    const int d3 = ((X + 128) & 255) - 128;
+    X = (X - d3) >> 8;
+    const int d2 = ((X + 128) & 255) - 128;
+    X = (X - d2) >> 8;
+    const int d1 = ((X + 128) & 255) - 128;
+    const int d0 = (X - d1) >> 8;  // in [-64, 64]
+    const int sh = 8 * (e & 3);
+    limb[0][e >> 2] |= (static_cast<uint32_t>(d0) & 255u) << sh;
+    limb[1][e >> 2] |= (static_cast<uint32_t>(d1) & 255u) << sh;
+    limb[2][e >> 2] |= (static_cast<uint32_t>(d2) & 255u) << sh;
+    limb[3][e >> 2] |= (static_cast<uint32_t>(d3) & 255u) << sh;
+  }
+  int8_t* lb = (is_k ? klimb : qlimb);
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    int8_t* row = lb + ((static_cast<size_t>(bh) * 4 + a) * g.T + c) * kLimbRow;
+    if constexpr (EPT == 8) {
+      *reinterpret_cast<uint2*>(row + chunk * EPT) = make_uint2(limb[a][0], limb[a][1]);
+      if (D < kLimbRow) *reinterpret_cast<uint2*>(row + D + chunk * EPT) = make_uint2(0u, 0u);
+    } else {
+      *reinterpret_cast<uint4*>(row + chunk * EPT) = make_uint4(limb[a][0], limb[a][1], limb[a][2], limb[a][3]);
+      if (D < kLimbRow) *reinterpret_cast<uint4*>(row + D + chunk * EPT) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  if (chunk == 0) {
+    if (is_k) {
+      kexp[rowid] = E;
+      atomicMax(kexp_max + bh, static_cast<unsigned>(E + kExpBias));
+    } else {
+      qexp[rowid] = E;
+      ql1[rowid] = l1;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------ exact scores
+namespace rsc {
+constexpr int kThreads = 320;  // warp 0 TMA, warp 1 TMEM owner + MMA, warps 2-9 epilogue
+constexpr uint32_t OFF_Q = 0;                      // 4 limbs x [128 rows][128 B]
+constexpr uint32_t OFF_K = 65536;                  // 2 stages x 4 limbs x [128 keys][128 B]
+constexpr uint32_t OFF_BAR = OFF_K + 2 * 65536;
+constexpr uint32_t OFF_SLOT = OFF_BAR + 128;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
+constexpr uint32_t TMEM_COLS = 512;                // level w at columns 128w
+enum { B_QF = 0, B_QE = 1, B_KF = 2, B_KE = 4, B_TF = 6, B_TE = 7, B_FIN = 8, NBAR = 9 };
+}  // namespace rsc
+
+struct ScoreArgs {
+  const int* qexp;
+  const int* kexp;
+  const double* ql1;
+  const unsigned* kexp_max;
+  int* keys;        // [BH*T, Tk]
+  RowMeta* meta;    // [BH*T]
+  DevStatus* st;
+  int T, Tk, BH;
+  double scale;
+  unsigned long long timeout_ns;
+};
+
+// KS = D / 32 k-steps of 32 int8 per product.  Work item = one 128 x 128 tile of (query
+// cubes, key cubes) of one head; each CTA takes a contiguous run of items, so consecutive
+// items share their query rows (loaded once per row block).
+template <int KS>
+__global__ void __launch_bounds__(rsc::kThreads, 1)
+    score_keys_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const ScoreArgs a) {
+  using namespace rsc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_SLOT);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = a.T;
+  const int nrb = (T + 127) >> 7;
+  const long long n_items = static_cast<long long>(a.BH) * nrb * nrb;
+  const long long t0 = n_items * blockIdx.x / gridDim.x, t1 = n_items * (blockIdx.x + 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < NBAR; ++b) mbar_init(&bars[b], b == B_TE ? 256u : 1u);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool skip_all = aborted(a.st);
+
+  if (warp == 0) {
+    if (lane == 0 && !skip_all) {
+      uint32_t ks = 0;
+      int qn = 0;
+      long long prev = -1;
+      bool ok = true;
+      for (long long t = t0; ok && t < t1; ++t) {
+        const int bh = static_cast<int>(t / (static_cast<long long>(nrb) * nrb));
+        const int rem = static_cast<int>(t % (static_cast<long long>(nrb) * nrb));
+        const int rb = rem / nrb, cb = rem % nrb;
+        const long long rbk = static_cast<long long>(bh) * nrb + rb;
+        if (rbk != prev) {
+          if (qn >= 1 && !mbar_wait(&bars[B_QE], (qn - 1) & 1, a.st, a.timeout_ns, 101)) break;
+          mbar_arrive_expect_tx(&bars[B_QF], 65536);
+#pragma unroll
+          for (int l = 0; l < 4; ++l) tma_load_3d(smem + OFF_Q + l * 16384, &tm_q, &bars[B_QF], 0, rb * 128, bh * 4 + l);
+          ++qn;
+          prev = rbk;
+        }
+        const uint32_t st = ks & 1u;
+        if (ks >= 2 && !mbar_wait(&bars[B_KE + st], ((ks >> 1) + 1) & 1, a.st, a.timeout_ns, 102)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&bars[B_KF + st], 65536);
+#pragma unroll
+        for (int l = 0; l < 4; ++l)
+          tma_load_3d(smem + OFF_K + st * 65536 + l * 16384, &tm_k, &bars[B_KF + st], 0, cb * 128, bh * 4 + l);
+        ++ks;
+      }
+      // drain: never leave the CTA with copies in flight
+      if (qn > 0) mbar_wait_drain(&bars[B_QF], (qn - 1) & 1, a.st, a.timeout_ns, 103);
+      for (uint32_t s = (ks > 2 ? ks - 2 : 0); s < ks; ++s)
+        mbar_wait_drain(&bars[B_KF + (s & 1u)], (s >> 1) & 1, a.st, a.timeout_ns, 104);
+    }
+  } else if (warp == 1) {
+    if (!skip_all) {
+      const uint32_t idesc = make_idesc_s8(128, 128);
+      uint32_t ks = 0, tile = 0;
+      int qn = 0;
+      long long prev = -1;
+      bool ok = true;
+      for (long long t = t0; ok && t < t1; ++t) {
+        const int bh = static_cast<int>(t / (static_cast<long long>(nrb) * nrb));
+        const int rem = static_cast<int>(t % (static_cast<long long>(nrb) * nrb));
+        const int rb = rem / nrb;
+        const long long rbk = static_cast<long long>(bh) * nrb + rb;
+        if (rbk != prev) {
+          if (!mbar_wait_warp(&bars[B_QF], qn & 1, a.st, a.timeout_ns, 111)) break;
+          ++qn;
+          prev = rbk;
+        }
+        const long long tn = t + 1;
+        const bool last_of_rb =
+            tn >= t1 || (tn / (static_cast<long long>(nrb) * nrb)) * nrb +
+                                (tn % (static_cast<long long>(nrb) * nrb)) / nrb != rbk;
+        if (tile >= 1 && !mbar_wait_warp(&bars[B_TE], (tile - 1) & 1, a.st, a.timeout_ns, 112)) break;
+        const uint32_t st = ks & 1u;
+        if (!mbar_wait_warp(&bars[B_KF + st], (ks >> 1) & 1, a.st, a.timeout_ns, 113)) break;
+        tc_fence_after();
+        const uint32_t kb = sbase + OFF_K + st * 65536;
+        if (elect_one()) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+#pragma unroll
+            for (int la = 0; la <= w; ++la) {
+              const int lb = w - la;
+#pragma unroll
+              for (int kk = 0; kk < KS; ++kk)
+                umma_i8_ss(tmem + 128 * w, sw128_desc(sbase + OFF_Q + la * 16384 + kk * 32, 16, 1024),
+                           sw128_desc(kb + lb * 16384 + kk * 32, 16, 1024), idesc, (la > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&bars[B_KE + st]);
+          umma_commit(&bars[B_TF]);
+          if (last_of_rb) umma_commit(&bars[B_QE]);
+        }
+        __syncwarp();
+        ++ks;
+        ++tile;
+      }
+      if (elect_one()) umma_commit(&bars[B_FIN]);
+      __syncwarp();
+      mbar_wait_drain(&bars[B_FIN], 0, a.st, a.timeout_ns, 114);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int quarter = warp & 3, half = (warp - 2) >> 2;
+    const int r = quarter * 32 + lane;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    uint32_t tile = 0;
+    bool ok = !skip_all;
+    for (long long t = t0; ok && t < t1; ++t, ++tile) {
+      const int bh = static_cast<int>(t / (static_cast<long long>(nrb) * nrb));
+      const int rem = static_cast<int>(t % (static_cast<long long>(nrb) * nrb));
+      const int rb = rem / nrb, cb = rem % nrb;
+      const int i = rb * 128 + r;
+      const bool row_ok = i < T;
+      const size_t rowid = static_cast<size_t>(bh) * T + (row_ok ? i : 0);
+      // per-row scaling of the keys: |raw| <= |Qbar_i|_1 2^Ekmax < 2^e, keys in units of 2^(e - 30)
+      int A = 0;
+      int f = 0;
+      const int Eq = __ldg(a.qexp + rowid);
+      const int Ekm = static_cast<int>(__ldg(a.kexp_max + bh)) - kExpBias;
+      const double B = ldexp(__ldg(a.ql1 + rowid), Ekm);
+      const bool nonzero = Eq != kExpZero && Ekm != kExpZero && B > 0.0;
+      if (nonzero) {
+        int e;
+        frexp(B, &e);
+        f = e - 30;
+      }
+      A = 36 + f - Eq;
+      if (row_ok && cb == 0 && half == 0) {
+        RowMeta m;
+        m.cunit = ldexp(a.scale * 1.4426950408889634, f);
+        const double eps_raw = nonzero ? 4.03 * ldexp(1.0, Eq + Ekm - 23) : 0.0;
+        m.eps_key = eps_raw * ldexp(1.0, -f) + 1.0;
+        m.eps_s = (eps_raw + ldexp(1.0, f)) * a.scale;
+        m.pad = 0.0;
+        a.meta[rowid] = m;
+      }
+      if (!mbar_wait(&bars[B_TF], tile & 1, a.st, a.timeout_ns, 121)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      int* krow = a.keys + rowid * a.Tk;
+      const int* ekp = a.kexp + static_cast<size_t>(bh) * T;
+#pragma unroll 1
+      for (int ch = 0; ch < 2; ++ch) {
+        const int col0 = 64 * half + 32 * ch;
+        uint32_t L0[32], L1[32], L2[32], L3[32];
+        tmem_ld32(t_lane + 0 + col0, L0);
+        tmem_ld32(t_lane + 128 + col0, L1);
+        tmem_ld32(t_lane + 256 + col0, L2);
+        tmem_ld32(t_lane + 384 + col0, L3);
+        tmem_ld_wait();
+        if (ch == 1) {
+          tc_fence_before();
+          mbar_arrive(&bars[B_TE]);  // this thread's reads of the tile are complete
+        }
+        const int j0 = cb * 128 + col0;
+        if (!row_ok) continue;
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          int kv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int c = 4 * c4 + u;
+            const int j = j0 + c;
+            const long long hiw = static_cast<long long>(static_cast<int>(L0[c])) * 256 + static_cast<int>(L1[c]);
+            const long long low = static_cast<long long>(static_cast<int>(L2[c])) * 256 + static_cast<int>(L3[c]);
+            const long long v = hiw * 65536 + low;
+            int sh = A - (j < T ? __ldg(ekp + j) : 0);
+            sh = sh < 1 ? 1 : (sh > 62 ? 62 : sh);
+            kv[u] = static_cast<int>((v + (1LL << (sh - 1))) >> sh);
+          }
+          const int j = j0 + 4 * c4;
+          if (j + 3 < T) {
+            *reinterpret_cast<int4*>(krow + j) = make_int4(kv[0], kv[1], kv[2], kv[3]);
+          } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (j + u < T) krow[j + u] = kv[u];
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, rsc::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------------ key selection
+// 2^50 * 2^(-u c): the fixed-point mass of a score u key units below the row maximum.
+__device__ __forceinline__ unsigned long long mass_key(uint32_t u, double c) {
+  const double x = -static_cast<double>(u) * c;
+  if (x < -60.0) return 0ull;
+  const double fl = floor(x);
+  const float p2 = ex2_approx(static_cast<float>(x - fl));  // in [1, 2)
+  const int ex = static_cast<int>(fl) + 50;                 // >= -10
+  const double m = static_cast<double>(p2) * __longlong_as_double(static_cast<long long>(ex + 1023) << 52);
+  return static_cast<unsigned long long>(__double2ull_rz(m));
+}
+
+constexpr unsigned kDebugRouterFallback = 2u;  // debug flag: every row takes the fp64 path
+
+// One warp per row of keys.  Writes the row's list and count when its decision is certain;
+// otherwise appends the row to `flist` (length in st->router_fallback) for the fp64 path.
+__global__ void __launch_bounds__(256) select_keys_kernel(const int* __restrict__ keys, int Tk,
+                                                          const RowMeta* __restrict__ meta, int rows, int T, int top_k,
+                                                          float top_p, int cap, int32_t* __restrict__ kv_index,
+                                                          int32_t* __restrict__ kv_count, int* __restrict__ flist,
+                                                          DevStatus* st, unsigned debug) {
+  __shared__ uint32_t cnt_s[8][256];
+  __shared__ unsigned long long mass_s[8][256];
+  __shared__ unsigned long long cand_s[8][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= rows) return;
+  const int* kr = keys + static_cast<size_t>(row) * Tk;
+  uint32_t* cnt = cnt_s[warp];
+  unsigned long long* mass = mass_s[warp];
+  int32_t* out = kv_index + static_cast<size_t>(row) * cap;
+  const int nk = max(1, min(top_k, T));
+  if (top_p >= 1.0f || nk >= T) {  // every block
+    for (int j = lane; j < T && j < cap; j += 32) out[j] = j;
+    if (lane == 0) {
+      if (T > cap) flag_error(st, DEVERR_CAPACITY, 0);
+      kv_count[row] = min(T, cap);
+    }
+    return;
+  }
+  // ---- maximum and minimum key
+  int kmax = INT_MIN, kmin = INT_MAX;
+  for (int j0 = 0; j0 < T; j0 += 128) {
+    const int j = j0 + 4 * lane;
+    if (j < T) {
+      const int4 v = *reinterpret_cast<const int4*>(kr + j);
+      const int vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (j + u < T) {
+          kmax = max(kmax, vv[u]);
+          kmin = min(kmin, vv[u]);
+        }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+  }
+  const RowMeta m = meta[row];
+  const double c = m.cunit;
+  // ---- radix descent on u = kmax - key over [lo, hi]
+  uint32_t lo = 0, hi = static_cast<uint32_t>(kmax - kmin);
+  unsigned long long c_above = 0, m_above = 0, Z = 0;
+  double target = -1.0;
+  uint32_t bcnt = 0;
+  for (int level = 0;; ++level) {
+    const uint32_t span = hi - lo;
+    const int s = span < 256u ? 0 : (32 - __clz(span)) - 8;  // (hi - lo) >> s < 256
+    for (int d = lane; d < 256; d += 32) {
+      cnt[d] = 0;
+      mass[d] = 0ull;
+    }
+    __syncwarp();
+    for (int j0 = 0; j0 < T; j0 += 128) {
+      const int j = j0 + 4 * lane;
+      if (j < T) {
+        const int4 v = *reinterpret_cast<const int4*>(kr + j);
+        const int vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u4 = 0; u4 < 4; ++u4) {
+          const uint32_t uu = static_cast<uint32_t>(kmax - vv[u4]);
+          if (j + u4 < T && uu >= lo && uu <= hi) {
+            const int b = static_cast<int>((uu - lo) >> s);
+            atomicAdd(&cnt[b], 1u);
+            atomicAdd(&mass[b], mass_key(uu, c));
+          }
+        }
+      }
+    }
+    __syncwarp();
+    uint32_t lc = 0;
+    unsigned long long lm = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      lc += cnt[lane * 8 + u];
+      lm += mass[lane * 8 + u];
+    }
+    uint32_t ic = lc;
+    unsigned long long im = lm;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t oc = __shfl_up_sync(0xffffffffu, ic, o);
+      const unsigned long long om = __shfl_up_sync(0xffffffffu, im, o);
+      if (lane >= o) {
+        ic += oc;
+        im += om;
+      }
+    }
+    if (level == 0) {
+      Z = __shfl_sync(0xffffffffu, im, 31);
+      if (top_p > 0.0f) target = static_cast<double>(top_p) * static_cast<double>(Z);
+    }
+    unsigned long long c_run = c_above + (ic - lc), m_run = m_above + (im - lm);
+    int hit = -1;
+    unsigned long long c_before = 0, m_before = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t cu = cnt[lane * 8 + u];
+      const unsigned long long mu = mass[lane * 8 + u];
+      if (hit < 0 && cu > 0 && c_run + cu >= static_cast<unsigned long long>(nk) &&
+          static_cast<double>(m_run + mu) >= target) {
+        hit = lane * 8 + u;
+        c_before = c_run;
+        m_before = m_run;
+      }
+      c_run += cu;
+      m_run += mu;
+    }
+    const uint32_t bal = __ballot_sync(0xffffffffu, hit >= 0);
+    if (bal == 0u) {  // cannot happen (the totals meet both conditions); decide the row in fp64
+      bcnt = 0xffffffffu;
+      break;
+    }
+    const int src = __ffs(bal) - 1;
+    const int bstar = __shfl_sync(0xffffffffu, hit, src);
+    c_above = __shfl_sync(0xffffffffu, c_before, src);
+    m_above = __shfl_sync(0xffffffffu, m_before, src);
+    bcnt = cnt[bstar];
+    __syncwarp();
+    const unsigned long long nlo = static_cast<unsigned long long>(lo) + (static_cast<unsigned long long>(bstar) << s);
+    const unsigned long long nhi = nlo + (1ull << s) - 1ull;
+    lo = static_cast<uint32_t>(nlo);
+    hi = static_cast<uint32_t>(nhi < hi ? nhi : hi);
+    if (bcnt <= 32u || s == 0) break;
+  }
+  bool certain = bcnt <= 32u && (debug & kDebugRouterFallback) == 0u;
+  uint32_t ub = 0;
+  int jb = -1, n = 0;
+  unsigned long long cum_at = 0, cum_before = 0;
+  if (certain) {
+    // ---- the boundary bucket's candidates, sorted by (u, id)
+    int nc = 0;
+    for (int j0 = 0; j0 < T; j0 += 128) {
+      const int j = j0 + 4 * lane;
+      int4 v = make_int4(0, 0, 0, 0);
+      if (j < T) v = *reinterpret_cast<const int4*>(kr + j);
+      const int vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const uint32_t uu = static_cast<uint32_t>(kmax - vv[u4]);
+        const bool in = j + u4 < T && uu >= lo && uu <= hi;
+        const uint32_t b = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          const int pos = nc + __popc(b & ((1u << lane) - 1u));
+          if (pos < 32) cand_s[warp][pos] = (static_cast<unsigned long long>(uu) << 32) | static_cast<uint32_t>(j + u4);
+        }
+        nc += __popc(b);
+      }
+    }
+    __syncwarp();
+    unsigned long long key = lane < static_cast<int>(bcnt) ? cand_s[warp][lane] : ~0ull;
+    // bitonic sort of 32 keys across the warp, ascending
+#pragma unroll
+    for (int k2 = 2; k2 <= 32; k2 <<= 1) {
+#pragma unroll
+      for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
+        const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, j2);
+        const bool up = (lane & k2) == 0;
+        const bool lower = (lane & j2) == 0;
+        const bool take_min = (lower == up);
+        key = take_min ? (key < other ? key : other) : (key > other ? key : other);
+      }
+    }
+    const bool valid = lane < static_cast<int>(bcnt);
+    const uint32_t uu = static_cast<uint32_t>(key >> 32);
+    const unsigned long long ms = valid ? mass_key(uu, c) : 0ull;
+    unsigned long long pm = ms;
+    uint32_t pc = valid ? 1u : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long t1 = __shfl_up_sync(0xffffffffu, pm, o);
+      const uint32_t t2 = __shfl_up_sync(0xffffffffu, pc, o);
+      if (lane >= o) {
+        pm += t1;
+        pc += t2;
+      }
+    }
+    const bool okb = valid && (c_above + pc >= static_cast<unsigned long long>(nk)) &&
+                     (static_cast<double>(m_above + pm) >= target);
+    const uint32_t okm = __ballot_sync(0xffffffffu, okb);
+    if (okm == 0u) {
+      certain = false;
+    } else {
+      const int L = __ffs(okm) - 1;
+      ub = __shfl_sync(0xffffffffu, uu, L);
+      jb = static_cast<int>(__shfl_sync(0xffffffffu, static_cast<uint32_t>(key & 0xffffffffull), L));
+      n = static_cast<int>(c_above) + L + 1;
+      cum_at = m_above + __shfl_sync(0xffffffffu, pm, L);
+      cum_before = cum_at - __shfl_sync(0xffffffffu, ms, L);
+    }
+  }
+  if (certain) {
+    // ---- emit the kept ids in ascending order; the smallest u left out is the next key
+    int written = 0;
+    uint32_t unext = 0xffffffffu;
+    for (int j0 = 0; j0 < T; j0 += 128) {
+      const int j = j0 + 4 * lane;
+      int4 v = make_int4(0, 0, 0, 0);
+      if (j < T) v = *reinterpret_cast<const int4*>(kr + j);
+      const int vv[4] = {v.x, v.y, v.z, v.w};
+      bool sel[4];
+      int nsel = 0;
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const uint32_t uu = static_cast<uint32_t>(kmax - vv[u4]);
+        const bool in = j + u4 < T;
+        sel[u4] = in && (uu < ub || (uu == ub && j + u4 <= jb));
+        if (in && !sel[u4]) unext = min(unext, uu);
+        nsel += sel[u4] ? 1 : 0;
+      }
+      int incl = nsel;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int pos = written + incl - nsel;
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4)
+        if (sel[u4]) {
+          if (pos < cap) out[pos] = j + u4;
+          ++pos;
+        }
+      written += __shfl_sync(0xffffffffu, incl, 31);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) unext = min(unext, __shfl_xor_sync(0xffffffffu, unext, o));
+    // ---- is the decision certain within the error bounds?
+    const double Zd = static_cast<double>(Z);
+    const double delta = (2.0 * m.eps_s + 2.0 * 4.76837158203125e-07 + 1e-12) * Zd;  // 2^-21
+    bool gap_ok = unext == 0xffffffffu || static_cast<double>(unext - ub) > 2.0 * m.eps_key;
+    bool cross_ok = true;
+    if (top_p > 0.0f) {
+      if (n > nk)
+        cross_ok = fabs(static_cast<double>(cum_at) - target) > delta &&
+                   fabs(static_cast<double>(cum_before) - target) > delta;
+      else
+        cross_ok = static_cast<double>(cum_at) - target > delta;
+    }
+    certain = gap_ok && cross_ok && written == n;
+    if (certain && lane == 0) {
+      if (n > cap) flag_error(st, DEVERR_CAPACITY, 0);
+      kv_count[row] = min(n, cap);
+    }
+  }
+  if (!certain && lane == 0) {
+    const unsigned k = atomicAdd(&st->router_fallback, 1u);
+    flist[k] = row;
+  }
+}
+
+// The fp64 path for the rows the key selection queued: each warp recomputes the row's scores
+// Qbar_i . Kbar_j * scale in fp64 into its own scratch row, then selects as select_kernel does.
+__global__ void __launch_bounds__(128) router_fallback_kernel(const double* __restrict__ qbar,
+                                                              const double* __restrict__ kbar, int D, int T,
+                                                              double scale, const int* __restrict__ flist,
+                                                              double* __restrict__ scratch, int top_k, float top_p,
+                                                              int cap, int32_t* __restrict__ kv_index,
+                                                              int32_t* __restrict__ kv_count, DevStatus* st) {
+  __shared__ uint32_t cnt_s[4][256];
+  __shared__ unsigned long long mass_s[4][256];
+  __shared__ double qs[4][128];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * 4 + warp, nw = gridDim.x * 4;
+  const int nf = static_cast<int>(*reinterpret_cast<const volatile unsigned*>(&st->router_fallback));
+  double* s = scratch + static_cast<size_t>(gw) * T;
+  for (int k = gw; k < nf; k += nw) {
+    const int row = flist[k];
+    const size_t bh = static_cast<size_t>(row) / T;
+    for (int d = lane; d < D; d += 32) qs[warp][d] = qbar[static_cast<size_t>(row) * D + d];
+    __syncwarp();
+    for (int j = lane; j < T; j += 32) {
+      const double* kj = kbar + (bh * T + j) * D;
+      double acc = 0.0;
+      for (int d = 0; d < D; ++d) acc = fma(qs[warp][d], kj[d], acc);
+      s[j] = acc * scale;
+    }
+    __syncwarp();
+    select_row_fp64(s, T, top_k, top_p, cap, kv_index + static_cast<size_t>(row) * cap, kv_count + row, st,
+                    cnt_s[warp], mass_s[warp]);
+    __syncwarp();
   }
 }
 
@@ -425,6 +1137,66 @@ cudaError_t launch_pool(const void* q, const void* k, const Geom& g, int BH, int
 cudaError_t launch_select(const double* S, int32_t* kv_index, int32_t* kv_count, int rows, int T, int top_k,
                           float top_p, int cap, DevStatus* st, cudaStream_t stream) {
   select_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(S, kv_index, kv_count, rows, T, top_k, top_p, cap, st);
+  return cudaGetLastError();
+}
+
+// fixed (not the device's SM count) so that workspace sizes do not depend on the device
+int plan_fallback_ctas() { return 148; }
+
+cudaError_t launch_plan_fast(const void* q, const void* k, const float* q_scale, const float* k_scale,
+                             const CUtensorMap& tm_qlimb, const CUtensorMap& tm_klimb, const Geom& g, int BH, int D,
+                             bool fp8, double scale, int top_k, float top_p, int cap, unsigned debug,
+                             unsigned long long timeout_ns, const PlanFastWs& w, int32_t* kv_index, int32_t* kv_count,
+                             DevStatus* st, cudaStream_t stream, int* launches) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(score_keys_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         rsc::SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(score_keys_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsc::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  // the per-head maxima of the key exponents start at 0 (below every biased exponent)
+  if (cudaMemsetAsync(w.kexp_max, 0, static_cast<size_t>(BH) * sizeof(unsigned), stream) != cudaSuccess)
+    return cudaErrorUnknown;
+  dim3 pg((g.T + 3) / 4, BH, 2);
+  if (fp8)
+    pool_limbs_kernel<1><<<pg, 256, 0, stream>>>(static_cast<const uint8_t*>(q), static_cast<const uint8_t*>(k),
+                                                 q_scale, k_scale, w.qbar, w.kbar, w.qlimb, w.klimb, w.qexp, w.kexp,
+                                                 w.ql1, w.kexp_max, g, D);
+  else
+    pool_limbs_kernel<2><<<pg, 256, 0, stream>>>(static_cast<const uint8_t*>(q), static_cast<const uint8_t*>(k),
+                                                 q_scale, k_scale, w.qbar, w.kbar, w.qlimb, w.klimb, w.qexp, w.kexp,
+                                                 w.ql1, w.kexp_max, g, D);
+  ScoreArgs sa_;
+  sa_.qexp = w.qexp;
+  sa_.kexp = w.kexp;
+  sa_.ql1 = w.ql1;
+  sa_.kexp_max = w.kexp_max;
+  sa_.keys = w.keys;
+  sa_.meta = reinterpret_cast<RowMeta*>(w.meta);
+  sa_.st = st;
+  sa_.T = g.T;
+  sa_.Tk = w.Tk;
+  sa_.BH = BH;
+  sa_.scale = scale;
+  sa_.timeout_ns = timeout_ns;
+  const int nrb = (g.T + 127) / 128;
+  const long long items = static_cast<long long>(BH) * nrb * nrb;
+  const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
+  if (D == 64)
+    score_keys_kernel<2><<<grid, rsc::kThreads, rsc::SMEM_BYTES, stream>>>(tm_qlimb, tm_klimb, sa_);
+  else
+    score_keys_kernel<4><<<grid, rsc::kThreads, rsc::SMEM_BYTES, stream>>>(tm_qlimb, tm_klimb, sa_);
+  const int rows = BH * g.T;
+  select_keys_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(w.keys, w.Tk, reinterpret_cast<const RowMeta*>(w.meta), rows,
+                                                         g.T, top_k, top_p, cap, kv_index, kv_count, w.flist, st,
+                                                         debug);
+  router_fallback_kernel<<<plan_fallback_ctas(), 128, 0, stream>>>(w.qbar, w.kbar, D, g.T, scale, w.flist,
+                                                                   w.fb_scratch, top_k, top_p, cap, kv_index,
+                                                                   kv_count, st);
+  *launches = 5;
   return cudaGetLastError();
 }
 

@@ -80,6 +80,9 @@ typedef struct {
 /* Test hook: the forward kernel's producer issues no loads, so its consumers' bounded
  * waits run out and the call reports SA_ERR_DEVICE_TIMEOUT without faulting. */
 #define SA_DEBUG_SKIP_LOADS 1u
+/* Test hook: sa_plan decides every row on its fp64 path (normally taken only by the rows
+ * whose tensor-core decision is within the error bound of changing). */
+#define SA_DEBUG_ROUTER_FALLBACK 2u
 
 /* Padded token count Npad and cube count T implied by the latent grid (0 on bad input). */
 SA_API int sa_padded_tokens(const sa_params* p);
@@ -90,7 +93,9 @@ SA_API int sa_num_cubes(const sa_params* p);
 SA_API int sa_topk_from_fraction(double frac, int T);
 
 /* Bytes of device workspace `op` (sa_op) needs for these parameters; 0 on bad input.
- * Plan: status block + pooled Q and K (fp64) + block scores (fp64, B*H*T*T).
+ * Plan: status block + pooled Q and K (fp64, 2*B*H*T*D) + their int8 limbs (8*B*H*T*128) + per-row
+ * exponents, norms and key scaling (48*B*H*T) + the fixed-point score keys (int32, B*H*T*Tk, Tk = T
+ * rounded up to 4) + the fp64 rows' list (B*H*T) and scratch (fp64, 592*T).
  * Forward: status block + one 64-bit valid-slot mask per cube (T) + the union lists of
  * adjacent query-cube pairs (int32, B*H*ceil(T/2)*(1 + 2*kv_capacity)).  Backward: status block
  * + cube masks + Delta and -lse*log2(e) (fp32, 2*B*H*Npad) + the selection as a bit matrix
@@ -110,6 +115,27 @@ SA_API size_t sa_workspace_size(const sa_params* p, int op);
 SA_API sa_status sa_tile(const void* x_latent, void* x_tiled, const sa_params* p, int elem_bytes, sa_stream_t stream);
 SA_API sa_status sa_untile(const void* x_tiled, void* x_latent, const sa_params* p, int elem_bytes, sa_stream_t stream);
 
+/* The same permutation with the 3-D rotary position embedding fused in (VSA2 page, section 2.2
+ * "Permutation": the permutation to cube-major order is applied once at the start of the
+ * transformer with a matching permutation of the RoPE embeddings; RoFormer: channel pair
+ * (x_2i, x_2i+1) of a token at position m is rotated by m * theta_i).  The head dimension p->D
+ * splits into three even sections rope_dt + rope_dh + rope_dw = D, rotated by the token's t, h
+ * and w position.  rope_cos / rope_sin (fp32, device, caller-owned) hold the cosines and sines
+ * of the angles: lat_t rows of rope_dt/2 entries (axis t, row = position), then lat_h rows of
+ * rope_dh/2, then lat_w rows of rope_dw/2.  A pair (a, b) with cosine c and sine s becomes
+ * (a c - b s, a s + b c), computed in fp32 and rounded to the element type.
+ * sa_tile_rope: x_latent [B,H,L,D] -> x_tiled [B,H,Npad,D], padding slots 0.
+ * sa_untile_rope: x_tiled -> x_latent with the inverse rotation (a c + b s, -a s + b c), e.g. for
+ * gradients; padding slots are dropped.  elem_bytes: 2 (bf16) or 4 (fp32); D * elem_bytes a
+ * multiple of 16.  Errors: SA_ERR_INVALID_ARG (sections, sizes, NULL), SA_ERR_ALIGNMENT (tensors
+ * 16-byte, tables 4-byte aligned).  One launch, no workspace. */
+SA_API sa_status sa_tile_rope(const void* x_latent, void* x_tiled, const sa_params* p, int elem_bytes, int rope_dt,
+                              int rope_dh, int rope_dw, const float* rope_cos, const float* rope_sin,
+                              sa_stream_t stream);
+SA_API sa_status sa_untile_rope(const void* x_tiled, void* x_latent, const sa_params* p, int elem_bytes, int rope_dt,
+                                int rope_dh, int rope_dw, const float* rope_cos, const float* rope_sin,
+                                sa_stream_t stream);
+
 /* Router (SpargeAttention2 page, "Block-Pooled Attention", steps 2-4, and equation 9;
  * VSA page, "Kernel Implementation": contiguous arrays of block indices).
  * q, k: [B,H,Npad,D] bf16, or e4m3 bytes when qk_dtype == SA_FP8_E4M3, in which case
@@ -121,7 +147,13 @@ SA_API sa_status sa_untile(const void* x_tiled, void* x_latent, const sa_params*
  * Outputs: kv_count [B,H,T] int32 = number of kept blocks (clipped to kv_capacity, with
  * SA_ERR_CAPACITY recorded when clipping happened); kv_index [B,H,T,kv_capacity] int32
  * holds the kept block ids in ascending order in its first kv_count entries (the rest
- * are left untouched).  Deterministic. */
+ * are left untouched).  Deterministic.
+ * How it runs: the pooled rows are split into four exact 8-bit limbs and the scores come from
+ * integer tensor-core products (exact accumulation; each score within 4.03 * 2^-23 * 2^(Eq+Ek)
+ * * scale of its fp64 value, 2^Eq and 2^Ek bounding the two rows' entries), as 32-bit
+ * fixed-point keys; the selection runs on the keys with fixed-point masses, and every row whose
+ * decision could change within those error bounds (exact ties among them) is decided again from
+ * fp64 scores, so the result is the fp64 decision (sa_plan_fallback_rows counts those rows). */
 SA_API sa_status sa_plan(const void* q, const void* k, const float* q_scale, const float* k_scale, const sa_params* p,
                   int32_t* kv_index, int32_t* kv_count, void* ws, size_t ws_bytes, sa_stream_t stream);
 
@@ -258,6 +290,10 @@ SA_API sa_status sa_plan_static(const void* q, const void* k, const float* q_sca
  * SA_OK, SA_ERR_DEVICE_TIMEOUT, SA_ERR_DEVICE_INDEX or SA_ERR_CAPACITY (first that
  * applies, in that order of precedence: timeout, index, capacity). */
 SA_API sa_status sa_get_device_status(const void* ws, sa_stream_t stream);
+
+/* Synchronises `stream` and returns how many rows the last sa_plan on this workspace decided
+ * on its fp64 path; -1 on error. */
+SA_API int sa_plan_fallback_rows(const void* ws, sa_stream_t stream);
 
 SA_API const char* sa_status_string(sa_status s);
 

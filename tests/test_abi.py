@@ -39,7 +39,10 @@ def test_geometry_and_workspace(lib):
     assert lib.sa_topk_from_fraction(0.03, 1562) == 47
     T, BH = 1440, 40
     plan_ws = sa.workspace_size(p, sa.OP_PLAN)
-    assert plan_ws >= 256 + 2 * BH * T * 128 * 8 + BH * T * T * 8
+    # pooled rows (fp64) + their 4 int8 limbs + per-row data + int32 keys + fp64 rows' scratch
+    assert plan_ws >= 256 + 2 * BH * T * 128 * 8 + 2 * BH * 4 * T * 128 + BH * T * T * 4 + 592 * T * 8
+    # the routers that keep every fp64 score (coarse branch) need the full score matrix
+    assert sa.workspace_size(p, sa.OP_PLAN_COARSE) >= 256 + 2 * BH * T * 128 * 8 + BH * T * T * 8
     assert sa.workspace_size(p, sa.OP_FORWARD) >= 256 + 1440 * 8 + 40 * 720 * min(2 * 1440, 1440) * 4  # masks + pair unions
     assert sa.workspace_size(p, sa.OP_BACKWARD) >= BH * 92160 * 4 + BH * T * T * 4
 
@@ -91,9 +94,10 @@ def test_package_does_not_import_oracle():
 def test_coarse_entry_points_validate_on_the_host(lib):
     p = sa.make_params(2, 3, 64, (8, 8, 8), 4, 0.5)          # T = 8, B*H = 6
     T, BH, D, npad = 8, 6, 64, 512
-    plan, bwd = sa.workspace_size(p, sa.OP_PLAN), sa.workspace_size(p, sa.OP_BACKWARD)
-    # plan + Pc; backward + dOc^, three per-cube terms, delta_c, scores and dS (each 256-byte aligned)
-    assert sa.workspace_size(p, sa.OP_PLAN_COARSE) >= plan + BH * T * T * 4
+    bwd = sa.workspace_size(p, sa.OP_BACKWARD)
+    plan64 = 256 + 2 * BH * T * D * 8 + BH * T * T * 8      # status, fp64 Qbar, Kbar and every score
+    # fp64 plan + Pc; backward + dOc^, three per-cube terms, delta_c, scores and dS (each 256-byte aligned)
+    assert sa.workspace_size(p, sa.OP_PLAN_COARSE) >= plan64 + BH * T * T * 4
     assert sa.workspace_size(p, sa.OP_BACKWARD_GATED) >= bwd + 4 * BH * T * D * 4 + BH * T * 4 + 2 * BH * T * T * 4
     assert sa.workspace_size(p, 6) == 0
     bad = ctypes.c_void_p(16)
@@ -141,8 +145,8 @@ def test_recall_validates_on_the_host(lib):
 def test_plan_bq128_validates_on_the_host(lib):
     p = sa.make_params(1, 2, 64, (8, 8, 12), 4, 0.5)          # T = 12: 6 query blocks
     T, BH, M, D = 12, 2, 6, 64
-    plan = sa.workspace_size(p, sa.OP_PLAN)
-    # the plan's, then the block means (fp64) and the block lists and counts
+    plan = 256 + 2 * BH * T * D * 8 + BH * T * T * 8          # status, fp64 Qbar, Kbar and every score
+    # the fp64 plan's, then the block means (fp64) and the block lists and counts
     assert sa.workspace_size(p, sa.OP_PLAN_BQ128) >= plan + BH * M * D * 8 + BH * M * (T + 1) * 4
     bad = ctypes.c_void_p(16)
     assert lib.sa_plan_bq128(None, bad, ctypes.byref(p), bad, bad, bad, 1 << 30, None) == 1

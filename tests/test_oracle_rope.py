@@ -113,3 +113,12 @@ def test_planted_mistakes_fail(variant, monkeypatch):
         return y.reshape(lt, lw, lh, -1).transpose(0, 2, 1, 3).reshape(lt * lh * lw, -1)
     monkeypatch.setattr(R, "rope_3d", wrong)
     assert not _check_slots()
+
+
+def test_untile_rope_inverts_tile_rope():
+    rng = np.random.default_rng(2)
+    lat, sec = (5, 6, 7), (4, 6, 6)
+    lay = O.cube_layout(lat)
+    x = rng.standard_normal((lat[0] * lat[1] * lat[2], sum(sec)))
+    cos, sin = R.rope_tables(lat, sec, base=30.0)
+    assert np.allclose(R.untile_rope(R.tile_rope(x, lay, sec, cos, sin), lay, sec, cos, sin), x, rtol=0, atol=1e-13)
