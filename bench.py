@@ -17,6 +17,7 @@ sa_backward_gated), skipped with ``--no-fp8`` / ``--no-gated``.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -210,6 +211,7 @@ def run_ours(args, rank, world, dist):
             step(wl[s])
         torch.cuda.synchronize()
     clock_summary = clocks.summary(line0, line1)
+    balance = measure_balance(sa, p, x, res[0], res[1], flush)
     plan_ms, fwd_ms, bwd_ms = phases(recs)
     step_ms = [a + b + c for a, b, c in zip(plan_ms, fwd_ms, bwd_ms)]
     ms_per_step = max_over_ranks(statistics.median(step_ms), dist, dev)
@@ -266,6 +268,7 @@ def run_ours(args, rank, world, dist):
         "roofline": roofline,
         "gpu_launches": gpu_launches,
         "clocks": clock_summary,
+        "cta_balance": balance,
         "gen_s": round(t_gen, 1),
     }
     if args.e2e_steps > 0:
@@ -287,6 +290,43 @@ def run_ours(args, rank, world, dist):
         result["cpu_baseline"], result["parity_sample"] = cpu_baseline(cfg, host, gpu_sample, ntiles,
                                                                        seconds=args.cpu_seconds)
     return result
+
+
+def measure_balance(sa, p, x, idx, cnt, flush):
+    """One more forward + backward (not timed) with per-CTA clock records: for each attention
+    kernel, how long each CTA was busy (start to end, globaltimer) under the dynamic in-order
+    item schedule, and how its items and pipeline steps were spread."""
+    import torch
+    res = {"source": "globaltimer at each CTA's start and end (SA_DEBUG_CTA_CLOCKS), one untimed forward + backward "
+                     "per schedule, L2 flushed before each call"}
+    for sched, flag in (("dynamic", 0), ("static", sa.DEBUG_STATIC_ITEMS)):
+        pc = sa.make_params(p.B, p.H, p.D, (p.lat_t, p.lat_h, p.lat_w), p.top_k, p.top_p,
+                            kv_capacity=p.kv_capacity, debug_flags=sa.DEBUG_CTA_CLOCKS | flag)
+        wf, wb = sa.new_workspace(pc, sa.OP_FORWARD), sa.new_workspace(pc, sa.OP_BACKWARD)
+        flush.fill_(7)
+        out, lse, o32 = sa.forward(x["q"], x["k"], x["v"], idx, cnt, pc, ws=wf, with_f32=True)
+        flush.fill_(8)
+        sa.backward(x["q"], x["k"], x["v"], out, lse, x["do"], idx, cnt, pc, ws=wb, out_f32=o32)
+        torch.cuda.synchronize()
+        part = {"schedule": ("work items (cube pairs) in natural order from a per-launch counter, each to the next "
+                             "free CTA (the library's schedule)") if flag == 0 else
+                            "fixed round-robin share (CTA c: items c, c + grid, ...; SA_DEBUG_STATIC_ITEMS)"}
+        for kernel, name, ws in ((0, "attn_fwd_kernel", wf), (1, "attn_dq_kernel", wb), (2, "attn_dkdv_kernel", wb)):
+            r = sa.cta_clocks(ws, kernel).astype("float64")
+            if len(r) == 0:
+                continue
+            busy = (r[:, 1] - r[:, 0]) / 1e6
+            span = (r[:, 1].max() - r[:, 0].min()) / 1e6
+            part[name] = {"ctas": len(r), "span_ms": round(span, 4), "busy_ms_max": round(busy.max(), 4),
+                          "busy_ms_mean": round(busy.mean(), 4), "busy_ms_min": round(busy.min(), 4),
+                          "max_over_mean": round(busy.max() / busy.mean(), 4),
+                          "idle_frac": round(1.0 - busy.sum() / (len(r) * span), 4),
+                          "items": [int(r[:, 2].min()), int(r[:, 2].max())],
+                          "steps": [int(r[:, 3].min()), int(r[:, 3].max())],
+                          "steps_max_over_mean": round(r[:, 3].max() / r[:, 3].mean(), 4)}
+        res[sched] = part
+        del wf, wb, out, lse, o32
+    return res
 
 
 def valid_only_flops(sa, p, cfg, idx, cnt, dev):
@@ -534,8 +574,69 @@ def run_extras(args, sa, cfg, host, dev, flush, dist):
            "min_cube_recall": round(float(cube_cpu.min()), 4),
            "cubes_below_half": round(float((cube_cpu < 0.5).float().mean()), 4),
            "mean_blocks_per_row": round(float(cnt.float().mean()), 2)}
-    return {"config": f"{cfg.name}: sa_plan_bq128 + fine stage on its lists; recall of sa_plan's lists",
-            "steps": steps, "bq128": bq, "recall": rec}
+    # P_oracle (token-level softmax mass per block pair) and the best recall at the router's counts
+    pblock = sa.block_mass(t["q"], t["k"], lse_all, p)
+    best = sa.best_recall(pblock, cnt, p)
+    sel = torch.zeros_like(pblock)
+    ar = torch.arange(idx.shape[-1], device=dev)
+    keep = ar.view(1, 1, 1, -1) < cnt.unsqueeze(-1)
+    sel.scatter_(3, torch.where(keep, idx.long(), 0), keep.float())
+    got = (pblock * sel).sum(-1)
+    ratio = (got / best.clamp_min(1e-30)).float().cpu()
+    rec.update({"mean_oracle_recall": round(float(got.mean()), 4), "mean_best_recall": round(float(best.mean()), 4),
+                "mean_recall_over_best": round(float(ratio.mean()), 4),
+                "min_recall_over_best": round(float(ratio.min()), 4)})
+    del pblock, sel, lse_all
+    fine = run_fine_router(sa, cfg, t, p, T, dev, flush, steps)
+    return {"config": f"{cfg.name}: sa_plan_bq128 + fine stage on its lists; recall of sa_plan's lists "
+                      f"(token-level and against P_oracle's best at the same counts); VSA2 fine router",
+            "steps": steps, "bq128": bq, "recall": rec, "fine_router": fine}
+
+
+def run_fine_router(sa, cfg, t, p, T, dev, flush, steps, R=(2, 2, 2)):
+    """VSA2's fine-grained router (sa_plan_fine, group pooling R) timed alone and with the fine
+    forward and backward on its per-sequence Top-K lists."""
+    import torch
+    ws = {op: sa.new_workspace(p, op, dev) for op in (sa.OP_FORWARD, sa.OP_BACKWARD)}
+    idx = torch.empty((cfg.B, cfg.H, T, p.kv_capacity), dtype=torch.int32, device=dev)
+    cnt = torch.empty((cfg.B, cfg.H, T), dtype=torch.int32, device=dev)
+    n = int(sa.load_library().sa_plan_fine_workspace_size(ctypes.byref(p), *R))
+    wsf = torch.empty(n, dtype=torch.uint8, device=dev)
+
+    def step(rec=None):
+        if rec is not None:
+            rec[0].record()
+        sa.plan_fine(t["q"], t["k"], p, R=R, kv_index=idx, kv_count=cnt, ws=wsf)
+        if rec is not None:
+            rec[1].record()
+        out, lse, o32 = sa.forward(t["q"], t["k"], t["v"], idx, cnt, p, ws=ws[sa.OP_FORWARD], with_f32=True)
+        if rec is not None:
+            rec[2].record()
+        sa.backward(t["q"], t["k"], t["v"], out, lse, t["do"], idx, cnt, p, ws=ws[sa.OP_BACKWARD], out_f32=o32)
+        if rec is not None:
+            rec[3].record()
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    for w in list(ws.values()) + [wsf]:
+        st = sa.device_status(w)
+        if st != 0:
+            raise RuntimeError(f"fine router: device status {sa.STATUS_NAMES.get(st, st)}")
+    recs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for s in range(steps):
+        flush.fill_(s & 0xff)
+        step(recs[s])
+    torch.cuda.synchronize()
+    ms = [statistics.median(r[i].elapsed_time(r[i + 1]) for r in recs) for i in range(3)]
+    ntiles = int(cnt.sum().item())
+    fwd_fl, bwd_fl = tile_flops(cfg.D, ntiles)
+    c = cnt.float()
+    return {"R": list(R), "plan_fine_ms": round(ms[0], 4), "forward_ms": round(ms[1], 4),
+            "backward_ms": round(ms[2], 4), "selected_tiles": ntiles,
+            "density": round(ntiles / (cfg.B * cfg.H * T * T), 5),
+            "blocks_per_row": {"mean": round(float(c.mean()), 2), "min": int(c.min()), "max": int(c.max())},
+            "effective_tflops": round((fwd_fl + bwd_fl) / (sum(ms) * 1e-3) / 1e12, 3)}
 
 
 def cta_balance(masks, sms: int):
@@ -591,8 +692,10 @@ def selection_masks(idx, cnt):
 
 def run_sweep(args):
     """Config-4 sweep at the 720p shape: k = 4, p in {0.8, 0.9, 0.95}, locality amplitude calibrated
-    (at p = 0.9) for 80..98% sparsity.  One JSON line per point: step timings and the per-CTA
-    load balance of the persistent attention kernels."""
+    (at p = 0.9) for 80..98% sparsity.  One JSON line per point: step timings, the per-CTA load
+    balance of the persistent attention kernels predicted from the lists under a fixed
+    round-robin share, and the measured per-CTA busy times under the dynamic and the fixed
+    schedules."""
     import torch
 
     import block_sparse_attention_cubes_b200 as sa
@@ -646,7 +749,8 @@ def run_sweep(args):
                     "plan_ms": round(ms[0], 3), "forward_ms": round(ms[1], 3), "backward_ms": round(ms[2], 3),
                     "forward_tflops": round(fwd_fl / (ms[1] * 1e-3) / 1e12, 1),
                     "backward_tflops": round(bwd_fl / (ms[2] * 1e-3) / 1e12, 1),
-                    "balance": cta_balance(masks, sms)}
+                    "balance": cta_balance(masks, sms),
+                    "measured_balance": measure_balance(sa, p, x, idx, cnt, flush)}
             print(json.dumps(line), flush=True)
             del x, A
 

@@ -31,16 +31,19 @@ SA_OK = 0
 STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_ALIGNMENT",
                 4: "SA_ERR_CAPACITY", 5: "SA_ERR_WORKSPACE", 6: "SA_ERR_LAUNCH", 7: "SA_ERR_DEVICE_TIMEOUT",
                 8: "SA_ERR_DEVICE_INDEX"}
-OP_PLAN, OP_FORWARD, OP_BACKWARD, OP_PLAN_COARSE, OP_BACKWARD_GATED, OP_PLAN_BQ128 = 0, 1, 2, 3, 4, 5
+OP_PLAN, OP_FORWARD, OP_BACKWARD, OP_PLAN_COARSE, OP_BACKWARD_GATED, OP_PLAN_BQ128, OP_BLOCK_MASS = 0, 1, 2, 3, 4, 5, 6
 BF16, FP8_E4M3 = 0, 1
 DEBUG_SKIP_LOADS = 1
 DEBUG_ROUTER_FALLBACK = 2
+DEBUG_CTA_CLOCKS = 4
+DEBUG_STATIC_ITEMS = 8
 
 # every symbol include/sa.h declares
 EXPORTS = ("sa_padded_tokens", "sa_num_cubes", "sa_topk_from_fraction", "sa_workspace_size", "sa_tile",
            "sa_untile", "sa_plan", "sa_forward", "sa_backward", "sa_get_device_status", "sa_status_string",
            "sa_last_launch_count", "sa_plan_static", "sa_plan_coarse", "sa_forward_gated", "sa_backward_gated", "sa_recall", "sa_plan_bq128",
-           "sa_plan_fallback_rows", "sa_tile_rope", "sa_untile_rope")
+           "sa_plan_fallback_rows", "sa_tile_rope", "sa_untile_rope", "sa_block_mass", "sa_best_recall",
+           "sa_plan_fine_workspace_size", "sa_plan_fine", "sa_get_cta_clocks")
 
 
 class SAError(RuntimeError):
@@ -98,6 +101,11 @@ def load_library(path: str = LIB_PATH):
         "sa_plan_fallback_rows": (i32, [vp, vp]),
         "sa_tile_rope": (i32, [vp, vp, P, i32, i32, i32, i32, vp, vp, vp]),
         "sa_untile_rope": (i32, [vp, vp, P, i32, i32, i32, i32, vp, vp, vp]),
+        "sa_block_mass": (i32, [vp, vp, vp, P, vp, vp, sz, vp]),
+        "sa_best_recall": (i32, [vp, vp, P, vp, vp]),
+        "sa_plan_fine_workspace_size": (sz, [P, i32, i32, i32]),
+        "sa_plan_fine": (i32, [vp, vp, P, i32, i32, i32, vp, vp, vp, vp, sz, vp]),
+        "sa_get_cta_clocks": (i32, [vp, sz, i32, vp, i32, ctypes.POINTER(ctypes.c_int), vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -181,6 +189,18 @@ def new_workspace(p: Params, op: int, device=None):
 def device_status(ws, stream=None) -> int:
     """Synchronise the stream and return the status recorded in the workspace (0 = SA_OK)."""
     return int(load_library().sa_get_device_status(_ptr(ws), _stream(stream)))
+
+
+def cta_clocks(ws, kernel: int, stream=None):
+    """Per-CTA records ``[n, 4]`` uint64 (start ns, end ns, items, steps) of attention kernel
+    ``kernel`` (0 forward, 1 dQ, 2 dK/dV) from the last call on workspace ``ws`` made with
+    ``DEBUG_CTA_CLOCKS``; synchronises the stream."""
+    import numpy as np
+    out = np.zeros((1024, 4), dtype=np.uint64)
+    n = ctypes.c_int(0)
+    _check(load_library().sa_get_cta_clocks(_ptr(ws), ws.numel(), int(kernel), out.ctypes.data, 1024,
+                                            ctypes.byref(n), _stream(stream)), "sa_get_cta_clocks")
+    return out[:n.value].copy()
 
 
 def plan_fallback_rows(ws, stream=None) -> int:
@@ -537,6 +557,60 @@ def recall(lse_kept, lse_all, p: Params, stream=None):
                                   _stream(stream))
     _check(st, "sa_recall")
     return tau, cube
+
+
+def plan_fine(q, k, p: Params, R=(2, 2, 2), kv_index=None, kv_count=None, with_scores: bool = False, ws=None,
+              stream=None):
+    """VSA2's fine-grained router with per-sequence Top-K (``p.top_k`` blocks per query cube on
+    average): returns (kv_index, kv_count), plus P_r ``[B,H,T,T]`` fp32 when ``with_scores``."""
+    torch = _torch()
+    T, dev = _router_args(q, k, p, None, None, kv_index, kv_count)
+    if kv_index is None:
+        kv_index = torch.empty((p.B, p.H, T, p.kv_capacity), dtype=torch.int32, device=dev)
+    if kv_count is None:
+        kv_count = torch.empty((p.B, p.H, T), dtype=torch.int32, device=dev)
+    pr = torch.empty((p.B, p.H, T, T), dtype=torch.float32, device=dev) if with_scores else None
+    lib = load_library()
+    if ws is None:
+        n = int(lib.sa_plan_fine_workspace_size(ctypes.byref(p), *R))
+        if n == 0:
+            raise SAError(2, "sa_plan_fine_workspace_size")
+        ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    _check(lib.sa_plan_fine(_ptr(q), _ptr(k), ctypes.byref(p), *R, _ptr(kv_index), _ptr(kv_count), _ptr(pr),
+                            _ptr(ws), ws.numel(), _stream(stream)), "sa_plan_fine")
+    return (kv_index, kv_count, pr) if with_scores else (kv_index, kv_count)
+
+
+def block_mass(q, k, lse_all, p: Params, ws=None, stream=None):
+    """P_oracle ``[B,H,T,T]`` fp32: the token-level softmax mass per (query cube, key cube),
+    averaged over the query cube's valid tokens (``lse_all``: lse of :func:`forward` on lists
+    holding every block)."""
+    torch = _torch()
+    npad, T = geometry(p)
+    _token_tensor(q, p, "q", 2)
+    _token_tensor(k, p, "k", 2)
+    _contig(lse_all, "lse_all", torch.float32)
+    _shape(lse_all, (p.B, p.H, npad), "lse_all")
+    out = torch.empty((p.B, p.H, T, T), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = new_workspace(p, OP_BLOCK_MASS, q.device)
+    _check(load_library().sa_block_mass(_ptr(q), _ptr(k), _ptr(lse_all), ctypes.byref(p), _ptr(out), _ptr(ws),
+                                        ws.numel(), _stream(stream)), "sa_block_mass")
+    return out
+
+
+def best_recall(pblock, kv_count, p: Params, stream=None):
+    """``[B,H,T]`` fp32: the sum of the kv_count largest entries of each row of ``pblock``."""
+    torch = _torch()
+    _, T = geometry(p)
+    _contig(pblock, "pblock", torch.float32)
+    _shape(pblock, (p.B, p.H, T, T), "pblock")
+    _contig(kv_count, "kv_count", torch.int32)
+    _shape(kv_count, (p.B, p.H, T), "kv_count")
+    out = torch.empty((p.B, p.H, T), dtype=torch.float32, device=pblock.device)
+    _check(load_library().sa_best_recall(_ptr(pblock), _ptr(kv_count), ctypes.byref(p), _ptr(out), _stream(stream)),
+           "sa_best_recall")
+    return out
 
 
 @dataclass

@@ -14,6 +14,8 @@ using sa::Geom;
 thread_local int g_last_launches = 0;
 
 constexpr size_t kHeader = 256;
+// forward / backward: per-CTA clock records of the three attention kernels after the header
+constexpr size_t kClockBytes = 3ull * sa::kClockCtas * 4 * sizeof(unsigned long long);
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -60,15 +62,17 @@ int union_cap(const sa_params* p, const Geom& g) { return 2 * p->kv_capacity < g
 struct WsLayout {
   size_t cmask = 0;                                        // forward, backward: [T] cube masks
   size_t ulist = 0, ucnt = 0;                              // forward: query-pair union lists
+  size_t v16 = 0;                                          // forward: fp16 copy of V
   size_t qbar = 0, kbar = 0, scores = 0;                   // plan
   size_t delta = 0, nlse2 = 0, bits = 0;                  // backward
   size_t ukcnt = 0, uklist = 0;                            // backward: key-pair unions
+  size_t h16[4] = {0, 0, 0, 0};                            // backward: fp16 copies of Q, K, V, dO
   size_t p32 = 0;                                          // plan + coarse: Pc [BH, T, T] fp32
   size_t doc = 0, dltc = 0, s32 = 0, ds32 = 0;             // gated backward: coarse scratch
   size_t cq = 0, ck = 0, cv = 0;
   size_t qpair = 0, blk_index = 0, blk_count = 0;          // plan with 128-token query blocks
   size_t qlimb = 0, klimb = 0, qexp = 0, kexp = 0, ql1 = 0;  // plan on the tensor cores
-  size_t kexpmax = 0, meta = 0, keys = 0, flist = 0, fbs = 0;
+  size_t kexpmax = 0, meta = 0, keys = 0, flist = 0, rkmax = 0, rkmin = 0;
   int Tk = 0;
   size_t total = 0;
 };
@@ -136,7 +140,7 @@ WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
     w.qexp = off;
     off = align256(off + rows * sizeof(int));
     w.kexp = off;
-    off = align256(off + rows * sizeof(int));
+    off = align256(off + BH * static_cast<size_t>((g.T + 3) & ~3) * sizeof(int));
     w.ql1 = off;
     off = align256(off + rows * sizeof(double));
     w.kexpmax = off;
@@ -148,8 +152,10 @@ WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
     off = align256(off + rows * static_cast<size_t>(w.Tk) * sizeof(int));
     w.flist = off;
     off = align256(off + rows * sizeof(int));
-    w.fbs = off;
-    off = align256(off + static_cast<size_t>(sa::plan_fallback_ctas()) * 4 * g.T * sizeof(double));
+    w.rkmax = off;
+    off = align256(off + rows * sizeof(int));
+    w.rkmin = off;
+    off = align256(off + rows * sizeof(int));
   } else if (op == kOpPlanFp64) {
     w.qbar = off;
     off = align256(off + BH * g.T * p->D * sizeof(double));
@@ -157,7 +163,11 @@ WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
     off = align256(off + BH * g.T * p->D * sizeof(double));
     w.scores = off;
     off = align256(off + BH * g.T * static_cast<size_t>(g.T) * sizeof(double));
+  } else if (op == SA_OP_BLOCK_MASS) {
+    w.cmask = off;
+    off = align256(off + static_cast<size_t>(g.T) * sizeof(unsigned long long));
   } else if (op == SA_OP_FORWARD) {
+    off += kClockBytes;
     w.cmask = off;
     off = align256(off + static_cast<size_t>(g.T) * sizeof(unsigned long long));
     const size_t P = static_cast<size_t>((g.T + 1) / 2);
@@ -165,7 +175,10 @@ WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
     off = align256(off + BH * P * sizeof(int32_t));
     w.ulist = off;
     off = align256(off + BH * P * static_cast<size_t>(union_cap(p, g)) * sizeof(int32_t));
+    w.v16 = off;  // fp16 copy of V for the single-product P V when the fp32 output is kept
+    off = align256(off + BH * g.Npad * static_cast<size_t>(p->D) * 2);
   } else if (op == SA_OP_BACKWARD) {
+    off += kClockBytes;
     w.cmask = off;
     off = align256(off + static_cast<size_t>(g.T) * sizeof(unsigned long long));
     w.delta = off;
@@ -183,6 +196,10 @@ WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
     off = align256(off + BH * P * sizeof(int32_t));
     w.uklist = off;
     off = align256(off + BH * P * static_cast<size_t>(g.T) * sizeof(int32_t));
+    for (int t = 0; t < 4; ++t) {  // fp16 copies for the single-product path
+      w.h16[t] = off;
+      off = align256(off + BH * g.Npad * static_cast<size_t>(p->D) * 2);
+    }
   }
   w.total = off;
   return w;
@@ -233,8 +250,27 @@ bool make_limb_map(CUtensorMap* m, const void* base, int T, long long slabs) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over the router's keys {T columns, T rows, BH heads} (int32, row stride Tk): 32 x 32
+// boxes with the 128-byte swizzle; rows and columns past T are outside the map.
+bool make_keys_map(CUtensorMap* m, void* base, int T, int Tk, int BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(Tk) * 4, static_cast<cuuint64_t>(T) * Tk * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_INT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 sa_status reset_status(void* ws, cudaStream_t s) {
   return cudaMemsetAsync(ws, 0, kHeader, s) == cudaSuccess ? SA_OK : SA_ERR_LAUNCH;
+}
+
+unsigned long long timeout_ns_of(const sa_params* p) {
+  const unsigned ms = p->timeout_ms ? p->timeout_ms : 2000u;
+  return static_cast<unsigned long long>(ms) * 1000000ull;
 }
 
 sa::AttnArgs base_args(const sa_params* p, const Geom& g, void* ws) {
@@ -252,6 +288,11 @@ sa::AttnArgs base_args(const sa_params* p, const Geom& g, void* ws) {
   a.timeout_ns = static_cast<unsigned long long>(ms) * 1000000ull;
   a.debug = p->debug_flags;
   a.st = static_cast<sa::DevStatus*>(ws);
+  a.item_next = a.st->item_next;
+  if (p->debug_flags & SA_DEBUG_CTA_CLOCKS) {  // forward and backward workspaces hold the records
+    a.cta_clock = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(ws) + kHeader);
+    a.clock_grid = a.st->grid;
+  }
   return a;
 }
 
@@ -305,14 +346,16 @@ sa_status plan_on_scratch(const void* q, const void* k, const float* q_scale, co
   f.keys = reinterpret_cast<int*>(wb + w.keys);
   f.Tk = w.Tk;
   f.flist = reinterpret_cast<int*>(wb + w.flist);
-  f.fb_scratch = reinterpret_cast<double*>(wb + w.fbs);
-  CUtensorMap tq, tk;
-  if (!make_limb_map(&tq, f.qlimb, g.T, 4LL * BH) || !make_limb_map(&tk, f.klimb, g.T, 4LL * BH))
+  f.rkmax = reinterpret_cast<int*>(wb + w.rkmax);
+  f.rkmin = reinterpret_cast<int*>(wb + w.rkmin);
+  CUtensorMap tq, tk, tkeys;
+  if (!make_limb_map(&tq, f.qlimb, g.T, 4LL * BH) || !make_limb_map(&tk, f.klimb, g.T, 4LL * BH) ||
+      !make_keys_map(&tkeys, f.keys, g.T, f.Tk, BH))
     return SA_ERR_LAUNCH;
   if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
   const unsigned ms = p->timeout_ms ? p->timeout_ms : 2000u;
   int launches = 0;
-  if (launch_plan_fast(q, k, q_scale, k_scale, tq, tk, g, BH, p->D, fp8, softmax_scale(p), p->top_k, p->top_p,
+  if (launch_plan_fast(q, k, q_scale, k_scale, tq, tk, tkeys, g, BH, p->D, fp8, softmax_scale(p), p->top_k, p->top_p,
                        p->kv_capacity, p->debug_flags, static_cast<unsigned long long>(ms) * 1000000ull, f, kv_index,
                        kv_count, static_cast<DevStatus*>(ws), st, &launches) != cudaSuccess)
     return SA_ERR_LAUNCH;
@@ -341,7 +384,7 @@ int sa_topk_from_fraction(double frac, int T) {
 
 size_t sa_workspace_size(const sa_params* p, int op) {
   Geom g;
-  if (check_params(p, &g) != SA_OK || op < SA_OP_PLAN || op > SA_OP_PLAN_BQ128) return 0;
+  if (check_params(p, &g) != SA_OK || op < SA_OP_PLAN || op > SA_OP_BLOCK_MASS) return 0;
   return ws_layout(p, g, op).total;
 }
 
@@ -405,9 +448,13 @@ sa_status sa_plan(const void* q, const void* k, const float* q_scale, const floa
                              reinterpret_cast<cudaStream_t>(stream));
 }
 
-sa_status sa_forward(const void* q, const void* k, const void* v, const float* q_scale, const float* k_scale,
-                     const int32_t* kv_index, const int32_t* kv_count, const sa_params* p, void* out, float* lse,
-                     float* out_f32, void* ws, size_t ws_bytes, sa_stream_t stream) {
+namespace {
+
+// sa_forward, and with `gate` / `oc` set sa_forward_gated (the combination in the epilogue).
+sa_status forward_impl(const void* q, const void* k, const void* v, const float* q_scale, const float* k_scale,
+                       const int32_t* kv_index, const int32_t* kv_count, const sa_params* p, void* out, float* lse,
+                       float* out_f32, const float* gate, const float* oc, void* ws, size_t ws_bytes,
+                       sa_stream_t stream) {
   Geom g;
   g_last_launches = 0;
   sa_status s = check_params(p, &g);
@@ -429,6 +476,8 @@ sa_status sa_forward(const void* q, const void* k, const void* v, const float* q
   a.out = static_cast<__nv_bfloat16*>(out);
   a.out_f32 = out_f32;
   a.lse = lse;
+  a.gate = gate;
+  a.oc = oc;
   a.qk_fp8 = fp8 ? 1 : 0;
   if (fp8) {
     a.q_scale = q_scale;
@@ -450,9 +499,30 @@ sa_status sa_forward(const void* q, const void* k, const void* v, const float* q
                                   reinterpret_cast<int32_t*>(wb + w.ucnt), a.BH, g.T, p->kv_capacity, a.st,
                                   st) != cudaSuccess)
     return SA_ERR_LAUNCH;
-  if (sa::launch_forward(tq, tk, tv, a, st) != cudaSuccess) return SA_ERR_LAUNCH;
-  g_last_launches = 3;
+  CUtensorMap tv16 = tv;
+  int extra = 0;
+  if (out_f32) {
+    // fp16 copy of V (and a range flag in the status block) for the single fp16 P V product
+    void* v16 = wb + w.v16;
+    a.f16_bad = &static_cast<sa::DevStatus*>(ws)->f16_out_of_range;
+    if (!make_map(&tv16, v16, a.rows_total, p->D, 2) ||
+        sa::launch_to_f16(v, v16, static_cast<long long>(a.rows_total) * p->D,
+                          const_cast<unsigned int*>(a.f16_bad), st) != cudaSuccess)
+      return SA_ERR_LAUNCH;
+    extra = 1;
+  }
+  if (sa::launch_forward(tq, tk, tv, tv16, a, st) != cudaSuccess) return SA_ERR_LAUNCH;
+  g_last_launches = 3 + extra;
   return SA_OK;
+}
+
+}  // namespace
+
+sa_status sa_forward(const void* q, const void* k, const void* v, const float* q_scale, const float* k_scale,
+                     const int32_t* kv_index, const int32_t* kv_count, const sa_params* p, void* out, float* lse,
+                     float* out_f32, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  return forward_impl(q, k, v, q_scale, k_scale, kv_index, kv_count, p, out, lse, out_f32, nullptr, nullptr, ws,
+                      ws_bytes, stream);
 }
 
 }  // extern "C"
@@ -515,6 +585,21 @@ sa_status backward_impl(const void* q, const void* k, const void* v, const void*
   a.cube_mask = reinterpret_cast<unsigned long long*>(wb + w.cmask);
   if (sa::launch_cube_mask(g, reinterpret_cast<unsigned long long*>(wb + w.cmask), st) != cudaSuccess)
     return SA_ERR_LAUNCH;
+  // fp16 copies of Q, K, V and dO with a range flag and max|dO|, max|V|; the decision kernel sets
+  // the status block's single-product switch that both backward kernels read
+  sa::DevStatus* dst = static_cast<sa::DevStatus*>(ws);
+  CUtensorMap t16[4];
+  const void* src16[4] = {q, k, v, dout};
+  unsigned int* maxbits[4] = {nullptr, nullptr, &dst->f16_max[1], &dst->f16_max[0]};
+  for (int t = 0; t < 4; ++t) {
+    void* h = wb + w.h16[t];
+    if (!make_map(&t16[t], h, a.rows_total, p->D, 2) ||
+        sa::launch_to_f16(src16[t], h, static_cast<long long>(a.rows_total) * p->D, &dst->f16_out_of_range, st,
+                          maxbits[t]) != cudaSuccess)
+      return SA_ERR_LAUNCH;
+  }
+  if (sa::launch_f16_decide(dst, p->D, st) != cudaSuccess) return SA_ERR_LAUNCH;
+  a.f16_single = &dst->f16_single;
   float* delta = reinterpret_cast<float*>(wb + w.delta);
   float* nlse2 = reinterpret_cast<float*>(wb + w.nlse2);
   int coarse_launches = 0;
@@ -525,18 +610,18 @@ sa_status backward_impl(const void* q, const void* k, const void* v, const void*
                               reinterpret_cast<float*>(wb + w.cq),   reinterpret_cast<float*>(wb + w.ck),
                               reinterpret_cast<float*>(wb + w.cv)};
     if (sa::launch_coarse_backward(out, out_f32, dout, lse, gate, coarse_tensors(coarse), dgate, delta, nlse2, cw,
-                                   a.scale, g, a.BH, p->D, st, &coarse_launches) != cudaSuccess)
+                                   a.scale, g, a.BH, p->D, a.st, a.timeout_ns, st, &coarse_launches) != cudaSuccess)
       return SA_ERR_LAUNCH;
     add = sa::CoarseAdd{cw.cq, cw.ck, cw.cv};
   }
   int launches = 0;
   a.ucap = union_cap(p, g);
-  if (sa::launch_backward(tq, tk, tv, tdo, out, out_f32, dout, a, reinterpret_cast<uint32_t*>(wb + w.bits), delta,
+  if (sa::launch_backward(tq, tk, tv, tdo, t16, out, out_f32, dout, a, reinterpret_cast<uint32_t*>(wb + w.bits), delta,
                           nlse2, reinterpret_cast<int32_t*>(wb + w.ulist), reinterpret_cast<int32_t*>(wb + w.ucnt),
                           reinterpret_cast<int32_t*>(wb + w.uklist), reinterpret_cast<int32_t*>(wb + w.ukcnt), add,
                           gated, st, &launches) != cudaSuccess)
     return SA_ERR_LAUNCH;
-  g_last_launches = 1 + coarse_launches + launches;
+  g_last_launches = 6 + coarse_launches + launches;
   return SA_OK;
 }
 
@@ -578,7 +663,8 @@ sa_status sa_plan_coarse(const void* q, const void* k, const void* v, const sa_p
                       p->kv_capacity, kv_index, kv_count, qbar, kbar, S, static_cast<sa::DevStatus*>(ws), st,
                       &plan_launches) != cudaSuccess ||
       sa::launch_coarse_forward(v, qbar, kbar, S, reinterpret_cast<float*>(wb + w.p32), coarse_tensors(coarse), g, BH,
-                                p->D, st, &coarse_launches) != cudaSuccess)
+                                p->D, static_cast<sa::DevStatus*>(ws), timeout_ns_of(p), st,
+                                &coarse_launches) != cudaSuccess)
     return SA_ERR_LAUNCH;
   g_last_launches = plan_launches + coarse_launches;
   return SA_OK;
@@ -597,14 +683,9 @@ sa_status sa_forward_gated(const void* q, const void* k, const void* v, const in
   if (!gate || !out_f32) return SA_ERR_INVALID_ARG;
   if ((s = check_coarse(coarse)) != SA_OK) return s;
   if (!aligned4(gate)) return SA_ERR_ALIGNMENT;
-  s = sa_forward(q, k, v, nullptr, nullptr, kv_index, kv_count, p, out, lse, out_f32, ws, ws_bytes, stream);
-  if (s != SA_OK) return s;
-  const int fine_launches = g_last_launches;
-  if (sa::launch_coarse_combine(out, out_f32, gate, coarse->oc, g, p->B * p->H, p->D,
-                                reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return SA_ERR_LAUNCH;
-  g_last_launches = fine_launches + 1;
-  return SA_OK;
+  // the forward kernel forms O = G Oc^ + O_f in its epilogue (fp32, then the bf16 copy)
+  return forward_impl(q, k, v, nullptr, nullptr, kv_index, kv_count, p, out, lse, out_f32, gate, coarse->oc, ws,
+                      ws_bytes, stream);
 }
 
 sa_status sa_backward_gated(const void* q, const void* k, const void* v, const void* out, const float* out_f32,
@@ -661,6 +742,156 @@ sa_status sa_recall(const float* lse_kept, const float* lse_all, const sa_params
   return SA_OK;
 }
 
+sa_status sa_block_mass(const void* q, const void* k, const float* lse_all, const sa_params* p, float* pblock,
+                        void* ws, size_t ws_bytes, sa_stream_t stream) {
+  Geom g;
+  g_last_launches = 0;
+  sa_status s = check_params(p, &g);
+  if (s != SA_OK) return s;
+  if (!q || !k || !lse_all || !pblock) return SA_ERR_INVALID_ARG;
+  if (p->qk_dtype != SA_BF16) return SA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(p->B) * p->H * g.T * g.T >= (1LL << 40)) return SA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned4(lse_all) || !aligned4(pblock)) return SA_ERR_ALIGNMENT;
+  const WsLayout w = ws_layout(p, g, SA_OP_BLOCK_MASS);
+  if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SA_ERR_ALIGNMENT;
+  const int BH = p->B * p->H;
+  CUtensorMap tq, tk;
+  if (!make_map(&tq, q, static_cast<long long>(BH) * g.Npad, p->D, 2) ||
+      !make_map(&tk, k, static_cast<long long>(BH) * g.Npad, p->D, 2))
+    return SA_ERR_LAUNCH;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  auto* cmask = reinterpret_cast<unsigned long long*>(wb + w.cmask);
+  const unsigned ms = p->timeout_ms ? p->timeout_ms : 2000u;
+  const double sc = softmax_scale(p);
+  if (sa::launch_cube_mask(g, cmask, st) != cudaSuccess ||
+      sa::launch_block_mass(tq, tk, lse_all, cmask, pblock, g, BH, p->D, static_cast<float>(sc * 1.4426950408889634),
+                            static_cast<sa::DevStatus*>(ws), static_cast<unsigned long long>(ms) * 1000000ull,
+                            st) != cudaSuccess)
+    return SA_ERR_LAUNCH;
+  g_last_launches = 2;
+  return SA_OK;
+}
+
+sa_status sa_best_recall(const float* pblock, const int32_t* kv_count, const sa_params* p, float* best,
+                         sa_stream_t stream) {
+  Geom g;
+  g_last_launches = 0;
+  sa_status s = check_params(p, &g);
+  if (s != SA_OK) return s;
+  if (!pblock || !kv_count || !best) return SA_ERR_INVALID_ARG;
+  if (!aligned4(pblock) || !aligned4(kv_count) || !aligned4(best)) return SA_ERR_ALIGNMENT;
+  if (sa::launch_best_recall(pblock, kv_count, best, p->B * p->H * g.T, g.T, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return SA_ERR_LAUNCH;
+  g_last_launches = 1;
+  return SA_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+struct FineLayout {
+  size_t qlimb, klimb, qexp, qvalid, ql1, kexp, kvalid, kexpmax, lse2, pr, total;
+  int TG, TGp;
+};
+
+bool fine_shape_ok(int rt, int rh, int rw) {
+  auto ok = [](int r) { return r == 1 || r == 2 || r == 4; };
+  if (!ok(rt) || !ok(rh) || !ok(rw)) return false;
+  const int G = 64 / (rt * rh * rw);
+  return G == 4 || G == 8 || G == 16;
+}
+
+FineLayout fine_layout(const sa_params* p, const Geom& g, int rt, int rh, int rw) {
+  FineLayout w;
+  const size_t BH = static_cast<size_t>(p->B) * p->H;
+  const int G = 64 / (rt * rh * rw);
+  w.TG = g.T * G;
+  w.TGp = (w.TG + 3) & ~3;
+  const size_t TG = static_cast<size_t>(w.TG), TGp = static_cast<size_t>(w.TGp);
+  size_t off = kHeader;
+  w.qlimb = off;
+  off = align256(off + BH * 4 * TG * 128);
+  w.klimb = off;
+  off = align256(off + BH * 4 * TG * 128);
+  w.qexp = off;
+  off = align256(off + BH * TG * sizeof(int));
+  w.qvalid = off;
+  off = align256(off + BH * TG * sizeof(int));
+  w.ql1 = off;
+  off = align256(off + BH * TG * sizeof(double));
+  w.kexp = off;
+  off = align256(off + BH * TGp * sizeof(int));
+  w.kvalid = off;
+  off = align256(off + BH * TGp * sizeof(int));
+  w.kexpmax = off;
+  off = align256(off + BH * sizeof(unsigned));
+  w.lse2 = off;
+  off = align256(off + BH * TG * sizeof(float));
+  w.pr = off;
+  off = align256(off + BH * g.T * static_cast<size_t>(g.T) * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sa_plan_fine_workspace_size(const sa_params* p, int rt, int rh, int rw) {
+  Geom g;
+  if (check_params(p, &g) != SA_OK || !fine_shape_ok(rt, rh, rw)) return 0;
+  return fine_layout(p, g, rt, rh, rw).total;
+}
+
+sa_status sa_plan_fine(const void* q, const void* k, const sa_params* p, int rt, int rh, int rw, int32_t* kv_index,
+                       int32_t* kv_count, float* p_r, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  Geom g;
+  g_last_launches = 0;
+  sa_status s = check_params(p, &g);
+  if (s != SA_OK) return s;
+  if (!q || !k || !kv_index || !kv_count) return SA_ERR_INVALID_ARG;
+  if (!fine_shape_ok(rt, rh, rw)) return SA_ERR_UNSUPPORTED;
+  if (p->qk_dtype != SA_BF16) return SA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned4(kv_index) || !aligned4(kv_count) || (p_r && !aligned4(p_r)))
+    return SA_ERR_ALIGNMENT;
+  const FineLayout w = fine_layout(p, g, rt, rh, rw);
+  if (static_cast<long long>(p->B) * p->H * 4 * w.TG >= (1LL << 31)) return SA_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SA_ERR_ALIGNMENT;
+  const int BH = p->B * p->H;
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  sa::FineWs f;
+  f.qlimb = reinterpret_cast<int8_t*>(wb + w.qlimb);
+  f.klimb = reinterpret_cast<int8_t*>(wb + w.klimb);
+  f.qexp = reinterpret_cast<int*>(wb + w.qexp);
+  f.qvalid = reinterpret_cast<int*>(wb + w.qvalid);
+  f.ql1 = reinterpret_cast<double*>(wb + w.ql1);
+  f.kexp = reinterpret_cast<int*>(wb + w.kexp);
+  f.kvalid = reinterpret_cast<int*>(wb + w.kvalid);
+  f.kexp_max = reinterpret_cast<unsigned*>(wb + w.kexpmax);
+  f.lse2 = reinterpret_cast<float*>(wb + w.lse2);
+  f.pr = p_r ? p_r : reinterpret_cast<float*>(wb + w.pr);
+  f.TGp = w.TGp;
+  CUtensorMap tq, tk;
+  if (!make_limb_map(&tq, f.qlimb, w.TG, 4LL * BH) || !make_limb_map(&tk, f.klimb, w.TG, 4LL * BH))
+    return SA_ERR_LAUNCH;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
+  const unsigned ms = p->timeout_ms ? p->timeout_ms : 2000u;
+  int launches = 0;
+  if (sa::launch_plan_fine(q, k, tq, tk, g, BH, p->D, rt, rh, rw, softmax_scale(p), p->top_k, p->kv_capacity, f,
+                           kv_index, kv_count, static_cast<sa::DevStatus*>(ws),
+                           static_cast<unsigned long long>(ms) * 1000000ull, st, &launches) != cudaSuccess)
+    return SA_ERR_LAUNCH;
+  g_last_launches = launches;
+  return SA_OK;
+}
+
 sa_status sa_get_device_status(const void* ws, sa_stream_t stream) {
   if (!ws) return SA_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SA_ERR_LAUNCH;
@@ -678,6 +909,28 @@ int sa_plan_fallback_rows(const void* ws, sa_stream_t stream) {
   sa::DevStatus h;
   if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return -1;
   return static_cast<int>(h.router_fallback);
+}
+
+sa_status sa_get_cta_clocks(const void* ws, size_t ws_bytes, int kernel, unsigned long long* out, int max_ctas,
+                            int* n_ctas, sa_stream_t stream) {
+  if (!ws || !out || !n_ctas || kernel < 0 || kernel > 2 || max_ctas < 0 || ws_bytes < kHeader + kClockBytes)
+    return SA_ERR_INVALID_ARG;
+  *n_ctas = 0;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SA_ERR_LAUNCH;
+  sa::DevStatus h;
+  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return SA_ERR_LAUNCH;
+  int n = static_cast<int>(h.grid[kernel]);
+  n = n < max_ctas ? n : max_ctas;
+  n = n < sa::kClockCtas ? n : sa::kClockCtas;
+  if (n > 0) {
+    const uint8_t* src = static_cast<const uint8_t*>(ws) + kHeader +
+                         static_cast<size_t>(kernel) * sa::kClockCtas * 4 * sizeof(unsigned long long);
+    if (cudaMemcpy(out, src, static_cast<size_t>(n) * 4 * sizeof(unsigned long long), cudaMemcpyDeviceToHost) !=
+        cudaSuccess)
+      return SA_ERR_LAUNCH;
+  }
+  *n_ctas = n;
+  return SA_OK;
 }
 
 const char* sa_status_string(sa_status s) {

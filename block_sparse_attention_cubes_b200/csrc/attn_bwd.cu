@@ -15,6 +15,7 @@
 // All products are full-rate 128 x 128 tcgen05 MMAs with accumulators in TMEM; P and dS
 // enter the dV, dK and dQ products as bf16 hi + lo pairs read from TMEM.
 #include <cmath>
+#include <type_traits>
 
 #include "attn_common.cuh"
 #include "kernels.h"
@@ -101,11 +102,12 @@ constexpr uint32_t OFF_V = OFF_K + KST * 32768;
 constexpr uint32_t OFF_BAR = OFF_V + VST * 32768;
 constexpr uint32_t OFF_SLOT = OFF_BAR + 256;
 constexpr uint32_t OFF_ABORT = OFF_BAR + 264;
+constexpr uint32_t OFF_RING = OFF_BAR + 272;  // kItemRing item ids
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;
 constexpr uint32_t TMEM_COLS = 512;  // S/dS[b] at 128b, dP at 256, dQ at 384
 enum {
   B_QF = 0, B_QE = 1, B_KF = 2, B_KE = 5, B_VF = 8, B_VE = 10, B_SF = 12, B_DPF = 14, B_PF = 15, B_DQR = 16,
-  B_DQFREE = 17, B_FIN = 18, NBAR = 19
+  B_DQFREE = 17, B_FIN = 18, B_IF = 19, B_IE = 23, NBAR = 27
 };
 }  // namespace dqk
 
@@ -113,6 +115,7 @@ template <int KS>  // D / 16; MMA loops unrolled (a counted loop costs more than
 __global__ void __launch_bounds__(dqk::kThreads, 1)
     attn_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                   const __grid_constant__ CUtensorMap tm_q16, const __grid_constant__ CUtensorMap tm_k16,
                    const AttnArgs a, const CoarseAdd add) {
   using namespace dqk;
   extern __shared__ uint8_t smem_raw[];
@@ -128,7 +131,8 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
   const int n_items = a.BH * npairs;
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < NBAR; ++b) mbar_init(&bars[b], b == B_PF ? 256u : (b == B_DQFREE ? 8u : 1u));
+    for (int b = 0; b < NBAR; ++b)
+      mbar_init(&bars[b], b == B_PF ? 256u : (b == B_DQFREE ? 8u : ((b >= B_IE && b < B_IE + kItemRing) ? kRingReaders : 1u)));
     *sm_abort = aborted(a.st) ? 1 : 0;
     fence_barrier_init();
   }
@@ -141,15 +145,26 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const bool skip_all = *sm_abort != 0;
+  const ItemRing ring{reinterpret_cast<volatile int*>(smem + OFF_RING), &bars[B_IF], &bars[B_IE]};
+  const unsigned long long t_start = (threadIdx.x == 0 && a.cta_clock) ? globaltimer_ns() : 0ull;
+  int rec_items = 0;
+  uint32_t rec_steps = 0;
+  // fp16 single products (Q and K from their fp16 copies, dS as one fp16 value) when the
+  // conversion pass found every operand and the dS bound within fp16; else bf16, dS as hi + lo
+  const bool use16 = a.f16_single != nullptr && *reinterpret_cast<const volatile unsigned*>(a.f16_single) == 1u;
+  const CUtensorMap* mq = use16 ? &tm_q16 : &tm_q;
 
   if (warp == 0) {
     if (lane < 2 && !skip_all) {
-      const bool kq = lane == 0;  // lane 0: Q2, dO2 and K tiles; lane 1: V tiles
-      const CUtensorMap* tmap = kq ? &tm_k : &tm_v;
+      const bool kq = lane == 0;  // lane 0: item ids, Q2, dO2 and K tiles; lane 1: V tiles
+      const CUtensorMap* tmap = kq ? (use16 ? &tm_k16 : &tm_k) : &tm_v;
       uint32_t gs = 0;
       int issued_q = 0;
       bool ok = true;
-      for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+      int n = 0;
+      for (; ok; ++n) {
+        const int it = kq ? ring_publish(ring, n, n_items, a, a.item_next + 1, 45, ok) : ring_read(ring, n, a, 46, ok);
+        if (it < 0) break;
         const int bh = it / npairs, pr = it % npairs;
         const int nu = a.u_cnt[it];
         const int32_t* ul = a.u_list + static_cast<size_t>(it) * a.ucap;
@@ -158,10 +173,10 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
           const int r0 = bh * g.Npad + (2 * pr) * 64;
           const int r1 = (2 * pr + 1 < g.T) ? r0 + 64 : a.rows_total;
           mbar_arrive_expect_tx(&bars[B_QF], 65536);
-          tma_load_2d(smem + OFF_Q, &tm_q, &bars[B_QF], 0, r0);
-          tma_load_2d(smem + OFF_Q + 8192, &tm_q, &bars[B_QF], 0, r1);
-          tma_load_2d(smem + OFF_Q + 16384, &tm_q, &bars[B_QF], 64, r0);
-          tma_load_2d(smem + OFF_Q + 24576, &tm_q, &bars[B_QF], 64, r1);
+          tma_load_2d(smem + OFF_Q, mq, &bars[B_QF], 0, r0);
+          tma_load_2d(smem + OFF_Q + 8192, mq, &bars[B_QF], 0, r1);
+          tma_load_2d(smem + OFF_Q + 16384, mq, &bars[B_QF], 64, r0);
+          tma_load_2d(smem + OFF_Q + 24576, mq, &bars[B_QF], 64, r1);
           tma_load_2d(smem + OFF_DO, &tm_do, &bars[B_QF], 0, r0);
           tma_load_2d(smem + OFF_DO + 8192, &tm_do, &bars[B_QF], 0, r1);
           tma_load_2d(smem + OFF_DO + 16384, &tm_do, &bars[B_QF], 64, r0);
@@ -191,6 +206,10 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
           ++gs;
         }
       }
+      if (kq) {
+        rec_items = n;
+        rec_steps = gs;
+      }
       if (kq && issued_q > 0) mbar_wait_drain(&bars[B_QF], (issued_q - 1) & 1, a.st, a.timeout_ns, 43);
       const uint32_t nst = kq ? KST : VST;
       for (uint32_t s = (gs > nst ? gs - nst : 0); s < gs; ++s)
@@ -199,8 +218,9 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
   } else if (warp == 1) {
     // the whole warp runs the loop; one elected lane issues (see elect_one)
     if (!skip_all) {
-      const uint32_t idesc_kk = make_idesc(128, 128, FMT_BF16, false, false);
-      const uint32_t idesc_q = make_idesc(128, 128, FMT_BF16, false, true);
+      const uint32_t idesc_kk = make_idesc(128, 128, FMT_BF16, false, false);  // dP: bf16 dO, V
+      const uint32_t idesc_s = make_idesc(128, 128, use16 ? FMT_F16 : FMT_BF16, false, false);
+      const uint32_t idesc_q = make_idesc(128, 128, use16 ? FMT_F16 : FMT_BF16, false, true);
       uint32_t gs_s = 0, gs_p = 0, gs_q = 0;  // global steps whose S, dP, dQ products were issued
       bool ok = true;
       auto issue_s = [&]() -> bool {
@@ -213,7 +233,7 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
           for (int ks = 0; ks < KS; ++ks) {
             const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
             umma_f16_ss(tmem + sb * 128, sw128_desc(sbase + OFF_Q + off, 16, 1024), sw128_desc(kst + off, 16, 1024),
-                        idesc_kk, ks > 0 ? 1u : 0u);
+                        idesc_s, ks > 0 ? 1u : 0u);
           }
           umma_commit(&bars[B_SF + sb]);
         }
@@ -240,7 +260,9 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         ++gs_p;
         return true;
       };
-      for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+      for (int n = 0; ok; ++n) {
+        const int it = ring_read_warp(ring, n, a, 57, ok);
+        if (it < 0) break;
         const int nsteps = (a.u_cnt[it] + 1) >> 1;
         if (!mbar_wait_warp(&bars[B_QF], n & 1, a.st, a.timeout_ns, 53)) break;
         if (nsteps > 0) ok = issue_s() && issue_dp();
@@ -263,12 +285,21 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
           const uint32_t ks_i = gs_q % KST, sb = gs_q & 1;
           const uint32_t kst = sbase + OFF_K + ks_i * 32768;
           if (elect_one()) {
+            if (use16) {
 #pragma unroll
-            for (int ks = 0; ks < 16; ++ks) {  // 8 k-steps over dS_hi, then 8 over dS_lo
-              const uint32_t kk = ks & 7, part = ks >> 3;
-              const uint32_t acol = sb * 128 + (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
-              umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(kst + kk * 2048, 16384, 1024), idesc_q,
-                          (s > 0 || ks > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 8; ++kk) {  // 8 k-steps over dS (fp16)
+                const uint32_t acol = sb * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
+                umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(kst + kk * 2048, 16384, 1024), idesc_q,
+                            (s > 0 || kk > 0) ? 1u : 0u);
+              }
+            } else {
+#pragma unroll
+              for (int ks = 0; ks < 16; ++ks) {  // 8 k-steps over dS_hi, then 8 over dS_lo
+                const uint32_t kk = ks & 7, part = ks >> 3;
+                const uint32_t acol = sb * 128 + (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
+                umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(kst + kk * 2048, 16384, 1024), idesc_q,
+                            (s > 0 || ks > 0) ? 1u : 0u);
+              }
             }
             umma_commit(&bars[B_KE + ks_i]);  // K(s) was read by S(s) and dQ(s)
           }
@@ -294,7 +325,9 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     uint32_t gs = 0;
     bool ok = !skip_all;
-    for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+    for (int n = 0; ok; ++n) {
+      const int it = ring_read_group(ring, n, a, 64, sm_abort, ok);
+      if (it < 0) break;
       const int bh = it / npairs, pr = it % npairs;
       const int icube = 2 * pr + half;
       const bool row_exists = icube < g.T;
@@ -316,41 +349,56 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         const bool ok2 = mbar_wait(&bars[B_DPF], gs & 1, a.st, a.timeout_ns, 62);
         if (!(ok1 && ok2)) *sm_abort = 1;
         tc_fence_after();
-        uint32_t hi[32], lo[32];
-        if (w_active) {
-          uint32_t s0[32], s1[32], p0[32], p1[32];
-          tmem_ld32(t_lane + b * 128 + grp * 64, s0);
-          tmem_ld32(t_lane + b * 128 + grp * 64 + 32, s1);
-          tmem_ld32(t_lane + 256 + grp * 64, p0);
-          tmem_ld32(t_lane + 256 + grp * 64 + 32, p1);
-          tmem_ld_wait();
-          // the key mask is first used here, so its load (issued a step earlier) hides behind the waits
-          const unsigned long long km = active ? km_cur : 0ull;
-          const uint64_t sc2 = pk2(a.scale_log2, a.scale_log2), nl2 = pk2(-lse2, -lse2), dl2 = pk2(dlt, dlt);
-          const bool full = km == ~0ull;  // uniform over the warp
+        // one body per precision (each with its own registers): dS as fp16, or bf16 hi + lo
+        auto emit_ds = [&](auto f16_tag) {
+          constexpr bool F16 = decltype(f16_tag)::value;
+          uint32_t hi[32], lo[F16 ? 1 : 32];
+          if (w_active) {
+            uint32_t s0[32], s1[32], p0[32], p1[32];
+            tmem_ld32(t_lane + b * 128 + grp * 64, s0);
+            tmem_ld32(t_lane + b * 128 + grp * 64 + 32, s1);
+            tmem_ld32(t_lane + 256 + grp * 64, p0);
+            tmem_ld32(t_lane + 256 + grp * 64 + 32, p1);
+            tmem_ld_wait();
+            // the key mask is first used here, so its load (issued a step earlier) hides behind the waits
+            const unsigned long long km = active ? km_cur : 0ull;
+            const uint64_t sc2 = pk2(a.scale_log2, a.scale_log2), nl2 = pk2(-lse2, -lse2), dl2 = pk2(dlt, dlt);
+            const bool full = km == ~0ull;  // uniform over the warp
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int c0 = 2 * c, c1 = 2 * c + 1;
-            const uint32_t sa0 = c0 < 32 ? s0[c0] : s1[c0 - 32], sa1 = c1 < 32 ? s0[c1] : s1[c1 - 32];
-            const uint32_t pa0 = c0 < 32 ? p0[c0] : p1[c0 - 32], pa1 = c1 < 32 ? p0[c1] : p1[c1 - 32];
-            float x0, x1;
-            upk2(fma2(pk2(__uint_as_float(sa0), __uint_as_float(sa1)), sc2, nl2), x0, x1);
-            float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
-            if (!full) {
-              if (!((km >> c0) & 1ull)) e0 = 0.0f;
-              if (!((km >> c1) & 1ull)) e1 = 0.0f;
+            for (int c = 0; c < 32; ++c) {
+              const int c0 = 2 * c, c1 = 2 * c + 1;
+              const uint32_t sa0 = c0 < 32 ? s0[c0] : s1[c0 - 32], sa1 = c1 < 32 ? s0[c1] : s1[c1 - 32];
+              const uint32_t pa0 = c0 < 32 ? p0[c0] : p1[c0 - 32], pa1 = c1 < 32 ? p0[c1] : p1[c1 - 32];
+              float x0, x1;
+              upk2(fma2(pk2(__uint_as_float(sa0), __uint_as_float(sa1)), sc2, nl2), x0, x1);
+              float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+              if (!full) {
+                if (!((km >> c0) & 1ull)) e0 = 0.0f;
+                if (!((km >> c1) & 1ull)) e1 = 0.0f;
+              }
+              float d0, d1;
+              upk2(mul2(pk2(e0, e1), sub2(pk2(__uint_as_float(pa0), __uint_as_float(pa1)), dl2)), d0, d1);
+              if constexpr (F16)
+                hi[c] = pack_f16x2(d0, d1);
+              else
+                split_bf16x2(d0, d1, hi[c], lo[c]);
             }
-            float d0, d1;
-            upk2(mul2(pk2(e0, e1), sub2(pk2(__uint_as_float(pa0), __uint_as_float(pa1)), dl2)), d0, d1);
-            split_bf16x2(d0, d1, hi[c], lo[c]);
-          }
-        } else {
+          } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) hi[c] = lo[c] = 0u;
-        }
-        // dS over this group's own S columns: hi at +0, lo at +32
-        tmem_st32(t_lane + b * 128 + grp * 64, hi);
-        tmem_st32(t_lane + b * 128 + grp * 64 + 32, lo);
+            for (int c = 0; c < 32; ++c) hi[c] = 0u;
+            if constexpr (!F16) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) lo[c] = 0u;
+            }
+          }
+          // dS over this group's own S columns: hi at +0, lo at +32
+          tmem_st32(t_lane + b * 128 + grp * 64, hi);
+          if constexpr (!F16) tmem_st32(t_lane + b * 128 + grp * 64 + 32, lo);
+        };
+        if (use16)
+          emit_ds(std::true_type{});
+        else
+          emit_ds(std::false_type{});
         e = e_next;
         km_cur = a.cube_mask[e >> 2];
         tmem_st_wait();
@@ -403,6 +451,7 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+  if (threadIdx.x == 0) cta_clock_record(a, 1, t_start, rec_items, rec_steps);
 }
 
 // ------------------------------------------------------------------------ dK, dV
@@ -424,11 +473,12 @@ constexpr uint32_t OFF_DLT = OFF_LSE + QST * 512;   // QST x [128] float
 constexpr uint32_t OFF_BAR = OFF_DLT + QST * 512;
 constexpr uint32_t OFF_SLOT = OFF_BAR + 256;
 constexpr uint32_t OFF_ABORT = OFF_BAR + 264;
+constexpr uint32_t OFF_RING = OFF_BAR + 272;  // kItemRing item ids
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;
 constexpr uint32_t TMEM_COLS = 512;  // S^T/P^T at 0, dP^T/dS^T at 128, dV at 256, dK at 384
 enum {
   B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DF = 6, B_DE = 8, B_SF = 10, B_DPF = 11, B_PF = 12, B_DSF = 13,
-  B_DVR = 14, B_DVFREE = 15, B_FIN = 16, NBAR = 17
+  B_DVR = 14, B_DVFREE = 15, B_FIN = 16, B_IF = 17, B_IE = 21, NBAR = 25
 };
 }  // namespace dkv
 
@@ -436,6 +486,8 @@ template <int KS>  // D / 16; MMA loops unrolled (a counted loop costs more than
 __global__ void __launch_bounds__(dkv::kThreads, 1)
     attn_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ CUtensorMap tm_q16, const __grid_constant__ CUtensorMap tm_k16,
+                     const __grid_constant__ CUtensorMap tm_v16, const __grid_constant__ CUtensorMap tm_do16,
                      const AttnArgs a, const CoarseAdd add) {
   using namespace dkv;
   extern __shared__ uint8_t smem_raw[];
@@ -454,7 +506,9 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < NBAR; ++b)
-      mbar_init(&bars[b], (b == B_PF || b == B_DSF) ? 256u : (b == B_DVFREE ? 8u : 1u));
+      mbar_init(&bars[b], (b == B_PF || b == B_DSF)
+                              ? 256u
+                              : (b == B_DVFREE ? 8u : ((b >= B_IE && b < B_IE + kItemRing) ? kRingReaders : 1u)));
     *sm_abort = aborted(a.st) ? 1 : 0;
     fence_barrier_init();
   }
@@ -467,16 +521,29 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const bool skip_all = *sm_abort != 0;
+  const ItemRing ring{reinterpret_cast<volatile int*>(smem + OFF_RING), &bars[B_IF], &bars[B_IE]};
+  const unsigned long long t_start = (threadIdx.x == 0 && a.cta_clock) ? globaltimer_ns() : 0ull;
+  int rec_items = 0;
+  uint32_t rec_steps = 0;
+  // fp16 single products (every operand from its fp16 copy, P^T and dS^T as one fp16 value) when
+  // the conversion pass found every operand and the dS bound within fp16; else bf16 with P^T and
+  // dS^T as hi + lo
+  const bool use16 = a.f16_single != nullptr && *reinterpret_cast<const volatile unsigned*>(a.f16_single) == 1u;
+  const CUtensorMap* mk = use16 ? &tm_k16 : &tm_k;
+  const CUtensorMap* mv = use16 ? &tm_v16 : &tm_v;
 
   if (warp == 0) {
     if (lane < 2 && !skip_all) {
-      const bool qside = lane == 0;  // lane 0: K2, V2, Q2 + lse; lane 1: dO2 + Delta
-      const CUtensorMap* tmap = qside ? &tm_q : &tm_do;
+      const bool qside = lane == 0;  // lane 0: item ids, K2, V2, Q2 + lse; lane 1: dO2 + Delta
+      const CUtensorMap* tmap = qside ? (use16 ? &tm_q16 : &tm_q) : (use16 ? &tm_do16 : &tm_do);
       const float* vec = qside ? a.nlse2 : a.delta;
       uint32_t gs = 0;
       int issued_kv = 0;
       bool ok = true;
-      for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+      int n = 0;
+      for (; ok; ++n) {
+        const int it = qside ? ring_publish(ring, n, n_items, a, a.item_next + 2, 75, ok) : ring_read(ring, n, a, 76, ok);
+        if (it < 0) break;
         const int bh = it / npairs, pr = it % npairs;
         const int nu = a.uk_cnt[it];
         const int32_t* ul = a.uk_list + static_cast<size_t>(it) * g.T;
@@ -485,14 +552,14 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
           const int r0 = bh * g.Npad + (2 * pr) * 64;
           const int r1 = (2 * pr + 1 < g.T) ? r0 + 64 : a.rows_total;
           mbar_arrive_expect_tx(&bars[B_KVF], 65536);
-          tma_load_2d(smem + OFF_K, &tm_k, &bars[B_KVF], 0, r0);
-          tma_load_2d(smem + OFF_K + 8192, &tm_k, &bars[B_KVF], 0, r1);
-          tma_load_2d(smem + OFF_K + 16384, &tm_k, &bars[B_KVF], 64, r0);
-          tma_load_2d(smem + OFF_K + 24576, &tm_k, &bars[B_KVF], 64, r1);
-          tma_load_2d(smem + OFF_V, &tm_v, &bars[B_KVF], 0, r0);
-          tma_load_2d(smem + OFF_V + 8192, &tm_v, &bars[B_KVF], 0, r1);
-          tma_load_2d(smem + OFF_V + 16384, &tm_v, &bars[B_KVF], 64, r0);
-          tma_load_2d(smem + OFF_V + 24576, &tm_v, &bars[B_KVF], 64, r1);
+          tma_load_2d(smem + OFF_K, mk, &bars[B_KVF], 0, r0);
+          tma_load_2d(smem + OFF_K + 8192, mk, &bars[B_KVF], 0, r1);
+          tma_load_2d(smem + OFF_K + 16384, mk, &bars[B_KVF], 64, r0);
+          tma_load_2d(smem + OFF_K + 24576, mk, &bars[B_KVF], 64, r1);
+          tma_load_2d(smem + OFF_V, mv, &bars[B_KVF], 0, r0);
+          tma_load_2d(smem + OFF_V + 8192, mv, &bars[B_KVF], 0, r1);
+          tma_load_2d(smem + OFF_V + 16384, mv, &bars[B_KVF], 64, r0);
+          tma_load_2d(smem + OFF_V + 24576, mv, &bars[B_KVF], 64, r1);
           ++issued_kv;
         }
         const int nsteps = (nu + 1) >> 1;
@@ -519,6 +586,10 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
           ++gs;
         }
       }
+      if (qside) {
+        rec_items = n;
+        rec_steps = gs;
+      }
       if (qside && issued_kv > 0) mbar_wait_drain(&bars[B_KVF], (issued_kv - 1) & 1, a.st, a.timeout_ns, 73);
       for (uint32_t s = (gs > QST ? gs - QST : 0); s < gs; ++s)
         mbar_wait_drain(&bars[(qside ? B_QF : B_DF) + s % QST], (s / QST) & 1, a.st, a.timeout_ns, 74);
@@ -526,11 +597,13 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
   } else if (warp == 1) {
     // the whole warp runs the loop; one elected lane issues (see elect_one)
     if (!skip_all) {
-      const uint32_t idesc_kk = make_idesc(128, 128, FMT_BF16, false, false);
-      const uint32_t idesc_mn = make_idesc(128, 128, FMT_BF16, false, true);
+      const uint32_t idesc_kk = make_idesc(128, 128, use16 ? FMT_F16 : FMT_BF16, false, false);
+      const uint32_t idesc_mn = make_idesc(128, 128, use16 ? FMT_F16 : FMT_BF16, false, true);
       uint32_t gs = 0;
       bool ok = true;
-      for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+      for (int n = 0; ok; ++n) {
+        const int it = ring_read_warp(ring, n, a, 89, ok);
+        if (it < 0) break;
         const int nsteps = (a.uk_cnt[it] + 1) >> 1;
         if (!mbar_wait_warp(&bars[B_KVF], n & 1, a.st, a.timeout_ns, 81)) break;
         // one phase of DVR / DVFREE per item, empty items included (see the dQ kernel)
@@ -569,12 +642,21 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
           }
           tc_fence_after();
           if (elect_one()) {
+            if (use16) {
 #pragma unroll
-            for (int ks = 0; ks < 16; ++ks) {  // dV += P^T dO2 (hi then lo), overlapping dS^T
-              const uint32_t kk = ks & 7, part = ks >> 3;
-              const uint32_t acol = (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
-              umma_f16_ts(tmem + 256, tmem + acol, sw128_desc(dst + kk * 2048, 16384, 1024), idesc_mn,
-                          (s > 0 || ks > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO2 (fp16), overlapping dS^T
+                const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
+                umma_f16_ts(tmem + 256, tmem + acol, sw128_desc(dst + kk * 2048, 16384, 1024), idesc_mn,
+                            (s > 0 || kk > 0) ? 1u : 0u);
+              }
+            } else {
+#pragma unroll
+              for (int ks = 0; ks < 16; ++ks) {  // dV += P^T dO2 (hi then lo), overlapping dS^T
+                const uint32_t kk = ks & 7, part = ks >> 3;
+                const uint32_t acol = (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
+                umma_f16_ts(tmem + 256, tmem + acol, sw128_desc(dst + kk * 2048, 16384, 1024), idesc_mn,
+                            (s > 0 || ks > 0) ? 1u : 0u);
+              }
             }
           }
           __syncwarp();
@@ -588,12 +670,21 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
           }
           tc_fence_after();
           if (elect_one()) {
+            if (use16) {
 #pragma unroll
-            for (int ks = 0; ks < 16; ++ks) {  // dK += dS^T Q2 (hi then lo)
-              const uint32_t kk = ks & 7, part = ks >> 3;
-              const uint32_t acol = 128 + (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
-              umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(qst + kk * 2048, 16384, 1024), idesc_mn,
-                          (s > 0 || ks > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 8; ++kk) {  // dK += dS^T Q2 (fp16)
+                const uint32_t acol = 128 + (kk >> 2) * 64 + (kk & 3) * 8;
+                umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(qst + kk * 2048, 16384, 1024), idesc_mn,
+                            (s > 0 || kk > 0) ? 1u : 0u);
+              }
+            } else {
+#pragma unroll
+              for (int ks = 0; ks < 16; ++ks) {  // dK += dS^T Q2 (hi then lo)
+                const uint32_t kk = ks & 7, part = ks >> 3;
+                const uint32_t acol = 128 + (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
+                umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(qst + kk * 2048, 16384, 1024), idesc_mn,
+                            (s > 0 || ks > 0) ? 1u : 0u);
+              }
             }
             // the Q and dO stages (with their lse and Delta, read by the softmax before DSF) are free
             umma_commit(&bars[B_QE + st]);
@@ -624,7 +715,9 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     uint32_t gs = 0;
     bool ok = !skip_all;
-    for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+    for (int n = 0; ok; ++n) {
+      const int it = ring_read_group(ring, n, a, 94, sm_abort, ok);
+      if (it < 0) break;
       const int bh = it / npairs, pr = it % npairs;
       const int kcube = 2 * pr + khalf;
       const bool key_exists = kcube < g.T;
@@ -644,7 +737,6 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
         // P^T = exp(S^T * scale - lse_q): written as soon as it is known so that dV can start
         float pe[64];
         {
-          uint32_t ph[32], pl[32];
           if (w_active) {
             uint32_t s0[32], s1[32];
             tmem_ld32(t_lane + grp * 64, s0);
@@ -666,21 +758,28 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
                 if (!full && !((qm >> c) & 1ull)) pe[c] = 0.0f;
               }
             }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) pe[c] = 0.0f;
+          }
+          // P^T over S^T (every S^T read of this thread's own columns is done): one fp16 value,
+          // or bf16 hi + lo
+          if (use16) {
+            uint32_t ph[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ph[c] = pack_f16x2(pe[2 * c], pe[2 * c + 1]);
+            tmem_st32(t_lane + grp * 64, ph);
+          } else {
+            uint32_t ph[32], pl[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
               ph[c] = pack_bf16x2(pe[2 * c], pe[2 * c + 1]);
               pl[c] = pack_bf16x2(pe[2 * c] - __uint_as_float(ph[c] << 16),
                                   pe[2 * c + 1] - __uint_as_float(ph[c] & 0xffff0000u));
             }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 64; ++c) pe[c] = 0.0f;
-#pragma unroll
-            for (int c = 0; c < 32; ++c) ph[c] = pl[c] = 0u;
+            tmem_st32(t_lane + grp * 64, ph);
+            tmem_st32(t_lane + grp * 64 + 32, pl);
           }
-          // P^T over S^T: every S^T read of this thread's own columns is done
-          tmem_st32(t_lane + grp * 64, ph);
-          tmem_st32(t_lane + grp * 64 + 32, pl);
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(&bars[B_PF]);
@@ -689,14 +788,13 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
         if (!mbar_wait(&bars[B_DPF], gs & 1, a.st, a.timeout_ns, 93)) *sm_abort = 1;
         tc_fence_after();
         {
-          uint32_t dh[32], dl[32];
+          // pe becomes dS^T in place (P^T is no longer needed once packed)
           if (w_active) {
             uint32_t p0[32], p1[32];
             tmem_ld32(t_lane + 128 + grp * 64, p0);
             tmem_ld32(t_lane + 128 + grp * 64 + 32, p1);
             tmem_ld_wait();
             const float* dq_ = dlt_sh + st * 128 + grp * 64;
-            float dsv[64];
 #pragma unroll
             for (int c4 = 0; c4 < 16; ++c4) {
               const float4 d4 = *reinterpret_cast<const float4*>(dq_ + 4 * c4);
@@ -705,21 +803,26 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
               for (int u = 0; u < 4; ++u) {
                 const int c = 4 * c4 + u;
                 const uint32_t pv = c < 32 ? p0[c] : p1[c - 32];
-                dsv[c] = pe[c] * (__uint_as_float(pv) - dv4[u]);
+                pe[c] = pe[c] * (__uint_as_float(pv) - dv4[u]);
               }
             }
+          }
+          if (use16) {
+            uint32_t dh[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) dh[c] = pack_f16x2(pe[2 * c], pe[2 * c + 1]);
+            tmem_st32(t_lane + 128 + grp * 64, dh);
+          } else {
+            uint32_t dh[32], dl[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              dh[c] = pack_bf16x2(dsv[2 * c], dsv[2 * c + 1]);
-              dl[c] = pack_bf16x2(dsv[2 * c] - __uint_as_float(dh[c] << 16),
-                                  dsv[2 * c + 1] - __uint_as_float(dh[c] & 0xffff0000u));
+              dh[c] = pack_bf16x2(pe[2 * c], pe[2 * c + 1]);
+              dl[c] = pack_bf16x2(pe[2 * c] - __uint_as_float(dh[c] << 16),
+                                  pe[2 * c + 1] - __uint_as_float(dh[c] & 0xffff0000u));
             }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) dh[c] = dl[c] = 0u;
+            tmem_st32(t_lane + 128 + grp * 64, dh);
+            tmem_st32(t_lane + 128 + grp * 64 + 32, dl);
           }
-          tmem_st32(t_lane + 128 + grp * 64, dh);
-          tmem_st32(t_lane + 128 + grp * 64 + 32, dl);
           e = e_next;
           qm_cur = a.cube_mask[e >> 2];
           tmem_st_wait();
@@ -781,11 +884,13 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+  if (threadIdx.x == 0) cta_clock_record(a, 2, t_start, rec_items, rec_steps);
 }
 
 // ------------------------------------------------------------------------ launch
 cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const void* out, const float* out_f32, const void* dout,
+                            const CUtensorMap& tdo, const CUtensorMap (&t16)[4], const void* out, const float* out_f32,
+                            const void* dout,
                             AttnArgs a, uint32_t* bits, float* delta, float* nlse2,
                             int32_t* uq_list,
                             int32_t* uq_cnt, int32_t* uk_list, int32_t* uk_cnt, const CoarseAdd& add,
@@ -820,11 +925,13 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   const int items = a.BH * ((g.T + 1) >> 1);
   const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
   if (a.D == 64) {
-    attn_dq_kernel<4><<<grid, dqk::kThreads, dqk::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a, add);
-    attn_dkdv_kernel<4><<<grid, dkv::kThreads, dkv::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a, add);
+    attn_dq_kernel<4><<<grid, dqk::kThreads, dqk::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, t16[0], t16[1], a, add);
+    attn_dkdv_kernel<4><<<grid, dkv::kThreads, dkv::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, t16[0], t16[1], t16[2],
+                                                                         t16[3], a, add);
   } else {
-    attn_dq_kernel<8><<<grid, dqk::kThreads, dqk::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a, add);
-    attn_dkdv_kernel<8><<<grid, dkv::kThreads, dkv::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a, add);
+    attn_dq_kernel<8><<<grid, dqk::kThreads, dqk::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, t16[0], t16[1], a, add);
+    attn_dkdv_kernel<8><<<grid, dkv::kThreads, dkv::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, t16[0], t16[1], t16[2],
+                                                                         t16[3], a, add);
   }
   *launches = delta_ready ? 5 : 6;
   return cudaGetLastError();

@@ -14,6 +14,10 @@ struct AttnArgs {
   const float* k_scale;
   __nv_bfloat16* out;       // forward output [BH, Npad, D]
   float* out_f32;           // optional fp32 copy of the forward output
+  const unsigned int* f16_bad;  // forward with out_f32: nonzero when V did not fit fp16 (then P as bf16 hi + lo)
+  const unsigned int* f16_single;  // backward: 1 when Q, K, V, dO and dS fit fp16 (single fp16 products)
+  const float* gate;        // gated forward: G per token [BH, Npad] and the coarse output Oc^ [BH, T, D]
+  const float* oc;          //   (O = G Oc^[cube] + O_f on the valid rows, formed in the epilogue)
   const unsigned long long* cube_mask;  // [T] valid-slot mask of every cube
   const int32_t* u_list;    // query-pair unions: [BH, ceil(T/2), ucap] (block << 2 | membership bits)
   const int32_t* u_cnt;     // [BH, ceil(T/2)]
@@ -35,7 +39,102 @@ struct AttnArgs {
   float scale_log2;         // softmax scale * log2(e)
   unsigned long long timeout_ns;
   unsigned int debug;
+  unsigned int* item_next;        // work-item counters [3] (forward, dQ, dK/dV), zeroed before the launch
+  unsigned long long* cta_clock;  // optional per-CTA records [3][kClockCtas][4]: start, end (ns), items, steps
+  unsigned int* clock_grid;       // with cta_clock: [3] grid sizes
 };
+constexpr int kClockCtas = 1024;  // per-CTA clock records kept per kernel
+
+// ------------------------------------------------------------------ dynamic item order
+// Work items (pairs of cubes) go, in their natural order, to whichever CTA is free: CTA c
+// starts with item c and takes each later one from a per-launch counter.  Neighbouring items
+// belong to the same head and share most of their K/V tiles, so the CTAs at work at any
+// moment keep reading the same lines of L2, and no CTA is left with a longer static share.
+// One thread (the first producer lane) fetches every id into a small shared ring; each of
+// the kernel's other roles reads the same sequence from it and signals the slot free.
+constexpr int kItemRing = 4;
+constexpr unsigned int kDebugStaticItems = 8u;  // debug flag: item n of CTA c is c + n * gridDim.x
+constexpr uint32_t kRingReaders = 10;  // the second producer lane, the MMA warp, eight epilogue warps
+struct ItemRing {
+  volatile int* ids;  // [kItemRing]; -1 once no item is left
+  uint64_t* full;     // [kItemRing], one arrival (the fetching thread)
+  uint64_t* empty;    // [kItemRing], kRingReaders arrivals
+};
+
+// The fetching thread: item n of this CTA, published in slot n % kItemRing.
+__device__ __forceinline__ int ring_publish(const ItemRing& r, int n, int n_items, const AttnArgs& a,
+                                            unsigned int* counter, unsigned int where, bool& ok) {
+  const int slot = n % kItemRing;
+  if (n >= kItemRing && !mbar_wait(&r.empty[slot], ((n / kItemRing) + 1) & 1, a.st, a.timeout_ns, where)) {
+    ok = false;
+    return -1;
+  }
+  int it;
+  if (a.debug & kDebugStaticItems)  // measurement hook: the fixed round-robin share instead
+    it = static_cast<int>(blockIdx.x) + n * static_cast<int>(gridDim.x);
+  else
+    it = n == 0 ? static_cast<int>(blockIdx.x) : static_cast<int>(gridDim.x + atomicAdd(counter, 1u));
+  if (it >= n_items) it = -1;
+  r.ids[slot] = it;
+  mbar_arrive(&r.full[slot]);
+  return it;
+}
+
+// One reading thread (a producer lane).
+__device__ __forceinline__ int ring_read(const ItemRing& r, int n, const AttnArgs& a, unsigned int where, bool& ok) {
+  const int slot = n % kItemRing;
+  if (!mbar_wait(&r.full[slot], (n / kItemRing) & 1, a.st, a.timeout_ns, where)) {
+    ok = false;
+    return -1;
+  }
+  const int it = r.ids[slot];
+  mbar_arrive(&r.empty[slot]);
+  return it;
+}
+
+// A whole converged warp (the MMA warp): one arrival.
+__device__ __forceinline__ int ring_read_warp(const ItemRing& r, int n, const AttnArgs& a, unsigned int where,
+                                              bool& ok) {
+  const int slot = n % kItemRing;
+  if (!mbar_wait_warp(&r.full[slot], (n / kItemRing) & 1, a.st, a.timeout_ns, where)) {
+    ok = false;
+    return -1;
+  }
+  const int it = r.ids[slot];
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&r.empty[slot]);
+  return it;
+}
+
+// The 256 epilogue threads (named barrier 1): they agree on success through the shared abort
+// flag behind the barrier, so they leave their loops together; one arrival per warp.
+__device__ __forceinline__ int ring_read_group(const ItemRing& r, int n, const AttnArgs& a, unsigned int where,
+                                               volatile int* sm_abort, bool& ok) {
+  const int slot = n % kItemRing;
+  if (!mbar_wait(&r.full[slot], (n / kItemRing) & 1, a.st, a.timeout_ns, where)) *sm_abort = 1;
+  named_bar_sync(1, 256);
+  if (*sm_abort) {
+    ok = false;
+    return -1;
+  }
+  const int it = r.ids[slot];
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&r.empty[slot]);
+  return it;
+}
+
+// Per-CTA clock record of kernel `kid` (thread 0, when records were asked for): start and end
+// in globaltimer nanoseconds, the items and steps this CTA processed.
+__device__ __forceinline__ void cta_clock_record(const AttnArgs& a, int kid, unsigned long long t0, int items,
+                                                 uint32_t steps) {
+  if (a.cta_clock == nullptr || blockIdx.x >= static_cast<unsigned>(kClockCtas)) return;
+  if (blockIdx.x == 0) a.clock_grid[kid] = gridDim.x;
+  unsigned long long* c = a.cta_clock + 4ull * (static_cast<unsigned long long>(kid) * kClockCtas + blockIdx.x);
+  c[0] = t0;
+  c[1] = globaltimer_ns();
+  c[2] = static_cast<unsigned long long>(items);
+  c[3] = steps;
+}
 
 // bf16 pair of (v0, v1) into hi, and with the remainders (v - bf16(v)) as a second bf16 pair
 // into lo: hi + lo carries v to about 16 bits.

@@ -21,7 +21,8 @@
 //   warps 2-9   two groups of 128 threads; thread r of group g owns query row r and the 64
 //               key columns of tile t_g.  The two halves' row maxima are exchanged once per
 //               step through shared memory; the running maximum is raised (and that row of O
-//               rescaled in TMEM) only when a score exceeds it by more than 2^16.
+//               rescaled in TMEM) only when a score exceeds it by more than 2^15.
+#include <type_traits>
 #include <cmath>
 
 #include "attn_common.cuh"
@@ -31,7 +32,7 @@ namespace sa {
 
 namespace fwd {
 constexpr int kThreads = 320;
-constexpr float kTau = 16.0f;      // log2 headroom before a running maximum is raised
+constexpr float kTau = 15.0f;      // log2 headroom before a running maximum is raised (P <= 2^15: fp16 holds it)
 constexpr float kNegBig = -1e30f;  // finite "minus infinity" for running maxima
 constexpr int KST = 3, VST = 2;    // K and V ring depths
 constexpr uint32_t OFF_Q = 0;                    // Q2: [2 halves][128 rows][128 B]
@@ -40,6 +41,7 @@ constexpr uint32_t OFF_V = OFF_K + KST * 32768;  // VST x same
 constexpr uint32_t OFF_BAR = OFF_V + VST * 32768;
 constexpr uint32_t OFF_SLOT = OFF_BAR + 256;
 constexpr uint32_t OFF_ABORT = OFF_BAR + 264;
+constexpr uint32_t OFF_RING = OFF_BAR + 272;     // kItemRing item ids
 constexpr uint32_t OFF_XMAX = OFF_BAR + 512;     // [2 step parities][2 groups][128 rows] float
 constexpr uint32_t OFF_XL = OFF_XMAX + 2048;     // [2 groups][128 rows] float
 constexpr uint32_t SMEM_BYTES = OFF_XL + 1024 + 1024;
@@ -49,7 +51,7 @@ constexpr uint32_t TMEM_COLS = 512;  // S/P[b] at 128b (b = 0,1), O[ob] at 256 +
 // phases unobserved.  The softmax of step s+2 needs S(s+2), issued only after PV(s).
 enum {
   B_QF = 0, B_QE = 1, B_KF = 2, B_KE = 5, B_VF = 8, B_VE = 10, B_SF = 12, B_PF = 14, B_PFREE = 16, B_OR = 17,
-  B_OFREE = 19, B_FIN = 21, NBAR = 22
+  B_OFREE = 19, B_FIN = 21, B_IF = 22, B_IE = 26, NBAR = 30
 };
 }  // namespace fwd
 
@@ -62,7 +64,8 @@ enum {
 template <int KS, bool FP8>
 __global__ void __launch_bounds__(fwd::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_v16,
+                    const AttnArgs a) {
   using namespace fwd;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -84,6 +87,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       uint32_t cnt = 1;
       if (b == B_PF || b == B_PF + 1) cnt = 256;
       if (b == B_OFREE || b == B_OFREE + 1) cnt = 8;
+      if (b >= B_IE && b < B_IE + kItemRing) cnt = kRingReaders;
       mbar_init(&bars[b], cnt);
     }
     *sm_abort = aborted(a.st) ? 1 : 0;
@@ -103,19 +107,30 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const bool skip_all = *sm_abort != 0;
-  // When the caller keeps the fp32 output (for the backward's Delta), P enters the PV
-  // product as bf16 hi + lo so that O is exact to ~2^-16 instead of bf16's 2^-9.
-  const bool split_pv = a.out_f32 != nullptr;
+  const ItemRing ring{reinterpret_cast<volatile int*>(smem + OFF_RING), &bars[B_IF], &bars[B_IE]};
+  const unsigned long long t_start = (threadIdx.x == 0 && a.cta_clock) ? globaltimer_ns() : 0ull;
+  int rec_items = 0;
+  uint32_t rec_steps = 0;
+  // With the fp32 output kept (for the backward's Delta), P must enter P V to ~2^-11 or better: as one fp16 product against
+  // the fp16 copy of V when V fits fp16 (a flag the conversion pass left in device memory, the
+  // same for every thread of the launch), else as bf16 hi + lo against V.
+  const bool keep32 = a.out_f32 != nullptr;
+  const bool use16 = keep32 && a.f16_bad != nullptr && *reinterpret_cast<const volatile unsigned*>(a.f16_bad) == 0u;
+  const bool split_pv = keep32 && !use16;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producers
-    if (lane < 2 && !skip_all && !(a.debug & 1u)) {
-      const bool kq = lane == 0;  // lane 0: Q2 and K tiles; lane 1: V tiles
-      const CUtensorMap* tmap = kq ? &tm_k : &tm_v;
+    if (lane < 2 && !skip_all) {
+      const bool kq = lane == 0;  // lane 0: item ids, Q2 and K tiles; lane 1: V (or its fp16 copy) tiles
+      const CUtensorMap* tmap = kq ? &tm_k : (use16 ? &tm_v16 : &tm_v);
       uint32_t gs = 0;
       int issued_q = 0;
       bool ok = true;
-      for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+      int n = 0;
+      for (; ok; ++n) {
+        const int it = kq ? ring_publish(ring, n, n_items, a, a.item_next + 0, 15, ok) : ring_read(ring, n, a, 16, ok);
+        if (it < 0) break;
+        if (a.debug & 1u) break;  // SA_DEBUG_SKIP_LOADS: the item is published, nothing is loaded
         const int bh = it / npairs, pr = it % npairs;
         const int nu = a.u_cnt[it];
         const int32_t* ul = a.u_list + static_cast<size_t>(it) * ucap;
@@ -158,6 +173,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           ++gs;
         }
       }
+      if (kq) {
+        rec_items = n;
+        rec_steps = gs;
+      }
       // drain: never leave the CTA with copies in flight
       if (kq && issued_q > 0) mbar_wait_drain(&bars[B_QF], (issued_q - 1) & 1, a.st, a.timeout_ns, 13);
       const uint32_t nst = kq ? KST : VST;
@@ -169,7 +188,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     if (!skip_all) {
       const uint32_t idesc_s = make_idesc(128, 128, FMT_BF16, false, false);
       const uint32_t idesc_s8 = make_idesc(128, 128, FMT_E4M3, false, false);
-      const uint32_t idesc_o = make_idesc(128, 128, FMT_BF16, false, true);
+      const uint32_t idesc_o = make_idesc(128, 128, use16 ? FMT_F16 : FMT_BF16, false, true);
       uint32_t gs_s = 0, gs_o = 0;
       bool ok = true;
       // S for the next global step into S buffer gs_s & 1.  That buffer last held P of step
@@ -201,7 +220,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         ++gs_s;
         return true;
       };
-      for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+      for (int n = 0; ok; ++n) {
+        const int it = ring_read_warp(ring, n, a, 27, ok);
+        if (it < 0) break;
         const int nsteps = (a.u_cnt[it] + 1) >> 1;
         const int ob = n & 1;
         if (!mbar_wait_warp(&bars[B_QF], n & 1, a.st, a.timeout_ns, 22)) break;
@@ -252,7 +273,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     uint32_t gs = 0;
     bool ok = !skip_all;
-    for (int it = blockIdx.x, n = 0; ok && it < n_items; it += gridDim.x, ++n) {
+    for (int n = 0; ok; ++n) {
+      const int it = ring_read_group(ring, n, a, 34, sm_abort, ok);
+      if (it < 0) break;
       const int bh = it / npairs, pr = it % npairs;
       const int icube = 2 * pr + half;
       const bool row_exists = icube < g.T;
@@ -334,31 +357,52 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           tmem_st32(oc + 32, o1);
           tmem_st_wait();
         }
-        uint32_t ph[32], pl[32];
-        if (active) {
-          const uint64_t sc2 = pk2(sc, sc), nm2 = pk2(-m_run, -m_run);
-          uint64_t l2 = pk2(0.0f, 0.0f);
+        // one body per P format, each with its own registers: 0 = bf16, 1 = bf16 hi + lo (the fp32
+        // output's P V), 2 = fp16
+        auto emit_p = [&](auto mode_tag) {
+          constexpr int M = decltype(mode_tag)::value;
+          uint32_t ph[32], pl[M == 1 ? 32 : 1];
+          if (active) {
+            const uint64_t sc2 = pk2(sc, sc), nm2 = pk2(-m_run, -m_run);
+            uint64_t l2 = pk2(0.0f, 0.0f);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float d0, d1;
-            upk2(fma2(pk2(x[2 * c], x[2 * c + 1]), sc2, nm2), d0, d1);
-            const float p0 = ex2_approx(d0), p1 = ex2_approx(d1);
-            const uint64_t pp = pk2(p0, p1);
-            l2 = add2(l2, pp);
-            ph[c] = pack_bf16x2(p0, p1);
-            float r0, r1;
-            upk2(sub2(pp, pk2(__uint_as_float(ph[c] << 16), __uint_as_float(ph[c] & 0xffff0000u))), r0, r1);
-            pl[c] = pack_bf16x2(r0, r1);
+            for (int c = 0; c < 32; ++c) {
+              float d0, d1;
+              upk2(fma2(pk2(x[2 * c], x[2 * c + 1]), sc2, nm2), d0, d1);
+              const float p0 = ex2_approx(d0), p1 = ex2_approx(d1);
+              const uint64_t pp = pk2(p0, p1);
+              l2 = add2(l2, pp);
+              if constexpr (M == 2) {
+                ph[c] = pack_f16x2(p0, p1);
+              } else {
+                ph[c] = pack_bf16x2(p0, p1);
+                if constexpr (M == 1) {
+                  float r0, r1;
+                  upk2(sub2(pp, pk2(__uint_as_float(ph[c] << 16), __uint_as_float(ph[c] & 0xffff0000u))), r0, r1);
+                  pl[c] = pack_bf16x2(r0, r1);
+                }
+              }
+            }
+            float la, lb;
+            upk2(l2, la, lb);
+            l_part += la + lb;
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ph[c] = 0u;
+            if constexpr (M == 1) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) pl[c] = 0u;
+            }
           }
-          float la, lb;
-          upk2(l2, la, lb);
-          l_part += la + lb;
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) ph[c] = pl[c] = 0u;
-        }
-        tmem_st32(t_lane + b * 128 + grp * 32, ph);
-        if (split_pv) tmem_st32(t_lane + b * 128 + 64 + grp * 32, pl);
+          tmem_st32(t_lane + b * 128 + grp * 32, ph);
+          if constexpr (M == 1) tmem_st32(t_lane + b * 128 + 64 + grp * 32, pl);
+        };
+        if (use16)
+          emit_p(std::integral_constant<int, 2>{});
+        else if (split_pv)
+          emit_p(std::integral_constant<int, 1>{});
+        else
+          emit_p(std::integral_constant<int, 0>{});
         e = e_next;
         km = a.cube_mask[e >> 2];
         tmem_st_wait();
@@ -397,6 +441,19 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_OFREE + ob]);
       if (row_exists && grp * 64 < a.D) {
+        if (a.gate && row_valid) {  // the gated combination, with the coarse branch's row of this cube
+          const float gv = a.gate[qrow];
+          const float4* ocp =
+              reinterpret_cast<const float4*>(a.oc + (static_cast<size_t>(bh) * g.T + icube) * a.D + grp * 64);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float4 t = __ldg(ocp + c);
+            o[4 * c] = fmaf(gv, t.x, o[4 * c]);
+            o[4 * c + 1] = fmaf(gv, t.y, o[4 * c + 1]);
+            o[4 * c + 2] = fmaf(gv, t.z, o[4 * c + 2]);
+            o[4 * c + 3] = fmaf(gv, t.w, o[4 * c + 3]);
+          }
+        }
         uint4* dst = reinterpret_cast<uint4*>(a.out + qrow * a.D + grp * 64);
 #pragma unroll
         for (int c = 0; c < 8; ++c)
@@ -413,6 +470,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+  if (threadIdx.x == 0) cta_clock_record(a, 0, t_start, rec_items, rec_steps);
 }
 
 // 64-bit mask of the valid token slots of every cube (bit s = slot s holds a real token).
@@ -443,8 +501,59 @@ int num_sms() {
   return n;
 }
 
-cudaError_t launch_forward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
-                           cudaStream_t stream) {
+// bf16 -> fp16 copy of a tensor (n16 = elements / 8, one 16-byte vector per thread); any value
+// an fp16 cannot hold (|x| > 65504, or not finite) sets *bad.  Values below fp16's normal range
+// become fp16 subnormals (absolute error at most 2^-25).
+// With maxbits set, the largest |x| (fp32 bits, a non-negative float orders as its bits) is
+// also recorded there.
+__global__ void __launch_bounds__(256) to_f16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                     long long n16, unsigned int* bad, unsigned int* maxbits) {
+  const long long i = blockIdx.x * 256LL + threadIdx.x;
+  bool out = false;
+  float mx = 0.0f;
+  if (i < n16) {
+    const uint4 v = src[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float a = __uint_as_float(w[u] << 16), b = __uint_as_float(w[u] & 0xffff0000u);
+      out |= !(fabsf(a) <= 65504.0f) || !(fabsf(b) <= 65504.0f);
+      mx = fmaxf(mx, fmaxf(fabsf(a), fabsf(b)));
+      o[u] = pack_f16x2(a, b);
+    }
+    dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (__any_sync(0xffffffffu, out) && (threadIdx.x & 31) == 0) atomicOr(bad, 1u);
+  if (maxbits) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) atomicMax(maxbits, __float_as_uint(mx));
+  }
+}
+
+cudaError_t launch_to_f16(const void* src, void* dst, long long elems, unsigned int* bad, cudaStream_t stream,
+                          unsigned int* maxbits) {
+  const long long n16 = elems / 8;
+  to_f16_kernel<<<static_cast<unsigned>((n16 + 255) / 256), 256, 0, stream>>>(
+      static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16, bad, maxbits);
+  return cudaGetLastError();
+}
+
+// The backward's single-product decision: every converted tensor fit fp16, and the bound
+// |dS| <= |dP| + |Delta| <= 2 D max|dO| max|V| leaves fp16 (and the forward's P) headroom.
+__global__ void f16_decide_kernel(DevStatus* st, int D) {
+  const float mdo = __uint_as_float(st->f16_max[0]), mv = __uint_as_float(st->f16_max[1]);
+  st->f16_single = (st->f16_out_of_range == 0u && 2.0f * static_cast<float>(D) * mdo * mv <= 32768.0f) ? 1u : 0u;
+}
+
+cudaError_t launch_f16_decide(DevStatus* st, int D, cudaStream_t stream) {
+  f16_decide_kernel<<<1, 1, 0, stream>>>(st, D);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_forward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const CUtensorMap& tv16, const AttnArgs& a, cudaStream_t stream) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaSuccess;
@@ -458,7 +567,7 @@ cudaError_t launch_forward(const CUtensorMap& tq, const CUtensorMap& tk, const C
   const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
   // e4m3 Q/K is built for D = 128 only (the host rejects other head sizes)
   auto fn = a.qk_fp8 ? attn_fwd_kernel<8, true> : (a.D == 64 ? attn_fwd_kernel<4, false> : attn_fwd_kernel<8, false>);
-  fn<<<grid, fwd::kThreads, fwd::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  fn<<<grid, fwd::kThreads, fwd::SMEM_BYTES, stream>>>(tq, tk, tv, tv16, a);
   return cudaGetLastError();
 }
 

@@ -9,22 +9,24 @@
 //
 //   coarse_pool_kernel      Vc (fp32 mean of the valid tokens) and fp32 copies of Qc, Kc
 //   coarse_softmax_kernel   Pc rows (fp32) and lse_c from the fp64 scores
-//   coarse_gemm_kernel      batched fp32 products of the cube-level matrices, with the
-//                           epilogues the branch needs (plain, dS = P (dP - delta), and
-//                           the mean-pool adjoint 1/n per cube)
-//   coarse_combine_kernel   O = G * Oc^[cube] + O_f on the valid rows, in place
+//   coarse_mma_kernel       batched products of the cube-level matrices on the tensor cores
+//                           (fp32 operands split into bf16 hi + lo), with the epilogues the
+//                           branch needs (plain, dS = P (dP - delta), and the mean-pool
+//                           adjoint 1/n per cube)
 //   coarse_gate_bwd_kernel  one pass over dO: dG, the fine branch's Delta and -lse*log2(e),
 //                           dOc^ = sum_t G_t dO_t and delta_c = <dOc^, Oc^> per cube
 //
 // The cube-level matrices are T x T per head (T = 1440 at the 720p shape), so the six products
-// of a forward and backward are about 1/250 of the fine stage's FLOPs at 95% sparsity; they run
-// on the fp32 FMA pipe, which keeps the branch within fp32 rounding of the fp64 definition.
+// of a forward and backward are about 1/250 of the fine stage's FLOPs at 95% sparsity.  They
+// run on the tensor cores with every fp32 operand split into a bf16 pair (three products per
+// tile: about 2^-16 relative per term, fp32 accumulation).
 #include <cuda_bf16.h>
 
 #include <cmath>
 
 #include "geometry.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace sa {
 namespace {
@@ -134,8 +136,7 @@ __global__ void __launch_bounds__(256) coarse_softmax_kernel(const double* __res
 }
 
 // ------------------------------------------------------------------------ products
-// C[b] (M x N) = alpha * op(A[b]) op(B[b]), fp32, 64 x 64 tiles, 16-deep k slices, 4 x 4
-// outputs per thread, the next slice loaded into registers while the current one is used.
+// C[b] (M x N) = alpha * op(A[b]) op(B[b]), fp32 in and out, with
 // op(A)(m, k) = TA ? A[k * lda + m] : A[m * lda + k];  op(B)(k, n) = TB ? B[n * ldb + k] : B[k * ldb + n].
 enum : int { EPI_STORE = 0, EPI_DS = 1, EPI_UNPOOL = 2 };
 struct GemmArgs {
@@ -151,152 +152,255 @@ struct GemmArgs {
   const float* row_dlt;  // EPI_DS: delta_c per row
   long long sRow;
   Geom g;                // EPI_UNPOOL: row m is cube m, divided by its valid-token count
+  DevStatus* st;         // bounded waits of the tensor-core kernel report here
+  unsigned long long timeout_ns;
 };
 
-constexpr int GBM = 64, GBN = 64, GBK = 16, GPAD = 4;
+// ------------------------------------------------------------------------ products on the tensor cores
+// The same products on tcgen05: each fp32 operand value x enters as the bf16 pair
+// hi = bf16(x), lo = bf16(x - hi) (x to about 2^-16 relative), and a product accumulates
+// hi*hi + hi*lo + lo*hi in fp32 in tensor memory (the dropped lo*lo term is below 2^-16 of
+// |a||b|).  One CTA per 128 x 128 output tile: eight warps load 64-deep k slices of both
+// operands from global memory (fp32, coalesced), split them and store them in the 128-byte
+// swizzled layouts the MMA reads (K-major when k is the contiguous index of the source,
+// MN-major when m or n is), two slices in flight; warp 8 owns tensor memory and issues the
+// MMAs; the same eight warps run the epilogue from tensor memory.
+namespace cmm {
+constexpr int kThreads = 288;
+constexpr int BK = 64;                       // k slice
+constexpr uint32_t OP_BYTES = 16384;         // one operand part: 128 x 64 bf16
+constexpr uint32_t STAGE_BYTES = 4 * OP_BYTES;  // A hi, A lo, B hi, B lo
+constexpr uint32_t OFF_BAR = 2 * STAGE_BYTES;
+constexpr uint32_t OFF_SLOT = OFF_BAR + 64;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 128 + 1024;
+enum { B_FULL = 0, B_EMPTY = 2, B_DONE = 4, NBAR = 5 };
+}  // namespace cmm
 
+// bf16 hi and lo of 8 consecutive values as two 16-byte chunks
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    h[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+    l[i] = pack_bf16x2(x[2 * i] - __uint_as_float(h[i] << 16), x[2 * i + 1] - __uint_as_float(h[i] & 0xffff0000u));
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// 8 consecutive fp32 values of a source row from column c0 (zeros past `ncols`); vec: rows
+// 16-byte aligned, so whole float4 loads are legal where they are in range.
+__device__ __forceinline__ void load8(const float* row, int c0, int ncols, bool vec, float (&x)[8]) {
+  if (vec && c0 + 8 <= ncols) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(row + c0));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(row + c0 + 4));
+    x[0] = a.x, x[1] = a.y, x[2] = a.z, x[3] = a.w, x[4] = b.x, x[5] = b.y, x[6] = b.z, x[7] = b.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = c0 + i < ncols ? __ldg(row + c0 + i) : 0.0f;
+  }
+}
+
+// One operand slice (128 rows of the MMA's M or N by 64 k) into shared memory as hi and lo.
+// KMAJ: the source holds row r's k values contiguously (src[r * ld + k]); the slice is
+// stored K-major ([128 rows][128 B]).  Otherwise the source holds k row by k row
+// (src[k * ld + r]) and the slice is stored MN-major ([2 halves of 64 r][64 k][128 B]).
+template <bool KMAJ>
+__device__ __forceinline__ void load_slice(const float* src, int ld, int r0, int rows, int k0, int K, bool vec,
+                                           uint32_t s_hi, uint32_t s_lo, int tid) {
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {  // 256 threads x 4 chunks of 8 values = 128 x 64
+    const int u = tid + 256 * it;
+    float x[8];
+    uint32_t off;
+    if (KMAJ) {
+      const int r = u >> 3, c = u & 7;  // row r, k chunk c
+      const int gr = r0 + r;
+      if (gr < rows) {
+        load8(src + static_cast<long long>(gr) * ld, k0 + 8 * c, K, vec, x);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = 0.0f;
+      }
+      off = sw128_offset(r, c);
+    } else {
+      const int k = u >> 4, c = u & 15;  // k row k, r chunk c (8 values)
+      const int gk = k0 + k;
+      if (gk < K) {
+        load8(src + static_cast<long long>(gk) * ld, r0 + 8 * c, rows, vec, x);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = 0.0f;
+      }
+      off = (c >> 3) * 8192u + sw128_offset(k, c & 7);
+    }
+    uint4 h, l;
+    split8(x, h, l);
+    st_shared_v4(s_hi + off, h.x, h.y, h.z, h.w);
+    st_shared_v4(s_lo + off, l.x, l.y, l.z, l.w);
+  }
+}
+
+// C[b] = alpha * op(A[b]) op(B[b]) with the epilogues of the fp32 kernel; TA / TB as there
+// (TA: A is stored k-major by row, i.e. the MMA reads it MN-major).
 template <bool TA, bool TB, int EPI>
-__global__ void __launch_bounds__(256) coarse_gemm_kernel(GemmArgs p) {
-  __shared__ __align__(16) float As[2][GBK][GBM + GPAD];
-  __shared__ __align__(16) float Bs[2][GBK][GBN + GPAD];
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const int m0 = blockIdx.y * GBM, n0 = blockIdx.x * GBN;
+__global__ void __launch_bounds__(cmm::kThreads, 1) coarse_mma_kernel(GemmArgs p) {
+  using namespace cmm;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_SLOT);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * 128, n0 = blockIdx.x * 128;
   const long long b = blockIdx.z;
   const float* A = p.A + b * p.sA;
   const float* B = p.B + b * p.sB;
-  float ra[4], rb[4];
-  // element i of this thread's share of the A slice: (m, k) within the tile
-  auto a_pos = [&](int i, int& m, int& k) {
-    const int idx = tid + 256 * i;
-    if (TA) k = idx >> 6, m = idx & 63;
-    else m = idx >> 4, k = idx & 15;
-  };
-  auto b_pos = [&](int i, int& k, int& n) {
-    const int idx = tid + 256 * i;
-    if (TB) n = idx >> 4, k = idx & 15;
-    else k = idx >> 6, n = idx & 63;
-  };
-  auto load = [&](int k0) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      int m, k, n, kb;
-      a_pos(i, m, k);
-      const int gm = m0 + m, gk = k0 + k;
-      ra[i] = (gm < p.M && gk < p.K) ? (TA ? A[static_cast<long long>(gk) * p.lda + gm]
-                                            : A[static_cast<long long>(gm) * p.lda + gk])
-                                     : 0.0f;
-      b_pos(i, kb, n);
-      const int gn = n0 + n, gkb = k0 + kb;
-      rb[i] = (gn < p.N && gkb < p.K) ? (TB ? B[static_cast<long long>(gn) * p.ldb + gkb]
-                                             : B[static_cast<long long>(gkb) * p.ldb + gn])
-                                      : 0.0f;
-    }
-  };
-  auto store = [&](int buf) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      int m, k, n, kb;
-      a_pos(i, m, k);
-      As[buf][k][m] = ra[i];
-      b_pos(i, kb, n);
-      Bs[buf][kb][n] = rb[i];
-    }
-  };
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-  const int nk = (p.K + GBK - 1) / GBK;
-  load(0);
-  store(0);
-  __syncthreads();
-  for (int t = 0; t < nk; ++t) {
-    const int cur = t & 1;
-    if (t + 1 < nk) load((t + 1) * GBK);
-#pragma unroll
-    for (int k = 0; k < GBK; ++k) {
-      const float4 a4 = *reinterpret_cast<const float4*>(&As[cur][k][ty * 4]);
-      const float4 b4 = *reinterpret_cast<const float4*>(&Bs[cur][k][tx * 4]);
-      const float a[4] = {a4.x, a4.y, a4.z, a4.w}, bb[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
-    }
-    // the other buffer was last read before the previous barrier
-    if (t + 1 < nk) store(cur ^ 1);
-    __syncthreads();
+  const int nk = (p.K + BK - 1) / BK;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[B_FULL], 256);
+    mbar_init(&bars[B_FULL + 1], 256);
+    mbar_init(&bars[B_EMPTY], 1);
+    mbar_init(&bars[B_EMPTY + 1], 1);
+    mbar_init(&bars[B_DONE], 1);
+    fence_barrier_init();
   }
-  float* C = p.C + b * p.sC;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + ty * 4 + i;
-    if (m >= p.M) continue;
-    float rs = p.alpha, lse = 0.0f, dlt = 0.0f;
-    if (EPI == EPI_UNPOOL) rs = p.alpha / static_cast<float>(cube_valid_count(p.g, m));
-    if (EPI == EPI_DS) {
-      lse = p.row_lse[b * p.sRow + m];
-      dlt = p.row_dlt[b * p.sRow + m];
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool skip_all = aborted(p.st);
+  // A is K-major in shared memory unless TA; B (the MMA's N x K operand) is K-major when TB
+  const bool vec_a = (p.lda & 3) == 0 && (reinterpret_cast<uintptr_t>(A) & 15) == 0;
+  const bool vec_b = (p.ldb & 3) == 0 && (reinterpret_cast<uintptr_t>(B) & 15) == 0;
+  if (warp < 8) {
+    const int tid = threadIdx.x;
+    bool ok = !skip_all;
+    for (int c = 0; ok && c < nk; ++c) {
+      const int st = c & 1;
+      if (c >= 2 && !mbar_wait(&bars[B_EMPTY + st], ((c >> 1) + 1) & 1, p.st, p.timeout_ns, 141)) {
+        ok = false;
+        break;
+      }
+      const uint32_t sb = sbase + st * STAGE_BYTES;
+      load_slice<!TA>(A, p.lda, m0, p.M, c * BK, p.K, vec_a, sb, sb + OP_BYTES, tid);
+      load_slice<TB>(B, p.ldb, n0, p.N, c * BK, p.K, vec_b, sb + 2 * OP_BYTES, sb + 3 * OP_BYTES, tid);
+      fence_proxy_async_smem();  // generic-proxy stores, read next by the tensor cores
+      mbar_arrive(&bars[B_FULL + st]);
     }
+    // epilogue: warp w reads TMEM lanes 32 (w % 4).. and columns 64 (w / 4)..
+    if (ok && mbar_wait(&bars[B_DONE], 0, p.st, p.timeout_ns, 142)) {
+      tc_fence_after();
+      const int q = warp & 3, ch = warp >> 2;
+      const int m = m0 + q * 32 + lane;
+      float* C = p.C + b * p.sC;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx * 4 + j;
-      if (n >= p.N) continue;
-      const long long o = static_cast<long long>(m) * p.ldc + n;
-      if (EPI == EPI_DS) {
-        float* aux = p.aux + b * p.sC;
-        const float pr = expf(aux[o] - lse);
-        aux[o] = pr;
-        C[o] = pr * (acc[i][j] - dlt);
-      } else {
-        C[o] = acc[i][j] * rs;
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 64 + hh * 32, v);
+        tmem_ld_wait();
+        if (m < p.M) {
+          float rs = p.alpha, lse = 0.0f, dlt = 0.0f;
+          if (EPI == EPI_UNPOOL) rs = p.alpha / static_cast<float>(cube_valid_count(p.g, m));
+          if (EPI == EPI_DS) {
+            lse = p.row_lse[b * p.sRow + m];
+            dlt = p.row_dlt[b * p.sRow + m];
+          }
+          const int nb = n0 + ch * 64 + hh * 32;
+          const long long o0 = static_cast<long long>(m) * p.ldc + nb;
+          float* aux = EPI == EPI_DS ? p.aux + b * p.sC : nullptr;
+          if (nb + 32 <= p.N && (p.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(C) & 15) == 0 &&
+              (EPI != EPI_DS || (reinterpret_cast<uintptr_t>(aux) & 15) == 0)) {
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {  // whole float4 rows of 32 columns
+              float r[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) r[u] = __uint_as_float(v[4 * j4 + u]);
+              if (EPI == EPI_DS) {
+                float4* ap = reinterpret_cast<float4*>(aux + o0) + j4;
+                const float4 sv = *ap;
+                const float pr[4] = {expf(sv.x - lse), expf(sv.y - lse), expf(sv.z - lse), expf(sv.w - lse)};
+                *ap = make_float4(pr[0], pr[1], pr[2], pr[3]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) r[u] = pr[u] * (r[u] - dlt);
+              } else {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) r[u] *= rs;
+              }
+              reinterpret_cast<float4*>(C + o0)[j4] = make_float4(r[0], r[1], r[2], r[3]);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (nb + j >= p.N) break;
+              const long long o = o0 + j;
+              const float acc = __uint_as_float(v[j]);
+              if (EPI == EPI_DS) {
+                const float pr = expf(aux[o] - lse);
+                aux[o] = pr;
+                C[o] = pr * (acc - dlt);
+              } else {
+                C[o] = acc * rs;
+              }
+            }
+          }
+        }
       }
     }
+  } else if (!skip_all) {
+    // warp 8: the whole warp runs the loop, one elected lane issues
+    const uint32_t idesc = make_idesc(128, 128, FMT_BF16, TA, !TB);
+    bool ok = true;
+    for (int c = 0; c < nk; ++c) {
+      const int st = c & 1;
+      if (!mbar_wait_warp(&bars[B_FULL + st], (c >> 1) & 1, p.st, p.timeout_ns, 143)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t sb = sbase + st * STAGE_BYTES;
+      if (elect_one()) {
+#pragma unroll
+        for (int prod = 0; prod < 3; ++prod) {  // hi*hi, hi*lo, lo*hi
+          const uint32_t a_s = sb + (prod == 2 ? OP_BYTES : 0u);
+          const uint32_t b_s = sb + 2 * OP_BYTES + (prod == 1 ? OP_BYTES : 0u);
+#pragma unroll
+          for (int ks = 0; ks < BK / 16; ++ks) {
+            // K-major: k step = 32 bytes along the row; MN-major: 16 k rows = 2048 bytes
+            const uint64_t ad = TA ? sw128_desc(a_s + ks * 2048, 8192, 1024) : sw128_desc(a_s + ks * 32, 16, 1024);
+            const uint64_t bd = TB ? sw128_desc(b_s + ks * 32, 16, 1024) : sw128_desc(b_s + ks * 2048, 8192, 1024);
+            umma_f16_ss(tmem, ad, bd, idesc, (c > 0 || prod > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(&bars[B_EMPTY + st]);
+        if (c == nk - 1) umma_commit(&bars[B_DONE]);
+      }
+      __syncwarp();
+    }
+    if (ok) mbar_wait_drain(&bars[B_DONE], 0, p.st, p.timeout_ns, 144);  // every MMA done before TMEM is freed
   }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) tmem_dealloc(tmem, 128);
 }
 
 template <bool TA, bool TB, int EPI>
 cudaError_t gemm(const GemmArgs& a, int batch, cudaStream_t stream) {
-  const dim3 grid(static_cast<unsigned>((a.N + GBN - 1) / GBN), static_cast<unsigned>((a.M + GBM - 1) / GBM),
-                  static_cast<unsigned>(batch));
-  coarse_gemm_kernel<TA, TB, EPI><<<grid, 256, 0, stream>>>(a);
-  return cudaGetLastError();
-}
-
-// ------------------------------------------------------------------------ combine
-// O = G * Oc^[cube] + O_f on valid rows, in place on the bf16 output and, when present, its
-// fp32 copy (then the bf16 value is the rounded fp32 sum; the C ABI always passes the copy).
-// One thread per 4 columns of a row.
-__global__ void __launch_bounds__(256) coarse_combine_kernel(__nv_bfloat16* __restrict__ out,
-                                                             float* __restrict__ o32, const float* __restrict__ gate,
-                                                             const float* __restrict__ oc, Geom g, int BH, int D) {
-  const int q4 = D >> 2;
-  const long long u = blockIdx.x * 256LL + threadIdx.x;
-  const long long rows = static_cast<long long>(BH) * g.Npad;
-  if (u >= rows * q4) return;
-  const long long row = u / q4;
-  const int c = static_cast<int>(u % q4) * 4;
-  const int bh = static_cast<int>(row / g.Npad), slot = static_cast<int>(row % g.Npad);
-  if (!token_valid(g, slot >> 6, slot & 63)) return;  // padding rows stay 0
-  const float gv = gate[row];
-  const float4 ov = *reinterpret_cast<const float4*>(oc + (static_cast<long long>(bh) * g.T + (slot >> 6)) * D + c);
-  float x[4];
-  if (o32) {
-    load_f<4>(o32 + row * D + c, x);
-  } else {
-    load_bf<4>(out + row * D + c, x);
+  static bool attr_set = false;
+  if (!attr_set) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(coarse_mma_kernel<TA, TB, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, cmm::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
   }
-  x[0] = fmaf(gv, ov.x, x[0]);
-  x[1] = fmaf(gv, ov.y, x[1]);
-  x[2] = fmaf(gv, ov.z, x[2]);
-  x[3] = fmaf(gv, ov.w, x[3]);
-  if (o32) store_f<4>(o32 + row * D + c, x);
-  const __nv_bfloat162 lo = __floats2bfloat162_rn(x[0], x[1]), hi = __floats2bfloat162_rn(x[2], x[3]);
-  uint2 w;
-  w.x = *reinterpret_cast<const uint32_t*>(&lo);
-  w.y = *reinterpret_cast<const uint32_t*>(&hi);
-  *reinterpret_cast<uint2*>(out + row * D + c) = w;
+  const dim3 grid(static_cast<unsigned>((a.N + 127) / 128), static_cast<unsigned>((a.M + 127) / 128),
+                  static_cast<unsigned>(batch));
+  coarse_mma_kernel<TA, TB, EPI><<<grid, cmm::kThreads, cmm::SMEM_BYTES, stream>>>(a);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------------ gate backward
@@ -381,7 +485,7 @@ __global__ void __launch_bounds__(256) coarse_gate_bwd_kernel(
 // ------------------------------------------------------------------------ launch
 cudaError_t launch_coarse_forward(const void* v, const double* qbar64, const double* kbar64, const double* S64,
                                   float* P32, const CoarseTensors& c, const Geom& g, int BH, int D,
-                                  cudaStream_t stream, int* launches) {
+                                  DevStatus* st, unsigned long long timeout_ns, cudaStream_t stream, int* launches) {
   const long long cubes = static_cast<long long>(BH) * g.T;
   const unsigned blocks = static_cast<unsigned>((cubes + 7) / 8);
   const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
@@ -397,23 +501,17 @@ cudaError_t launch_coarse_forward(const void* v, const double* qbar64, const dou
   a.M = g.T, a.N = D, a.K = g.T;
   a.alpha = 1.0f;
   a.g = g;
+  a.st = st;
+  a.timeout_ns = timeout_ns;
   cudaError_t e = gemm<false, false, EPI_STORE>(a, BH, stream);
   *launches = 3;
   return e;
 }
 
-cudaError_t launch_coarse_combine(void* out, float* out_f32, const float* gate, const float* oc, const Geom& g,
-                                  int BH, int D, cudaStream_t stream) {
-  const long long units = static_cast<long long>(BH) * g.Npad * (D / 4);
-  coarse_combine_kernel<<<static_cast<unsigned>((units + 255) / 256), 256, 0, stream>>>(
-      static_cast<__nv_bfloat16*>(out), out_f32, gate, oc, g, BH, D);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_coarse_backward(const void* out, const float* out_f32, const void* dout, const float* lse,
                                    const float* gate, const CoarseTensors& c, float* dgate, float* delta,
                                    float* nlse2, const CoarseGradWs& w, float scale, const Geom& g, int BH, int D,
-                                   cudaStream_t stream, int* launches) {
+                                   DevStatus* st, unsigned long long timeout_ns, cudaStream_t stream, int* launches) {
   const long long cubes = static_cast<long long>(BH) * g.T;
   const unsigned blocks = static_cast<unsigned>((cubes + 7) / 8);
   const __nv_bfloat16* ob = static_cast<const __nv_bfloat16*>(out);
@@ -434,6 +532,8 @@ cudaError_t launch_coarse_backward(const void* out, const float* out_f32, const 
   a.M = g.T, a.N = g.T, a.K = D;
   a.alpha = scale;
   a.g = g;
+  a.st = st;
+  a.timeout_ns = timeout_ns;
   if (e == cudaSuccess) e = gemm<false, true, EPI_STORE>(a, BH, stream);
   // dP = dOc^ Vc^T;  P = exp(S - lse_c) over S;  dS = P (dP - delta_c)
   GemmArgs d = a;
@@ -449,6 +549,8 @@ cudaError_t launch_coarse_backward(const void* out, const float* out_f32, const 
   q.M = g.T, q.N = D, q.K = g.T;
   q.alpha = scale;
   q.g = g;
+  q.st = st;
+  q.timeout_ns = timeout_ns;
   if (e == cudaSuccess) e = gemm<false, false, EPI_UNPOOL>(q, BH, stream);
   // dKc / n = scale * dS^T Qc / n
   GemmArgs k = q;

@@ -15,7 +15,12 @@ struct DevStatus {
   unsigned int abort;      // set once any CTA gave up; later CTAs return at once
   unsigned int where;      // code of the first wait that timed out
   unsigned int router_fallback;  // rows the router decided again in fp64 (and the length of its row list)
-  unsigned int pad[60];
+  unsigned int f16_out_of_range; // a tensor converted to fp16 for the single-product path did not fit
+  unsigned int f16_max[2];       // backward: largest |dO| and |V| (fp32 bits) seen by the conversions
+  unsigned int f16_single;       // backward: 1 when every product takes the fp16 single-product path
+  unsigned int item_next[3];     // work-item counters of the forward, dQ and dK/dV kernels
+  unsigned int grid[3];          // their grid sizes (the number of per-CTA clock records)
+  unsigned int pad[50];
 };
 enum : unsigned int {
   DEVERR_TIMEOUT = 1u,
@@ -153,6 +158,19 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
+// 3-D tiled store shared -> global (bulk group of this thread); coordinates must be >= 0
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y,
+                                             int32_t z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until the shared-memory sources of this thread's committed bulk stores have been read
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// wait until this thread's committed bulk stores have completed
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // 1-D bulk copy global -> shared (both 16-byte aligned, size a multiple of 16), this CTA only
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -279,6 +297,7 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t M, uint32_t N, uint32
   return (1u << 4) | (ab_format << 7) | (ab_format << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
          ((N >> 3) << 17) | ((M >> 4) << 24);
 }
+constexpr uint32_t FMT_F16 = 0u;
 constexpr uint32_t FMT_BF16 = 1u;
 constexpr uint32_t FMT_E4M3 = 0u;
 // kind::i8 with signed 8-bit A and B (format 1) and a signed 32-bit accumulator (D format 2)
@@ -326,6 +345,12 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

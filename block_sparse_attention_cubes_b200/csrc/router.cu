@@ -21,18 +21,11 @@
 #include "geometry.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
+#include "router_common.cuh"
 
 namespace sa {
 
 // ------------------------------------------------------------------------ pooling
-__device__ __forceinline__ float e4m3_value(uint32_t b) {
-  // 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits; exponent 0 is subnormal.
-  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
-  float v = (e == 0u) ? static_cast<float>(m) * (1.0f / 512.0f)
-                      : __uint_as_float(((e + 120u) << 23) | (m << 20));
-  if (e == 15u && m == 7u) v = __uint_as_float(0x7fc00000u);
-  return (b & 0x80u) ? -v : v;
-}
 
 // grid (ceil(T/4), BH, 2); 256 threads = 4 groups of 64, one cube per group.
 // ESZ = bytes per element (2: bf16, 1: e4m3).
@@ -431,133 +424,205 @@ struct RowMeta {
   double pad;
 };
 
-constexpr int kLimbRow = 128;  // bytes per limb row: K = 128 int8 (D = 64 rows are zero-padded)
-constexpr int kExpZero = -1100;  // exponent recorded for an all-zero row
-constexpr int kExpBias = 2048;   // exponents are kept as E + 2048 > 0 for the per-head atomicMax
 
-// grid (ceil(T/4), BH, 2); as pool_kernel, plus the limbs, exponents and (Q) 1-norms.
-template <int ESZ>
-__global__ void __launch_bounds__(256) pool_limbs_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ k,
-                                                         const float* __restrict__ q_scale,
-                                                         const float* __restrict__ k_scale, double* __restrict__ qbar,
-                                                         double* __restrict__ kbar, int8_t* __restrict__ qlimb,
-                                                         int8_t* __restrict__ klimb, int* __restrict__ qexp,
-                                                         int* __restrict__ kexp, double* __restrict__ ql1,
-                                                         unsigned* __restrict__ kexp_max, Geom g, int D) {
-  constexpr int EPT = 16 / ESZ;  // elements per 16-byte vector
-  __shared__ double red[4][64][EPT];
-  const int grp = threadIdx.x >> 6, t64 = threadIdx.x & 63;
-  const int c = blockIdx.x * 4 + grp;
-  const int bh = blockIdx.y;
-  const bool is_k = blockIdx.z == 1;
-  const uint8_t* src = is_k ? k : q;
-  const int tpr = D * ESZ / 16;  // threads per token row (4, 8 or 16: lanes 0..tpr-1 of the group's first warp)
-  const int rows_per_iter = 64 / tpr;
-  const int chunk = t64 % tpr, roff = t64 / tpr;
-  double acc[EPT];
-#pragma unroll
-  for (int e = 0; e < EPT; ++e) acc[e] = 0.0;
-  int vt = 0, vh = 0, vw = 0;
-  if (c < g.T) {
-    cube_extent(g, c, vt, vh, vw);
-    const size_t row_bytes = static_cast<size_t>(D) * ESZ;
-    const uint8_t* base = src + (static_cast<size_t>(bh) * g.Npad + static_cast<size_t>(c) * 64) * row_bytes;
-    // eight rows' loads in flight per thread before any of them is accumulated
-    for (int r0 = roff; r0 < 64; r0 += 8 * rows_per_iter) {
-      uint4 v[8];
-      bool ok[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int r = r0 + u * rows_per_iter;
-        ok[u] = r < 64 && slot_valid(vt, vh, vw, r);
-        v[u] = ok[u] ? __ldg(reinterpret_cast<const uint4*>(base + r * row_bytes) + chunk) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (!ok[u]) continue;
-        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-          float f;
-          if constexpr (ESZ == 2) {
-            f = __uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
-          } else {
-            f = e4m3_value((w[e >> 2] >> (8 * (e & 3))) & 0xffu);
+// Pooling for the tensor-core router.  Persistent CTAs, one per SM; items are (head, cube, Q or
+// K), dealt round-robin so the CTAs stream neighbouring cubes together.  Warp 16 (one lane)
+// brings each item's rows (up to the cube's last valid slot) into a 24-stage shared-memory ring
+// with 1-D bulk copies, half a cube (32 slots) per stage; warps 0-15 take the items in turn,
+// each lane summing D/32 columns over the cube's valid rows in fp64 and releasing each half as
+// soon as it is summed, and write the mean, its limbs, the row's binary exponent and (Q) its
+// 1-norm.  Half-cube stages keep 16 cubes in progress and 8 halves in flight per SM.
+namespace rpl {
+constexpr int kConsumers = 16;
+constexpr int kThreads = (kConsumers + 1) * 32;
+constexpr int kStages = 24;
+constexpr uint32_t kStageBytes = 8192;  // half a cube: 32 rows x 256 bytes (bf16, D = 128)
+constexpr uint32_t OFF_BAR = kStages * kStageBytes;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 2 * kStages * 8 + 1024;
+}  // namespace rpl
+
+struct PoolArgs {
+  const uint8_t* q;
+  const uint8_t* k;
+  const float* q_scale;
+  const float* k_scale;
+  double* qbar;
+  double* kbar;
+  int8_t* qlimb;
+  int8_t* klimb;
+  int* qexp;
+  int* kexp;
+  double* ql1;
+  unsigned* kexp_max;
+  int* rkmax;
+  int* rkmin;
+  DevStatus* st;
+  Geom g;
+  int BH, D, Tk;
+  unsigned long long timeout_ns;
+};
+
+// ESZ = bytes per element (2: bf16, 1: e4m3); EPL = D / 32 elements per lane.
+template <int ESZ, int EPL>
+__global__ void __launch_bounds__(rpl::kThreads, 1) pool_limbs_kernel(const PoolArgs a) {
+  using namespace rpl;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* empty = full + kStages;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Geom& g = a.g;
+  const int D = a.D;
+  const size_t row_bytes = static_cast<size_t>(D) * ESZ;
+  const long long n_items = 2LL * a.BH * g.T;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (aborted(a.st)) return;
+  if (warp == kConsumers) {
+    if (lane == 0) {
+      long long i = 0;  // stage sequence: item j of this CTA fills stages 2j (slots 0-31) and 2j+1 (32-63)
+      bool ok = true;
+      for (long long it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+        const int which = static_cast<int>(it & 1);
+        const long long cube = it >> 1;  // bh * T + c
+        const int c = static_cast<int>(cube % g.T);
+        int vt, vh, vw;
+        cube_extent(g, c, vt, vh, vw);
+        const uint32_t nrows = static_cast<uint32_t>(16 * (vt - 1) + 4 * (vh - 1) + vw);  // through the last valid slot
+        const uint8_t* src = (which ? a.k : a.q) + (static_cast<size_t>(cube / g.T) * g.Npad + static_cast<size_t>(c) * 64) *
+                                                       row_bytes;
+        for (uint32_t h = 0; h < 2; ++h, ++i) {
+          const int stage = static_cast<int>(i % kStages);
+          if (i >= kStages && !mbar_wait(&empty[stage], ((i / kStages) + 1) & 1, a.st, a.timeout_ns, 131)) {
+            ok = false;
+            break;
           }
-          acc[e] += static_cast<double>(f);
+          const uint32_t r0 = 32 * h, r1 = nrows < r0 + 32 ? nrows : r0 + 32;
+          if (r1 > r0) {
+            const uint32_t bytes = (r1 - r0) * static_cast<uint32_t>(row_bytes);
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            bulk_load(smem + stage * kStageBytes, src + r0 * row_bytes, bytes, &full[stage]);
+          } else {
+            mbar_arrive(&full[stage]);  // no valid slot in this half: an empty stage
+          }
         }
       }
+      // drain: the copies still in flight land before the CTA exits
+      const long long issued = i;
+      for (long long d = (issued > kStages ? issued - kStages : 0); d < issued; ++d)
+        mbar_wait_drain(&full[d % kStages], (d / kStages) & 1, a.st, a.timeout_ns, 132);
     }
+    return;
   }
+  long long j = warp;  // this CTA's item counter
+  for (long long it = blockIdx.x + static_cast<long long>(warp) * gridDim.x; it < n_items;
+       it += static_cast<long long>(kConsumers) * gridDim.x, j += kConsumers) {
+    const int which = static_cast<int>(it & 1);
+    const long long cube = it >> 1;
+    const int bh = static_cast<int>(cube / g.T), c = static_cast<int>(cube % g.T);
+    int vt, vh, vw;
+    cube_extent(g, c, vt, vh, vw);
+    // four accumulator sets (slot d0 of each row of 4) keep independent fp64 chains in flight
+    double acc4[4][EPL];
 #pragma unroll
-  for (int e = 0; e < EPT; ++e) red[grp][t64][e] = acc[e];
-  __syncthreads();
-  if (c >= g.T || t64 >= tpr) return;
-  const int n = vt * vh * vw;
-  double scale = 1.0;
-  if constexpr (ESZ == 1) {
-    const float* sc = is_k ? k_scale : q_scale;
-    scale = static_cast<double>(sc[static_cast<size_t>(bh) * g.T + c]);
-  }
-  const size_t rowid = static_cast<size_t>(bh) * g.T + c;
-  double* dst = (is_k ? kbar : qbar) + rowid * D + chunk * EPT;
-  double x[EPT];
-  double amax = 0.0, l1 = 0.0;
+    for (int u = 0; u < 4; ++u)
 #pragma unroll
-  for (int e = 0; e < EPT; ++e) {
-    double s = 0.0;
-    for (int r = 0; r < rows_per_iter; ++r) s += red[grp][t64 + r * tpr][e];
-    x[e] = s * scale / static_cast<double>(n);
-    dst[e] = x[e];
-    amax = fmax(amax, fabs(x[e]));
-    l1 += fabs(x[e]);
-  }
-  // row maximum and 1-norm over the tpr lanes holding the row
-  const unsigned mask = (tpr >= 32) ? 0xffffffffu : ((1u << tpr) - 1u);
-  for (int o = 1; o < tpr; o <<= 1) {
-    amax = fmax(amax, __shfl_xor_sync(mask, amax, o));
-    l1 += __shfl_xor_sync(mask, l1, o);
-  }
-  int E = kExpZero;
-  if (amax > 0.0) frexp(amax, &E);  // amax = m 2^E, m in [0.5, 1): every |x_d| < 2^E
-  const double up = amax > 0.0 ? ldexp(1.0, 30 - E) : 0.0;
-  uint32_t limb[4][EPT / 4];
+      for (int e = 0; e < EPL; ++e) acc4[u][e] = 0.0;
+    bool ok = true;
+    for (int h = 0; h < 2; ++h) {  // the two half-cube stages: slot rows a0 in {2h, 2h + 1}
+      const long long i = 2 * j + h;
+      const int stage = static_cast<int>(i % kStages);
+      if (!mbar_wait_warp(&full[stage], (i / kStages) & 1, a.st, a.timeout_ns, 133)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* tile = smem + stage * kStageBytes + lane * EPL * ESZ;
+      const int a_end = vt < 2 * h + 2 ? vt : 2 * h + 2;
+    for (int a0 = 2 * h; a0 < a_end; ++a0)
+      for (int b0 = 0; b0 < vh; ++b0)
 #pragma unroll
-  for (int w = 0; w < EPT / 4; ++w) limb[0][w] = limb[1][w] = limb[2][w] = limb[3][w] = 0u;
+        for (int d0 = 0; d0 < 4; ++d0) {
+          if (d0 >= vw) break;
+          double* acc = acc4[d0];
+          const uint8_t* rp = tile + ((a0 - 2 * h) * 16 + b0 * 4 + d0) * row_bytes;
+          if constexpr (ESZ == 2) {
+            uint32_t wv[EPL / 2];
+            if constexpr (EPL == 4) {
+              const uint2 t2 = *reinterpret_cast<const uint2*>(rp);
+              wv[0] = t2.x;
+              wv[1] = t2.y;
+            } else {
+              wv[0] = *reinterpret_cast<const uint32_t*>(rp);
+            }
 #pragma unroll
-  for (int e = 0; e < EPT; ++e) {
-    int X = static_cast<int>(rint(x[e] * up));  // |X| <= 2^30
-    const int d3 = ((X + 128) & 255) - 128;
-    X = (X - d3) >> 8;
-    const int d2 = ((X + 128) & 255) - 128;
-    X = (X - d2) >> 8;
-    const int d1 = ((X + 128) & 255) - 128;
-    const int d0 = (X - d1) >> 8;  // in [-64, 64]
-    const int sh = 8 * (e & 3);
-    limb[0][e >> 2] |= (static_cast<uint32_t>(d0) & 255u) << sh;
-    limb[1][e >> 2] |= (static_cast<uint32_t>(d1) & 255u) << sh;
-    limb[2][e >> 2] |= (static_cast<uint32_t>(d2) & 255u) << sh;
-    limb[3][e >> 2] |= (static_cast<uint32_t>(d3) & 255u) << sh;
-  }
-  int8_t* lb = (is_k ? klimb : qlimb);
+            for (int e = 0; e < EPL; ++e)
+              acc[e] += static_cast<double>(
+                  __uint_as_float((e & 1) ? (wv[e >> 1] & 0xffff0000u) : (wv[e >> 1] << 16)));
+          } else {
+            uint32_t wv = EPL == 4 ? *reinterpret_cast<const uint32_t*>(rp)
+                                   : static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(rp));
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    int8_t* row = lb + ((static_cast<size_t>(bh) * 4 + a) * g.T + c) * kLimbRow;
-    if constexpr (EPT == 8) {
-      *reinterpret_cast<uint2*>(row + chunk * EPT) = make_uint2(limb[a][0], limb[a][1]);
-      if (D < kLimbRow) *reinterpret_cast<uint2*>(row + D + chunk * EPT) = make_uint2(0u, 0u);
-    } else {
-      *reinterpret_cast<uint4*>(row + chunk * EPT) = make_uint4(limb[a][0], limb[a][1], limb[a][2], limb[a][3]);
-      if (D < kLimbRow) *reinterpret_cast<uint4*>(row + D + chunk * EPT) = make_uint4(0u, 0u, 0u, 0u);
+            for (int e = 0; e < EPL; ++e) acc[e] += static_cast<double>(e4m3_value((wv >> (8 * e)) & 0xffu));
+          }
+        }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);  // the half's rows have been read
     }
-  }
-  if (chunk == 0) {
-    if (is_k) {
-      kexp[rowid] = E;
-      atomicMax(kexp_max + bh, static_cast<unsigned>(E + kExpBias));
-    } else {
-      qexp[rowid] = E;
-      ql1[rowid] = l1;
+    if (!ok) break;
+    double acc[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] = (acc4[0][e] + acc4[1][e]) + (acc4[2][e] + acc4[3][e]);
+    const int n = vt * vh * vw;
+    double scale = 1.0;
+    if constexpr (ESZ == 1) scale = static_cast<double>((which ? a.k_scale : a.q_scale)[cube]);
+    double x[EPL];
+    double amax = 0.0, l1 = 0.0;
+    double* dst = (which ? a.kbar : a.qbar) + static_cast<size_t>(cube) * D + lane * EPL;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      x[e] = acc[e] * scale / static_cast<double>(n);
+      dst[e] = x[e];
+      amax = fmax(amax, fabs(x[e]));
+      l1 += fabs(x[e]);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+    int E = kExpZero;
+    if (amax > 0.0) frexp(amax, &E);  // amax = m 2^E, m in [0.5, 1): every |x_d| < 2^E
+    const double up = amax > 0.0 ? ldexp(1.0, 30 - E) : 0.0;
+    uint32_t limb[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) limb_digits(x[e], up, e, limb);
+    int8_t* lb = which ? a.klimb : a.qlimb;
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+      int8_t* rowp = lb + ((static_cast<size_t>(bh) * 4 + l) * g.T + c) * kLimbRow;
+      if constexpr (EPL == 4) {
+        reinterpret_cast<uint32_t*>(rowp)[lane] = limb[l];
+      } else {  // D = 64: 64 bytes of limbs, then 64 zero bytes
+        reinterpret_cast<uint16_t*>(rowp)[lane] = static_cast<uint16_t>(limb[l]);
+        reinterpret_cast<uint16_t*>(rowp + 64)[lane] = 0;
+      }
+    }
+    if (lane == 0) {
+      if (which) {
+        a.kexp[static_cast<size_t>(bh) * a.Tk + c] = E;  // rows of Tk entries: 16-byte aligned per head
+        atomicMax(a.kexp_max + bh, static_cast<unsigned>(E + kExpBias));
+      } else {
+        a.qexp[cube] = E;
+        a.ql1[cube] = l1;
+        a.rkmax[cube] = INT_MIN;  // the score kernel's per-row key extrema start here
+        a.rkmin[cube] = INT_MAX;
+      }
     }
   }
 }
@@ -567,7 +632,8 @@ namespace rsc {
 constexpr int kThreads = 320;  // warp 0 TMA, warp 1 TMEM owner + MMA, warps 2-9 epilogue
 constexpr uint32_t OFF_Q = 0;                      // 4 limbs x [128 rows][128 B]
 constexpr uint32_t OFF_K = 65536;                  // 2 stages x 4 limbs x [128 keys][128 B]
-constexpr uint32_t OFF_BAR = OFF_K + 2 * 65536;
+constexpr uint32_t OFF_STG = OFF_K + 2 * 65536;   // 8 epilogue warps x [32 rows][128 B] key staging
+constexpr uint32_t OFF_BAR = OFF_STG + 8 * 4096;
 constexpr uint32_t OFF_SLOT = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
 constexpr uint32_t TMEM_COLS = 512;                // level w at columns 128w
@@ -580,9 +646,11 @@ struct ScoreArgs {
   const double* ql1;
   const unsigned* kexp_max;
   int* keys;        // [BH*T, Tk]
+  int* rkmax;       // [BH*T] largest and smallest key of each row (atomics)
+  int* rkmin;
   RowMeta* meta;    // [BH*T]
   DevStatus* st;
-  int T, Tk, BH;
+  int T, Tk, BH;    // kexp rows have Tk entries per head
   double scale;
   unsigned long long timeout_ns;
 };
@@ -593,7 +661,7 @@ struct ScoreArgs {
 template <int KS>
 __global__ void __launch_bounds__(rsc::kThreads, 1)
     score_keys_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const ScoreArgs a) {
+                      const __grid_constant__ CUtensorMap tm_keys, const ScoreArgs a) {
   using namespace rsc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -661,7 +729,6 @@ __global__ void __launch_bounds__(rsc::kThreads, 1)
     }
   } else if (warp == 1) {
     if (!skip_all) {
-      const uint32_t idesc = make_idesc_s8(128, 128);
       uint32_t ks = 0, tile = 0;
       int qn = 0;
       long long prev = -1;
@@ -686,17 +753,7 @@ __global__ void __launch_bounds__(rsc::kThreads, 1)
         tc_fence_after();
         const uint32_t kb = sbase + OFF_K + st * 65536;
         if (elect_one()) {
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-#pragma unroll
-            for (int la = 0; la <= w; ++la) {
-              const int lb = w - la;
-#pragma unroll
-              for (int kk = 0; kk < KS; ++kk)
-                umma_i8_ss(tmem + 128 * w, sw128_desc(sbase + OFF_Q + la * 16384 + kk * 32, 16, 1024),
-                           sw128_desc(kb + lb * 16384 + kk * 32, 16, 1024), idesc, (la > 0 || kk > 0) ? 1u : 0u);
-            }
-          }
+          issue_limb_products<KS>(tmem, sbase + OFF_Q, kb);
           umma_commit(&bars[B_KE + st]);
           umma_commit(&bars[B_TF]);
           if (last_of_rb) umma_commit(&bars[B_QE]);
@@ -716,6 +773,9 @@ __global__ void __launch_bounds__(rsc::kThreads, 1)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     uint32_t tile = 0;
     bool ok = !skip_all;
+    long long prev_rbk = -1;
+    int A = 0, f = 0, Eq = 0, Ekm = 0;
+    bool nonzero = false;
     for (long long t = t0; ok && t < t1; ++t, ++tile) {
       const int bh = static_cast<int>(t / (static_cast<long long>(nrb) * nrb));
       const int rem = static_cast<int>(t % (static_cast<long long>(nrb) * nrb));
@@ -723,19 +783,22 @@ __global__ void __launch_bounds__(rsc::kThreads, 1)
       const int i = rb * 128 + r;
       const bool row_ok = i < T;
       const size_t rowid = static_cast<size_t>(bh) * T + (row_ok ? i : 0);
-      // per-row scaling of the keys: |raw| <= |Qbar_i|_1 2^Ekmax < 2^e, keys in units of 2^(e - 30)
-      int A = 0;
-      int f = 0;
-      const int Eq = __ldg(a.qexp + rowid);
-      const int Ekm = static_cast<int>(__ldg(a.kexp_max + bh)) - kExpBias;
-      const double B = ldexp(__ldg(a.ql1 + rowid), Ekm);
-      const bool nonzero = Eq != kExpZero && Ekm != kExpZero && B > 0.0;
-      if (nonzero) {
-        int e;
-        frexp(B, &e);
-        f = e - 30;
+      const long long rbk = static_cast<long long>(bh) * nrb + rb;
+      if (rbk != prev_rbk) {
+        // per-row scaling of the keys: |raw| <= |Qbar_i|_1 2^Ekmax < 2^e, keys in units of 2^(e - 30)
+        prev_rbk = rbk;
+        f = 0;
+        Eq = __ldg(a.qexp + rowid);
+        Ekm = static_cast<int>(__ldg(a.kexp_max + bh)) - kExpBias;
+        const double B = ldexp(__ldg(a.ql1 + rowid), Ekm);
+        nonzero = Eq != kExpZero && Ekm != kExpZero && B > 0.0;
+        if (nonzero) {
+          int e;
+          frexp(B, &e);
+          f = e - 30;
+        }
+        A = 36 + f - Eq;
       }
-      A = 36 + f - Eq;
       if (row_ok && cb == 0 && half == 0) {
         RowMeta m;
         m.cunit = ldexp(a.scale * 1.4426950408889634, f);
@@ -745,16 +808,30 @@ __global__ void __launch_bounds__(rsc::kThreads, 1)
         m.pad = 0.0;
         a.meta[rowid] = m;
       }
-      if (!mbar_wait(&bars[B_TF], tile & 1, a.st, a.timeout_ns, 121)) {
+      if (!mbar_wait_warp(&bars[B_TF], tile & 1, a.st, a.timeout_ns, 121)) {  // warp-uniform (warp ops below)
         ok = false;
         break;
       }
       tc_fence_after();
-      int* krow = a.keys + rowid * a.Tk;
-      const int* ekp = a.kexp + static_cast<size_t>(bh) * T;
+      const int* ekp = a.kexp + static_cast<size_t>(bh) * a.Tk;  // padded rows: 16-byte aligned
+      int lmax = INT_MIN, lmin = INT_MAX;
+      uint8_t* stg = smem + OFF_STG + (warp - 2) * 4096;
 #pragma unroll 1
       for (int ch = 0; ch < 2; ++ch) {
         const int col0 = 64 * half + 32 * ch;
+        // the 32 key exponents of this chunk (entries past T are never stored: any value will do)
+        int ekc[32];
+        {
+          const int jc = cb * 128 + col0;
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4) {
+            const int4 e4 = jc + 4 * v4 < a.Tk ? __ldg(reinterpret_cast<const int4*>(ekp + jc) + v4) : make_int4(0, 0, 0, 0);
+            ekc[4 * v4] = e4.x;
+            ekc[4 * v4 + 1] = e4.y;
+            ekc[4 * v4 + 2] = e4.z;
+            ekc[4 * v4 + 3] = e4.w;
+          }
+        }
         uint32_t L0[32], L1[32], L2[32], L3[32];
         tmem_ld32(t_lane + 0 + col0, L0);
         tmem_ld32(t_lane + 128 + col0, L1);
@@ -766,32 +843,42 @@ __global__ void __launch_bounds__(rsc::kThreads, 1)
           mbar_arrive(&bars[B_TE]);  // this thread's reads of the tile are complete
         }
         const int j0 = cb * 128 + col0;
-        if (!row_ok) continue;
+        // this warp's previous store has read its staging rows
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
+          const int j = j0 + 4 * c4;
           int kv[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int c = 4 * c4 + u;
-            const int j = j0 + c;
-            const long long hiw = static_cast<long long>(static_cast<int>(L0[c])) * 256 + static_cast<int>(L1[c]);
-            const long long low = static_cast<long long>(static_cast<int>(L2[c])) * 256 + static_cast<int>(L3[c]);
-            const long long v = hiw * 65536 + low;
-            int sh = A - (j < T ? __ldg(ekp + j) : 0);
+            const long long v = limb_levels(L0[c], L1[c], L2[c], L3[c]);
+            int sh = A - ekc[c];
             sh = sh < 1 ? 1 : (sh > 62 ? 62 : sh);
             kv[u] = static_cast<int>((v + (1LL << (sh - 1))) >> sh);
+            if (row_ok && j + u < T) {
+              lmax = max(lmax, kv[u]);
+              lmin = min(lmin, kv[u]);
+            }
           }
-          const int j = j0 + 4 * c4;
-          if (j + 3 < T) {
-            *reinterpret_cast<int4*>(krow + j) = make_int4(kv[0], kv[1], kv[2], kv[3]);
-          } else {
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              if (j + u < T) krow[j + u] = kv[u];
-          }
+          // row `lane` of the warp's 32 x 32 staging tile, 16-byte chunk c4, 128-byte swizzle
+          st_shared_v4(smem_u32(stg) + sw128_offset(lane, c4), kv[0], kv[1], kv[2], kv[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        // rows and columns past T fall outside the map and are not written
+        if (lane == 0) {
+          tma_store_3d(&tm_keys, stg, j0, rb * 128 + quarter * 32, bh);
+          bulk_commit_group();
         }
       }
+      if (row_ok && lmax >= lmin) {
+        atomicMax(a.rkmax + rowid, lmax);
+        atomicMin(a.rkmin + rowid, lmin);
+      }
     }
+    if (lane == 0) bulk_wait0();  // the key stores are complete before the CTA leaves
   }
   tc_fence_before();
   __syncthreads();
@@ -799,35 +886,70 @@ __global__ void __launch_bounds__(rsc::kThreads, 1)
 }
 
 // ------------------------------------------------------------------------ key selection
-// 2^50 * 2^(-u c): the fixed-point mass of a score u key units below the row maximum.
+// 2^36 * 2^(-u c): the fixed-point mass of a score u key units below the row maximum.  A row's
+// masses sum to at most T 2^36 < 2^50 (T <= 8192), so a histogram bucket packs its count in
+// bits 50-63 and its mass in bits 0-49 of one 64-bit word, and sums of such words (buckets,
+// prefixes) stay packed.
+constexpr int kMassBits = 36;
+constexpr unsigned long long kMassMask = (1ull << 50) - 1ull;
+constexpr unsigned long long kCountOne = 1ull << 50;
 __device__ __forceinline__ unsigned long long mass_key(uint32_t u, double c) {
-  const double x = -static_cast<double>(u) * c;
+  // Two conversion-pipe operations per entry (f64 -> f32 and ex2); the rest is fp64 and integer
+  // arithmetic.  u as fp64 exactly: 2^52 + u has u in its low word.
+  const double ud = __hiloint2double(0x43300000, static_cast<int>(u)) - 4503599627370496.0;
+  const double x = -ud * c;  // log2 of the mass relative to the row maximum, <= 0
   if (x < -60.0) return 0ull;
-  const double fl = floor(x);
-  const float p2 = ex2_approx(static_cast<float>(x - fl));  // in [1, 2)
-  const int ex = static_cast<int>(fl) + 50;                 // >= -10
-  const double m = static_cast<double>(p2) * __longlong_as_double(static_cast<long long>(ex + 1023) << 52);
-  return static_cast<unsigned long long>(__double2ull_rz(m));
+  // x = n + f with n = round(x) (round-to-nearest through 1.5 * 2^52) and f in [-1/2, 1/2]
+  const double t = x + 6755399441055744.0;
+  const int n = __double2loint(t);
+  const double f = x - (t - 6755399441055744.0);
+  const float p2 = ex2_approx(__double2float_rn(f));  // in [2^-1/2, 2^1/2]
+  // 2^(36 + n) * p2 as an integer: p2 = m * 2^(e - 23) with m the 24-bit significand
+  const uint32_t pb = __float_as_uint(p2);
+  const unsigned long long m = static_cast<unsigned long long>((pb & 0x7fffffu) | 0x800000u);
+  const int sh = kMassBits + n + static_cast<int>((pb >> 23) & 0xffu) - 127 - 23;
+  return sh >= 0 ? (m << sh) : (sh > -64 ? (m >> -sh) : 0ull);
 }
 
 constexpr unsigned kDebugRouterFallback = 2u;  // debug flag: every row takes the fp64 path
 
-// One warp per row of keys.  Writes the row's list and count when its decision is certain;
-// otherwise appends the row to `flist` (length in st->router_fallback) for the fp64 path.
-__global__ void __launch_bounds__(256) select_keys_kernel(const int* __restrict__ keys, int Tk,
-                                                          const RowMeta* __restrict__ meta, int rows, int T, int top_k,
-                                                          float top_p, int cap, int32_t* __restrict__ kv_index,
-                                                          int32_t* __restrict__ kv_count, int* __restrict__ flist,
-                                                          DevStatus* st, unsigned debug) {
-  __shared__ uint32_t cnt_s[8][256];
-  __shared__ unsigned long long mass_s[8][256];
+// Visit a row of keys 128 at a time (int4 of 4 consecutive keys per lane), in order.  Every
+// lane calls f for every chunk (the chunk loop is uniform), so f may use warp collectives;
+// keys past T arrive as 0 and f must check j + u < T.  The loads of four chunks are issued
+// together, so a pass over a row waits for L2 a quarter as often.
+template <class F>
+__device__ __forceinline__ void for_key_chunks(const int* kr, int T, int lane, F&& f) {
+  for (int j0 = 0; j0 < T; j0 += 512) {
+    int4 x[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = j0 + 128 * c + 4 * lane;
+      x[c] = j < T ? *reinterpret_cast<const int4*>(kr + j) : make_int4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      if (j0 + 128 * c < T) f(j0 + 128 * c + 4 * lane, x[c]);
+  }
+}
+
+// One warp per row; every pass reads the row from global memory (after the first, from L2).
+__global__ void __launch_bounds__(256, 4) select_keys_kernel(const int* __restrict__ keys, int Tk,
+                                                                         const int* __restrict__ rkmax,
+                                                                         const int* __restrict__ rkmin,
+                                                                         const RowMeta* __restrict__ meta, int rows,
+                                                                         int T, int top_k, float top_p, int cap,
+                                                                         int32_t* __restrict__ kv_index,
+                                                                         int32_t* __restrict__ kv_count,
+                                                                         int* __restrict__ flist, DevStatus* st,
+                                                                         unsigned debug,
+                                                                         unsigned long long timeout_ns) {
+  __shared__ unsigned long long hist_s[8][256];  // packed (count << 50) + mass per bucket
   __shared__ unsigned long long cand_s[8][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + warp;
   if (row >= rows) return;
   const int* kr = keys + static_cast<size_t>(row) * Tk;
-  uint32_t* cnt = cnt_s[warp];
-  unsigned long long* mass = mass_s[warp];
+  unsigned long long* hist = hist_s[warp];
   int32_t* out = kv_index + static_cast<size_t>(row) * cap;
   const int nk = max(1, min(top_k, T));
   if (top_p >= 1.0f || nk >= T) {  // every block
@@ -838,29 +960,10 @@ __global__ void __launch_bounds__(256) select_keys_kernel(const int* __restrict_
     }
     return;
   }
-  // ---- maximum and minimum key
-  int kmax = INT_MIN, kmin = INT_MAX;
-  for (int j0 = 0; j0 < T; j0 += 128) {
-    const int j = j0 + 4 * lane;
-    if (j < T) {
-      const int4 v = *reinterpret_cast<const int4*>(kr + j);
-      const int vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (j + u < T) {
-          kmax = max(kmax, vv[u]);
-          kmin = min(kmin, vv[u]);
-        }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-  }
+  const int kmax = rkmax[row], kmin = rkmin[row];
   const RowMeta m = meta[row];
   const double c = m.cunit;
-  // ---- radix descent on u = kmax - key over [lo, hi]
+  // ---- (1) radix descent on u = kmax - key over [lo, hi]
   uint32_t lo = 0, hi = static_cast<uint32_t>(kmax - kmin);
   unsigned long long c_above = 0, m_above = 0, Z = 0;
   double target = -1.0;
@@ -868,57 +971,39 @@ __global__ void __launch_bounds__(256) select_keys_kernel(const int* __restrict_
   for (int level = 0;; ++level) {
     const uint32_t span = hi - lo;
     const int s = span < 256u ? 0 : (32 - __clz(span)) - 8;  // (hi - lo) >> s < 256
-    for (int d = lane; d < 256; d += 32) {
-      cnt[d] = 0;
-      mass[d] = 0ull;
-    }
+    for (int d = lane; d < 256; d += 32) hist[d] = 0ull;
     __syncwarp();
-    for (int j0 = 0; j0 < T; j0 += 128) {
-      const int j = j0 + 4 * lane;
-      if (j < T) {
-        const int4 v = *reinterpret_cast<const int4*>(kr + j);
-        const int vv[4] = {v.x, v.y, v.z, v.w};
+    for_key_chunks(kr, T, lane, [&](int j, const int4& v) {
+      const int vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4) {
-          const uint32_t uu = static_cast<uint32_t>(kmax - vv[u4]);
-          if (j + u4 < T && uu >= lo && uu <= hi) {
-            const int b = static_cast<int>((uu - lo) >> s);
-            atomicAdd(&cnt[b], 1u);
-            atomicAdd(&mass[b], mass_key(uu, c));
-          }
-        }
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const uint32_t uu = static_cast<uint32_t>(kmax - vv[u4]);
+        if (j + u4 < T && uu >= lo && uu <= hi) atomicAdd(&hist[(uu - lo) >> s], kCountOne + mass_key(uu, c));
       }
-    }
+    });
     __syncwarp();
-    uint32_t lc = 0;
-    unsigned long long lm = 0;
+    unsigned long long lw = 0;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      lc += cnt[lane * 8 + u];
-      lm += mass[lane * 8 + u];
-    }
-    uint32_t ic = lc;
-    unsigned long long im = lm;
+    for (int u = 0; u < 8; ++u) lw += hist[lane * 8 + u];
+    unsigned long long iw = lw;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t oc = __shfl_up_sync(0xffffffffu, ic, o);
-      const unsigned long long om = __shfl_up_sync(0xffffffffu, im, o);
-      if (lane >= o) {
-        ic += oc;
-        im += om;
-      }
+      const unsigned long long ow = __shfl_up_sync(0xffffffffu, iw, o);
+      if (lane >= o) iw += ow;
     }
     if (level == 0) {
-      Z = __shfl_sync(0xffffffffu, im, 31);
+      Z = __shfl_sync(0xffffffffu, iw, 31) & kMassMask;
       if (top_p > 0.0f) target = static_cast<double>(top_p) * static_cast<double>(Z);
     }
-    unsigned long long c_run = c_above + (ic - lc), m_run = m_above + (im - lm);
+    const unsigned long long ex = iw - lw;  // packed sums of the buckets before this lane's
+    unsigned long long c_run = c_above + (ex >> 50), m_run = m_above + (ex & kMassMask);
     int hit = -1;
     unsigned long long c_before = 0, m_before = 0;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const uint32_t cu = cnt[lane * 8 + u];
-      const unsigned long long mu = mass[lane * 8 + u];
+      const unsigned long long wu = hist[lane * 8 + u];
+      const uint32_t cu = static_cast<uint32_t>(wu >> 50);
+      const unsigned long long mu = wu & kMassMask;
       if (hit < 0 && cu > 0 && c_run + cu >= static_cast<unsigned long long>(nk) &&
           static_cast<double>(m_run + mu) >= target) {
         hit = lane * 8 + u;
@@ -937,7 +1022,7 @@ __global__ void __launch_bounds__(256) select_keys_kernel(const int* __restrict_
     const int bstar = __shfl_sync(0xffffffffu, hit, src);
     c_above = __shfl_sync(0xffffffffu, c_before, src);
     m_above = __shfl_sync(0xffffffffu, m_before, src);
-    bcnt = cnt[bstar];
+    bcnt = static_cast<uint32_t>(hist[bstar] >> 50);
     __syncwarp();
     const unsigned long long nlo = static_cast<unsigned long long>(lo) + (static_cast<unsigned long long>(bstar) << s);
     const unsigned long long nhi = nlo + (1ull << s) - 1ull;
@@ -945,33 +1030,56 @@ __global__ void __launch_bounds__(256) select_keys_kernel(const int* __restrict_
     hi = static_cast<uint32_t>(nhi < hi ? nhi : hi);
     if (bcnt <= 32u || s == 0) break;
   }
-  bool certain = bcnt <= 32u && (debug & kDebugRouterFallback) == 0u;
+  // the provisional list (ids above the bucket and the candidates) must fit the row
+  bool certain = bcnt <= 32u && c_above + bcnt <= static_cast<unsigned long long>(cap) &&
+                 (debug & kDebugRouterFallback) == 0u;
   uint32_t ub = 0;
   int jb = -1, n = 0;
   unsigned long long cum_at = 0, cum_before = 0;
+  uint32_t unext = 0xffffffffu;
   if (certain) {
-    // ---- the boundary bucket's candidates, sorted by (u, id)
-    int nc = 0;
-    for (int j0 = 0; j0 < T; j0 += 128) {
-      const int j = j0 + 4 * lane;
-      int4 v = make_int4(0, 0, 0, 0);
-      if (j < T) v = *reinterpret_cast<const int4*>(kr + j);
+    // ---- (2) write ids above the bucket and the marked candidates in ascending id order
+    int written = 0, nc = 0;
+    uint32_t umin_below = 0xffffffffu;
+    for_key_chunks(kr, T, lane, [&](int j, const int4& v) {
       const int vv[4] = {v.x, v.y, v.z, v.w};
+      int tag[4];
+      int nsel = 0;
 #pragma unroll
       for (int u4 = 0; u4 < 4; ++u4) {
         const uint32_t uu = static_cast<uint32_t>(kmax - vv[u4]);
-        const bool in = j + u4 < T && uu >= lo && uu <= hi;
-        const uint32_t b = __ballot_sync(0xffffffffu, in);
-        if (in) {
+        const bool in = j + u4 < T;
+        tag[u4] = !in ? 0 : (uu < lo ? 1 : (uu <= hi ? 2 : 0));  // 1: kept, 2: candidate
+        if (in && uu > hi) umin_below = min(umin_below, uu);
+        nsel += tag[u4] ? 1 : 0;
+        const bool isc = tag[u4] == 2;
+        const uint32_t b = __ballot_sync(0xffffffffu, isc);
+        if (isc) {
           const int pos = nc + __popc(b & ((1u << lane) - 1u));
           if (pos < 32) cand_s[warp][pos] = (static_cast<unsigned long long>(uu) << 32) | static_cast<uint32_t>(j + u4);
         }
         nc += __popc(b);
       }
-    }
+      int incl = nsel;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int pos = written + incl - nsel;
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4)
+        if (tag[u4]) {
+          if (pos < cap) out[pos] = (j + u4) | (tag[u4] == 2 ? static_cast<int>(0x80000000u) : 0);
+          ++pos;
+        }
+      written += __shfl_sync(0xffffffffu, incl, 31);
+    });
+#pragma unroll
+    for (int o = 16; o; o >>= 1) umin_below = min(umin_below, __shfl_xor_sync(0xffffffffu, umin_below, o));
     __syncwarp();
+    // ---- (3) the candidates sorted by (u, id): bitonic sort of 32 keys across the warp
     unsigned long long key = lane < static_cast<int>(bcnt) ? cand_s[warp][lane] : ~0ull;
-    // bitonic sort of 32 keys across the warp, ascending
 #pragma unroll
     for (int k2 = 2; k2 <= 32; k2 <<= 1) {
 #pragma unroll
@@ -979,8 +1087,7 @@ __global__ void __launch_bounds__(256) select_keys_kernel(const int* __restrict_
         const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, j2);
         const bool up = (lane & k2) == 0;
         const bool lower = (lane & j2) == 0;
-        const bool take_min = (lower == up);
-        key = take_min ? (key < other ? key : other) : (key > other ? key : other);
+        key = (lower == up) ? (key < other ? key : other) : (key > other ? key : other);
       }
     }
     const bool valid = lane < static_cast<int>(bcnt);
@@ -1000,7 +1107,7 @@ __global__ void __launch_bounds__(256) select_keys_kernel(const int* __restrict_
     const bool okb = valid && (c_above + pc >= static_cast<unsigned long long>(nk)) &&
                      (static_cast<double>(m_above + pm) >= target);
     const uint32_t okm = __ballot_sync(0xffffffffu, okb);
-    if (okm == 0u) {
+    if (okm == 0u || written != static_cast<int>(c_above + bcnt)) {
       certain = false;
     } else {
       const int L = __ffs(okm) - 1;
@@ -1009,48 +1116,36 @@ __global__ void __launch_bounds__(256) select_keys_kernel(const int* __restrict_
       n = static_cast<int>(c_above) + L + 1;
       cum_at = m_above + __shfl_sync(0xffffffffu, pm, L);
       cum_before = cum_at - __shfl_sync(0xffffffffu, ms, L);
+      // the next element in order: the next candidate, else the first key below the bucket
+      const uint32_t un = __shfl_sync(0xffffffffu, uu, (L + 1) & 31);
+      unext = (L + 1 < static_cast<int>(bcnt)) ? un : umin_below;
+      // ---- (4) drop the candidates the boundary leaves out, in place (reads stay ahead of writes)
+      int wpos = 0;
+      for (int r0 = 0; r0 < written; r0 += 32) {
+        const int r = r0 + lane;
+        int e = r < written ? out[r] : 0;
+        bool keep = r < written;
+        if (keep && e < 0) {
+          const int jj = e & 0x7fffffff;
+          const uint32_t uj = static_cast<uint32_t>(kmax - kr[jj]);
+          keep = uj < ub || (uj == ub && jj <= jb);
+          e = jj;
+        }
+        const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+        __syncwarp();
+        if (keep) out[wpos + __popc(kb & ((1u << lane) - 1u))] = e;
+        wpos += __popc(kb);
+      }
+      if (wpos != n) certain = false;
     }
   }
   if (certain) {
-    // ---- emit the kept ids in ascending order; the smallest u left out is the next key
-    int written = 0;
-    uint32_t unext = 0xffffffffu;
-    for (int j0 = 0; j0 < T; j0 += 128) {
-      const int j = j0 + 4 * lane;
-      int4 v = make_int4(0, 0, 0, 0);
-      if (j < T) v = *reinterpret_cast<const int4*>(kr + j);
-      const int vv[4] = {v.x, v.y, v.z, v.w};
-      bool sel[4];
-      int nsel = 0;
-#pragma unroll
-      for (int u4 = 0; u4 < 4; ++u4) {
-        const uint32_t uu = static_cast<uint32_t>(kmax - vv[u4]);
-        const bool in = j + u4 < T;
-        sel[u4] = in && (uu < ub || (uu == ub && j + u4 <= jb));
-        if (in && !sel[u4]) unext = min(unext, uu);
-        nsel += sel[u4] ? 1 : 0;
-      }
-      int incl = nsel;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-      }
-      int pos = written + incl - nsel;
-#pragma unroll
-      for (int u4 = 0; u4 < 4; ++u4)
-        if (sel[u4]) {
-          if (pos < cap) out[pos] = j + u4;
-          ++pos;
-        }
-      written += __shfl_sync(0xffffffffu, incl, 31);
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) unext = min(unext, __shfl_xor_sync(0xffffffffu, unext, o));
     // ---- is the decision certain within the error bounds?
     const double Zd = static_cast<double>(Z);
-    const double delta = (2.0 * m.eps_s + 2.0 * 4.76837158203125e-07 + 1e-12) * Zd;  // 2^-21
-    bool gap_ok = unext == 0xffffffffu || static_cast<double>(unext - ub) > 2.0 * m.eps_key;
+    // masses: ex2.approx within 2^-21 relative, scores within eps_s, and one fixed-point unit
+    // of truncation per element
+    const double delta = (2.0 * m.eps_s + 2.0 * 4.76837158203125e-07 + 1e-12) * Zd + static_cast<double>(T);
+    const bool gap_ok = unext == 0xffffffffu || static_cast<double>(unext - ub) > 2.0 * m.eps_key;
     bool cross_ok = true;
     if (top_p > 0.0f) {
       if (n > nk)
@@ -1059,11 +1154,8 @@ __global__ void __launch_bounds__(256) select_keys_kernel(const int* __restrict_
       else
         cross_ok = static_cast<double>(cum_at) - target > delta;
     }
-    certain = gap_ok && cross_ok && written == n;
-    if (certain && lane == 0) {
-      if (n > cap) flag_error(st, DEVERR_CAPACITY, 0);
-      kv_count[row] = min(n, cap);
-    }
+    certain = gap_ok && cross_ok;
+    if (certain && lane == 0) kv_count[row] = n;  // n <= cap (checked above)
   }
   if (!certain && lane == 0) {
     const unsigned k = atomicAdd(&st->router_fallback, 1u);
@@ -1071,36 +1163,52 @@ __global__ void __launch_bounds__(256) select_keys_kernel(const int* __restrict_
   }
 }
 
-// The fp64 path for the rows the key selection queued: each warp recomputes the row's scores
-// Qbar_i . Kbar_j * scale in fp64 into its own scratch row, then selects as select_kernel does.
+// The fp64 path for the rows the key selection queued: one CTA per row (grid-stride over the
+// queue).  Its four warps compute the row's scores Qbar_i . Kbar_j * scale in fp64 into shared
+// memory, lanes splitting each dot product over D (coalesced reads of every Kbar row, then a
+// shuffle reduction), and warp 0 selects from there as select_kernel does.
 __global__ void __launch_bounds__(128) router_fallback_kernel(const double* __restrict__ qbar,
                                                               const double* __restrict__ kbar, int D, int T,
-                                                              double scale, const int* __restrict__ flist,
-                                                              double* __restrict__ scratch, int top_k, float top_p,
-                                                              int cap, int32_t* __restrict__ kv_index,
+                                                              double scale, const int* __restrict__ flist, int top_k,
+                                                              float top_p, int cap, int32_t* __restrict__ kv_index,
                                                               int32_t* __restrict__ kv_count, DevStatus* st) {
-  __shared__ uint32_t cnt_s[4][256];
-  __shared__ unsigned long long mass_s[4][256];
-  __shared__ double qs[4][128];
+  extern __shared__ double srow[];  // [T] scores
+  __shared__ uint32_t cnt_s[256];
+  __shared__ unsigned long long mass_s[256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * 4 + warp, nw = gridDim.x * 4;
   const int nf = static_cast<int>(*reinterpret_cast<const volatile unsigned*>(&st->router_fallback));
-  double* s = scratch + static_cast<size_t>(gw) * T;
-  for (int k = gw; k < nf; k += nw) {
+  const int per = D >> 5;  // doubles per lane (2 or 4)
+  for (int k = blockIdx.x; k < nf; k += gridDim.x) {
     const int row = flist[k];
     const size_t bh = static_cast<size_t>(row) / T;
-    for (int d = lane; d < D; d += 32) qs[warp][d] = qbar[static_cast<size_t>(row) * D + d];
-    __syncwarp();
-    for (int j = lane; j < T; j += 32) {
-      const double* kj = kbar + (bh * T + j) * D;
-      double acc = 0.0;
-      for (int d = 0; d < D; ++d) acc = fma(qs[warp][d], kj[d], acc);
-      s[j] = acc * scale;
+    double qv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) qv[e] = e < per ? qbar[static_cast<size_t>(row) * D + lane * per + e] : 0.0;
+    // eight keys per warp per round, every load issued before the arithmetic
+    for (int j0 = warp * 8; j0 < T; j0 += 32) {
+      double kv[8][4];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u < T ? j0 + u : T - 1;
+        const double* kj = kbar + (bh * T + j) * D + lane * per;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) kv[u][e] = e < per ? kj[e] : 0.0;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        double acc = 0.0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc = fma(qv[e], kv[u][e], acc);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0 && j0 + u < T) srow[j0 + u] = acc * scale;
+      }
     }
-    __syncwarp();
-    select_row_fp64(s, T, top_k, top_p, cap, kv_index + static_cast<size_t>(row) * cap, kv_count + row, st,
-                    cnt_s[warp], mass_s[warp]);
-    __syncwarp();
+    __syncthreads();
+    if (warp == 0)
+      select_row_fp64(srow, T, top_k, top_p, cap, kv_index + static_cast<size_t>(row) * cap, kv_count + row, st,
+                      cnt_s, mass_s);
+    __syncthreads();
   }
 }
 
@@ -1140,11 +1248,12 @@ cudaError_t launch_select(const double* S, int32_t* kv_index, int32_t* kv_count,
   return cudaGetLastError();
 }
 
-// fixed (not the device's SM count) so that workspace sizes do not depend on the device
-int plan_fallback_ctas() { return 148; }
+// fixed (not the device's SM count): one row per CTA, grid-stride over the queue (4 CTAs per SM)
+int plan_fallback_ctas() { return 592; }
 
 cudaError_t launch_plan_fast(const void* q, const void* k, const float* q_scale, const float* k_scale,
-                             const CUtensorMap& tm_qlimb, const CUtensorMap& tm_klimb, const Geom& g, int BH, int D,
+                             const CUtensorMap& tm_qlimb, const CUtensorMap& tm_klimb, const CUtensorMap& tm_keys,
+                             const Geom& g, int BH, int D,
                              bool fp8, double scale, int top_k, float top_p, int cap, unsigned debug,
                              unsigned long long timeout_ns, const PlanFastWs& w, int32_t* kv_index, int32_t* kv_count,
                              DevStatus* st, cudaStream_t stream, int* launches) {
@@ -1154,27 +1263,58 @@ cudaError_t launch_plan_fast(const void* q, const void* k, const float* q_scale,
                                          rsc::SMEM_BYTES);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(score_keys_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsc::SMEM_BYTES);
+    if (e == cudaSuccess)  // one fp64 score row of up to 8192 cubes
+      e = cudaFuncSetAttribute(router_fallback_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 8192 * 8);
+    for (auto fn : {pool_limbs_kernel<2, 4>, pool_limbs_kernel<2, 2>, pool_limbs_kernel<1, 4>, pool_limbs_kernel<1, 2>})
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, rpl::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   // the per-head maxima of the key exponents start at 0 (below every biased exponent)
   if (cudaMemsetAsync(w.kexp_max, 0, static_cast<size_t>(BH) * sizeof(unsigned), stream) != cudaSuccess)
     return cudaErrorUnknown;
-  dim3 pg((g.T + 3) / 4, BH, 2);
-  if (fp8)
-    pool_limbs_kernel<1><<<pg, 256, 0, stream>>>(static_cast<const uint8_t*>(q), static_cast<const uint8_t*>(k),
-                                                 q_scale, k_scale, w.qbar, w.kbar, w.qlimb, w.klimb, w.qexp, w.kexp,
-                                                 w.ql1, w.kexp_max, g, D);
-  else
-    pool_limbs_kernel<2><<<pg, 256, 0, stream>>>(static_cast<const uint8_t*>(q), static_cast<const uint8_t*>(k),
-                                                 q_scale, k_scale, w.qbar, w.kbar, w.qlimb, w.klimb, w.qexp, w.kexp,
-                                                 w.ql1, w.kexp_max, g, D);
+  PoolArgs pa;
+  pa.q = static_cast<const uint8_t*>(q);
+  pa.k = static_cast<const uint8_t*>(k);
+  pa.q_scale = q_scale;
+  pa.k_scale = k_scale;
+  pa.qbar = w.qbar;
+  pa.kbar = w.kbar;
+  pa.qlimb = w.qlimb;
+  pa.klimb = w.klimb;
+  pa.qexp = w.qexp;
+  pa.kexp = w.kexp;
+  pa.ql1 = w.ql1;
+  pa.kexp_max = w.kexp_max;
+  pa.rkmax = w.rkmax;
+  pa.rkmin = w.rkmin;
+  pa.st = st;
+  pa.g = g;
+  pa.BH = BH;
+  pa.D = D;
+  pa.Tk = w.Tk;
+  pa.timeout_ns = timeout_ns;
+  const long long pitems = 2LL * BH * g.T;
+  const int pgrid = static_cast<int>(pitems < num_sms() ? pitems : num_sms());
+  if (fp8) {
+    if (D == 128)
+      pool_limbs_kernel<1, 4><<<pgrid, rpl::kThreads, rpl::SMEM_BYTES, stream>>>(pa);
+    else
+      pool_limbs_kernel<1, 2><<<pgrid, rpl::kThreads, rpl::SMEM_BYTES, stream>>>(pa);
+  } else {
+    if (D == 128)
+      pool_limbs_kernel<2, 4><<<pgrid, rpl::kThreads, rpl::SMEM_BYTES, stream>>>(pa);
+    else
+      pool_limbs_kernel<2, 2><<<pgrid, rpl::kThreads, rpl::SMEM_BYTES, stream>>>(pa);
+  }
   ScoreArgs sa_;
   sa_.qexp = w.qexp;
   sa_.kexp = w.kexp;
   sa_.ql1 = w.ql1;
   sa_.kexp_max = w.kexp_max;
   sa_.keys = w.keys;
+  sa_.rkmax = w.rkmax;
+  sa_.rkmin = w.rkmin;
   sa_.meta = reinterpret_cast<RowMeta*>(w.meta);
   sa_.st = st;
   sa_.T = g.T;
@@ -1186,16 +1326,15 @@ cudaError_t launch_plan_fast(const void* q, const void* k, const float* q_scale,
   const long long items = static_cast<long long>(BH) * nrb * nrb;
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
   if (D == 64)
-    score_keys_kernel<2><<<grid, rsc::kThreads, rsc::SMEM_BYTES, stream>>>(tm_qlimb, tm_klimb, sa_);
+    score_keys_kernel<2><<<grid, rsc::kThreads, rsc::SMEM_BYTES, stream>>>(tm_qlimb, tm_klimb, tm_keys, sa_);
   else
-    score_keys_kernel<4><<<grid, rsc::kThreads, rsc::SMEM_BYTES, stream>>>(tm_qlimb, tm_klimb, sa_);
+    score_keys_kernel<4><<<grid, rsc::kThreads, rsc::SMEM_BYTES, stream>>>(tm_qlimb, tm_klimb, tm_keys, sa_);
   const int rows = BH * g.T;
-  select_keys_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(w.keys, w.Tk, reinterpret_cast<const RowMeta*>(w.meta), rows,
-                                                         g.T, top_k, top_p, cap, kv_index, kv_count, w.flist, st,
-                                                         debug);
-  router_fallback_kernel<<<plan_fallback_ctas(), 128, 0, stream>>>(w.qbar, w.kbar, D, g.T, scale, w.flist,
-                                                                   w.fb_scratch, top_k, top_p, cap, kv_index,
-                                                                   kv_count, st);
+  select_keys_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(
+        w.keys, w.Tk, w.rkmax, w.rkmin, reinterpret_cast<const RowMeta*>(w.meta), rows, g.T, top_k, top_p, cap,
+        kv_index, kv_count, w.flist, st, debug, timeout_ns);
+  router_fallback_kernel<<<plan_fallback_ctas(), 128, static_cast<size_t>(g.T) * sizeof(double), stream>>>(
+      w.qbar, w.kbar, D, g.T, scale, w.flist, top_k, top_p, cap, kv_index, kv_count, st);
   *launches = 5;
   return cudaGetLastError();
 }

@@ -62,7 +62,8 @@ typedef enum {
   SA_OP_BACKWARD = 2,
   SA_OP_PLAN_COARSE = 3,      /* sa_plan_coarse */
   SA_OP_BACKWARD_GATED = 4,   /* sa_backward_gated */
-  SA_OP_PLAN_BQ128 = 5        /* sa_plan_bq128 */
+  SA_OP_PLAN_BQ128 = 5,       /* sa_plan_bq128 */
+  SA_OP_BLOCK_MASS = 6        /* sa_block_mass */
 } sa_op;
 
 typedef struct {
@@ -83,6 +84,12 @@ typedef struct {
 /* Test hook: sa_plan decides every row on its fp64 path (normally taken only by the rows
  * whose tensor-core decision is within the error bound of changing). */
 #define SA_DEBUG_ROUTER_FALLBACK 2u
+/* Measurement hook: sa_forward and sa_backward record, for every CTA of their attention
+ * kernels, its start and end time and the work it did (read with sa_get_cta_clocks). */
+#define SA_DEBUG_CTA_CLOCKS 4u
+/* Measurement hook: the attention kernels take the fixed round-robin share of work items
+ * (CTA c: items c, c + grid, ...) instead of fetching them in order from a shared counter. */
+#define SA_DEBUG_STATIC_ITEMS 8u
 
 /* Padded token count Npad and cube count T implied by the latent grid (0 on bad input). */
 SA_API int sa_padded_tokens(const sa_params* p);
@@ -95,7 +102,7 @@ SA_API int sa_topk_from_fraction(double frac, int T);
 /* Bytes of device workspace `op` (sa_op) needs for these parameters; 0 on bad input.
  * Plan: status block + pooled Q and K (fp64, 2*B*H*T*D) + their int8 limbs (8*B*H*T*128) + per-row
  * exponents, norms and key scaling (48*B*H*T) + the fixed-point score keys (int32, B*H*T*Tk, Tk = T
- * rounded up to 4) + the fp64 rows' list (B*H*T) and scratch (fp64, 592*T).
+ * rounded up to 4) + the list of rows decided in fp64 (B*H*T).
  * Forward: status block + one 64-bit valid-slot mask per cube (T) + the union lists of
  * adjacent query-cube pairs (int32, B*H*ceil(T/2)*(1 + 2*kv_capacity)).  Backward: status block
  * + cube masks + Delta and -lse*log2(e) (fp32, 2*B*H*Npad) + the selection as a bit matrix
@@ -221,10 +228,11 @@ SA_API sa_status sa_plan_coarse(const void* q, const void* k, const void* v, con
                                 int32_t* kv_count, const sa_coarse* coarse, void* ws, size_t ws_bytes,
                                 sa_stream_t stream);
 
-/* sa_forward (arguments, errors and outputs as there, bf16 only), then
- * O = G (.) Repeat_64(coarse->oc) + O_f written in place over out_f32 and out (out is the
- * bf16 rounding of the fp32 sum).  out_f32 is REQUIRED (SA_ERR_INVALID_ARG when NULL):
- * summing into an already rounded bf16 O_f rounds twice, past the output error bounds.
+/* sa_forward (arguments, errors and outputs as there, bf16 only) with the gated combination
+ * O = G (.) Repeat_64(coarse->oc) + O_f formed in the forward kernel's epilogue from the fp32
+ * O_f of each valid row (one fused multiply-add per value): out_f32 receives the fp32 sum and
+ * out its bf16 rounding; padding rows stay 0.  out_f32 is REQUIRED (SA_ERR_INVALID_ARG when
+ * NULL): sa_backward_gated recovers the fine branch's Delta from it.
  * gate: [B,H,Npad] fp32.  lse is the fine stage's.  Workspace:
  * sa_workspace_size(p, SA_OP_FORWARD).  Deterministic. */
 SA_API sa_status sa_forward_gated(const void* q, const void* k, const void* v, const int32_t* kv_index,
@@ -260,6 +268,26 @@ SA_API sa_status sa_backward_gated(const void* q, const void* k, const void* v, 
 SA_API sa_status sa_plan_bq128(const void* q, const void* k, const sa_params* p, int32_t* kv_index, int32_t* kv_count,
                                void* ws, size_t ws_bytes, sa_stream_t stream);
 
+/* VSA2's fine-grained router with per-sequence Top-K (VSA2 page, section 2.2, router
+ * equations): each cube splits into G = 64 / (rt*rh*rw) groups (an rt x rh x rw box of its
+ * (t, h, w) offsets), each group is pooled over its valid tokens (Q_r, K_r = MeanPool_R), the
+ * group-level scores Q_r K_r^T * scale get a softmax over every key group of the sequence per
+ * query group, the G x G aggregation gives one score per (query cube, key cube) (P_r[i, j] = the
+ * mass a query group of cube i puts on the key groups of cube j, averaged over cube i's valid
+ * query groups), and per-sequence Top-K keeps the min(top_k * T, T^2) largest entries of P_r of
+ * each (batch, head), ties by the smaller row-major index (top_p is not used).  A group without
+ * valid tokens takes no part.  Each R_x is 1, 2 or 4 with G in {4, 8, 16} (else
+ * SA_ERR_UNSUPPORTED); bf16 only.  Outputs: kv_index / kv_count in sa_plan's layout (a row may
+ * keep no block; more than kv_capacity records SA_ERR_CAPACITY), and P_r [B,H,T,T] fp32 in p_r when
+ * it is not NULL.  The scores are exact integer limb products on the tensor cores (as sa_plan's);
+ * the softmax uses fp32 exponentials, so P_r is within a few 1e-6 relative of its fp64 value and
+ * the selection is that of this fp32 P_r.  Workspace: sa_plan_fine_workspace_size(p, rt, rh, rw).
+ * Deterministic. */
+SA_API size_t sa_plan_fine_workspace_size(const sa_params* p, int rt, int rh, int rw);
+SA_API sa_status sa_plan_fine(const void* q, const void* k, const sa_params* p, int rt, int rh, int rw,
+                              int32_t* kv_index, int32_t* kv_count, float* p_r, void* ws, size_t ws_bytes,
+                              sa_stream_t stream);
+
 /* Router recall diagnostic (SpargeAttention2 page, equation 8: tau = sum_j p_j m_j, the share of a
  * query's true softmax mass inside its kept blocks; VSA page, "Kernel Implementation": Top-32
  * keeps 50-90%).  Since lse is the log of a row's softmax normaliser, tau = exp(lse_kept -
@@ -270,6 +298,28 @@ SA_API sa_status sa_plan_bq128(const void* q, const void* k, const sa_params* p,
  * Asynchronous, one launch, no workspace.  Deterministic. */
 SA_API sa_status sa_recall(const float* lse_kept, const float* lse_all, const sa_params* p, float* recall,
                            float* cube_recall, sa_stream_t stream);
+
+/* Oracle block scores P_oracle (VSA2 page, section 2.2: MeanPool over the B x B tiles of the
+ * token-level softmax P, the reference the router approximates): pblock[b,h,i,j] = the softmax
+ * mass the valid query tokens of cube i put on the valid keys of cube j, averaged over cube i's
+ * valid tokens (each row sums to 1).  lse_all: [B,H,Npad] fp32, the lse of sa_forward on lists
+ * holding every block; then P_rc = exp(s_rc * scale - lse_r) and one dense tensor-core pass of
+ * S = Q K^T gives every entry.  q, k: [B,H,Npad,D] bf16; pblock: [B,H,T,T] fp32.  Workspace:
+ * sa_workspace_size(p, SA_OP_BLOCK_MASS) (status block + cube masks); bounded waits report
+ * SA_ERR_DEVICE_TIMEOUT through sa_get_device_status.  Cost: a dense S product over every token
+ * pair (2 * B*H*Npad^2*D FLOP) plus one exponential per pair: a diagnostic, not the step.
+ * Deterministic. */
+SA_API sa_status sa_block_mass(const void* q, const void* k, const float* lse_all, const sa_params* p, float* pblock,
+                               void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* Best recall of a selection size (VSA2 page, section 2.2, P_oracle; VSA page, "Kernel
+ * Implementation": Top-32 keeps 50-90% of the mass): best[b,h,i] = the sum of the n largest
+ * entries of row i of pblock, n = kv_count[b,h,i] clamped to [0, T]: the most recall any choice
+ * of n key cubes could reach, beside sa_recall's cube_recall of the router's own choice.
+ * pblock: [B,H,T,T] fp32 (non-negative); kv_count: [B,H,T] int32; best: [B,H,T] fp32.  One
+ * launch, no workspace.  Deterministic. */
+SA_API sa_status sa_best_recall(const float* pblock, const int32_t* kv_count, const sa_params* p, float* best,
+                                sa_stream_t stream);
 
 /* sa_plan without a workspace: the same router and the same results, for callers that
  * cannot allocate device memory (code running under a CUDA stream capture, serving
@@ -294,6 +344,20 @@ SA_API sa_status sa_get_device_status(const void* ws, sa_stream_t stream);
 /* Synchronises `stream` and returns how many rows the last sa_plan on this workspace decided
  * on its fp64 path; -1 on error. */
 SA_API int sa_plan_fallback_rows(const void* ws, sa_stream_t stream);
+
+/* Per-CTA clock records of the attention kernels, written by the last sa_forward (kernel 0,
+ * the forward) or sa_backward / sa_backward_gated (kernel 1, dQ; kernel 2, dK/dV) that ran on
+ * this workspace with SA_DEBUG_CTA_CLOCKS in p->debug_flags.  Synchronises `stream`, then
+ * copies min(grid, max_ctas, 1024) records into `out` (host memory, 4 values each: start and
+ * end in globaltimer nanoseconds, the work items and the pipeline steps the CTA processed) and
+ * sets *n_ctas to that number (0 when the call ran without the flag).  The kernels take their
+ * work items in order from a shared counter, each CTA the next one when it is free, so the
+ * records measure how evenly the dynamic schedule loaded the SMs.
+ * ws / ws_bytes: a workspace of sa_workspace_size(p, SA_OP_FORWARD or SA_OP_BACKWARD[_GATED]).
+ * Returns SA_ERR_INVALID_ARG for a null pointer, kernel outside 0..2 or a workspace too small
+ * to hold the records, SA_ERR_LAUNCH when the copy fails. */
+SA_API sa_status sa_get_cta_clocks(const void* ws, size_t ws_bytes, int kernel, unsigned long long* out,
+                                   int max_ctas, int* n_ctas, sa_stream_t stream);
 
 SA_API const char* sa_status_string(sa_status s);
 

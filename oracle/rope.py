@@ -22,7 +22,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .attention import CubeLayout, tile
+from .attention import CubeLayout, tile, untile
 
 
 def rope_tables(lat, sections, base: float = 10000.0):
@@ -72,3 +72,8 @@ def rope_3d(x: np.ndarray, lat, sections, cos: np.ndarray, sin: np.ndarray) -> n
 def tile_rope(x: np.ndarray, lay: CubeLayout, sections, cos, sin) -> np.ndarray:
     """Reading r4: the cube-major tensor of the rotated tokens ``[n_pad, D]``."""
     return tile(rope_3d(x, lay.lat, sections, cos, sin), lay)
+
+
+def untile_rope(y: np.ndarray, lay: CubeLayout, sections, cos, sin) -> np.ndarray:
+    """The inverse: latent order ``[L, D]``, each token rotated back (the angle negated)."""
+    return rope_3d(untile(y, lay), lay.lat, sections, cos, -sin)

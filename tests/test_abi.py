@@ -39,8 +39,8 @@ def test_geometry_and_workspace(lib):
     assert lib.sa_topk_from_fraction(0.03, 1562) == 47
     T, BH = 1440, 40
     plan_ws = sa.workspace_size(p, sa.OP_PLAN)
-    # pooled rows (fp64) + their 4 int8 limbs + per-row data + int32 keys + fp64 rows' scratch
-    assert plan_ws >= 256 + 2 * BH * T * 128 * 8 + 2 * BH * 4 * T * 128 + BH * T * T * 4 + 592 * T * 8
+    # pooled rows (fp64) + their 4 int8 limbs + per-row data + int32 keys
+    assert plan_ws >= 256 + 2 * BH * T * 128 * 8 + 2 * BH * 4 * T * 128 + BH * T * T * 4
     # the routers that keep every fp64 score (coarse branch) need the full score matrix
     assert sa.workspace_size(p, sa.OP_PLAN_COARSE) >= 256 + 2 * BH * T * 128 * 8 + BH * T * T * 8
     assert sa.workspace_size(p, sa.OP_FORWARD) >= 256 + 1440 * 8 + 40 * 720 * min(2 * 1440, 1440) * 4  # masks + pair unions
@@ -99,7 +99,8 @@ def test_coarse_entry_points_validate_on_the_host(lib):
     # fp64 plan + Pc; backward + dOc^, three per-cube terms, delta_c, scores and dS (each 256-byte aligned)
     assert sa.workspace_size(p, sa.OP_PLAN_COARSE) >= plan64 + BH * T * T * 4
     assert sa.workspace_size(p, sa.OP_BACKWARD_GATED) >= bwd + 4 * BH * T * D * 4 + BH * T * 4 + 2 * BH * T * T * 4
-    assert sa.workspace_size(p, 6) == 0
+    assert sa.workspace_size(p, sa.OP_BLOCK_MASS) == 256 + 256     # status block + cube masks
+    assert sa.workspace_size(p, 7) == 0
     bad = ctypes.c_void_p(16)
     c = sa.CoarseC(16, 16, 16, 16, 16)
     cref = ctypes.byref(c)
@@ -198,3 +199,22 @@ def test_fine_stage_layout_and_static_plan_validate_on_the_host(lib):
     assert lib.sa_plan_static(bad, bad, None, None, ctypes.byref(huge), bad, bad, None) == 5
     assert lib.sa_get_device_status(None, None) == 1
     assert lib.sa_last_launch_count() == 0
+
+
+def test_cta_clocks_validate_on_the_host(lib):
+    """sa_get_cta_clocks rejects bad arguments before touching the device, and forward and
+    backward workspaces carry room for the records (three kernels x 1024 CTAs x 32 bytes)."""
+    p = sa.make_params(1, 2, 64, (8, 8, 8), 2, 0.9)
+    rec = 3 * 1024 * 32
+    assert sa.workspace_size(p, sa.OP_FORWARD) >= 256 + rec
+    assert sa.workspace_size(p, sa.OP_BACKWARD) >= 256 + rec
+    out = (ctypes.c_ulonglong * 16)()
+    n = ctypes.c_int(-1)
+    fake = ctypes.c_void_p(16)
+    for ws, size, kernel, o, np_ in ((None, 10 ** 6, 0, out, ctypes.byref(n)),      # null workspace
+                                     (fake, 10 ** 6, 3, out, ctypes.byref(n)),      # kernel outside 0..2
+                                     (fake, 10 ** 6, -1, out, ctypes.byref(n)),
+                                     (fake, 256 + rec - 1, 0, out, ctypes.byref(n)),  # too small for the records
+                                     (fake, 10 ** 6, 0, None, ctypes.byref(n)),     # null output
+                                     (fake, 10 ** 6, 0, out, None)):                # null count
+        assert lib.sa_get_cta_clocks(ws, size, kernel, o, 4, np_, None) == 1

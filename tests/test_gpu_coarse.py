@@ -114,9 +114,11 @@ def test_gated_forward_backward(case):
 def test_zero_gate_reproduces_the_fine_stage():
     """G = 0 (VSA's zero-initialised coarse gate): the gated output is the fine output bit
     for bit; the gradients equal sa_backward's up to the order of Delta's sum.  dS enters
-    the tensor-core products as a bf16 hi + lo pair (about 16 significant bits), so a
-    last-bit change in Delta can move a gradient by about 2^-16 of its magnitude (O(1) here):
-    the bound is 1e-4 (measured 1.3e-5)."""
+    the tensor-core products as one fp16 value (11 significant bits) when every operand fits
+    fp16, as here, else as a bf16 hi + lo pair (about 16 bits); both calls take the same path.
+    A last-bit change in Delta can flip the rounding of dS, moving a gradient by about 2^-11
+    of its magnitude: the bound is 2^-9 of the largest gradient (measured 4.3e-4 on O(1)
+    gradients)."""
     cfg = synth.small_config(*SMALL["b2h3_d64"])
     x, p, t = gpu_inputs(cfg)
     idx, cnt, co = sa.plan_coarse(t["q"], t["k"], t["v"], p)
@@ -130,7 +132,7 @@ def test_zero_gate_reproduces_the_fine_stage():
     fq, fk, fv = sa.backward(t["q"], t["k"], t["v"], out_f, lse_f, t["do"], idx, cnt, p, out_f32=o32_f)
     torch.cuda.synchronize()
     for a, b in ((gq, fq), (gk, fk), (gv, fv)):
-        assert float((a - b).abs().max()) < 1e-4
+        assert float((a - b).abs().max()) <= 2.0 ** -9 * max(1.0, float(b.abs().max()))
     # dG = <dO, Oc^> still flows with G = 0
     lay = O.cube_layout(cfg.lat)
     q, k, v, do = (oracle_head(x, n, 1, 2, lay) for n in ("q", "k", "v", "do"))

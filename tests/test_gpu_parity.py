@@ -134,6 +134,41 @@ def test_backward_small(D, lat, k, pp):
     _bwd_case(synth.small_config("b", 1, 2, D, lat, k, pp))
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_fp16_and_bf16_operand_paths(D):
+    """The backward multiplies P and dS as single fp16 values when Q, K, V and dO all fit fp16
+    and the bound |dS| <= 2 D max|dO| max|V| stays within 2^15, else as bf16 hi + lo pairs (the
+    forward with the fp32 output likewise takes P in fp16 when V fits); the choice is made on
+    the device for each call.  (a) dO scaled by 2^12 (exact in bf16, still inside fp16) breaks
+    the dS bound: the gradients, scaled back, must still match the oracle.  (b) one padding
+    slot of V set to 2^17 (outside fp16; padding keys never take part) forces the bf16 path in
+    both forward and backward with results inside the same bounds."""
+    cfg = synth.small_config("bp", 1, 2, D, (5, 8, 12), 3, 0.9)
+    x, p, t, idx, cnt, out, lse, out32, trs = _fwd_case(cfg)
+    lay = O.cube_layout(cfg.lat)
+    refs = {hh: O.attention_backward_head(*(oracle_head(x, n, 0, hh, lay) for n in ("q", "k", "v", "do")),
+                                          trs[(0, hh)], lay.valid) for hh in range(p.H)}
+    s = 2.0 ** 12
+    assert float(t["do"].abs().max()) * s < 65504.0
+    ga = sa.backward(t["q"], t["k"], t["v"], out, lse, t["do"] * s, idx, cnt, p, out_f32=out32)
+    pad = int(np.flatnonzero(~lay.valid)[0])
+    v_pad = t["v"].clone()
+    v_pad[0, :, pad, 0] = 2.0 ** 17
+    out_b, lse_b, o32_b = sa.forward(t["q"], t["k"], v_pad, idx, cnt, p, with_f32=True)
+    gb = sa.backward(t["q"], t["k"], v_pad, out_b, lse_b, t["do"], idx, cnt, p, out_f32=o32_b)
+    torch.cuda.synchronize()
+    for hh in range(p.H):
+        o_ref, _ = O.attention_forward_head(*(oracle_head(x, n, 0, hh, lay) for n in ("q", "k", "v")),
+                                            trs[(0, hh)], lay.valid)
+        assert_close(f"out (V out of fp16 range) h{hh}", out_b[0, hh].float().cpu().numpy()[lay.valid],
+                     o_ref[lay.valid])
+        for name, g_a, g_b, ref in zip(("dq", "dk", "dv"), ga, gb, refs[hh]):
+            assert_close(f"{name} (dO x 2^12) h{hh}", g_a[0, hh].cpu().numpy() / s, ref)
+            b_ = g_b[0, hh].cpu().numpy()
+            assert_close(f"{name} (V out of fp16 range) h{hh}", b_, ref)
+            assert np.all(b_[~lay.valid] == 0)
+
+
 def test_end_to_end_with_gpu_lists():
     cfg = synth.small_config("e2e", 1, 4, 128, (8, 16, 20), 4, 0.9)
     x, p, t, idx, cnt = _router_case(cfg, names=("q", "k", "v", "do"))

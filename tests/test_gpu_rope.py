@@ -1,8 +1,8 @@
 """sa_tile_rope / sa_untile_rope against the oracle's 3-D RoPE with the cube-major permutation
 (GPU, through the C ABI).  Both sides take the same fp32 cosine and sine tables (RoFormer's
 frequencies); the CUDA path rotates in fp32 and rounds to the element type, so bf16 outputs
-are compared within half a bf16 ulp (2^-9 relative) plus the fp32 rotation's error, fp32
-outputs within 1e-6 relative."""
+are compared within half a bf16 ulp (at most 2^-8 of the value, just above a power of two)
+plus the fp32 rotation's error, fp32 outputs within 1e-6 relative."""
 import numpy as np
 import pytest
 import torch
@@ -35,7 +35,7 @@ def test_tile_rope_matches_oracle(lat, D, sec):
     cs32, sn32 = torch.from_numpy(cos).float(), torch.from_numpy(sin).float()
     p = sa.make_params(B, H, D, lat, 1, 0.5)
     cs_d, sn_d = cs32.cuda(), sn32.cuda()
-    for dtype, rel in ((torch.bfloat16, 2.0 ** -9 + 2.0 ** -20), (torch.float32, 1e-6)):
+    for dtype, rel in ((torch.bfloat16, 2.0 ** -8 + 2.0 ** -20), (torch.float32, 1e-6)):
         x = x32.to(dtype)
         y = sa.tile_rope(x.cuda(), p, sec, cs_d, sn_d)
         torch.cuda.synchronize()
