@@ -787,7 +787,7 @@ def traffic_for(kernel: str, ntiles: int):
 # What decides the forward kernel's DRAM traffic: its own source and device headers, and in
 # the C ABI the tensor-map encoding, the argument setup and the forward entry point.
 FWD_SOURCES = ("attn_fwd.cu", "attn_common.cuh", "geometry.cuh", "ptx.cuh")
-FWD_ABI_FUNCTIONS = ("bool make_map(", "sa::AttnArgs base_args(", "sa_status sa_forward(")
+FWD_ABI_FUNCTIONS = ("bool make_map(", "sa::AttnArgs base_args(", "sa_status forward_impl(", "sa_status sa_forward(")
 
 
 def source_sha() -> str:

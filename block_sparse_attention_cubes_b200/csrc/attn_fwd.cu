@@ -9,19 +9,23 @@
 // one work item is a pair of adjacent query cubes (128 query rows) walking the union of
 // their two KV lists, two key tiles (128 keys) per step:
 //     S[128 q x 128 keys]  = Q2 . [K_t0; K_t1]^T        (SS, M=128, N=128, K=D)
-//     O[128 q x D]        += P . [V_t0; V_t1]          (TS: P read from TMEM, N=128)
-// P overwrites S in TMEM (bf16 pairs), so it never goes through shared memory.  A tile that
-// only one cube of the pair selected is masked for the other cube's rows (its products are
-// spent, its exponentials are skipped).  Persistent CTAs walk the pairs round-robin.
+//     O_g[128 q x D]      += P_g . V_tg   (g = 0, 1)   (TS: P_g read from TMEM, N=128, K=64)
+// P_g overwrites group g's S columns in TMEM (fp16 or bf16 pairs), so it never goes through
+// shared memory.  A tile that only one cube of the pair selected is masked for the other
+// cube's rows (its products are spent, its exponentials are skipped).  Persistent CTAs take
+// the pairs in order from a shared counter.
 // Warp roles (320 threads):
 //   warp 0      TMA producers: lane 0 loads Q2 and K tile pairs (3-stage ring, released when
 //               S is done), lane 1 loads V tile pairs (2-stage ring, released after PV)
 //   warp 1      TMEM owner and MMA warp: the whole warp runs the issue loop and one elected
 //               lane issues every tcgen05.mma / commit
 //   warps 2-9   two groups of 128 threads; thread r of group g owns query row r and the 64
-//               key columns of tile t_g.  The two halves' row maxima are exchanged once per
-//               step through shared memory; the running maximum is raised (and that row of O
-//               rescaled in TMEM) only when a score exceeds it by more than 2^15.
+//               key columns of tile t_g, with its own running maximum, sum and accumulator
+//               O_g (split-key online softmax), so the groups never wait on each other
+//               within a pair; the running maximum is raised (and that row of O_g rescaled in
+//               TMEM) only when a score exceeds it by more than 2^15.  At the end of a pair
+//               the two partial results of each row are combined once:
+//               O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)).
 #include <type_traits>
 #include <cmath>
 
@@ -42,16 +46,18 @@ constexpr uint32_t OFF_BAR = OFF_V + VST * 32768;
 constexpr uint32_t OFF_SLOT = OFF_BAR + 256;
 constexpr uint32_t OFF_ABORT = OFF_BAR + 264;
 constexpr uint32_t OFF_RING = OFF_BAR + 272;     // kItemRing item ids
-constexpr uint32_t OFF_XMAX = OFF_BAR + 512;     // [2 step parities][2 groups][128 rows] float
-constexpr uint32_t OFF_XL = OFF_XMAX + 2048;     // [2 groups][128 rows] float
+constexpr uint32_t OFF_XMAX = OFF_BAR + 512;     // [2 groups][128 rows] float: running maxima at the item's end
+constexpr uint32_t OFF_XL = OFF_XMAX + 1024;     // [2 groups][128 rows] float: partial sums
 constexpr uint32_t SMEM_BYTES = OFF_XL + 1024 + 1024;
-constexpr uint32_t TMEM_COLS = 512;  // S/P[b] at 128b (b = 0,1), O[ob] at 256 + 128ob
-// P-full is one barrier per S buffer: the softmax of step s+1 can start before the MMA thread
-// has observed P(s) (S(s+1) is issued ahead of PV(s)), so a single barrier could complete two
-// phases unobserved.  The softmax of step s+2 needs S(s+2), issued only after PV(s).
+// S/P[b] at 128b (b = 0,1): group g's 64 key columns at 128b + 64g, its P over them; O_g at 256 + 128g
+constexpr uint32_t TMEM_COLS = 512;
+// P-full is one barrier per (S buffer, group): the softmax of step s+1 can start before the MMA
+// thread has observed P(s) (S(s+1) is issued ahead of PV(s)), so a single barrier per group
+// could complete two phases unobserved.  The softmax of step s+2 needs S(s+2), issued only
+// after PV(s).  PV-done is one barrier per group (its rescales wait for its previous PV).
 enum {
-  B_QF = 0, B_QE = 1, B_KF = 2, B_KE = 5, B_VF = 8, B_VE = 10, B_SF = 12, B_PF = 14, B_PFREE = 16, B_OR = 17,
-  B_OFREE = 19, B_FIN = 21, B_IF = 22, B_IE = 26, NBAR = 30
+  B_QF = 0, B_QE = 1, B_KF = 2, B_KE = 5, B_VF = 8, B_VE = 10, B_SF = 12, B_PF = 14, B_PFREE = 18, B_OR = 20,
+  B_OFREE = 21, B_FIN = 22, B_IF = 23, B_IE = 27, NBAR = 31
 };
 }  // namespace fwd
 
@@ -85,8 +91,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int b = 0; b < NBAR; ++b) {
       uint32_t cnt = 1;
-      if (b == B_PF || b == B_PF + 1) cnt = 256;
-      if (b == B_OFREE || b == B_OFREE + 1) cnt = 8;
+      if (b >= B_PF && b < B_PF + 4) cnt = 128;
+      if (b == B_OFREE) cnt = 8;
       if (b >= B_IE && b < B_IE + kItemRing) cnt = kRingReaders;
       mbar_init(&bars[b], cnt);
     }
@@ -224,39 +230,50 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         const int it = ring_read_warp(ring, n, a, 27, ok);
         if (it < 0) break;
         const int nsteps = (a.u_cnt[it] + 1) >> 1;
-        const int ob = n & 1;
         if (!mbar_wait_warp(&bars[B_QF], n & 1, a.st, a.timeout_ns, 22)) break;
         for (int s = 0; ok && s < nsteps && s < 2; ++s) ok = issue_s();
-        if (ok && n >= 2) ok = mbar_wait_warp(&bars[B_OFREE + ob], ((n >> 1) + 1) & 1, a.st, a.timeout_ns, 23);
+        // O_0 and O_1 of the previous pair must have been read out before this pair's first PV
+        if (ok && n >= 1) ok = mbar_wait_warp(&bars[B_OFREE], (n - 1) & 1, a.st, a.timeout_ns, 23);
         for (int s = 0; ok && s < nsteps; ++s) {
           const uint32_t vs = gs_o % VST, pb = gs_o & 1;
-          ok = mbar_wait_warp(&bars[B_PF + pb], (gs_o >> 1) & 1, a.st, a.timeout_ns, 24) &&
-               mbar_wait_warp(&bars[B_VF + vs], (gs_o / VST) & 1, a.st, a.timeout_ns, 25);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t vst = sbase + OFF_V + vs * 32768;
-          const uint32_t o_acc = tmem + 256 + ob * 128, p_col = tmem + pb * 128;
-          if (elect_one()) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // 8 k-steps over P (or P_hi) ...
-              umma_f16_ts(o_acc, p_col + kk * 8, sw128_desc(vst + kk * 2048, 16384, 1024), idesc_o,
-                          (s > 0 || kk > 0) ? 1u : 0u);
-            if (split_pv) {
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk)  // ... then 8 over P_lo
-                umma_f16_ts(o_acc, p_col + 64 + kk * 8, sw128_desc(vst + kk * 2048, 16384, 1024), idesc_o, 1u);
-            }
-            umma_commit(&bars[B_VE + vs]);
-            umma_commit(&bars[B_PFREE]);
+          if (!mbar_wait_warp(&bars[B_VF + vs], (gs_o / VST) & 1, a.st, a.timeout_ns, 25)) {
+            ok = false;
+            break;
           }
-          __syncwarp();
+          const uint32_t vst = sbase + OFF_V + vs * 32768;
+#pragma unroll
+          for (int gq = 0; gq < 2; ++gq) {
+            // O_g += P_g V_g as soon as group g's P is written: keys 64g.. of the step, K = 64
+            if (!mbar_wait_warp(&bars[B_PF + 2 * pb + gq], (gs_o >> 1) & 1, a.st, a.timeout_ns, 24)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t o_acc = tmem + 256 + gq * 128, p_col = tmem + pb * 128 + gq * 64;
+            if (elect_one()) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)  // 4 k-steps over P (or P_hi) ...
+                umma_f16_ts(o_acc, p_col + kk * 8, sw128_desc(vst + (4 * gq + kk) * 2048, 16384, 1024), idesc_o,
+                            (s > 0 || kk > 0) ? 1u : 0u);
+              if (split_pv) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)  // ... then 4 over P_lo
+                  umma_f16_ts(o_acc, p_col + 32 + kk * 8, sw128_desc(vst + (4 * gq + kk) * 2048, 16384, 1024),
+                              idesc_o, 1u);
+              }
+              umma_commit(&bars[B_PFREE + gq]);
+              if (gq == 1) umma_commit(&bars[B_VE + vs]);
+            }
+            __syncwarp();
+          }
+          if (!ok) break;
           ++gs_o;
           if (s + 2 < nsteps) ok = issue_s();
         }
         if (!ok) break;
         if (elect_one()) {
-          umma_commit(&bars[B_QE]);       // every product reading Q2 has been issued
-          umma_commit(&bars[B_OR + ob]);  // O of this pair is final once these complete
+          umma_commit(&bars[B_QE]);  // every product reading Q2 has been issued
+          umma_commit(&bars[B_OR]);  // O_0 and O_1 of this pair are final once these complete
         }
         __syncwarp();
       }
@@ -283,7 +300,6 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       const int nu = a.u_cnt[it];
       const int32_t* ul = a.u_list + static_cast<size_t>(it) * ucap;
       const int nsteps = (nu + 1) >> 1;
-      const int ob = n & 1;
       float qs = 1.0f;
       if (a.q_scale && row_exists) qs = a.q_scale[static_cast<size_t>(bh) * g.T + icube];
       float m_run = kNegBig, l_part = 0.0f;
@@ -321,16 +337,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], x[c]);
           pmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
         }
-        // exchange the two halves' row maxima (double-buffered by step parity); the barrier
-        // also orders every S read of this step before the P writes below
-        float* xm = xmax + (gs & 1) * 256;
-        xm[grp * 128 + r] = pmax;
-        named_bar_sync(1, 256);
-        if (*sm_abort) {
-          ok = false;
-          break;
-        }
-        const float rmax = fmaxf(pmax, xm[(grp ^ 1) * 128 + r]);
+        // each group keeps its own running maximum, sum and O_g (combined once per pair at the
+        // end), so the groups never wait on each other within a pair; P_g overwrites the
+        // group's own S columns
+        const float rmax = pmax;
         bool rescale = false;
         float alpha = 1.0f;
         if (rmax > m_run + kTau) {
@@ -340,21 +350,19 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           rescale = s > 0;
         }
         if (__any_sync(0xffffffffu, rescale)) {
-          // O is read-modified here: the previous PV product must have finished
-          if (!mbar_wait(&bars[B_PFREE], (gs - 1) & 1, a.st, a.timeout_ns, 32)) *sm_abort = 1;
+          // O_g is read-modified here: the group's previous PV product must have finished
+          if (!mbar_wait(&bars[B_PFREE + grp], (gs - 1) & 1, a.st, a.timeout_ns, 32)) *sm_abort = 1;
           tc_fence_after();
-          uint32_t o0[32], o1[32];
-          const uint32_t oc = t_lane + 256 + ob * 128 + grp * 64;
-          tmem_ld32(oc, o0);
-          tmem_ld32(oc + 32, o1);
-          tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            o0[c] = __float_as_uint(__uint_as_float(o0[c]) * alpha);
-            o1[c] = __float_as_uint(__uint_as_float(o1[c]) * alpha);
+          for (int q4 = 0; q4 < 4; ++q4) {  // the row's 128 accumulator columns, 32 at a time
+            uint32_t o0[32];
+            const uint32_t oc = t_lane + 256 + grp * 128 + q4 * 32;
+            tmem_ld32(oc, o0);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o0[c] = __float_as_uint(__uint_as_float(o0[c]) * alpha);
+            tmem_st32(oc, o0);
           }
-          tmem_st32(oc, o0);
-          tmem_st32(oc + 32, o1);
           tmem_st_wait();
         }
         // one body per P format, each with its own registers: 0 = bf16, 1 = bf16 hi + lo (the fp32
@@ -394,8 +402,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
               for (int c = 0; c < 32; ++c) pl[c] = 0u;
             }
           }
-          tmem_st32(t_lane + b * 128 + grp * 32, ph);
-          if constexpr (M == 1) tmem_st32(t_lane + b * 128 + 64 + grp * 32, pl);
+          tmem_st32(t_lane + b * 128 + grp * 64, ph);
+          if constexpr (M == 1) tmem_st32(t_lane + b * 128 + grp * 64 + 32, pl);
         };
         if (use16)
           emit_p(std::integral_constant<int, 2>{});
@@ -407,62 +415,72 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         km = a.cube_mask[e >> 2];
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bars[B_PF + b]);
+        mbar_arrive(&bars[B_PF + 2 * b + grp]);
       }
-      if (!ok) break;
       // -------------------------------------------------------------- epilogue
+      // the two groups' partial results of each row: O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / l
+      xmax[grp * 128 + r] = m_run;
       xl[grp * 128 + r] = l_part;
       named_bar_sync(1, 256);
       if (*sm_abort) break;
-      const float l = l_part + xl[(grp ^ 1) * 128 + r];
+      const float m_oth = xmax[(grp ^ 1) * 128 + r];
+      const float m_all = fmaxf(m_run, m_oth);
+      const float a_self = ex2_approx(m_run - m_all), a_oth = ex2_approx(m_oth - m_all);
+      const float l = l_part * a_self + xl[(grp ^ 1) * 128 + r] * a_oth;
       const bool has = nsteps > 0 && l > 0.0f;
       const float linv = (row_valid && has) ? 1.0f / l : 0.0f;
       const size_t qrow = static_cast<size_t>(bh) * g.Npad + static_cast<size_t>(icube) * 64 + (r & 63);
       if (grp == 0 && row_exists)
-        a.lse[qrow] = row_valid ? (has ? (m_run + log2f(l)) * 0.69314718055994531f : -INFINITY) : 0.0f;
-      float o[64];
-      if (!mbar_wait(&bars[B_OR + ob], (n >> 1) & 1, a.st, a.timeout_ns, 33)) *sm_abort = 1;  // every item
-      if (nsteps > 0) {
-        tc_fence_after();
-        uint32_t o0[32], o1[32];
-        tmem_ld32(t_lane + 256 + ob * 128 + grp * 64, o0);
-        tmem_ld32(t_lane + 256 + ob * 128 + grp * 64 + 32, o1);
-        tmem_ld_wait();
+        a.lse[qrow] = row_valid ? (has ? (m_all + log2f(l)) * 0.69314718055994531f : -INFINITY) : 0.0f;
+      if (!mbar_wait(&bars[B_OR], n & 1, a.st, a.timeout_ns, 33)) *sm_abort = 1;  // every item
+      tc_fence_after();
+      // output columns 64grp + 32h.. from O_0 (TMEM 256 + 64grp) and O_1 (384 + 64grp), 32 at a time
+      const float f0 = (grp == 0 ? a_self : a_oth) * linv, f1 = (grp == 0 ? a_oth : a_self) * linv;
+      const bool writes = row_exists && grp * 64 < a.D;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          o[c] = __uint_as_float(o0[c]) * linv;
-          o[c + 32] = __uint_as_float(o1[c]) * linv;
+      for (int h = 0; h < 2; ++h) {
+        float o[32];
+        if (nsteps > 0) {
+          uint32_t u0[32], u1[32];
+          tmem_ld32(t_lane + 256 + grp * 64 + h * 32, u0);
+          tmem_ld32(t_lane + 384 + grp * 64 + h * 32, u1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = fmaf(__uint_as_float(u0[c]), f0, __uint_as_float(u1[c]) * f1);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0.0f;
         }
-      } else {
+        if (h == 1) {  // both accumulators have been read: the next pair's PV may overwrite them
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[B_OFREE]);
+        }
+        if (writes) {
+          const int col = grp * 64 + h * 32;
+          if (a.gate && row_valid) {  // the gated combination, with the coarse branch's row of this cube
+            const float gv = a.gate[qrow];
+            const float4* ocp =
+                reinterpret_cast<const float4*>(a.oc + (static_cast<size_t>(bh) * g.T + icube) * a.D + col);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) o[c] = 0.0f;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_OFREE + ob]);
-      if (row_exists && grp * 64 < a.D) {
-        if (a.gate && row_valid) {  // the gated combination, with the coarse branch's row of this cube
-          const float gv = a.gate[qrow];
-          const float4* ocp =
-              reinterpret_cast<const float4*>(a.oc + (static_cast<size_t>(bh) * g.T + icube) * a.D + grp * 64);
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float4 t = __ldg(ocp + c);
-            o[4 * c] = fmaf(gv, t.x, o[4 * c]);
-            o[4 * c + 1] = fmaf(gv, t.y, o[4 * c + 1]);
-            o[4 * c + 2] = fmaf(gv, t.z, o[4 * c + 2]);
-            o[4 * c + 3] = fmaf(gv, t.w, o[4 * c + 3]);
+            for (int c = 0; c < 8; ++c) {
+              const float4 t = __ldg(ocp + c);
+              o[4 * c] = fmaf(gv, t.x, o[4 * c]);
+              o[4 * c + 1] = fmaf(gv, t.y, o[4 * c + 1]);
+              o[4 * c + 2] = fmaf(gv, t.z, o[4 * c + 2]);
+              o[4 * c + 3] = fmaf(gv, t.w, o[4 * c + 3]);
+            }
           }
-        }
-        uint4* dst = reinterpret_cast<uint4*>(a.out + qrow * a.D + grp * 64);
+          uint4* dst = reinterpret_cast<uint4*>(a.out + qrow * a.D + col);
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          dst[c] = make_uint4(pack_bf16x2(o[8 * c], o[8 * c + 1]), pack_bf16x2(o[8 * c + 2], o[8 * c + 3]),
-                              pack_bf16x2(o[8 * c + 4], o[8 * c + 5]), pack_bf16x2(o[8 * c + 6], o[8 * c + 7]));
-        if (a.out_f32) {
-          float4* df = reinterpret_cast<float4*>(a.out_f32 + qrow * a.D + grp * 64);
+          for (int c = 0; c < 4; ++c)
+            dst[c] = make_uint4(pack_bf16x2(o[8 * c], o[8 * c + 1]), pack_bf16x2(o[8 * c + 2], o[8 * c + 3]),
+                                pack_bf16x2(o[8 * c + 4], o[8 * c + 5]), pack_bf16x2(o[8 * c + 6], o[8 * c + 7]));
+          if (a.out_f32) {
+            float4* df = reinterpret_cast<float4*>(a.out_f32 + qrow * a.D + col);
 #pragma unroll
-          for (int c = 0; c < 16; ++c) df[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+            for (int c = 0; c < 8; ++c) df[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          }
         }
       }
     }

@@ -41,6 +41,10 @@ namespace fpl {
 constexpr int kConsumers = 8;
 constexpr int kThreads = (kConsumers + 1) * 32;
 constexpr int kStages = 12;
+// A consumer's next stage is kConsumers stages past its last one; a parity wait tells apart only
+// a barrier's current phase and the one before, so the previous fill of that stage must have
+// landed already: kStages >= kConsumers guarantees it.
+static_assert(kStages >= kConsumers, "a full-barrier wait could pass on a fill two phases old");
 constexpr uint32_t kStageBytes = 16384;  // one cube of 64 rows x 256 bytes (bf16, D = 128)
 constexpr uint32_t OFF_BAR = kStages * kStageBytes;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 2 * kStages * 8 + 1024;

@@ -176,10 +176,13 @@ __device__ __forceinline__ uint64_t mass_fx(double x, double m) {
 // by an 8-bit radix descent over the 64-bit order keys in which every bucket carries
 // its count and its exact fixed-point mass.  Then writes the kept ids in ascending order.
 // `s` is the row's T scores, `cnt` / `mass` a 256-entry scratch histogram of this warp; the
-// kept ids go to `out` (at most cap) and their number to *count.  Called by a whole warp.
+// kept ids go to `out` (at most cap) and their number to *count.  `mrow`, when given, holds
+// every score's mass mass_fx(s_j, max) already (else each pass computes the masses it needs).
+// Called by a whole warp.
 __device__ void select_row_fp64(const double* __restrict__ s, int T, int top_k, float top_p, int cap,
                                 int32_t* __restrict__ out, int32_t* __restrict__ count, DevStatus* st,
-                                uint32_t* cnt, unsigned long long* mass) {
+                                uint32_t* cnt, unsigned long long* mass,
+                                const unsigned long long* __restrict__ mrow = nullptr) {
   const int lane = threadIdx.x & 31;
 
   double m = -DBL_MAX;
@@ -226,7 +229,7 @@ __device__ void select_row_fp64(const double* __restrict__ s, int T, int top_k, 
             if (shift == 56 || (kj >> (shift + 8)) == (prefix >> (shift + 8))) {
               part = true;
               d = static_cast<int>((kj >> shift) & 255u);
-              mj = static_cast<unsigned long long>(mass_fx(x, m));
+              mj = mrow ? mrow[j] : static_cast<unsigned long long>(mass_fx(x, m));
             }
           }
           const uint32_t act = __ballot_sync(0xffffffffu, part);
@@ -317,7 +320,7 @@ __device__ void select_row_fp64(const double* __restrict__ s, int T, int top_k, 
               const double x = xs[u];
               kj = desc_key(x);
               cand = (kj & mask) == prefix;
-              if (cand) mj = mass_fx(x, m);
+              if (cand) mj = mrow ? mrow[j] : mass_fx(x, m);
             }
             // candidates share one key when shift == 0; a single candidate otherwise
             const uint32_t cb = __ballot_sync(0xffffffffu, cand);
@@ -426,16 +429,21 @@ struct RowMeta {
 
 
 // Pooling for the tensor-core router.  Persistent CTAs, one per SM; items are (head, cube, Q or
-// K), dealt round-robin so the CTAs stream neighbouring cubes together.  Warp 16 (one lane)
+// K), dealt round-robin so the CTAs stream neighbouring cubes together.  Warp 12 (one lane)
 // brings each item's rows (up to the cube's last valid slot) into a 24-stage shared-memory ring
-// with 1-D bulk copies, half a cube (32 slots) per stage; warps 0-15 take the items in turn,
+// with 1-D bulk copies, half a cube (32 slots) per stage; warps 0-11 take the items in turn,
 // each lane summing D/32 columns over the cube's valid rows in fp64 and releasing each half as
 // soon as it is summed, and write the mean, its limbs, the row's binary exponent and (Q) its
-// 1-norm.  Half-cube stages keep 16 cubes in progress and 8 halves in flight per SM.
+// 1-norm.  Half-cube stages keep 12 cubes in progress per SM with halves still in flight.
 namespace rpl {
-constexpr int kConsumers = 16;
+constexpr int kConsumers = 12;
 constexpr int kThreads = (kConsumers + 1) * 32;
 constexpr int kStages = 24;
+// A consumer's next stage is 2 * kConsumers stages past its last one.  A parity wait tells
+// apart only the current phase of a barrier and the one before it, so the previous fill of
+// that stage must already have landed: kStages >= 2 * kConsumers - 1 guarantees it (the
+// consumer has seen the producer pass its last stage).
+static_assert(kStages >= 2 * kConsumers - 1, "a full-barrier wait could pass on a fill two phases old");
 constexpr uint32_t kStageBytes = 8192;  // half a cube: 32 rows x 256 bytes (bf16, D = 128)
 constexpr uint32_t OFF_BAR = kStages * kStageBytes;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 2 * kStages * 8 + 1024;
@@ -1166,15 +1174,19 @@ __global__ void __launch_bounds__(256, 4) select_keys_kernel(const int* __restri
 // The fp64 path for the rows the key selection queued: one CTA per row (grid-stride over the
 // queue).  Its four warps compute the row's scores Qbar_i . Kbar_j * scale in fp64 into shared
 // memory, lanes splitting each dot product over D (coalesced reads of every Kbar row, then a
-// shuffle reduction), and warp 0 selects from there as select_kernel does.
+// shuffle reduction), then every score's fixed-point mass once (the selection's passes would
+// otherwise evaluate the fp64 exponential again in each pass), and warp 0 selects from there
+// as select_kernel does.
 __global__ void __launch_bounds__(128) router_fallback_kernel(const double* __restrict__ qbar,
                                                               const double* __restrict__ kbar, int D, int T,
                                                               double scale, const int* __restrict__ flist, int top_k,
                                                               float top_p, int cap, int32_t* __restrict__ kv_index,
                                                               int32_t* __restrict__ kv_count, DevStatus* st) {
-  extern __shared__ double srow[];  // [T] scores
+  extern __shared__ double srow[];  // [T] scores, then [T] masses
   __shared__ uint32_t cnt_s[256];
   __shared__ unsigned long long mass_s[256];
+  __shared__ double wmax[4];
+  unsigned long long* mrow = reinterpret_cast<unsigned long long*>(srow + T);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nf = static_cast<int>(*reinterpret_cast<const volatile unsigned*>(&st->router_fallback));
   const int per = D >> 5;  // doubles per lane (2 or 4)
@@ -1205,9 +1217,18 @@ __global__ void __launch_bounds__(128) router_fallback_kernel(const double* __re
       }
     }
     __syncthreads();
+    double mx = -DBL_MAX;
+    for (int j = threadIdx.x; j < T; j += 128) mx = fmax(mx, srow[j]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) wmax[warp] = mx;
+    __syncthreads();
+    mx = fmax(fmax(wmax[0], wmax[1]), fmax(wmax[2], wmax[3]));
+    for (int j = threadIdx.x; j < T; j += 128) mrow[j] = mass_fx(srow[j], mx);
+    __syncthreads();
     if (warp == 0)
       select_row_fp64(srow, T, top_k, top_p, cap, kv_index + static_cast<size_t>(row) * cap, kv_count + row, st,
-                      cnt_s, mass_s);
+                      cnt_s, mass_s, mrow);
     __syncthreads();
   }
 }
@@ -1263,8 +1284,8 @@ cudaError_t launch_plan_fast(const void* q, const void* k, const float* q_scale,
                                          rsc::SMEM_BYTES);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(score_keys_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsc::SMEM_BYTES);
-    if (e == cudaSuccess)  // one fp64 score row of up to 8192 cubes
-      e = cudaFuncSetAttribute(router_fallback_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 8192 * 8);
+    if (e == cudaSuccess)  // one fp64 score row and its masses, up to 8192 cubes
+      e = cudaFuncSetAttribute(router_fallback_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 8192 * 16);
     for (auto fn : {pool_limbs_kernel<2, 4>, pool_limbs_kernel<2, 2>, pool_limbs_kernel<1, 4>, pool_limbs_kernel<1, 2>})
       if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, rpl::SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -1333,7 +1354,7 @@ cudaError_t launch_plan_fast(const void* q, const void* k, const float* q_scale,
   select_keys_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(
         w.keys, w.Tk, w.rkmax, w.rkmin, reinterpret_cast<const RowMeta*>(w.meta), rows, g.T, top_k, top_p, cap,
         kv_index, kv_count, w.flist, st, debug, timeout_ns);
-  router_fallback_kernel<<<plan_fallback_ctas(), 128, static_cast<size_t>(g.T) * sizeof(double), stream>>>(
+  router_fallback_kernel<<<plan_fallback_ctas(), 128, static_cast<size_t>(g.T) * 16, stream>>>(
       w.qbar, w.kbar, D, g.T, scale, w.flist, top_k, top_p, cap, kv_index, kv_count, st);
   *launches = 5;
   return cudaGetLastError();
