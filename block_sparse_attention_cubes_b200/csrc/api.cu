@@ -100,7 +100,7 @@ WsLayout ws_layout(const sa_params* p, const Geom& g, int op) {
   }
   if (op == SA_OP_PLAN_COARSE || op == SA_OP_BACKWARD_GATED) {
     // the plain layout, then the coarse branch's buffers
-    w = ws_layout(p, g, op == SA_OP_PLAN_COARSE ? kOpPlanFp64 : SA_OP_BACKWARD);
+    w = ws_layout(p, g, op == SA_OP_PLAN_COARSE ? SA_OP_PLAN : SA_OP_BACKWARD);
     const size_t TT = BH * g.T * static_cast<size_t>(g.T) * sizeof(float);
     const size_t TD = BH * g.T * static_cast<size_t>(p->D) * sizeof(float);
     size_t off = w.total;
@@ -320,7 +320,7 @@ sa_status plan_check(const void* q, const void* k, const float* q_scale, const f
 // (a caller's workspace, or the fixed array of sa_plan_static); records the launch count.
 sa_status plan_on_scratch(const void* q, const void* k, const float* q_scale, const float* k_scale,
                           const sa_params* p, int32_t* kv_index, int32_t* kv_count, void* ws, size_t ws_bytes,
-                          cudaStream_t st) {
+                          cudaStream_t st, float* s32) {
   g_last_launches = 0;
   size_t need = 0;
   sa_status s = plan_check(q, k, q_scale, k_scale, p, kv_index, kv_count, &need);
@@ -348,6 +348,7 @@ sa_status plan_on_scratch(const void* q, const void* k, const float* q_scale, co
   f.flist = reinterpret_cast<int*>(wb + w.flist);
   f.rkmax = reinterpret_cast<int*>(wb + w.rkmax);
   f.rkmin = reinterpret_cast<int*>(wb + w.rkmin);
+  f.s32 = s32;
   CUtensorMap tq, tk, tkeys;
   if (!make_limb_map(&tq, f.qlimb, g.T, 4LL * BH) || !make_limb_map(&tk, f.klimb, g.T, 4LL * BH) ||
       !make_keys_map(&tkeys, f.keys, g.T, f.Tk, BH))
@@ -652,19 +653,18 @@ sa_status sa_plan_coarse(const void* q, const void* k, const void* v, const sa_p
   if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
   if (!aligned16(ws)) return SA_ERR_ALIGNMENT;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (reset_status(ws, st) != SA_OK) return SA_ERR_LAUNCH;
   uint8_t* wb = static_cast<uint8_t*>(ws);
   const int BH = p->B * p->H;
-  double* qbar = reinterpret_cast<double*>(wb + w.qbar);
-  double* kbar = reinterpret_cast<double*>(wb + w.kbar);
-  double* S = reinterpret_cast<double*>(wb + w.scores);
-  int plan_launches = 0, coarse_launches = 0;
-  if (sa::launch_plan(q, k, nullptr, nullptr, g, BH, p->D, false, softmax_scale(p), p->top_k, p->top_p,
-                      p->kv_capacity, kv_index, kv_count, qbar, kbar, S, static_cast<sa::DevStatus*>(ws), st,
-                      &plan_launches) != cudaSuccess ||
-      sa::launch_coarse_forward(v, qbar, kbar, S, reinterpret_cast<float*>(wb + w.p32), coarse_tensors(coarse), g, BH,
-                                p->D, static_cast<sa::DevStatus*>(ws), timeout_ns_of(p), st,
-                                &coarse_launches) != cudaSuccess)
+  float* P32 = reinterpret_cast<float*>(wb + w.p32);
+  // the router of sa_plan (same kernels, same lists), which also writes every scaled score in
+  // fp32 into P32; then the coarse branch from its fp64 means and those scores
+  if ((s = sa::plan_on_scratch(q, k, nullptr, nullptr, p, kv_index, kv_count, ws, ws_bytes, st, P32)) != SA_OK)
+    return s;
+  const int plan_launches = g_last_launches;
+  int coarse_launches = 0;
+  if (sa::launch_coarse_forward(v, reinterpret_cast<double*>(wb + w.qbar), reinterpret_cast<double*>(wb + w.kbar), P32,
+                                coarse_tensors(coarse), g, BH, p->D, static_cast<sa::DevStatus*>(ws), timeout_ns_of(p),
+                                st, &coarse_launches) != cudaSuccess)
     return SA_ERR_LAUNCH;
   g_last_launches = plan_launches + coarse_launches;
   return SA_OK;

@@ -519,18 +519,20 @@ int num_sms() {
   return n;
 }
 
-// bf16 -> fp16 copy of a tensor (n16 = elements / 8, one 16-byte vector per thread); any value
-// an fp16 cannot hold (|x| > 65504, or not finite) sets *bad.  Values below fp16's normal range
+// bf16 -> fp16 copy of a tensor (n16 = elements / 8 vectors of 16 bytes); any value an fp16
+// cannot hold (|x| > 65504, or not finite) sets *bad.  Values below fp16's normal range
 // become fp16 subnormals (absolute error at most 2^-25).
 // With maxbits set, the largest |x| (fp32 bits, a non-negative float orders as its bits) is
 // also recorded there.
-__global__ void __launch_bounds__(256) to_f16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+__global__ void __launch_bounds__(512) to_f16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
                                                      long long n16, unsigned int* bad, unsigned int* maxbits) {
-  const long long i = blockIdx.x * 256LL + threadIdx.x;
+  // grid-stride, four 16-byte loads in flight per thread; the range flag and the maximum are
+  // reduced over the block, so one atomic per block reaches each status word
+  __shared__ float s_mx[16];
+  __shared__ int s_out[16];
   bool out = false;
   float mx = 0.0f;
-  if (i < n16) {
-    const uint4 v = src[i];
+  auto cvt = [&](const uint4 v) -> uint4 {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t o[4];
 #pragma unroll
@@ -540,21 +542,48 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const uint4* __restrict__ s
       mx = fmaxf(mx, fmaxf(fabsf(a), fabsf(b)));
       o[u] = pack_f16x2(a, b);
     }
-    dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
-  }
-  if (__any_sync(0xffffffffu, out) && (threadIdx.x & 31) == 0) atomicOr(bad, 1u);
-  if (maxbits) {
+    return make_uint4(o[0], o[1], o[2], o[3]);
+  };
+  const long long stride = static_cast<long long>(gridDim.x) * 512;
+  long long i = static_cast<long long>(blockIdx.x) * 512 + threadIdx.x;
+  for (; i + 3 * stride < n16; i += 4 * stride) {
+    uint4 v[4];
 #pragma unroll
-    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if ((threadIdx.x & 31) == 0) atomicMax(maxbits, __float_as_uint(mx));
+    for (int u = 0; u < 4; ++u) v[u] = __ldcs(src + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) __stcs(dst + i + u * stride, cvt(v[u]));
+  }
+  for (; i < n16; i += stride) __stcs(dst + i, cvt(__ldcs(src + i)));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const bool wout = __any_sync(0xffffffffu, out);
+  if (lane == 0) {
+    s_mx[warp] = mx;
+    s_out[warp] = wout ? 1 : 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.0f;
+    int o = 0;
+    for (int w = 0; w < 16; ++w) {
+      m = fmaxf(m, s_mx[w]);
+      o |= s_out[w];
+    }
+    if (o) atomicOr(bad, 1u);
+    if (maxbits) atomicMax(maxbits, __float_as_uint(m));
   }
 }
 
 cudaError_t launch_to_f16(const void* src, void* dst, long long elems, unsigned int* bad, cudaStream_t stream,
                           unsigned int* maxbits) {
   const long long n16 = elems / 8;
-  to_f16_kernel<<<static_cast<unsigned>((n16 + 255) / 256), 256, 0, stream>>>(
-      static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16, bad, maxbits);
+  long long blocks = (n16 + 511) / 512;
+  const long long cap = 4LL * num_sms();  // persistent: a few blocks per SM stream the whole tensor
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  to_f16_kernel<<<static_cast<unsigned>(blocks), 512, 0, stream>>>(static_cast<const uint4*>(src),
+                                                                   static_cast<uint4*>(dst), n16, bad, maxbits);
   return cudaGetLastError();
 }
 

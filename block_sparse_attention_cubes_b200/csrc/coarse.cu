@@ -113,26 +113,26 @@ __global__ void __launch_bounds__(256) coarse_pool_kernel(const __nv_bfloat16* _
 }
 
 // ------------------------------------------------------------------------ softmax
-// One warp per cube row: max, sum of exp(s - max), then P = exp(s - max) / sum.  The row
-// (T doubles) is read three times; after the first pass it comes from L1/L2.
-__global__ void __launch_bounds__(256) coarse_softmax_kernel(const double* __restrict__ S, float* __restrict__ P,
-                                                             float* __restrict__ lse, long long rows, int T) {
+// One warp per cube row: max, sum of exp(s - max), then P = exp(s - max) / sum, in place over
+// the row's fp32 scores (each lane rewrites only the entries it read).  The row is read three
+// times; after the first pass it comes from L1/L2.
+__global__ void __launch_bounds__(256) coarse_softmax_kernel(float* __restrict__ SP, float* __restrict__ lse,
+                                                             long long rows, int T) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = blockIdx.x * 8LL + warp;
   if (row >= rows) return;
-  const double* s = S + row * T;
-  double m = -INFINITY;
-  for (int j = lane; j < T; j += 32) m = fmax(m, s[j]);
+  float* s = SP + row * T;
+  float m = -INFINITY;
+  for (int j = lane; j < T; j += 32) m = fmaxf(m, s[j]);
 #pragma unroll
-  for (int off = 16; off; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+  for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
   float l = 0.0f;
-  for (int j = lane; j < T; j += 32) l += expf(static_cast<float>(s[j] - m));
+  for (int j = lane; j < T; j += 32) l += expf(s[j] - m);
 #pragma unroll
   for (int off = 16; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
   const float inv = 1.0f / l;
-  float* p = P + row * T;
-  for (int j = lane; j < T; j += 32) p[j] = expf(static_cast<float>(s[j] - m)) * inv;
-  if (lane == 0) lse[row] = static_cast<float>(m) + logf(l);
+  for (int j = lane; j < T; j += 32) s[j] = expf(s[j] - m) * inv;
+  if (lane == 0) lse[row] = m + logf(l);
 }
 
 // ------------------------------------------------------------------------ products
@@ -201,41 +201,38 @@ __device__ __forceinline__ void load8(const float* row, int c0, int ncols, bool 
   }
 }
 
-// One operand slice (128 rows of the MMA's M or N by 64 k) into shared memory as hi and lo.
-// KMAJ: the source holds row r's k values contiguously (src[r * ld + k]); the slice is
-// stored K-major ([128 rows][128 B]).  Otherwise the source holds k row by k row
+// One operand slice (128 rows of the MMA's M or N by 64 k) into shared memory as hi and lo, in
+// two halves so that a caller can issue the loads of both operands before converting either:
+// gather_slice loads the thread's four 8-value chunks into registers, store_slice splits and
+// stores them.  KMAJ: the source holds row r's k values contiguously (src[r * ld + k]); the
+// slice is stored K-major ([128 rows][128 B]).  Otherwise the source holds k row by k row
 // (src[k * ld + r]) and the slice is stored MN-major ([2 halves of 64 r][64 k][128 B]).
 template <bool KMAJ>
-__device__ __forceinline__ void load_slice(const float* src, int ld, int r0, int rows, int k0, int K, bool vec,
-                                           uint32_t s_hi, uint32_t s_lo, int tid) {
+__device__ __forceinline__ void gather_slice(const float* src, int ld, int r0, int rows, int k0, int K, bool vec,
+                                             int tid, float (&x)[4][8]) {
 #pragma unroll
   for (int it = 0; it < 4; ++it) {  // 256 threads x 4 chunks of 8 values = 128 x 64
     const int u = tid + 256 * it;
-    float x[8];
-    uint32_t off;
-    if (KMAJ) {
-      const int r = u >> 3, c = u & 7;  // row r, k chunk c
-      const int gr = r0 + r;
-      if (gr < rows) {
-        load8(src + static_cast<long long>(gr) * ld, k0 + 8 * c, K, vec, x);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = 0.0f;
-      }
-      off = sw128_offset(r, c);
+    const int outer = KMAJ ? (u >> 3) : (u >> 4);           // row r (K-major) or k row (MN-major)
+    const int c0 = KMAJ ? 8 * (u & 7) : 8 * (u & 15);       // first value of the chunk in that row
+    const int g_outer = (KMAJ ? r0 : k0) + outer, lim_outer = KMAJ ? rows : K;
+    if (g_outer < lim_outer) {
+      load8(src + static_cast<long long>(g_outer) * ld, (KMAJ ? k0 : r0) + c0, KMAJ ? K : rows, vec, x[it]);
     } else {
-      const int k = u >> 4, c = u & 15;  // k row k, r chunk c (8 values)
-      const int gk = k0 + k;
-      if (gk < K) {
-        load8(src + static_cast<long long>(gk) * ld, r0 + 8 * c, rows, vec, x);
-      } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = 0.0f;
-      }
-      off = (c >> 3) * 8192u + sw128_offset(k, c & 7);
+      for (int i = 0; i < 8; ++i) x[it][i] = 0.0f;
     }
+  }
+}
+
+template <bool KMAJ>
+__device__ __forceinline__ void store_slice(const float (&x)[4][8], uint32_t s_hi, uint32_t s_lo, int tid) {
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int u = tid + 256 * it;
+    const uint32_t off = KMAJ ? sw128_offset(u >> 3, u & 7) : ((u & 15) >> 3) * 8192u + sw128_offset(u >> 4, u & 7);
     uint4 h, l;
-    split8(x, h, l);
+    split8(x[it], h, l);
     st_shared_v4(s_hi + off, h.x, h.y, h.z, h.w);
     st_shared_v4(s_lo + off, l.x, l.y, l.z, l.w);
   }
@@ -287,8 +284,11 @@ __global__ void __launch_bounds__(cmm::kThreads, 1) coarse_mma_kernel(GemmArgs p
         break;
       }
       const uint32_t sb = sbase + st * STAGE_BYTES;
-      load_slice<!TA>(A, p.lda, m0, p.M, c * BK, p.K, vec_a, sb, sb + OP_BYTES, tid);
-      load_slice<TB>(B, p.ldb, n0, p.N, c * BK, p.K, vec_b, sb + 2 * OP_BYTES, sb + 3 * OP_BYTES, tid);
+      float xa[4][8], xb[4][8];  // both operands' loads in flight before either is converted
+      gather_slice<!TA>(A, p.lda, m0, p.M, c * BK, p.K, vec_a, tid, xa);
+      gather_slice<TB>(B, p.ldb, n0, p.N, c * BK, p.K, vec_b, tid, xb);
+      store_slice<!TA>(xa, sb, sb + OP_BYTES, tid);
+      store_slice<TB>(xb, sb + 2 * OP_BYTES, sb + 3 * OP_BYTES, tid);
       fence_proxy_async_smem();  // generic-proxy stores, read next by the tensor cores
       mbar_arrive(&bars[B_FULL + st]);
     }
@@ -483,9 +483,9 @@ __global__ void __launch_bounds__(256) coarse_gate_bwd_kernel(
 }  // namespace
 
 // ------------------------------------------------------------------------ launch
-cudaError_t launch_coarse_forward(const void* v, const double* qbar64, const double* kbar64, const double* S64,
-                                  float* P32, const CoarseTensors& c, const Geom& g, int BH, int D,
-                                  DevStatus* st, unsigned long long timeout_ns, cudaStream_t stream, int* launches) {
+cudaError_t launch_coarse_forward(const void* v, const double* qbar64, const double* kbar64, float* P32,
+                                  const CoarseTensors& c, const Geom& g, int BH, int D, DevStatus* st,
+                                  unsigned long long timeout_ns, cudaStream_t stream, int* launches) {
   const long long cubes = static_cast<long long>(BH) * g.T;
   const unsigned blocks = static_cast<unsigned>((cubes + 7) / 8);
   const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
@@ -493,7 +493,7 @@ cudaError_t launch_coarse_forward(const void* v, const double* qbar64, const dou
     coarse_pool_kernel<4><<<blocks, 256, 0, stream>>>(vb, qbar64, kbar64, c.qbar, c.kbar, c.vbar, g, BH);
   else
     coarse_pool_kernel<2><<<blocks, 256, 0, stream>>>(vb, qbar64, kbar64, c.qbar, c.kbar, c.vbar, g, BH);
-  coarse_softmax_kernel<<<blocks, 256, 0, stream>>>(S64, P32, c.lse, cubes, g.T);
+  coarse_softmax_kernel<<<blocks, 256, 0, stream>>>(P32, c.lse, cubes, g.T);
   GemmArgs a{};
   a.A = P32, a.B = c.vbar, a.C = c.oc;
   a.sA = static_cast<long long>(g.T) * g.T, a.sB = static_cast<long long>(g.T) * D, a.sC = a.sB;

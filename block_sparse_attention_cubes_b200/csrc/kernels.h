@@ -16,10 +16,11 @@ sa_status plan_check(const void* q, const void* k, const float* q_scale, const f
                      const int32_t* kv_index, const int32_t* kv_count, size_t* ws_needed);
 // sa_plan on the scratch `ws` of `ws_bytes` (a caller's workspace or the library's fixed
 // array): the host checks, the workspace carving and the launches of sa_plan, and the launch
-// count that sa_last_launch_count reports (api.cu).
+// count that sa_last_launch_count reports (api.cu).  s32 (optional, [B*H*T, T] fp32) also
+// receives every scaled score.
 sa_status plan_on_scratch(const void* q, const void* k, const float* q_scale, const float* k_scale,
                           const sa_params* p, int32_t* kv_index, int32_t* kv_count, void* ws, size_t ws_bytes,
-                          cudaStream_t stream);
+                          cudaStream_t stream, float* s32 = nullptr);
 
 struct DevStatus;
 struct AttnArgs;
@@ -52,6 +53,7 @@ struct PlanFastWs {
   int* rkmin;
   int Tk;              // row stride of keys (T rounded up to 4)
   int* flist;          // [BH*T] rows left to the fp64 path
+  float* s32 = nullptr;  // optional [BH*T, T]: every scaled score in fp32 (the coarse branch reads them)
 };
 int plan_fallback_ctas();
 // Router on the tensor cores (pool + limbs, exact limb products -> keys, key selection, fp64
@@ -172,11 +174,11 @@ struct CoarseGradWs {
   float* cv;
 };
 
-// Vc pooled from v, fp32 copies of the router's fp64 Qc and Kc, Pc from the router's fp64
-// scores and Oc^ = Pc Vc (3 launches).
-cudaError_t launch_coarse_forward(const void* v, const double* qbar64, const double* kbar64, const double* S64,
-                                  float* P32, const CoarseTensors& c, const Geom& g, int BH, int D,
-                                  DevStatus* st, unsigned long long timeout_ns, cudaStream_t stream, int* launches);
+// Vc pooled from v, fp32 copies of the router's fp64 Qc and Kc, Pc from the router's fp32 scores
+// (P32 holds them on entry and Pc on return) and Oc^ = Pc Vc (3 launches).
+cudaError_t launch_coarse_forward(const void* v, const double* qbar64, const double* kbar64, float* P32,
+                                  const CoarseTensors& c, const Geom& g, int BH, int D, DevStatus* st,
+                                  unsigned long long timeout_ns, cudaStream_t stream, int* launches);
 // dG, the fine branch's Delta and -lse*log2(e), and the coarse branch's per-cube gradient
 // terms w.cq, w.ck, w.cv (6 launches).
 cudaError_t launch_coarse_backward(const void* out, const float* out_f32, const void* dout, const float* lse,

@@ -429,22 +429,22 @@ struct RowMeta {
 
 
 // Pooling for the tensor-core router.  Persistent CTAs, one per SM; items are (head, cube, Q or
-// K), dealt round-robin so the CTAs stream neighbouring cubes together.  Warp 12 (one lane)
-// brings each item's rows (up to the cube's last valid slot) into a 24-stage shared-memory ring
-// with 1-D bulk copies, half a cube (32 slots) per stage; warps 0-11 take the items in turn,
-// each lane summing D/32 columns over the cube's valid rows in fp64 and releasing each half as
-// soon as it is summed, and write the mean, its limbs, the row's binary exponent and (Q) its
-// 1-norm.  Half-cube stages keep 12 cubes in progress per SM with halves still in flight.
+// K), dealt round-robin so the CTAs stream neighbouring cubes together.  Warp 8 (one lane)
+// brings each item's rows (up to the cube's last valid slot: one contiguous range) into a
+// 12-stage shared-memory ring with 1-D bulk copies; warps 0-7 take the items in turn, each lane
+// summing D/32 columns over the cube's valid rows in fp64, and write the mean, its limbs, the
+// row's binary exponent and (Q) its 1-norm.  (Half-cube stages with 12 consumers measured
+// slower: 0.63 against 0.50 ms at 720p.)
 namespace rpl {
-constexpr int kConsumers = 12;
+constexpr int kConsumers = 8;
 constexpr int kThreads = (kConsumers + 1) * 32;
-constexpr int kStages = 24;
-// A consumer's next stage is 2 * kConsumers stages past its last one.  A parity wait tells
-// apart only the current phase of a barrier and the one before it, so the previous fill of
-// that stage must already have landed: kStages >= 2 * kConsumers - 1 guarantees it (the
-// consumer has seen the producer pass its last stage).
-static_assert(kStages >= 2 * kConsumers - 1, "a full-barrier wait could pass on a fill two phases old");
-constexpr uint32_t kStageBytes = 8192;  // half a cube: 32 rows x 256 bytes (bf16, D = 128)
+constexpr int kStages = 12;
+// A consumer's next stage is kConsumers stages past its last one.  A parity wait tells apart
+// only the current phase of a barrier and the one before it, so the previous fill of that
+// stage must already have landed: kStages >= kConsumers guarantees it (the consumer has seen
+// the producer pass its last stage).
+static_assert(kStages >= kConsumers, "a full-barrier wait could pass on a fill two phases old");
+constexpr uint32_t kStageBytes = 16384;  // one cube of 64 rows x 256 bytes (bf16, D = 128)
 constexpr uint32_t OFF_BAR = kStages * kStageBytes;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 2 * kStages * 8 + 1024;
 }  // namespace rpl
@@ -494,9 +494,9 @@ __global__ void __launch_bounds__(rpl::kThreads, 1) pool_limbs_kernel(const Pool
   if (aborted(a.st)) return;
   if (warp == kConsumers) {
     if (lane == 0) {
-      long long i = 0;  // stage sequence: item j of this CTA fills stages 2j (slots 0-31) and 2j+1 (32-63)
+      long long i = 0;  // item j of this CTA fills stage j % kStages
       bool ok = true;
-      for (long long it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+      for (long long it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++i) {
         const int which = static_cast<int>(it & 1);
         const long long cube = it >> 1;  // bh * T + c
         const int c = static_cast<int>(cube % g.T);
@@ -505,21 +505,14 @@ __global__ void __launch_bounds__(rpl::kThreads, 1) pool_limbs_kernel(const Pool
         const uint32_t nrows = static_cast<uint32_t>(16 * (vt - 1) + 4 * (vh - 1) + vw);  // through the last valid slot
         const uint8_t* src = (which ? a.k : a.q) + (static_cast<size_t>(cube / g.T) * g.Npad + static_cast<size_t>(c) * 64) *
                                                        row_bytes;
-        for (uint32_t h = 0; h < 2; ++h, ++i) {
-          const int stage = static_cast<int>(i % kStages);
-          if (i >= kStages && !mbar_wait(&empty[stage], ((i / kStages) + 1) & 1, a.st, a.timeout_ns, 131)) {
-            ok = false;
-            break;
-          }
-          const uint32_t r0 = 32 * h, r1 = nrows < r0 + 32 ? nrows : r0 + 32;
-          if (r1 > r0) {
-            const uint32_t bytes = (r1 - r0) * static_cast<uint32_t>(row_bytes);
-            mbar_arrive_expect_tx(&full[stage], bytes);
-            bulk_load(smem + stage * kStageBytes, src + r0 * row_bytes, bytes, &full[stage]);
-          } else {
-            mbar_arrive(&full[stage]);  // no valid slot in this half: an empty stage
-          }
+        const int stage = static_cast<int>(i % kStages);
+        if (i >= kStages && !mbar_wait(&empty[stage], ((i / kStages) + 1) & 1, a.st, a.timeout_ns, 131)) {
+          ok = false;
+          break;
         }
+        const uint32_t bytes = nrows * static_cast<uint32_t>(row_bytes);
+        mbar_arrive_expect_tx(&full[stage], bytes);
+        bulk_load(smem + stage * kStageBytes, src, bytes, &full[stage]);
       }
       // drain: the copies still in flight land before the CTA exits
       const long long issued = i;
@@ -542,23 +535,17 @@ __global__ void __launch_bounds__(rpl::kThreads, 1) pool_limbs_kernel(const Pool
     for (int u = 0; u < 4; ++u)
 #pragma unroll
       for (int e = 0; e < EPL; ++e) acc4[u][e] = 0.0;
-    bool ok = true;
-    for (int h = 0; h < 2; ++h) {  // the two half-cube stages: slot rows a0 in {2h, 2h + 1}
-      const long long i = 2 * j + h;
-      const int stage = static_cast<int>(i % kStages);
-      if (!mbar_wait_warp(&full[stage], (i / kStages) & 1, a.st, a.timeout_ns, 133)) {
-        ok = false;
-        break;
-      }
+    {
+      const int stage = static_cast<int>(j % kStages);
+      if (!mbar_wait_warp(&full[stage], (j / kStages) & 1, a.st, a.timeout_ns, 133)) break;
       const uint8_t* tile = smem + stage * kStageBytes + lane * EPL * ESZ;
-      const int a_end = vt < 2 * h + 2 ? vt : 2 * h + 2;
-    for (int a0 = 2 * h; a0 < a_end; ++a0)
+    for (int a0 = 0; a0 < vt; ++a0)
       for (int b0 = 0; b0 < vh; ++b0)
 #pragma unroll
         for (int d0 = 0; d0 < 4; ++d0) {
           if (d0 >= vw) break;
           double* acc = acc4[d0];
-          const uint8_t* rp = tile + ((a0 - 2 * h) * 16 + b0 * 4 + d0) * row_bytes;
+          const uint8_t* rp = tile + (a0 * 16 + b0 * 4 + d0) * row_bytes;
           if constexpr (ESZ == 2) {
             uint32_t wv[EPL / 2];
             if constexpr (EPL == 4) {
@@ -580,9 +567,8 @@ __global__ void __launch_bounds__(rpl::kThreads, 1) pool_limbs_kernel(const Pool
           }
         }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[stage]);  // the half's rows have been read
+      if (lane == 0) mbar_arrive(&empty[stage]);  // the cube's rows have been read
     }
-    if (!ok) break;
     double acc[EPL];
 #pragma unroll
     for (int e = 0; e < EPL; ++e) acc[e] = (acc4[0][e] + acc4[1][e]) + (acc4[2][e] + acc4[3][e]);
@@ -657,6 +643,7 @@ struct ScoreArgs {
   int* rkmax;       // [BH*T] largest and smallest key of each row (atomics)
   int* rkmin;
   RowMeta* meta;    // [BH*T]
+  float* s32;       // optional [BH*T, T]: the scaled scores in fp32
   DevStatus* st;
   int T, Tk, BH;    // kexp rows have Tk entries per head
   double scale;
@@ -862,6 +849,13 @@ __global__ void __launch_bounds__(rsc::kThreads, 1)
           for (int u = 0; u < 4; ++u) {
             const int c = 4 * c4 + u;
             const long long v = limb_levels(L0[c], L1[c], L2[c], L3[c]);
+            if (a.s32 && row_ok && j + u < T) {  // v in units of 2^(Eq + Ek - 36), times the softmax scale
+              const int e2 = Eq + ekc[c] - 36;      // a zero row (exponent kExpZero) has v = 0
+              a.s32[rowid * T + j + u] =
+                  (v != 0 && e2 > -1000 && e2 < 1000)
+                      ? static_cast<float>(static_cast<double>(v) * a.scale * __hiloint2double((1023 + e2) << 20, 0))
+                      : 0.0f;
+            }
             int sh = A - ekc[c];
             sh = sh < 1 ? 1 : (sh > 62 ? 62 : sh);
             kv[u] = static_cast<int>((v + (1LL << (sh - 1))) >> sh);
@@ -1337,6 +1331,7 @@ cudaError_t launch_plan_fast(const void* q, const void* k, const float* q_scale,
   sa_.rkmax = w.rkmax;
   sa_.rkmin = w.rkmin;
   sa_.meta = reinterpret_cast<RowMeta*>(w.meta);
+  sa_.s32 = w.s32;
   sa_.st = st;
   sa_.T = g.T;
   sa_.Tk = w.Tk;
