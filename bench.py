@@ -755,6 +755,30 @@ def run_sweep(args):
             del x, A
 
 
+def run_one_pass(args):
+    """One pass of every hot kernel on the seeded inputs of --config, nothing timed: sa_plan,
+    sa_forward (fp32 copy), sa_backward, sa_plan_fine (R = 2x2x2), sa_plan_coarse,
+    sa_forward_gated, sa_backward_gated.  Prints the selected tile counts."""
+    import torch
+
+    import block_sparse_attention_cubes_b200 as sa
+    import synth
+    cfg = synth.get_config(args.config)
+    host = synth.make_inputs(cfg, 0)
+    p = sa.make_params(cfg.B, cfg.H, cfg.D, cfg.lat, cfg.top_k, cfg.top_p)
+    x = {n: sa.tile(host[n].cuda(), p) for n in ("q", "k", "v", "do")}
+    idx, cnt = sa.plan(x["q"], x["k"], p)
+    out, lse, o32 = sa.forward(x["q"], x["k"], x["v"], idx, cnt, p, with_f32=True)
+    sa.backward(x["q"], x["k"], x["v"], out, lse, x["do"], idx, cnt, p, out_f32=o32)
+    _, fcnt = sa.plan_fine(x["q"], x["k"], p, R=(2, 2, 2))
+    idx2, cnt2, co = sa.plan_coarse(x["q"], x["k"], x["v"], p)
+    gate = synth.make_gate(cfg, 0).cuda()
+    og, lg, o32g = sa.forward_gated(x["q"], x["k"], x["v"], idx2, cnt2, p, co, gate)
+    sa.backward_gated(x["q"], x["k"], x["v"], og, lg, x["do"], gate, idx2, cnt2, p, co, out_f32=o32g)
+    torch.cuda.synchronize()
+    print(json.dumps({"one_pass": cfg.name, "tiles": int(cnt.sum()), "fine_tiles": int(fcnt.sum())}), flush=True)
+
+
 def max_over_ranks(x: float, dist, device) -> float:
     """Max of a per-rank scalar over all ranks (identity without a process group)."""
     if dist is None:
@@ -1066,6 +1090,10 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="config-4 sweep (k=4, p x sparsity grid): one JSON line per point with load balance")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--one-pass", action="store_true",
+                    help="one untimed pass of every hot kernel at --config (router, forward with the fp32 copy, "
+                         "backward, fine router, coarse branch and gated layer) and exit: the command the "
+                         "kernel profiles are captured on")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -1074,6 +1102,10 @@ def main():
     if args.sweep:
         if rank == 0:
             run_sweep(args)
+        return
+    if args.one_pass:
+        if rank == 0:
+            run_one_pass(args)
         return
     if args.impl == "reference":
         if rank == 0:

@@ -494,9 +494,9 @@ constexpr uint32_t OFF_RING = OFF_BAR + 272;  // kItemRing item ids
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;
 constexpr uint32_t TMEM_COLS = 512;  // S^T/P^T at 0, dP^T/dS^T at 128, dV at 256, dK at 384
 enum {
-  B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DF = 6, B_DE = 8, B_SF = 10, B_DPF = 12, B_PF = 14, B_DSF = 16,
-  B_DVR = 18, B_DVFREE = 19, B_FIN = 20, B_IF = 21, B_IE = 25, NBAR = 29
-};  // S^T, dP^T, P-full and dS-full are one barrier per softmax group (+ g)
+  B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DF = 6, B_DE = 8, B_SF = 10, B_DPF = 11, B_PF = 12, B_DSF = 13,
+  B_DVR = 14, B_DVFREE = 15, B_FIN = 16, B_IF = 17, B_IE = 21, NBAR = 25
+};
 }  // namespace dkv
 
 template <int KS>  // D / 16; MMA loops unrolled (a counted loop costs more than the MMA)
@@ -523,8 +523,8 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < NBAR; ++b)
-      mbar_init(&bars[b], (b == B_PF || b == B_PF + 1 || b == B_DSF || b == B_DSF + 1)
-                              ? 128u
+      mbar_init(&bars[b], (b == B_PF || b == B_DSF)
+                              ? 256u
                               : (b == B_DVFREE ? 8u : ((b >= B_IE && b < B_IE + kItemRing) ? kRingReaders : 1u)));
     *sm_abort = aborted(a.st) ? 1 : 0;
     fence_barrier_init();
@@ -614,7 +614,7 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
   } else if (warp == 1) {
     // the whole warp runs the loop; one elected lane issues (see elect_one)
     if (!skip_all) {
-      const uint32_t idesc_n64 = make_idesc(128, 64, use16 ? FMT_F16 : FMT_BF16, false, false);
+      const uint32_t idesc_kk = make_idesc(128, 128, use16 ? FMT_F16 : FMT_BF16, false, false);
       const uint32_t idesc_mn = make_idesc(128, 128, use16 ? FMT_F16 : FMT_BF16, false, true);
       uint32_t gs = 0;
       bool ok = true;
@@ -625,96 +625,92 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
         if (!mbar_wait_warp(&bars[B_KVF], n & 1, a.st, a.timeout_ns, 81)) break;
         // one phase of DVR / DVFREE per item, empty items included (see the dQ kernel)
         if (n >= 1 && !mbar_wait_warp(&bars[B_DVFREE], (n - 1) & 1, a.st, a.timeout_ns, 82)) break;
-        // Each softmax group g owns query cube g of a step and runs its own pipeline: S^T_g and
-        // dP^T_g are N = 64 products into the group's own TMEM columns, and per step the issue
-        // order is  dV += P^T_0 dO_0, S^T_0(s+1), dV += P^T_1 dO_1, S^T_1(s+1), then
-        // dK += dS^T_0 Q_0, dP^T_0(s+1), dK += dS^T_1 Q_1, dP^T_1(s+1).  S^T_g(s+1) overwrites
-        // P^T_g(s), read by the dV product just issued; dP^T_g(s+1) overwrites dS^T_g(s), read by
-        // the dK product just issued (one lane issues everything, so the products execute in
-        // this order).  A group never waits for the other: while one runs its exponentials the
-        // tensor cores work on the other's products.
-        auto issue_sdp = [&](uint32_t g, int gq, bool want_s) -> bool {
+        // Issue order per step s:  dV(s), S^T(s+1), dK(s), dP^T(s+1).  S^T(s+1) overwrites P^T(s),
+        // already read by dV(s); dP^T(s+1) overwrites dS^T(s), already read by dK(s) (one lane
+        // issues everything, so the products execute in this order).  The exponentials of step
+        // s+1 then overlap dK(s), and dS^T(s+1) overlaps dV(s+1).
+        auto issue_sdp = [&](uint32_t g, bool want_s) -> bool {
           const uint32_t st = g % QST;
           if (!mbar_wait_warp(want_s ? &bars[B_QF + st] : &bars[B_DF + st], (g / QST) & 1, a.st, a.timeout_ns,
                               want_s ? 83 : 84))
             return false;
           tc_fence_after();
-          // rows 64 gq.. of the step's Q2 (dO2) tile: query cube gq
-          const uint32_t opnd = sbase + (want_s ? OFF_Q : OFF_DO) + st * 32768 + gq * 8192;
+          const uint32_t opnd = sbase + (want_s ? OFF_Q : OFF_DO) + st * 32768;
           const uint32_t kv = sbase + (want_s ? OFF_K : OFF_V);
           if (elect_one()) {
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
               const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-              umma_f16_ss(tmem + (want_s ? 0 : 128) + gq * 64, sw128_desc(kv + off, 16, 1024),
-                          sw128_desc(opnd + off, 16, 1024), idesc_n64, ks > 0 ? 1u : 0u);
+              umma_f16_ss(tmem + (want_s ? 0 : 128), sw128_desc(kv + off, 16, 1024), sw128_desc(opnd + off, 16, 1024),
+                          idesc_kk, ks > 0 ? 1u : 0u);
             }
-            umma_commit(&bars[(want_s ? B_SF : B_DPF) + gq]);
+            umma_commit(&bars[want_s ? B_SF : B_DPF]);
           }
           __syncwarp();
           return true;
         };
-        if (nsteps > 0)
-          ok = issue_sdp(gs, 0, true) && issue_sdp(gs, 1, true) && issue_sdp(gs, 0, false) &&
-               issue_sdp(gs, 1, false);
+        if (nsteps > 0) ok = issue_sdp(gs, true) && issue_sdp(gs, false);
         for (int s = 0; ok && s < nsteps; ++s, ++gs) {
           const uint32_t st = gs % QST;
           const uint32_t qst = sbase + OFF_Q + st * 32768, dst = sbase + OFF_DO + st * 32768;
+          if (!mbar_wait_warp(&bars[B_PF], gs & 1, a.st, a.timeout_ns, 85)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one()) {
+            if (use16) {
 #pragma unroll
-          for (int gq = 0; gq < 2; ++gq) {  // dV += P^T_g dO_g (K = the group's 64 queries)
-            if (!mbar_wait_warp(&bars[B_PF + gq], gs & 1, a.st, a.timeout_ns, 85)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            if (elect_one()) {
-#pragma unroll
-              for (int part = 0; part < 2; ++part) {  // P^T (or P^T_hi), then P^T_lo
-                if (part == 1 && use16) break;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  const uint32_t acol = gq * 64 + part * 32 + kk * 8;
-                  umma_f16_ts(tmem + 256, tmem + acol, sw128_desc(dst + (4 * gq + kk) * 2048, 16384, 1024), idesc_mn,
-                              (s > 0 || gq > 0 || part > 0 || kk > 0) ? 1u : 0u);
-                }
+              for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO2 (fp16), overlapping dS^T
+                const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
+                umma_f16_ts(tmem + 256, tmem + acol, sw128_desc(dst + kk * 2048, 16384, 1024), idesc_mn,
+                            (s > 0 || kk > 0) ? 1u : 0u);
               }
-            }
-            __syncwarp();
-            if (s + 1 < nsteps && !issue_sdp(gs + 1, gq, true)) {
-              ok = false;
-              break;
+            } else {
+#pragma unroll
+              for (int ks = 0; ks < 16; ++ks) {  // dV += P^T dO2 (hi then lo), overlapping dS^T
+                const uint32_t kk = ks & 7, part = ks >> 3;
+                const uint32_t acol = (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
+                umma_f16_ts(tmem + 256, tmem + acol, sw128_desc(dst + kk * 2048, 16384, 1024), idesc_mn,
+                            (s > 0 || ks > 0) ? 1u : 0u);
+              }
             }
           }
-          if (!ok) break;
+          __syncwarp();
+          if (s + 1 < nsteps && !issue_sdp(gs + 1, true)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait_warp(&bars[B_DSF], gs & 1, a.st, a.timeout_ns, 87)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one()) {
+            if (use16) {
 #pragma unroll
-          for (int gq = 0; gq < 2; ++gq) {  // dK += dS^T_g Q_g
-            if (!mbar_wait_warp(&bars[B_DSF + gq], gs & 1, a.st, a.timeout_ns, 87)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            if (elect_one()) {
-#pragma unroll
-              for (int part = 0; part < 2; ++part) {  // dS^T (or dS^T_hi), then dS^T_lo
-                if (part == 1 && use16) break;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  const uint32_t acol = 128 + gq * 64 + part * 32 + kk * 8;
-                  umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(qst + (4 * gq + kk) * 2048, 16384, 1024), idesc_mn,
-                              (s > 0 || gq > 0 || part > 0 || kk > 0) ? 1u : 0u);
-                }
+              for (int kk = 0; kk < 8; ++kk) {  // dK += dS^T Q2 (fp16)
+                const uint32_t acol = 128 + (kk >> 2) * 64 + (kk & 3) * 8;
+                umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(qst + kk * 2048, 16384, 1024), idesc_mn,
+                            (s > 0 || kk > 0) ? 1u : 0u);
               }
-              if (gq == 1) {
-                // the Q and dO stages (with their lse and Delta, read by the softmax before DSF) are free
-                umma_commit(&bars[B_QE + st]);
-                umma_commit(&bars[B_DE + st]);
+            } else {
+#pragma unroll
+              for (int ks = 0; ks < 16; ++ks) {  // dK += dS^T Q2 (hi then lo)
+                const uint32_t kk = ks & 7, part = ks >> 3;
+                const uint32_t acol = 128 + (kk >> 2) * 64 + part * 32 + (kk & 3) * 8;
+                umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(qst + kk * 2048, 16384, 1024), idesc_mn,
+                            (s > 0 || ks > 0) ? 1u : 0u);
               }
             }
-            __syncwarp();
-            if (s + 1 < nsteps && !issue_sdp(gs + 1, gq, false)) {
-              ok = false;
-              break;
-            }
+            // the Q and dO stages (with their lse and Delta, read by the softmax before DSF) are free
+            umma_commit(&bars[B_QE + st]);
+            umma_commit(&bars[B_DE + st]);
+          }
+          __syncwarp();
+          if (s + 1 < nsteps && !issue_sdp(gs + 1, false)) {
+            ok = false;
+            break;
           }
         }
         if (!ok) break;
@@ -753,7 +749,7 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
         const int e_next = (2 * s + 2 + grp < nu) ? ul[2 * s + 2 + grp] : 0;
         const bool active = ((e >> khalf) & 1) && key_valid;
         const bool w_active = __any_sync(0xffffffffu, active);
-        if (!mbar_wait(&bars[B_SF + grp], gs & 1, a.st, a.timeout_ns, 91)) *sm_abort = 1;
+        if (!mbar_wait(&bars[B_SF], gs & 1, a.st, a.timeout_ns, 91)) *sm_abort = 1;
         tc_fence_after();
         // P^T = exp(S^T * scale - lse_q): written as soon as it is known so that dV can start
         float pe[64];
@@ -803,10 +799,10 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
           }
           tmem_st_wait();
           tc_fence_before();
-          mbar_arrive(&bars[B_PF + grp]);
+          mbar_arrive(&bars[B_PF]);
         }
         // dS^T = P^T (dP^T - Delta_q)
-        if (!mbar_wait(&bars[B_DPF + grp], gs & 1, a.st, a.timeout_ns, 93)) *sm_abort = 1;
+        if (!mbar_wait(&bars[B_DPF], gs & 1, a.st, a.timeout_ns, 93)) *sm_abort = 1;
         tc_fence_after();
         {
           // pe becomes dS^T in place (P^T is no longer needed once packed)
@@ -848,7 +844,7 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
           qm_cur = a.cube_mask[e >> 2];
           tmem_st_wait();
           tc_fence_before();
-          mbar_arrive(&bars[B_DSF + grp]);
+          mbar_arrive(&bars[B_DSF]);
         }
       }
       // epilogue: key row r, columns 64grp..64grp+63 of dV and dK (dK times the scale)
