@@ -43,24 +43,22 @@ constexpr uint32_t OFF_Q = 0;                    // Q2: [2 halves][128 rows][128
 constexpr uint32_t OFF_K = 32768;                // KST x [2 halves][128 keys][128 B]
 constexpr uint32_t OFF_V = OFF_K + KST * 32768;  // VST x same
 constexpr uint32_t OFF_BAR = OFF_V + VST * 32768;
-constexpr uint32_t OFF_SLOT = OFF_BAR + 320;     // after up to 40 mbarriers
-constexpr uint32_t OFF_ABORT = OFF_BAR + 328;
-constexpr uint32_t OFF_RING = OFF_BAR + 336;     // kItemRing item ids
+constexpr uint32_t OFF_SLOT = OFF_BAR + 256;
+constexpr uint32_t OFF_ABORT = OFF_BAR + 264;
+constexpr uint32_t OFF_RING = OFF_BAR + 272;     // kItemRing item ids
 constexpr uint32_t OFF_XMAX = OFF_BAR + 512;     // [2 groups][128 rows] float: running maxima at the item's end
 constexpr uint32_t OFF_XL = OFF_XMAX + 1024;     // [2 groups][128 rows] float: partial sums
 constexpr uint32_t SMEM_BYTES = OFF_XL + 1024 + 1024;
 // S/P[b] at 128b (b = 0,1): group g's 64 key columns at 128b + 64g, its P over them; O_g at 256 + 128g
 constexpr uint32_t TMEM_COLS = 512;
-// S-full and P-full are one barrier per (S buffer, group): the softmax of step s+1 can start
-// before the MMA thread has observed P(s) (S(s+1) is issued ahead of PV(s)), so a single
-// barrier per group could complete two phases unobserved.  The softmax of step s+2 needs
-// S(s+2), issued only after PV(s).  PV-done is one barrier per group (its rescales wait for its
-// previous PV).
+// P-full is one barrier per (S buffer, group): the softmax of step s+1 can start before the MMA
+// thread has observed P(s) (S(s+1) is issued ahead of PV(s)), so a single barrier per group
+// could complete two phases unobserved.  The softmax of step s+2 needs S(s+2), issued only
+// after PV(s).  PV-done is one barrier per group (its rescales wait for its previous PV).
 enum {
-  B_QF = 0, B_QE = 1, B_KF = 2, B_KE = 5, B_VF = 8, B_VE = 10, B_SF = 12, B_PF = 16, B_PFREE = 20, B_OR = 22,
-  B_OFREE = 23, B_FIN = 24, B_IF = 25, B_IE = 29, NBAR = 33
+  B_QF = 0, B_QE = 1, B_KF = 2, B_KE = 5, B_VF = 8, B_VE = 10, B_SF = 12, B_PF = 14, B_PFREE = 18, B_OR = 20,
+  B_OFREE = 21, B_FIN = 22, B_IF = 23, B_IE = 27, NBAR = 31
 };
-static_assert(NBAR * 8 <= OFF_SLOT - OFF_BAR, "mbarriers overlap the TMEM slot");
 }  // namespace fwd
 
 // KS = D / 16 k-steps per S product.  Every MMA loop below has a compile-time trip count and
@@ -194,43 +192,38 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (!skip_all) {
-      const uint32_t idesc_s = make_idesc(128, 64, FMT_BF16, false, false);   // S_g: N = 64 keys
-      const uint32_t idesc_s8 = make_idesc(128, 64, FMT_E4M3, false, false);
+      const uint32_t idesc_s = make_idesc(128, 128, FMT_BF16, false, false);
+      const uint32_t idesc_s8 = make_idesc(128, 128, FMT_E4M3, false, false);
       const uint32_t idesc_o = make_idesc(128, 128, use16 ? FMT_F16 : FMT_BF16, false, true);
       uint32_t gs_s = 0, gs_o = 0;
       bool ok = true;
       // S for the next global step into S buffer gs_s & 1.  That buffer last held P of step
       // gs_s - 2, read by PV(gs_s - 2), which this thread issued earlier; the tcgen05.mma
       // operations of one thread execute in issue order.
-      // S_g for one softmax group: its 64 keys (rows 64g.. of the K2 stage) into its own columns of
-      // the S buffer, N = 64, so each group's step can start as soon as its own product is done.
-      // Buffer gs_s & 1 last held P of step gs_s - 2, read by that group's PV(gs_s - 2), issued
-      // earlier by this thread; the tcgen05.mma operations of one thread execute in issue order.
-      auto issue_s = [&](int gq) -> bool {
+      auto issue_s = [&]() -> bool {
         const uint32_t kst_i = gs_s % KST, sb = gs_s & 1;
         if (!mbar_wait_warp(&bars[B_KF + kst_i], (gs_s / KST) & 1, a.st, a.timeout_ns, 21)) return false;
         tc_fence_after();
-        const uint32_t kst = sbase + OFF_K + kst_i * 32768 + gq * 8192;
-        const uint32_t d_s = tmem + sb * 128 + gq * 64;
+        const uint32_t kst = sbase + OFF_K + kst_i * 32768;
         if (elect_one()) {
           if (FP8) {
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)  // 32 e4m3 elements = 32 bytes per k-step
-              umma_f8_ss(d_s, sw128_desc(sbase + OFF_Q + ks * 32, 16, 1024), sw128_desc(kst + ks * 32, 16, 1024),
-                         idesc_s8, ks > 0 ? 1u : 0u);
+              umma_f8_ss(tmem + sb * 128, sw128_desc(sbase + OFF_Q + ks * 32, 16, 1024),
+                         sw128_desc(kst + ks * 32, 16, 1024), idesc_s8, ks > 0 ? 1u : 0u);
           } else {
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
               const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-              umma_f16_ss(d_s, sw128_desc(sbase + OFF_Q + off, 16, 1024), sw128_desc(kst + off, 16, 1024), idesc_s,
-                          ks > 0 ? 1u : 0u);
+              umma_f16_ss(tmem + sb * 128, sw128_desc(sbase + OFF_Q + off, 16, 1024),
+                          sw128_desc(kst + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
             }
           }
-          umma_commit(&bars[B_SF + 2 * sb + gq]);
-          if (gq == 1) umma_commit(&bars[B_KE + kst_i]);  // both halves of the K stage have been read
+          umma_commit(&bars[B_SF + sb]);
+          umma_commit(&bars[B_KE + kst_i]);
         }
         __syncwarp();
-        if (gq == 1) ++gs_s;
+        ++gs_s;
         return true;
       };
       for (int n = 0; ok; ++n) {
@@ -238,7 +231,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         if (it < 0) break;
         const int nsteps = (a.u_cnt[it] + 1) >> 1;
         if (!mbar_wait_warp(&bars[B_QF], n & 1, a.st, a.timeout_ns, 22)) break;
-        for (int s = 0; ok && s < nsteps && s < 2; ++s) ok = issue_s(0) && issue_s(1);
+        for (int s = 0; ok && s < nsteps && s < 2; ++s) ok = issue_s();
         // O_0 and O_1 of the previous pair must have been read out before this pair's first PV
         if (ok && n >= 1) ok = mbar_wait_warp(&bars[B_OFREE], (n - 1) & 1, a.st, a.timeout_ns, 23);
         for (int s = 0; ok && s < nsteps; ++s) {
@@ -272,14 +265,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
               if (gq == 1) umma_commit(&bars[B_VE + vs]);
             }
             __syncwarp();
-            // S_g(s+2) right behind PV_g(s), which read the group's P(s) from the same columns
-            if (s + 2 < nsteps && !issue_s(gq)) {
-              ok = false;
-              break;
-            }
           }
           if (!ok) break;
           ++gs_o;
+          if (s + 2 < nsteps) ok = issue_s();
         }
         if (!ok) break;
         if (elect_one()) {
@@ -324,7 +313,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         const bool active = ((e >> half) & 1) && row_exists;  // uniform over each warp
         float sc = a.scale_log2 * qs;
         if (a.k_scale && active) sc *= a.k_scale[static_cast<size_t>(bh) * g.T + tile];
-        if (!mbar_wait(&bars[B_SF + 2 * b + grp], (gs >> 1) & 1, a.st, a.timeout_ns, 31)) *sm_abort = 1;
+        if (!mbar_wait(&bars[B_SF + b], (gs >> 1) & 1, a.st, a.timeout_ns, 31)) *sm_abort = 1;
         tc_fence_after();
         float x[64];
         float pmax = -INFINITY;
