@@ -495,8 +495,8 @@ constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;
 constexpr uint32_t TMEM_COLS = 512;  // S^T/P^T at 0, dP^T/dS^T at 128, dV at 256, dK at 384
 enum {
   B_KVF = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_DF = 6, B_DE = 8, B_SF = 10, B_DPF = 11, B_PF = 12, B_DSF = 13,
-  B_DVR = 14, B_DVFREE = 15, B_FIN = 16, B_IF = 17, B_IE = 21, B_SRD = 25, NBAR = 26
-};  // B_SRD (fp16 path): every softmax thread has read S^T of the step
+  B_DVR = 14, B_DVFREE = 15, B_FIN = 16, B_IF = 17, B_IE = 21, NBAR = 25
+};
 }  // namespace dkv
 
 template <int KS>  // D / 16; MMA loops unrolled (a counted loop costs more than the MMA)
@@ -523,7 +523,7 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < NBAR; ++b)
-      mbar_init(&bars[b], (b == B_PF || b == B_DSF || b == B_SRD)
+      mbar_init(&bars[b], (b == B_PF || b == B_DSF)
                               ? 256u
                               : (b == B_DVFREE ? 8u : ((b >= B_IE && b < B_IE + kItemRing) ? kRingReaders : 1u)));
     *sm_abort = aborted(a.st) ? 1 : 0;
@@ -650,49 +650,7 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
           return true;
         };
         if (nsteps > 0) ok = issue_sdp(gs, true) && issue_sdp(gs, false);
-        // fp16 path: the softmax writes P^T and dS^T (fp16 pairs, 32 columns each) into its group's dP^T
-        // columns once it has read them, so S^T(s+1) can go out as soon as every softmax thread has read
-        // S^T(s): the exponentials of step s+1 then overlap dV(s), dK(s) and dP^T(s+1).  Order per step:
-        // S^T(s+1) (after the S^T reads of step s), dV(s) and dK(s) (after P^T, dS^T of step s),
-        // dP^T(s+1) (after dV(s), dK(s) in issue order).
-        for (int s = 0; use16 && ok && s < nsteps; ++s, ++gs) {
-          const uint32_t st = gs % QST;
-          const uint32_t qst = sbase + OFF_Q + st * 32768, dst = sbase + OFF_DO + st * 32768;
-          if (s + 1 < nsteps) {
-            if (!mbar_wait_warp(&bars[B_SRD], gs & 1, a.st, a.timeout_ns, 88) || !issue_sdp(gs + 1, true)) {
-              ok = false;
-              break;
-            }
-          }
-          if (!mbar_wait_warp(&bars[B_PF], gs & 1, a.st, a.timeout_ns, 85)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (elect_one()) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO2: P^T of group kk / 4 at 128 + 64 g + 32
-              const uint32_t acol = 128 + (kk >> 2) * 64 + 32 + (kk & 3) * 8;
-              umma_f16_ts(tmem + 256, tmem + acol, sw128_desc(dst + kk * 2048, 16384, 1024), idesc_mn,
-                          (s > 0 || kk > 0) ? 1u : 0u);
-            }
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {  // dK += dS^T Q2: dS^T of group kk / 4 at 128 + 64 g
-              const uint32_t acol = 128 + (kk >> 2) * 64 + (kk & 3) * 8;
-              umma_f16_ts(tmem + 384, tmem + acol, sw128_desc(qst + kk * 2048, 16384, 1024), idesc_mn,
-                          (s > 0 || kk > 0) ? 1u : 0u);
-            }
-            // the Q and dO stages (with their lse and Delta, read by the softmax before PF) are free
-            umma_commit(&bars[B_QE + st]);
-            umma_commit(&bars[B_DE + st]);
-          }
-          __syncwarp();
-          if (s + 1 < nsteps && !issue_sdp(gs + 1, false)) {
-            ok = false;
-            break;
-          }
-        }
-        for (int s = 0; !use16 && ok && s < nsteps; ++s, ++gs) {
+        for (int s = 0; ok && s < nsteps; ++s, ++gs) {
           const uint32_t st = gs % QST;
           const uint32_t qst = sbase + OFF_Q + st * 32768, dst = sbase + OFF_DO + st * 32768;
           if (!mbar_wait_warp(&bars[B_PF], gs & 1, a.st, a.timeout_ns, 85)) {
@@ -793,74 +751,8 @@ __global__ void __launch_bounds__(dkv::kThreads, 1)
         const bool w_active = __any_sync(0xffffffffu, active);
         if (!mbar_wait(&bars[B_SF], gs & 1, a.st, a.timeout_ns, 91)) *sm_abort = 1;
         tc_fence_after();
+        // P^T = exp(S^T * scale - lse_q): written as soon as it is known so that dV can start
         float pe[64];
-        if (use16) {
-          // fp16 path: S^T is released as soon as it is read; P^T and dS^T go into the dP^T columns
-          if (w_active) {
-            uint32_t s0[32], s1[32];
-            tmem_ld32(t_lane + grp * 64, s0);
-            tmem_ld32(t_lane + grp * 64 + 32, s1);
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive(&bars[B_SRD]);
-            const unsigned long long qm = active ? qm_cur : 0ull;
-            const bool full = qm == ~0ull;  // uniform over the warp
-            const float* lq = lse_sh + st * 128 + grp * 64;
-#pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4) {
-              const float4 l4 = *reinterpret_cast<const float4*>(lq + 4 * c4);
-              const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int c = 4 * c4 + u;
-                const uint32_t sv = c < 32 ? s0[c] : s1[c - 32];
-                pe[c] = ex2_approx(fmaf(__uint_as_float(sv), a.scale_log2, lv[u]));  // lv = -lse log2(e)
-                if (!full && !((qm >> c) & 1ull)) pe[c] = 0.0f;
-              }
-            }
-          } else {
-            tc_fence_before();
-            mbar_arrive(&bars[B_SRD]);
-#pragma unroll
-            for (int c = 0; c < 64; ++c) pe[c] = 0.0f;
-          }
-          if (!mbar_wait(&bars[B_DPF], gs & 1, a.st, a.timeout_ns, 93)) *sm_abort = 1;
-          tc_fence_after();
-          // dS^T = P^T (dP^T - Delta_q), dP^T read 32 columns at a time; both halves are read before
-          // anything is written over them
-          uint32_t dsp[32];
-          if (w_active) {
-            const float* dq_ = dlt_sh + st * 128 + grp * 64;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              uint32_t pp[32];
-              tmem_ld32(t_lane + 128 + grp * 64 + 32 * h, pp);
-              tmem_ld_wait();
-#pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                const int c0 = 32 * h + 2 * c;
-                const float2 d2 = *reinterpret_cast<const float2*>(dq_ + c0);
-                dsp[16 * h + c] = pack_f16x2(pe[c0] * (__uint_as_float(pp[2 * c]) - d2.x),
-                                             pe[c0 + 1] * (__uint_as_float(pp[2 * c + 1]) - d2.y));
-              }
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) dsp[c] = 0u;
-          }
-          uint32_t ph[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) ph[c] = pack_f16x2(pe[2 * c], pe[2 * c + 1]);
-          tmem_st32(t_lane + 128 + grp * 64, dsp);
-          tmem_st32(t_lane + 128 + grp * 64 + 32, ph);
-          e = e_next;
-          qm_cur = a.cube_mask[e >> 2];
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(&bars[B_PF]);
-          continue;
-        }
-        // bf16 path: P^T = exp(S^T * scale - lse_q), written as soon as it is known so that dV can start
         {
           if (w_active) {
             uint32_t s0[32], s1[32];
