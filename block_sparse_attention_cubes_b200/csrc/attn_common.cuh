@@ -106,13 +106,13 @@ __device__ __forceinline__ int ring_read_warp(const ItemRing& r, int n, const At
   return it;
 }
 
-// The 256 epilogue threads (named barrier 1): they agree on success through the shared abort
-// flag behind the barrier, so they leave their loops together; one arrival per warp.
+// The epilogue threads (named barrier 1 over `nthreads`): they agree on success through the
+// shared abort flag behind the barrier, so they leave their loops together; one arrival per warp.
 __device__ __forceinline__ int ring_read_group(const ItemRing& r, int n, const AttnArgs& a, unsigned int where,
-                                               volatile int* sm_abort, bool& ok) {
+                                               volatile int* sm_abort, bool& ok, uint32_t nthreads = 256) {
   const int slot = n % kItemRing;
   if (!mbar_wait(&r.full[slot], (n / kItemRing) & 1, a.st, a.timeout_ns, where)) *sm_abort = 1;
-  named_bar_sync(1, 256);
+  named_bar_sync(1, nthreads);
   if (*sm_abort) {
     ok = false;
     return -1;
