@@ -185,20 +185,31 @@ __device__ void select_row_fp64(const double* __restrict__ s, int T, int top_k, 
                                 const unsigned long long* __restrict__ mrow = nullptr) {
   const int lane = threadIdx.x & 31;
 
-  double m = -DBL_MAX;
+  double m = -DBL_MAX, mn = DBL_MAX;
 #pragma unroll 4
-  for (int j = lane; j < T; j += 32) m = fmax(m, s[j]);
+  for (int j = lane; j < T; j += 32) {
+    m = fmax(m, s[j]);
+    mn = fmin(mn, s[j]);
+  }
 #pragma unroll
-  for (int o = 16; o; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+  for (int o = 16; o; o >>= 1) {
+    m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+    mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  }
 
   const int nk = max(1, min(top_k, T));
   const bool keep_all = (top_p >= 1.0f) || nk >= T;
   uint64_t kb = ~0ull;  // boundary key
   int jb = T;           // boundary id (elements with key == kb and id <= jb are kept)
   if (!keep_all) {
-    uint64_t prefix = 0, cnt_above = 0, mass_above = 0;
+    // every key of the row lies between those of its maximum and minimum, so the bytes above the
+    // highest bit in which those two differ are common to all: the descent starts below them
+    const uint64_t kmx = desc_key(m), kdiff = kmx ^ desc_key(mn);
+    const int shift0 = kdiff ? ((63 - __clzll(static_cast<long long>(kdiff))) & ~7) : 0;
+    uint64_t prefix = shift0 >= 56 ? 0ull : (kmx & ~((1ull << (shift0 + 8)) - 1ull));
+    uint64_t cnt_above = 0, mass_above = 0;
     double target = -1.0;  // p <= 0: the mass test always passes
-    for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int shift = shift0; shift >= 0; shift -= 8) {
       for (int d = lane; d < 256; d += 32) {
         cnt[d] = 0;
         mass[d] = 0ull;
@@ -226,7 +237,7 @@ __device__ void select_row_fp64(const double* __restrict__ s, int T, int top_k, 
           if (j < T) {
             const double x = xs[u];
             const uint64_t kj = desc_key(x);
-            if (shift == 56 || (kj >> (shift + 8)) == (prefix >> (shift + 8))) {
+            if (shift == 56 || (kj >> (shift + 8)) == (prefix >> (shift + 8))) {  // all keys at shift0
               part = true;
               d = static_cast<int>((kj >> shift) & 255u);
               mj = mrow ? mrow[j] : static_cast<unsigned long long>(mass_fx(x, m));
@@ -268,7 +279,7 @@ __device__ void select_row_fp64(const double* __restrict__ s, int T, int top_k, 
           im += om;
         }
       }
-      if (shift == 56) {
+      if (shift == shift0) {  // the first pass counts every key: the row's total mass
         const unsigned long long Z = __shfl_sync(0xffffffffu, im, 31);
         if (top_p > 0.0f) target = static_cast<double>(top_p) * static_cast<double>(Z);
       }
