@@ -332,10 +332,12 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             for (int c = 0; c < 64; ++c)
               if (!((km >> c) & 1ull)) x[c] = -INFINITY;
           }
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          float m8[8];  // eight independent chains of eight
 #pragma unroll
-          for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], x[c]);
-          pmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
+          for (int u = 0; u < 8; ++u) m8[u] = x[u];
+#pragma unroll
+          for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], x[c]);
+          pmax = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sc;
         }
         // each group keeps its own running maximum, sum and O_g (combined once per pair at the
         // end), so the groups never wait on each other within a pair; P_g overwrites the
@@ -372,14 +374,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           uint32_t ph[32], pl[M == 1 ? 32 : 1];
           if (active) {
             const uint64_t sc2 = pk2(sc, sc), nm2 = pk2(-m_run, -m_run);
-            uint64_t l2 = pk2(0.0f, 0.0f);
+            uint64_t l2[4] = {pk2(0.0f, 0.0f), pk2(0.0f, 0.0f), pk2(0.0f, 0.0f), pk2(0.0f, 0.0f)};  // 4 chains
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
               float d0, d1;
               upk2(fma2(pk2(x[2 * c], x[2 * c + 1]), sc2, nm2), d0, d1);
               const float p0 = ex2_approx(d0), p1 = ex2_approx(d1);
               const uint64_t pp = pk2(p0, p1);
-              l2 = add2(l2, pp);
+              l2[c & 3] = add2(l2[c & 3], pp);
               if constexpr (M == 2) {
                 ph[c] = pack_f16x2(p0, p1);
               } else {
@@ -392,7 +394,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
               }
             }
             float la, lb;
-            upk2(l2, la, lb);
+            upk2(add2(add2(l2[0], l2[1]), add2(l2[2], l2[3])), la, lb);
             l_part += la + lb;
           } else {
 #pragma unroll

@@ -1182,7 +1182,8 @@ __global__ void __launch_bounds__(256, 4) select_keys_kernel(const int* __restri
 // shuffle reduction), then every score's fixed-point mass once (the selection's passes would
 // otherwise evaluate the fp64 exponential again in each pass), and warp 0 selects from there
 // as select_kernel does.
-__global__ void __launch_bounds__(128) router_fallback_kernel(const double* __restrict__ qbar,
+constexpr int kFallbackThreads = 512;  // 16 warps: each key's dot product is one warp's, 8 keys per round
+__global__ void __launch_bounds__(kFallbackThreads) router_fallback_kernel(const double* __restrict__ qbar,
                                                               const double* __restrict__ kbar, int D, int T,
                                                               double scale, const int* __restrict__ flist, int top_k,
                                                               float top_p, int cap, int32_t* __restrict__ kv_index,
@@ -1190,8 +1191,9 @@ __global__ void __launch_bounds__(128) router_fallback_kernel(const double* __re
   extern __shared__ double srow[];  // [T] scores, then [T] masses
   __shared__ uint32_t cnt_s[256];
   __shared__ unsigned long long mass_s[256];
-  __shared__ double wmax[4];
+  __shared__ double wmax[kFallbackThreads / 32];
   unsigned long long* mrow = reinterpret_cast<unsigned long long*>(srow + T);
+  constexpr int kWarps = kFallbackThreads / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nf = static_cast<int>(*reinterpret_cast<const volatile unsigned*>(&st->router_fallback));
   const int per = D >> 5;  // doubles per lane (2 or 4)
@@ -1202,7 +1204,7 @@ __global__ void __launch_bounds__(128) router_fallback_kernel(const double* __re
 #pragma unroll
     for (int e = 0; e < 4; ++e) qv[e] = e < per ? qbar[static_cast<size_t>(row) * D + lane * per + e] : 0.0;
     // eight keys per warp per round, every load issued before the arithmetic
-    for (int j0 = warp * 8; j0 < T; j0 += 32) {
+    for (int j0 = warp * 8; j0 < T; j0 += 8 * kWarps) {
       double kv[8][4];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -1223,13 +1225,15 @@ __global__ void __launch_bounds__(128) router_fallback_kernel(const double* __re
     }
     __syncthreads();
     double mx = -DBL_MAX;
-    for (int j = threadIdx.x; j < T; j += 128) mx = fmax(mx, srow[j]);
+    for (int j = threadIdx.x; j < T; j += kFallbackThreads) mx = fmax(mx, srow[j]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if (lane == 0) wmax[warp] = mx;
     __syncthreads();
-    mx = fmax(fmax(wmax[0], wmax[1]), fmax(wmax[2], wmax[3]));
-    for (int j = threadIdx.x; j < T; j += 128) mrow[j] = mass_fx(srow[j], mx);
+    mx = wmax[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) mx = fmax(mx, wmax[w]);
+    for (int j = threadIdx.x; j < T; j += kFallbackThreads) mrow[j] = mass_fx(srow[j], mx);
     __syncthreads();
     if (warp == 0)
       select_row_fp64(srow, T, top_k, top_p, cap, kv_index + static_cast<size_t>(row) * cap, kv_count + row, st,
@@ -1360,7 +1364,7 @@ cudaError_t launch_plan_fast(const void* q, const void* k, const float* q_scale,
   select_keys_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(
         w.keys, w.Tk, w.rkmax, w.rkmin, reinterpret_cast<const RowMeta*>(w.meta), rows, g.T, top_k, top_p, cap,
         kv_index, kv_count, w.flist, st, debug, timeout_ns);
-  router_fallback_kernel<<<plan_fallback_ctas(), 128, static_cast<size_t>(g.T) * 16, stream>>>(
+  router_fallback_kernel<<<plan_fallback_ctas(), kFallbackThreads, static_cast<size_t>(g.T) * 16, stream>>>(
       w.qbar, w.kbar, D, g.T, scale, w.flist, top_k, top_p, cap, kv_index, kv_count, st);
   *launches = 5;
   return cudaGetLastError();
