@@ -661,10 +661,10 @@ struct ScoreArgs {
   unsigned long long timeout_ns;
 };
 
-// KS = D / 32 k-steps of 32 int8 per product.  Work item = one 128 x 128 tile of (query
-// cubes, key cubes) of one head; each CTA takes a contiguous run of items, so consecutive
-// items share their query rows (loaded once per row block).
-template <int KS>
+// KS = D / 32 k-steps of 32 int8 per product.  S32: also write every scaled score in fp32 (a.s32).
+// Work item = one 128 x 128 tile of (query cubes, key cubes) of one head; each CTA takes a
+// contiguous run of items, so consecutive items share their query rows (loaded once per row block).
+template <int KS, bool S32>
 __global__ void __launch_bounds__(rsc::kThreads, 1)
     score_keys_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_keys, const ScoreArgs a) {
@@ -856,16 +856,16 @@ __global__ void __launch_bounds__(rsc::kThreads, 1)
         for (int c4 = 0; c4 < 8; ++c4) {
           const int j = j0 + 4 * c4;
           int kv[4];
+          float sv[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int c = 4 * c4 + u;
             const long long v = limb_levels(L0[c], L1[c], L2[c], L3[c]);
-            if (a.s32 && row_ok && j + u < T) {  // v in units of 2^(Eq + Ek - 36), times the softmax scale
-              const int e2 = Eq + ekc[c] - 36;      // a zero row (exponent kExpZero) has v = 0
-              a.s32[rowid * T + j + u] =
-                  (v != 0 && e2 > -1000 && e2 < 1000)
-                      ? static_cast<float>(static_cast<double>(v) * a.scale * __hiloint2double((1023 + e2) << 20, 0))
-                      : 0.0f;
+            if constexpr (S32) {  // v in units of 2^(Eq + Ek - 36), times the softmax scale
+              const int e2 = Eq + ekc[c] - 36;  // a zero row (exponent kExpZero) has v = 0
+              sv[u] = (v != 0 && e2 > -1000 && e2 < 1000)
+                          ? static_cast<float>(static_cast<double>(v) * a.scale * __hiloint2double((1023 + e2) << 20, 0))
+                          : 0.0f;
             }
             int sh = A - ekc[c];
             sh = sh < 1 ? 1 : (sh > 62 ? 62 : sh);
@@ -873,6 +873,16 @@ __global__ void __launch_bounds__(rsc::kThreads, 1)
             if (row_ok && j + u < T) {
               lmax = max(lmax, kv[u]);
               lmin = min(lmin, kv[u]);
+            }
+          }
+          if (S32 && row_ok) {  // four consecutive scores of this row: one 16-byte store when aligned
+            float* dst = a.s32 + rowid * T + j;
+            if ((T & 3) == 0 && j + 3 < T) {
+              *reinterpret_cast<float4*>(dst) = make_float4(sv[0], sv[1], sv[2], sv[3]);
+            } else {
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                if (j + u < T) dst[u] = sv[u];
             }
           }
           // row `lane` of the warp's 32 x 32 staging tile, 16-byte chunk c4, 128-byte swizzle
@@ -1182,7 +1192,7 @@ __global__ void __launch_bounds__(256, 4) select_keys_kernel(const int* __restri
 // shuffle reduction), then every score's fixed-point mass once (the selection's passes would
 // otherwise evaluate the fp64 exponential again in each pass), and warp 0 selects from there
 // as select_kernel does.
-constexpr int kFallbackThreads = 512;  // 16 warps: each key's dot product is one warp's, 8 keys per round
+constexpr int kFallbackThreads = 128;  // 4 warps: each key's dot product is one warp's, 8 keys per round (16 warps measured slower)
 __global__ void __launch_bounds__(kFallbackThreads) router_fallback_kernel(const double* __restrict__ qbar,
                                                               const double* __restrict__ kbar, int D, int T,
                                                               double scale, const int* __restrict__ flist, int top_k,
@@ -1289,10 +1299,10 @@ cudaError_t launch_plan_fast(const void* q, const void* k, const float* q_scale,
                              DevStatus* st, cudaStream_t stream, int* launches) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(score_keys_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         rsc::SMEM_BYTES);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(score_keys_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsc::SMEM_BYTES);
+    cudaError_t e = cudaSuccess;
+    for (auto fn : {score_keys_kernel<4, false>, score_keys_kernel<2, false>, score_keys_kernel<4, true>,
+                    score_keys_kernel<2, true>})
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, rsc::SMEM_BYTES);
     if (e == cudaSuccess)  // one fp64 score row and its masses, up to 8192 cubes
       e = cudaFuncSetAttribute(router_fallback_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 8192 * 16);
     for (auto fn : {pool_limbs_kernel<2, 4>, pool_limbs_kernel<2, 2>, pool_limbs_kernel<1, 4>, pool_limbs_kernel<1, 2>})
@@ -1356,10 +1366,9 @@ cudaError_t launch_plan_fast(const void* q, const void* k, const float* q_scale,
   const int nrb = (g.T + 127) / 128;
   const long long items = static_cast<long long>(BH) * nrb * nrb;
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  if (D == 64)
-    score_keys_kernel<2><<<grid, rsc::kThreads, rsc::SMEM_BYTES, stream>>>(tm_qlimb, tm_klimb, tm_keys, sa_);
-  else
-    score_keys_kernel<4><<<grid, rsc::kThreads, rsc::SMEM_BYTES, stream>>>(tm_qlimb, tm_klimb, tm_keys, sa_);
+  auto kern = D == 64 ? (w.s32 ? score_keys_kernel<2, true> : score_keys_kernel<2, false>)
+                      : (w.s32 ? score_keys_kernel<4, true> : score_keys_kernel<4, false>);
+  kern<<<grid, rsc::kThreads, rsc::SMEM_BYTES, stream>>>(tm_qlimb, tm_klimb, tm_keys, sa_);
   const int rows = BH * g.T;
   select_keys_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(
         w.keys, w.Tk, w.rkmax, w.rkmin, reinterpret_cast<const RowMeta*>(w.meta), rows, g.T, top_k, top_p, cap,

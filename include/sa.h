@@ -221,7 +221,8 @@ typedef struct {
 
 /* Router and coarse branch in one call: the same kv_index / kv_count as sa_plan (same
  * kernels, bit-identical), and the cube-level tensors of `coarse` (written).  Q and K are
- * pooled once for both (the coarse branch reads the router's fp64 means and scores).
+ * pooled once for both (the coarse branch reads the router's fp64 means, and every scaled score, which
+ * the router's score kernel also writes in fp32 for this call: the exact limb dot product rounded once).
  * v: [B,H,Npad,D] bf16.  Workspace: sa_workspace_size(p, SA_OP_PLAN_COARSE).
  * Deterministic. */
 SA_API sa_status sa_plan_coarse(const void* q, const void* k, const void* v, const sa_params* p, int32_t* kv_index,
