@@ -186,6 +186,7 @@ def run_ours(args, rank, world, dist):
             st = sa.device_status(A._ws[op])
             if st != 0:
                 raise RuntimeError(f"device status {sa.STATUS_NAMES.get(st, st)} after warm-up")
+        fallback_rows = sa.plan_fallback_rows(A._ws[sa.OP_PLAN])  # rows the last plan decided in fp64
         cnt = last[1]
         ntiles = int(cnt.sum().item())
         valid_fl = valid_only_flops(sa, p, cfg, last[0], cnt, dev)
@@ -264,7 +265,8 @@ def run_ours(args, rank, world, dist):
         "valid_only": {"flops_fwd_bwd": valid_fl, "tflops": round(valid_fl / ((fwd_med + bwd_med) * 1e-3) / 1e12, 3),
                        "note": "4*D and 10*D FLOPs per valid (query row, key) pair of the selected tiles"},
         "router": {"achieved_gbs": round(router_gbs, 1), "peak_gbs": peaks.get("hbm_gbs"),
-                   "frac": round(router_gbs / peaks.get("hbm_gbs"), 4), "algorithmic_bytes": router_bytes},
+                   "frac": round(router_gbs / peaks.get("hbm_gbs"), 4), "algorithmic_bytes": router_bytes,
+                   "fallback_rows": fallback_rows, "rows": int(cnt.numel())},
         "roofline": roofline,
         "gpu_launches": gpu_launches,
         "clocks": clock_summary,

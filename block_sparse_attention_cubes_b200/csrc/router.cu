@@ -550,33 +550,52 @@ __global__ void __launch_bounds__(rpl::kThreads, 1) pool_limbs_kernel(const Pool
       const int stage = static_cast<int>(j % kStages);
       if (!mbar_wait_warp(&full[stage], (j / kStages) & 1, a.st, a.timeout_ns, 133)) break;
       const uint8_t* tile = smem + stage * kStageBytes + lane * EPL * ESZ;
-    for (int a0 = 0; a0 < vt; ++a0)
-      for (int b0 = 0; b0 < vh; ++b0)
-#pragma unroll
-        for (int d0 = 0; d0 < 4; ++d0) {
-          if (d0 >= vw) break;
-          double* acc = acc4[d0];
-          const uint8_t* rp = tile + (a0 * 16 + b0 * 4 + d0) * row_bytes;
-          if constexpr (ESZ == 2) {
-            uint32_t wv[EPL / 2];
-            if constexpr (EPL == 4) {
-              const uint2 t2 = *reinterpret_cast<const uint2*>(rp);
-              wv[0] = t2.x;
-              wv[1] = t2.y;
-            } else {
-              wv[0] = *reinterpret_cast<const uint32_t*>(rp);
-            }
-#pragma unroll
-            for (int e = 0; e < EPL; ++e)
-              acc[e] += static_cast<double>(
-                  __uint_as_float((e & 1) ? (wv[e >> 1] & 0xffff0000u) : (wv[e >> 1] << 16)));
-          } else {
-            uint32_t wv = EPL == 4 ? *reinterpret_cast<const uint32_t*>(rp)
-                                   : static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(rp));
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[e] += static_cast<double>(e4m3_value((wv >> (8 * e)) & 0xffu));
-          }
+      // this lane's EPL elements of one row: loaded from shared memory as NW words, then
+      // widened to fp64 and added
+      constexpr int NW = ESZ == 2 ? EPL / 2 : 1;
+      auto load_row = [&](const uint8_t* rp, uint32_t (&wv)[NW]) {
+        if constexpr (ESZ == 2 && EPL == 4) {
+          const uint2 t2 = *reinterpret_cast<const uint2*>(rp);
+          wv[0] = t2.x;
+          wv[1] = t2.y;
+        } else if constexpr (ESZ == 1 && EPL == 2) {
+          wv[0] = *reinterpret_cast<const uint16_t*>(rp);
+        } else {
+          wv[0] = *reinterpret_cast<const uint32_t*>(rp);
         }
+      };
+      auto add_words = [&](double* acc, const uint32_t (&wv)[NW]) {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          if constexpr (ESZ == 2)
+            acc[e] += static_cast<double>(
+                __uint_as_float((e & 1) ? (wv[e >> 1] & 0xffff0000u) : (wv[e >> 1] << 16)));
+          else
+            acc[e] += static_cast<double>(e4m3_value((wv[0] >> (8 * e)) & 0xffu));
+        }
+      };
+      if (vt == 4 && vh == 4 && vw == 4) {
+        // a whole cube: 64 consecutive rows, sixteen at a time with every load of the group
+        // issued before its arithmetic (one shared-memory round trip per sixteen rows)
+#pragma unroll 1
+        for (int r0 = 0; r0 < 64; r0 += 16) {
+          uint32_t w16[16][NW];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) load_row(tile + (r0 + u) * row_bytes, w16[u]);
+#pragma unroll
+          for (int u = 0; u < 16; ++u) add_words(acc4[u & 3], w16[u]);
+        }
+      } else {
+        for (int a0 = 0; a0 < vt; ++a0)
+          for (int b0 = 0; b0 < vh; ++b0)
+#pragma unroll
+            for (int d0 = 0; d0 < 4; ++d0) {
+              if (d0 >= vw) break;
+              uint32_t wv[NW];
+              load_row(tile + (a0 * 16 + b0 * 4 + d0) * row_bytes, wv);
+              add_words(acc4[d0], wv);
+            }
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[stage]);  // the cube's rows have been read
     }
@@ -856,7 +875,7 @@ __global__ void __launch_bounds__(rsc::kThreads, 1)
         for (int c4 = 0; c4 < 8; ++c4) {
           const int j = j0 + 4 * c4;
           int kv[4];
-          float sv[4];
+          float sv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int c = 4 * c4 + u;
@@ -1186,13 +1205,239 @@ __global__ void __launch_bounds__(256, 4) select_keys_kernel(const int* __restri
   }
 }
 
+// The same decision as select_row_fp64, taken by a whole CTA of NWARP warps: the radix levels
+// split the row's keys over the warps (one shared histogram), warp 0 scans each level's 256
+// buckets and publishes the hit through shared memory, and the two passes in id order (the
+// boundary candidate, the emission) give each warp a contiguous range of ids, offset by the
+// counts of the warps before it.  `s` and `mrow` (scores and their fixed-point masses against
+// the row maximum m) are in shared memory; mn is the row minimum.  Called by every thread.
+struct SelCtl {
+  unsigned long long cnt_above, mass_above, bmass, kb;
+  double target;
+  int dstar, cstar, jb;
+  uint32_t bucket;
+  int wcount[32];
+};
+
+template <int NWARP>
+__device__ void select_row_fp64_cta(const double* __restrict__ s, const unsigned long long* __restrict__ mrow,
+                                    double m, double mn, int T, int top_k, float top_p, int cap,
+                                    int32_t* __restrict__ out, int32_t* __restrict__ count, DevStatus* st,
+                                    uint32_t* cnt, unsigned long long* mass, SelCtl* ctl) {
+  constexpr int NT = NWARP * 32;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nk = max(1, min(top_k, T));
+  const bool keep_all = (top_p >= 1.0f) || nk >= T;
+  // contiguous id range of this warp for the passes in id order (whole chunks of 32)
+  const int per = ((T + NT - 1) / NT) * 32;
+  const int w_lo = min(T, warp * per), w_hi = min(T, w_lo + per);
+  uint64_t kb = ~0ull;  // boundary key; ids with this key up to jb are kept
+  int jb = T;
+  if (!keep_all) {
+    const uint64_t kmx = desc_key(m), kdiff = kmx ^ desc_key(mn);
+    const int shift0 = kdiff ? ((63 - __clzll(static_cast<long long>(kdiff))) & ~7) : 0;
+    uint64_t prefix = shift0 >= 56 ? 0ull : (kmx & ~((1ull << (shift0 + 8)) - 1ull));
+    uint64_t cnt_above = 0, mass_above = 0;
+    double target = -1.0;
+    for (int shift = shift0; shift >= 0; shift -= 8) {
+      for (int d = tid; d < 256; d += NT) {
+        cnt[d] = 0;
+        mass[d] = 0ull;
+      }
+      __syncthreads();
+      // chunks of 32 keys dealt to the warps in turn; a warp whose keys share one bucket adds
+      // its count and mass once
+      for (int j0 = warp * 32; j0 < T; j0 += NT) {
+        const int j = j0 + lane;
+        bool part = false;
+        int d = 0;
+        unsigned long long mj = 0ull;
+        if (j < T) {
+          const uint64_t kj = desc_key(s[j]);
+          if (shift == 56 || (kj >> (shift + 8)) == (prefix >> (shift + 8))) {
+            part = true;
+            d = static_cast<int>((kj >> shift) & 255u);
+            mj = mrow[j];
+          }
+        }
+        const uint32_t act = __ballot_sync(0xffffffffu, part);
+        if (act == 0u) continue;
+        const int dl = __shfl_sync(0xffffffffu, d, __ffs(act) - 1);
+        if (__all_sync(0xffffffffu, !part || d == dl)) {
+          unsigned long long ms = mj;
+#pragma unroll
+          for (int o = 16; o; o >>= 1) ms += __shfl_xor_sync(0xffffffffu, ms, o);
+          if (lane == 0) {
+            atomicAdd(&cnt[dl], static_cast<uint32_t>(__popc(act)));
+            atomicAdd(&mass[dl], ms);
+          }
+        } else if (part) {
+          atomicAdd(&cnt[d], 1u);
+          atomicAdd(&mass[d], mj);
+        }
+      }
+      __syncthreads();
+      if (warp == 0) {
+        uint32_t lc = 0;
+        unsigned long long lm = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          lc += cnt[lane * 8 + u];
+          lm += mass[lane * 8 + u];
+        }
+        uint32_t ic = lc;
+        unsigned long long im = lm;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t oc = __shfl_up_sync(0xffffffffu, ic, o);
+          const unsigned long long om = __shfl_up_sync(0xffffffffu, im, o);
+          if (lane >= o) {
+            ic += oc;
+            im += om;
+          }
+        }
+        if (shift == shift0) {  // the first level counts every key: the row's total mass
+          const unsigned long long Z = __shfl_sync(0xffffffffu, im, 31);
+          if (top_p > 0.0f) target = static_cast<double>(top_p) * static_cast<double>(Z);
+        }
+        uint64_t c_run = cnt_above + (ic - lc), m_run = mass_above + (im - lm);
+        int hit = -1;
+        uint64_t c_before = 0, m_before = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t cu = cnt[lane * 8 + u];
+          const unsigned long long mu = mass[lane * 8 + u];
+          if (hit < 0 && cu > 0 && c_run + cu >= static_cast<uint64_t>(nk) &&
+              static_cast<double>(m_run + mu) >= target) {
+            hit = lane * 8 + u;
+            c_before = c_run;
+            m_before = m_run;
+          }
+          c_run += cu;
+          m_run += mu;
+        }
+        const uint32_t bal = __ballot_sync(0xffffffffu, hit >= 0);
+        const int src = __ffs(bal) - 1;  // the totals meet both conditions: some bucket hits
+        const int dstar = __shfl_sync(0xffffffffu, hit, src);
+        const uint64_t ca = __shfl_sync(0xffffffffu, c_before, src);
+        const uint64_t ma = __shfl_sync(0xffffffffu, m_before, src);
+        if (lane == 0) {
+          ctl->dstar = dstar;
+          ctl->cnt_above = ca;
+          ctl->mass_above = ma;
+          ctl->target = target;
+          ctl->bucket = cnt[dstar];
+          ctl->bmass = mass[dstar];
+        }
+      }
+      __syncthreads();
+      const int dstar = ctl->dstar;
+      cnt_above = ctl->cnt_above;
+      mass_above = ctl->mass_above;
+      target = ctl->target;
+      const uint32_t bucket = ctl->bucket;
+      prefix |= static_cast<uint64_t>(dstar) << shift;
+      if (bucket == 1u || shift == 0) {
+        // The candidates (keys with this prefix) share one key, hence one mass: the boundary is
+        // the c-th of them in id order for the least c meeting both conditions (c = 1 for a
+        // single candidate, where the hit guarantees both).
+        const uint64_t mask = (shift == 0) ? ~0ull : ~((1ull << shift) - 1ull);
+        if (warp == 0) {
+          const unsigned long long mj = ctl->bmass / bucket;
+          int cs = -1;
+          for (uint32_t c0 = 1; c0 <= bucket && cs < 0; c0 += 32) {
+            const uint32_t c = c0 + lane;
+            const bool ok = c <= bucket && cnt_above + c >= static_cast<uint64_t>(nk) &&
+                            static_cast<double>(mass_above + c * mj) >= target;
+            const uint32_t okb = __ballot_sync(0xffffffffu, ok);
+            if (okb) cs = static_cast<int>(c0) + __ffs(okb) - 1;
+          }
+          if (lane == 0) {
+            ctl->cstar = cs < 0 ? static_cast<int>(bucket) : cs;
+            ctl->jb = 0;  // overwritten below by the warp holding the boundary candidate
+          }
+        }
+        // this warp's candidates in its id range
+        int wc = 0;
+        for (int j0 = w_lo; j0 < w_hi; j0 += 32) {
+          const int j = j0 + lane;
+          const bool cand = j < w_hi && (desc_key(s[j]) & mask) == prefix;
+          wc += __popc(__ballot_sync(0xffffffffu, cand));
+        }
+        if (lane == 0) ctl->wcount[warp] = wc;
+        __syncthreads();
+        const int cs = ctl->cstar;
+        int before = 0;
+        for (int w = 0; w < warp; ++w) before += ctl->wcount[w];
+        if (cs > before && cs <= before + wc) {  // the boundary candidate is in this warp's range
+          int seen = before;
+          for (int j0 = w_lo; j0 < w_hi; j0 += 32) {
+            const int j = j0 + lane;
+            const bool cand = j < w_hi && (desc_key(s[j]) & mask) == prefix;
+            const uint32_t cb = __ballot_sync(0xffffffffu, cand);
+            if (seen + __popc(cb) >= cs) {
+              // the (cs - seen)-th set bit of cb
+              uint32_t bits = cb;
+              for (int r = cs - seen; r > 1; --r) bits &= bits - 1u;
+              if (lane == 0) ctl->jb = j0 + __ffs(bits) - 1;
+              break;
+            }
+            seen += __popc(cb);
+          }
+        }
+        __syncthreads();
+        jb = ctl->jb;
+        kb = desc_key(s[jb]);  // the boundary's whole key (below `shift`, a lone candidate's own bits)
+        break;
+      }
+    }
+  }
+  // emit the kept ids in ascending order: count per warp range, then write at the offsets
+  int wn = 0;
+  for (int j0 = w_lo; j0 < w_hi; j0 += 32) {
+    const int j = j0 + lane;
+    bool sel = false;
+    if (j < w_hi) {
+      const uint64_t kj = desc_key(s[j]);
+      sel = kj < kb || (kj == kb && j <= jb);
+    }
+    wn += __popc(__ballot_sync(0xffffffffu, sel));
+  }
+  if (lane == 0) ctl->wcount[warp] = wn;
+  __syncthreads();
+  int n = 0, pos0 = 0;
+  for (int w = 0; w < NWARP; ++w) {
+    const int c = ctl->wcount[w];
+    if (w < warp) pos0 += c;
+    n += c;
+  }
+  for (int j0 = w_lo; j0 < w_hi; j0 += 32) {
+    const int j = j0 + lane;
+    bool sel = false;
+    if (j < w_hi) {
+      const uint64_t kj = desc_key(s[j]);
+      sel = kj < kb || (kj == kb && j <= jb);
+    }
+    const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+    const int pos = pos0 + __popc(bal & ((1u << lane) - 1u));
+    if (sel && pos < cap) out[pos] = j;
+    pos0 += __popc(bal);
+  }
+  if (tid == 0) {
+    if (n > cap) flag_error(st, DEVERR_CAPACITY, 0);
+    *count = min(n, cap);
+  }
+  __syncthreads();  // the control block and histogram are reused by the CTA's next row
+}
+
 // The fp64 path for the rows the key selection queued: one CTA per row (grid-stride over the
-// queue).  Its four warps compute the row's scores Qbar_i . Kbar_j * scale in fp64 into shared
+// queue).  Its eight warps compute the row's scores Qbar_i . Kbar_j * scale in fp64 into shared
 // memory, lanes splitting each dot product over D (coalesced reads of every Kbar row, then a
 // shuffle reduction), then every score's fixed-point mass once (the selection's passes would
-// otherwise evaluate the fp64 exponential again in each pass), and warp 0 selects from there
-// as select_kernel does.
-constexpr int kFallbackThreads = 128;  // 4 warps: each key's dot product is one warp's, 8 keys per round (16 warps measured slower)
+// otherwise evaluate the fp64 exponential again in each pass), and the whole CTA selects from
+// there (select_row_fp64_cta: the decision of select_row_fp64, with the work of each pass
+// split over the warps instead of one warp walking the row while the others wait).
+constexpr int kFallbackThreads = 256;  // 8 warps: each key's dot product is one warp's, 8 keys per round
 __global__ void __launch_bounds__(kFallbackThreads) router_fallback_kernel(const double* __restrict__ qbar,
                                                               const double* __restrict__ kbar, int D, int T,
                                                               double scale, const int* __restrict__ flist, int top_k,
@@ -1201,7 +1446,8 @@ __global__ void __launch_bounds__(kFallbackThreads) router_fallback_kernel(const
   extern __shared__ double srow[];  // [T] scores, then [T] masses
   __shared__ uint32_t cnt_s[256];
   __shared__ unsigned long long mass_s[256];
-  __shared__ double wmax[kFallbackThreads / 32];
+  __shared__ double wmax[kFallbackThreads / 32], wmin[kFallbackThreads / 32];
+  __shared__ SelCtl ctl;
   unsigned long long* mrow = reinterpret_cast<unsigned long long*>(srow + T);
   constexpr int kWarps = kFallbackThreads / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1234,21 +1480,32 @@ __global__ void __launch_bounds__(kFallbackThreads) router_fallback_kernel(const
       }
     }
     __syncthreads();
-    double mx = -DBL_MAX;
-    for (int j = threadIdx.x; j < T; j += kFallbackThreads) mx = fmax(mx, srow[j]);
+    double mx = -DBL_MAX, mn = DBL_MAX;
+    for (int j = threadIdx.x; j < T; j += kFallbackThreads) {
+      mx = fmax(mx, srow[j]);
+      mn = fmin(mn, srow[j]);
+    }
 #pragma unroll
-    for (int o = 16; o; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if (lane == 0) wmax[warp] = mx;
+    for (int o = 16; o; o >>= 1) {
+      mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    }
+    if (lane == 0) {
+      wmax[warp] = mx;
+      wmin[warp] = mn;
+    }
     __syncthreads();
     mx = wmax[0];
+    mn = wmin[0];
 #pragma unroll
-    for (int w = 1; w < kWarps; ++w) mx = fmax(mx, wmax[w]);
+    for (int w = 1; w < kWarps; ++w) {
+      mx = fmax(mx, wmax[w]);
+      mn = fmin(mn, wmin[w]);
+    }
     for (int j = threadIdx.x; j < T; j += kFallbackThreads) mrow[j] = mass_fx(srow[j], mx);
     __syncthreads();
-    if (warp == 0)
-      select_row_fp64(srow, T, top_k, top_p, cap, kv_index + static_cast<size_t>(row) * cap, kv_count + row, st,
-                      cnt_s, mass_s, mrow);
-    __syncthreads();
+    select_row_fp64_cta<kWarps>(srow, mrow, mx, mn, T, top_k, top_p, cap, kv_index + static_cast<size_t>(row) * cap,
+                                kv_count + row, st, cnt_s, mass_s, &ctl);
   }
 }
 
