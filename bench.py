@@ -832,26 +832,23 @@ def source_sha() -> str:
 
 
 def run_e2e(args, sa, A, p, host, dev, flops, world, dist):
-    """Same step through the public API with host buffers: pinned latent-order inputs are
-    copied in, tiled, routed, run forward and backward, and out/dq/dk/dv are untiled and
-    copied back, all inside the timed region."""
+    """Same step through the public API with host buffers (sa_step_host): pinned latent-order
+    inputs are copied in, tiled, routed, run forward and backward, and out/dq/dk/dv are untiled
+    and copied back, all inside the timed region, the copies of one chunk of heads overlapping
+    the work on the neighbouring chunks.  The results of the last timed step are then compared
+    with the device entry points run on the same inputs (they must be equal bit for bit)."""
     import torch
-    pinned = {n: host[n].pin_memory() for n in ("q", "k", "v", "do")}
+    pinned = {n: host[n].contiguous().pin_memory() for n in ("q", "k", "v", "do")}
     L = p.lat_t * p.lat_h * p.lat_w
-    outs = {"out": torch.empty((p.B, p.H, L, p.D), dtype=torch.bfloat16).pin_memory()}
-    for n in ("dq", "dk", "dv"):
-        outs[n] = torch.empty((p.B, p.H, L, p.D), dtype=torch.float32).pin_memory()
+    outs = [torch.empty((p.B, p.H, L, p.D), dtype=torch.bfloat16).pin_memory()]
+    outs += [torch.empty((p.B, p.H, L, p.D), dtype=torch.float32).pin_memory() for _ in range(3)]
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    chunk = max(1, min(args.e2e_chunk, p.B * p.H))
+    ws = torch.empty(sa.step_host_workspace_size(p, chunk), dtype=torch.uint8, device=dev)
 
     def e2e_step():
-        d = {n: t.to(dev, non_blocking=True) for n, t in pinned.items()}
-        x = {n: sa.tile(d[n], p) for n in d}
-        idx, cnt = A.plan(x["q"], x["k"])
-        out, lse, out32 = A.forward(x["q"], x["k"], x["v"], idx, cnt)
-        dq, dk, dv = A.backward(x["q"], x["k"], x["v"], out, lse, x["do"], idx, cnt, out_f32=out32)
-        for n, t in (("out", out), ("dq", dq), ("dk", dk), ("dv", dv)):
-            outs[n].copy_(sa.untile(t, p), non_blocking=True)
+        sa.step_host(pinned["q"], pinned["k"], pinned["v"], pinned["do"], p, chunk, *outs, ws=ws)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -864,8 +861,19 @@ def run_e2e(args, sa, A, p, host, dev, flops, world, dist):
     e1.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dist, dev)
+    status = sa.device_status(ws)
+    # the device path on the same inputs
+    x = {n: sa.tile(pinned[n].to(dev), p) for n in pinned}
+    idx, cnt = A.plan(x["q"], x["k"])
+    out, lse, out32 = A.forward(x["q"], x["k"], x["v"], idx, cnt)
+    grads = A.backward(x["q"], x["k"], x["v"], out, lse, x["do"], idx, cnt, out_f32=out32)
+    same = all(torch.equal(sa.untile(r, p).cpu(), o) for r, o in zip((out, *grads), outs))
+    del x, idx, cnt, out, lse, out32, grads
     return {"value": round(flops * world / (ms * 1e-3) / 1e12, 3), "unit": UNIT, "ms_per_step": round(ms, 3),
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "how": f"sa_step_host, {chunk} heads per chunk: chunk c copied in while c-1 is computed and c-2 "
+                   f"copied out (pinned host buffers)",
+            "device_status": sa.STATUS_NAMES.get(status, status), "equals_device_path": bool(same)}
 
 
 # ---------------------------------------------------------------------------------- oracle
@@ -1084,6 +1092,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="720p")
     ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-chunk", type=int, default=5,
+                    help="(batch, head) problems per chunk of the end-to-end step (sa_step_host)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the e4m3 Q/K forward section")
     ap.add_argument("--no-gated", action="store_true", help="skip the gated (coarse + fine) layer section")

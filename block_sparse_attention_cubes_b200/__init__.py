@@ -43,7 +43,8 @@ EXPORTS = ("sa_padded_tokens", "sa_num_cubes", "sa_topk_from_fraction", "sa_work
            "sa_untile", "sa_plan", "sa_forward", "sa_backward", "sa_get_device_status", "sa_status_string",
            "sa_last_launch_count", "sa_plan_static", "sa_plan_coarse", "sa_forward_gated", "sa_backward_gated", "sa_recall", "sa_plan_bq128",
            "sa_plan_fallback_rows", "sa_tile_rope", "sa_untile_rope", "sa_block_mass", "sa_best_recall",
-           "sa_plan_fine_workspace_size", "sa_plan_fine", "sa_get_cta_clocks")
+           "sa_plan_fine_workspace_size", "sa_plan_fine", "sa_get_cta_clocks", "sa_step_host_workspace_size",
+           "sa_step_host")
 
 
 class SAError(RuntimeError):
@@ -106,6 +107,8 @@ def load_library(path: str = LIB_PATH):
         "sa_plan_fine_workspace_size": (sz, [P, i32, i32, i32]),
         "sa_plan_fine": (i32, [vp, vp, P, i32, i32, i32, vp, vp, vp, vp, sz, vp]),
         "sa_get_cta_clocks": (i32, [vp, sz, i32, vp, i32, ctypes.POINTER(ctypes.c_int), vp]),
+        "sa_step_host_workspace_size": (sz, [P, i32]),
+        "sa_step_host": (i32, [vp, vp, vp, vp, P, i32, vp, vp, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -611,6 +614,47 @@ def best_recall(pblock, kv_count, p: Params, stream=None):
     _check(load_library().sa_best_recall(_ptr(pblock), _ptr(kv_count), ctypes.byref(p), _ptr(out), _stream(stream)),
            "sa_best_recall")
     return out
+
+
+def step_host_workspace_size(p: Params, chunk_heads: int) -> int:
+    return int(load_library().sa_step_host_workspace_size(ctypes.byref(p), int(chunk_heads)))
+
+
+def step_host(q, k, v, dout, p: Params, chunk_heads: int, out=None, dq=None, dk=None, dv=None, ws=None,
+              stream=None):
+    """One step (layout, router, forward, backward, layout back) from and to HOST memory with
+    the copies overlapped with the work, ``chunk_heads`` (batch, head) problems at a time
+    (``sa_step_host``).  q, k, v, dout: CPU ``[B,H,L,D]`` bf16 in latent order, best pinned;
+    returns CPU ``(out bf16, dq, dk, dv fp32)``, each ``[B,H,L,D]``.  The results are final
+    once ``stream`` (default: the current one) has been synchronised."""
+    torch = _torch()
+    L = p.lat_t * p.lat_h * p.lat_w
+    shape = (p.B, p.H, L, p.D)
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
+        if t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be a contiguous CPU bf16 tensor")
+        _shape(t, shape, name)
+    def host_out(t, name, dtype):
+        if t is None:
+            return torch.empty(shape, dtype=dtype).pin_memory()
+        if t.is_cuda or not t.is_contiguous() or t.dtype != dtype:
+            raise ValueError(f"{name} must be a contiguous CPU {dtype} tensor")
+        _shape(t, shape, name)
+        return t
+    out = host_out(out, "out", torch.bfloat16)
+    dq, dk, dv = (host_out(t, n, torch.float32) for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")))
+    need = step_host_workspace_size(p, chunk_heads)
+    if need == 0:
+        raise SAError(1, "sa_step_host_workspace_size")
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+        if stream is not None:  # the allocator hands this memory out again only after `stream`'s work
+            ws.record_stream(stream)
+    _contig(ws, "ws", torch.uint8)
+    _check(load_library().sa_step_host(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), ctypes.byref(p), int(chunk_heads),
+                                       _ptr(out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
+                                       _stream(stream)), "sa_step_host")
+    return out, dq, dk, dv
 
 
 @dataclass

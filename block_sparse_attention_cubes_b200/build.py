@@ -9,7 +9,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = ["api.cu", "layout.cu", "router.cu", "attn_fwd.cu", "attn_bwd.cu", "pairs.cu", "plan_static.cu", "coarse.cu", "recall.cu", "blocks128.cu", "fine_router.cu"]
+SOURCES = ["api.cu", "layout.cu", "router.cu", "attn_fwd.cu", "attn_bwd.cu", "pairs.cu", "plan_static.cu", "coarse.cu", "recall.cu", "blocks128.cu", "fine_router.cu", "step_host.cu"]
 LIB = os.path.join(HERE, "libsa.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

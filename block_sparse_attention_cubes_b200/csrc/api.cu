@@ -300,6 +300,9 @@ sa::AttnArgs base_args(const sa_params* p, const Geom& g, void* ws) {
 
 namespace sa {
 
+// the launch count sa_last_launch_count reports, for entry points defined in other files
+void set_last_launches(int n) { g_last_launches = n; }
+
 // sa_plan's host-side argument checks (nothing touches the device); *ws_needed receives the
 // workspace size the router needs.
 sa_status plan_check(const void* q, const void* k, const float* q_scale, const float* k_scale, const sa_params* p,

@@ -337,6 +337,32 @@ SA_API sa_status sa_best_recall(const float* pblock, const int32_t* kv_count, co
 SA_API sa_status sa_plan_static(const void* q, const void* k, const float* q_scale, const float* k_scale,
                                 const sa_params* p, int32_t* kv_index, int32_t* kv_count, sa_stream_t stream);
 
+/* ---- One step from and to host memory ----
+ * The whole hot path of one training step on host buffers: the layout of the VSA page
+ * ("Cube Partitioning and Token Re-Indexing"), sa_plan, sa_forward (with its fp32 output)
+ * and sa_backward as documented above, and the layout back, with the host<->device copies
+ * overlapped with the work.  The B*H (batch, head) problems are independent, so the step
+ * runs over chunks of chunk_heads consecutive problems of the flattened [B*H] axis (the
+ * last chunk may be shorter): chunk c's inputs are copied in while chunk c-1 is computed
+ * and chunk c-2's results are copied out (two internal copy streams, two buffer slots in
+ * the workspace, events between them).  Results equal those of the device entry points
+ * run on the same data.  bf16 only (qk_dtype SA_BF16, else SA_ERR_UNSUPPORTED); B*H <= 65535.
+ * q, k, v, dout: HOST [B,H,lat_t*lat_h*lat_w,D] bf16 in latent (t, h, w) order.
+ * out: HOST [B,H,L,D] bf16; dq, dk, dv: HOST [B,H,L,D] fp32 (L = lat_t*lat_h*lat_w).
+ * Host buffers should be page-locked (cudaHostAlloc, or pinned tensors) for the copies to
+ * run asynchronously; pageable memory works but serialises the copies with the host.  The
+ * caller keeps every host buffer alive and unmodified until `stream` has been synchronised.
+ * ws: device workspace of sa_step_host_workspace_size(p, chunk_heads) bytes, 16-byte
+ * aligned; its first 256 bytes gather the device status of every chunk's calls
+ * (sa_get_device_status(ws, stream)).  All device work is ordered on `stream`: it starts
+ * after the work already queued there, and work queued after the call starts after the
+ * last copy-out.  Returns the first host-side error of any chunk's calls (SA_ERR_* as for
+ * those entry points); nothing more is issued after it. */
+SA_API size_t sa_step_host_workspace_size(const sa_params* p, int chunk_heads);
+SA_API sa_status sa_step_host(const void* q, const void* k, const void* v, const void* dout, const sa_params* p,
+                              int chunk_heads, void* out, float* dq, float* dk, float* dv, void* ws,
+                              size_t ws_bytes, sa_stream_t stream);
+
 /* Synchronises `stream`, then maps the workspace's device status block to a status:
  * SA_OK, SA_ERR_DEVICE_TIMEOUT, SA_ERR_DEVICE_INDEX or SA_ERR_CAPACITY (first that
  * applies, in that order of precedence: timeout, index, capacity). */

@@ -218,3 +218,32 @@ def test_cta_clocks_validate_on_the_host(lib):
                                      (fake, 10 ** 6, 0, None, ctypes.byref(n)),     # null output
                                      (fake, 10 ** 6, 0, out, None)):                # null count
         assert lib.sa_get_cta_clocks(ws, size, kernel, o, 4, np_, None) == 1
+
+
+def test_step_host_validates_on_the_host(lib):
+    """sa_step_host_workspace_size and the error paths of sa_step_host that return before any
+    stream, event or copy is made."""
+    p = sa.make_params(2, 3, 64, (8, 8, 8), 4, 0.5)            # B*H = 6 problems, T = 8, L = 512
+    P = ctypes.byref(p)
+    npad, T, L, D = 512, 8, 512, 64
+    w1, w2, w6 = (lib.sa_step_host_workspace_size(P, c) for c in (1, 2, 6))
+    assert 0 < w1 < w2 < w6
+    assert lib.sa_step_host_workspace_size(P, 100) == w6       # chunks never exceed B*H
+    assert lib.sa_step_host_workspace_size(P, 0) == 0
+    # per problem at least: two slots of latent inputs and outputs, the cube-major tensors, the lists
+    per = 2 * 4 * L * D * 2 + 4 * npad * D * 2 + T * T * 4 + npad * D * (2 + 4 + 3 * 4) + 2 * L * D * (2 + 3 * 4)
+    assert w2 >= 2 * per + sum(sa.workspace_size(sa.make_params(1, 2, 64, (8, 8, 8), 4, 0.5), op)
+                               for op in (sa.OP_PLAN, sa.OP_FORWARD, sa.OP_BACKWARD))
+    bad, odd = ctypes.c_void_p(16), ctypes.c_void_p(24)
+    # sa_step_host(q, k, v, dout, p, chunk_heads, out, dq, dk, dv, ws, ws_bytes, stream)
+    assert lib.sa_step_host(bad, bad, bad, None, P, 2, bad, bad, bad, bad, bad, w2, None) == 1
+    assert lib.sa_step_host(bad, bad, bad, bad, P, 0, bad, bad, bad, bad, bad, w2, None) == 1
+    assert lib.sa_step_host(bad, bad, bad, bad, P, 2, bad, bad, bad, bad, None, w2, None) == 5
+    assert lib.sa_step_host(bad, bad, bad, bad, P, 2, bad, bad, bad, bad, bad, w2 - 1, None) == 5
+    assert lib.sa_step_host(bad, bad, bad, bad, P, 2, bad, bad, bad, bad, odd, w2, None) == 3
+    f8 = sa.make_params(1, 2, 128, (8, 8, 8), 4, 0.5, qk_dtype=sa.FP8_E4M3)
+    assert lib.sa_step_host(bad, bad, bad, bad, ctypes.byref(f8), 1, bad, bad, bad, bad, bad, 1 << 30, None) == 2
+    d96 = sa.make_params(1, 2, 96, (8, 8, 8), 4, 0.5)
+    assert lib.sa_step_host_workspace_size(ctypes.byref(d96), 1) == 0
+    assert lib.sa_step_host(bad, bad, bad, bad, ctypes.byref(d96), 1, bad, bad, bad, bad, bad, 1 << 30, None) == 2
+    assert lib.sa_last_launch_count() == 0
