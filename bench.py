@@ -1092,7 +1092,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="720p")
     ap.add_argument("--e2e-steps", type=int, default=2)
-    ap.add_argument("--e2e-chunk", type=int, default=5,
+    ap.add_argument("--e2e-chunk", type=int, default=2,
                     help="(batch, head) problems per chunk of the end-to-end step (sa_step_host)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the e4m3 Q/K forward section")
