@@ -440,14 +440,15 @@ struct RowMeta {
 
 
 // Pooling for the tensor-core router.  Persistent CTAs, one per SM; items are (head, cube, Q or
-// K), dealt round-robin so the CTAs stream neighbouring cubes together.  Warp 8 (one lane)
-// brings each item's rows (up to the cube's last valid slot: one contiguous range) into a
-// 12-stage shared-memory ring with 1-D bulk copies; warps 0-7 take the items in turn, each lane
-// summing D/32 columns over the cube's valid rows in fp64, and write the mean, its limbs, the
-// row's binary exponent and (Q) its 1-norm.  (Half-cube stages with 12 consumers measured
-// slower: 0.63 against 0.50 ms at 720p.)
+// K), dealt round-robin so the CTAs stream neighbouring cubes together.  The last warp (one
+// lane) brings each item's rows (up to the cube's last valid slot: one contiguous range) into a
+// 12-stage shared-memory ring with 1-D bulk copies; the kConsumers warps before it take the items
+// in turn, each lane summing D/32 columns over the cube's valid rows in fp64, and write the mean,
+// its limbs, the row's binary exponent and (Q) its 1-norm.  Measured at 720p (sa_plan alone):
+// ten consumers 1.24 ms, eight 1.26, twelve (one stage each, no lookahead) 1.26; half-cube
+// stages with twelve consumers were slower still (0.63 against 0.50 ms for the pooling).
 namespace rpl {
-constexpr int kConsumers = 8;
+constexpr int kConsumers = 10;
 constexpr int kThreads = (kConsumers + 1) * 32;
 constexpr int kStages = 12;
 // A consumer's next stage is kConsumers stages past its last one.  A parity wait tells apart
