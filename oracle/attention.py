@@ -149,7 +149,7 @@ def hybrid_ids(row: np.ndarray, k: int, p: float) -> np.ndarray:
 
 @dataclass
 class RouterTrace:
-    """Everything the parity tests need to judge one (b, h) slice of the router."""
+    """Everything the parity tests need to check one (b, h) slice of the router."""
     pbar: np.ndarray      # [T, T] fp64 block probabilities
     lists: list           # T arrays of ascending kv block ids
     n_k: np.ndarray       # [T] Top-k size

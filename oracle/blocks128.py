@@ -12,7 +12,7 @@ What it restates:
 * recall ............... SpargeAttention2 page, equation 8: tau = sum_j p_j m_j, the share of a
                          query's true attention mass inside its kept blocks; VSA2 page, section
                          2.2: P_oracle = MeanPool_{B x B}(P), against which a selection of n
-                         blocks per query cube can be judged (VSA page, "Kernel Implementation":
+                         blocks per query cube can be measured (VSA page, "Kernel Implementation":
                          Top-32 captures 50-90% of the mass)
 
 Readings where the pages are silent:

@@ -1,5 +1,5 @@
 """Helpers shared by the GPU parity tests: run the CUDA path and the oracle on the same
-seeded inputs and judge the results.  Test infrastructure only."""
+seeded inputs and compare the results.  Test infrastructure only."""
 import math
 
 import numpy as np

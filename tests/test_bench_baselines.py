@@ -1,6 +1,6 @@
 """The bench's oracle baselines run on the host alone (CPU only): the plain step's and the
 gated layer's, on a small configuration, with a bounded sample and the contract's keys.
-The plain step's leg also judges the last timed step's lists and outputs; here it is fed
+The plain step's leg also checks the last timed step's lists and outputs; here it is fed
 the oracle's own results (everything equal, errors zero) and then one planted wrong list."""
 import numpy as np
 import torch
